@@ -1,0 +1,270 @@
+/*
+ * sgmv.h -- C ABI of libsgmv_b200.so: the multi-LoRA delta on one B200 (sm_100a).
+ *
+ * The library computes, for every token t of a batch whose tokens carry
+ * different LoRA adapters a(t),
+ *
+ *     y_t  <-  y_t + scale * B_{a(t)} ( A_{a(t)} x_t )
+ *
+ * where y already holds the base output W x_t.  Pages cited by title:
+ *
+ *   [SGMV post] "Multi-LoRA serving: the single translator with a thousand
+ *               glossaries -- shared base, thousands of concurrent adapters
+ *               and the SGMV kernel" (blog.lo0.es)
+ *   [Glossary]  "Multi-LoRA Serving" (skillsintelligence.tools glossary)
+ *   [ClusterBid] "Multi-LoRA Inference Serving: Serving Thousands of
+ *               Fine-Tuned Models on One GPU" (clusterbid.com)
+ *
+ * Orientation ([SGMV post], "The bare mechanism", equations W' = W + BA and
+ * y = Wx + B(Ax)): A is r x d_in, B is d_out x r.  The per-token form and its
+ * two phases, shrink (d_in -> r) and expand (r -> d_out), are those of
+ * [SGMV post], "SGMV: the kernel that holds it all up".
+ *
+ * Conventions shared by every call
+ *   - All matrices are row-major.  bf16 data is passed as raw 16-bit words.
+ *   - "device" pointers are CUDA global-memory addresses on the pool's
+ *     device; "host" pointers are ordinary process memory.
+ *   - Calls that take a stream enqueue work on it and return without
+ *     waiting, except where stated.  NULL is the legacy default stream.
+ *   - A call that returns anything but SGMV_OK has launched nothing and
+ *     changed no caller memory; sgmv_last_error() describes the failure.
+ *   - Kernels never trap.  Device-side checks (a page id outside the pool,
+ *     a token row outside the batch, a wait that gave up) set a device error
+ *     word and skip the access; sgmv_check_errors() reports and clears it.
+ *   - The caller owns x, y, v and the plan table; the pool owns its pages
+ *     and its page table.  Nothing here is thread-safe on the same pool.
+ */
+#ifndef SGMV_B200_H
+#define SGMV_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SGMV_API __attribute__((visibility("default")))
+#else
+#define SGMV_API
+#endif
+
+typedef struct CUstream_st* sgmv_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    SGMV_OK = 0,
+    SGMV_ERR_INVALID = 1,      /* malformed argument (null pointer, bad size, misaligned row) */
+    SGMV_ERR_UNSUPPORTED = 2,  /* well-formed but outside what this build handles            */
+    SGMV_ERR_NOT_RESIDENT = 3, /* an adapter id of the batch is not loaded in the pool        */
+    SGMV_ERR_OUT_OF_PAGES = 4, /* the pool has too few free pages for an adapter              */
+    SGMV_ERR_CUDA = 5,         /* a CUDA runtime call failed                                  */
+    SGMV_ERR_BOUNDS = 6,       /* a device-side bounds check failed (from sgmv_check_errors)  */
+    SGMV_ERR_TIMEOUT = 7,      /* a device-side wait gave up (from sgmv_check_errors)         */
+    SGMV_ERR_CAPACITY = 8      /* a caller-provided buffer is too small                       */
+} sgmv_status;
+
+/* Text of a status code (static storage). */
+SGMV_API const char* sgmv_status_string(sgmv_status s);
+/* Detail of the last failure on the calling thread (thread-local storage). */
+SGMV_API const char* sgmv_last_error(void);
+
+/* ------------------------------------------------------------------------ */
+/* Paged adapter pool                                                         */
+/* ------------------------------------------------------------------------ */
+/*
+ * Adapter weights live in one device buffer of equal-size pages, in the
+ * spirit of the unified paging that [SGMV post] describes (TL;DR, and
+ * "Operational pitfalls": memory fragmentation -- weights kept in a pool of
+ * interchangeable blocks) and of the fixed-size adapter pool with slots of
+ * [ClusterBid] (paragraph on vLLM's GPU memory pool).
+ *
+ * Layout.  A page holds page_elems bf16 values.  For each adapter and each
+ * projection p the pool stores
+ *     A   as r rows of d_in[p]  values (the logical r x d_in matrix), and
+ *     B^T as r rows of d_out[p] values (the transpose of the d_out x r B),
+ * each row cut into d/page_elems pages.  The page table (int32 page ids) maps
+ * (adapter, projection, matrix, rank row k, chunk c) to a page; entries of one
+ * (adapter, projection, matrix) are contiguous:
+ *     entry = base + k * (d / page_elems) + c.
+ * Pages are taken from a free list in any order, so consecutive chunks of a
+ * row are in general not adjacent in memory.
+ *
+ * The payload of a rank-r adapter is exactly sum_p (d_in[p]*r + r*d_out[p])*2
+ * bytes -- the bytes-per-matrix formula of [SGMV post], "The maths that
+ * matters" -- because page_elems must divide every d_in[p] and d_out[p].
+ */
+typedef struct sgmv_pool sgmv_pool;
+
+typedef struct {
+    int64_t num_pages;         /* pages in the pool                                 */
+    int64_t free_pages;        /* pages not holding adapter data                    */
+    int64_t page_bytes;        /* page_elems * 2                                    */
+    int64_t payload_bytes;     /* (num_pages - free_pages) * page_bytes             */
+    int32_t resident_adapters; /* adapters currently loaded                         */
+    int32_t page_elems;
+} sgmv_pool_stats;
+
+/*
+ * Create a pool on `device` (CUDA ordinal) with `num_pages` pages of
+ * `page_elems` bf16 values (a power of two in [64, 65536]), for adapters over
+ * `n_proj` projections with shapes d_in[p] -> d_out[p] (host arrays of n_proj
+ * entries, each a multiple of page_elems) and ranks up to max_rank (<= 128).
+ * device = -1 creates a host-only pool that keeps the bookkeeping (page
+ * allocation, page table) without device memory; its loads copy nothing and
+ * accept NULL matrix pointers.  A device pool allocates
+ * num_pages * page_elems * 2 bytes of pages and 2 * num_pages + 1024 int32
+ * page-table entries on `device`, which must be the current device of every
+ * later call that uses the pool.  On success *out owns that memory until
+ * sgmv_pool_destroy.
+ */
+SGMV_API sgmv_status sgmv_pool_create(int device, int64_t num_pages, int32_t page_elems, int32_t n_proj,
+                             const int32_t* d_in, const int32_t* d_out, int32_t max_rank,
+                             sgmv_pool** out);
+SGMV_API sgmv_status sgmv_pool_destroy(sgmv_pool* pool);
+
+/*
+ * Load (or replace) adapter `adapter_id` (>= 0) of rank `rank` (0..max_rank).
+ * A[p] points to the r x d_in[p] matrix of projection p, B[p] to its
+ * d_out[p] x r matrix (bf16, row-major, logical orientation); A and B are host
+ * arrays of n_proj pointers.  The pointed-to data is device memory when
+ * src_on_device != 0, host memory otherwise.  The copies are enqueued on
+ * `stream` and the call waits for them before returning, so the sources may be
+ * freed afterwards.  SGMV_ERR_OUT_OF_PAGES leaves the pool unchanged.
+ */
+SGMV_API sgmv_status sgmv_pool_load(sgmv_pool* pool, int32_t adapter_id, int32_t rank,
+                           const void* const* A, const void* const* B, int src_on_device,
+                           sgmv_stream_t stream);
+/* Remove an adapter and return its pages to the free list.  The caller must
+ * not evict an adapter that an enqueued kernel may still read. */
+SGMV_API sgmv_status sgmv_pool_evict(sgmv_pool* pool, int32_t adapter_id);
+SGMV_API sgmv_status sgmv_pool_get_stats(const sgmv_pool* pool, sgmv_pool_stats* out);
+/* Rank of a resident adapter; SGMV_ERR_NOT_RESIDENT otherwise. */
+SGMV_API sgmv_status sgmv_pool_adapter_rank(const sgmv_pool* pool, int32_t adapter_id, int32_t* rank);
+/*
+ * Copy the page ids of (adapter, projection, matrix) into page_ids (host,
+ * capacity `cap`), in page-table order; matrix 0 = A, 1 = B^T.  *n receives
+ * the count (r * d / page_elems).  For inspection and tests.
+ */
+SGMV_API sgmv_status sgmv_pool_adapter_pages(const sgmv_pool* pool, int32_t adapter_id, int32_t proj,
+                                    int32_t matrix, int32_t* page_ids, int64_t cap, int64_t* n);
+/*
+ * Reorder the free-page list pseudo-randomly (seeded), so that later loads
+ * place consecutive chunks of a row on scattered pages.  Changes no resident
+ * adapter.  For exercising the page-table indirection.
+ */
+SGMV_API sgmv_status sgmv_pool_shuffle_free_pages(sgmv_pool* pool, uint64_t seed);
+/* Device address of the page buffer (bf16 [num_pages][page_elems]); NULL for a
+ * host-only pool.  For inspection and tests. */
+SGMV_API const void* sgmv_pool_pages_device(const sgmv_pool* pool);
+
+/* ------------------------------------------------------------------------ */
+/* Segment builder and dispatch plan                                          */
+/* ------------------------------------------------------------------------ */
+/*
+ * SGMV "groups the batch's tokens by adapter" and picks, per segment, tensor
+ * cores for large segments and a batched gather path for small ones
+ * ([SGMV post], "SGMV: the kernel that holds it all up", and the figure in
+ * that section; heterogeneous ranks in one batch: TL;DR and the S-LoRA
+ * MBGMM/MBGMV paragraph).
+ *
+ * The builder runs on the host.  It writes one table (host memory, 16-byte
+ * aligned arrays at the byte offsets below) that the caller copies to the
+ * device as is, and fills the plan header, which stays on the host.
+ *
+ *   token_idx   int32 [num_rows]         sorted row -> token (row of x and y)
+ *   seg_offsets int32 [num_segments+1]   rows of segment s: [off[s], off[s+1])
+ *   seg_adapter int32 [num_segments]
+ *   seg_rank    int32 [num_segments]
+ *   seg_a_pt    int64 [num_segments*n_proj]  first page-table entry of A, per projection
+ *   seg_b_pt    int64 [num_segments*n_proj]  first page-table entry of B^T
+ *   simt_items  int32x4 [num_simt_items] {segment, row_begin, row_end, 0}
+ *   tc_tiles    int32x4 [num_tc_tiles]   {segment, row_begin, row_end, 0}, <= 128 rows
+ *
+ * Segments are in ascending adapter id; rows of a segment keep batch order
+ * (stable).  Tokens with adapter id -1 are in no segment and their y rows
+ * are never touched.  Segments of rank 0 produce no work item.  A segment
+ * with at least `long_threshold` rows goes to the tensor-core path as
+ * 128-row tiles; shorter segments go to the SIMT path as items of at most
+ * 64 rows (long_threshold <= 0 selects the built-in default; a huge value
+ * keeps every segment on the SIMT path; 1 sends every segment to tensor cores).
+ */
+typedef struct {
+    int32_t T;              /* tokens in the batch                                   */
+    int32_t num_segments;   /* S                                                     */
+    int32_t num_rows;       /* tokens in some segment (= off[S]); rows of v           */
+    int32_t max_rank;       /* R = max segment rank; v needs ldv >= R                */
+    int32_t n_proj;
+    int32_t num_simt_items;
+    int32_t num_tc_tiles;
+    int32_t long_threshold; /* the threshold actually used                           */
+    int32_t max_item_rows;  /* largest SIMT item                                     */
+    int32_t reserved;
+    int64_t table_bytes;    /* bytes of the table to copy to the device              */
+    int64_t off_token_idx, off_seg_offsets, off_seg_adapter, off_seg_rank;
+    int64_t off_seg_a_pt, off_seg_b_pt, off_simt_items, off_tc_tiles;
+} sgmv_plan;
+
+/* Bytes a table may need for a batch of T tokens over n_proj projections. */
+SGMV_API int64_t sgmv_plan_table_capacity(int32_t T, int32_t n_proj);
+
+/*
+ * adapter_ids: host int32[T], -1 = no adapter.  Every other id must be
+ * resident in `pool` (else SGMV_ERR_NOT_RESIDENT).  `table` is host memory of
+ * `table_capacity` bytes (see sgmv_plan_table_capacity), 16-byte aligned.
+ * Host only; touches no device memory.
+ */
+SGMV_API sgmv_status sgmv_build_plan(const int32_t* adapter_ids, int32_t T, const sgmv_pool* pool,
+                            int32_t long_threshold, void* table, int64_t table_capacity,
+                            sgmv_plan* plan);
+
+/* ------------------------------------------------------------------------ */
+/* SGMV-shrink and SGMV-expand                                               */
+/* ------------------------------------------------------------------------ */
+/*
+ * SGMV-shrink ([SGMV post], "SGMV: the kernel that holds it all up", phase 1:
+ * projection d_in -> r with A_{a(t)}):
+ *
+ *   v[i][k] = sum_c A_s[k][c] * x[token_idx[i]][c]     for rows i of segment s, k < r_s
+ *
+ * x       device bf16 [T][ldx], ldx >= d_in, row starts 16-byte aligned
+ * v       device fp32 [plan->num_rows][ldv], ldv >= plan->max_rank; written
+ *         for k < r_s (other entries are left as they were); fp32 accumulation
+ * proj    projection index, d_in must equal the pool's d_in[proj]
+ * table   device copy of the table that built `plan`
+ * One launch covers every SIMT item (all short segments, any mix of ranks)
+ * and one more covers every tensor-core tile, in stream order.
+ */
+SGMV_API sgmv_status sgmv_shrink(const void* x, int64_t ldx, int32_t T, int32_t d_in, int32_t proj,
+                        const sgmv_plan* plan, const void* table, const sgmv_pool* pool,
+                        float* v, int64_t ldv, sgmv_stream_t stream);
+
+/*
+ * SGMV-expand ([SGMV post], "SGMV: the kernel that holds it all up", phase 2:
+ * projection r -> d_out with B_{a(t)}, accumulated into Y as in the TL;DR's
+ * "Y +=" form):
+ *
+ *   y[t][j] <- round( y[t][j] + scale * sum_{k < r_s} B_s[j][k] * v[i][k] ),  t = token_idx[i]
+ *
+ * computed in fp32 with one rounding to the output type.
+ * y        device [T][ldy] updated in place, ldy >= d_out, rows 16-byte aligned;
+ *          y_dtype 0 = bf16 (round to nearest even), 1 = fp32.
+ * Rows of tokens in no segment are not read or written.
+ */
+SGMV_API sgmv_status sgmv_expand(const float* v, int64_t ldv, int32_t T, int32_t d_out, int32_t proj,
+                        const sgmv_plan* plan, const void* table, const sgmv_pool* pool,
+                        float scale, void* y, int64_t ldy, int32_t y_dtype,
+                        sgmv_stream_t stream);
+
+/*
+ * Wait for `stream`, then return and clear the device error word:
+ * SGMV_OK, SGMV_ERR_BOUNDS or SGMV_ERR_TIMEOUT.  *flags (may be NULL) receives
+ * the raw bits (1 = page id out of range, 2 = token row out of range,
+ * 4 = wait timed out, 8 = segment rows out of range).
+ */
+SGMV_API sgmv_status sgmv_check_errors(sgmv_stream_t stream, uint32_t* flags);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SGMV_B200_H */

@@ -1,0 +1,335 @@
+"""Python binding of libsgmv_b200.so -- the multi-LoRA delta on one B200.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library behind the C ABI declared in include/sgmv.h.  PyTorch supplies device
+memory and streams.  If the compiled library is missing this module raises on
+import of any entry point; there is no fallback.
+
+    pool = AdapterPool([(d_in, d_out), ...], num_pages=..., device=0)
+    pool.load(adapter_id, rank, [A_p ...], [B_p ...])    # A_p: [r, d_in], B_p: [d_out, r] bf16
+    plan = pool.plan(adapter_ids)                         # segment builder + dispatch (host)
+    plan.upload()                                         # one host->device copy of the table
+    v = plan.new_v()
+    shrink(x, plan, pool, v, proj)                        # v = A_{a(t)} x_t
+    expand(v, plan, pool, y, proj, scale)                 # y_t += scale * B_{a(t)} v_t
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libsgmv_b200.so")
+
+_STATUS = {0: "SGMV_OK", 1: "SGMV_ERR_INVALID", 2: "SGMV_ERR_UNSUPPORTED", 3: "SGMV_ERR_NOT_RESIDENT",
+           4: "SGMV_ERR_OUT_OF_PAGES", 5: "SGMV_ERR_CUDA", 6: "SGMV_ERR_BOUNDS", 7: "SGMV_ERR_TIMEOUT",
+           8: "SGMV_ERR_CAPACITY"}
+
+EXPORTED = ("sgmv_status_string", "sgmv_last_error", "sgmv_pool_create", "sgmv_pool_destroy", "sgmv_pool_load",
+            "sgmv_pool_evict", "sgmv_pool_get_stats", "sgmv_pool_adapter_rank", "sgmv_pool_adapter_pages",
+            "sgmv_pool_shuffle_free_pages", "sgmv_pool_pages_device", "sgmv_plan_table_capacity",
+            "sgmv_build_plan", "sgmv_shrink", "sgmv_expand", "sgmv_check_errors")
+
+
+class SgmvError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "T", "num_segments", "num_rows", "max_rank", "n_proj", "num_simt_items", "num_tc_tiles",
+        "long_threshold", "max_item_rows", "reserved")] + [(n, ctypes.c_int64) for n in (
+            "table_bytes", "off_token_idx", "off_seg_offsets", "off_seg_adapter", "off_seg_rank",
+            "off_seg_a_pt", "off_seg_b_pt", "off_simt_items", "off_tc_tiles")]
+
+
+class PoolStats(ctypes.Structure):
+    _fields_ = [("num_pages", ctypes.c_int64), ("free_pages", ctypes.c_int64), ("page_bytes", ctypes.c_int64),
+                ("payload_bytes", ctypes.c_int64), ("resident_adapters", ctypes.c_int32),
+                ("page_elems", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load the compiled library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with segmented_rank_gemm_sgmv_b200/build.py "
+                          "(there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    i32, i64, vp, f32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_float
+    st = ctypes.c_int
+    sig = {
+        "sgmv_status_string": (ctypes.c_char_p, [st]),
+        "sgmv_last_error": (ctypes.c_char_p, []),
+        "sgmv_pool_create": (st, [ctypes.c_int, i64, i32, i32, vp, vp, i32, ctypes.POINTER(vp)]),
+        "sgmv_pool_destroy": (st, [vp]),
+        "sgmv_pool_load": (st, [vp, i32, i32, vp, vp, ctypes.c_int, vp]),
+        "sgmv_pool_evict": (st, [vp, i32]),
+        "sgmv_pool_get_stats": (st, [vp, ctypes.POINTER(PoolStats)]),
+        "sgmv_pool_adapter_rank": (st, [vp, i32, ctypes.POINTER(i32)]),
+        "sgmv_pool_adapter_pages": (st, [vp, i32, i32, i32, vp, i64, ctypes.POINTER(i64)]),
+        "sgmv_pool_shuffle_free_pages": (st, [vp, ctypes.c_uint64]),
+        "sgmv_pool_pages_device": (vp, [vp]),
+        "sgmv_plan_table_capacity": (i64, [i32, i32]),
+        "sgmv_build_plan": (st, [vp, i32, vp, i32, vp, i64, ctypes.POINTER(Plan)]),
+        "sgmv_shrink": (st, [vp, i64, i32, i32, i32, ctypes.POINTER(Plan), vp, vp, vp, i64, vp]),
+        "sgmv_expand": (st, [vp, i64, i32, i32, i32, ctypes.POINTER(Plan), vp, vp, f32, vp, i64, i32, vp]),
+        "sgmv_check_errors": (st, [vp, ctypes.POINTER(ctypes.c_uint32)]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        msg = load_library().sgmv_last_error().decode(errors="replace")
+        raise SgmvError(status, msg)
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+class AdapterPool:
+    """Paged adapter pool (see include/sgmv.h, "Paged adapter pool")."""
+
+    def __init__(self, projections: Sequence[Tuple[int, int]], num_pages: int, page_elems: int = 512,
+                 max_rank: int = 128, device: int = 0):
+        lib = load_library()
+        self.projections = [(int(a), int(b)) for a, b in projections]
+        self.device = device
+        self.page_elems = page_elems
+        n = len(self.projections)
+        d_in = (ctypes.c_int32 * n)(*[p[0] for p in self.projections])
+        d_out = (ctypes.c_int32 * n)(*[p[1] for p in self.projections])
+        h = ctypes.c_void_p()
+        _check(lib.sgmv_pool_create(device, int(num_pages), int(page_elems), n, ctypes.cast(d_in, ctypes.c_void_p),
+                                    ctypes.cast(d_out, ctypes.c_void_p), int(max_rank), ctypes.byref(h)))
+        self.handle = h
+
+    def close(self):
+        if getattr(self, "handle", None):
+            load_library().sgmv_pool_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @staticmethod
+    def pages_needed(projections, rank: int, page_elems: int = 512) -> int:
+        return sum(rank * (a // page_elems + b // page_elems) for a, b in projections)
+
+    def load(self, adapter_id: int, rank: int, A: Optional[Sequence[torch.Tensor]] = None,
+             B: Optional[Sequence[torch.Tensor]] = None, stream=None) -> None:
+        """A[p]: bf16 [rank, d_in_p]; B[p]: bf16 [d_out_p, rank]; all on the pool's device or all on the
+        host.  A host-only pool (device=-1) takes A = B = None and records the bookkeeping only."""
+        n = len(self.projections)
+        if rank > 0 and self.device < 0 and A is None and B is None:
+            _check(load_library().sgmv_pool_load(self.handle, int(adapter_id), int(rank), None, None, 0, None))
+        elif rank > 0:
+            assert len(A) == n and len(B) == n
+            on_dev = A[0].is_cuda
+            keep = []
+            for p, (d_in, d_out) in enumerate(self.projections):
+                a = A[p].contiguous()
+                b = B[p].contiguous()
+                assert a.dtype == torch.bfloat16 and b.dtype == torch.bfloat16
+                assert tuple(a.shape) == (rank, d_in) and tuple(b.shape) == (d_out, rank), (a.shape, b.shape)
+                assert a.is_cuda == on_dev and b.is_cuda == on_dev
+                keep += [a, b]
+            a_ptrs = (ctypes.c_void_p * n)(*[keep[2 * p].data_ptr() for p in range(n)])
+            b_ptrs = (ctypes.c_void_p * n)(*[keep[2 * p + 1].data_ptr() for p in range(n)])
+            _check(load_library().sgmv_pool_load(self.handle, int(adapter_id), int(rank),
+                                                  ctypes.cast(a_ptrs, ctypes.c_void_p),
+                                                  ctypes.cast(b_ptrs, ctypes.c_void_p), 1 if on_dev else 0,
+                                                  _stream(stream) if self.device >= 0 else None))
+            del keep
+        else:
+            _check(load_library().sgmv_pool_load(self.handle, int(adapter_id), 0, None, None, 0,
+                                                  _stream(stream) if self.device >= 0 else None))
+
+    def evict(self, adapter_id: int) -> None:
+        _check(load_library().sgmv_pool_evict(self.handle, int(adapter_id)))
+
+    def shuffle_free_pages(self, seed: int) -> None:
+        _check(load_library().sgmv_pool_shuffle_free_pages(self.handle, int(seed)))
+
+    def stats(self) -> PoolStats:
+        s = PoolStats()
+        _check(load_library().sgmv_pool_get_stats(self.handle, ctypes.byref(s)))
+        return s
+
+    def rank_of(self, adapter_id: int) -> int:
+        r = ctypes.c_int32()
+        _check(load_library().sgmv_pool_adapter_rank(self.handle, int(adapter_id), ctypes.byref(r)))
+        return r.value
+
+    def page_ids(self, adapter_id: int, proj: int, matrix: int) -> np.ndarray:
+        n = ctypes.c_int64()
+        lib = load_library()
+        st = lib.sgmv_pool_adapter_pages(self.handle, adapter_id, proj, matrix, None, 0, ctypes.byref(n))
+        if st not in (0, 8):
+            _check(st)
+        out = np.zeros(max(n.value, 1), dtype=np.int32)
+        _check(lib.sgmv_pool_adapter_pages(self.handle, adapter_id, proj, matrix, out.ctypes.data, n.value,
+                                           ctypes.byref(n)))
+        return out[:n.value]
+
+    def pages_tensor(self) -> torch.Tensor:
+        """The page buffer as a bf16 [num_pages, page_elems] tensor view (device pools only)."""
+        addr = load_library().sgmv_pool_pages_device(self.handle)
+        s = self.stats()
+        storage = torch.cuda.memory  # noqa: F841  (keeps torch.cuda initialised)
+        arr = _DevicePtr(addr, s.num_pages * s.page_elems * 2, self.device)
+        t = torch.as_tensor(arr, device=f"cuda:{self.device}")
+        return t.view(torch.bfloat16).view(s.num_pages, s.page_elems)
+
+    def plan(self, adapter_ids, long_threshold: int = 0) -> "BatchPlan":
+        return BatchPlan(self, adapter_ids, long_threshold)
+
+
+class _DevicePtr:
+    """__cuda_array_interface__ wrapper around a raw device address (read-only inspection)."""
+
+    def __init__(self, addr: int, nbytes: int, device: int):
+        self.__cuda_array_interface__ = {"shape": (nbytes,), "typestr": "|u1", "data": (addr, True),
+                                         "version": 3}
+
+
+class BatchPlan:
+    """Segment table + dispatch for one batch (see include/sgmv.h, "Segment builder")."""
+
+    def __init__(self, pool: AdapterPool, adapter_ids, long_threshold: int = 0):
+        lib = load_library()
+        ids = np.ascontiguousarray(np.asarray(adapter_ids, dtype=np.int32).reshape(-1))
+        self.T = int(ids.size)
+        cap = int(lib.sgmv_plan_table_capacity(self.T, len(pool.projections)))
+        pinned = torch.cuda.is_available() and pool.device >= 0
+        self.host = torch.empty(cap, dtype=torch.uint8, pin_memory=pinned)
+        self.plan = Plan()
+        _check(lib.sgmv_build_plan(ids.ctypes.data if self.T else None, self.T, pool.handle, int(long_threshold),
+                                   self.host.data_ptr(), cap, ctypes.byref(self.plan)))
+        self.pool = pool
+        self.device_table: Optional[torch.Tensor] = None
+
+    # -- host views of the table
+    def _arr(self, off: int, count: int, dtype) -> np.ndarray:
+        nbytes = count * np.dtype(dtype).itemsize
+        return self.host.numpy()[off:off + nbytes].view(dtype).copy()
+
+    @property
+    def token_idx(self) -> np.ndarray:
+        return self._arr(self.plan.off_token_idx, self.plan.num_rows, np.int32)
+
+    @property
+    def seg_offsets(self) -> np.ndarray:
+        return self._arr(self.plan.off_seg_offsets, self.plan.num_segments + 1, np.int32)
+
+    @property
+    def seg_adapter(self) -> np.ndarray:
+        return self._arr(self.plan.off_seg_adapter, self.plan.num_segments, np.int32)
+
+    @property
+    def seg_rank(self) -> np.ndarray:
+        return self._arr(self.plan.off_seg_rank, self.plan.num_segments, np.int32)
+
+    def seg_pt(self, matrix: int) -> np.ndarray:
+        off = self.plan.off_seg_a_pt if matrix == 0 else self.plan.off_seg_b_pt
+        return self._arr(off, self.plan.num_segments * self.plan.n_proj, np.int64).reshape(
+            self.plan.num_segments, self.plan.n_proj)
+
+    @property
+    def simt_items(self) -> np.ndarray:
+        return self._arr(self.plan.off_simt_items, 4 * self.plan.num_simt_items, np.int32).reshape(-1, 4)
+
+    @property
+    def tc_tiles(self) -> np.ndarray:
+        return self._arr(self.plan.off_tc_tiles, 4 * self.plan.num_tc_tiles, np.int32).reshape(-1, 4)
+
+    @property
+    def num_rows(self) -> int:
+        return self.plan.num_rows
+
+    @property
+    def max_rank(self) -> int:
+        return self.plan.max_rank
+
+    # -- device side
+    def upload(self, stream=None) -> torch.Tensor:
+        n = max(int(self.plan.table_bytes), 16)
+        dev = torch.device("cuda", self.pool.device)
+        if self.device_table is None or self.device_table.numel() < n:
+            self.device_table = torch.empty(n, dtype=torch.uint8, device=dev)
+        s = torch.cuda.current_stream(dev) if stream is None else stream
+        with torch.cuda.stream(s):
+            self.device_table[:n].copy_(self.host[:n], non_blocking=True)
+        return self.device_table
+
+    def new_v(self, ldv: Optional[int] = None) -> torch.Tensor:
+        ldv = ldv or max(4, (self.plan.max_rank + 3) // 4 * 4)
+        return torch.empty(max(self.plan.num_rows, 1), ldv, dtype=torch.float32,
+                           device=torch.device("cuda", self.pool.device))
+
+
+def shrink(x: torch.Tensor, plan: BatchPlan, pool: AdapterPool, v: torch.Tensor, proj: int = 0,
+           stream=None) -> None:
+    """v[i, k] = sum_c A_s[k, c] x[token_idx[i], c]  (SGMV-shrink)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    assert v.dtype == torch.float32 and v.dim() == 2 and v.stride(1) == 1
+    table = plan.device_table if plan.device_table is not None else plan.upload(stream)
+    _check(load_library().sgmv_shrink(_ptr(x), x.stride(0), plan.T, x.shape[1], int(proj), ctypes.byref(plan.plan),
+                                      table.data_ptr(), pool.handle, _ptr(v), v.stride(0), _stream(stream)))
+
+
+def expand(v: torch.Tensor, plan: BatchPlan, pool: AdapterPool, y: torch.Tensor, proj: int = 0,
+           scale: float = 1.0, stream=None) -> None:
+    """y[t, j] += scale * sum_k B_s[j, k] v[i, k]  (SGMV-expand, in place, one rounding)."""
+    assert v.dtype == torch.float32 and v.dim() == 2 and v.stride(1) == 1
+    assert y.dim() == 2 and y.stride(1) == 1 and y.dtype in (torch.bfloat16, torch.float32)
+    table = plan.device_table if plan.device_table is not None else plan.upload(stream)
+    _check(load_library().sgmv_expand(_ptr(v), v.stride(0), plan.T, y.shape[1], int(proj), ctypes.byref(plan.plan),
+                                      table.data_ptr(), pool.handle, float(scale), _ptr(y), y.stride(0),
+                                      0 if y.dtype == torch.bfloat16 else 1, _stream(stream)))
+
+
+def check_errors(stream=None) -> int:
+    """Wait for the stream; raise SgmvError if a device-side check failed, else return 0."""
+    bits = ctypes.c_uint32()
+    _check(load_library().sgmv_check_errors(_stream(stream), ctypes.byref(bits)))
+    return bits.value
+
+
+def lora_delta(x: torch.Tensor, y: torch.Tensor, plan: BatchPlan, pool: AdapterPool, proj: int = 0,
+               scale: float = 1.0, v: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """y_t += scale * B_{a(t)} A_{a(t)} x_t for every token: shrink then expand on one stream."""
+    if v is None:
+        v = plan.new_v()
+    shrink(x, plan, pool, v, proj, stream)
+    expand(v, plan, pool, y, proj, scale, stream)
+    return v

@@ -1,0 +1,106 @@
+// Library-internal declarations shared by the translation units.
+#pragma once
+#include <cstdint>
+#include <map>
+#include <algorithm>
+#include <string>
+#include <unordered_map>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "../../include/sgmv.h"
+
+namespace sgmv {
+
+// --------------------------------------------------------------- status text
+sgmv_status fail(sgmv_status s, const std::string& msg);
+sgmv_status cuda_fail(cudaError_t e, const char* what);
+#define SGMV_CUDA_TRY(call)                                     \
+    do {                                                        \
+        cudaError_t e__ = (call);                               \
+        if (e__ != cudaSuccess) return ::sgmv::cuda_fail(e__, #call); \
+    } while (0)
+
+// ---------------------------------------------------------------------- pool
+struct AdapterRec {
+    int32_t rank = 0;
+    int64_t pt_begin = 0, pt_count = 0;      // contiguous page-table range
+    std::vector<int64_t> a_pt, b_pt;         // per projection, first entry of A / B^T
+};
+
+}  // namespace sgmv
+
+struct sgmv_pool {
+    int device = -1;
+    int64_t num_pages = 0;
+    int32_t page_elems = 0, page_log2 = 0;
+    int32_t n_proj = 0, max_rank = 0;
+    std::vector<int32_t> d_in, d_out;
+    void* pages_dev = nullptr;       // bf16 [num_pages][page_elems]
+    int32_t* pt_dev = nullptr;       // int32 [pt_capacity]
+    int64_t pt_capacity = 0;
+    std::vector<int32_t> pt_host;    // mirror of the page table
+    std::vector<int64_t> free_pages; // stack of free page ids
+    std::map<int64_t, int64_t> free_pt;  // free page-table ranges: start -> length
+    std::unordered_map<int32_t, sgmv::AdapterRec> adapters;
+    void* staging_dev = nullptr;     // device staging for host-source loads
+    size_t staging_bytes = 0;
+};
+
+namespace sgmv {
+
+// -------------------------------------------------------------- plan tables
+struct Item {
+    int32_t seg, row_begin, row_end, pad;
+};
+static_assert(sizeof(Item) == 16, "Item must be 16 bytes");
+
+constexpr int kSimtMaxItemRows = 64;   // rows per SIMT work item
+constexpr int kTcTileRows = 128;       // rows per tensor-core tile (MMA M)
+constexpr int kDefaultLongThreshold = 64;
+constexpr int kMaxRank = 128;
+
+// Device view of everything a kernel needs about the batch.
+struct BatchView {
+    const int32_t* token_idx;
+    const int32_t* seg_offsets;
+    const int32_t* seg_rank;
+    const int64_t* seg_a_pt;
+    const int64_t* seg_b_pt;
+    const Item* simt_items;
+    const Item* tc_tiles;
+    int32_t num_segments, num_rows, n_proj, proj, T;
+};
+
+struct PoolView {
+    const uint16_t* pages;
+    const int32_t* page_table;
+    int64_t num_pages;
+    int64_t pt_capacity;
+    int32_t page_log2;
+};
+
+// --------------------------------------------------------------- launchers
+cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, const BatchView& b,
+                               int32_t num_items, int32_t max_item_rows, int32_t max_rank, const PoolView& pool,
+                               float* v, int64_t ldv, cudaStream_t stream);
+cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const BatchView& b,
+                               int32_t num_items, int32_t max_item_rows, int32_t max_rank, const PoolView& pool,
+                               float scale, void* y, int64_t ldy, int32_t y_dtype, cudaStream_t stream);
+cudaError_t launch_shrink_tc(const uint16_t* x, int64_t ldx, int32_t d_in, const BatchView& b, int32_t num_tiles,
+                             int32_t max_rank, const PoolView& pool, float* v, int64_t ldv, cudaStream_t stream);
+cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const BatchView& b, int32_t num_tiles,
+                             int32_t max_rank, const PoolView& pool, float scale, void* y, int64_t ldy,
+                             int32_t y_dtype, cudaStream_t stream);
+
+// Read and clear the device error words of every translation unit.
+cudaError_t read_clear_errors_simt(uint32_t* bits, cudaStream_t stream);
+cudaError_t read_clear_errors_tc(uint32_t* bits, cudaStream_t stream);
+
+// Pool scatter kernels (sgmv_pool.cu).
+cudaError_t launch_pool_scatter(const uint16_t* src, int64_t rows, int64_t cols, bool transpose,
+                                const int32_t* page_table, int64_t pt_base, int32_t page_log2,
+                                uint16_t* pages, cudaStream_t stream);
+
+}  // namespace sgmv

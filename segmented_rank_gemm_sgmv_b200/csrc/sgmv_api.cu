@@ -1,0 +1,136 @@
+// C ABI entry points: argument validation, the size-based dispatch between
+// the SIMT and the tensor-core kernels, and error reporting.
+#include <cstdio>
+#include <string>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace sgmv {
+
+namespace {
+thread_local std::string t_last_error;
+}
+
+sgmv_status fail(sgmv_status s, const std::string& msg) {
+    t_last_error = msg;
+    return s;
+}
+
+sgmv_status cuda_fail(cudaError_t e, const char* what) {
+    t_last_error = std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
+    return SGMV_ERR_CUDA;
+}
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+sgmv_status make_views(const sgmv_plan* plan, const void* table, const sgmv_pool* pool, int32_t T, int32_t proj,
+                       BatchView* bv, PoolView* pv, const char* who) {
+    const std::string w(who);
+    if (!plan || !pool) return fail(SGMV_ERR_INVALID, w + ": plan and pool are required");
+    if (pool->device < 0 || !pool->pages_dev) return fail(SGMV_ERR_INVALID, w + ": pool has no device memory");
+    if (plan->T != T) return fail(SGMV_ERR_INVALID, w + ": T differs from the plan's T");
+    if (plan->n_proj != pool->n_proj) return fail(SGMV_ERR_INVALID, w + ": plan was built for another pool");
+    if (proj < 0 || proj >= pool->n_proj) return fail(SGMV_ERR_INVALID, w + ": projection index out of range");
+    if (plan->table_bytes > 0 && (!table || !aligned16(table)))
+        return fail(SGMV_ERR_INVALID, w + ": table must be a 16-byte aligned device pointer");
+    const uint8_t* base = static_cast<const uint8_t*>(table);
+    bv->token_idx = reinterpret_cast<const int32_t*>(base + plan->off_token_idx);
+    bv->seg_offsets = reinterpret_cast<const int32_t*>(base + plan->off_seg_offsets);
+    bv->seg_rank = reinterpret_cast<const int32_t*>(base + plan->off_seg_rank);
+    bv->seg_a_pt = reinterpret_cast<const int64_t*>(base + plan->off_seg_a_pt);
+    bv->seg_b_pt = reinterpret_cast<const int64_t*>(base + plan->off_seg_b_pt);
+    bv->simt_items = reinterpret_cast<const Item*>(base + plan->off_simt_items);
+    bv->tc_tiles = reinterpret_cast<const Item*>(base + plan->off_tc_tiles);
+    bv->num_segments = plan->num_segments;
+    bv->num_rows = plan->num_rows;
+    bv->n_proj = plan->n_proj;
+    bv->proj = proj;
+    bv->T = T;
+    pv->pages = static_cast<const uint16_t*>(pool->pages_dev);
+    pv->page_table = pool->pt_dev;
+    pv->num_pages = pool->num_pages;
+    pv->pt_capacity = pool->pt_capacity;
+    pv->page_log2 = pool->page_log2;
+    return SGMV_OK;
+}
+
+}  // namespace
+}  // namespace sgmv
+
+using namespace sgmv;
+
+extern "C" const char* sgmv_status_string(sgmv_status s) {
+    switch (s) {
+        case SGMV_OK: return "SGMV_OK";
+        case SGMV_ERR_INVALID: return "SGMV_ERR_INVALID";
+        case SGMV_ERR_UNSUPPORTED: return "SGMV_ERR_UNSUPPORTED";
+        case SGMV_ERR_NOT_RESIDENT: return "SGMV_ERR_NOT_RESIDENT";
+        case SGMV_ERR_OUT_OF_PAGES: return "SGMV_ERR_OUT_OF_PAGES";
+        case SGMV_ERR_CUDA: return "SGMV_ERR_CUDA";
+        case SGMV_ERR_BOUNDS: return "SGMV_ERR_BOUNDS";
+        case SGMV_ERR_TIMEOUT: return "SGMV_ERR_TIMEOUT";
+        case SGMV_ERR_CAPACITY: return "SGMV_ERR_CAPACITY";
+    }
+    return "SGMV_ERR_UNKNOWN";
+}
+
+extern "C" const char* sgmv_last_error(void) { return t_last_error.c_str(); }
+
+extern "C" sgmv_status sgmv_shrink(const void* x, int64_t ldx, int32_t T, int32_t d_in, int32_t proj,
+                                   const sgmv_plan* plan, const void* table, const sgmv_pool* pool, float* v,
+                                   int64_t ldv, sgmv_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    BatchView bv;
+    PoolView pv;
+    sgmv_status st = make_views(plan, table, pool, T, proj, &bv, &pv, "shrink");
+    if (st != SGMV_OK) return st;
+    if (d_in != pool->d_in[proj]) return fail(SGMV_ERR_INVALID, "shrink: d_in differs from the pool's projection");
+    if (plan->num_rows == 0 || (plan->num_simt_items == 0 && plan->num_tc_tiles == 0)) return SGMV_OK;
+    if (!x || !v) return fail(SGMV_ERR_INVALID, "shrink: x and v are required");
+    if (ldx < d_in || (ldx % 8) || !aligned16(x)) return fail(SGMV_ERR_INVALID, "shrink: x rows must be 16-byte aligned, ldx >= d_in");
+    if (ldv < plan->max_rank || ldv < 1 || (ldv % 4) || !aligned16(v))
+        return fail(SGMV_ERR_INVALID, "shrink: v needs ldv >= max_rank, ldv % 4 == 0, 16-byte alignment");
+    const uint16_t* xb = static_cast<const uint16_t*>(x);
+    SGMV_CUDA_TRY(launch_shrink_simt(xb, ldx, d_in, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, pv,
+                                     v, ldv, stream));
+    SGMV_CUDA_TRY(launch_shrink_tc(xb, ldx, d_in, bv, plan->num_tc_tiles, plan->max_rank, pv, v, ldv, stream));
+    return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_expand(const float* v, int64_t ldv, int32_t T, int32_t d_out, int32_t proj,
+                                   const sgmv_plan* plan, const void* table, const sgmv_pool* pool, float scale,
+                                   void* y, int64_t ldy, int32_t y_dtype, sgmv_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    BatchView bv;
+    PoolView pv;
+    sgmv_status st = make_views(plan, table, pool, T, proj, &bv, &pv, "expand");
+    if (st != SGMV_OK) return st;
+    if (d_out != pool->d_out[proj]) return fail(SGMV_ERR_INVALID, "expand: d_out differs from the pool's projection");
+    if (y_dtype != 0 && y_dtype != 1) return fail(SGMV_ERR_INVALID, "expand: y_dtype must be 0 (bf16) or 1 (fp32)");
+    if (plan->num_rows == 0 || (plan->num_simt_items == 0 && plan->num_tc_tiles == 0)) return SGMV_OK;
+    if (!v || !y) return fail(SGMV_ERR_INVALID, "expand: v and y are required");
+    const int64_t esz = y_dtype == 0 ? 2 : 4;
+    if (ldy < d_out || ((ldy * esz) % 16) || !aligned16(y))
+        return fail(SGMV_ERR_INVALID, "expand: y rows must be 16-byte aligned, ldy >= d_out");
+    if (ldv < plan->max_rank || ldv < 1 || (ldv % 4) || !aligned16(v))
+        return fail(SGMV_ERR_INVALID, "expand: v needs ldv >= max_rank, ldv % 4 == 0, 16-byte alignment");
+    SGMV_CUDA_TRY(launch_expand_simt(v, ldv, d_out, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, pv,
+                                     scale, y, ldy, y_dtype, stream));
+    SGMV_CUDA_TRY(launch_expand_tc(v, ldv, d_out, bv, plan->num_tc_tiles, plan->max_rank, pv, scale, y, ldy, y_dtype,
+                                   stream));
+    return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_check_errors(sgmv_stream_t stream_, uint32_t* flags) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    uint32_t bits = 0;
+    SGMV_CUDA_TRY(read_clear_errors_simt(&bits, stream));
+    SGMV_CUDA_TRY(read_clear_errors_tc(&bits, stream));
+    if (flags) *flags = bits;
+    if (bits & kErrTimeout) return fail(SGMV_ERR_TIMEOUT, "a device-side wait timed out");
+    if (bits) return fail(SGMV_ERR_BOUNDS, "a device-side bounds check failed");
+    return SGMV_OK;
+}

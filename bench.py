@@ -1,0 +1,441 @@
+"""Benchmark of the multi-LoRA delta (SGMV shrink + expand) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one pass of the whole hot path over one batch: the host segment
+builder (run every step, overlapped with the previous device work), one
+host-to-device copy of the segment table, then SGMV-shrink and SGMV-expand for
+every adapted projection of the workload.  The device time of a step (CUDA
+events on the launching stream, from the table copy to the last expand) is
+what `value` measures; L2 is flushed (a 512 MiB write) between steps, outside
+the timed windows.  `e2e` repeats the step through the same public API with
+host buffers: the step's x and y rows go host->device from pinned memory and y
+comes back device->host, all inside the timed window, with the host builder.
+
+With N > 1 (torchrun) every rank runs its own batch of the same shape (weak
+scaling, no collective on the data path: the tokens of a batch are
+independent); the reported time is the max over ranks.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "LoRA-delta tokens/s per adapted layer; SGMV achieved HBM GB/s vs B200 peak"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 512 << 20
+
+
+# ---------------------------------------------------------------------------- helpers
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(wl: workloads.Workload, proj: int):
+    """Minimum bytes of one shrink and one expand: each distinct adapter's A and B
+    once, x read once, v written and read in fp32, y read and written."""
+    _, d_in, d_out = wl.projections[proj]
+    ids = wl.adapter_ids[wl.adapter_ids >= 0]
+    distinct = np.unique(ids)
+    r_of = {int(a): wl.rank_of(int(a)) for a in distinct}
+    sum_r_adapters = sum(r_of.values())
+    rows = [t for t in range(wl.T) if wl.adapter_ids[t] >= 0 and r_of[int(wl.adapter_ids[t])] > 0]
+    sum_r_tokens = sum(r_of[int(wl.adapter_ids[t])] for t in rows)
+    shrink = 2 * sum_r_adapters * d_in + 2 * len(rows) * d_in + 4 * sum_r_tokens
+    expand = 2 * sum_r_adapters * d_out + 4 * sum_r_tokens + 4 * len(rows) * d_out
+    flops = 2 * sum_r_tokens * (d_in + d_out)
+    return shrink, expand, flops
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report what is known
+            self.err = str(e)
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                for b, name in self.REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def read_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when the
+    kernel sources changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "segmented_rank_gemm_sgmv_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    digest = h.hexdigest()[:16]
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) == 4 and parts[0] == workload and parts[1] == kernel and parts[3] == digest:
+                return float(parts[2])
+    return None
+
+
+# ---------------------------------------------------------------------------- our arm
+def setup(wl_name: str, rank: int, device: int):
+    import segmented_rank_gemm_sgmv_b200 as sg
+    wl = workloads.make(wl_name, seed=rank)
+    bank = workloads.AdapterBank(wl, device=f"cuda:{device}")
+    projs = [(d_in, d_out) for _, d_in, d_out in wl.projections]
+    need = sum(sg.AdapterPool.pages_needed(projs, int(r)) for r in wl.pool_ranks)
+    pool = sg.AdapterPool(projs, num_pages=need + 64, page_elems=512,
+                          max_rank=max(16, int(wl.pool_ranks.max())), device=device)
+    pool.shuffle_free_pages(1234 + rank)
+    for a, r in zip(wl.pool_ids.tolist(), wl.pool_ranks.tolist()):
+        A, B = zip(*[bank.get(a, p) for p in range(len(projs))])
+        pool.load(a, int(r), list(A), list(B))
+    acts = [workloads.activations(wl, p, device=f"cuda:{device}") for p in range(len(projs))]
+    del bank
+    torch.cuda.empty_cache()
+    return sg, wl, pool, acts
+
+
+def run_ours(args, rank, world, device):
+    sg, wl, pool, acts = setup(args.workload, rank, device)
+    n_proj = len(wl.projections)
+    stream = torch.cuda.current_stream(device)
+    plans = [sg.BatchPlan(pool, capacity_tokens=wl.T) for _ in range(2)]
+    for pl in plans:
+        pl.build(wl.adapter_ids)
+        pl.upload(stream)
+    v = plans[0].new_v()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=f"cuda:{device}")
+    ys = [y for _, y in acts]
+
+    def step(i, evs=None):
+        pl = plans[i % 2]
+        pl.build(wl.adapter_ids)                     # host segment builder + dispatch
+        if evs:
+            evs[0].record(stream)
+        table = pl.upload(stream)                    # one host->device copy of the table
+        k = 1
+        for p in range(n_proj):
+            x, y = acts[p]
+            if evs:
+                evs[k].record(stream)
+            sg.shrink(x, pl, pool, v, p, stream)
+            if evs:
+                evs[k + 1].record(stream)
+            sg.expand(v, pl, pool, y, p, wl.scale, stream)
+            k += 2
+        if evs:
+            evs[k].record(stream)
+        return table
+
+    n_ev = 2 + 2 * n_proj
+    for i in range(args.warmup):
+        flush.zero_()
+        step(i)
+    sg.check_errors(stream)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    records = []
+    with ClockSampler(device) as clk:
+        for i in range(args.steps):
+            flush.zero_()                            # L2 flush, outside the timed window
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+            step(i, evs)
+            records.append(evs)
+        torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    sg.check_errors(stream)
+    step_ms = [e[0].elapsed_time(e[-1]) for e in records]
+    shrink_ms = [sum(e[1 + 2 * p].elapsed_time(e[2 + 2 * p]) for p in range(n_proj)) for e in records]
+    expand_ms = [sum(e[2 + 2 * p].elapsed_time(e[3 + 2 * p]) for p in range(n_proj)) for e in records]
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=f"cuda:{device}")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # roofline of the dominant kernel (the phase with the larger device time)
+    shrink_b = expand_b = flops = 0
+    for p in range(n_proj):
+        s_b, e_b, f = algorithmic_bytes(wl, p)
+        shrink_b += s_b
+        expand_b += e_b
+        flops += f
+    peak, peak_kind = measured_peaks()
+    per = {"shrink": (float(np.mean(shrink_ms)), shrink_b), "expand": (float(np.mean(expand_ms)), expand_b)}
+    dom = max(per, key=lambda k: per[k][0])
+    launches_per_phase = n_proj * (int(plans[0].plan.num_simt_items > 0) + int(plans[0].plan.num_tc_tiles > 0))
+    dom_ms, dom_bytes = per[dom]
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    traffic_total = read_traffic(args.workload, dom)
+    res = dict(total_ms=total_ms, step_ms=step_ms, per=per, dom=dom, achieved=achieved, peak=peak,
+               peak_kind=peak_kind, launches=plans[0].launches(n_proj), clocks=clk.summary(),
+               step_bytes=shrink_b + expand_b, flops=flops, launches_per_phase=launches_per_phase,
+               traffic=traffic_total, plan=plans[0].plan)
+
+    # end to end through the public API with host buffers
+    res["e2e"] = e2e_ours(sg, wl, pool, acts, args, device, stream, world)
+    return wl, res
+
+
+def e2e_ours(sg, wl, pool, acts, args, device, stream, world):
+    n_proj = len(wl.projections)
+    host_x = [x.cpu().pin_memory() for x, _ in acts]
+    host_y = [y.cpu().pin_memory() for _, y in acts]
+    dev_x = [torch.empty_like(x) for x, _ in acts]
+    dev_y = [torch.empty_like(y) for _, y in acts]
+    out_y = [torch.empty_like(h).pin_memory() for h in host_y]
+    plan = sg.BatchPlan(pool, capacity_tokens=wl.T)
+    v = None
+    h2d = d2h = 0
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=f"cuda:{device}")
+
+    def one(timed):
+        nonlocal v, h2d, d2h
+        b_in = b_out = 0
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        plan.build(wl.adapter_ids)
+        plan.upload(stream)
+        b_in += int(plan.plan.table_bytes)
+        if v is None:
+            v = plan.new_v()
+        for p in range(n_proj):
+            dev_x[p].copy_(host_x[p], non_blocking=True)
+            dev_y[p].copy_(host_y[p], non_blocking=True)
+            b_in += host_x[p].numel() * 2 + host_y[p].numel() * 2
+            sg.shrink(dev_x[p], plan, pool, v, p, stream)
+            sg.expand(v, plan, pool, dev_y[p], p, wl.scale, stream)
+            out_y[p].copy_(dev_y[p], non_blocking=True)
+            b_out += out_y[p].numel() * 2
+        e1.record(stream)
+        e1.synchronize()
+        h2d, d2h = b_in, b_out
+        return e0.elapsed_time(e1)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        torch.cuda.synchronize(device)
+        one(False)
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        torch.cuda.synchronize(device)
+        times.append(one(True))
+    total = float(sum(times))
+    if world > 1:
+        t = torch.tensor([total], dtype=torch.float64, device=f"cuda:{device}")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total = float(t.item())
+    return dict(total_ms=total, h2d=h2d, d2h=d2h)
+
+
+# ---------------------------------------------------------------------------- oracle arm
+def oracle_inputs(wl, device):
+    """fp64 host copies of the batch's inputs (x, y, A, B of the adapters in use)."""
+    bank = workloads.AdapterBank(wl, device=device)
+    import oracle
+    tix, off, seg_ad = oracle.group_by_adapter(wl.adapter_ids.tolist())
+    per_proj = []
+    for p in range(len(wl.projections)):
+        x, y = workloads.activations(wl, p, device=device)
+        A = [workloads.bf16_to_f64(bank.get(a, p)[0]) for a in seg_ad]
+        B = [workloads.bf16_to_f64(bank.get(a, p)[1]) for a in seg_ad]
+        per_proj.append((workloads.bf16_to_f64(x), workloads.bf16_to_f64(y), A, B))
+    ranks = [wl.rank_of(a) for a in seg_ad]
+    del bank
+    return tix, off, ranks, per_proj
+
+
+def time_oracle(prepared, wl, budget_s: float, threads: int):
+    """Run the oracle over the whole batch (all projections) until about budget_s
+    seconds have passed; returns (tokens/s, reps, elapsed, threads used)."""
+    import oracle
+    tix, off, ranks, per_proj = prepared
+    used = oracle.threads_used(threads)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        for x, y, A, B in per_proj:
+            oracle.lora_delta(x, y, off, ranks, A, B, token_idx=tix, scale=wl.scale, threads=threads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return len(tix) * reps / el, reps, el, used
+
+
+def run_reference(args, rank, world, device):
+    if rank != 0:
+        return
+    wl = workloads.make(args.workload, seed=0)
+    threads = os.cpu_count() or 1
+    dev = f"cuda:{device}" if torch.cuda.is_available() else "cpu"
+    prepared = oracle_inputs(wl, dev)
+    for _ in range(args.warmup):
+        time_oracle(prepared, wl, 0.0, threads)
+    per_step_budget = max(0.05, 60.0 / max(args.steps, 1))
+    t_all, reps_all, used = 0.0, 0, 1
+    for _ in range(args.steps):
+        _, reps, el, used = time_oracle(prepared, wl, per_step_budget, threads)
+        t_all += el
+        reps_all += reps
+    n_tok = len(prepared[0])
+    value = reps_all * n_tok / t_all
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_all / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(wl),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
+                             "sample": f"whole batch ({n_tok} tokens x {len(wl.projections)} projections) "
+                                       f"repeated {reps_all} times over {args.steps} steps"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl):
+    ranks = sorted(set(int(wl.rank_of(a)) for a in np.unique(wl.adapter_ids[wl.adapter_ids >= 0])))
+    return {"workload": wl.name, "tokens": wl.T,
+            "projections": [f"{n}:{a}->{b}" for n, a, b in wl.projections],
+            "ranks": ranks, "pool_adapters": int(wl.pool_ids.size),
+            "distinct_adapters": wl.distinct_adapters, "page_elems": 512,
+            "l2": "flushed between steps (512 MiB write outside the timed window)",
+            "parallelism": "replicas"}
+
+
+# ---------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode_q_proj", choices=workloads.WORKLOAD_NAMES)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        if torch.cuda.is_available():
+            torch.cuda.set_device(0)
+
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world, local)
+            return
+        wl, res = run_ours(args, rank, world, local)
+        if rank != 0:
+            return
+        n_tok = int((wl.adapter_ids >= 0).sum())
+        value = world * n_tok * args.steps / (res["total_ms"] * 1e-3)
+        e2e = res["e2e"]
+        e2e_value = world * n_tok * args.steps / (e2e["total_ms"] * 1e-3)
+        dom_ms, dom_bytes = res["per"][res["dom"]]
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res["total_ms"] / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_of(wl),
+            "hbm_gbs_step": res["step_bytes"] / (res["total_ms"] / args.steps * 1e-3) / 1e9,
+            "phases_ms": {k: v[0] for k, v in res["per"].items()},
+            "roofline": {"bound": "hbm", "kernel": f"sgmv_{res['dom']}", "achieved": res["achieved"],
+                         "peak": res["peak"], "unit": "GB/s", "frac": res["achieved"] / res["peak"],
+                         "peak_source": f"{res['peak_kind']} (MEASURED_PEAKS.json hbm_gbs)" if res["peak_kind"] ==
+                         "measured" else "fallback 6650 GB/s",
+                         "algorithmic_bytes_per_step": dom_bytes,
+                         "launches_per_step": res["launches_per_phase"],
+                         "traffic": res["traffic"]},
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
+                    "d2h_bytes_per_step": e2e["d2h"]},
+            "gpu_launches": res["launches"] * args.steps,
+            "clocks": res["clocks"],
+        }
+        if not args.no_cpu_baseline and world == 1:
+            prepared = oracle_inputs(wl, f"cuda:{local}")
+            rate, reps, el, used = time_oracle(prepared, wl, args.cpu_budget, os.cpu_count() or 1)
+            line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": used, "kind": "oracle",
+                                    "sample": f"whole batch ({n_tok} tokens x {len(wl.projections)} projections)"
+                                              f" repeated {reps} times in {el:.1f} s"}
+        print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -218,25 +218,44 @@ class _DevicePtr:
     """__cuda_array_interface__ wrapper around a raw device address (read-only inspection)."""
 
     def __init__(self, addr: int, nbytes: int, device: int):
-        self.__cuda_array_interface__ = {"shape": (nbytes,), "typestr": "|u1", "data": (addr, True),
+        self.__cuda_array_interface__ = {"shape": (nbytes,), "typestr": "|u1", "data": (addr, False),
                                          "version": 3}
 
 
 class BatchPlan:
-    """Segment table + dispatch for one batch (see include/sgmv.h, "Segment builder")."""
+    """Segment table + dispatch for one batch (see include/sgmv.h, "Segment builder").
 
-    def __init__(self, pool: AdapterPool, adapter_ids, long_threshold: int = 0):
-        lib = load_library()
-        ids = np.ascontiguousarray(np.asarray(adapter_ids, dtype=np.int32).reshape(-1))
-        self.T = int(ids.size)
-        cap = int(lib.sgmv_plan_table_capacity(self.T, len(pool.projections)))
-        pinned = torch.cuda.is_available() and pool.device >= 0
-        self.host = torch.empty(cap, dtype=torch.uint8, pin_memory=pinned)
-        self.plan = Plan()
-        _check(lib.sgmv_build_plan(ids.ctypes.data if self.T else None, self.T, pool.handle, int(long_threshold),
-                                   self.host.data_ptr(), cap, ctypes.byref(self.plan)))
+    The host table lives in pinned memory and the device copy in a device buffer,
+    both reused by later build() calls; build() first waits for the previous
+    upload from the host buffer to finish, so a plan can be rebuilt every step.
+    """
+
+    def __init__(self, pool: AdapterPool, adapter_ids=None, long_threshold: int = 0,
+                 capacity_tokens: Optional[int] = None):
         self.pool = pool
+        self.long_threshold = int(long_threshold)
+        ids = None if adapter_ids is None else np.asarray(adapter_ids, dtype=np.int32).reshape(-1)
+        cap_t = capacity_tokens if capacity_tokens is not None else (0 if ids is None else ids.size)
+        self.capacity = int(load_library().sgmv_plan_table_capacity(int(cap_t), len(pool.projections)))
+        pinned = torch.cuda.is_available() and pool.device >= 0
+        self.host = torch.empty(self.capacity, dtype=torch.uint8, pin_memory=pinned)
+        self.plan = Plan()
         self.device_table: Optional[torch.Tensor] = None
+        self._uploaded: Optional[torch.cuda.Event] = None
+        self.T = 0
+        if ids is not None:
+            self.build(ids)
+
+    def build(self, adapter_ids, long_threshold: Optional[int] = None) -> "BatchPlan":
+        ids = np.ascontiguousarray(np.asarray(adapter_ids, dtype=np.int32).reshape(-1))
+        if self._uploaded is not None:
+            self._uploaded.synchronize()      # the previous upload has read the host buffer
+        lt = self.long_threshold if long_threshold is None else int(long_threshold)
+        _check(load_library().sgmv_build_plan(ids.ctypes.data if ids.size else None, int(ids.size),
+                                              self.pool.handle, lt, self.host.data_ptr(), self.capacity,
+                                              ctypes.byref(self.plan)))
+        self.T = int(ids.size)
+        return self
 
     # -- host views of the table
     def _arr(self, off: int, count: int, dtype) -> np.ndarray:
@@ -280,15 +299,24 @@ class BatchPlan:
     def max_rank(self) -> int:
         return self.plan.max_rank
 
+    def launches(self, projections: int = 1) -> int:
+        """Kernel launches one shrink + expand pass makes per projection, times `projections`."""
+        per = 2 * (int(self.plan.num_simt_items > 0) + int(self.plan.num_tc_tiles > 0))
+        return per * projections
+
     # -- device side
     def upload(self, stream=None) -> torch.Tensor:
+        """Copy the table to the device on `stream` (one host-to-device copy)."""
         n = max(int(self.plan.table_bytes), 16)
         dev = torch.device("cuda", self.pool.device)
-        if self.device_table is None or self.device_table.numel() < n:
-            self.device_table = torch.empty(n, dtype=torch.uint8, device=dev)
+        if self.device_table is None or self.device_table.numel() < max(n, self.capacity):
+            self.device_table = torch.empty(max(n, self.capacity), dtype=torch.uint8, device=dev)
         s = torch.cuda.current_stream(dev) if stream is None else stream
         with torch.cuda.stream(s):
             self.device_table[:n].copy_(self.host[:n], non_blocking=True)
+            if self._uploaded is None:
+                self._uploaded = torch.cuda.Event()
+            self._uploaded.record(s)
         return self.device_table
 
     def new_v(self, ldv: Optional[int] = None) -> torch.Tensor:

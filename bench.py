@@ -64,7 +64,7 @@ def algorithmic_bytes(wl: workloads.Workload, proj: int):
     shrink = 2 * sum_r_adapters * d_in + 2 * len(rows) * d_in + 4 * sum_r_tokens
     expand = 2 * sum_r_adapters * d_out + 4 * sum_r_tokens + 4 * len(rows) * d_out
     flops = 2 * sum_r_tokens * (d_in + d_out)
-    return shrink, expand, flops
+    return shrink, expand, flops, 4 * sum_r_tokens
 
 
 class ClockSampler:
@@ -170,29 +170,34 @@ def run_ours(args, rank, world, device):
         pl.upload(stream)
     v = plans[0].new_v()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=f"cuda:{device}")
-    ys = [y for _, y in acts]
+    # Hold the stream for ~200 us after the flush so that the host has enqueued the
+    # whole step before the device reaches it: event times are then device times.
+    gate_cycles = int(2e-4 * 2.0e9)
+    split = args.split_phases
 
     def step(i, evs=None):
         pl = plans[i % 2]
         pl.build(wl.adapter_ids)                     # host segment builder + dispatch
         if evs:
             evs[0].record(stream)
-        table = pl.upload(stream)                    # one host->device copy of the table
-        k = 1
+        pl.upload(stream)                            # one host->device copy of the table
         for p in range(n_proj):
             x, y = acts[p]
             if evs:
-                evs[k].record(stream)
-            sg.shrink(x, pl, pool, v, p, stream)
+                evs[1 + 3 * p].record(stream)
+            if split:                                # an event between the phases (no launch overlap)
+                sg.shrink(x, pl, pool, v, p, stream)
+                if evs:
+                    evs[2 + 3 * p].record(stream)
+                sg.expand(v, pl, pool, y, p, wl.scale, stream)
+            else:                                    # shrink, then expand overlapping it (PDL)
+                sg.lora_delta(x, pl, pool, y, p, wl.scale, v=v, stream=stream)
             if evs:
-                evs[k + 1].record(stream)
-            sg.expand(v, pl, pool, y, p, wl.scale, stream)
-            k += 2
+                evs[3 + 3 * p].record(stream)
         if evs:
-            evs[k].record(stream)
-        return table
+            evs[-1].record(stream)
 
-    n_ev = 2 + 2 * n_proj
+    n_ev = 2 + 3 * n_proj
     for i in range(args.warmup):
         flush.zero_()
         step(i)
@@ -204,6 +209,7 @@ def run_ours(args, rank, world, device):
     with ClockSampler(device) as clk:
         for i in range(args.steps):
             flush.zero_()                            # L2 flush, outside the timed window
+            torch.cuda._sleep(gate_cycles)
             evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
             step(i, evs)
             records.append(evs)
@@ -213,34 +219,34 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize(device)
     sg.check_errors(stream)
     step_ms = [e[0].elapsed_time(e[-1]) for e in records]
-    shrink_ms = [sum(e[1 + 2 * p].elapsed_time(e[2 + 2 * p]) for p in range(n_proj)) for e in records]
-    expand_ms = [sum(e[2 + 2 * p].elapsed_time(e[3 + 2 * p]) for p in range(n_proj)) for e in records]
+    proj_ms = [sum(e[1 + 3 * p].elapsed_time(e[3 + 3 * p]) for p in range(n_proj)) for e in records]
     total_ms = float(sum(step_ms))
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=f"cuda:{device}")
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         total_ms = float(t.item())
 
-    # roofline of the dominant kernel (the phase with the larger device time)
     shrink_b = expand_b = flops = 0
     for p in range(n_proj):
-        s_b, e_b, f = algorithmic_bytes(wl, p)
+        s_b, e_b, f, _ = algorithmic_bytes(wl, p)
         shrink_b += s_b
         expand_b += e_b
         flops += f
     peak, peak_kind = measured_peaks()
-    per = {"shrink": (float(np.mean(shrink_ms)), shrink_b), "expand": (float(np.mean(expand_ms)), expand_b)}
-    dom = max(per, key=lambda k: per[k][0])
-    launches_per_phase = n_proj * (int(plans[0].plan.num_simt_items > 0) + int(plans[0].plan.num_tc_tiles > 0))
-    dom_ms, dom_bytes = per[dom]
-    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
-    traffic_total = read_traffic(args.workload, dom)
-    res = dict(total_ms=total_ms, step_ms=step_ms, per=per, dom=dom, achieved=achieved, peak=peak,
-               peak_kind=peak_kind, launches=plans[0].launches(n_proj), clocks=clk.summary(),
-               step_bytes=shrink_b + expand_b, flops=flops, launches_per_phase=launches_per_phase,
-               traffic=traffic_total, plan=plans[0].plan)
-
-    # end to end through the public API with host buffers
+    plan0 = plans[0].plan
+    simt, tc = plan0.num_simt_items > 0, plan0.num_tc_tiles > 0
+    kinds = [k for k, on in (("simt", simt), ("tc", tc)) if on]
+    names = " + ".join(f"shrink_{k}_kernel" for k in kinds) + " + " + " + ".join(f"expand_{k}_kernel" for k in kinds)
+    res = dict(total_ms=total_ms, proj_ms=float(np.mean(proj_ms)), kernel_name=f"sgmv_lora_delta ({names})",
+               step_bytes=shrink_b + expand_b, flops=flops, peak=peak, peak_kind=peak_kind,
+               launches=2 * n_proj * len(kinds), clocks=clk.summary(), dom_launches=n_proj,
+               traffic=read_traffic(args.workload, "lora_delta"), split=split)
+    if split:
+        res["phase_ms"] = {"shrink": float(np.mean([sum(e[1 + 3 * p].elapsed_time(e[2 + 3 * p]) for p in range(n_proj))
+                                                    for e in records])),
+                           "expand": float(np.mean([sum(e[2 + 3 * p].elapsed_time(e[3 + 3 * p]) for p in range(n_proj))
+                                                    for e in records]))}
+    res["achieved"] = res["step_bytes"] / (res["proj_ms"] * 1e-3) / 1e9
     res["e2e"] = e2e_ours(sg, wl, pool, acts, args, device, stream, world)
     return wl, res
 
@@ -271,8 +277,7 @@ def e2e_ours(sg, wl, pool, acts, args, device, stream, world):
             dev_x[p].copy_(host_x[p], non_blocking=True)
             dev_y[p].copy_(host_y[p], non_blocking=True)
             b_in += host_x[p].numel() * 2 + host_y[p].numel() * 2
-            sg.shrink(dev_x[p], plan, pool, v, p, stream)
-            sg.expand(v, plan, pool, dev_y[p], p, wl.scale, stream)
+            v = sg.lora_delta(dev_x[p], plan, pool, dev_y[p], p, wl.scale, v=v, stream=stream)
             out_y[p].copy_(dev_y[p], non_blocking=True)
             b_out += out_y[p].numel() * 2
         e1.record(stream)
@@ -378,6 +383,8 @@ def main():
     ap.add_argument("--workload", default="decode_q_proj", choices=workloads.WORKLOAD_NAMES)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--split-phases", action="store_true",
+                    help="record an event between shrink and expand (times each phase; removes their overlap)")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -405,26 +412,26 @@ def main():
         value = world * n_tok * args.steps / (res["total_ms"] * 1e-3)
         e2e = res["e2e"]
         e2e_value = world * n_tok * args.steps / (e2e["total_ms"] * 1e-3)
-        dom_ms, dom_bytes = res["per"][res["dom"]]
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["total_ms"] / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config_of(wl),
             "hbm_gbs_step": res["step_bytes"] / (res["total_ms"] / args.steps * 1e-3) / 1e9,
-            "phases_ms": {k: v[0] for k, v in res["per"].items()},
-            "roofline": {"bound": "hbm", "kernel": f"sgmv_{res['dom']}", "achieved": res["achieved"],
+            "roofline": {"bound": "hbm", "kernel": res["kernel_name"], "achieved": res["achieved"],
                          "peak": res["peak"], "unit": "GB/s", "frac": res["achieved"] / res["peak"],
-                         "peak_source": f"{res['peak_kind']} (MEASURED_PEAKS.json hbm_gbs)" if res["peak_kind"] ==
-                         "measured" else "fallback 6650 GB/s",
-                         "algorithmic_bytes_per_step": dom_bytes,
-                         "launches_per_step": res["launches_per_phase"],
+                         "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if res["peak_kind"] == "measured"
+                         else "fallback 6650 GB/s",
+                         "algorithmic_bytes_per_step": res["step_bytes"],
+                         "launches_per_step": res["dom_launches"],
                          "traffic": res["traffic"]},
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
                     "d2h_bytes_per_step": e2e["d2h"]},
             "gpu_launches": res["launches"] * args.steps,
             "clocks": res["clocks"],
         }
+        if "phase_ms" in res:
+            line["phase_ms"] = res["phase_ms"]
         if not args.no_cpu_baseline and world == 1:
             prepared = oracle_inputs(wl, f"cuda:{local}")
             rate, reps, el, used = time_oracle(prepared, wl, args.cpu_budget, os.cpu_count() or 1)

@@ -178,15 +178,17 @@ SGMV_API const void* sgmv_pool_pages_device(const sgmv_pool* pool);
  *   seg_rank    int32 [num_segments]
  *   seg_a_pt    int64 [num_segments*n_proj]  first page-table entry of A, per projection
  *   seg_b_pt    int64 [num_segments*n_proj]  first page-table entry of B^T
- *   simt_items  int32x4 [num_simt_items] {segment, row_begin, row_end, 0}
- *   tc_tiles    int32x4 [num_tc_tiles]   {segment, row_begin, row_end, 0}, <= 128 rows
+ *   simt_items  record [num_simt_items][n_proj]
+ *   tc_tiles    record [num_tc_tiles][n_proj]   (<= 128 rows each)
+ *               record = {int32 segment, row_begin, row_end, rank;
+ *                         int64 first page-table entry of A, of B^T (for that projection)}
  *
  * Segments are in ascending adapter id; rows of a segment keep batch order
  * (stable).  Tokens with adapter id -1 are in no segment and their y rows
  * are never touched.  Segments of rank 0 produce no work item.  A segment
  * with at least `long_threshold` rows goes to the tensor-core path as
  * 128-row tiles; shorter segments go to the SIMT path as items of at most
- * 64 rows (long_threshold <= 0 selects the built-in default; a huge value
+ * 8 rows (long_threshold <= 0 selects the built-in default, 16; a huge value
  * keeps every segment on the SIMT path; 1 sends every segment to tensor cores).
  */
 typedef struct {
@@ -233,7 +235,8 @@ SGMV_API sgmv_status sgmv_build_plan(const int32_t* adapter_ids, int32_t T, cons
  * proj    projection index, d_in must equal the pool's d_in[proj]
  * table   device copy of the table that built `plan`
  * One launch covers every SIMT item (all short segments, any mix of ranks)
- * and one more covers every tensor-core tile, in stream order.
+ * and one more covers every tensor-core tile, in stream order.  The SIMT
+ * path needs the pool's page_elems <= 1024 (else SGMV_ERR_UNSUPPORTED).
  */
 SGMV_API sgmv_status sgmv_shrink(const void* x, int64_t ldx, int32_t T, int32_t d_in, int32_t proj,
                         const sgmv_plan* plan, const void* table, const sgmv_pool* pool,
@@ -250,11 +253,34 @@ SGMV_API sgmv_status sgmv_shrink(const void* x, int64_t ldx, int32_t T, int32_t 
  * y        device [T][ldy] updated in place, ldy >= d_out, rows 16-byte aligned;
  *          y_dtype 0 = bf16 (round to nearest even), 1 = fp32.
  * Rows of tokens in no segment are not read or written.
+ * The SIMT launch is a programmatic dependent of the kernel before it in the
+ * stream: it stages adapter pages while that kernel runs and reads v and y
+ * only after that kernel has completed.
  */
 SGMV_API sgmv_status sgmv_expand(const float* v, int64_t ldv, int32_t T, int32_t d_out, int32_t proj,
                         const sgmv_plan* plan, const void* table, const sgmv_pool* pool,
                         float scale, void* y, int64_t ldy, int32_t y_dtype,
                         sgmv_stream_t stream);
+
+/*
+ * Both phases in one call ([SGMV post], "SGMV: the kernel that holds it all
+ * up": one pass computes the delta of every token):
+ *
+ *   y[t][j] <- round( y[t][j] + scale * sum_k B_s[j][k] * sum_c A_s[k][c] * x[t][c] )
+ *
+ * = sgmv_shrink into v, then sgmv_expand from v, on `stream`; the expand's
+ * SIMT launch overlaps the shrink (programmatic dependent launch), so the
+ * second launch costs little ([Glossary], "Limits and open questions", names
+ * the extra launch per adapted layer as a cost of unmerged adapters).
+ * x, y, y_dtype, d_in, d_out, proj as for sgmv_shrink / sgmv_expand.
+ * v        device fp32 [plan->num_rows][ldv], ldv >= plan->max_rank: workspace
+ *          for the intermediate A x (required whenever the plan has work);
+ *          on return it holds v as sgmv_shrink writes it.
+ */
+SGMV_API sgmv_status sgmv_lora_delta(const void* x, int64_t ldx, int32_t T, int32_t d_in, int32_t d_out,
+                                     int32_t proj, const sgmv_plan* plan, const void* table,
+                                     const sgmv_pool* pool, float scale, void* y, int64_t ldy,
+                                     int32_t y_dtype, float* v, int64_t ldv, sgmv_stream_t stream);
 
 /*
  * Wait for `stream`, then return and clear the device error word:

@@ -32,7 +32,7 @@ _STATUS = {0: "SGMV_OK", 1: "SGMV_ERR_INVALID", 2: "SGMV_ERR_UNSUPPORTED", 3: "S
 EXPORTED = ("sgmv_status_string", "sgmv_last_error", "sgmv_pool_create", "sgmv_pool_destroy", "sgmv_pool_load",
             "sgmv_pool_evict", "sgmv_pool_get_stats", "sgmv_pool_adapter_rank", "sgmv_pool_adapter_pages",
             "sgmv_pool_shuffle_free_pages", "sgmv_pool_pages_device", "sgmv_plan_table_capacity",
-            "sgmv_build_plan", "sgmv_shrink", "sgmv_expand", "sgmv_check_errors")
+            "sgmv_build_plan", "sgmv_shrink", "sgmv_expand", "sgmv_lora_delta", "sgmv_check_errors")
 
 
 class SgmvError(RuntimeError):
@@ -85,6 +85,8 @@ def load_library() -> ctypes.CDLL:
         "sgmv_build_plan": (st, [vp, i32, vp, i32, vp, i64, ctypes.POINTER(Plan)]),
         "sgmv_shrink": (st, [vp, i64, i32, i32, i32, ctypes.POINTER(Plan), vp, vp, vp, i64, vp]),
         "sgmv_expand": (st, [vp, i64, i32, i32, i32, ctypes.POINTER(Plan), vp, vp, f32, vp, i64, i32, vp]),
+        "sgmv_lora_delta": (st, [vp, i64, i32, i32, i32, i32, ctypes.POINTER(Plan), vp, vp, f32, vp, i64, i32,
+                                 vp, i64, vp]),
         "sgmv_check_errors": (st, [vp, ctypes.POINTER(ctypes.c_uint32)]),
     }
     for name, (res, args) in sig.items():
@@ -283,13 +285,33 @@ class BatchPlan:
         return self._arr(off, self.plan.num_segments * self.plan.n_proj, np.int64).reshape(
             self.plan.num_segments, self.plan.n_proj)
 
+    def _records(self, off: int, n: int) -> np.ndarray:
+        """[n][n_proj] records as an int64 array [..., 6]: seg, row_begin, row_end, rank, a_pt, b_pt."""
+        npj = self.plan.n_proj
+        raw = self._arr(off, 8 * n * npj, np.int32).reshape(n, npj, 8)
+        out = np.zeros((n, npj, 6), dtype=np.int64)
+        out[..., :4] = raw[..., :4]
+        out[..., 4] = raw[..., 4:6].copy().view(np.int64)[..., 0]
+        out[..., 5] = raw[..., 6:8].copy().view(np.int64)[..., 0]
+        return out
+
+    @property
+    def simt_records(self) -> np.ndarray:
+        return self._records(self.plan.off_simt_items, self.plan.num_simt_items)
+
+    @property
+    def tc_records(self) -> np.ndarray:
+        return self._records(self.plan.off_tc_tiles, self.plan.num_tc_tiles)
+
     @property
     def simt_items(self) -> np.ndarray:
-        return self._arr(self.plan.off_simt_items, 4 * self.plan.num_simt_items, np.int32).reshape(-1, 4)
+        """[n][3]: segment, row_begin, row_end of each SIMT item."""
+        return self.simt_records[:, 0, :3].astype(np.int32).reshape(-1, 3)
 
     @property
     def tc_tiles(self) -> np.ndarray:
-        return self._arr(self.plan.off_tc_tiles, 4 * self.plan.num_tc_tiles, np.int32).reshape(-1, 4)
+        """[n][3]: segment, row_begin, row_end of each tensor-core tile."""
+        return self.tc_records[:, 0, :3].astype(np.int32).reshape(-1, 3)
 
     @property
     def num_rows(self) -> int:
@@ -353,11 +375,18 @@ def check_errors(stream=None) -> int:
     return bits.value
 
 
-def lora_delta(x: torch.Tensor, y: torch.Tensor, plan: BatchPlan, pool: AdapterPool, proj: int = 0,
+def lora_delta(x: torch.Tensor, plan: BatchPlan, pool: AdapterPool, y: torch.Tensor, proj: int = 0,
                scale: float = 1.0, v: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """y_t += scale * B_{a(t)} A_{a(t)} x_t for every token: shrink then expand on one stream."""
+    """y_t += scale * B_{a(t)} A_{a(t)} x_t for every token in one call (SGMV-shrink into the
+    workspace v, then SGMV-expand).  Returns v."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    assert y.dim() == 2 and y.stride(1) == 1 and y.dtype in (torch.bfloat16, torch.float32)
     if v is None:
         v = plan.new_v()
-    shrink(x, plan, pool, v, proj, stream)
-    expand(v, plan, pool, y, proj, scale, stream)
+    assert v.dtype == torch.float32 and v.dim() == 2 and v.stride(1) == 1
+    table = plan.device_table if plan.device_table is not None else plan.upload(stream)
+    _check(load_library().sgmv_lora_delta(
+        _ptr(x), x.stride(0), plan.T, x.shape[1], y.shape[1], int(proj), ctypes.byref(plan.plan),
+        table.data_ptr(), pool.handle, float(scale), _ptr(y), y.stride(0),
+        0 if y.dtype == torch.bfloat16 else 1, _ptr(v), v.stride(0), _stream(stream)))
     return v

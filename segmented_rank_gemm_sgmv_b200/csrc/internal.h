@@ -51,14 +51,19 @@ struct sgmv_pool {
 namespace sgmv {
 
 // -------------------------------------------------------------- plan tables
-struct Item {
-    int32_t seg, row_begin, row_end, pad;
+// One work item as a kernel sees it for one projection: the rows of a
+// segment it covers, its rank, and the first page-table entries of A and B^T
+// of its adapter for that projection.  Records are stored [item][projection]
+// so that a CTA finds everything about its item with one 32-byte load.
+struct ItemRec {
+    int32_t seg, row_begin, row_end, rank;
+    int64_t a_pt, b_pt;
 };
-static_assert(sizeof(Item) == 16, "Item must be 16 bytes");
+static_assert(sizeof(ItemRec) == 32, "ItemRec must be 32 bytes");
 
-constexpr int kSimtMaxItemRows = 64;   // rows per SIMT work item
+constexpr int kSimtMaxItemRows = 8;    // rows per SIMT work item
 constexpr int kTcTileRows = 128;       // rows per tensor-core tile (MMA M)
-constexpr int kDefaultLongThreshold = 64;
+constexpr int kDefaultLongThreshold = 16;
 constexpr int kMaxRank = 128;
 
 // Device view of everything a kernel needs about the batch.
@@ -68,8 +73,8 @@ struct BatchView {
     const int32_t* seg_rank;
     const int64_t* seg_a_pt;
     const int64_t* seg_b_pt;
-    const Item* simt_items;
-    const Item* tc_tiles;
+    const ItemRec* simt_items;   // [num_simt_items][n_proj]
+    const ItemRec* tc_tiles;     // [num_tc_tiles][n_proj]
     int32_t num_segments, num_rows, n_proj, proj, T;
 };
 

@@ -42,8 +42,8 @@ sgmv_status make_views(const sgmv_plan* plan, const void* table, const sgmv_pool
     bv->seg_rank = reinterpret_cast<const int32_t*>(base + plan->off_seg_rank);
     bv->seg_a_pt = reinterpret_cast<const int64_t*>(base + plan->off_seg_a_pt);
     bv->seg_b_pt = reinterpret_cast<const int64_t*>(base + plan->off_seg_b_pt);
-    bv->simt_items = reinterpret_cast<const Item*>(base + plan->off_simt_items);
-    bv->tc_tiles = reinterpret_cast<const Item*>(base + plan->off_tc_tiles);
+    bv->simt_items = reinterpret_cast<const ItemRec*>(base + plan->off_simt_items);
+    bv->tc_tiles = reinterpret_cast<const ItemRec*>(base + plan->off_tc_tiles);
     bv->num_segments = plan->num_segments;
     bv->num_rows = plan->num_rows;
     bv->n_proj = plan->n_proj;
@@ -93,6 +93,8 @@ extern "C" sgmv_status sgmv_shrink(const void* x, int64_t ldx, int32_t T, int32_
     if (ldx < d_in || (ldx % 8) || !aligned16(x)) return fail(SGMV_ERR_INVALID, "shrink: x rows must be 16-byte aligned, ldx >= d_in");
     if (ldv < plan->max_rank || ldv < 1 || (ldv % 4) || !aligned16(v))
         return fail(SGMV_ERR_INVALID, "shrink: v needs ldv >= max_rank, ldv % 4 == 0, 16-byte alignment");
+    if (plan->num_simt_items > 0 && pool->page_elems > 1024)
+        return fail(SGMV_ERR_UNSUPPORTED, "shrink: the SIMT path takes page_elems <= 1024");
     const uint16_t* xb = static_cast<const uint16_t*>(x);
     SGMV_CUDA_TRY(launch_shrink_simt(xb, ldx, d_in, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, pv,
                                      v, ldv, stream));
@@ -117,11 +119,24 @@ extern "C" sgmv_status sgmv_expand(const float* v, int64_t ldv, int32_t T, int32
         return fail(SGMV_ERR_INVALID, "expand: y rows must be 16-byte aligned, ldy >= d_out");
     if (ldv < plan->max_rank || ldv < 1 || (ldv % 4) || !aligned16(v))
         return fail(SGMV_ERR_INVALID, "expand: v needs ldv >= max_rank, ldv % 4 == 0, 16-byte alignment");
+    if (plan->num_simt_items > 0 && pool->page_elems > 1024)
+        return fail(SGMV_ERR_UNSUPPORTED, "expand: the SIMT path takes page_elems <= 1024");
     SGMV_CUDA_TRY(launch_expand_simt(v, ldv, d_out, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, pv,
                                      scale, y, ldy, y_dtype, stream));
     SGMV_CUDA_TRY(launch_expand_tc(v, ldv, d_out, bv, plan->num_tc_tiles, plan->max_rank, pv, scale, y, ldy, y_dtype,
                                    stream));
     return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_lora_delta(const void* x, int64_t ldx, int32_t T, int32_t d_in, int32_t d_out,
+                                       int32_t proj, const sgmv_plan* plan, const void* table, const sgmv_pool* pool,
+                                       float scale, void* y, int64_t ldy, int32_t y_dtype, float* v, int64_t ldv,
+                                       sgmv_stream_t stream) {
+    if (plan && plan->num_rows > 0 && (plan->num_simt_items > 0 || plan->num_tc_tiles > 0) && !v)
+        return fail(SGMV_ERR_INVALID, "lora_delta: the workspace v is required");
+    sgmv_status st = sgmv_shrink(x, ldx, T, d_in, proj, plan, table, pool, v, ldv, stream);
+    if (st != SGMV_OK) return st;
+    return sgmv_expand(v, ldv, T, d_out, proj, plan, table, pool, scale, y, ldy, y_dtype, stream);
 }
 
 extern "C" sgmv_status sgmv_check_errors(sgmv_stream_t stream_, uint32_t* flags) {

@@ -30,8 +30,8 @@ Layout layout_for(int64_t rows, int64_t S, int64_t n_proj, int64_t n_simt, int64
     L.seg_rank = o;    o = align16(o + S * 4);
     L.seg_a_pt = o;    o = align16(o + S * n_proj * 8);
     L.seg_b_pt = o;    o = align16(o + S * n_proj * 8);
-    L.simt_items = o;  o = align16(o + n_simt * 16);
-    L.tc_tiles = o;    o = align16(o + n_tc * 16);
+    L.simt_items = o;  o = align16(o + n_simt * n_proj * 32);
+    L.tc_tiles = o;    o = align16(o + n_tc * n_proj * 32);
     L.end = o;
     return L;
 }
@@ -44,7 +44,7 @@ using namespace sgmv;
 extern "C" int64_t sgmv_plan_table_capacity(int32_t T, int32_t n_proj) {
     if (T < 0 || n_proj < 0) return -1;
     // rows <= T, segments <= T, items <= T and tiles <= T (each holds >= 1 row)
-    return layout_for(T, T, n_proj, T, T).end;
+    return layout_for(T, T, std::max<int64_t>(n_proj, 1), T, T).end;
 }
 
 extern "C" sgmv_status sgmv_build_plan(const int32_t* adapter_ids, int32_t T, const sgmv_pool* pool,
@@ -110,8 +110,14 @@ extern "C" sgmv_status sgmv_build_plan(const int32_t* adapter_ids, int32_t T, co
     int32_t* seg_rank = reinterpret_cast<int32_t*>(base + L.seg_rank);
     int64_t* seg_a_pt = reinterpret_cast<int64_t*>(base + L.seg_a_pt);
     int64_t* seg_b_pt = reinterpret_cast<int64_t*>(base + L.seg_b_pt);
-    Item* simt = reinterpret_cast<Item*>(base + L.simt_items);
-    Item* tc = reinterpret_cast<Item*>(base + L.tc_tiles);
+    auto recs_rank = [&](int32_t s) { return recs[s]->rank; };
+    auto recs_pt = [&](int32_t s, int64_t p, int m) { return m == 0 ? recs[s]->a_pt[p] : recs[s]->b_pt[p]; };
+    ItemRec* simt = reinterpret_cast<ItemRec*>(base + L.simt_items);
+    ItemRec* tc = reinterpret_cast<ItemRec*>(base + L.tc_tiles);
+    auto put = [&](ItemRec* recs, int64_t idx, int32_t s, int32_t r0, int32_t r1) {
+        for (int64_t p = 0; p < n_proj; ++p)
+            recs[idx * n_proj + p] = ItemRec{s, r0, r1, recs_rank(s), recs_pt(s, p, 0), recs_pt(s, p, 1)};
+    };
 
     std::vector<int32_t> fill(offsets.begin(), offsets.end() - 1);
     for (int32_t t = 0; t < T; ++t)  // ascending t keeps each segment in batch order
@@ -128,13 +134,12 @@ extern "C" sgmv_status sgmv_build_plan(const int32_t* adapter_ids, int32_t T, co
         const int32_t b = offsets[s], e = offsets[s + 1], n = e - b;
         if (recs[s]->rank == 0 || n == 0) continue;
         if (n >= long_threshold) {
-            for (int32_t r0 = b; r0 < e; r0 += kTcTileRows)
-                tc[i_tc++] = Item{(int32_t)s, r0, std::min(e, r0 + kTcTileRows), 0};
+            for (int32_t r0 = b; r0 < e; r0 += kTcTileRows) put(tc, i_tc++, (int32_t)s, r0, std::min(e, r0 + kTcTileRows));
         } else {
             for (int32_t r0 = b; r0 < e; r0 += kSimtMaxItemRows) {
                 const int32_t r1 = std::min(e, r0 + kSimtMaxItemRows);
                 max_item = std::max(max_item, r1 - r0);
-                simt[i_simt++] = Item{(int32_t)s, r0, r1, 0};
+                put(simt, i_simt++, (int32_t)s, r0, r1);
             }
         }
     }

@@ -6,19 +6,27 @@
 // small segments take a batched gather path.  One launch per phase covers
 // every short segment of the batch, whatever its rank, with no padded work.
 //
-// shrink:  a thread-block cluster of C CTAs per work item (<= 64 rows of one
-//          segment) splits d_in into C chunks.  Each CTA streams its chunk of
-//          every rank row of A from the page pool into shared memory with bulk
-//          asynchronous copies (one per page, completion on an mbarrier), keeps
-//          8 columns of up to 4 tokens' x in registers, and reduces the
-//          per-thread partial dot products with warp shuffles.  The C partial
-//          results are summed in a fixed order through distributed shared
-//          memory and written to v: deterministic, no atomics, no scratch.
+// Decode batches move a few MB per phase, so both kernels are built around
+// latency: a CTA first reads the page ids of everything it will touch in one
+// round of independent loads, then keeps up to four 16 KB stages of adapter
+// rows in flight with 16-byte cp.async copies issued by all threads (pages are
+// 1 KiB and scattered, which is too fine-grained for one bulk copy per page),
+// the token rows are fetched while those copies fly, and the expand is launched
+// as a programmatic dependent of the shrink so that its B^T stages stream in
+// while the shrink is still running.
 //
-// expand:  one CTA per (work item, tile of d_out columns).  v of the item is
-//          staged in shared memory; each thread owns 8 consecutive output
-//          columns, streams the B^T rank rows for them with 16-byte loads and
-//          updates y in place with a single rounding.
+// shrink:  a thread-block cluster of C CTAs per work item (<= 8 rows of one
+//          segment); CTA q owns d_in columns [q kc, (q+1) kc).  Stages are 8
+//          rank rows x up to 1024 columns; each thread owns 8 columns and
+//          keeps the item's (up to 8) tokens' x in registers; partial dot products are
+//          reduced with warp shuffles and shared memory, then the C partial
+//          tiles are summed in a fixed order through distributed shared memory
+//          and written to v.  Deterministic, no atomics, no scratch memory.
+// expand:  CTAs per work item each cover one or more 1024-column passes of
+//          d_out (about four CTAs per SM in total).  B^T rank rows are staged by
+//          bulk copies before the kernel waits for the shrink; then v of the
+//          item is read, each thread accumulates its 8 output columns for up to
+//          8 tokens and updates y with one rounding, pass by pass.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -29,7 +37,13 @@ namespace {
 
 __device__ unsigned int g_err_simt;
 
-constexpr int kMaxStages = 4;
+constexpr int kThreads = 128;
+constexpr int kVec = 8;                    // columns per thread
+constexpr int kPass = kThreads * kVec;     // 1024 columns per stage
+constexpr int kRowGroup = 8;               // rank rows per stage
+constexpr int kShrinkStages = 4;
+constexpr int kExpandStages = 3;
+constexpr int kStageElems = kRowGroup * kPass;
 
 struct ShrinkArgs {
     const uint16_t* x;
@@ -41,8 +55,9 @@ struct ShrinkArgs {
     int64_t ldv;
     int32_t cluster;     // C
     int32_t kc;          // columns of d_in per CTA (multiple of the page size)
-    int32_t stages;      // depth of the A ring
-    int32_t part_floats; // capacity of the partial buffer
+    int32_t stages;
+    int32_t max_rank;
+    int32_t ring_offset; // byte offset of the stage ring in shared memory
 };
 
 struct ExpandArgs {
@@ -55,10 +70,41 @@ struct ExpandArgs {
     void* y;
     int64_t ldy;
     int32_t y_dtype;
-    int32_t tile_cols;   // output columns per CTA = 8 * blockDim.x
-    int32_t num_tiles;
-    int32_t span;        // pages of one rank row covered by a tile
+    int32_t ctas_per_item;  // CTAs covering d_out for one item
+    int32_t npass;          // 1024-column passes per CTA
+    int32_t stages;
+    int32_t max_rank;
+    int32_t ring_offset;    // byte offset of the stage ring in shared memory
 };
+
+struct ItemInfo {
+    int i0, n, r;
+    int64_t pt;          // first page-table entry of the matrix for this projection
+    bool ok;
+};
+
+__device__ __forceinline__ ItemInfo load_item(const BatchView& b, int idx, int max_rows, int max_rank, int matrix) {
+    ItemInfo m;
+    const int4* rp = reinterpret_cast<const int4*>(b.simt_items + ((int64_t)idx * b.n_proj + b.proj));
+    const int4 h = rp[0], t = rp[1];  // {seg, row_begin, row_end, rank}, {a_pt, b_pt}
+    m.i0 = h.y;
+    m.n = h.z - h.y;
+    m.r = h.w;
+    m.ok = h.x >= 0 && h.x < b.num_segments && h.y >= 0 && m.n > 0 && m.n <= max_rows && h.z <= b.num_rows &&
+           m.r > 0 && m.r <= max_rank;
+    m.pt = matrix == 0 ? (int64_t)(((uint64_t)(uint32_t)t.y << 32) | (uint32_t)t.x)
+                       : (int64_t)(((uint64_t)(uint32_t)t.w << 32) | (uint32_t)t.z);
+    if (!m.ok) {
+        m.n = 0;
+        m.r = 0;
+    }
+    return m;
+}
+
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ float dot8(const float (&a)[8], const float (&b)[8]) {
     float s = a[0] * b[0];
@@ -67,15 +113,15 @@ __device__ __forceinline__ float dot8(const float (&a)[8], const float (&b)[8]) 
     return s;
 }
 
-// Sum N values per thread over the whole CTA.  On return, thread t < N holds
-// the CTA-wide sum of value index t.  N is 8, 16 or 32.
+// Sum N values per thread over the CTA.  Thread t < N gets the CTA-wide sum of
+// value index t.  N is 8, 16, 32 or 64.
 template <int N>
-__device__ __forceinline__ float block_reduce(float (&vals)[N], float* red, int nwarps) {
+__device__ __forceinline__ float block_reduce(float (&vals)[N], float* red) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    constexpr int LOGN = (N == 8) ? 3 : (N == 16) ? 4 : 5;
-    // transpose-reduce: each step halves the values a lane keeps
+    constexpr int LOGN = (N == 8) ? 3 : (N == 16) ? 4 : (N == 32) ? 5 : 6;
+    constexpr int STEPS = LOGN < 5 ? LOGN : 5;
 #pragma unroll
-    for (int step = 0; step < LOGN; ++step) {
+    for (int step = 0; step < STEPS; ++step) {  // transpose-reduce: halve the values a lane keeps
         const int o = 16 >> step;
         const int half = N >> (step + 1);
         const bool upper = (lane & o) != 0;
@@ -86,150 +132,219 @@ __device__ __forceinline__ float block_reduce(float (&vals)[N], float* red, int 
             vals[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
         }
     }
+    if constexpr (N < 32) {
 #pragma unroll
-    for (int o = (16 >> LOGN); o >= 1; o >>= 1) vals[0] += __shfl_xor_sync(0xFFFFFFFFu, vals[0], o);
-    constexpr int SPAN = 32 / N;  // lanes sharing one value index
-    if ((lane & (SPAN - 1)) == 0) red[warp * N + (lane >> (5 - LOGN))] = vals[0];
+        for (int o = (16 >> LOGN); o >= 1; o >>= 1) vals[0] += __shfl_xor_sync(0xFFFFFFFFu, vals[0], o);
+    }
+    if constexpr (N <= 32) {
+        constexpr int SPAN = 32 / N;  // lanes sharing one value index
+        if ((lane & (SPAN - 1)) == 0) red[warp * N + (lane >> (5 - LOGN))] = vals[0];
+    } else {
+        // after five steps lane l holds values i < N/32 of index l * (N/32) + i
+#pragma unroll
+        for (int i = 0; i < N / 32; ++i) red[warp * N + lane * (N / 32) + i] = vals[i];
+    }
     __syncthreads();
     float s = 0.f;
     if (threadIdx.x < N)
-        for (int w = 0; w < nwarps; ++w) s += red[w * N + threadIdx.x];
+#pragma unroll
+        for (int w = 0; w < kThreads / 32; ++w) s += red[w * N + threadIdx.x];
     __syncthreads();
     return s;
 }
 
+// Stage u of a CTA holds rank rows [8 g, 8 g + 8) x columns [c, c + W) of one
+// matrix (W <= 1024), row-major with row stride W.  All 128 threads fill it
+// with 16-byte cp.async copies: consecutive threads take consecutive 16-byte
+// granules of a row (512 contiguous bytes per warp instruction, conflict-free
+// shared-memory writes), each granule's page found in the CTA's page-id table.
+// Every stage is one commit group; the prologue commits kStages groups and
+// each consumed stage commits one more (possibly empty), so waiting for all but
+// the newest kStages - 1 groups always means "this stage has landed".
+struct StageGeom {  // stage u -> rows and columns
+    int NG, npass, span, col_base, rank, pages_per_row;
+    int64_t pt;
+    const int32_t* pid;  // page ids of the CTA's span, [rank row][chunk], in shared memory
+    int span_pages;
+    __device__ void at(int u, bool pass_outer, int& g, int& c, int& W) const {
+        const int s = pass_outer ? u / NG : u % npass;
+        g = pass_outer ? u % NG : u / npass;
+        c = s * kPass;
+        W = min(kPass, span - c);
+    }
+};
+
+template <int kStages>
+struct Pipe {
+    uint16_t* data;
+    int issued = 0, consumed = 0, total = 0;
+};
+
+template <int kStages>
+__device__ __forceinline__ void pipe_issue(const PoolView& pool, Pipe<kStages>& pp, const StageGeom& sg,
+                                           bool pass_outer) {
+    if (pp.issued < pp.total) {
+        const int P_log2 = pool.page_log2, P = 1 << P_log2;
+        int g, c, W;
+        sg.at(pp.issued, pass_outer, g, c, W);
+        const int rows = min(kRowGroup, sg.rank - kRowGroup * g);
+        const int gpr = W >> 3;  // granules per row
+        uint16_t* dst0 = pp.data + (size_t)(pp.issued % kStages) * kStageElems;
+#pragma unroll
+        for (int i = 0; i < kStageElems / 8 / kThreads; ++i) {
+            const int gi = threadIdx.x + kThreads * i;
+            const int kk = gi / gpr, cg = gi - kk * gpr;
+            if (kk < rows) {
+                const int col = c + cg * 8;
+                const int32_t page = sg.pid[(kRowGroup * g + kk) * sg.span_pages + (col >> P_log2)];
+                cp_async16(dst0 + (size_t)kk * W + cg * 8,
+                           pool.pages + ((int64_t)page << P_log2) + (col & (P - 1)), true);
+            }
+        }
+    }
+    ++pp.issued;
+    cp_async_commit();
+}
+
+template <int kStages>
+__device__ __forceinline__ const uint16_t* pipe_acquire(Pipe<kStages>& pp) {
+    cp_async_wait<kStages - 1>();
+    __syncthreads();
+    return pp.data + (size_t)(pp.consumed % kStages) * kStageElems;
+}
+
+template <int kStages>
+__device__ __forceinline__ void pipe_release(const PoolView& pool, Pipe<kStages>& pp, const StageGeom& sg,
+                                             bool pass_outer) {
+    __syncthreads();  // every thread is done with the slot before it is refilled
+    ++pp.consumed;
+    pipe_issue(pool, pp, sg, pass_outer);
+}
+
+// All threads: fetch the page ids of every rank row over the CTA's column span
+// into shared memory in one round of independent loads.  Out-of-range ids are
+// flagged and replaced by page 0 (in bounds; the result is flagged).
+__device__ void load_page_ids(const PoolView& pool, StageGeom& sg, int32_t* pid, unsigned int* err) {
+    const int P_log2 = pool.page_log2;
+    sg.span_pages = sg.span > 0 ? (sg.span + (1 << P_log2) - 1) >> P_log2 : 0;
+    const int n = sg.rank * sg.span_pages;
+    for (int i = threadIdx.x; i < n; i += kThreads) {
+        const int k = i / sg.span_pages, pc = i - k * sg.span_pages;
+        const int64_t e = sg.pt + (int64_t)k * sg.pages_per_row + (sg.col_base >> P_log2) + pc;
+        int32_t page = (e >= 0 && e < pool.pt_capacity) ? pool.page_table[e] : -1;
+        if (page < 0 || page >= pool.num_pages) {
+            atomicOr(err, kErrPage);
+            page = 0;
+        }
+        pid[i] = page;
+    }
+    sg.pid = pid;
+}
+
 // ------------------------------------------------------------------ shrink
 template <int G>
-__device__ void shrink_item(const ShrinkArgs& a, int i0, int n, int r, int64_t a_base, uint32_t q, uint64_t* bars,
-                            uint16_t* ring, float* part, float* red, int* abort_flag) {
-    const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5;
-    const int P_log2 = a.pool.page_log2, P = 1 << P_log2;
-    const int kc = a.kc, c0 = (int)q * kc;
-    const int pages_per_row = a.d_in >> P_log2, cpr = kc >> P_log2;
-    const int n_groups = (r + 7) >> 3;
-    const int NS = a.stages;
-
-    auto issue = [&](int g) {  // warp 0: bulk-copy the chunk of rank rows [8g, 8g+8) into the ring
-        const int slot = g % NS;
-        const int rows = min(8, r - 8 * g);
-        if (lane == 0) mbar_arrive_expect_tx(&bars[slot], (uint32_t)(rows * kc * 2));
-        __syncwarp();
-        for (int idx = lane; idx < rows * cpr; idx += 32) {
-            const int kk = idx / cpr, pq = idx - kk * cpr;
-            const int64_t e = a_base + (int64_t)(8 * g + kk) * pages_per_row + (c0 >> P_log2) + pq;
-            int32_t page = (e >= 0 && e < a.pool.pt_capacity) ? a.pool.page_table[e] : -1;
-            if (page < 0 || page >= a.pool.num_pages) {
-                atomicOr(&g_err_simt, kErrPage);
-                page = 0;  // keep the transaction count exact; the result is flagged
-            }
-            bulk_g2s(ring + ((size_t)slot * 8 + kk) * kc + (size_t)pq * P,
-                     a.pool.pages + ((int64_t)page << P_log2), (uint32_t)P * 2u, &bars[slot]);
+__device__ void shrink_item(const ShrinkArgs& a, const ItemInfo& m, uint32_t q, Pipe<kShrinkStages>& pp,
+                            const StageGeom& sg, float* part, float* red) {
+    const int tid = threadIdx.x, col = kVec * tid;
+    const uint16_t* xrow[G];
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+        xrow[j] = nullptr;
+        if (j < m.n) {
+            const int t = a.b.token_idx[m.i0 + j];
+            if (t >= 0 && t < a.b.T) xrow[j] = a.x + (int64_t)t * a.ldx + (int64_t)q * a.kc;
+            else atomicOr(&g_err_simt, kErrToken);
         }
-    };
-    if (warp == 0)
-        for (int g = 0; g < min(NS, n_groups); ++g) issue(g);
-
-    for (int g = 0; g < n_groups; ++g) {
-        const int slot = g % NS;
-        const uint32_t parity = (uint32_t)((g / NS) & 1);
-        if (!mbar_wait(&bars[slot], parity, &g_err_simt)) *abort_flag = 1;
-        const uint16_t* As = ring + (size_t)slot * 8 * kc;
-        const int rows = min(8, r - 8 * g);
-        for (int j0 = 0; j0 < n; j0 += G) {
-            float p[8 * G];
+    }
+    for (int g = 0; g < sg.NG; ++g) {
+        float p[kRowGroup * G];
 #pragma unroll
-            for (int i = 0; i < 8 * G; ++i) p[i] = 0.f;
-            const uint16_t* xrow[G];
+        for (int i = 0; i < kRowGroup * G; ++i) p[i] = 0.f;
+        for (int s = 0; s < sg.npass; ++s) {
+            const int c = s * kPass, W = min(kPass, sg.span - c);
+            const bool active = col < W;
+            float xf[G][8];
 #pragma unroll
-            for (int jj = 0; jj < G; ++jj) {
-                xrow[jj] = nullptr;
-                if (j0 + jj < n) {
-                    const int t = a.b.token_idx[i0 + j0 + jj];
-                    if (t >= 0 && t < a.b.T) xrow[jj] = a.x + (int64_t)t * a.ldx + c0;
-                    else atomicOr(&g_err_simt, kErrToken);
+            for (int j = 0; j < G; ++j) {
+                if (active && xrow[j]) {
+                    unpack8(__ldg(reinterpret_cast<const uint4*>(xrow[j] + c + col)), xf[j]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) xf[j][e] = 0.f;
                 }
             }
-            for (int col = 8 * tid; col < kc; col += 8 * nthr) {
-                float xf[G][8];
+            const uint16_t* st = pipe_acquire(pp);
+            if (active) {
 #pragma unroll
-                for (int jj = 0; jj < G; ++jj) {
-                    if (xrow[jj]) {
-                        const uint4 xq = __ldg(reinterpret_cast<const uint4*>(xrow[jj] + col));
-                        unpack8(xq, xf[jj]);
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) xf[jj][e] = 0.f;
-                    }
-                }
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint4 aq = *reinterpret_cast<const uint4*>(As + (size_t)kk * kc + col);
+                for (int kk = 0; kk < kRowGroup; ++kk) {
                     float af[8];
-                    unpack8(aq, af);
+                    unpack8(*reinterpret_cast<const uint4*>(st + (size_t)kk * W + col), af);
 #pragma unroll
-                    for (int jj = 0; jj < G; ++jj) p[kk * G + jj] += dot8(af, xf[jj]);
+                    for (int j = 0; j < G; ++j) p[kk * G + j] += dot8(af, xf[j]);
                 }
             }
-            const float s = block_reduce<8 * G>(p, red, nthr >> 5);
-            if (tid < 8 * G) {
-                const int kk = tid / G, jj = tid - (tid / G) * G;
-                if (kk < rows && j0 + jj < n) part[(j0 + jj) * r + 8 * g + kk] = s;
-            }
+            pipe_release(a.pool, pp, sg, false);
         }
-        __syncthreads();  // every thread is done with this slot
-        if (warp == 0 && g + NS < n_groups) issue(g + NS);
+        const float sum = block_reduce<kRowGroup * G>(p, red);
+        if (tid < kRowGroup * G) {
+            const int kk = tid / G, j = tid - (tid / G) * G;
+            if (kRowGroup * g + kk < m.r && j < m.n) part[j * m.r + kRowGroup * g + kk] = sum;
+        }
     }
 }
 
-__global__ void __launch_bounds__(256) shrink_simt_kernel(const ShrinkArgs a) {
+template <int MAXG>
+__global__ void __launch_bounds__(kThreads, MAXG == 8 ? 2 : 3) shrink_simt_kernel(const ShrinkArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ int abort_flag;
+    pdl_launch_dependents();  // the expand may start staging its B^T pages now
     const int C = a.cluster;
     const int item_idx = blockIdx.x / C;
     const uint32_t q = cluster_ctarank();
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    uint16_t* ring = reinterpret_cast<uint16_t*>(smem + 128);
-    float* part = reinterpret_cast<float*>(smem + 128 + (size_t)a.stages * 8 * a.kc * 2);
-    float* red = part + a.part_floats;
+    float* part = reinterpret_cast<float*>(smem);
+    float* red = part + kSimtMaxItemRows * a.max_rank;  // [4 warps][64]
+    int32_t* pid = reinterpret_cast<int32_t*>(red + 4 * 64);
 
-    const Item it = a.b.simt_items[item_idx];
-    int n = it.row_end - it.row_begin, r = 0;
-    int64_t a_base = 0;
-    if (it.seg < 0 || it.seg >= a.b.num_segments || it.row_begin < 0 || n < 0 || it.row_end > a.b.num_rows) {
-        if (threadIdx.x == 0) atomicOr(&g_err_simt, kErrRows);
-        n = 0;
-    } else {
-        r = a.b.seg_rank[it.seg];
-        a_base = a.b.seg_a_pt[(int64_t)it.seg * a.b.n_proj + a.b.proj];
-        if (r < 0 || n * r > a.part_floats) {
-            if (threadIdx.x == 0) atomicOr(&g_err_simt, kErrRows);
-            n = 0;
-        }
-    }
-    if (threadIdx.x == 0) {
-        abort_flag = 0;
-        for (int i = 0; i < a.stages; ++i) mbar_init(&bars[i], 1);
-        fence_mbar_init();
-    }
+    const ItemInfo m = load_item(a.b, item_idx, MAXG, a.max_rank, 0);
+    if (!m.ok && threadIdx.x == 0) atomicOr(&g_err_simt, kErrRows);
+    StageGeom sg;
+    sg.NG = (m.r + kRowGroup - 1) / kRowGroup;
+    sg.span = a.kc;
+    sg.npass = (a.kc + kPass - 1) / kPass;
+    sg.col_base = (int)q * a.kc;
+    sg.rank = m.r;
+    sg.pages_per_row = a.d_in >> a.pool.page_log2;
+    sg.pt = m.pt;
+    Pipe<kShrinkStages> pp;
+    pp.data = reinterpret_cast<uint16_t*>(smem + a.ring_offset);
+    pp.total = m.ok ? sg.NG * sg.npass : 0;
+    if (m.ok) load_page_ids(a.pool, sg, pid, &g_err_simt);
     __syncthreads();
-
-    if (n > 0 && r > 0) {
-        if (n == 1) shrink_item<1>(a, it.row_begin, n, r, a_base, q, bars, ring, part, red, &abort_flag);
-        else if (n == 2) shrink_item<2>(a, it.row_begin, n, r, a_base, q, bars, ring, part, red, &abort_flag);
-        else shrink_item<4>(a, it.row_begin, n, r, a_base, q, bars, ring, part, red, &abort_flag);
+#pragma unroll 1
+    for (int i = 0; i < kShrinkStages; ++i) pipe_issue(a.pool, pp, sg, false);
+    if (m.ok) {  // MAXG bounds the token group, and with it the registers of the launch
+        if (MAXG == 1 || m.n == 1) shrink_item<1>(a, m, q, pp, sg, part, red);
+        else if (MAXG == 2 || m.n == 2) shrink_item<(MAXG < 2 ? MAXG : 2)>(a, m, q, pp, sg, part, red);
+        else if (MAXG == 4 || m.n <= 4) shrink_item<(MAXG < 4 ? MAXG : 4)>(a, m, q, pp, sg, part, red);
+        else shrink_item<MAXG>(a, m, q, pp, sg, part, red);
     }
+    cp_async_wait<0>();
 
-    // Sum the C partial results in a fixed order through distributed shared memory.
+    // Sum the C partial tiles in a fixed order through distributed shared memory.
     cluster_sync();
-    if (n > 0 && r > 0 && !abort_flag) {
-        const int E = n * r;
+    if (m.ok) {
+        const int E = m.n * m.r;
         const int e0 = (int)(((int64_t)E * q) / C), e1 = (int)(((int64_t)E * (q + 1)) / C);
         const uint32_t part_s = smem_u32(part);
-        for (int e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
+        for (int e = e0 + threadIdx.x; e < e1; e += kThreads) {
+            float pv[8];
+#pragma unroll
+            for (int qq = 0; qq < 8; ++qq)  // all loads in flight before the sum
+                pv[qq] = qq < C ? ld_cluster_f32(map_cluster(part_s + 4u * (uint32_t)e, (uint32_t)qq)) : 0.f;
             float s = 0.f;
-            for (int qq = 0; qq < C; ++qq) s += ld_cluster_f32(map_cluster(part_s + 4u * (uint32_t)e, (uint32_t)qq));
-            const int jrow = e / r, k = e - jrow * r;
-            a.v[(int64_t)(it.row_begin + jrow) * a.ldv + k] = s;
+#pragma unroll
+            for (int qq = 0; qq < 8; ++qq) s += pv[qq];
+            const int jrow = e / m.r, k = e - jrow * m.r;
+            a.v[(int64_t)(m.i0 + jrow) * a.ldv + k] = s;
         }
     }
     cluster_sync();  // peers keep their shared memory until every read is done
@@ -237,128 +352,174 @@ __global__ void __launch_bounds__(256) shrink_simt_kernel(const ShrinkArgs a) {
 
 // ------------------------------------------------------------------ expand
 template <int G>
-__device__ void expand_item(const ExpandArgs& a, int i0, int n, int r, const float* vs, const int32_t* pg, int j,
-                            int pc) {
-    const int P_log2 = a.pool.page_log2;
-    const int off = j & ((1 << P_log2) - 1);
-    for (int j0 = 0; j0 < n; j0 += G) {
-        float acc[G][8];
+__device__ void expand_item(const ExpandArgs& a, const ItemInfo& m, Pipe<kExpandStages>& pp, const StageGeom& sg,
+                            const float* vs) {
+    const int tid = threadIdx.x, col = kVec * tid;
+    int trow[G];
 #pragma unroll
-        for (int jj = 0; jj < G; ++jj)
+    for (int j = 0; j < G; ++j) {
+        trow[j] = -1;
+        if (j < m.n) {
+            const int t = a.b.token_idx[m.i0 + j];
+            if (t >= 0 && t < a.b.T) trow[j] = t;
+            else if (tid == 0) atomicOr(&g_err_simt, kErrToken);
+        }
+    }
+    for (int s = 0; s < sg.npass; ++s) {
+        const int c = s * kPass, W = min(kPass, sg.span - c);
+        const bool active = col < W;
+        const int jcol = sg.col_base + c + col;
+        // y of this pass: issued now, used after the accumulation
+        uint4 yb[G];
+        float4 yf0[G], yf1[G];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[jj][e] = 0.f;
-#pragma unroll 4
-        for (int k = 0; k < r; ++k) {
-            const int32_t page = pg[k * a.span + pc];
-            const uint4 bq = __ldg(reinterpret_cast<const uint4*>(a.pool.pages + ((int64_t)page << P_log2) + off));
-            float bf[8];
-            unpack8(bq, bf);
-#pragma unroll
-            for (int jj = 0; jj < G; ++jj) {
-                const float w = vs[min(j0 + jj, n - 1) * r + k];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[jj][e] = fmaf(w, bf[e], acc[jj][e]);
+        for (int j = 0; j < G; ++j) {
+            if (active && trow[j] >= 0) {
+                if (a.y_dtype == 0) {
+                    yb[j] = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.y) +
+                                                             (int64_t)trow[j] * a.ldy + jcol);
+                } else {
+                    const float* yp = static_cast<const float*>(a.y) + (int64_t)trow[j] * a.ldy + jcol;
+                    yf0[j] = *reinterpret_cast<const float4*>(yp);
+                    yf1[j] = *reinterpret_cast<const float4*>(yp + 4);
+                }
             }
         }
+        float acc[G][8];
 #pragma unroll
-        for (int jj = 0; jj < G; ++jj) {
-            if (j0 + jj >= n) break;
-            const int t = a.b.token_idx[i0 + j0 + jj];
-            if (t < 0 || t >= a.b.T) {
-                atomicOr(&g_err_simt, kErrToken);
-                continue;
+        for (int j = 0; j < G; ++j)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+        for (int g = 0; g < sg.NG; ++g) {
+            const uint16_t* st = pipe_acquire(pp);
+            if (active) {
+#pragma unroll
+                for (int kk = 0; kk < kRowGroup; ++kk) {
+                    const int k = kRowGroup * g + kk;
+                    if (k < m.r) {
+                        float bf[8];
+                        unpack8(*reinterpret_cast<const uint4*>(st + (size_t)kk * W + col), bf);
+#pragma unroll
+                        for (int j = 0; j < G; ++j) {
+                            const float w = vs[min(j, m.n - 1) * m.r + k];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) acc[j][e] = fmaf(w, bf[e], acc[j][e]);
+                        }
+                    }
+                }
             }
+            pipe_release(a.pool, pp, sg, true);
+        }
+        if (!active) continue;
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+            if (trow[j] < 0) continue;
             if (a.y_dtype == 0) {
-                uint16_t* yp = static_cast<uint16_t*>(a.y) + (int64_t)t * a.ldy + j;
-                uint4 yq = *reinterpret_cast<const uint4*>(yp);
-                float yf[8];
-                unpack8(yq, yf);
+                float yv[8];
+                unpack8(yb[j], yv);
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float lo = fmaf(a.scale, acc[jj][2 * e], yf[2 * e]);
-                    const float hi = fmaf(a.scale, acc[jj][2 * e + 1], yf[2 * e + 1]);
+                    const float lo = fmaf(a.scale, acc[j][2 * e], yv[2 * e]);
+                    const float hi = fmaf(a.scale, acc[j][2 * e + 1], yv[2 * e + 1]);
                     w[e] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
                            ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
                 }
-                *reinterpret_cast<uint4*>(yp) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.y) + (int64_t)trow[j] * a.ldy + jcol) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
             } else {
-                float* yp = static_cast<float*>(a.y) + (int64_t)t * a.ldy + j;
-                float4 y0 = *reinterpret_cast<const float4*>(yp);
-                float4 y1 = *reinterpret_cast<const float4*>(yp + 4);
-                y0.x = fmaf(a.scale, acc[jj][0], y0.x); y0.y = fmaf(a.scale, acc[jj][1], y0.y);
-                y0.z = fmaf(a.scale, acc[jj][2], y0.z); y0.w = fmaf(a.scale, acc[jj][3], y0.w);
-                y1.x = fmaf(a.scale, acc[jj][4], y1.x); y1.y = fmaf(a.scale, acc[jj][5], y1.y);
-                y1.z = fmaf(a.scale, acc[jj][6], y1.z); y1.w = fmaf(a.scale, acc[jj][7], y1.w);
-                *reinterpret_cast<float4*>(yp) = y0;
-                *reinterpret_cast<float4*>(yp + 4) = y1;
+                float* yp = static_cast<float*>(a.y) + (int64_t)trow[j] * a.ldy + jcol;
+                float4 o0 = yf0[j], o1 = yf1[j];
+                o0.x = fmaf(a.scale, acc[j][0], o0.x); o0.y = fmaf(a.scale, acc[j][1], o0.y);
+                o0.z = fmaf(a.scale, acc[j][2], o0.z); o0.w = fmaf(a.scale, acc[j][3], o0.w);
+                o1.x = fmaf(a.scale, acc[j][4], o1.x); o1.y = fmaf(a.scale, acc[j][5], o1.y);
+                o1.z = fmaf(a.scale, acc[j][6], o1.z); o1.w = fmaf(a.scale, acc[j][7], o1.w);
+                *reinterpret_cast<float4*>(yp) = o0;
+                *reinterpret_cast<float4*>(yp + 4) = o1;
             }
         }
     }
 }
 
-__global__ void __launch_bounds__(256) expand_simt_kernel(const ExpandArgs a) {
-    extern __shared__ __align__(16) uint8_t smem_e[];
-    uint8_t* smem = smem_e;
-    const int tile = blockIdx.x % a.num_tiles, item_idx = blockIdx.x / a.num_tiles;
-    const Item it = a.b.simt_items[item_idx];
-    const int n = it.row_end - it.row_begin;
-    if (it.seg < 0 || it.seg >= a.b.num_segments || it.row_begin < 0 || n <= 0 || it.row_end > a.b.num_rows) {
-        if (threadIdx.x == 0) atomicOr(&g_err_simt, kErrRows);
-        return;
-    }
-    const int r = a.b.seg_rank[it.seg];
-    if (r <= 0 || r > kMaxRank || n > kSimtMaxItemRows) {
-        if (threadIdx.x == 0 && r != 0) atomicOr(&g_err_simt, kErrRows);
-        return;
-    }
-    const int64_t b_base = a.b.seg_b_pt[(int64_t)it.seg * a.b.n_proj + a.b.proj];
-    const int P_log2 = a.pool.page_log2;
-    const int j0 = tile * a.tile_cols;
-    const int pages_per_row = a.d_out >> P_log2;
-    const int first_page = j0 >> P_log2;
+template <int MAXG>
+__global__ void __launch_bounds__(kThreads, MAXG == 8 ? 2 : 3) expand_simt_kernel(const ExpandArgs a) {
+    extern __shared__ __align__(128) uint8_t smem_e[];
+    const int part_idx = blockIdx.x % a.ctas_per_item, item_idx = blockIdx.x / a.ctas_per_item;
+    float* vs = reinterpret_cast<float*>(smem_e);
+    int32_t* pid = reinterpret_cast<int32_t*>(vs + kSimtMaxItemRows * a.max_rank);
 
-    float* vs = reinterpret_cast<float*>(smem);
-    int32_t* pg = reinterpret_cast<int32_t*>(vs + kSimtMaxItemRows * kMaxRank);
-    for (int e = threadIdx.x; e < n * r; e += blockDim.x) {
-        const int jrow = e / r, k = e - jrow * r;
-        vs[e] = a.v[(int64_t)(it.row_begin + jrow) * a.ldv + k];
-    }
-    for (int e = threadIdx.x; e < r * a.span; e += blockDim.x) {
-        const int k = e / a.span, pc = e - k * a.span;
-        int32_t page = 0;
-        if (first_page + pc < pages_per_row) {
-            const int64_t ent = b_base + (int64_t)k * pages_per_row + first_page + pc;
-            page = (ent >= 0 && ent < a.pool.pt_capacity) ? a.pool.page_table[ent] : -1;
-            if (page < 0 || page >= a.pool.num_pages) {
-                atomicOr(&g_err_simt, kErrPage);
-                page = 0;
-            }
-        }
-        pg[e] = page;
-    }
+    const ItemInfo m = load_item(a.b, item_idx, MAXG, a.max_rank, 1);
+    const int j0 = part_idx * a.npass * kPass;
+    StageGeom sg;
+    sg.NG = (m.r + kRowGroup - 1) / kRowGroup;
+    sg.span = min(a.npass * kPass, a.d_out - j0);
+    sg.npass = (sg.span + kPass - 1) / kPass;
+    sg.col_base = j0;
+    sg.rank = m.r;
+    sg.pages_per_row = a.d_out >> a.pool.page_log2;
+    sg.pt = m.pt;
+    const bool work = m.ok && sg.span > 0;
+    Pipe<kExpandStages> pp;
+    pp.data = reinterpret_cast<uint16_t*>(smem_e + a.ring_offset);
+    pp.total = work ? sg.NG * sg.npass : 0;
+    if (work) load_page_ids(a.pool, sg, pid, &g_err_simt);
     __syncthreads();
-    const int j = j0 + 8 * threadIdx.x;
-    if (j >= a.d_out) return;
-    const int pc = (j >> P_log2) - first_page;
-    if (n == 1) expand_item<1>(a, it.row_begin, n, r, vs, pg, j, pc);
-    else if (n == 2) expand_item<2>(a, it.row_begin, n, r, vs, pg, j, pc);
-    else expand_item<4>(a, it.row_begin, n, r, vs, pg, j, pc);
+    // B^T pages do not depend on the shrink: start them before waiting for it
+#pragma unroll 1
+    for (int i = 0; i < kExpandStages; ++i) pipe_issue(a.pool, pp, sg, true);
+    pdl_wait();  // v (and y) are final once the preceding kernel has completed
+    if (!work) {
+        if (threadIdx.x == 0 && !m.ok) atomicOr(&g_err_simt, kErrRows);
+        cp_async_wait<0>();
+        return;
+    }
+    for (int e = threadIdx.x; e < m.n * m.r; e += kThreads) {
+        const int jrow = e / m.r, k = e - jrow * m.r;
+        vs[e] = a.v[(int64_t)(m.i0 + jrow) * a.ldv + k];
+    }
+    // (the first pipe_acquire's barrier publishes vs)
+    if (MAXG == 1 || m.n == 1) expand_item<1>(a, m, pp, sg, vs);
+    else if (MAXG == 2 || m.n == 2) expand_item<(MAXG < 2 ? MAXG : 2)>(a, m, pp, sg, vs);
+    else if (MAXG == 4 || m.n <= 4) expand_item<(MAXG < 4 ? MAXG : 4)>(a, m, pp, sg, vs);
+    else expand_item<MAXG>(a, m, pp, sg, vs);
+    cp_async_wait<0>();
+}
+
+int num_sms() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            n = 148;
+    }
+    return n;
 }
 
 }  // namespace
+
+template <typename K1, typename K2, typename K4, typename K8>
+auto pick(int max_item_rows, K1 k1, K2 k2, K4 k4, K8 k8) {
+    return max_item_rows <= 1 ? k1 : max_item_rows <= 2 ? k2 : max_item_rows <= 4 ? k4 : k8;
+}
 
 cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, const BatchView& b, int32_t num_items,
                                int32_t max_item_rows, int32_t max_rank, const PoolView& pool, float* v, int64_t ldv,
                                cudaStream_t stream) {
     if (num_items <= 0) return cudaSuccess;
+    auto kern = pick(max_item_rows, shrink_simt_kernel<1>, shrink_simt_kernel<2>, shrink_simt_kernel<4>,
+                     shrink_simt_kernel<8>);
+    // Cluster size: enough CTAs for two per SM, chunks of >= 1024 columns, at most 8.
     const int pages = d_in >> pool.page_log2;
+    const int target = (2 * num_sms() + num_items - 1) / num_items;
     int C = 1;
-    for (int c = 8; c >= 1; --c)
-        if (pages % c == 0) {
+    for (int c = 1; c <= 8; ++c) {
+        if (pages % c || (c > 1 && d_in / c < kPass)) continue;
+        if (c >= target) {
             C = c;
             break;
         }
+        C = c;
+    }
     ShrinkArgs a;
     a.x = x;
     a.ldx = ldx;
@@ -369,17 +530,20 @@ cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, con
     a.ldv = ldv;
     a.cluster = C;
     a.kc = d_in / C;
-    const size_t stage_bytes = (size_t)8 * a.kc * 2;
-    a.stages = (int)std::max<size_t>(2, std::min<size_t>(kMaxStages, (96u << 10) / stage_bytes));
-    a.part_floats = std::max(1, max_item_rows * max_rank);
-    int threads = std::min(256, std::max(32, a.kc / 8));
-    threads = (threads + 31) / 32 * 32;
-    const size_t smem = 128 + (size_t)a.stages * stage_bytes + (size_t)a.part_floats * 4 + (size_t)(threads / 32) * 32 * 4;
-    cudaError_t e = cudaFuncSetAttribute(shrink_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    a.max_rank = std::max(8, max_rank);
+    const int NG = (a.max_rank + kRowGroup - 1) / kRowGroup;
+    const int npass = (a.kc + kPass - 1) / kPass;
+    (void)NG;
+    (void)npass;
+    a.stages = kShrinkStages;
+    const size_t pid_bytes = (size_t)a.max_rank * (a.kc >> pool.page_log2) * 4;
+    a.ring_offset = (int)(((size_t)kSimtMaxItemRows * a.max_rank * 4 + 1024 + pid_bytes + 127) & ~(size_t)127);
+    const size_t smem = (size_t)a.ring_offset + (size_t)kShrinkStages * kStageElems * 2;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(C * num_items), 1, 1);
-    cfg.blockDim = dim3((unsigned)threads, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -389,15 +553,15 @@ cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, con
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, shrink_simt_kernel, a);
+    return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const BatchView& b, int32_t num_items,
                                int32_t max_item_rows, int32_t max_rank, const PoolView& pool, float scale, void* y,
                                int64_t ldy, int32_t y_dtype, cudaStream_t stream) {
-    (void)max_item_rows;
-    (void)max_rank;
     if (num_items <= 0) return cudaSuccess;
+    auto kern = pick(max_item_rows, expand_simt_kernel<1>, expand_simt_kernel<2>, expand_simt_kernel<4>,
+                     expand_simt_kernel<8>);
     ExpandArgs a;
     a.v = v;
     a.ldv = ldv;
@@ -408,17 +572,31 @@ cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const
     a.y = y;
     a.ldy = ldy;
     a.y_dtype = y_dtype;
-    int threads = 128;
-    if ((int64_t)num_items * ((d_out + 1023) / 1024) < 2 * 148) threads = 64;
-    a.tile_cols = threads * 8;
-    a.num_tiles = (d_out + a.tile_cols - 1) / a.tile_cols;
-    const int P = 1 << pool.page_log2;
-    a.span = a.tile_cols >= P ? a.tile_cols / P : 1;
-    const size_t smem = (size_t)kSimtMaxItemRows * kMaxRank * 4 + (size_t)kMaxRank * a.span * 4;
-    cudaError_t e = cudaFuncSetAttribute(expand_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // About four CTAs per SM: CTAs per item k, each covering npass 1024-column passes.
+    const int tiles = (d_out + kPass - 1) / kPass;
+    const int k = std::max(1, std::min(tiles, (4 * num_sms() + num_items / 2) / num_items));
+    a.npass = (tiles + k - 1) / k;
+    a.ctas_per_item = (tiles + a.npass - 1) / a.npass;
+    a.max_rank = std::max(8, max_rank);
+    const int NG = (a.max_rank + kRowGroup - 1) / kRowGroup;
+    (void)NG;
+    a.stages = kExpandStages;
+    const size_t pid_bytes = (size_t)a.max_rank * ((a.npass * kPass) >> pool.page_log2) * 4;
+    a.ring_offset = (int)(((size_t)kSimtMaxItemRows * a.max_rank * 4 + pid_bytes + 127) & ~(size_t)127);
+    const size_t smem = (size_t)a.ring_offset + (size_t)kExpandStages * kStageElems * 2;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    expand_simt_kernel<<<(unsigned)(a.num_tiles * num_items), threads, smem, stream>>>(a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.ctas_per_item * num_items), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 cudaError_t read_clear_errors_simt(uint32_t* bits, cudaStream_t stream) {

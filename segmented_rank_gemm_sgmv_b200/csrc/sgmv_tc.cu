@@ -89,14 +89,14 @@ __global__ void __launch_bounds__(kThreads) shrink_tc_kernel(const ShrinkTcArgs 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int tile_idx = blockIdx.x / a.ks;
     const uint32_t q = cluster_ctarank();
-    const Item it = a.b.tc_tiles[tile_idx];
+    const ItemRec it = a.b.tc_tiles[(int64_t)tile_idx * a.b.n_proj + a.b.proj];
     int rows = it.row_end - it.row_begin, r = 0;
     int64_t a_base = 0;
     bool ok = !(it.seg < 0 || it.seg >= a.b.num_segments || it.row_begin < 0 || rows <= 0 ||
                 rows > kTcTileRows || it.row_end > a.b.num_rows);
     if (ok) {
-        r = a.b.seg_rank[it.seg];
-        a_base = a.b.seg_a_pt[(int64_t)it.seg * a.b.n_proj + a.b.proj];
+        r = it.rank;
+        a_base = it.a_pt;
         ok = r > 0 && ((r + 15) & ~15) <= a.npad_max;
     }
     if (!ok && tid == 0) atomicOr(&g_err_tc, kErrRows);
@@ -248,14 +248,14 @@ __global__ void __launch_bounds__(kThreads) expand_tc_kernel(const ExpandTcArgs 
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ntile = blockIdx.x % a.n_tiles, tile_idx = blockIdx.x / a.n_tiles;
-    const Item it = a.b.tc_tiles[tile_idx];
+    const ItemRec it = a.b.tc_tiles[(int64_t)tile_idx * a.b.n_proj + a.b.proj];
     int rows = it.row_end - it.row_begin, r = 0;
     int64_t b_base = 0;
     bool ok = !(it.seg < 0 || it.seg >= a.b.num_segments || it.row_begin < 0 || rows <= 0 ||
                 rows > kTcTileRows || it.row_end > a.b.num_rows);
     if (ok) {
-        r = a.b.seg_rank[it.seg];
-        b_base = a.b.seg_b_pt[(int64_t)it.seg * a.b.n_proj + a.b.proj];
+        r = it.rank;
+        b_base = it.b_pt;
         ok = r > 0 && ((r + 15) & ~15) <= a.kpad_max;
     }
     if (!ok) {  // uniform across the CTA: nothing is allocated yet

@@ -41,15 +41,20 @@ def build_pool(wl: workloads.Workload, bank: workloads.AdapterBank, page_elems: 
 
 
 def run_gpu(pool, wl, proj, x, y, long_threshold=0, y_dtype=torch.bfloat16, scale=None,
-            adapter_ids=None):
+            adapter_ids=None, mode="separate"):
+    """mode "separate": sgmv_shrink then sgmv_expand; "lora_delta": both in one call."""
     ids = wl.adapter_ids if adapter_ids is None else adapter_ids
     plan = pool.plan(ids, long_threshold=long_threshold)
     plan.upload()
     v = plan.new_v()
     v.fill_(float("nan"))
     y_out = y.to(y_dtype).clone()
-    sg.shrink(x, plan, pool, v, proj)
-    sg.expand(v, plan, pool, y_out, proj, wl.scale if scale is None else scale)
+    sc = wl.scale if scale is None else scale
+    if mode == "separate":
+        sg.shrink(x, plan, pool, v, proj)
+        sg.expand(v, plan, pool, y_out, proj, sc)
+    else:
+        sg.lora_delta(x, plan, pool, y_out, proj, sc, v=v)
     sg.check_errors()
     return plan, v, y_out
 

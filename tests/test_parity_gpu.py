@@ -67,53 +67,61 @@ def custom_case(seg_lens, ranks, d_in, d_out, seed=0, minus_one=0, shuffle=True,
     return wl, bank, x, y
 
 
-def check(wl, bank, x, y, long_threshold, y_dtype=torch.bfloat16, proj=0, **kw):
+def check(wl, bank, x, y, long_threshold, y_dtype=torch.bfloat16, proj=0, mode="separate", **kw):
     pool = build_pool(wl, bank)
-    plan, v, y_out = run_gpu(pool, wl, proj, x, y, long_threshold, y_dtype, **kw)
+    plan, v, y_out = run_gpu(pool, wl, proj, x, y, long_threshold, y_dtype, mode=mode, **kw)
     ref = run_oracle(wl, bank, proj, x, y, **kw)
     errs = compare(plan, v, y_out, y, ref)
     return plan, v, y_out, ref, errs
 
 
 # ------------------------------------------------------------------ workloads
+MODES = pytest.mark.parametrize("mode", ["separate", "lora_delta"])
+
+
+@MODES
 @pytest.mark.parametrize("path", [SIMT, TC], ids=["simt", "tc"])
 @pytest.mark.parametrize("y_dtype", [torch.bfloat16, torch.float32], ids=["ybf16", "yfp32"])
-def test_tiny(path, y_dtype):
+def test_tiny(path, y_dtype, mode):
     wl = workloads.make("tiny")
     bank = workloads.AdapterBank(wl, device="cuda")
     x, y = workloads.activations(wl, 0, device="cuda")
-    plan, *_ = check(wl, bank, x, y, path, y_dtype)
+    plan, *_ = check(wl, bank, x, y, path, y_dtype, mode=mode)
     assert (plan.plan.num_tc_tiles > 0) == (path == TC)
 
 
-def test_decode_q_proj():
+@MODES
+def test_decode_q_proj(mode):
     wl = workloads.make("decode_q_proj")
     bank = workloads.AdapterBank(wl, device="cuda")
     x, y = workloads.activations(wl, 0, device="cuda")
-    plan, *_ = check(wl, bank, x, y, 0)
+    plan, *_ = check(wl, bank, x, y, 0, mode=mode)
     assert plan.plan.num_tc_tiles == 0 and plan.plan.num_segments == wl.distinct_adapters
 
 
+@MODES
 @pytest.mark.parametrize("y_dtype", [torch.bfloat16, torch.float32], ids=["ybf16", "yfp32"])
-def test_mixed_rank_mlp_up(y_dtype):
+def test_mixed_rank_mlp_up(y_dtype, mode):
     wl = workloads.make("mixed_rank_mlp_up")
     bank = workloads.AdapterBank(wl, device="cuda")
     x, y = workloads.activations(wl, 0, device="cuda")
-    plan, *_ = check(wl, bank, x, y, 0, y_dtype)
+    plan, *_ = check(wl, bank, x, y, 0, y_dtype, mode=mode)
     assert len(set(plan.seg_rank.tolist())) == 4
 
 
-@pytest.mark.parametrize("path", [0, SIMT], ids=["dispatch", "simt"])
-def test_prefill_long(path):
+@pytest.mark.parametrize("path,mode", [(0, "separate"), (0, "lora_delta"), (SIMT, "separate")],
+                         ids=["dispatch", "dispatch-lora_delta", "simt"])
+def test_prefill_long(path, mode):
     wl = workloads.make("prefill_long")
     bank = workloads.AdapterBank(wl, device="cuda")
     x, y = workloads.activations(wl, 0, device="cuda")
-    plan, *_ = check(wl, bank, x, y, path)
+    plan, *_ = check(wl, bank, x, y, path, mode=mode)
     if path == 0:
         assert plan.plan.num_tc_tiles == 32 and plan.plan.num_simt_items == 0
 
 
-def test_llama70b_layer_sampled():
+@MODES
+def test_llama70b_layer_sampled(mode):
     """Full-size layer (pool of 2000 rank-16 adapters, 7 projections, 256 tokens on
     distinct adapters) in the launch configuration the benchmark times; the oracle
     recomputes a sample of 32 tokens one by one for every projection."""
@@ -124,7 +132,7 @@ def test_llama70b_layer_sampled():
     sample = sorted(rng.choice(wl.T, size=32, replace=False).tolist())
     for p in range(len(wl.projections)):
         x, y = workloads.activations(wl, p, device="cuda")
-        plan, v, y_out = run_gpu(pool, wl, p, x, y)
+        plan, v, y_out = run_gpu(pool, wl, p, x, y, mode=mode)
         ref = run_oracle(wl, bank, p, x, y, rows_of_tokens=sample)
         compare(plan, v, y_out, y, ref, check_rows=sample)
         # every token is its own segment; untouched rows do not exist in this workload
@@ -132,14 +140,16 @@ def test_llama70b_layer_sampled():
 
 
 # ------------------------------------------------------------------ exact pins
+@MODES
 @pytest.mark.parametrize("path", [SIMT, TC], ids=["simt", "tc"])
 @pytest.mark.parametrize("d", [512, 1024, 1536])
-def test_exact_integer_inputs_bit_exact(path, d):
+def test_exact_integer_inputs_bit_exact(path, d, mode):
     """Integer inputs whose every partial sum is exact in bf16/fp32/fp64: the GPU must
     equal the oracle bit for bit, in v and in y, on both paths."""
-    wl, bank, x, y = custom_case([3, 70, 1, 130], [4, 3, 1, 2], d, d, seed=5, minus_one=5, ints=True)
+    wl, bank, x, y = custom_case([3, 70, 1, 130, 5, 8], [4, 3, 1, 2, 16, 9], d, 2 * d, seed=5, minus_one=5,
+                                 ints=True)
     pool = build_pool(wl, bank)
-    plan, v, y_out = run_gpu(pool, wl, 0, x, y, path)
+    plan, v, y_out = run_gpu(pool, wl, 0, x, y, path, mode=mode)
     ref = run_oracle(wl, bank, 0, x, y)
     vg = v.double().cpu().numpy()
     row = {t: i for i, t in enumerate(plan.token_idx.tolist())}
@@ -149,36 +159,39 @@ def test_exact_integer_inputs_bit_exact(path, d):
     assert np.array_equal(y_out.double().cpu().numpy(), ref["y"])
 
 
+@MODES
 @pytest.mark.parametrize("path", [SIMT, TC], ids=["simt", "tc"])
-def test_zero_B_and_zero_scale_leave_y_unchanged(path):
+def test_zero_B_and_zero_scale_leave_y_unchanged(path, mode):
     wl, bank, x, y = custom_case([5, 90], [8, 16], 512, 1024, seed=6)
     for a in range(2):
         A, B = bank.m[(a, 0)]
         bank.m[(a, 0)] = (A, torch.zeros_like(B))
     pool = build_pool(wl, bank)
-    _, _, y_out = run_gpu(pool, wl, 0, x, y, path)
+    _, _, y_out = run_gpu(pool, wl, 0, x, y, path, mode=mode)
     assert torch.equal(y_out.view(torch.int16), y.view(torch.int16))
     wl2, bank2, x2, y2 = custom_case([5, 90], [8, 16], 512, 1024, seed=7)
     pool2 = build_pool(wl2, bank2)
-    _, _, y_out2 = run_gpu(pool2, wl2, 0, x2, y2, path, scale=0.0)
+    _, _, y_out2 = run_gpu(pool2, wl2, 0, x2, y2, path, scale=0.0, mode=mode)
     assert torch.equal(y_out2.view(torch.int16), y2.view(torch.int16))
 
 
 # ------------------------------------------------------------------ edge cases
+@MODES
 @pytest.mark.parametrize("path", [0, SIMT, TC], ids=["dispatch", "simt", "tc"])
-def test_ragged_lengths_and_odd_ranks(path):
-    lens = [1, 63, 64, 65, 127, 128, 129, 200, 2]
-    ranks = [5, 24, 100, 128, 16, 8, 40, 64, 128]
+def test_ragged_lengths_and_odd_ranks(path, mode):
+    lens = [1, 63, 64, 65, 127, 128, 129, 200, 2, 3, 5, 7, 8, 9, 15, 16, 17]
+    ranks = [5, 24, 100, 128, 16, 8, 40, 64, 128, 8, 16, 32, 64, 12, 72, 8, 16]
     wl, bank, x, y = custom_case(lens, ranks, 1536, 2560, seed=8, minus_one=11)
-    check(wl, bank, x, y, path, torch.float32)
+    check(wl, bank, x, y, path, torch.float32, mode=mode)
 
 
+@MODES
 @pytest.mark.parametrize("path", [SIMT, TC], ids=["simt", "tc"])
-def test_single_token_and_rank_zero(path):
+def test_single_token_and_rank_zero(path, mode):
     wl, bank, x, y = custom_case([1], [16], 512, 512, seed=9)
-    check(wl, bank, x, y, path)
+    check(wl, bank, x, y, path, mode=mode)
     wl, bank, x, y = custom_case([3, 4], [0, 8], 512, 512, seed=10, minus_one=2)
-    check(wl, bank, x, y, path)
+    check(wl, bank, x, y, path, mode=mode)
 
 
 def test_empty_batches():
@@ -232,7 +245,8 @@ def test_pool_pages_hold_A_rows_and_Bt_rows():
     assert P == 512
 
 
-def test_device_bounds_checks_report_without_faulting():
+@MODES
+def test_device_bounds_checks_report_without_faulting(mode):
     """A corrupted device table (token row past the batch) is caught by the kernels'
     own bounds checks: the access is skipped and sgmv_check_errors reports it."""
     for path in (SIMT, TC):
@@ -245,9 +259,25 @@ def test_device_bounds_checks_report_without_faulting():
         tix[0] = wl.T + 5
         v = plan.new_v()
         y2 = y.clone()
-        sg.shrink(x, plan, pool, v, 0)
-        sg.expand(v, plan, pool, y2, 0)
+        if mode == "separate":
+            sg.shrink(x, plan, pool, v, 0)
+            sg.expand(v, plan, pool, y2, 0)
+        else:
+            sg.lora_delta(x, plan, pool, y2, 0, v=v)
         with pytest.raises(sg.SgmvError) as e:
             sg.check_errors()
         assert e.value.status == 6
         assert sg.check_errors() == 0   # cleared
+
+
+def test_lora_delta_requires_workspace():
+    wl, bank, x, y = custom_case([1, 2, 3], [16, 8, 32], 1024, 1024, seed=21, minus_one=3)
+    pool = build_pool(wl, bank)
+    plan = pool.plan(wl.adapter_ids)
+    plan.upload()
+    lib = sg.load_library()
+    import ctypes
+    st = lib.sgmv_lora_delta(x.data_ptr(), x.stride(0), plan.T, 1024, 1024, 0, ctypes.byref(plan.plan),
+                             plan.device_table.data_ptr(), pool.handle, 1.0, y.data_ptr(), y.stride(0), 0, None, 0,
+                             None)
+    assert st == 1

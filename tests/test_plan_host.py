@@ -29,17 +29,19 @@ def _check_plan(plan, pool, ids, ranks, thr):
     assert plan.seg_rank.tolist() == [ranks[a] for a in seg_ad]
     assert plan.num_rows == len(tix)
     assert plan.max_rank == max([ranks[a] for a in seg_ad], default=0)
-    # page-table bases agree with the pool's own record
+    # every work record repeats its segment's rank and page-table bases, per projection
     a_pt, b_pt = plan.seg_pt(0), plan.seg_pt(1)
-    for s, a in enumerate(seg_ad):
-        for p in range(len(pool.projections)):
-            for m, base in ((0, a_pt[s, p]), (1, b_pt[s, p])):
-                ids_pool = pool.page_ids(a, p, m)
-                assert ids_pool.size == 0 or True
+    for recs in (plan.simt_records, plan.tc_records):
+        for rec in recs:
+            for p in range(len(pool.projections)):
+                seg = int(rec[p, 0])
+                assert rec[p, 3] == ranks[seg_ad[seg]]
+                assert rec[p, 4] == a_pt[seg, p] and rec[p, 5] == b_pt[seg, p]
+                assert tuple(rec[p, :3]) == tuple(rec[0, :3])
     # dispatch covers every row of every non-empty, non-zero-rank segment exactly once
     covered = []
-    for items, lim, is_tc in ((plan.simt_items, 64, False), (plan.tc_tiles, 128, True)):
-        for s, b, e, _ in items.tolist():
+    for items, lim, is_tc in ((plan.simt_items, 8, False), (plan.tc_tiles, 128, True)):
+        for s, b, e in items.tolist():
             n = off[s + 1] - off[s]
             assert off[s] <= b < e <= off[s + 1] and e - b <= lim
             assert (n >= thr) == is_tc

@@ -283,6 +283,31 @@ SGMV_API sgmv_status sgmv_lora_delta(const void* x, int64_t ldx, int32_t T, int3
                                      int32_t y_dtype, float* v, int64_t ldv, sgmv_stream_t stream);
 
 /*
+ * sgmv_lora_delta for callers that cannot give the library device memory.
+ * No counterpart on the pages: this is a deployment convenience.
+ *
+ * Some callers cannot allocate (their device memory belongs to another
+ * runtime's fixed arena, or the library must not grow the process's device
+ * footprint or trigger cudaMalloc's synchronisation).  This call takes the
+ * same arguments as sgmv_lora_delta without v: the intermediate lives in a
+ * fixed array of 2^19 fp32 (2 MiB) compiled into the library, which every GPU
+ * that loads the library holds until the process exits.  It allocates nothing
+ * and calls no allocating routine.
+ *   - The batch must fit: plan->num_rows * max(4, round_up(plan->max_rank, 4))
+ *     <= 2^19, else SGMV_ERR_CAPACITY (nothing launched).
+ *   - The first call on a device looks up the array's device address, with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls on a device share the array, which keeps the last call's
+ *     contents (nothing in it needs to start at zero).  Calls whose kernels
+ *     overlap on the same device race on it: serialise them (one stream).
+ */
+SGMV_API sgmv_status sgmv_lora_delta_noalloc(const void* x, int64_t ldx, int32_t T, int32_t d_in,
+                                             int32_t d_out, int32_t proj, const sgmv_plan* plan,
+                                             const void* table, const sgmv_pool* pool, float scale,
+                                             void* y, int64_t ldy, int32_t y_dtype,
+                                             sgmv_stream_t stream);
+
+/*
  * Wait for `stream`, then return and clear the device error word:
  * SGMV_OK, SGMV_ERR_BOUNDS or SGMV_ERR_TIMEOUT.  *flags (may be NULL) receives
  * the raw bits (1 = page id out of range, 2 = token row out of range,

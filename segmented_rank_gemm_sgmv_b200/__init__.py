@@ -32,7 +32,8 @@ _STATUS = {0: "SGMV_OK", 1: "SGMV_ERR_INVALID", 2: "SGMV_ERR_UNSUPPORTED", 3: "S
 EXPORTED = ("sgmv_status_string", "sgmv_last_error", "sgmv_pool_create", "sgmv_pool_destroy", "sgmv_pool_load",
             "sgmv_pool_evict", "sgmv_pool_get_stats", "sgmv_pool_adapter_rank", "sgmv_pool_adapter_pages",
             "sgmv_pool_shuffle_free_pages", "sgmv_pool_pages_device", "sgmv_plan_table_capacity",
-            "sgmv_build_plan", "sgmv_shrink", "sgmv_expand", "sgmv_lora_delta", "sgmv_check_errors")
+            "sgmv_build_plan", "sgmv_shrink", "sgmv_expand", "sgmv_lora_delta", "sgmv_lora_delta_noalloc",
+            "sgmv_check_errors")
 
 
 class SgmvError(RuntimeError):
@@ -87,6 +88,8 @@ def load_library() -> ctypes.CDLL:
         "sgmv_expand": (st, [vp, i64, i32, i32, i32, ctypes.POINTER(Plan), vp, vp, f32, vp, i64, i32, vp]),
         "sgmv_lora_delta": (st, [vp, i64, i32, i32, i32, i32, ctypes.POINTER(Plan), vp, vp, f32, vp, i64, i32,
                                  vp, i64, vp]),
+        "sgmv_lora_delta_noalloc": (st, [vp, i64, i32, i32, i32, i32, ctypes.POINTER(Plan), vp, vp, f32, vp, i64,
+                                         i32, vp]),
         "sgmv_check_errors": (st, [vp, ctypes.POINTER(ctypes.c_uint32)]),
     }
     for name, (res, args) in sig.items():
@@ -366,6 +369,19 @@ def expand(v: torch.Tensor, plan: BatchPlan, pool: AdapterPool, y: torch.Tensor,
     _check(load_library().sgmv_expand(_ptr(v), v.stride(0), plan.T, y.shape[1], int(proj), ctypes.byref(plan.plan),
                                       table.data_ptr(), pool.handle, float(scale), _ptr(y), y.stride(0),
                                       0 if y.dtype == torch.bfloat16 else 1, _stream(stream)))
+
+
+def lora_delta_noalloc(x: torch.Tensor, plan: BatchPlan, pool: AdapterPool, y: torch.Tensor, proj: int = 0,
+                       scale: float = 1.0, stream=None) -> None:
+    """lora_delta with the intermediate in the library's fixed device array (no workspace
+    argument, nothing allocated); see sgmv_lora_delta_noalloc in include/sgmv.h."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    assert y.dim() == 2 and y.stride(1) == 1 and y.dtype in (torch.bfloat16, torch.float32)
+    table = plan.device_table if plan.device_table is not None else plan.upload(stream)
+    _check(load_library().sgmv_lora_delta_noalloc(
+        _ptr(x), x.stride(0), plan.T, x.shape[1], y.shape[1], int(proj), ctypes.byref(plan.plan),
+        table.data_ptr(), pool.handle, float(scale), _ptr(y), y.stride(0),
+        0 if y.dtype == torch.bfloat16 else 1, _stream(stream)))
 
 
 def check_errors(stream=None) -> int:

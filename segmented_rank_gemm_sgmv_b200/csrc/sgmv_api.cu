@@ -1,6 +1,7 @@
 // C ABI entry points: argument validation, the size-based dispatch between
 // the SIMT and the tensor-core kernels, and error reporting.
 #include <cstdio>
+#include <mutex>
 #include <string>
 
 #include "internal.h"
@@ -137,6 +138,60 @@ extern "C" sgmv_status sgmv_lora_delta(const void* x, int64_t ldx, int32_t T, in
     sgmv_status st = sgmv_shrink(x, ldx, T, d_in, proj, plan, table, pool, v, ldv, stream);
     if (st != SGMV_OK) return st;
     return sgmv_expand(v, ldv, T, d_out, proj, plan, table, pool, scale, y, ldy, y_dtype, stream);
+}
+
+// ---------------------------------------------------------------------------
+// sgmv_lora_delta without a caller workspace.
+//
+// Some callers cannot hand this library a device buffer for the intermediate
+// v: their device memory is owned by another runtime's fixed arena, or the
+// library is not allowed to grow the process's device footprint or to pay for
+// cudaMalloc's device-wide synchronisation.  For them the workspace lives in
+// the fixed array below, which every GPU that loads this library holds until
+// the process exits.  All calls on a device share it: calls whose kernels
+// overlap on that device race on it, and it keeps whatever the last call left
+// (nothing in it has to start at zero -- the shrink writes every entry the
+// expand then reads).
+constexpr int64_t kNoAllocScratchFloats = int64_t(1) << 19;  // 2 MiB of fp32
+static __device__ __align__(256) float g_noalloc_v[kNoAllocScratchFloats];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+float* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_v on the current device (looked up once per device).
+sgmv_status noalloc_scratch(float** out) {
+    int dev = 0;
+    SGMV_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return fail(SGMV_ERR_UNSUPPORTED, "lora_delta_noalloc: device ordinal too large");
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_v);
+        if (e != cudaSuccess || !p) return cuda_fail(e, "lora_delta_noalloc: cudaGetSymbolAddress");
+        g_noalloc_ptr[dev] = static_cast<float*>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return SGMV_OK;
+}
+}  // namespace
+
+extern "C" sgmv_status sgmv_lora_delta_noalloc(const void* x, int64_t ldx, int32_t T, int32_t d_in, int32_t d_out,
+                                               int32_t proj, const sgmv_plan* plan, const void* table,
+                                               const sgmv_pool* pool, float scale, void* y, int64_t ldy,
+                                               int32_t y_dtype, sgmv_stream_t stream) {
+    if (!plan) return fail(SGMV_ERR_INVALID, "lora_delta_noalloc: plan is required");
+    const int64_t ldv = std::max<int64_t>(4, ((int64_t)plan->max_rank + 3) / 4 * 4);
+    if ((int64_t)plan->num_rows * ldv > kNoAllocScratchFloats)
+        return fail(SGMV_ERR_CAPACITY, "lora_delta_noalloc: the batch needs " +
+                                           std::to_string((int64_t)plan->num_rows * ldv) +
+                                           " fp32 of workspace, above the fixed " +
+                                           std::to_string(kNoAllocScratchFloats) + "; use sgmv_lora_delta");
+    float* v = nullptr;
+    const sgmv_status st = noalloc_scratch(&v);
+    if (st != SGMV_OK) return st;
+    return sgmv_lora_delta(x, ldx, T, d_in, d_out, proj, plan, table, pool, scale, y, ldy, y_dtype, v, ldv, stream);
 }
 
 extern "C" sgmv_status sgmv_check_errors(sgmv_stream_t stream_, uint32_t* flags) {

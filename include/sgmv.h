@@ -201,10 +201,14 @@ typedef struct {
     int32_t num_tc_tiles;
     int32_t long_threshold; /* the threshold actually used                           */
     int32_t max_item_rows;  /* largest SIMT item                                     */
-    int32_t reserved;
+    int32_t needs_device_table; /* 0: the kernels take everything from `host_table` as
+                               launch arguments (<= 64 SIMT items, no tensor-core tiles);
+                               the device table may then be NULL and need not be copied */
     int64_t table_bytes;    /* bytes of the table to copy to the device              */
     int64_t off_token_idx, off_seg_offsets, off_seg_adapter, off_seg_rank;
     int64_t off_seg_a_pt, off_seg_b_pt, off_simt_items, off_tc_tiles;
+    const void* host_table; /* the host table the builder wrote; it must still hold that
+                               table when sgmv_shrink / sgmv_expand are called          */
 } sgmv_plan;
 
 /* Bytes a table may need for a batch of T tokens over n_proj projections. */
@@ -233,7 +237,9 @@ SGMV_API sgmv_status sgmv_build_plan(const int32_t* adapter_ids, int32_t T, cons
  * v       device fp32 [plan->num_rows][ldv], ldv >= plan->max_rank; written
  *         for k < r_s (other entries are left as they were); fp32 accumulation
  * proj    projection index, d_in must equal the pool's d_in[proj]
- * table   device copy of the table that built `plan`
+ * table   device copy of the table that built `plan` (may be NULL when
+ *         plan->needs_device_table is 0: the work items then travel as launch
+ *         arguments, read from plan->host_table at the call)
  * One launch covers every SIMT item (all short segments, any mix of ranks)
  * and one more covers every tensor-core tile, in stream order.  The SIMT
  * path needs the pool's page_elems <= 1024 (else SGMV_ERR_UNSUPPORTED).

@@ -45,9 +45,9 @@ class SgmvError(RuntimeError):
 class Plan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "T", "num_segments", "num_rows", "max_rank", "n_proj", "num_simt_items", "num_tc_tiles",
-        "long_threshold", "max_item_rows", "reserved")] + [(n, ctypes.c_int64) for n in (
+        "long_threshold", "max_item_rows", "needs_device_table")] + [(n, ctypes.c_int64) for n in (
             "table_bytes", "off_token_idx", "off_seg_offsets", "off_seg_adapter", "off_seg_rank",
-            "off_seg_a_pt", "off_seg_b_pt", "off_simt_items", "off_tc_tiles")]
+            "off_seg_a_pt", "off_seg_b_pt", "off_simt_items", "off_tc_tiles")] + [("host_table", ctypes.c_void_p)]
 
 
 class PoolStats(ctypes.Structure):
@@ -330,8 +330,20 @@ class BatchPlan:
         return per * projections
 
     # -- device side
-    def upload(self, stream=None) -> torch.Tensor:
-        """Copy the table to the device on `stream` (one host-to-device copy)."""
+    def table_ptr(self, stream=None) -> Optional[int]:
+        """Device address of the table for the kernel calls, or None when the plan's work
+        items travel as launch arguments (no copy needed)."""
+        if not self.plan.needs_device_table:
+            return None
+        if self.device_table is None:
+            self.upload(stream)
+        return self.device_table.data_ptr()
+
+    def upload(self, stream=None) -> Optional[torch.Tensor]:
+        """Copy the table to the device on `stream` (one host-to-device copy); nothing to do
+        when the plan's work items travel as launch arguments."""
+        if not self.plan.needs_device_table:
+            return None
         n = max(int(self.plan.table_bytes), 16)
         dev = torch.device("cuda", self.pool.device)
         if self.device_table is None or self.device_table.numel() < max(n, self.capacity):
@@ -355,9 +367,8 @@ def shrink(x: torch.Tensor, plan: BatchPlan, pool: AdapterPool, v: torch.Tensor,
     """v[i, k] = sum_c A_s[k, c] x[token_idx[i], c]  (SGMV-shrink)."""
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     assert v.dtype == torch.float32 and v.dim() == 2 and v.stride(1) == 1
-    table = plan.device_table if plan.device_table is not None else plan.upload(stream)
     _check(load_library().sgmv_shrink(_ptr(x), x.stride(0), plan.T, x.shape[1], int(proj), ctypes.byref(plan.plan),
-                                      table.data_ptr(), pool.handle, _ptr(v), v.stride(0), _stream(stream)))
+                                      plan.table_ptr(stream), pool.handle, _ptr(v), v.stride(0), _stream(stream)))
 
 
 def expand(v: torch.Tensor, plan: BatchPlan, pool: AdapterPool, y: torch.Tensor, proj: int = 0,
@@ -365,9 +376,8 @@ def expand(v: torch.Tensor, plan: BatchPlan, pool: AdapterPool, y: torch.Tensor,
     """y[t, j] += scale * sum_k B_s[j, k] v[i, k]  (SGMV-expand, in place, one rounding)."""
     assert v.dtype == torch.float32 and v.dim() == 2 and v.stride(1) == 1
     assert y.dim() == 2 and y.stride(1) == 1 and y.dtype in (torch.bfloat16, torch.float32)
-    table = plan.device_table if plan.device_table is not None else plan.upload(stream)
     _check(load_library().sgmv_expand(_ptr(v), v.stride(0), plan.T, y.shape[1], int(proj), ctypes.byref(plan.plan),
-                                      table.data_ptr(), pool.handle, float(scale), _ptr(y), y.stride(0),
+                                      plan.table_ptr(stream), pool.handle, float(scale), _ptr(y), y.stride(0),
                                       0 if y.dtype == torch.bfloat16 else 1, _stream(stream)))
 
 
@@ -377,10 +387,9 @@ def lora_delta_noalloc(x: torch.Tensor, plan: BatchPlan, pool: AdapterPool, y: t
     argument, nothing allocated); see sgmv_lora_delta_noalloc in include/sgmv.h."""
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     assert y.dim() == 2 and y.stride(1) == 1 and y.dtype in (torch.bfloat16, torch.float32)
-    table = plan.device_table if plan.device_table is not None else plan.upload(stream)
     _check(load_library().sgmv_lora_delta_noalloc(
         _ptr(x), x.stride(0), plan.T, x.shape[1], y.shape[1], int(proj), ctypes.byref(plan.plan),
-        table.data_ptr(), pool.handle, float(scale), _ptr(y), y.stride(0),
+        plan.table_ptr(stream), pool.handle, float(scale), _ptr(y), y.stride(0),
         0 if y.dtype == torch.bfloat16 else 1, _stream(stream)))
 
 
@@ -400,9 +409,8 @@ def lora_delta(x: torch.Tensor, plan: BatchPlan, pool: AdapterPool, y: torch.Ten
     if v is None:
         v = plan.new_v()
     assert v.dtype == torch.float32 and v.dim() == 2 and v.stride(1) == 1
-    table = plan.device_table if plan.device_table is not None else plan.upload(stream)
     _check(load_library().sgmv_lora_delta(
         _ptr(x), x.stride(0), plan.T, x.shape[1], y.shape[1], int(proj), ctypes.byref(plan.plan),
-        table.data_ptr(), pool.handle, float(scale), _ptr(y), y.stride(0),
+        plan.table_ptr(stream), pool.handle, float(scale), _ptr(y), y.stride(0),
         0 if y.dtype == torch.bfloat16 else 1, _ptr(v), v.stride(0), _stream(stream)))
     return v

@@ -62,6 +62,21 @@ struct ItemRec {
 static_assert(sizeof(ItemRec) == 32, "ItemRec must be 32 bytes");
 
 constexpr int kSimtMaxItemRows = 8;    // rows per SIMT work item
+constexpr int kInlineItems = 64;       // SIMT items that can travel as launch arguments
+
+// A SIMT work item passed by value in the kernel's parameters: the record for
+// the launch's projection plus the item's token rows.
+struct InlineItem {
+    int32_t seg, row_begin, row_end, rank;
+    int64_t a_pt, b_pt;
+    int32_t tok[kSimtMaxItemRows];
+};
+static_assert(sizeof(InlineItem) == 64, "InlineItem must be 64 bytes");
+template <int N>
+struct InlineTable {
+    int32_t count, pad[3];
+    InlineItem items[N];
+};
 constexpr int kTcTileRows = 128;       // rows per tensor-core tile (MMA M)
 constexpr int kDefaultLongThreshold = 16;
 constexpr int kMaxRank = 128;
@@ -87,12 +102,16 @@ struct PoolView {
 };
 
 // --------------------------------------------------------------- launchers
+// `inl` (may be null) holds the items as launch arguments when they fit.
 cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, const BatchView& b,
                                int32_t num_items, int32_t max_item_rows, int32_t max_rank, const PoolView& pool,
-                               float* v, int64_t ldv, cudaStream_t stream);
+                               float* v, int64_t ldv, const InlineTable<kInlineItems>* inl, cudaStream_t stream);
+// y_early: y may be read before the preceding kernel completes (that kernel is
+// the shrink of the same call, which does not write y).
 cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const BatchView& b,
                                int32_t num_items, int32_t max_item_rows, int32_t max_rank, const PoolView& pool,
-                               float scale, void* y, int64_t ldy, int32_t y_dtype, cudaStream_t stream);
+                               float scale, void* y, int64_t ldy, int32_t y_dtype,
+                               const InlineTable<kInlineItems>* inl, bool y_early, cudaStream_t stream);
 cudaError_t launch_shrink_tc(const uint16_t* x, int64_t ldx, int32_t d_in, const BatchView& b, int32_t num_tiles,
                              int32_t max_rank, const PoolView& pool, float* v, int64_t ldv, cudaStream_t stream);
 cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const BatchView& b, int32_t num_tiles,

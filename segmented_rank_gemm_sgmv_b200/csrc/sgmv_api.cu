@@ -35,16 +35,21 @@ sgmv_status make_views(const sgmv_plan* plan, const void* table, const sgmv_pool
     if (plan->T != T) return fail(SGMV_ERR_INVALID, w + ": T differs from the plan's T");
     if (plan->n_proj != pool->n_proj) return fail(SGMV_ERR_INVALID, w + ": plan was built for another pool");
     if (proj < 0 || proj >= pool->n_proj) return fail(SGMV_ERR_INVALID, w + ": projection index out of range");
-    if (plan->table_bytes > 0 && (!table || !aligned16(table)))
-        return fail(SGMV_ERR_INVALID, w + ": table must be a 16-byte aligned device pointer");
+    if (plan->needs_device_table && (!table || !aligned16(table)))
+        return fail(SGMV_ERR_INVALID, w + ": this plan needs its table as a 16-byte aligned device pointer");
+    if (!plan->needs_device_table && !table && !plan->host_table)
+        return fail(SGMV_ERR_INVALID, w + ": plan->host_table is NULL and no device table was given");
     const uint8_t* base = static_cast<const uint8_t*>(table);
-    bv->token_idx = reinterpret_cast<const int32_t*>(base + plan->off_token_idx);
-    bv->seg_offsets = reinterpret_cast<const int32_t*>(base + plan->off_seg_offsets);
-    bv->seg_rank = reinterpret_cast<const int32_t*>(base + plan->off_seg_rank);
-    bv->seg_a_pt = reinterpret_cast<const int64_t*>(base + plan->off_seg_a_pt);
-    bv->seg_b_pt = reinterpret_cast<const int64_t*>(base + plan->off_seg_b_pt);
-    bv->simt_items = reinterpret_cast<const ItemRec*>(base + plan->off_simt_items);
-    bv->tc_tiles = reinterpret_cast<const ItemRec*>(base + plan->off_tc_tiles);
+    *bv = BatchView{};
+    if (base) {
+        bv->token_idx = reinterpret_cast<const int32_t*>(base + plan->off_token_idx);
+        bv->seg_offsets = reinterpret_cast<const int32_t*>(base + plan->off_seg_offsets);
+        bv->seg_rank = reinterpret_cast<const int32_t*>(base + plan->off_seg_rank);
+        bv->seg_a_pt = reinterpret_cast<const int64_t*>(base + plan->off_seg_a_pt);
+        bv->seg_b_pt = reinterpret_cast<const int64_t*>(base + plan->off_seg_b_pt);
+        bv->simt_items = reinterpret_cast<const ItemRec*>(base + plan->off_simt_items);
+        bv->tc_tiles = reinterpret_cast<const ItemRec*>(base + plan->off_tc_tiles);
+    }
     bv->num_segments = plan->num_segments;
     bv->num_rows = plan->num_rows;
     bv->n_proj = plan->n_proj;
@@ -58,7 +63,40 @@ sgmv_status make_views(const sgmv_plan* plan, const void* table, const sgmv_pool
     return SGMV_OK;
 }
 
+// The SIMT items of `plan` for projection `proj` as launch arguments, read from
+// the host table; false when they do not fit (the kernels then read the
+// device table).
+bool inline_items(const sgmv_plan* plan, int32_t proj, InlineTable<kInlineItems>* t) {
+    if (!plan->host_table || plan->num_simt_items <= 0 || plan->num_simt_items > kInlineItems) return false;
+    const uint8_t* base = static_cast<const uint8_t*>(plan->host_table);
+    const ItemRec* recs = reinterpret_cast<const ItemRec*>(base + plan->off_simt_items);
+    const int32_t* tix = reinterpret_cast<const int32_t*>(base + plan->off_token_idx);
+    t->count = plan->num_simt_items;
+    for (int i = 0; i < plan->num_simt_items; ++i) {
+        const ItemRec& r = recs[(int64_t)i * plan->n_proj + proj];
+        InlineItem& it = t->items[i];
+        it.seg = r.seg;
+        it.row_begin = r.row_begin;
+        it.row_end = r.row_end;
+        it.rank = r.rank;
+        it.a_pt = r.a_pt;
+        it.b_pt = r.b_pt;
+        for (int j = 0; j < kSimtMaxItemRows; ++j) {
+            const int row = r.row_begin + j;
+            it.tok[j] = (row < r.row_end && row >= 0 && row < plan->num_rows) ? tix[row] : -1;
+        }
+    }
+    return true;
+}
+
 }  // namespace
+
+sgmv_status shrink_impl(const void* x, int64_t ldx, int32_t T, int32_t d_in, int32_t proj, const sgmv_plan* plan,
+                        const void* table, const sgmv_pool* pool, float* v, int64_t ldv, cudaStream_t stream);
+sgmv_status expand_impl(const float* v, int64_t ldv, int32_t T, int32_t d_out, int32_t proj, const sgmv_plan* plan,
+                        const void* table, const sgmv_pool* pool, float scale, void* y, int64_t ldy, int32_t y_dtype,
+                        bool y_early, cudaStream_t stream);
+
 }  // namespace sgmv
 
 using namespace sgmv;
@@ -82,8 +120,20 @@ extern "C" const char* sgmv_last_error(void) { return t_last_error.c_str(); }
 
 extern "C" sgmv_status sgmv_shrink(const void* x, int64_t ldx, int32_t T, int32_t d_in, int32_t proj,
                                    const sgmv_plan* plan, const void* table, const sgmv_pool* pool, float* v,
-                                   int64_t ldv, sgmv_stream_t stream_) {
-    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+                                   int64_t ldv, sgmv_stream_t stream) {
+    return shrink_impl(x, ldx, T, d_in, proj, plan, table, pool, v, ldv, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" sgmv_status sgmv_expand(const float* v, int64_t ldv, int32_t T, int32_t d_out, int32_t proj,
+                                   const sgmv_plan* plan, const void* table, const sgmv_pool* pool, float scale,
+                                   void* y, int64_t ldy, int32_t y_dtype, sgmv_stream_t stream) {
+    return expand_impl(v, ldv, T, d_out, proj, plan, table, pool, scale, y, ldy, y_dtype, false,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+sgmv_status sgmv::shrink_impl(const void* x, int64_t ldx, int32_t T, int32_t d_in, int32_t proj,
+                              const sgmv_plan* plan, const void* table, const sgmv_pool* pool, float* v,
+                              int64_t ldv, cudaStream_t stream) {
     BatchView bv;
     PoolView pv;
     sgmv_status st = make_views(plan, table, pool, T, proj, &bv, &pv, "shrink");
@@ -97,16 +147,17 @@ extern "C" sgmv_status sgmv_shrink(const void* x, int64_t ldx, int32_t T, int32_
     if (plan->num_simt_items > 0 && pool->page_elems > 1024)
         return fail(SGMV_ERR_UNSUPPORTED, "shrink: the SIMT path takes page_elems <= 1024");
     const uint16_t* xb = static_cast<const uint16_t*>(x);
+    InlineTable<kInlineItems> inl;
+    const bool use_inl = inline_items(plan, proj, &inl);
     SGMV_CUDA_TRY(launch_shrink_simt(xb, ldx, d_in, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, pv,
-                                     v, ldv, stream));
+                                     v, ldv, use_inl ? &inl : nullptr, stream));
     SGMV_CUDA_TRY(launch_shrink_tc(xb, ldx, d_in, bv, plan->num_tc_tiles, plan->max_rank, pv, v, ldv, stream));
     return SGMV_OK;
 }
 
-extern "C" sgmv_status sgmv_expand(const float* v, int64_t ldv, int32_t T, int32_t d_out, int32_t proj,
-                                   const sgmv_plan* plan, const void* table, const sgmv_pool* pool, float scale,
-                                   void* y, int64_t ldy, int32_t y_dtype, sgmv_stream_t stream_) {
-    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+sgmv_status sgmv::expand_impl(const float* v, int64_t ldv, int32_t T, int32_t d_out, int32_t proj,
+                              const sgmv_plan* plan, const void* table, const sgmv_pool* pool, float scale, void* y,
+                              int64_t ldy, int32_t y_dtype, bool y_early, cudaStream_t stream) {
     BatchView bv;
     PoolView pv;
     sgmv_status st = make_views(plan, table, pool, T, proj, &bv, &pv, "expand");
@@ -122,8 +173,10 @@ extern "C" sgmv_status sgmv_expand(const float* v, int64_t ldv, int32_t T, int32
         return fail(SGMV_ERR_INVALID, "expand: v needs ldv >= max_rank, ldv % 4 == 0, 16-byte alignment");
     if (plan->num_simt_items > 0 && pool->page_elems > 1024)
         return fail(SGMV_ERR_UNSUPPORTED, "expand: the SIMT path takes page_elems <= 1024");
+    InlineTable<kInlineItems> inl;
+    const bool use_inl = inline_items(plan, proj, &inl);
     SGMV_CUDA_TRY(launch_expand_simt(v, ldv, d_out, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, pv,
-                                     scale, y, ldy, y_dtype, stream));
+                                     scale, y, ldy, y_dtype, use_inl ? &inl : nullptr, y_early, stream));
     SGMV_CUDA_TRY(launch_expand_tc(v, ldv, d_out, bv, plan->num_tc_tiles, plan->max_rank, pv, scale, y, ldy, y_dtype,
                                    stream));
     return SGMV_OK;
@@ -135,9 +188,11 @@ extern "C" sgmv_status sgmv_lora_delta(const void* x, int64_t ldx, int32_t T, in
                                        sgmv_stream_t stream) {
     if (plan && plan->num_rows > 0 && (plan->num_simt_items > 0 || plan->num_tc_tiles > 0) && !v)
         return fail(SGMV_ERR_INVALID, "lora_delta: the workspace v is required");
-    sgmv_status st = sgmv_shrink(x, ldx, T, d_in, proj, plan, table, pool, v, ldv, stream);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    sgmv_status st = shrink_impl(x, ldx, T, d_in, proj, plan, table, pool, v, ldv, s);
     if (st != SGMV_OK) return st;
-    return sgmv_expand(v, ldv, T, d_out, proj, plan, table, pool, scale, y, ldy, y_dtype, stream);
+    // the expand's predecessor is this shrink, which does not write y: y may be read early
+    return expand_impl(v, ldv, T, d_out, proj, plan, table, pool, scale, y, ldy, y_dtype, true, s);
 }
 
 // ---------------------------------------------------------------------------

@@ -29,6 +29,9 @@
 //          8 tokens and updates y with one rounding, pass by pass.
 #include <cuda_bf16.h>
 
+#include <map>
+#include <mutex>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -70,6 +73,7 @@ struct ExpandArgs {
     void* y;
     int64_t ldy;
     int32_t y_dtype;
+    int32_t y_early;        // y may be read before the preceding kernel (the shrink) completes
     int32_t ctas_per_item;  // CTAs covering d_out for one item
     int32_t npass;          // 1024-column passes per CTA
     int32_t stages;
@@ -81,8 +85,32 @@ struct ItemInfo {
     int i0, n, r;
     int64_t pt;          // first page-table entry of the matrix for this projection
     bool ok;
+    int tok[kSimtMaxItemRows];  // token rows of the item (-1 past n or when out of range)
 };
 
+__device__ __forceinline__ void check_item(const BatchView& b, ItemInfo& m, int seg, int row_end, int max_rows,
+                                           int max_rank) {
+    m.ok = seg >= 0 && seg < b.num_segments && m.i0 >= 0 && m.n > 0 && m.n <= max_rows && row_end <= b.num_rows &&
+           m.r > 0 && m.r <= max_rank;
+    if (!m.ok) {
+        m.n = 0;
+        m.r = 0;
+    }
+}
+
+__device__ __forceinline__ void finish_tokens(const BatchView& b, ItemInfo& m) {
+#pragma unroll
+    for (int j = 0; j < kSimtMaxItemRows; ++j) {
+        if (j >= m.n) {
+            m.tok[j] = -1;
+        } else if (m.tok[j] < 0 || m.tok[j] >= b.T) {
+            if (threadIdx.x == 0) atomicOr(&g_err_simt, kErrToken);
+            m.tok[j] = -1;
+        }
+    }
+}
+
+// Work item `idx` from the device table: one 32-byte record, then the token rows.
 __device__ __forceinline__ ItemInfo load_item(const BatchView& b, int idx, int max_rows, int max_rank, int matrix) {
     ItemInfo m;
     const int4* rp = reinterpret_cast<const int4*>(b.simt_items + ((int64_t)idx * b.n_proj + b.proj));
@@ -90,14 +118,29 @@ __device__ __forceinline__ ItemInfo load_item(const BatchView& b, int idx, int m
     m.i0 = h.y;
     m.n = h.z - h.y;
     m.r = h.w;
-    m.ok = h.x >= 0 && h.x < b.num_segments && h.y >= 0 && m.n > 0 && m.n <= max_rows && h.z <= b.num_rows &&
-           m.r > 0 && m.r <= max_rank;
+    check_item(b, m, h.x, h.z, max_rows, max_rank);
     m.pt = matrix == 0 ? (int64_t)(((uint64_t)(uint32_t)t.y << 32) | (uint32_t)t.x)
                        : (int64_t)(((uint64_t)(uint32_t)t.w << 32) | (uint32_t)t.z);
-    if (!m.ok) {
-        m.n = 0;
-        m.r = 0;
-    }
+#pragma unroll
+    for (int j = 0; j < kSimtMaxItemRows; ++j) m.tok[j] = j < m.n ? b.token_idx[m.i0 + j] : -1;
+    finish_tokens(b, m);
+    return m;
+}
+
+// Work item `idx` from the launch arguments.
+template <int N>
+__device__ __forceinline__ ItemInfo load_item(const BatchView& b, const InlineTable<N>& t, int idx, int max_rows,
+                                              int max_rank, int matrix) {
+    ItemInfo m;
+    const InlineItem& it = t.items[idx];
+    m.i0 = it.row_begin;
+    m.n = it.row_end - it.row_begin;
+    m.r = it.rank;
+    check_item(b, m, it.seg, it.row_end, max_rows, max_rank);
+    m.pt = matrix == 0 ? it.a_pt : it.b_pt;
+#pragma unroll
+    for (int j = 0; j < kSimtMaxItemRows; ++j) m.tok[j] = it.tok[j];
+    finish_tokens(b, m);
     return m;
 }
 
@@ -248,14 +291,7 @@ __device__ void shrink_item(const ShrinkArgs& a, const ItemInfo& m, uint32_t q, 
     const int tid = threadIdx.x, col = kVec * tid;
     const uint16_t* xrow[G];
 #pragma unroll
-    for (int j = 0; j < G; ++j) {
-        xrow[j] = nullptr;
-        if (j < m.n) {
-            const int t = a.b.token_idx[m.i0 + j];
-            if (t >= 0 && t < a.b.T) xrow[j] = a.x + (int64_t)t * a.ldx + (int64_t)q * a.kc;
-            else atomicOr(&g_err_simt, kErrToken);
-        }
-    }
+    for (int j = 0; j < G; ++j) xrow[j] = m.tok[j] >= 0 ? a.x + (int64_t)m.tok[j] * a.ldx + (int64_t)q * a.kc : nullptr;
     for (int g = 0; g < sg.NG; ++g) {
         float p[kRowGroup * G];
 #pragma unroll
@@ -293,8 +329,9 @@ __device__ void shrink_item(const ShrinkArgs& a, const ItemInfo& m, uint32_t q, 
     }
 }
 
-template <int MAXG>
-__global__ void __launch_bounds__(kThreads, MAXG == 8 ? 2 : 3) shrink_simt_kernel(const ShrinkArgs a) {
+template <int MAXG, int NI>
+__global__ void __launch_bounds__(kThreads, MAXG == 8 ? 2 : 3)
+    shrink_simt_kernel(const ShrinkArgs a, const __grid_constant__ InlineTable<NI> inl) {
     extern __shared__ __align__(128) uint8_t smem[];
     pdl_launch_dependents();  // the expand may start staging its B^T pages now
     const int C = a.cluster;
@@ -304,7 +341,8 @@ __global__ void __launch_bounds__(kThreads, MAXG == 8 ? 2 : 3) shrink_simt_kerne
     float* red = part + kSimtMaxItemRows * a.max_rank;  // [4 warps][64]
     int32_t* pid = reinterpret_cast<int32_t*>(red + 4 * 64);
 
-    const ItemInfo m = load_item(a.b, item_idx, MAXG, a.max_rank, 0);
+    const ItemInfo m = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 0)
+                              : load_item(a.b, item_idx, MAXG, a.max_rank, 0);
     if (!m.ok && threadIdx.x == 0) atomicOr(&g_err_simt, kErrRows);
     StageGeom sg;
     sg.NG = (m.r + kRowGroup - 1) / kRowGroup;
@@ -353,25 +391,16 @@ __global__ void __launch_bounds__(kThreads, MAXG == 8 ? 2 : 3) shrink_simt_kerne
 // ------------------------------------------------------------------ expand
 template <int G>
 __device__ void expand_item(const ExpandArgs& a, const ItemInfo& m, Pipe<kExpandStages>& pp, const StageGeom& sg,
-                            const float* vs) {
+                            float* vs) {
     const int tid = threadIdx.x, col = kVec * tid;
     int trow[G];
 #pragma unroll
-    for (int j = 0; j < G; ++j) {
-        trow[j] = -1;
-        if (j < m.n) {
-            const int t = a.b.token_idx[m.i0 + j];
-            if (t >= 0 && t < a.b.T) trow[j] = t;
-            else if (tid == 0) atomicOr(&g_err_simt, kErrToken);
-        }
-    }
-    for (int s = 0; s < sg.npass; ++s) {
-        const int c = s * kPass, W = min(kPass, sg.span - c);
-        const bool active = col < W;
+    for (int j = 0; j < G; ++j) trow[j] = m.tok[j];
+    uint4 yb[G];
+    float4 yf0[G], yf1[G];
+    auto load_y = [&](int c) {  // y of the pass starting at column c, kept for after the accumulation
         const int jcol = sg.col_base + c + col;
-        // y of this pass: issued now, used after the accumulation
-        uint4 yb[G];
-        float4 yf0[G], yf1[G];
+        const bool active = col < min(kPass, sg.span - c);
 #pragma unroll
         for (int j = 0; j < G; ++j) {
             if (active && trow[j] >= 0) {
@@ -385,6 +414,19 @@ __device__ void expand_item(const ExpandArgs& a, const ItemInfo& m, Pipe<kExpand
                 }
             }
         }
+    };
+    if (a.y_early) load_y(0);
+    pdl_wait();  // v (and, unless y_early, y) are final once the preceding kernel has completed
+    for (int e = tid; e < m.n * m.r; e += kThreads) {
+        const int jrow = e / m.r, k = e - jrow * m.r;
+        vs[e] = a.v[(int64_t)(m.i0 + jrow) * a.ldv + k];
+    }
+    // (the first pipe_acquire's barrier publishes vs)
+    for (int s = 0; s < sg.npass; ++s) {
+        const int c = s * kPass, W = min(kPass, sg.span - c);
+        const bool active = col < W;
+        const int jcol = sg.col_base + c + col;
+        if (s > 0 || !a.y_early) load_y(c);
         float acc[G][8];
 #pragma unroll
         for (int j = 0; j < G; ++j)
@@ -441,14 +483,16 @@ __device__ void expand_item(const ExpandArgs& a, const ItemInfo& m, Pipe<kExpand
     }
 }
 
-template <int MAXG>
-__global__ void __launch_bounds__(kThreads, MAXG == 8 ? 2 : 3) expand_simt_kernel(const ExpandArgs a) {
+template <int MAXG, int NI>
+__global__ void __launch_bounds__(kThreads, MAXG == 8 ? 2 : 3)
+    expand_simt_kernel(const ExpandArgs a, const __grid_constant__ InlineTable<NI> inl) {
     extern __shared__ __align__(128) uint8_t smem_e[];
     const int part_idx = blockIdx.x % a.ctas_per_item, item_idx = blockIdx.x / a.ctas_per_item;
     float* vs = reinterpret_cast<float*>(smem_e);
     int32_t* pid = reinterpret_cast<int32_t*>(vs + kSimtMaxItemRows * a.max_rank);
 
-    const ItemInfo m = load_item(a.b, item_idx, MAXG, a.max_rank, 1);
+    const ItemInfo m = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 1)
+                              : load_item(a.b, item_idx, MAXG, a.max_rank, 1);
     const int j0 = part_idx * a.npass * kPass;
     StageGeom sg;
     sg.NG = (m.r + kRowGroup - 1) / kRowGroup;
@@ -467,17 +511,12 @@ __global__ void __launch_bounds__(kThreads, MAXG == 8 ? 2 : 3) expand_simt_kerne
     // B^T pages do not depend on the shrink: start them before waiting for it
 #pragma unroll 1
     for (int i = 0; i < kExpandStages; ++i) pipe_issue(a.pool, pp, sg, true);
-    pdl_wait();  // v (and y) are final once the preceding kernel has completed
     if (!work) {
+        pdl_wait();
         if (threadIdx.x == 0 && !m.ok) atomicOr(&g_err_simt, kErrRows);
         cp_async_wait<0>();
         return;
     }
-    for (int e = threadIdx.x; e < m.n * m.r; e += kThreads) {
-        const int jrow = e / m.r, k = e - jrow * m.r;
-        vs[e] = a.v[(int64_t)(m.i0 + jrow) * a.ldv + k];
-    }
-    // (the first pipe_acquire's barrier publishes vs)
     if (MAXG == 1 || m.n == 1) expand_item<1>(a, m, pp, sg, vs);
     else if (MAXG == 2 || m.n == 2) expand_item<(MAXG < 2 ? MAXG : 2)>(a, m, pp, sg, vs);
     else if (MAXG == 4 || m.n <= 4) expand_item<(MAXG < 4 ? MAXG : 4)>(a, m, pp, sg, vs);
@@ -497,6 +536,22 @@ int num_sms() {
 
 }  // namespace
 
+// Raise a kernel's dynamic shared-memory limit when a launch needs more than
+// any earlier launch of that kernel did.
+template <typename K>
+cudaError_t set_smem(K kern, size_t bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<int, const void*>, size_t> done;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    size_t& cur = done[{dev, reinterpret_cast<const void*>(kern)}];
+    if (bytes <= cur) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) cur = bytes;
+    return e;
+}
+
 template <typename K1, typename K2, typename K4, typename K8>
 auto pick(int max_item_rows, K1 k1, K2 k2, K4 k4, K8 k8) {
     return max_item_rows <= 1 ? k1 : max_item_rows <= 2 ? k2 : max_item_rows <= 4 ? k4 : k8;
@@ -504,10 +559,8 @@ auto pick(int max_item_rows, K1 k1, K2 k2, K4 k4, K8 k8) {
 
 cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, const BatchView& b, int32_t num_items,
                                int32_t max_item_rows, int32_t max_rank, const PoolView& pool, float* v, int64_t ldv,
-                               cudaStream_t stream) {
+                               const InlineTable<kInlineItems>* inl, cudaStream_t stream) {
     if (num_items <= 0) return cudaSuccess;
-    auto kern = pick(max_item_rows, shrink_simt_kernel<1>, shrink_simt_kernel<2>, shrink_simt_kernel<4>,
-                     shrink_simt_kernel<8>);
     // Cluster size: enough CTAs for two per SM, chunks of >= 1024 columns, at most 8.
     const int pages = d_in >> pool.page_log2;
     const int target = (2 * num_sms() + num_items - 1) / num_items;
@@ -539,8 +592,6 @@ cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, con
     const size_t pid_bytes = (size_t)a.max_rank * (a.kc >> pool.page_log2) * 4;
     a.ring_offset = (int)(((size_t)kSimtMaxItemRows * a.max_rank * 4 + 1024 + pid_bytes + 127) & ~(size_t)127);
     const size_t smem = (size_t)a.ring_offset + (size_t)kShrinkStages * kStageElems * 2;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(C * num_items), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -553,15 +604,25 @@ cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, con
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a);
+    if (inl) {
+        auto kern = pick(max_item_rows, shrink_simt_kernel<1, kInlineItems>, shrink_simt_kernel<2, kInlineItems>,
+                         shrink_simt_kernel<4, kInlineItems>, shrink_simt_kernel<8, kInlineItems>);
+        cudaError_t e = set_smem(kern, smem);
+        if (e != cudaSuccess) return e;
+        return cudaLaunchKernelEx(&cfg, kern, a, *inl);
+    }
+    auto kern = pick(max_item_rows, shrink_simt_kernel<1, 1>, shrink_simt_kernel<2, 1>, shrink_simt_kernel<4, 1>,
+                     shrink_simt_kernel<8, 1>);
+    cudaError_t e = set_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&cfg, kern, a, InlineTable<1>{});
 }
 
 cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const BatchView& b, int32_t num_items,
                                int32_t max_item_rows, int32_t max_rank, const PoolView& pool, float scale, void* y,
-                               int64_t ldy, int32_t y_dtype, cudaStream_t stream) {
+                               int64_t ldy, int32_t y_dtype, const InlineTable<kInlineItems>* inl, bool y_early,
+                               cudaStream_t stream) {
     if (num_items <= 0) return cudaSuccess;
-    auto kern = pick(max_item_rows, expand_simt_kernel<1>, expand_simt_kernel<2>, expand_simt_kernel<4>,
-                     expand_simt_kernel<8>);
     ExpandArgs a;
     a.v = v;
     a.ldv = ldv;
@@ -572,6 +633,7 @@ cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const
     a.y = y;
     a.ldy = ldy;
     a.y_dtype = y_dtype;
+    a.y_early = y_early ? 1 : 0;
     // About four CTAs per SM: CTAs per item k, each covering npass 1024-column passes.
     const int tiles = (d_out + kPass - 1) / kPass;
     const int k = std::max(1, std::min(tiles, (4 * num_sms() + num_items / 2) / num_items));
@@ -584,8 +646,6 @@ cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const
     const size_t pid_bytes = (size_t)a.max_rank * ((a.npass * kPass) >> pool.page_log2) * 4;
     a.ring_offset = (int)(((size_t)kSimtMaxItemRows * a.max_rank * 4 + pid_bytes + 127) & ~(size_t)127);
     const size_t smem = (size_t)a.ring_offset + (size_t)kExpandStages * kStageElems * 2;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.ctas_per_item * num_items), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -596,7 +656,18 @@ cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a);
+    if (inl) {
+        auto kern = pick(max_item_rows, expand_simt_kernel<1, kInlineItems>, expand_simt_kernel<2, kInlineItems>,
+                         expand_simt_kernel<4, kInlineItems>, expand_simt_kernel<8, kInlineItems>);
+        cudaError_t e = set_smem(kern, smem);
+        if (e != cudaSuccess) return e;
+        return cudaLaunchKernelEx(&cfg, kern, a, *inl);
+    }
+    auto kern = pick(max_item_rows, expand_simt_kernel<1, 1>, expand_simt_kernel<2, 1>, expand_simt_kernel<4, 1>,
+                     expand_simt_kernel<8, 1>);
+    cudaError_t e = set_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&cfg, kern, a, InlineTable<1>{});
 }
 
 cudaError_t read_clear_errors_simt(uint32_t* bits, cudaStream_t stream) {

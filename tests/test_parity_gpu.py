@@ -253,9 +253,12 @@ def test_device_bounds_checks_report_without_faulting(mode):
         wl, bank, x, y = custom_case([3, 130], [8, 16], 512, 512, seed=15)
         pool = build_pool(wl, bank)
         plan = pool.plan(wl.adapter_ids, long_threshold=path)
-        table = plan.upload()
-        torch.cuda.synchronize()
-        tix = table[plan.plan.off_token_idx:plan.plan.off_token_idx + 4 * plan.num_rows].view(torch.int32)
+        if plan.plan.needs_device_table:     # the kernels read the device copy: corrupt that
+            table = plan.upload()
+            torch.cuda.synchronize()
+            tix = table[plan.plan.off_token_idx:plan.plan.off_token_idx + 4 * plan.num_rows].view(torch.int32)
+        else:                                # the work items travel as launch arguments, built from the host table
+            tix = plan.host[plan.plan.off_token_idx:plan.plan.off_token_idx + 4 * plan.num_rows].view(torch.int32)
         tix[0] = wl.T + 5
         v = plan.new_v()
         y2 = y.clone()
@@ -278,6 +281,6 @@ def test_lora_delta_requires_workspace():
     lib = sg.load_library()
     import ctypes
     st = lib.sgmv_lora_delta(x.data_ptr(), x.stride(0), plan.T, 1024, 1024, 0, ctypes.byref(plan.plan),
-                             plan.device_table.data_ptr(), pool.handle, 1.0, y.data_ptr(), y.stride(0), 0, None, 0,
+                             plan.table_ptr(), pool.handle, 1.0, y.data_ptr(), y.stride(0), 0, None, 0,
                              None)
     assert st == 1

@@ -43,7 +43,7 @@ def _case(seed, lens, ranks, d_in, d_out):
 def _call_noalloc(x, plan, pool, y):
     lib = sg.load_library()
     return lib.sgmv_lora_delta_noalloc(x.data_ptr(), x.stride(0), plan.T, x.shape[1], y.shape[1], 0,
-                                       ctypes.byref(plan.plan), plan.device_table.data_ptr(), pool.handle, 1.0,
+                                       ctypes.byref(plan.plan), plan.table_ptr(), pool.handle, 1.0,
                                        y.data_ptr(), y.stride(0), 0, torch.cuda.current_stream().cuda_stream)
 
 

@@ -188,7 +188,7 @@ SGMV_API const void* sgmv_pool_pages_device(const sgmv_pool* pool);
  * are never touched.  Segments of rank 0 produce no work item.  A segment
  * with at least `long_threshold` rows goes to the tensor-core path as
  * 128-row tiles; shorter segments go to the SIMT path as items of at most
- * 8 rows (long_threshold <= 0 selects the built-in default, 16; a huge value
+ * 4 rows (long_threshold <= 0 selects the built-in default, 16; a huge value
  * keeps every segment on the SIMT path; 1 sends every segment to tensor cores).
  */
 typedef struct {

@@ -61,7 +61,7 @@ struct ItemRec {
 };
 static_assert(sizeof(ItemRec) == 32, "ItemRec must be 32 bytes");
 
-constexpr int kSimtMaxItemRows = 8;    // rows per SIMT work item
+constexpr int kSimtMaxItemRows = 4;    // rows per SIMT work item
 constexpr int kInlineItems = 64;       // SIMT items that can travel as launch arguments
 
 // A SIMT work item passed by value in the kernel's parameters: the record for
@@ -71,7 +71,7 @@ struct InlineItem {
     int64_t a_pt, b_pt;
     int32_t tok[kSimtMaxItemRows];
 };
-static_assert(sizeof(InlineItem) == 64, "InlineItem must be 64 bytes");
+static_assert(sizeof(InlineItem) == 48, "InlineItem must be 48 bytes");
 template <int N>
 struct InlineTable {
     int32_t count, pad[3];

@@ -15,10 +15,10 @@
 // as a programmatic dependent of the shrink so that its B^T stages stream in
 // while the shrink is still running.
 //
-// shrink:  a thread-block cluster of C CTAs per work item (<= 8 rows of one
+// shrink:  a thread-block cluster of C CTAs per work item (<= 4 rows of one
 //          segment); CTA q owns d_in columns [q kc, (q+1) kc).  Stages are 8
 //          rank rows x up to 1024 columns; each thread owns 8 columns and
-//          keeps the item's (up to 8) tokens' x in registers; partial dot products are
+//          keeps the item's (up to 4) tokens' x in registers; partial dot products are
 //          reduced with warp shuffles and shared memory, then the C partial
 //          tiles are summed in a fixed order through distributed shared memory
 //          and written to v.  Deterministic, no atomics, no scratch memory.
@@ -26,7 +26,7 @@
 //          d_out (about four CTAs per SM in total).  B^T rank rows are staged by
 //          bulk copies before the kernel waits for the shrink; then v of the
 //          item is read, each thread accumulates its 8 output columns for up to
-//          8 tokens and updates y with one rounding, pass by pass.
+//          4 tokens and updates y with one rounding, pass by pass.
 #include <cuda_bf16.h>
 
 #include <map>
@@ -330,7 +330,7 @@ __device__ void shrink_item(const ShrinkArgs& a, const ItemInfo& m, uint32_t q, 
 }
 
 template <int MAXG, int NI>
-__global__ void __launch_bounds__(kThreads, MAXG == 8 ? 2 : 3)
+__global__ void __launch_bounds__(kThreads, 3)
     shrink_simt_kernel(const ShrinkArgs a, const __grid_constant__ InlineTable<NI> inl) {
     extern __shared__ __align__(128) uint8_t smem[];
     pdl_launch_dependents();  // the expand may start staging its B^T pages now
@@ -362,7 +362,6 @@ __global__ void __launch_bounds__(kThreads, MAXG == 8 ? 2 : 3)
     if (m.ok) {  // MAXG bounds the token group, and with it the registers of the launch
         if (MAXG == 1 || m.n == 1) shrink_item<1>(a, m, q, pp, sg, part, red);
         else if (MAXG == 2 || m.n == 2) shrink_item<(MAXG < 2 ? MAXG : 2)>(a, m, q, pp, sg, part, red);
-        else if (MAXG == 4 || m.n <= 4) shrink_item<(MAXG < 4 ? MAXG : 4)>(a, m, q, pp, sg, part, red);
         else shrink_item<MAXG>(a, m, q, pp, sg, part, red);
     }
     cp_async_wait<0>();
@@ -484,7 +483,7 @@ __device__ void expand_item(const ExpandArgs& a, const ItemInfo& m, Pipe<kExpand
 }
 
 template <int MAXG, int NI>
-__global__ void __launch_bounds__(kThreads, MAXG == 8 ? 2 : 3)
+__global__ void __launch_bounds__(kThreads, 3)
     expand_simt_kernel(const ExpandArgs a, const __grid_constant__ InlineTable<NI> inl) {
     extern __shared__ __align__(128) uint8_t smem_e[];
     const int part_idx = blockIdx.x % a.ctas_per_item, item_idx = blockIdx.x / a.ctas_per_item;
@@ -519,7 +518,6 @@ __global__ void __launch_bounds__(kThreads, MAXG == 8 ? 2 : 3)
     }
     if (MAXG == 1 || m.n == 1) expand_item<1>(a, m, pp, sg, vs);
     else if (MAXG == 2 || m.n == 2) expand_item<(MAXG < 2 ? MAXG : 2)>(a, m, pp, sg, vs);
-    else if (MAXG == 4 || m.n <= 4) expand_item<(MAXG < 4 ? MAXG : 4)>(a, m, pp, sg, vs);
     else expand_item<MAXG>(a, m, pp, sg, vs);
     cp_async_wait<0>();
 }
@@ -552,9 +550,9 @@ cudaError_t set_smem(K kern, size_t bytes) {
     return e;
 }
 
-template <typename K1, typename K2, typename K4, typename K8>
-auto pick(int max_item_rows, K1 k1, K2 k2, K4 k4, K8 k8) {
-    return max_item_rows <= 1 ? k1 : max_item_rows <= 2 ? k2 : max_item_rows <= 4 ? k4 : k8;
+template <typename K1, typename K2, typename K4>
+auto pick(int max_item_rows, K1 k1, K2 k2, K4 k4) {
+    return max_item_rows <= 1 ? k1 : max_item_rows <= 2 ? k2 : k4;
 }
 
 cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, const BatchView& b, int32_t num_items,
@@ -606,13 +604,12 @@ cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, con
     cfg.numAttrs = 1;
     if (inl) {
         auto kern = pick(max_item_rows, shrink_simt_kernel<1, kInlineItems>, shrink_simt_kernel<2, kInlineItems>,
-                         shrink_simt_kernel<4, kInlineItems>, shrink_simt_kernel<8, kInlineItems>);
+                         shrink_simt_kernel<4, kInlineItems>);
         cudaError_t e = set_smem(kern, smem);
         if (e != cudaSuccess) return e;
         return cudaLaunchKernelEx(&cfg, kern, a, *inl);
     }
-    auto kern = pick(max_item_rows, shrink_simt_kernel<1, 1>, shrink_simt_kernel<2, 1>, shrink_simt_kernel<4, 1>,
-                     shrink_simt_kernel<8, 1>);
+    auto kern = pick(max_item_rows, shrink_simt_kernel<1, 1>, shrink_simt_kernel<2, 1>, shrink_simt_kernel<4, 1>);
     cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
     return cudaLaunchKernelEx(&cfg, kern, a, InlineTable<1>{});
@@ -658,13 +655,12 @@ cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const
     cfg.numAttrs = 1;
     if (inl) {
         auto kern = pick(max_item_rows, expand_simt_kernel<1, kInlineItems>, expand_simt_kernel<2, kInlineItems>,
-                         expand_simt_kernel<4, kInlineItems>, expand_simt_kernel<8, kInlineItems>);
+                         expand_simt_kernel<4, kInlineItems>);
         cudaError_t e = set_smem(kern, smem);
         if (e != cudaSuccess) return e;
         return cudaLaunchKernelEx(&cfg, kern, a, *inl);
     }
-    auto kern = pick(max_item_rows, expand_simt_kernel<1, 1>, expand_simt_kernel<2, 1>, expand_simt_kernel<4, 1>,
-                     expand_simt_kernel<8, 1>);
+    auto kern = pick(max_item_rows, expand_simt_kernel<1, 1>, expand_simt_kernel<2, 1>, expand_simt_kernel<4, 1>);
     cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
     return cudaLaunchKernelEx(&cfg, kern, a, InlineTable<1>{});

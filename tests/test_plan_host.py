@@ -40,7 +40,7 @@ def _check_plan(plan, pool, ids, ranks, thr):
                 assert tuple(rec[p, :3]) == tuple(rec[0, :3])
     # dispatch covers every row of every non-empty, non-zero-rank segment exactly once
     covered = []
-    for items, lim, is_tc in ((plan.simt_items, 8, False), (plan.tc_tiles, 128, True)):
+    for items, lim, is_tc in ((plan.simt_items, 4, False), (plan.tc_tiles, 128, True)):
         for s, b, e in items.tolist():
             n = off[s + 1] - off[s]
             assert off[s] <= b < e <= off[s + 1] and e - b <= lim

@@ -142,9 +142,9 @@ def read_traffic(workload: str, kernel: str):
 
 
 # ---------------------------------------------------------------------------- our arm
-def setup(wl_name: str, rank: int, device: int):
+def setup(wl_name: str, rank: int, device: int, pool_override: int = 0):
     import segmented_rank_gemm_sgmv_b200 as sg
-    wl = workloads.make(wl_name, seed=rank)
+    wl = workloads.make(wl_name, seed=rank, **({"pool": pool_override} if pool_override else {}))
     bank = workloads.AdapterBank(wl, device=f"cuda:{device}")
     projs = [(d_in, d_out) for _, d_in, d_out in wl.projections]
     need = sum(sg.AdapterPool.pages_needed(projs, int(r)) for r in wl.pool_ranks)
@@ -161,7 +161,7 @@ def setup(wl_name: str, rank: int, device: int):
 
 
 def run_ours(args, rank, world, device):
-    sg, wl, pool, acts = setup(args.workload, rank, device)
+    sg, wl, pool, acts = setup(args.workload, rank, device, args.pool)
     n_proj = len(wl.projections)
     stream = torch.cuda.current_stream(device)
     plans = [sg.BatchPlan(pool, capacity_tokens=wl.T) for _ in range(2)]
@@ -242,6 +242,10 @@ def run_ours(args, rank, world, device):
                launches=2 * n_proj * len(kinds), clocks=clk.summary(), dom_launches=n_proj,
                traffic=read_traffic(args.workload, "lora_delta"), split=split)
     if split:
+        res["phase_us_per_proj"] = {
+            name: [round(1e3 * float(np.mean([e[1 + 3 * p].elapsed_time(e[2 + 3 * p]) for e in records])), 2),
+                   round(1e3 * float(np.mean([e[2 + 3 * p].elapsed_time(e[3 + 3 * p]) for e in records])), 2)]
+            for p, (name, _, _) in enumerate(wl.projections)}
         res["phase_ms"] = {"shrink": float(np.mean([sum(e[1 + 3 * p].elapsed_time(e[2 + 3 * p]) for p in range(n_proj))
                                                     for e in records])),
                            "expand": float(np.mean([sum(e[2 + 3 * p].elapsed_time(e[3 + 3 * p]) for p in range(n_proj))
@@ -383,6 +387,9 @@ def main():
     ap.add_argument("--workload", default="decode_q_proj", choices=workloads.WORKLOAD_NAMES)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pool", type=int, default=0,
+                    help="resident adapters of the pool (llama70b_layer only; for small profiler captures, "
+                         "the kernels see the same batch shape)")
     ap.add_argument("--split-phases", action="store_true",
                     help="record an event between shrink and expand (times each phase; removes their overlap)")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
@@ -432,6 +439,7 @@ def main():
         }
         if "phase_ms" in res:
             line["phase_ms"] = res["phase_ms"]
+            line["phase_us_per_proj"] = res["phase_us_per_proj"]
         if not args.no_cpu_baseline and world == 1:
             prepared = oracle_inputs(wl, f"cuda:{local}")
             rate, reps, el, used = time_oracle(prepared, wl, args.cpu_budget, os.cpu_count() or 1)

@@ -19,9 +19,10 @@
 //          segment); CTA q owns d_in columns [q kc, (q+1) kc).  Stages are 8
 //          rank rows x up to 1024 columns; each thread owns 8 columns and
 //          keeps the item's (up to 4) tokens' x in registers; partial dot products are
-//          reduced with warp shuffles and shared memory, then the C partial
-//          tiles are summed in a fixed order through distributed shared memory
-//          and written to v.  Deterministic, no atomics, no scratch memory.
+//          reduced with warp shuffles and shared memory; the other CTAs of the
+//          cluster push their partial tiles into rank 0's shared memory, which
+//          sums them in a fixed order and writes v.  Deterministic, no atomics,
+//          no scratch memory.
 // expand:  CTAs per work item each cover one or more 1024-column passes of
 //          d_out (about four CTAs per SM in total).  B^T rank rows are staged by
 //          bulk copies before the kernel waits for the shrink; then v of the
@@ -31,6 +32,7 @@
 
 #include <map>
 #include <mutex>
+#include <tuple>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -204,23 +206,21 @@ __device__ __forceinline__ float block_reduce(float (&vals)[N], float* red) {
 // Every stage is one commit group; the prologue commits kStages groups and
 // each consumed stage commits one more (possibly empty), so waiting for all but
 // the newest kStages - 1 groups always means "this stage has landed".
-struct StageGeom {  // stage u -> rows and columns
+struct StageGeom {  // rows and columns of the CTA's stages
     int NG, npass, span, col_base, rank, pages_per_row;
     int64_t pt;
     const int32_t* pid;  // page ids of the CTA's span, [rank row][chunk], in shared memory
     int span_pages;
-    __device__ void at(int u, bool pass_outer, int& g, int& c, int& W) const {
-        const int s = pass_outer ? u / NG : u % npass;
-        g = pass_outer ? u % NG : u / npass;
-        c = s * kPass;
-        W = min(kPass, span - c);
-    }
 };
 
+// The ring: stage `issued` goes to slot `islot`, its row group / pass advance
+// incrementally (row group outer for the shrink, pass outer for the expand).
 template <int kStages>
 struct Pipe {
     uint16_t* data;
-    int issued = 0, consumed = 0, total = 0;
+    int issued = 0, total = 0;
+    int islot = 0, cslot = 0;  // slots of the next issued / consumed stage
+    int ig = 0, is = 0;        // row group and pass of the next issued stage
 };
 
 template <int kStages>
@@ -228,22 +228,40 @@ __device__ __forceinline__ void pipe_issue(const PoolView& pool, Pipe<kStages>& 
                                            bool pass_outer) {
     if (pp.issued < pp.total) {
         const int P_log2 = pool.page_log2, P = 1 << P_log2;
-        int g, c, W;
-        sg.at(pp.issued, pass_outer, g, c, W);
+        const int g = pp.ig, c = pp.is * kPass;
+        const int W = min(kPass, sg.span - c);
         const int rows = min(kRowGroup, sg.rank - kRowGroup * g);
-        const int gpr = W >> 3;  // granules per row
-        uint16_t* dst0 = pp.data + (size_t)(pp.issued % kStages) * kStageElems;
+        uint16_t* dst0 = pp.data + (size_t)pp.islot * kStageElems;
+        const int32_t* pidg = sg.pid + kRowGroup * g * sg.span_pages;
+        if (W == kPass) {  // full pass: thread t copies granule t of each of the stage's rows
+            const int col = c + kVec * threadIdx.x;
+            const int32_t* pidc = pidg + (col >> P_log2);
+            const uint16_t* src0 = pool.pages + (col & (P - 1));
+            uint16_t* dst = dst0 + kVec * threadIdx.x;
 #pragma unroll
-        for (int i = 0; i < kStageElems / 8 / kThreads; ++i) {
-            const int gi = threadIdx.x + kThreads * i;
-            const int kk = gi / gpr, cg = gi - kk * gpr;
-            if (kk < rows) {
-                const int col = c + cg * 8;
-                const int32_t page = sg.pid[(kRowGroup * g + kk) * sg.span_pages + (col >> P_log2)];
-                cp_async16(dst0 + (size_t)kk * W + cg * 8,
-                           pool.pages + ((int64_t)page << P_log2) + (col & (P - 1)), true);
+            for (int kk = 0; kk < kRowGroup; ++kk)
+                if (kk < rows)
+                    cp_async16(dst + kk * kPass, src0 + ((int64_t)pidc[kk * sg.span_pages] << P_log2), true);
+        } else {
+            const int gpr = W >> 3;  // granules per row
+#pragma unroll
+            for (int i = 0; i < kStageElems / 8 / kThreads; ++i) {
+                const int gi = threadIdx.x + kThreads * i;
+                const int kk = gi / gpr, cg = gi - kk * gpr;
+                if (kk < rows) {
+                    const int col = c + cg * 8;
+                    const int32_t page = pidg[kk * sg.span_pages + (col >> P_log2)];
+                    cp_async16(dst0 + (size_t)kk * W + cg * 8,
+                               pool.pages + ((int64_t)page << P_log2) + (col & (P - 1)), true);
+                }
             }
         }
+        if (pass_outer) {
+            if (++pp.ig == sg.NG) { pp.ig = 0; ++pp.is; }
+        } else {
+            if (++pp.is == sg.npass) { pp.is = 0; ++pp.ig; }
+        }
+        pp.islot = pp.islot + 1 == kStages ? 0 : pp.islot + 1;
     }
     ++pp.issued;
     cp_async_commit();
@@ -253,14 +271,14 @@ template <int kStages>
 __device__ __forceinline__ const uint16_t* pipe_acquire(Pipe<kStages>& pp) {
     cp_async_wait<kStages - 1>();
     __syncthreads();
-    return pp.data + (size_t)(pp.consumed % kStages) * kStageElems;
+    return pp.data + (size_t)pp.cslot * kStageElems;
 }
 
 template <int kStages>
 __device__ __forceinline__ void pipe_release(const PoolView& pool, Pipe<kStages>& pp, const StageGeom& sg,
                                              bool pass_outer) {
     __syncthreads();  // every thread is done with the slot before it is refilled
-    ++pp.consumed;
+    pp.cslot = pp.cslot + 1 == kStages ? 0 : pp.cslot + 1;
     pipe_issue(pool, pp, sg, pass_outer);
 }
 
@@ -292,25 +310,32 @@ __device__ void shrink_item(const ShrinkArgs& a, const ItemInfo& m, uint32_t q, 
     const uint16_t* xrow[G];
 #pragma unroll
     for (int j = 0; j < G; ++j) xrow[j] = m.tok[j] >= 0 ? a.x + (int64_t)m.tok[j] * a.ldx + (int64_t)q * a.kc : nullptr;
+    // x of the unit after the current one is in flight while the current one is
+    // consumed (units: row group g outer, column pass s inner)
+    const int units = sg.NG * sg.npass;
+    uint4 xcur[G], xnext[G];
+    auto load_x = [&](int sp, uint4 (&dst)[G]) {  // x of pass sp
+        const int c = sp * kPass;
+        const bool active = col < min(kPass, sg.span - c);
+#pragma unroll
+        for (int j = 0; j < G; ++j)
+            dst[j] = (active && xrow[j]) ? __ldg(reinterpret_cast<const uint4*>(xrow[j] + c + col)) : make_uint4(0, 0, 0, 0);
+    };
+    load_x(0, xcur);
+    int u = 0;
     for (int g = 0; g < sg.NG; ++g) {
         float p[kRowGroup * G];
 #pragma unroll
         for (int i = 0; i < kRowGroup * G; ++i) p[i] = 0.f;
-        for (int s = 0; s < sg.npass; ++s) {
+        for (int s = 0; s < sg.npass; ++s, ++u) {
             const int c = s * kPass, W = min(kPass, sg.span - c);
             const bool active = col < W;
-            float xf[G][8];
-#pragma unroll
-            for (int j = 0; j < G; ++j) {
-                if (active && xrow[j]) {
-                    unpack8(__ldg(reinterpret_cast<const uint4*>(xrow[j] + c + col)), xf[j]);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) xf[j][e] = 0.f;
-                }
-            }
+            if (u + 1 < units) load_x(s + 1 == sg.npass ? 0 : s + 1, xnext);
             const uint16_t* st = pipe_acquire(pp);
             if (active) {
+                float xf[G][8];
+#pragma unroll
+                for (int j = 0; j < G; ++j) unpack8(xcur[j], xf[j]);
 #pragma unroll
                 for (int kk = 0; kk < kRowGroup; ++kk) {
                     float af[8];
@@ -320,6 +345,8 @@ __device__ void shrink_item(const ShrinkArgs& a, const ItemInfo& m, uint32_t q, 
                 }
             }
             pipe_release(a.pool, pp, sg, false);
+#pragma unroll
+            for (int j = 0; j < G; ++j) xcur[j] = xnext[j];
         }
         const float sum = block_reduce<kRowGroup * G>(p, red);
         if (tid < kRowGroup * G) {
@@ -335,10 +362,14 @@ __global__ void __launch_bounds__(kThreads, 3)
     extern __shared__ __align__(128) uint8_t smem[];
     pdl_launch_dependents();  // the expand may start staging its B^T pages now
     const int C = a.cluster;
+    // First cluster phase: every CTA has started.  Its wait, just before the
+    // partial tiles are pushed, makes rank 0's shared memory a valid target.
+    if (C > 1) cluster_arrive_relaxed();
     const int item_idx = blockIdx.x / C;
     const uint32_t q = cluster_ctarank();
-    float* part = reinterpret_cast<float*>(smem);
-    float* red = part + kSimtMaxItemRows * a.max_rank;  // [4 warps][64]
+    const int slot = kSimtMaxItemRows * a.max_rank;  // floats of one partial tile
+    float* part = reinterpret_cast<float*>(smem);     // [C slots][slot]; slot 0 is this CTA's own
+    float* red = part + C * slot;                      // [4 warps][64]
     int32_t* pid = reinterpret_cast<int32_t*>(red + 4 * 64);
 
     const ItemInfo m = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 0)
@@ -366,25 +397,34 @@ __global__ void __launch_bounds__(kThreads, 3)
     }
     cp_async_wait<0>();
 
-    // Sum the C partial tiles in a fixed order through distributed shared memory.
-    cluster_sync();
+    // Sum the C partial tiles in a fixed order.  Every CTA but rank 0 pushes its
+    // tile into slot q of rank 0's shared memory and arrives on the cluster
+    // barrier without waiting (it may then exit: nobody reads its memory); rank 0
+    // arrives, waits for all, sums slots 0..C-1 and writes v.  Slot 0 is rank 0's
+    // own tile, so the order of the sum is fixed.
+    const int E = m.n * m.r;
+    __syncthreads();  // part[] complete in this CTA
+    if (C > 1) {
+        cluster_wait_acquire();
+        if (q != 0) {
+            if (m.ok) {
+                const uint32_t dst = map_cluster(smem_u32(part + (size_t)q * slot), 0u);
+                for (int e = threadIdx.x; e < E; e += kThreads) st_cluster_f32(dst + 4u * (uint32_t)e, part[e]);
+            }
+            cluster_arrive_release();
+            return;
+        }
+        cluster_arrive_release();
+        cluster_wait_acquire();
+    }
     if (m.ok) {
-        const int E = m.n * m.r;
-        const int e0 = (int)(((int64_t)E * q) / C), e1 = (int)(((int64_t)E * (q + 1)) / C);
-        const uint32_t part_s = smem_u32(part);
-        for (int e = e0 + threadIdx.x; e < e1; e += kThreads) {
-            float pv[8];
-#pragma unroll
-            for (int qq = 0; qq < 8; ++qq)  // all loads in flight before the sum
-                pv[qq] = qq < C ? ld_cluster_f32(map_cluster(part_s + 4u * (uint32_t)e, (uint32_t)qq)) : 0.f;
+        for (int e = threadIdx.x; e < E; e += kThreads) {
             float s = 0.f;
-#pragma unroll
-            for (int qq = 0; qq < 8; ++qq) s += pv[qq];
+            for (int qq = 0; qq < C; ++qq) s += part[(size_t)qq * slot + e];
             const int jrow = e / m.r, k = e - jrow * m.r;
             a.v[(int64_t)(m.i0 + jrow) * a.ldv + k] = s;
         }
     }
-    cluster_sync();  // peers keep their shared memory until every read is done
 }
 
 // ------------------------------------------------------------------ expand
@@ -395,26 +435,27 @@ __device__ void expand_item(const ExpandArgs& a, const ItemInfo& m, Pipe<kExpand
     int trow[G];
 #pragma unroll
     for (int j = 0; j < G; ++j) trow[j] = m.tok[j];
-    uint4 yb[G];
-    float4 yf0[G], yf1[G];
-    auto load_y = [&](int c) {  // y of the pass starting at column c, kept for after the accumulation
-        const int jcol = sg.col_base + c + col;
+    // y of a pass is loaded one pass ahead of its update (two buffers)
+    // (bf16 y: the 16 bytes live in the first float4)
+    float4 y0[G], y1[G], n0[G], n1[G];
+    auto load_y = [&](int s, float4 (&d0)[G], float4 (&d1)[G]) {
+        const int c = s * kPass, jcol = sg.col_base + c + col;
         const bool active = col < min(kPass, sg.span - c);
 #pragma unroll
         for (int j = 0; j < G; ++j) {
             if (active && trow[j] >= 0) {
                 if (a.y_dtype == 0) {
-                    yb[j] = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.y) +
+                    d0[j] = *reinterpret_cast<const float4*>(static_cast<const uint16_t*>(a.y) +
                                                              (int64_t)trow[j] * a.ldy + jcol);
                 } else {
                     const float* yp = static_cast<const float*>(a.y) + (int64_t)trow[j] * a.ldy + jcol;
-                    yf0[j] = *reinterpret_cast<const float4*>(yp);
-                    yf1[j] = *reinterpret_cast<const float4*>(yp + 4);
+                    d0[j] = *reinterpret_cast<const float4*>(yp);
+                    d1[j] = *reinterpret_cast<const float4*>(yp + 4);
                 }
             }
         }
     };
-    if (a.y_early) load_y(0);
+    if (a.y_early) load_y(0, y0, y1);
     pdl_wait();  // v (and, unless y_early, y) are final once the preceding kernel has completed
     for (int e = tid; e < m.n * m.r; e += kThreads) {
         const int jrow = e / m.r, k = e - jrow * m.r;
@@ -425,7 +466,8 @@ __device__ void expand_item(const ExpandArgs& a, const ItemInfo& m, Pipe<kExpand
         const int c = s * kPass, W = min(kPass, sg.span - c);
         const bool active = col < W;
         const int jcol = sg.col_base + c + col;
-        if (s > 0 || !a.y_early) load_y(c);
+        if (s == 0 && !a.y_early) load_y(0, y0, y1);
+        if (s + 1 < sg.npass) load_y(s + 1, n0, n1);
         float acc[G][8];
 #pragma unroll
         for (int j = 0; j < G; ++j)
@@ -451,13 +493,14 @@ __device__ void expand_item(const ExpandArgs& a, const ItemInfo& m, Pipe<kExpand
             }
             pipe_release(a.pool, pp, sg, true);
         }
-        if (!active) continue;
 #pragma unroll
         for (int j = 0; j < G; ++j) {
-            if (trow[j] < 0) continue;
+            if (!active || trow[j] < 0) continue;
             if (a.y_dtype == 0) {
                 float yv[8];
-                unpack8(yb[j], yv);
+                const float4 q = y0[j];
+                unpack8(make_uint4(__float_as_uint(q.x), __float_as_uint(q.y), __float_as_uint(q.z),
+                                   __float_as_uint(q.w)), yv);
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -470,7 +513,7 @@ __device__ void expand_item(const ExpandArgs& a, const ItemInfo& m, Pipe<kExpand
                     make_uint4(w[0], w[1], w[2], w[3]);
             } else {
                 float* yp = static_cast<float*>(a.y) + (int64_t)trow[j] * a.ldy + jcol;
-                float4 o0 = yf0[j], o1 = yf1[j];
+                float4 o0 = y0[j], o1 = y1[j];
                 o0.x = fmaf(a.scale, acc[j][0], o0.x); o0.y = fmaf(a.scale, acc[j][1], o0.y);
                 o0.z = fmaf(a.scale, acc[j][2], o0.z); o0.w = fmaf(a.scale, acc[j][3], o0.w);
                 o1.x = fmaf(a.scale, acc[j][4], o1.x); o1.y = fmaf(a.scale, acc[j][5], o1.y);
@@ -478,6 +521,11 @@ __device__ void expand_item(const ExpandArgs& a, const ItemInfo& m, Pipe<kExpand
                 *reinterpret_cast<float4*>(yp) = o0;
                 *reinterpret_cast<float4*>(yp + 4) = o1;
             }
+        }
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+            y0[j] = n0[j];
+            y1[j] = n1[j];
         }
     }
 }
@@ -535,19 +583,45 @@ int num_sms() {
 }  // namespace
 
 // Raise a kernel's dynamic shared-memory limit when a launch needs more than
-// any earlier launch of that kernel did.
-template <typename K>
-cudaError_t set_smem(K kern, size_t bytes) {
+// any earlier launch of that kernel did (never lowers it).
+cudaError_t raise_smem(const void* kern, size_t bytes) {
     static std::mutex mu;
     static std::map<std::pair<int, const void*>, size_t> done;
     int dev = 0;
     cudaGetDevice(&dev);
     std::lock_guard<std::mutex> lock(mu);
-    size_t& cur = done[{dev, reinterpret_cast<const void*>(kern)}];
+    size_t& cur = done[{dev, kern}];
     if (bytes <= cur) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e == cudaSuccess) cur = bytes;
     return e;
+}
+template <typename K>
+cudaError_t set_smem(K kern, size_t bytes) {
+    return raise_smem(reinterpret_cast<const void*>(kern), bytes);
+}
+
+// CTAs of 128 threads with `smem` bytes of dynamic shared memory that one SM
+// holds at once (cached per device, kernel and size).
+int resident_ctas(const void* kern, size_t smem) {
+    static std::mutex mu;
+    static std::map<std::tuple<int, const void*, size_t>, int> done;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = done.find({dev, kern, smem});
+        if (it != done.end()) return it->second;
+    }
+    int n = 0;
+    if (raise_smem(kern, smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, smem) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        n = 1;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    done[{dev, kern, smem}] = n;
+    return n;
 }
 
 template <typename K1, typename K2, typename K4>
@@ -559,17 +633,31 @@ cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, con
                                int32_t max_item_rows, int32_t max_rank, const PoolView& pool, float* v, int64_t ldv,
                                const InlineTable<kInlineItems>* inl, cudaStream_t stream) {
     if (num_items <= 0) return cudaSuccess;
-    // Cluster size: enough CTAs for two per SM, chunks of >= 1024 columns, at most 8.
+    auto kern_inl = pick(max_item_rows, shrink_simt_kernel<1, kInlineItems>, shrink_simt_kernel<2, kInlineItems>,
+                         shrink_simt_kernel<4, kInlineItems>);
+    auto kern_tab = pick(max_item_rows, shrink_simt_kernel<1, 1>, shrink_simt_kernel<2, 1>, shrink_simt_kernel<4, 1>);
+    const int mr = std::max(8, max_rank);
+    const size_t pid_bytes_max = (size_t)mr * (d_in >> pool.page_log2) * 4;
+    auto smem_for = [&](int c) {
+        const size_t part_bytes = (size_t)c * kSimtMaxItemRows * mr * 4;
+        const size_t pidb = pid_bytes_max / c;
+        return (((part_bytes + 1024 + pidb + 127) & ~(size_t)127)) + (size_t)kShrinkStages * kStageElems * 2;
+    };
+    // Cluster size C: the largest split (chunks of >= 1024 columns, C <= 8,
+    // dividing the page count) whose grid still fits in one wave of resident
+    // CTAs, so that every CTA streams its share from the start and none waits
+    // for a second wave.  More CTAs per item shorten the per-item chain.
     const int pages = d_in >> pool.page_log2;
-    const int target = (2 * num_sms() + num_items - 1) / num_items;
     int C = 1;
-    for (int c = 1; c <= 8; ++c) {
+    for (int c = 8; c >= 1; --c) {
         if (pages % c || (c > 1 && d_in / c < kPass)) continue;
-        if (c >= target) {
+        const size_t sm = smem_for(c);
+        const void* kp = inl ? reinterpret_cast<const void*>(kern_inl) : reinterpret_cast<const void*>(kern_tab);
+        const int per_sm = resident_ctas(kp, sm);
+        if ((int64_t)num_items * c <= (int64_t)per_sm * num_sms()) {
             C = c;
             break;
         }
-        C = c;
     }
     ShrinkArgs a;
     a.x = x;
@@ -582,14 +670,9 @@ cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, con
     a.cluster = C;
     a.kc = d_in / C;
     a.max_rank = std::max(8, max_rank);
-    const int NG = (a.max_rank + kRowGroup - 1) / kRowGroup;
-    const int npass = (a.kc + kPass - 1) / kPass;
-    (void)NG;
-    (void)npass;
     a.stages = kShrinkStages;
-    const size_t pid_bytes = (size_t)a.max_rank * (a.kc >> pool.page_log2) * 4;
-    a.ring_offset = (int)(((size_t)kSimtMaxItemRows * a.max_rank * 4 + 1024 + pid_bytes + 127) & ~(size_t)127);
-    const size_t smem = (size_t)a.ring_offset + (size_t)kShrinkStages * kStageElems * 2;
+    const size_t smem = smem_for(C);
+    a.ring_offset = (int)(smem - (size_t)kShrinkStages * kStageElems * 2);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(C * num_items), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -603,16 +686,13 @@ cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, con
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (inl) {
-        auto kern = pick(max_item_rows, shrink_simt_kernel<1, kInlineItems>, shrink_simt_kernel<2, kInlineItems>,
-                         shrink_simt_kernel<4, kInlineItems>);
-        cudaError_t e = set_smem(kern, smem);
+        cudaError_t e = set_smem(kern_inl, smem);
         if (e != cudaSuccess) return e;
-        return cudaLaunchKernelEx(&cfg, kern, a, *inl);
+        return cudaLaunchKernelEx(&cfg, kern_inl, a, *inl);
     }
-    auto kern = pick(max_item_rows, shrink_simt_kernel<1, 1>, shrink_simt_kernel<2, 1>, shrink_simt_kernel<4, 1>);
-    cudaError_t e = set_smem(kern, smem);
+    cudaError_t e = set_smem(kern_tab, smem);
     if (e != cudaSuccess) return e;
-    return cudaLaunchKernelEx(&cfg, kern, a, InlineTable<1>{});
+    return cudaLaunchKernelEx(&cfg, kern_tab, a, InlineTable<1>{});
 }
 
 cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const BatchView& b, int32_t num_items,
@@ -631,18 +711,30 @@ cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const
     a.ldy = ldy;
     a.y_dtype = y_dtype;
     a.y_early = y_early ? 1 : 0;
-    // About four CTAs per SM: CTAs per item k, each covering npass 1024-column passes.
-    const int tiles = (d_out + kPass - 1) / kPass;
-    const int k = std::max(1, std::min(tiles, (4 * num_sms() + num_items / 2) / num_items));
-    a.npass = (tiles + k - 1) / k;
-    a.ctas_per_item = (tiles + a.npass - 1) / a.npass;
+    // CTAs per item k, each covering npass 1024-column passes: the largest k
+    // whose grid fits in one wave of resident CTAs.
+    auto kern_inl = pick(max_item_rows, expand_simt_kernel<1, kInlineItems>, expand_simt_kernel<2, kInlineItems>,
+                         expand_simt_kernel<4, kInlineItems>);
+    auto kern_tab = pick(max_item_rows, expand_simt_kernel<1, 1>, expand_simt_kernel<2, 1>, expand_simt_kernel<4, 1>);
+    const void* kp = inl ? reinterpret_cast<const void*>(kern_inl) : reinterpret_cast<const void*>(kern_tab);
     a.max_rank = std::max(8, max_rank);
-    const int NG = (a.max_rank + kRowGroup - 1) / kRowGroup;
-    (void)NG;
+    auto smem_for = [&](int npass) {
+        const size_t pid_bytes = (size_t)a.max_rank * ((npass * kPass) >> pool.page_log2) * 4;
+        return (((size_t)kSimtMaxItemRows * a.max_rank * 4 + pid_bytes + 127) & ~(size_t)127) +
+               (size_t)kExpandStages * kStageElems * 2;
+    };
+    const int tiles = (d_out + kPass - 1) / kPass;
+    a.npass = tiles;
+    for (int k = tiles; k >= 1; --k) {
+        const int np = (tiles + k - 1) / k, cpi = (tiles + np - 1) / np;
+        if (k > 1 && (int64_t)num_items * cpi > (int64_t)resident_ctas(kp, smem_for(np)) * num_sms()) continue;
+        a.npass = np;
+        break;
+    }
+    a.ctas_per_item = (tiles + a.npass - 1) / a.npass;
     a.stages = kExpandStages;
-    const size_t pid_bytes = (size_t)a.max_rank * ((a.npass * kPass) >> pool.page_log2) * 4;
-    a.ring_offset = (int)(((size_t)kSimtMaxItemRows * a.max_rank * 4 + pid_bytes + 127) & ~(size_t)127);
-    const size_t smem = (size_t)a.ring_offset + (size_t)kExpandStages * kStageElems * 2;
+    const size_t smem = smem_for(a.npass);
+    a.ring_offset = (int)(smem - (size_t)kExpandStages * kStageElems * 2);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.ctas_per_item * num_items), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -654,16 +746,13 @@ cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (inl) {
-        auto kern = pick(max_item_rows, expand_simt_kernel<1, kInlineItems>, expand_simt_kernel<2, kInlineItems>,
-                         expand_simt_kernel<4, kInlineItems>);
-        cudaError_t e = set_smem(kern, smem);
+        cudaError_t e = set_smem(kern_inl, smem);
         if (e != cudaSuccess) return e;
-        return cudaLaunchKernelEx(&cfg, kern, a, *inl);
+        return cudaLaunchKernelEx(&cfg, kern_inl, a, *inl);
     }
-    auto kern = pick(max_item_rows, expand_simt_kernel<1, 1>, expand_simt_kernel<2, 1>, expand_simt_kernel<4, 1>);
-    cudaError_t e = set_smem(kern, smem);
+    cudaError_t e = set_smem(kern_tab, smem);
     if (e != cudaSuccess) return e;
-    return cudaLaunchKernelEx(&cfg, kern, a, InlineTable<1>{});
+    return cudaLaunchKernelEx(&cfg, kern_tab, a, InlineTable<1>{});
 }
 
 cudaError_t read_clear_errors_simt(uint32_t* bits, cudaStream_t stream) {

@@ -82,6 +82,18 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
+// Arrive on `bar` once all cp.async copies this thread issued so far have
+// completed; the arrival counts against the count the barrier was created with.
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Barrier `id` (1..15) among `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -181,6 +193,26 @@ __device__ __forceinline__ uint64_t smem_desc_noswizzle(uint32_t saddr, uint32_t
     // base offset 0, lbo mode 0, layout type 0 (no swizzle)
     return d;
 }
+// Shared-memory matrix descriptor, 128-byte swizzle: atoms of 8 rows x 128
+// bytes whose 16-byte chunks are permuted by XOR with the row index (bits 4-6
+// of the address XOR bits 7-9), atoms 1024-byte aligned.  K-major operands:
+// lbo unused (1), sbo = stride of 8-row groups; MN-major operands: lbo = stride
+// of 64-element MN atoms, sbo = stride of 8-row K groups.  Layout type 2 in
+// bits 61-63, version 1 in bits 46-47.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
+}
+// Byte offset of 16-byte chunk `chunk` (0-7) of row `row` inside a 128B-swizzled atom.
+__host__ __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t chunk) {
+    return (row & 7u) * 128u + ((chunk ^ (row & 7u)) & 7u) * 16u;
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
     return (1u << 4)                           // D format: f32

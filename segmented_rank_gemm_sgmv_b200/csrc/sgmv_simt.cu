@@ -46,7 +46,11 @@ constexpr int kThreads = 128;
 constexpr int kVec = 8;                    // columns per thread
 constexpr int kPass = kThreads * kVec;     // 1024 columns per stage
 constexpr int kRowGroup = 8;               // rank rows per stage
-constexpr int kShrinkStages = 4;
+// shrink ring depth by token group: 1-token items stream long adapter rows with
+// 4 stages; items of 2-4 tokens carry larger x slices and keep 3 CTAs per SM
+// with 3 stages
+template <int MAXG>
+__host__ __device__ constexpr int shrink_stages() { return MAXG == 1 ? 4 : 3; }
 constexpr int kExpandStages = 3;
 constexpr int kStageElems = kRowGroup * kPass;
 
@@ -223,13 +227,31 @@ struct Pipe {
     int ig = 0, is = 0;        // row group and pass of the next issued stage
 };
 
+// x slices that travel with the shrink's stages: token row j's columns of the
+// stage's pass go to ring[slot][j] (maxg rows per slot), so their latency is
+// hidden by the same ring as the adapter rows.
+struct XStage {
+    uint16_t* ring;                              // null: no x slices (expand)
+    const uint16_t* rows[kSimtMaxItemRows];      // start of the CTA's chunk of each token row, or null
+    const uint16_t* any;                         // a valid address for zero-filled copies
+    int maxg;
+};
+
 template <int kStages>
 __device__ __forceinline__ void pipe_issue(const PoolView& pool, Pipe<kStages>& pp, const StageGeom& sg,
-                                           bool pass_outer) {
+                                           bool pass_outer, const XStage& xs) {
     if (pp.issued < pp.total) {
         const int P_log2 = pool.page_log2, P = 1 << P_log2;
         const int g = pp.ig, c = pp.is * kPass;
         const int W = min(kPass, sg.span - c);
+        if (xs.ring && kVec * (int)threadIdx.x < W) {
+            uint16_t* xd = xs.ring + (size_t)pp.islot * xs.maxg * kPass + kVec * threadIdx.x;
+#pragma unroll
+            for (int j = 0; j < kSimtMaxItemRows; ++j)
+                if (j < xs.maxg)
+                    cp_async16(xd + j * kPass, xs.rows[j] ? xs.rows[j] + c + kVec * threadIdx.x : xs.any,
+                               xs.rows[j] != nullptr);
+        }
         const int rows = min(kRowGroup, sg.rank - kRowGroup * g);
         uint16_t* dst0 = pp.data + (size_t)pp.islot * kStageElems;
         const int32_t* pidg = sg.pid + kRowGroup * g * sg.span_pages;
@@ -276,10 +298,10 @@ __device__ __forceinline__ const uint16_t* pipe_acquire(Pipe<kStages>& pp) {
 
 template <int kStages>
 __device__ __forceinline__ void pipe_release(const PoolView& pool, Pipe<kStages>& pp, const StageGeom& sg,
-                                             bool pass_outer) {
+                                             bool pass_outer, const XStage& xs) {
     __syncthreads();  // every thread is done with the slot before it is refilled
     pp.cslot = pp.cslot + 1 == kStages ? 0 : pp.cslot + 1;
-    pipe_issue(pool, pp, sg, pass_outer);
+    pipe_issue(pool, pp, sg, pass_outer, xs);
 }
 
 // All threads: fetch the page ids of every rank row over the CTA's column span
@@ -303,39 +325,23 @@ __device__ void load_page_ids(const PoolView& pool, StageGeom& sg, int32_t* pid,
 }
 
 // ------------------------------------------------------------------ shrink
-template <int G>
-__device__ void shrink_item(const ShrinkArgs& a, const ItemInfo& m, uint32_t q, Pipe<kShrinkStages>& pp,
-                            const StageGeom& sg, float* part, float* red) {
+template <int G, int kStages>
+__device__ void shrink_item(const ShrinkArgs& a, const ItemInfo& m, Pipe<kStages>& pp, const StageGeom& sg,
+                            const XStage& xs, float* part, float* red) {
     const int tid = threadIdx.x, col = kVec * tid;
-    const uint16_t* xrow[G];
-#pragma unroll
-    for (int j = 0; j < G; ++j) xrow[j] = m.tok[j] >= 0 ? a.x + (int64_t)m.tok[j] * a.ldx + (int64_t)q * a.kc : nullptr;
-    // x of the unit after the current one is in flight while the current one is
-    // consumed (units: row group g outer, column pass s inner)
-    const int units = sg.NG * sg.npass;
-    uint4 xcur[G], xnext[G];
-    auto load_x = [&](int sp, uint4 (&dst)[G]) {  // x of pass sp
-        const int c = sp * kPass;
-        const bool active = col < min(kPass, sg.span - c);
-#pragma unroll
-        for (int j = 0; j < G; ++j)
-            dst[j] = (active && xrow[j]) ? __ldg(reinterpret_cast<const uint4*>(xrow[j] + c + col)) : make_uint4(0, 0, 0, 0);
-    };
-    load_x(0, xcur);
-    int u = 0;
     for (int g = 0; g < sg.NG; ++g) {
         float p[kRowGroup * G];
 #pragma unroll
         for (int i = 0; i < kRowGroup * G; ++i) p[i] = 0.f;
-        for (int s = 0; s < sg.npass; ++s, ++u) {
+        for (int s = 0; s < sg.npass; ++s) {
             const int c = s * kPass, W = min(kPass, sg.span - c);
             const bool active = col < W;
-            if (u + 1 < units) load_x(s + 1 == sg.npass ? 0 : s + 1, xnext);
             const uint16_t* st = pipe_acquire(pp);
+            const uint16_t* xst = xs.ring + (size_t)pp.cslot * xs.maxg * kPass + col;
             if (active) {
                 float xf[G][8];
 #pragma unroll
-                for (int j = 0; j < G; ++j) unpack8(xcur[j], xf[j]);
+                for (int j = 0; j < G; ++j) unpack8(*reinterpret_cast<const uint4*>(xst + j * kPass), xf[j]);
 #pragma unroll
                 for (int kk = 0; kk < kRowGroup; ++kk) {
                     float af[8];
@@ -344,9 +350,7 @@ __device__ void shrink_item(const ShrinkArgs& a, const ItemInfo& m, uint32_t q, 
                     for (int j = 0; j < G; ++j) p[kk * G + j] += dot8(af, xf[j]);
                 }
             }
-            pipe_release(a.pool, pp, sg, false);
-#pragma unroll
-            for (int j = 0; j < G; ++j) xcur[j] = xnext[j];
+            pipe_release(a.pool, pp, sg, false, xs);
         }
         const float sum = block_reduce<kRowGroup * G>(p, red);
         if (tid < kRowGroup * G) {
@@ -383,17 +387,25 @@ __global__ void __launch_bounds__(kThreads, 3)
     sg.rank = m.r;
     sg.pages_per_row = a.d_in >> a.pool.page_log2;
     sg.pt = m.pt;
+    constexpr int kShrinkStages = shrink_stages<MAXG>();
     Pipe<kShrinkStages> pp;
     pp.data = reinterpret_cast<uint16_t*>(smem + a.ring_offset);
     pp.total = m.ok ? sg.NG * sg.npass : 0;
+    XStage xs;
+    xs.ring = pp.data + (size_t)kShrinkStages * kStageElems;
+    xs.maxg = MAXG;
+    xs.any = a.x;
+#pragma unroll
+    for (int j = 0; j < kSimtMaxItemRows; ++j)
+        xs.rows[j] = (j < MAXG && m.tok[j] >= 0) ? a.x + (int64_t)m.tok[j] * a.ldx + (int64_t)q * a.kc : nullptr;
     if (m.ok) load_page_ids(a.pool, sg, pid, &g_err_simt);
     __syncthreads();
 #pragma unroll 1
-    for (int i = 0; i < kShrinkStages; ++i) pipe_issue(a.pool, pp, sg, false);
+    for (int i = 0; i < kShrinkStages; ++i) pipe_issue(a.pool, pp, sg, false, xs);
     if (m.ok) {  // MAXG bounds the token group, and with it the registers of the launch
-        if (MAXG == 1 || m.n == 1) shrink_item<1>(a, m, q, pp, sg, part, red);
-        else if (MAXG == 2 || m.n == 2) shrink_item<(MAXG < 2 ? MAXG : 2)>(a, m, q, pp, sg, part, red);
-        else shrink_item<MAXG>(a, m, q, pp, sg, part, red);
+        if (MAXG == 1 || m.n == 1) shrink_item<1, kShrinkStages>(a, m, pp, sg, xs, part, red);
+        else if (MAXG == 2 || m.n == 2) shrink_item<(MAXG < 2 ? MAXG : 2), kShrinkStages>(a, m, pp, sg, xs, part, red);
+        else shrink_item<MAXG, kShrinkStages>(a, m, pp, sg, xs, part, red);
     }
     cp_async_wait<0>();
 
@@ -491,7 +503,7 @@ __device__ void expand_item(const ExpandArgs& a, const ItemInfo& m, Pipe<kExpand
                     }
                 }
             }
-            pipe_release(a.pool, pp, sg, true);
+            pipe_release(a.pool, pp, sg, true, XStage{});
         }
 #pragma unroll
         for (int j = 0; j < G; ++j) {
@@ -557,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 3)
     __syncthreads();
     // B^T pages do not depend on the shrink: start them before waiting for it
 #pragma unroll 1
-    for (int i = 0; i < kExpandStages; ++i) pipe_issue(a.pool, pp, sg, true);
+    for (int i = 0; i < kExpandStages; ++i) pipe_issue(a.pool, pp, sg, true, XStage{});
     if (!work) {
         pdl_wait();
         if (threadIdx.x == 0 && !m.ok) atomicOr(&g_err_simt, kErrRows);
@@ -638,10 +650,13 @@ cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, con
     auto kern_tab = pick(max_item_rows, shrink_simt_kernel<1, 1>, shrink_simt_kernel<2, 1>, shrink_simt_kernel<4, 1>);
     const int mr = std::max(8, max_rank);
     const size_t pid_bytes_max = (size_t)mr * (d_in >> pool.page_log2) * 4;
+    const int maxg = max_item_rows <= 1 ? 1 : max_item_rows <= 2 ? 2 : 4;
+    const int stages = maxg == 1 ? shrink_stages<1>() : shrink_stages<4>();
+    const size_t ring_bytes = (size_t)stages * (kStageElems + (size_t)maxg * kPass) * 2;  // A rows + x slices
     auto smem_for = [&](int c) {
         const size_t part_bytes = (size_t)c * kSimtMaxItemRows * mr * 4;
         const size_t pidb = pid_bytes_max / c;
-        return (((part_bytes + 1024 + pidb + 127) & ~(size_t)127)) + (size_t)kShrinkStages * kStageElems * 2;
+        return (((part_bytes + 1024 + pidb + 127) & ~(size_t)127)) + ring_bytes;
     };
     // Cluster size C: the largest split (chunks of >= 1024 columns, C <= 8,
     // dividing the page count) whose grid still fits in one wave of resident
@@ -670,9 +685,9 @@ cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, con
     a.cluster = C;
     a.kc = d_in / C;
     a.max_rank = std::max(8, max_rank);
-    a.stages = kShrinkStages;
+    a.stages = stages;
     const size_t smem = smem_for(C);
-    a.ring_offset = (int)(smem - (size_t)kShrinkStages * kStageElems * 2);
+    a.ring_offset = (int)(smem - ring_bytes);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(C * num_items), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);

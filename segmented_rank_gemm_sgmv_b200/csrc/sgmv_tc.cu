@@ -31,9 +31,9 @@ namespace {
 
 __device__ unsigned int g_err_tc;
 
-constexpr int kThreads = 128;
 constexpr int kKTile = 64;          // K columns per pipeline stage (shrink)
 constexpr int kShrinkStages = 4;
+constexpr int kShrinkThreads = 160;  // 4 producer / epilogue warps + 1 MMA warp
 
 struct ShrinkTcArgs {
     const uint16_t* x;
@@ -81,12 +81,19 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return p + ((1024u - (s & 1023u)) & 1023u);
 }
 
-__global__ void __launch_bounds__(kThreads) shrink_tc_kernel(const ShrinkTcArgs a) {
+// Warp roles: warps 0-3 (128 threads) fill the stage ring with cp.async and
+// then read the accumulator out; warp 4 owns the tensor memory and one of its
+// lanes issues the MMAs.  Stage s is "full" once all 128 producers' copies
+// into it have landed (cp.async.mbarrier.arrive.noinc, count 128) and "empty"
+// once the MMAs that read it have completed (tcgen05.commit).  Every wait is
+// bounded; a wait that gives up sets kErrTimeout and the CTA's abort flag, and
+// the remaining waits of the CTA are skipped.
+__global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkTcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
-    __shared__ uint64_t mma_bar[kShrinkStages];
+    __shared__ uint64_t full_bar[kShrinkStages], empty_bar[kShrinkStages], acc_bar;
     __shared__ uint32_t tmem_slot;
-    __shared__ int abort_flag;
+    __shared__ volatile int abort_flag;
     __shared__ int32_t tok_s[kTcTileRows];
 
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -112,24 +119,26 @@ __global__ void __launch_bounds__(kThreads) shrink_tc_kernel(const ShrinkTcArgs 
 
     if (tid == 0) {
         abort_flag = 0;
-        for (int i = 0; i < kShrinkStages; ++i) mbar_init(&mma_bar[i], 1);
+        for (int i = 0; i < kShrinkStages; ++i) {
+            mbar_init(&full_bar[i], kTcTileRows);
+            mbar_init(&empty_bar[i], 1);
+        }
+        mbar_init(&acc_bar, 1);
         fence_mbar_init();
     }
-    if (warp == 0) {
+    if (warp == 4) {
         tmem_alloc(&tmem_slot, (uint32_t)a.tmem_cols);
         tmem_relinquish();
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = tmem_slot;
 
     const int P_log2 = a.pool.page_log2;
     const int pages_per_row = a.d_in >> P_log2;
     const int k_begin = (int)q * a.kcols;
     const int nk = a.kcols / kKTile;
 
-    // token of each tile row (-1: none), read once
+    // token of each tile row (-1: none) and the page ids of the A rows over this
+    // CTA's K range ([rank row][page]; the range may start and end inside a page),
+    // each in one round of independent loads
     if (tid < kTcTileRows) {
         int t = -1;
         if (ok && tid < rows) {
@@ -141,102 +150,91 @@ __global__ void __launch_bounds__(kThreads) shrink_tc_kernel(const ShrinkTcArgs 
         }
         tok_s[tid] = t;
     }
-    __syncthreads();
-
-    // page ids of the A rows over this CTA's K range, [rank row][page], one round
-    // (the range may start and end inside a page)
     const int first_page = k_begin >> P_log2;
     const int span_pages = ((k_begin + a.kcols - 1) >> P_log2) - first_page + 1;
     int32_t* pid_s = reinterpret_cast<int32_t*>(smem + a.pid_offset);
-    for (int e = tid; e < r * span_pages; e += kThreads) {
+    for (int e = tid; e < r * span_pages; e += kShrinkThreads) {
         const int n = e / span_pages, pc = e - n * span_pages;
         pid_s[e] = safe_page(a.pool, a_base + (int64_t)n * pages_per_row + first_page + pc);
     }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;
 
-    // Granule g of a tile (16 bytes): row (g & 7) + 8 (g >> 6), K granule (g >> 3) & 7.
-    // A warp reads 8 rows x 64 contiguous bytes; each 8-lane phase writes one
-    // contiguous 128-byte line of a core-matrix column (no bank conflicts).
-    auto load_tile = [&](int kt, int slot) {
-        uint8_t* xs = stage0 + (size_t)slot * stage_bytes;
-        uint8_t* as = xs + x_tile_bytes;
-        const int c = k_begin + kt * kKTile;
+    if (warp < 4) {
+        // ---- producers.  Tiles are K-major with the 128-byte swizzle (8-row atoms of
+        // 128-byte rows, 1024-byte aligned).  Granule g (16 bytes): row g >> 3,
+        // chunk g & 7, so each 8-lane quarter of a warp copies one row's 128
+        // contiguous bytes into one (permuted) 128-byte row of shared memory.
+        for (int kt = 0; kt < nk; ++kt) {
+            const int st = kt % kShrinkStages;
+            if (kt >= kShrinkStages && !abort_flag &&
+                !mbar_wait(&empty_bar[st], (uint32_t)((kt / kShrinkStages - 1) & 1), &g_err_tc))
+                abort_flag = 1;
+            uint8_t* xs = stage0 + (size_t)st * stage_bytes;
+            uint8_t* as = xs + x_tile_bytes;
+            const int c = k_begin + kt * kKTile;
 #pragma unroll
-        for (int i = 0; i < (kTcTileRows * 8) / kThreads; ++i) {
-            const int g = tid + i * kThreads;
-            const int row = (g & 7) + 8 * (g >> 6), kg = (g >> 3) & 7;
-            const int t = tok_s[row];
-            const uint32_t off = (uint32_t)(row >> 3) * 1024 + kg * 128 + (row & 7) * 16;
-            const uint16_t* src = t >= 0 ? a.x + (int64_t)t * a.ldx + c + kg * 8 : a.x;
-            cp_async16(xs + off, src, t >= 0);
-        }
-        // A: rank rows n < npad, zero past r; the 64 columns lie in one page
-        const int page_rel = (c >> P_log2) - first_page, in_page = c & ((1 << P_log2) - 1);
-        for (int g = tid; g < npad * 8; g += kThreads) {
-            const int n = (g & 7) + 8 * (g >> 6), kg = (g >> 3) & 7;
-            const uint32_t off = (uint32_t)(n >> 3) * 1024 + kg * 128 + (n & 7) * 16;
-            const bool valid = ok && n < r;
-            const uint16_t* src = a.pool.pages;
-            if (valid) src = a.pool.pages + ((int64_t)pid_s[n * span_pages + page_rel] << P_log2) + in_page + kg * 8;
-            cp_async16(as + off, src, valid);
-        }
-    };
-
-    const uint32_t idesc = idesc_bf16_f32(128, npad, false, false);
-#pragma unroll 1
-    for (int s = 0; s < kShrinkStages - 1; ++s) {
-        if (s < nk) load_tile(s, s);
-        cp_async_commit();
-    }
-#pragma unroll 1
-    for (int kt = 0; kt < nk; ++kt) {
-        const int nxt = kt + kShrinkStages - 1;
-        if (nxt < nk) {
-            if (kt >= 1) {  // the slot of tile kt-1 is free once its MMAs completed
-                const int ps = (kt - 1) % kShrinkStages;
-                if (!mbar_wait(&mma_bar[ps], (uint32_t)(((kt - 1) / kShrinkStages) & 1), &g_err_tc))
-                    abort_flag = 1;
+            for (int i = 0; i < (kTcTileRows * 8) / kTcTileRows; ++i) {
+                const int g = tid + i * kTcTileRows;
+                const int row = g >> 3, kg = g & 7;
+                const int t = tok_s[row];
+                const uint32_t off = (uint32_t)(row >> 3) * 1024 + sw128_off((uint32_t)row, (uint32_t)kg);
+                const uint16_t* src = t >= 0 ? a.x + (int64_t)t * a.ldx + c + kg * 8 : a.x;
+                cp_async16(xs + off, src, t >= 0);
             }
-            load_tile(nxt, nxt % kShrinkStages);
+            // A: rank rows n < npad, zero past r; the 64 columns lie in one page
+            const int page_rel = (c >> P_log2) - first_page, in_page = c & ((1 << P_log2) - 1);
+            for (int g = tid; g < npad * 8; g += kTcTileRows) {
+                const int n = g >> 3, kg = g & 7;
+                const uint32_t off = (uint32_t)(n >> 3) * 1024 + sw128_off((uint32_t)n, (uint32_t)kg);
+                const bool valid = ok && n < r;
+                const uint16_t* src = a.pool.pages;
+                if (valid)
+                    src = a.pool.pages + ((int64_t)pid_s[n * span_pages + page_rel] << P_log2) + in_page + kg * 8;
+                cp_async16(as + off, src, valid);
+            }
+            cp_async_mbar_arrive_noinc(&full_bar[st]);
         }
-        cp_async_commit();
-        cp_async_wait<kShrinkStages - 1>();
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == 0) {
+    } else if (tid == 4 * 32) {
+        // ---- MMA issuer
+        const uint32_t idesc = idesc_bf16_f32(128, npad, false, false);
+        for (int kt = 0; kt < nk; ++kt) {
+            const int st = kt % kShrinkStages;
+            if (!abort_flag && !mbar_wait(&full_bar[st], (uint32_t)((kt / kShrinkStages) & 1), &g_err_tc))
+                abort_flag = 1;
+            fence_proxy_async_smem();  // the copies above were made through the generic proxy
             tc_fence_after();
-            const int slot = kt % kShrinkStages;
-            const uint32_t xs = smem_u32(stage0 + (size_t)slot * stage_bytes);
+            const uint32_t xs = smem_u32(stage0 + (size_t)st * stage_bytes);
             const uint32_t as = xs + (uint32_t)x_tile_bytes;
 #pragma unroll
-            for (int ks = 0; ks < kKTile / 16; ++ks) {
-                const uint64_t ad = smem_desc_noswizzle(xs + ks * 256, 128, 1024);
-                const uint64_t bd = smem_desc_noswizzle(as + ks * 256, 128, 1024);
+            for (int ks = 0; ks < kKTile / 16; ++ks) {  // K step of 16 = 32 bytes inside the swizzled rows
+                const uint64_t ad = smem_desc_sw128(xs + ks * 32, 16, 1024);
+                const uint64_t bd = smem_desc_sw128(as + ks * 32, 16, 1024);
                 tc_mma_bf16(tmem, ad, bd, idesc, kt > 0 || ks > 0);
             }
-            tc_commit(&mma_bar[slot]);
+            tc_commit(&empty_bar[st]);
         }
+        tc_commit(&acc_bar);  // every MMA of the tile has completed
     }
-    // accumulator complete once the last commit arrives
-    if (nk > 0) {
-        const int ls = (nk - 1) % kShrinkStages;
-        if (!mbar_wait(&mma_bar[ls], (uint32_t)(((nk - 1) / kShrinkStages) & 1), &g_err_tc)) abort_flag = 1;
-    }
-    tc_fence_after();
-    cp_async_wait<0>();
-    __syncthreads();
+    __syncwarp();  // warp 4 reconverges before the warp-collective instructions below
 
-    // tensor memory -> shared memory partial tile red[128][npad_max] (reuses the stages)
+    // ---- epilogue: tensor memory -> red[128][RS] (reuses the stages; RS odd: conflict-free)
     float* red = reinterpret_cast<float*>(smem);
-    const int RS = a.npad_max;
-    const int m = warp * 32 + (tid & 31);
-    for (int c0 = 0; c0 < npad; c0 += 32) {
-        uint32_t regs[32];
-        tmem_ld_32x32b_x32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, regs);
-        tmem_ld_wait();
+    const int RS = a.npad_max + 1;
+    if (warp < 4) {
+        if (!abort_flag && !mbar_wait(&acc_bar, 0u, &g_err_tc)) abort_flag = 1;
+        tc_fence_after();
+        const int m = warp * 32 + (tid & 31);
+        for (int c0 = 0; c0 < npad; c0 += 32) {
+            uint32_t regs[32];
+            tmem_ld_32x32b_x32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, regs);
+            tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-            if (c0 + e < RS) red[m * RS + c0 + e] = __uint_as_float(nk > 0 ? regs[e] : 0u);
+            for (int e = 0; e < 32; ++e)
+                if (c0 + e < a.npad_max) red[m * RS + c0 + e] = __uint_as_float(regs[e]);
+        }
     }
     tc_fence_before();
     cluster_sync();
@@ -245,21 +243,21 @@ __global__ void __launch_bounds__(kThreads) shrink_tc_kernel(const ShrinkTcArgs 
         const int KS = a.ks;
         const int m0 = (int)((kTcTileRows * q) / KS), m1 = (int)((kTcTileRows * (q + 1)) / KS);
         const uint32_t red_s = smem_u32(red);
-        for (int e = tid; e < (m1 - m0) * r; e += kThreads) {
+        for (int e = tid; e < (m1 - m0) * r; e += kShrinkThreads) {
             const int mm = m0 + e / r, k = e % r;
             if (mm >= rows) continue;
             float pv[8];
 #pragma unroll
             for (int qq = 0; qq < 8; ++qq)  // all loads in flight before the fixed-order sum
                 pv[qq] = qq < KS ? ld_cluster_f32(map_cluster(red_s + 4u * (uint32_t)(mm * RS + k), (uint32_t)qq)) : 0.f;
-            float s = 0.f;
+            float sum = 0.f;
 #pragma unroll
-            for (int qq = 0; qq < 8; ++qq) s += pv[qq];
-            a.v[(int64_t)(it.row_begin + mm) * a.ldv + k] = s;
+            for (int qq = 0; qq < 8; ++qq) sum += pv[qq];
+            a.v[(int64_t)(it.row_begin + mm) * a.ldv + k] = sum;
         }
     }
     cluster_sync();
-    if (warp == 0) {
+    if (warp == 4) {
         tc_fence_after();
         tmem_dealloc(tmem, (uint32_t)a.tmem_cols);
     }
@@ -268,24 +266,32 @@ __global__ void __launch_bounds__(kThreads) shrink_tc_kernel(const ShrinkTcArgs 
 // ------------------------------------------------------------------ expand
 // Persistent: CTA b takes a contiguous run of units (tile of <= 128 rows, block
 // of kYRowBytes of y columns), so consecutive units mostly share the tile and
-// its v rows.  The y rows and the B^T block of the next S-1 units are in flight
-// (cp.async) while the current unit is multiplied and written back:
-//   V_hi/V_lo [128 x kpad] (K-major)  <- v rows of the tile, split once per tile
-//   B^T block [kpad x NB]  (MN-major) <- page table
-//   Y block   [128 x NB]   (row stride kYStride: 16-byte accesses conflict-free)
-//   TMEM acc  [128 lanes x NB fp32]   <- V_hi B + V_lo B (tcgen05.mma, one thread)
-// The epilogue adds scale * acc to the Y block in shared memory (one row per
-// thread) and the block is stored with coalesced 16-byte stores.
+// its v rows.  Warp roles:
+//   warps 4-7 (producers): per unit, fetch the token rows and B^T page ids, then
+//     cp.async the y rows and the B^T block into stage slot s; when the tile
+//     changes, write V_hi / V_lo (v split into bf16 hi + lo, K-major)
+//   warp 8 (one lane): tcgen05.mma  acc[i & 1] = V_hi B + V_lo B  (N = block)
+//   warps 0-3 (epilogue): tcgen05.ld acc -> Y block += scale * acc in shared
+//     memory (row per thread) -> coalesced 16-byte stores of the block
+// mbarriers: full[s] (128 producer copies landed, cp.async.mbarrier.arrive),
+// yfree[s] (128 epilogue threads stored the block), accf[b] (MMAs done,
+// tcgen05.commit), acce[b] (128 epilogue threads read acc[b] out), vfull /
+// vempty (V of a tile written / its last MMA done).  The tensor-memory
+// accumulator is double-buffered, so the MMAs of unit i+1 overlap the epilogue
+// of unit i.  Every wait is bounded.
 constexpr int kYRowBytes = 256;             // y bytes of one tile row per unit (128 bf16 / 64 fp32)
 constexpr int kMaxPagesPerUnit = 2;         // pages of one B^T row a unit spans (page_elems >= 64)
 constexpr int kYStride = kYRowBytes + 16;   // padded shared-memory row stride
+constexpr int kExpandThreads = 288;         // 4 epilogue + 4 producer warps + 1 MMA warp
+constexpr int kMaxExpandStages = 3;
 
 template <int S>
-__global__ void __launch_bounds__(kThreads, 1) expand_tc_kernel(const ExpandTcArgs a) {
+__global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const ExpandTcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
-    __shared__ uint64_t mma_bar;
+    __shared__ uint64_t full_bar[S], yfree_bar[S], accf_bar[2], acce_bar[2], vfull_bar, vempty_bar;
     __shared__ uint32_t tmem_slot;
+    __shared__ volatile int abort_flag;
     __shared__ int32_t tok_s[S][kTcTileRows];
     __shared__ int32_t pid_s[S][kMaxRank * kMaxPagesPerUnit];  // B^T page ids of a unit [rank row][page]
 
@@ -295,20 +301,34 @@ __global__ void __launch_bounds__(kThreads, 1) expand_tc_kernel(const ExpandTcAr
     const int esz = a.y_dtype == 0 ? 2 : 4;
     const int NB = kYRowBytes / esz;              // output columns per unit
     const int kpm = a.kpad_max;
-    const uint32_t sbo = (uint32_t)(kpm / 8) * 128;  // 8-row (A) / 8-column (B) group stride
+    // V_hi / V_lo: K-major, 128-byte swizzle, blocks of 64 K columns (128 rows x 128 bytes each)
+    const int kpmv = (kpm + 63) & ~63;
     uint8_t* vhi = smem;
-    uint8_t* vlo = vhi + (size_t)kTcTileRows * kpm * 2;
-    uint8_t* bst = vlo + (size_t)kTcTileRows * kpm * 2;          // [S][kpm x NB]
+    uint8_t* vlo = vhi + (size_t)kTcTileRows * kpmv * 2;
+    // B^T block: MN-major, 128-byte swizzle: atoms of 8 K rows x 64 columns; atoms along N
+    // 1024 bytes apart (lbo), 8-row K groups sbo_b apart
+    const uint32_t sbo_b = (uint32_t)(NB / 64) * 1024;
+    uint8_t* bst = vlo + (size_t)kTcTileRows * kpmv * 2;          // [S][kpm x NB]
     const size_t b_bytes = (size_t)kpm * NB * 2;
     uint8_t* yst = bst + (size_t)S * b_bytes;                      // [S][128 x kYStride]
     const size_t y_bytes = (size_t)kTcTileRows * kYStride;
 
     if (tid == 0) {
-        mbar_init(&mma_bar, 1);
+        abort_flag = 0;
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&full_bar[i], kTcTileRows);
+            mbar_init(&yfree_bar[i], kTcTileRows);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&accf_bar[i], 1);
+            mbar_init(&acce_bar[i], kTcTileRows);
+        }
+        mbar_init(&vfull_bar, 1);
+        mbar_init(&vempty_bar, 1);
         fence_mbar_init();
     }
-    if (warp == 0) {
-        tmem_alloc(&tmem_slot, (uint32_t)NB);
+    if (warp == 8) {
+        tmem_alloc(&tmem_slot, (uint32_t)(2 * NB));
         tmem_relinquish();
     }
     tc_fence_before();
@@ -320,17 +340,18 @@ __global__ void __launch_bounds__(kThreads, 1) expand_tc_kernel(const ExpandTcAr
     const int pages_per_row = a.d_out >> P_log2;
     uint8_t* const ybase = static_cast<uint8_t*>(a.y);
 
-    // tile record of unit u; ok is uniform across the CTA
+    // unit u: its tile record; ok depends on the tile only, so it is the same for
+    // every unit of a tile and for every thread
     struct Unit {
-        int row_begin, rows, r, j0;
+        int tile, row_begin, rows, r, j0;
         int64_t b_base;
         bool ok;
     };
     auto unit = [&](int u) {
         Unit w;
-        const int tile = u / a.n_blocks;
-        w.j0 = (u - tile * a.n_blocks) * NB;
-        const ItemRec it = a.b.tc_tiles[(int64_t)tile * a.b.n_proj + a.b.proj];
+        w.tile = u / a.n_blocks;
+        w.j0 = (u - w.tile * a.n_blocks) * NB;
+        const ItemRec it = a.b.tc_tiles[(int64_t)w.tile * a.b.n_proj + a.b.proj];
         w.row_begin = it.row_begin;
         w.rows = it.row_end - it.row_begin;
         w.r = it.rank;
@@ -339,143 +360,149 @@ __global__ void __launch_bounds__(kThreads, 1) expand_tc_kernel(const ExpandTcAr
                  w.rows > kTcTileRows || it.row_end > a.b.num_rows || w.r <= 0 || ((w.r + 15) & ~15) > kpm);
         return w;
     };
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+        if (!abort_flag && !mbar_wait(bar, parity, &g_err_tc)) abort_flag = 1;
+    };
 
-    // Issue the copies of unit u into stage slot `slot` (one commit group).
-    // All threads call it.  First every index the copies need (token rows, B^T
-    // page ids) is fetched into shared memory in one round of independent loads,
-    // then the copies are issued from there.
-    auto issue = [&](int u, int slot) {
-        const Unit w = unit(u);
-        const int kpad = (w.r + 15) & ~15;
-        const int npc = NB > (1 << P_log2) ? (NB >> P_log2) : 1;  // pages a B^T row spans in one unit
-        if (w.ok) {
-            if (tid < kTcTileRows) {
+    if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ producers
+        const int pt = tid - 128;
+        int ts = -1, cur_tile = -1;
+        for (int u = u0; u < u1; ++u) {
+            const int i = u - u0, st = i % S;
+            const Unit w = unit(u);
+            if (i >= S) wait(&yfree_bar[st], (uint32_t)((i / S - 1) & 1));
+            if (w.ok && w.tile != cur_tile) {
+                if (ts >= 0) wait(&vempty_bar, (uint32_t)(ts & 1));  // the MMAs of the previous tile are done
+                const int m = pt, kpad = (w.r + 15) & ~15;
+                const bool row_ok = m < w.rows;
+                const float* vrow = a.v + (int64_t)(w.row_begin + (row_ok ? m : 0)) * a.ldv;
+                for (int kg = 0; kg < kpad / 8; ++kg) {
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int k = kg * 8 + e;
+                        f[e] = (row_ok && k < w.r) ? vrow[k] : 0.f;
+                    }
+                    uint32_t hw[4], lw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat16 h0 = __float2bfloat16_rn(f[2 * e]);
+                        const __nv_bfloat16 h1 = __float2bfloat16_rn(f[2 * e + 1]);
+                        const __nv_bfloat16 l0 = __float2bfloat16_rn(f[2 * e] - __bfloat162float(h0));
+                        const __nv_bfloat16 l1 = __float2bfloat16_rn(f[2 * e + 1] - __bfloat162float(h1));
+                        hw[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+                        lw[e] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+                    }
+                    const uint32_t off = (uint32_t)(kg >> 3) * (kTcTileRows * 128) + (uint32_t)(m >> 3) * 1024 +
+                                         sw128_off((uint32_t)m, (uint32_t)kg);
+                    *reinterpret_cast<uint4*>(vhi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4*>(vlo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
+                fence_proxy_async_smem();  // the tensor core reads V through the async proxy
+                named_bar_sync(1, 128);
+                if (pt == 0) mbar_arrive(&vfull_bar);
+                ++ts;
+                cur_tile = w.tile;
+            }
+            if (w.ok) {
+                // indices of the unit, one round of independent loads
+                const int npc = NB > (1 << P_log2) ? (NB >> P_log2) : 1;
                 int t = -1;
-                if (tid < w.rows) {
-                    t = a.b.token_idx[w.row_begin + tid];
+                if (pt < w.rows) {
+                    t = a.b.token_idx[w.row_begin + pt];
                     if (t < 0 || t >= a.b.T) {
                         atomicOr(&g_err_tc, kErrToken);
                         t = -1;
                     }
                 }
-                tok_s[slot][tid] = t;
-            }
-            for (int e = tid; e < w.r * npc; e += kThreads) {
-                const int k = e / npc, pc = e - k * npc;
-                pid_s[slot][e] = safe_page(a.pool, w.b_base + (int64_t)k * pages_per_row + (w.j0 >> P_log2) + pc);
-            }
-        } else if (tid == 0) {
-            atomicOr(&g_err_tc, kErrRows);
-        }
-        __syncthreads();
-        if (w.ok) {
-            uint8_t* ys = yst + (size_t)slot * y_bytes;
-            // y rows: 16 threads per row, 16 bytes each
+                tok_s[st][pt] = t;
+                for (int e = pt; e < w.r * npc; e += 128) {
+                    const int k = e / npc, pc = e - k * npc;
+                    pid_s[st][e] = safe_page(a.pool, w.b_base + (int64_t)k * pages_per_row + (w.j0 >> P_log2) + pc);
+                }
+                named_bar_sync(1, 128);
+                // y rows: 16 threads per row, 16 bytes each
+                uint8_t* ys = yst + (size_t)st * y_bytes;
 #pragma unroll 4
-            for (int i = 0; i < kTcTileRows * (kYRowBytes / 16) / kThreads; ++i) {
-                const int g = tid + i * kThreads;
-                const int m = g >> 4, q16 = g & 15;
-                const int t = tok_s[slot][m];
-                if (t >= 0)
-                    cp_async16(ys + m * kYStride + q16 * 16,
-                               ybase + ((int64_t)t * a.ldy + w.j0) * esz + q16 * 16, true);
-            }
-            // B^T block: granule (k, jg) = B^T[k][j0 + 8 jg .. +8], zero past r
-            uint8_t* bs = bst + (size_t)slot * b_bytes;
-            for (int g = tid; g < kpad * (NB / 8); g += kThreads) {
-                const int jg = g % (NB / 8), k = g / (NB / 8);
-                const int j = w.j0 + jg * 8;
-                const uint32_t off = (uint32_t)jg * sbo + (uint32_t)(k >> 3) * 128 + (uint32_t)(k & 7) * 16;
-                const bool valid = k < w.r;
-                const uint16_t* src = a.pool.pages;
-                if (valid) {
-                    const int32_t page = pid_s[slot][k * npc + ((j - w.j0) >> P_log2)];
-                    src = a.pool.pages + ((int64_t)page << P_log2) + (j & ((1 << P_log2) - 1));
+                for (int k16 = 0; k16 < kTcTileRows * (kYRowBytes / 16) / 128; ++k16) {
+                    const int g = pt + k16 * 128;
+                    const int m = g >> 4, q16 = g & 15;
+                    const int tm = tok_s[st][m];
+                    if (tm >= 0)
+                        cp_async16(ys + m * kYStride + q16 * 16, ybase + ((int64_t)tm * a.ldy + w.j0) * esz + q16 * 16,
+                                   true);
                 }
-                cp_async16(bs + off, src, valid);
+                // B^T block: granule (k, jg) = B^T[k][j0 + 8 jg .. +8], zero past r
+                uint8_t* bs = bst + (size_t)st * b_bytes;
+                const int kpad = (w.r + 15) & ~15;
+                for (int g = pt; g < kpad * (NB / 8); g += 128) {
+                    const int jg = g % (NB / 8), k = g / (NB / 8);
+                    const int j = w.j0 + jg * 8;
+                    const uint32_t off = (uint32_t)(k >> 3) * sbo_b + (uint32_t)(jg >> 3) * 1024 +
+                                         sw128_off((uint32_t)k, (uint32_t)jg);
+                    const bool valid = k < w.r;
+                    const uint16_t* src = a.pool.pages;
+                    if (valid)
+                        src = a.pool.pages + ((int64_t)pid_s[st][k * npc + ((j - w.j0) >> P_log2)] << P_log2) +
+                              (j & ((1 << P_log2) - 1));
+                    cp_async16(bs + off, src, valid);
+                }
+            } else if (pt == 0) {
+                atomicOr(&g_err_tc, kErrRows);
             }
+            cp_async_mbar_arrive_noinc(&full_bar[st]);
         }
-        cp_async_commit();
-    };
-
-#pragma unroll 1
-    for (int i = 0; i < S - 1; ++i) {
-        if (u0 + i < u1) issue(u0 + i, i);
-        else cp_async_commit();
-    }
-
-    int cur_tile = -1;
-    uint32_t phase = 0;
-    bool alive = true;
-#pragma unroll 1
-    for (int u = u0; u < u1; ++u) {
-        const int i = u - u0, slot = i % S;
-        __syncthreads();  // slot (i + S - 1) % S was fully read by the stores of unit i - 1
-        if (u + S - 1 < u1) issue(u + S - 1, (i + S - 1) % S);
-        else cp_async_commit();
-        const Unit w = unit(u);
-        const int tile = u / a.n_blocks;
-        if (w.ok && tile != cur_tile) {
-            // v rows of the tile -> bf16 hi + lo, row m = tid (the previous MMA has completed)
-            const int m = tid, kpad = (w.r + 15) & ~15;
-            const bool row_ok = m < w.rows;
-            const float* vrow = a.v + (int64_t)(w.row_begin + (row_ok ? m : 0)) * a.ldv;
-            for (int kg = 0; kg < kpad / 8; ++kg) {
-                float f[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int k = kg * 8 + e;
-                    f[e] = (row_ok && k < w.r) ? vrow[k] : 0.f;
-                }
-                uint32_t hw[4], lw[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const __nv_bfloat16 h0 = __float2bfloat16_rn(f[2 * e]);
-                    const __nv_bfloat16 h1 = __float2bfloat16_rn(f[2 * e + 1]);
-                    const __nv_bfloat16 l0 = __float2bfloat16_rn(f[2 * e] - __bfloat162float(h0));
-                    const __nv_bfloat16 l1 = __float2bfloat16_rn(f[2 * e + 1] - __bfloat162float(h1));
-                    hw[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-                    lw[e] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
-                }
-                const uint32_t off = (uint32_t)(m >> 3) * sbo + (uint32_t)kg * 128 + (uint32_t)(m & 7) * 16;
-                *reinterpret_cast<uint4*>(vhi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                *reinterpret_cast<uint4*>(vlo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-            }
-            cur_tile = tile;
-        }
-        if (S == 3) cp_async_wait<2>();
-        else cp_async_wait<1>();
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (!w.ok || !alive) continue;  // uniform
-
-        const int kpad = (w.r + 15) & ~15;
-        if (tid == 0) {
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        if ((tid & 31) == 0) {
             const uint32_t idesc = idesc_bf16_f32(128, NB, false, true);
             const uint32_t ah = smem_u32(vhi), al = smem_u32(vlo);
-            const uint32_t bb = smem_u32(bst + (size_t)slot * b_bytes);
-            for (int ks = 0; ks < kpad / 16; ++ks)
-                tc_mma_bf16(tmem, smem_desc_noswizzle(ah + ks * 256, 128, sbo),
-                            smem_desc_noswizzle(bb + ks * 256, 128, sbo), idesc, ks > 0);
-            for (int ks = 0; ks < kpad / 16; ++ks)
-                tc_mma_bf16(tmem, smem_desc_noswizzle(al + ks * 256, 128, sbo),
-                            smem_desc_noswizzle(bb + ks * 256, 128, sbo), idesc, true);
-            tc_commit(&mma_bar);
+            int ts = -1, cur_tile = -1;
+            for (int u = u0; u < u1; ++u) {
+                const int i = u - u0, st = i % S, bsel = i & 1;
+                const Unit w = unit(u);
+                if (w.ok && w.tile != cur_tile) {
+                    ++ts;
+                    cur_tile = w.tile;
+                    wait(&vfull_bar, (uint32_t)(ts & 1));
+                }
+                if (i >= 2) wait(&acce_bar[bsel], (uint32_t)((i / 2 - 1) & 1));
+                wait(&full_bar[st], (uint32_t)((i / S) & 1));
+                fence_proxy_async_smem();  // the copies were made through the generic proxy
+                tc_fence_after();
+                if (w.ok) {
+                    const int kpad = (w.r + 15) & ~15;
+                    const uint32_t acc = tmem + (uint32_t)(bsel * NB);
+                    const uint32_t bb = smem_u32(bst + (size_t)st * b_bytes);
+                    // K step ks: V at block ks / 4, 32 bytes per step inside its rows; B^T two K groups on
+                    for (int ks = 0; ks < kpad / 16; ++ks)
+                        tc_mma_bf16(acc, smem_desc_sw128(ah + (ks >> 2) * (kTcTileRows * 128) + (ks & 3) * 32, 16, 1024),
+                                    smem_desc_sw128(bb + ks * 2 * sbo_b, 1024, sbo_b), idesc, ks > 0);
+                    for (int ks = 0; ks < kpad / 16; ++ks)
+                        tc_mma_bf16(acc, smem_desc_sw128(al + (ks >> 2) * (kTcTileRows * 128) + (ks & 3) * 32, 16, 1024),
+                                    smem_desc_sw128(bb + ks * 2 * sbo_b, 1024, sbo_b), idesc, true);
+                }
+                tc_commit(&accf_bar[bsel]);
+                if (w.ok && (u + 1 == u1 || (u + 1) / a.n_blocks != w.tile))
+                    tc_commit(&vempty_bar);  // last MMA of the tile: V may be rewritten once it completes
+            }
         }
-        const bool done = mbar_wait(&mma_bar, phase, &g_err_tc);
-        phase ^= 1u;
-        tc_fence_after();
-
-        // epilogue: row m = tid of the Y block += scale * acc, 32 columns per tcgen05.ld
-        {
-            const int m = tid;
-            uint8_t* yrow = yst + (size_t)slot * y_bytes + (size_t)m * kYStride;
-            const bool row_ok = m < w.rows && done;
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int m = tid;
+        for (int u = u0; u < u1; ++u) {
+            const int i = u - u0, st = i % S, bsel = i & 1;
+            const Unit w = unit(u);
+            wait(&accf_bar[bsel], (uint32_t)((i / 2) & 1));
+            wait(&full_bar[st], (uint32_t)((i / S) & 1));  // (completed: makes the staged y visible here)
+            tc_fence_after();
+            uint8_t* yrow = yst + (size_t)st * y_bytes + (size_t)m * kYStride;
+            const bool row_ok = w.ok && m < w.rows && !abort_flag;
             for (int c0 = 0; c0 < NB; c0 += 32) {
                 uint32_t regs[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, regs);
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(bsel * NB + c0), regs);
                 tmem_ld_wait();
                 if (!row_ok) continue;
                 if (a.y_dtype == 0) {
@@ -507,28 +534,29 @@ __global__ void __launch_bounds__(kThreads, 1) expand_tc_kernel(const ExpandTcAr
                     }
                 }
             }
-        }
-        tc_fence_before();
-        alive = __syncthreads_and(done) != 0;  // uniform: a wait that gave up stops the CTA's work
-        if (!alive) continue;
-        // coalesced store of the Y block: 16 threads per row
-        {
-            const uint8_t* ys = yst + (size_t)slot * y_bytes;
-            for (int g = tid; g < kTcTileRows * (kYRowBytes / 16); g += kThreads) {
-                const int m = g >> 4, q16 = g & 15;
-                const int t = tok_s[slot][m];
-                if (m < w.rows && t >= 0)
-                    *reinterpret_cast<uint4*>(ybase + ((int64_t)t * a.ldy + w.j0) * esz + q16 * 16) =
-                        *reinterpret_cast<const uint4*>(ys + m * kYStride + q16 * 16);
+            tc_fence_before();
+            mbar_arrive(&acce_bar[bsel]);  // acc[bsel] has been read out
+            named_bar_sync(2, 128);        // the Y block is complete
+            if (w.ok && !abort_flag) {
+                const uint8_t* ys = yst + (size_t)st * y_bytes;
+#pragma unroll 4
+                for (int k16 = 0; k16 < kTcTileRows * (kYRowBytes / 16) / 128; ++k16) {
+                    const int g = m + k16 * 128;
+                    const int mm = g >> 4, q16 = g & 15;
+                    const int t = tok_s[st][mm];
+                    if (mm < w.rows && t >= 0)
+                        *reinterpret_cast<uint4*>(ybase + ((int64_t)t * a.ldy + w.j0) * esz + q16 * 16) =
+                            *reinterpret_cast<const uint4*>(ys + mm * kYStride + q16 * 16);
+                }
             }
+            mbar_arrive(&yfree_bar[st]);  // slot st may be refilled
         }
     }
-    cp_async_wait<0>();
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 8) {
         tc_fence_after();
-        tmem_dealloc(tmem, (uint32_t)NB);
+        tmem_dealloc(tmem, (uint32_t)(2 * NB));
     }
 }
 
@@ -564,7 +592,7 @@ cudaError_t launch_shrink_tc(const uint16_t* x, int64_t ldx, int32_t d_in, const
     a.ks = ks;
     a.kcols = d_in / ks;
     const size_t stage_bytes = (size_t)kTcTileRows * kKTile * 2 + (size_t)a.npad_max * kKTile * 2;
-    const size_t main_bytes = std::max(stage_bytes * kShrinkStages, (size_t)kTcTileRows * a.npad_max * 4);
+    const size_t main_bytes = std::max(stage_bytes * kShrinkStages, (size_t)kTcTileRows * (a.npad_max + 1) * 4);
     const size_t span_pages = ((size_t)a.kcols >> pool.page_log2) + 2;  // pages one K range can touch
     a.pid_offset = (int)main_bytes;
     const size_t pid_bytes = ((size_t)a.npad_max * span_pages * 4 + 15) & ~(size_t)15;
@@ -575,7 +603,7 @@ cudaError_t launch_shrink_tc(const uint16_t* x, int64_t ldx, int32_t d_in, const
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(ks * num_tiles), 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(kShrinkThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -608,12 +636,13 @@ cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const B
     a.n_blocks = d_out / NB;
     a.num_units = a.n_blocks * num_tiles;
     // shared memory: V hi + lo, S stages of (B^T block, Y block); three stages when they fit
-    const size_t v_bytes = (size_t)2 * kTcTileRows * a.kpad_max * 2;
+    const size_t v_bytes = (size_t)2 * kTcTileRows * ((a.kpad_max + 63) & ~63) * 2;
     const size_t stage = (size_t)a.kpad_max * NB * 2 + (size_t)kTcTileRows * kYStride;
-    // the opt-in limit covers dynamic (+1 KB alignment) and static (index tables) shared memory
-    const size_t limit = (227u << 10) - 1024 - 3 * kTcTileRows * 4 - 3 * kMaxRank * kMaxPagesPerUnit * 4;
+    // the opt-in limit covers dynamic (+1 KB alignment) and static (index tables, barriers) shared memory
+    const size_t limit = (227u << 10) - 1024 - 1024 - (size_t)kMaxExpandStages * kTcTileRows * 4 -
+                         (size_t)kMaxExpandStages * kMaxRank * kMaxPagesPerUnit * 4;
     const int S = (v_bytes + 3 * stage <= limit) ? 3 : 2;
-    // at least 116 KB: one CTA per SM, so tensor memory (NB <= 128 columns) is never oversubscribed
+    // at least 116 KB: one CTA per SM, so tensor memory (2 x NB <= 256 columns) is never oversubscribed
     const size_t smem = std::max(v_bytes + S * stage, (size_t)116 << 10) + 1024;
     // one CTA per SM, each a contiguous run of units
     static int sms = 0;
@@ -629,11 +658,11 @@ cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const B
     if (S == 3) {
         cudaError_t e = cudaFuncSetAttribute(expand_tc_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        expand_tc_kernel<3><<<(unsigned)blocks, kThreads, smem, stream>>>(a);
+        expand_tc_kernel<3><<<(unsigned)blocks, kExpandThreads, smem, stream>>>(a);
     } else {
         cudaError_t e = cudaFuncSetAttribute(expand_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        expand_tc_kernel<2><<<(unsigned)blocks, kThreads, smem, stream>>>(a);
+        expand_tc_kernel<2><<<(unsigned)blocks, kExpandThreads, smem, stream>>>(a);
     }
     return cudaGetLastError();
 }

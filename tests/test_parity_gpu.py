@@ -3,10 +3,11 @@ same seeded inputs, element by element.  Gates and tolerances: tests/sgmv_cases.
 
 The five workloads are the pages' shapes (see workloads/): tiny, decode q_proj,
 mixed ranks (MLP up), long prefill segments, and a full Llama-3-70B layer; the
-rest are edge cases of the method: ragged segment lengths around the 64-row
-SIMT items and 128-row tensor-core tiles, ranks that are not multiples of 8 or
-16, the largest rank, tokens without an adapter, empty batches, and the pins
-that fix the arithmetic exactly (integer inputs, zero B, zero scale).
+rest are edge cases of the method: ragged segment lengths around the 4-row
+SIMT items, the 16-row dispatch threshold and the 128-row tensor-core tiles,
+ranks that are not multiples of 8 or 16, the largest rank, tokens without an
+adapter, empty batches, page sizes other than 512 elements, and the pins that
+fix the arithmetic exactly (integer inputs, zero B, zero scale).
 """
 from __future__ import annotations
 
@@ -284,3 +285,20 @@ def test_lora_delta_requires_workspace():
                              plan.table_ptr(), pool.handle, 1.0, y.data_ptr(), y.stride(0), 0, None, 0,
                              None)
     assert st == 1
+
+
+@pytest.mark.parametrize("page_elems,d_in,d_out", [(64, 1536, 2560), (256, 1536, 2560), (1024, 2048, 3072)],
+                         ids=["P64", "P256", "P1024"])
+@pytest.mark.parametrize("path", [SIMT, TC], ids=["simt", "tc"])
+@pytest.mark.parametrize("y_dtype", [torch.bfloat16, torch.float32], ids=["ybf16", "yfp32"])
+def test_page_sizes(page_elems, d_in, d_out, path, y_dtype):
+    """Other page sizes: a B^T block or an A chunk spans several small pages, or a
+    CTA's column range starts inside a large one."""
+    wl, bank, x, y = custom_case([1, 3, 5, 17, 130, 40], [8, 16, 24, 64, 128, 32], d_in, d_out, seed=21,
+                                 minus_one=4)
+    pool = build_pool(wl, bank, page_elems=page_elems)
+    plan, v, y_out = run_gpu(pool, wl, 0, x, y, path, y_dtype, mode="lora_delta")
+    ref = run_oracle(wl, bank, 0, x, y)
+    errs = compare(plan, v, y_out, y, ref)
+    assert errs["v"] <= GATE_REL and errs["y"] <= GATE_REL, errs
+    assert sg.check_errors() == 0

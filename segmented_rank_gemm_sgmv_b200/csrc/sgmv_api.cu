@@ -96,6 +96,9 @@ sgmv_status shrink_impl(const void* x, int64_t ldx, int32_t T, int32_t d_in, int
 sgmv_status expand_impl(const float* v, int64_t ldv, int32_t T, int32_t d_out, int32_t proj, const sgmv_plan* plan,
                         const void* table, const sgmv_pool* pool, float scale, void* y, int64_t ldy, int32_t y_dtype,
                         bool y_early, cudaStream_t stream);
+sgmv_status delta_impl(const void* x, int64_t ldx, int32_t T, int32_t d_in, int32_t d_out, int32_t proj,
+                       const sgmv_plan* plan, const void* table, const sgmv_pool* pool, float scale, void* y,
+                       int64_t ldy, int32_t y_dtype, float* v, int64_t ldv, cudaStream_t stream);
 
 }  // namespace sgmv
 
@@ -131,21 +134,58 @@ extern "C" sgmv_status sgmv_expand(const float* v, int64_t ldv, int32_t T, int32
                        reinterpret_cast<cudaStream_t>(stream));
 }
 
-sgmv_status sgmv::shrink_impl(const void* x, int64_t ldx, int32_t T, int32_t d_in, int32_t proj,
-                              const sgmv_plan* plan, const void* table, const sgmv_pool* pool, float* v,
-                              int64_t ldv, cudaStream_t stream) {
-    BatchView bv;
-    PoolView pv;
-    sgmv_status st = make_views(plan, table, pool, T, proj, &bv, &pv, "shrink");
+namespace {
+
+// Argument checks of the shrink phase; fills the views.  Returns SGMV_OK with
+// *nothing = true when the batch has no work.
+sgmv_status check_shrink(const void* x, int64_t ldx, int32_t T, int32_t d_in, int32_t proj, const sgmv_plan* plan,
+                         const void* table, const sgmv_pool* pool, const float* v, int64_t ldv, BatchView* bv,
+                         PoolView* pv, bool* nothing) {
+    sgmv_status st = make_views(plan, table, pool, T, proj, bv, pv, "shrink");
     if (st != SGMV_OK) return st;
     if (d_in != pool->d_in[proj]) return fail(SGMV_ERR_INVALID, "shrink: d_in differs from the pool's projection");
-    if (plan->num_rows == 0 || (plan->num_simt_items == 0 && plan->num_tc_tiles == 0)) return SGMV_OK;
+    *nothing = plan->num_rows == 0 || (plan->num_simt_items == 0 && plan->num_tc_tiles == 0);
+    if (*nothing) return SGMV_OK;
     if (!x || !v) return fail(SGMV_ERR_INVALID, "shrink: x and v are required");
     if (ldx < d_in || (ldx % 8) || !aligned16(x)) return fail(SGMV_ERR_INVALID, "shrink: x rows must be 16-byte aligned, ldx >= d_in");
     if (ldv < plan->max_rank || ldv < 1 || (ldv % 4) || !aligned16(v))
         return fail(SGMV_ERR_INVALID, "shrink: v needs ldv >= max_rank, ldv % 4 == 0, 16-byte alignment");
     if (plan->num_simt_items > 0 && pool->page_elems > 1024)
         return fail(SGMV_ERR_UNSUPPORTED, "shrink: the SIMT path takes page_elems <= 1024");
+    return SGMV_OK;
+}
+
+// Argument checks of the expand phase; fills the views.
+sgmv_status check_expand(const float* v, int64_t ldv, int32_t T, int32_t d_out, int32_t proj, const sgmv_plan* plan,
+                         const void* table, const sgmv_pool* pool, const void* y, int64_t ldy, int32_t y_dtype,
+                         BatchView* bv, PoolView* pv, bool* nothing) {
+    sgmv_status st = make_views(plan, table, pool, T, proj, bv, pv, "expand");
+    if (st != SGMV_OK) return st;
+    if (d_out != pool->d_out[proj]) return fail(SGMV_ERR_INVALID, "expand: d_out differs from the pool's projection");
+    if (y_dtype != 0 && y_dtype != 1) return fail(SGMV_ERR_INVALID, "expand: y_dtype must be 0 (bf16) or 1 (fp32)");
+    *nothing = plan->num_rows == 0 || (plan->num_simt_items == 0 && plan->num_tc_tiles == 0);
+    if (*nothing) return SGMV_OK;
+    if (!v || !y) return fail(SGMV_ERR_INVALID, "expand: v and y are required");
+    const int64_t esz = y_dtype == 0 ? 2 : 4;
+    if (ldy < d_out || ((ldy * esz) % 16) || !aligned16(y))
+        return fail(SGMV_ERR_INVALID, "expand: y rows must be 16-byte aligned, ldy >= d_out");
+    if (ldv < plan->max_rank || ldv < 1 || (ldv % 4) || !aligned16(v))
+        return fail(SGMV_ERR_INVALID, "expand: v needs ldv >= max_rank, ldv % 4 == 0, 16-byte alignment");
+    if (plan->num_simt_items > 0 && pool->page_elems > 1024)
+        return fail(SGMV_ERR_UNSUPPORTED, "expand: the SIMT path takes page_elems <= 1024");
+    return SGMV_OK;
+}
+
+}  // namespace
+
+sgmv_status sgmv::shrink_impl(const void* x, int64_t ldx, int32_t T, int32_t d_in, int32_t proj,
+                              const sgmv_plan* plan, const void* table, const sgmv_pool* pool, float* v,
+                              int64_t ldv, cudaStream_t stream) {
+    BatchView bv;
+    PoolView pv;
+    bool nothing = false;
+    sgmv_status st = check_shrink(x, ldx, T, d_in, proj, plan, table, pool, v, ldv, &bv, &pv, &nothing);
+    if (st != SGMV_OK || nothing) return st;
     const uint16_t* xb = static_cast<const uint16_t*>(x);
     InlineTable<kInlineItems> inl;
     const bool use_inl = inline_items(plan, proj, &inl);
@@ -160,23 +200,41 @@ sgmv_status sgmv::expand_impl(const float* v, int64_t ldv, int32_t T, int32_t d_
                               int64_t ldy, int32_t y_dtype, bool y_early, cudaStream_t stream) {
     BatchView bv;
     PoolView pv;
-    sgmv_status st = make_views(plan, table, pool, T, proj, &bv, &pv, "expand");
-    if (st != SGMV_OK) return st;
-    if (d_out != pool->d_out[proj]) return fail(SGMV_ERR_INVALID, "expand: d_out differs from the pool's projection");
-    if (y_dtype != 0 && y_dtype != 1) return fail(SGMV_ERR_INVALID, "expand: y_dtype must be 0 (bf16) or 1 (fp32)");
-    if (plan->num_rows == 0 || (plan->num_simt_items == 0 && plan->num_tc_tiles == 0)) return SGMV_OK;
-    if (!v || !y) return fail(SGMV_ERR_INVALID, "expand: v and y are required");
-    const int64_t esz = y_dtype == 0 ? 2 : 4;
-    if (ldy < d_out || ((ldy * esz) % 16) || !aligned16(y))
-        return fail(SGMV_ERR_INVALID, "expand: y rows must be 16-byte aligned, ldy >= d_out");
-    if (ldv < plan->max_rank || ldv < 1 || (ldv % 4) || !aligned16(v))
-        return fail(SGMV_ERR_INVALID, "expand: v needs ldv >= max_rank, ldv % 4 == 0, 16-byte alignment");
-    if (plan->num_simt_items > 0 && pool->page_elems > 1024)
-        return fail(SGMV_ERR_UNSUPPORTED, "expand: the SIMT path takes page_elems <= 1024");
+    bool nothing = false;
+    sgmv_status st = check_expand(v, ldv, T, d_out, proj, plan, table, pool, y, ldy, y_dtype, &bv, &pv, &nothing);
+    if (st != SGMV_OK || nothing) return st;
     InlineTable<kInlineItems> inl;
     const bool use_inl = inline_items(plan, proj, &inl);
     SGMV_CUDA_TRY(launch_expand_simt(v, ldv, d_out, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, pv,
                                      scale, y, ldy, y_dtype, use_inl ? &inl : nullptr, y_early, stream));
+    SGMV_CUDA_TRY(launch_expand_tc(v, ldv, d_out, bv, plan->num_tc_tiles, plan->max_rank, pv, scale, y, ldy, y_dtype,
+                                   stream));
+    return SGMV_OK;
+}
+
+// Both phases in one call, arguments checked before anything is launched: the
+// SIMT shrink, the tensor-core shrink, then the SIMT expand as a programmatic
+// dependent launch (its adapter pages and y rows stream in while the shrinks
+// run) and the tensor-core expand.
+sgmv_status sgmv::delta_impl(const void* x, int64_t ldx, int32_t T, int32_t d_in, int32_t d_out, int32_t proj,
+                             const sgmv_plan* plan, const void* table, const sgmv_pool* pool, float scale, void* y,
+                             int64_t ldy, int32_t y_dtype, float* v, int64_t ldv, cudaStream_t stream) {
+    BatchView bv;
+    PoolView pv;
+    bool nothing = false;
+    sgmv_status st = check_shrink(x, ldx, T, d_in, proj, plan, table, pool, v, ldv, &bv, &pv, &nothing);
+    if (st != SGMV_OK || nothing) return st;
+    st = check_expand(v, ldv, T, d_out, proj, plan, table, pool, y, ldy, y_dtype, &bv, &pv, &nothing);
+    if (st != SGMV_OK || nothing) return st;
+    const uint16_t* xb = static_cast<const uint16_t*>(x);
+    InlineTable<kInlineItems> inl;
+    const bool use_inl = inline_items(plan, proj, &inl);
+    SGMV_CUDA_TRY(launch_shrink_simt(xb, ldx, d_in, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, pv,
+                                     v, ldv, use_inl ? &inl : nullptr, stream));
+    SGMV_CUDA_TRY(launch_shrink_tc(xb, ldx, d_in, bv, plan->num_tc_tiles, plan->max_rank, pv, v, ldv, stream));
+    // the expand's predecessor is this call's shrink, which does not write y: y may be read early
+    SGMV_CUDA_TRY(launch_expand_simt(v, ldv, d_out, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, pv,
+                                     scale, y, ldy, y_dtype, use_inl ? &inl : nullptr, true, stream));
     SGMV_CUDA_TRY(launch_expand_tc(v, ldv, d_out, bv, plan->num_tc_tiles, plan->max_rank, pv, scale, y, ldy, y_dtype,
                                    stream));
     return SGMV_OK;
@@ -188,11 +246,8 @@ extern "C" sgmv_status sgmv_lora_delta(const void* x, int64_t ldx, int32_t T, in
                                        sgmv_stream_t stream) {
     if (plan && plan->num_rows > 0 && (plan->num_simt_items > 0 || plan->num_tc_tiles > 0) && !v)
         return fail(SGMV_ERR_INVALID, "lora_delta: the workspace v is required");
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    sgmv_status st = shrink_impl(x, ldx, T, d_in, proj, plan, table, pool, v, ldv, s);
-    if (st != SGMV_OK) return st;
-    // the expand's predecessor is this shrink, which does not write y: y may be read early
-    return expand_impl(v, ldv, T, d_out, proj, plan, table, pool, scale, y, ldy, y_dtype, true, s);
+    return delta_impl(x, ldx, T, d_in, d_out, proj, plan, table, pool, scale, y, ldy, y_dtype, v, ldv,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------

@@ -6,28 +6,27 @@
 // small segments take a batched gather path.  One launch per phase covers
 // every short segment of the batch, whatever its rank, with no padded work.
 //
-// Decode batches move a few MB per phase, so both kernels are built around
+// Decode batches move a few MB per phase, so the kernels are built around
 // latency: a CTA first reads the page ids of everything it will touch in one
-// round of independent loads, then keeps up to four 16 KB stages of adapter
+// round of independent loads, then keeps three or four 16 KB stages of adapter
 // rows in flight with 16-byte cp.async copies issued by all threads (pages are
-// 1 KiB and scattered, which is too fine-grained for one bulk copy per page),
-// the token rows are fetched while those copies fly, and the expand is launched
-// as a programmatic dependent of the shrink so that its B^T stages stream in
-// while the shrink is still running.
+// 1 KiB and scattered, too fine-grained for one bulk copy per page); the token
+// rows' x slices travel in the same stages.  Grids are sized to one wave of
+// resident CTAs.
 //
 // shrink:  a thread-block cluster of C CTAs per work item (<= 4 rows of one
-//          segment); CTA q owns d_in columns [q kc, (q+1) kc).  Stages are 8
-//          rank rows x up to 1024 columns; each thread owns 8 columns and
-//          keeps the item's (up to 4) tokens' x in registers; partial dot products are
-//          reduced with warp shuffles and shared memory; the other CTAs of the
-//          cluster push their partial tiles into rank 0's shared memory, which
-//          sums them in a fixed order and writes v.  Deterministic, no atomics,
-//          no scratch memory.
+//          segment); CTA q owns a page-aligned share of d_in.  Stages are 8
+//          rank rows x up to 1024 columns; each thread owns 8 columns; partial
+//          dot products are reduced with warp shuffles and shared memory; the
+//          other CTAs of the cluster push their partial tiles into rank 0's
+//          shared memory, which sums them in a fixed order and writes v.
+//          Deterministic, no atomics, no scratch memory.
 // expand:  CTAs per work item each cover one or more 1024-column passes of
-//          d_out (about four CTAs per SM in total).  B^T rank rows are staged by
-//          bulk copies before the kernel waits for the shrink; then v of the
-//          item is read, each thread accumulates its 8 output columns for up to
-//          4 tokens and updates y with one rounding, pass by pass.
+//          d_out.  Launched as a programmatic dependent of the shrink: B^T rank
+//          rows are staged (and, inside sgmv_lora_delta, the first y rows read)
+//          before the kernel waits for the shrink; then v of the item is read,
+//          each thread accumulates its 8 output columns for up to 4 tokens and
+//          updates y with one rounding, pass by pass.
 #include <cuda_bf16.h>
 
 #include <map>

@@ -19,9 +19,13 @@
 // distributed shared memory into v.
 // expand: v (fp32) is split into bf16 hi + lo parts so that the delta keeps
 // ~16 bits of v: D = V_hi B + V_lo B, both products exact, fp32 accumulation.
+#include <cuda.h>  // CUtensorMap (the encoder is reached through the runtime's driver entry point)
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cstring>
+#include <mutex>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -48,6 +52,7 @@ struct ShrinkTcArgs {
     int32_t npad_max;    // largest padded rank of the launch (multiple of 16)
     int32_t tmem_cols;   // tensor-memory columns allocated per CTA
     int32_t pid_offset;  // byte offset of the page-id table in shared memory
+    int32_t use_tma;     // tmap_x is valid: tiles whose rows are consecutive tokens load X by TMA
 };
 
 struct ExpandTcArgs {
@@ -64,6 +69,7 @@ struct ExpandTcArgs {
     int32_t num_units;      // tiles x n_blocks
     int32_t units_per_cta;  // contiguous run of units per CTA
     int32_t kpad_max;
+    int32_t use_tma;        // tmap_y is valid: tiles of consecutive tokens move y by TMA
 };
 
 __device__ __forceinline__ int32_t safe_page(const PoolView& pool, int64_t entry) {
@@ -88,7 +94,8 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // once the MMAs that read it have completed (tcgen05.commit).  Every wait is
 // bounded; a wait that gives up sets kErrTimeout and the CTA's abort flag, and
 // the remaining waits of the CTA are skipped.
-__global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkTcArgs a) {
+__global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkTcArgs a,
+                                                                     const __grid_constant__ CUtensorMap tmap_x) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     __shared__ uint64_t full_bar[kShrinkStages], empty_bar[kShrinkStages], acc_bar;
@@ -161,6 +168,12 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
+    // rows that are consecutive tokens (a prefill segment): X tiles come by one TMA
+    // load each, 128 rows of 128 bytes in the same 128-byte swizzle (rows past the
+    // tile are other tokens or zero fill; their results are discarded)
+    const int t0 = tok_s[0];
+    const bool x_tma = __syncthreads_and(tid >= rows || tid >= kTcTileRows || (t0 >= 0 && tok_s[tid] == t0 + tid)) &&
+                       a.use_tma && ok;
 
     if (warp < 4) {
         // ---- producers.  Tiles are K-major with the 128-byte swizzle (8-row atoms of
@@ -175,14 +188,21 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
             uint8_t* xs = stage0 + (size_t)st * stage_bytes;
             uint8_t* as = xs + x_tile_bytes;
             const int c = k_begin + kt * kKTile;
+            if (x_tma) {
+                if (tid == 0) {
+                    mbar_expect_tx(&full_bar[st], (uint32_t)x_tile_bytes);
+                    tma_load_2d(xs, &tmap_x, c, t0, &full_bar[st]);
+                }
+            } else {
 #pragma unroll
-            for (int i = 0; i < (kTcTileRows * 8) / kTcTileRows; ++i) {
-                const int g = tid + i * kTcTileRows;
-                const int row = g >> 3, kg = g & 7;
-                const int t = tok_s[row];
-                const uint32_t off = (uint32_t)(row >> 3) * 1024 + sw128_off((uint32_t)row, (uint32_t)kg);
-                const uint16_t* src = t >= 0 ? a.x + (int64_t)t * a.ldx + c + kg * 8 : a.x;
-                cp_async16(xs + off, src, t >= 0);
+                for (int i = 0; i < (kTcTileRows * 8) / kTcTileRows; ++i) {
+                    const int g = tid + i * kTcTileRows;
+                    const int row = g >> 3, kg = g & 7;
+                    const int t = tok_s[row];
+                    const uint32_t off = (uint32_t)(row >> 3) * 1024 + sw128_off((uint32_t)row, (uint32_t)kg);
+                    const uint16_t* src = t >= 0 ? a.x + (int64_t)t * a.ldx + c + kg * 8 : a.x;
+                    cp_async16(xs + off, src, t >= 0);
+                }
             }
             // A: rank rows n < npad, zero past r; the 64 columns lie in one page
             const int page_rel = (c >> P_log2) - first_page, in_page = c & ((1 << P_log2) - 1);
@@ -195,6 +215,7 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
                     src = a.pool.pages + ((int64_t)pid_s[n * span_pages + page_rel] << P_log2) + in_page + kg * 8;
                 cp_async16(as + off, src, valid);
             }
+            cp_async_commit();  // close the group: the copies of every stage form their own
             cp_async_mbar_arrive_noinc(&full_bar[st]);
         }
     } else if (tid == 4 * 32) {
@@ -267,39 +288,46 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
 // Persistent: CTA b takes a contiguous run of units (tile of <= 128 rows, block
 // of kYRowBytes of y columns), so consecutive units mostly share the tile and
 // its v rows.  Warp roles:
-//   warps 4-7 (producers): per unit, fetch the token rows and B^T page ids, then
-//     cp.async the y rows and the B^T block into stage slot s; when the tile
-//     changes, write V_hi / V_lo (v split into bf16 hi + lo, K-major)
-//   warp 8 (one lane): tcgen05.mma  acc[i & 1] = V_hi B + V_lo B  (N = block)
-//   warps 0-3 (epilogue): tcgen05.ld acc -> Y block += scale * acc in shared
-//     memory (row per thread) -> coalesced 16-byte stores of the block
-// mbarriers: full[s] (128 producer copies landed, cp.async.mbarrier.arrive),
-// yfree[s] (128 epilogue threads stored the block), accf[b] (MMAs done,
-// tcgen05.commit), acce[b] (128 epilogue threads read acc[b] out), vfull /
-// vempty (V of a tile written / its last MMA done).  The tensor-memory
-// accumulator is double-buffered, so the MMAs of unit i+1 overlap the epilogue
-// of unit i.  Every wait is bounded.
+//   warps 8-11 (producers): per unit, fetch the token rows and B^T page ids;
+//     copy each y row segment (256 bytes) with one bulk copy that completes on
+//     the stage's mbarrier by bytes, and the B^T block with 16-byte cp.async;
+//     when the tile changes, write V_hi / V_lo (v split into bf16 hi + lo)
+//   warp 12 (one lane): tcgen05.mma  acc[i & 1] = V_hi B + V_lo B  (N = block)
+//   warps 0-7 (epilogue): two groups of four warps take alternate units (the
+//     group of unit i reads acc[i & 1]); warp w reads rows 32 (w % 4) .. + 31 of
+//     the accumulator (tcgen05.ld) and adds scale * acc to its y rows in shared
+//     memory; the group then stores the block: one TMA store per half for a full
+//     tile of consecutive tokens, coalesced 16-byte stores otherwise
+// mbarriers: full[s] (producers' copies landed: 128 cp.async arrivals plus the
+// TMA bytes), yfree[s] (the unit's epilogue group has stored slot s), accf[b]
+// (MMAs done, tcgen05.commit), acce[b] (the group has read acc[b] out),
+// vfull / vempty (V of a tile written / its last MMA done).  The accumulator
+// is double-buffered in tensor memory, so the MMAs of unit i+1 overlap the
+// epilogue of unit i.  Every wait is bounded.
 constexpr int kYRowBytes = 256;             // y bytes of one tile row per unit (128 bf16 / 64 fp32)
 constexpr int kMaxPagesPerUnit = 2;         // pages of one B^T row a unit spans (page_elems >= 64)
-constexpr int kYStride = kYRowBytes + 16;   // padded shared-memory row stride
-constexpr int kExpandThreads = 288;         // 4 epilogue + 4 producer warps + 1 MMA warp
+constexpr int kExpandThreads = 416;         // 8 epilogue + 4 producer warps + 1 MMA warp
+constexpr int kExpandProducers = 128;
+constexpr int kMmaWarp = 12;
 constexpr int kMaxExpandStages = 3;
 
-template <int S>
-__global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const ExpandTcArgs a) {
+template <int S, int ESZ>  // ESZ: bytes of a y element (2: bf16, 4: fp32)
+__global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const ExpandTcArgs a,
+                                                                      const __grid_constant__ CUtensorMap tmap_y) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     __shared__ uint64_t full_bar[S], yfree_bar[S], accf_bar[2], acce_bar[2], vfull_bar, vempty_bar;
     __shared__ uint32_t tmem_slot;
     __shared__ volatile int abort_flag;
-    __shared__ int32_t tok_s[S][kTcTileRows];
     __shared__ int32_t pid_s[S][kMaxRank * kMaxPagesPerUnit];  // B^T page ids of a unit [rank row][page]
+    __shared__ int32_t tok_s[S][kTcTileRows];                    // producers: token of each row of a unit
+    __shared__ int32_t tok_row[2][kTcTileRows];                  // epilogue groups: token of each row, -1 = none
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int u0 = blockIdx.x * a.units_per_cta, u1 = min(u0 + a.units_per_cta, a.num_units);
     if (u0 >= u1) return;  // uniform, before anything is allocated
-    const int esz = a.y_dtype == 0 ? 2 : 4;
-    const int NB = kYRowBytes / esz;              // output columns per unit
+    constexpr int esz = ESZ;
+    constexpr int NB = kYRowBytes / ESZ;          // output columns per unit
     const int kpm = a.kpad_max;
     // V_hi / V_lo: K-major, 128-byte swizzle, blocks of 64 K columns (128 rows x 128 bytes each)
     const int kpmv = (kpm + 63) & ~63;
@@ -307,17 +335,20 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
     uint8_t* vlo = vhi + (size_t)kTcTileRows * kpmv * 2;
     // B^T block: MN-major, 128-byte swizzle: atoms of 8 K rows x 64 columns; atoms along N
     // 1024 bytes apart (lbo), 8-row K groups sbo_b apart
-    const uint32_t sbo_b = (uint32_t)(NB / 64) * 1024;
+    constexpr uint32_t sbo_b = (uint32_t)(NB / 64) * 1024;
     uint8_t* bst = vlo + (size_t)kTcTileRows * kpmv * 2;          // [S][kpm x NB]
     const size_t b_bytes = (size_t)kpm * NB * 2;
-    uint8_t* yst = bst + (size_t)S * b_bytes;                      // [S][128 x kYStride]
-    const size_t y_bytes = (size_t)kTcTileRows * kYStride;
+    // Y block: two halves of 128 rows x 128 bytes, each in the 128-byte swizzle (as a
+    // TMA box lands): chunk q of row m of half h at h * 16 KB + m * 128 + (q ^ (m & 7)) * 16
+    uint8_t* yst = bst + (size_t)S * b_bytes;                      // [S][2][128 x 128 bytes]
+    constexpr int kYHalf = kTcTileRows * (kYRowBytes / 2);
+    const size_t y_bytes = 2 * (size_t)kYHalf;
 
     if (tid == 0) {
         abort_flag = 0;
         for (int i = 0; i < S; ++i) {
-            mbar_init(&full_bar[i], kTcTileRows);
-            mbar_init(&yfree_bar[i], kTcTileRows);
+            mbar_init(&full_bar[i], kExpandProducers);
+            mbar_init(&yfree_bar[i], kTcTileRows);  // one epilogue group per unit
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&accf_bar[i], 1);
@@ -327,7 +358,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
         mbar_init(&vempty_bar, 1);
         fence_mbar_init();
     }
-    if (warp == 8) {
+    if (warp == kMmaWarp) {
         tmem_alloc(&tmem_slot, (uint32_t)(2 * NB));
         tmem_relinquish();
     }
@@ -364,26 +395,70 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
         if (!abort_flag && !mbar_wait(bar, parity, &g_err_tc)) abort_flag = 1;
     };
 
-    if (warp >= 4 && warp < 8) {
+    if (warp >= 8 && warp < kMmaWarp) {
         // ------------------------------------------------------------ producers
-        const int pt = tid - 128;
+        const int pt = tid - 256;  // 0 .. 127: also the tile row this thread handles
+        const int npc = NB > (1 << P_log2) ? (NB >> P_log2) : 1;
+        // indices of a unit (token row of this thread's tile row, <= 2 B^T page ids),
+        // loaded one unit ahead so that their latency overlaps the current copies
+        auto fetch = [&](const Unit& w, int& t, int& t0, int32_t (&pg)[2]) {
+            t = t0 = -1;
+            pg[0] = pg[1] = 0;
+            if (!w.ok) return;
+            t0 = a.b.token_idx[w.row_begin];  // (checked by the thread of row 0)
+            if (pt < w.rows) {
+                t = a.b.token_idx[w.row_begin + pt];
+                if (t < 0 || t >= a.b.T) {
+                    atomicOr(&g_err_tc, kErrToken);
+                    t = -1;
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int e = pt + h * kExpandProducers;
+                if (e < w.r * npc) {
+                    const int k = e / npc, pc = e - k * npc;
+                    pg[h] = safe_page(a.pool, w.b_base + (int64_t)k * pages_per_row + (w.j0 >> P_log2) + pc);
+                }
+            }
+        };
+        int t_next, t0_next;
+        int32_t pg_next[2];
+        fetch(unit(u0), t_next, t0_next, pg_next);
         int ts = -1, cur_tile = -1;
         for (int u = u0; u < u1; ++u) {
             const int i = u - u0, st = i % S;
             const Unit w = unit(u);
+            const int t = t_next, t0 = t0_next;
+            const int32_t pg0 = pg_next[0], pg1 = pg_next[1];
+            if (u + 1 < u1) fetch(unit(u + 1), t_next, t0_next, pg_next);
             if (i >= S) wait(&yfree_bar[st], (uint32_t)((i / S - 1) & 1));
             if (w.ok && w.tile != cur_tile) {
                 if (ts >= 0) wait(&vempty_bar, (uint32_t)(ts & 1));  // the MMAs of the previous tile are done
                 const int m = pt, kpad = (w.r + 15) & ~15;
                 const bool row_ok = m < w.rows;
                 const float* vrow = a.v + (int64_t)(w.row_begin + (row_ok ? m : 0)) * a.ldv;
-                for (int kg = 0; kg < kpad / 8; ++kg) {
-                    float f[8];
+                // v row in chunks of 64 floats, each chunk's 16-byte loads all in flight
+                // (a load starts below r and below ldv, a multiple of 4: it stays in the row)
+                float4 vq[16];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int k = kg * 8 + e;
-                        f[e] = (row_ok && k < w.r) ? vrow[k] : 0.f;
+                for (int kg = 0; kg < kMaxRank / 8; ++kg) {
+                    if (kg >= kpad / 8) break;
+                    if ((kg & 7) == 0) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int k4 = kg * 8 + 4 * e;
+                            vq[e] = (row_ok && k4 < w.r && k4 < a.ldv) ? *reinterpret_cast<const float4*>(vrow + k4)
+                                                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
                     }
+                    float f[8];
+                    const float4 q0 = vq[2 * (kg & 7)], q1 = vq[2 * (kg & 7) + 1];
+                    f[0] = q0.x; f[1] = q0.y; f[2] = q0.z; f[3] = q0.w;
+                    f[4] = q1.x; f[5] = q1.y; f[6] = q1.z; f[7] = q1.w;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if (kg * 8 + e >= w.r) f[e] = 0.f;
                     uint32_t hw[4], lw[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -400,43 +475,44 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
                     *reinterpret_cast<uint4*>(vlo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
                 }
                 fence_proxy_async_smem();  // the tensor core reads V through the async proxy
-                named_bar_sync(1, 128);
+                named_bar_sync(1, kExpandProducers);
                 if (pt == 0) mbar_arrive(&vfull_bar);
                 ++ts;
                 cur_tile = w.tile;
             }
             if (w.ok) {
-                // indices of the unit, one round of independent loads
-                const int npc = NB > (1 << P_log2) ? (NB >> P_log2) : 1;
-                int t = -1;
-                if (pt < w.rows) {
-                    t = a.b.token_idx[w.row_begin + pt];
-                    if (t < 0 || t >= a.b.T) {
-                        atomicOr(&g_err_tc, kErrToken);
-                        t = -1;
-                    }
-                }
+                if (pt < w.r * npc) pid_s[st][pt] = pg0;
+                if (pt + kExpandProducers < w.r * npc) pid_s[st][pt + kExpandProducers] = pg1;
                 tok_s[st][pt] = t;
-                for (int e = pt; e < w.r * npc; e += 128) {
-                    const int k = e / npc, pc = e - k * npc;
-                    pid_s[st][e] = safe_page(a.pool, w.b_base + (int64_t)k * pages_per_row + (w.j0 >> P_log2) + pc);
-                }
-                named_bar_sync(1, 128);
-                // y rows: 16 threads per row, 16 bytes each
+                // page ids and token rows in shared memory; are the rows consecutive tokens?
+                const bool contig = named_bar_and(1, kExpandProducers, pt >= w.rows || (t == t0 + pt && t0 >= 0));
                 uint8_t* ys = yst + (size_t)st * y_bytes;
-#pragma unroll 4
-                for (int k16 = 0; k16 < kTcTileRows * (kYRowBytes / 16) / 128; ++k16) {
-                    const int g = pt + k16 * 128;
-                    const int m = g >> 4, q16 = g & 15;
-                    const int tm = tok_s[st][m];
-                    if (tm >= 0)
-                        cp_async16(ys + m * kYStride + q16 * 16, ybase + ((int64_t)tm * a.ldy + w.j0) * esz + q16 * 16,
-                                   true);
+                if (contig && a.use_tma) {
+                    if (pt == 0) {  // two boxes of 128 rows (rows past the tile: other tokens or zero fill)
+                        mbar_expect_tx(&full_bar[st], (uint32_t)y_bytes);
+                        tma_load_2d(ys, &tmap_y, w.j0, t0, &full_bar[st]);
+                        tma_load_2d(ys + kYHalf, &tmap_y, w.j0 + NB / 2, t0, &full_bar[st]);
+                    }
+                } else {
+                    // 16 threads per row; each 8-lane quarter copies 128 contiguous bytes
+#pragma unroll
+                    for (int k16 = 0; k16 < kTcTileRows * (kYRowBytes / 16) / kExpandProducers; ++k16) {
+                        const int g = pt + k16 * kExpandProducers;
+                        const int m = g >> 4, q16 = g & 15;
+                        const int tm = tok_s[st][m];
+                        if (tm >= 0)
+                            cp_async16(ys + (q16 >> 3) * kYHalf + m * 128 +
+                                           (((uint32_t)(q16 & 7) ^ (uint32_t)(m & 7)) << 4),
+                                       ybase + ((int64_t)tm * a.ldy + w.j0) * esz + q16 * 16, true);
+                    }
                 }
                 // B^T block: granule (k, jg) = B^T[k][j0 + 8 jg .. +8], zero past r
                 uint8_t* bs = bst + (size_t)st * b_bytes;
                 const int kpad = (w.r + 15) & ~15;
-                for (int g = pt; g < kpad * (NB / 8); g += 128) {
+#pragma unroll
+                for (int gi = 0; gi < kMaxRank * (kYRowBytes / 16) / kExpandProducers; ++gi) {  // <= 16 granules a row
+                    const int g = pt + gi * kExpandProducers;
+                    if (g >= kpad * (NB / 8)) break;
                     const int jg = g % (NB / 8), k = g / (NB / 8);
                     const int j = w.j0 + jg * 8;
                     const uint32_t off = (uint32_t)(k >> 3) * sbo_b + (uint32_t)(jg >> 3) * 1024 +
@@ -451,9 +527,10 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
             } else if (pt == 0) {
                 atomicOr(&g_err_tc, kErrRows);
             }
+            cp_async_commit();
             cp_async_mbar_arrive_noinc(&full_bar[st]);
         }
-    } else if (warp == 8) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if ((tid & 31) == 0) {
             const uint32_t idesc = idesc_bf16_f32(128, NB, false, true);
@@ -469,7 +546,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
                 }
                 if (i >= 2) wait(&acce_bar[bsel], (uint32_t)((i / 2 - 1) & 1));
                 wait(&full_bar[st], (uint32_t)((i / S) & 1));
-                fence_proxy_async_smem();  // the copies were made through the generic proxy
+                fence_proxy_async_smem();  // the B^T copies were made through the generic proxy
                 tc_fence_after();
                 if (w.ok) {
                     const int kpad = (w.r + 15) & ~15;
@@ -491,73 +568,137 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
-        const int m = tid;
-        for (int u = u0; u < u1; ++u) {
+        // Two warp groups take turns: group g (warps 4g .. 4g+3) handles the units
+        // i with i % 2 == g, whose accumulator is acc[g], over whole rows.
+        const int grp = warp >> 2;
+        const int m = (warp & 3) * 32 + (tid & 31);  // tile row (tensor-memory lane)
+        const int gt = tid & 127;                     // thread within the group
+        for (int u = u0 + grp; u < u1; u += 2) {
             const int i = u - u0, st = i % S, bsel = i & 1;
             const Unit w = unit(u);
             wait(&accf_bar[bsel], (uint32_t)((i / 2) & 1));
             wait(&full_bar[st], (uint32_t)((i / S) & 1));  // (completed: makes the staged y visible here)
             tc_fence_after();
-            uint8_t* yrow = yst + (size_t)st * y_bytes + (size_t)m * kYStride;
-            const bool row_ok = w.ok && m < w.rows && !abort_flag;
-            for (int c0 = 0; c0 < NB; c0 += 32) {
-                uint32_t regs[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(bsel * NB + c0), regs);
+            uint8_t* ys = yst + (size_t)st * y_bytes;
+            int t = -1;  // the row's token (the producer flags a bad one and leaves the row alone)
+            if (w.ok && m < w.rows) {
+                t = a.b.token_idx[w.row_begin + m];
+                if (t >= a.b.T) t = -1;
+            }
+            const bool row_ok = t >= 0 && !abort_flag;
+            for (int c00 = 0; c00 < NB; c00 += 64) {
+                uint32_t rr[2][32];  // two loads in flight per wait
+                const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(bsel * NB + c00);
+                tmem_ld_32x32b_x32(ta, rr[0]);
+                tmem_ld_32x32b_x32(ta + 32, rr[1]);
                 tmem_ld_wait();
                 if (!row_ok) continue;
-                if (a.y_dtype == 0) {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint4* yp = reinterpret_cast<uint4*>(yrow + (c0 + q4 * 8) * 2);
-                        float yf[8];
-                        unpack8(*yp, yf);
-                        uint32_t wv[4];
+                for (int h = 0; h < 2; ++h) {
+                    const int c0 = c00 + 32 * h;                 // column within the block
+                    const int hf = c0 / (NB / 2), cc = c0 % (NB / 2);  // half, column within it
+                    uint8_t* yrow = ys + (size_t)hf * kYHalf + (size_t)m * 128;  // swizzled row
+                    const uint32_t (&regs)[32] = rr[h];
+                    if (ESZ == 2) {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float lo = fmaf(a.scale, __uint_as_float(regs[q4 * 8 + 2 * e]), yf[2 * e]);
-                            const float hi = fmaf(a.scale, __uint_as_float(regs[q4 * 8 + 2 * e + 1]), yf[2 * e + 1]);
-                            wv[e] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
-                                    ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint4* yp = reinterpret_cast<uint4*>(yrow + ((((cc >> 3) + q4) ^ (m & 7)) << 4));
+                            float yf[8];
+                            unpack8(*yp, yf);
+                            uint32_t wv[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float lo = fmaf(a.scale, __uint_as_float(regs[q4 * 8 + 2 * e]), yf[2 * e]);
+                                const float hi = fmaf(a.scale, __uint_as_float(regs[q4 * 8 + 2 * e + 1]), yf[2 * e + 1]);
+                                wv[e] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+                                        ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+                            }
+                            *yp = make_uint4(wv[0], wv[1], wv[2], wv[3]);
                         }
-                        *yp = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                    }
-                } else {
+                    } else {
 #pragma unroll
-                    for (int q4 = 0; q4 < 8; ++q4) {
-                        float4* yp = reinterpret_cast<float4*>(yrow + (c0 + q4 * 4) * 4);
-                        float4 yv = *yp;
-                        yv.x = fmaf(a.scale, __uint_as_float(regs[q4 * 4 + 0]), yv.x);
-                        yv.y = fmaf(a.scale, __uint_as_float(regs[q4 * 4 + 1]), yv.y);
-                        yv.z = fmaf(a.scale, __uint_as_float(regs[q4 * 4 + 2]), yv.z);
-                        yv.w = fmaf(a.scale, __uint_as_float(regs[q4 * 4 + 3]), yv.w);
-                        *yp = yv;
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            float4* yp = reinterpret_cast<float4*>(yrow + ((((cc >> 2) + q4) ^ (m & 7)) << 4));
+                            float4 yv = *yp;
+                            yv.x = fmaf(a.scale, __uint_as_float(regs[q4 * 4 + 0]), yv.x);
+                            yv.y = fmaf(a.scale, __uint_as_float(regs[q4 * 4 + 1]), yv.y);
+                            yv.z = fmaf(a.scale, __uint_as_float(regs[q4 * 4 + 2]), yv.z);
+                            yv.w = fmaf(a.scale, __uint_as_float(regs[q4 * 4 + 3]), yv.w);
+                            *yp = yv;
+                        }
                     }
                 }
             }
             tc_fence_before();
             mbar_arrive(&acce_bar[bsel]);  // acc[bsel] has been read out
-            named_bar_sync(2, 128);        // the Y block is complete
-            if (w.ok && !abort_flag) {
-                const uint8_t* ys = yst + (size_t)st * y_bytes;
-#pragma unroll 4
-                for (int k16 = 0; k16 < kTcTileRows * (kYRowBytes / 16) / 128; ++k16) {
-                    const int g = m + k16 * 128;
-                    const int mm = g >> 4, q16 = g & 15;
-                    const int t = tok_s[st][mm];
-                    if (mm < w.rows && t >= 0)
-                        *reinterpret_cast<uint4*>(ybase + ((int64_t)t * a.ldy + w.j0) * esz + q16 * 16) =
-                            *reinterpret_cast<const uint4*>(ys + mm * kYStride + q16 * 16);
+            tok_row[grp][m] = t;
+            // a full tile of consecutive tokens goes back by TMA (a partial one must not
+            // touch the rows past it)
+            const int t0 = w.ok ? a.b.token_idx[w.row_begin] : -1;
+            const bool full = named_bar_and(2 + grp, kTcTileRows, w.ok && w.rows == kTcTileRows && t0 >= 0 &&
+                                                                      t == t0 + m && !abort_flag);
+            if (full && a.use_tma) {
+                fence_proxy_async_smem();  // this thread's row, to the async proxy
+                named_bar_sync(2 + grp, kTcTileRows);
+                if (gt == 0) {
+                    tma_store_2d(&tmap_y, w.j0, t0, ys);
+                    tma_store_2d(&tmap_y, w.j0 + NB / 2, t0, ys + kYHalf);
+                    bulk_commit();
+                    bulk_wait_read_all();  // the block has been read: slot st may be refilled
+                }
+            } else if (w.ok && !abort_flag) {
+                // coalesced 16-byte stores: 16 threads per row, two rows per warp instruction
+#pragma unroll
+                for (int k16 = 0; k16 < kTcTileRows * (kYRowBytes / 16) / kTcTileRows; ++k16) {
+                    const int mm = (gt >> 4) + k16 * (kTcTileRows / 16), q16 = gt & 15;
+                    const int tt = tok_row[grp][mm];
+                    if (tt >= 0)
+                        *reinterpret_cast<uint4*>(ybase + ((int64_t)tt * a.ldy + w.j0) * esz + q16 * 16) =
+                            *reinterpret_cast<const uint4*>(ys + (q16 >> 3) * kYHalf + mm * 128 +
+                                                             (((uint32_t)(q16 & 7) ^ (uint32_t)(mm & 7)) << 4));
                 }
             }
+            named_bar_sync(2 + grp, kTcTileRows);  // tok_row may be rewritten
             mbar_arrive(&yfree_bar[st]);  // slot st may be refilled
         }
+        if (gt == 0) bulk_wait_all();  // the TMA stores have reached global memory
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, (uint32_t)(2 * NB));
     }
+}
+
+// 2-D tensor map over a row-major matrix (rows x cols elements, row stride in
+// bytes), box of box_rows x box_cols with the 128-byte swizzle.  False if the
+// encoder is unavailable or rejects the layout (the kernels then gather).
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t cols, uint64_t rows,
+               uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows) {
+    static std::mutex mu;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static bool tried = false;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!tried) {
+            tried = true;
+            cudaDriverEntryPointQueryResult q;
+            void* f = nullptr;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+                q == cudaDriverEntryPointSuccess)
+                fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+            cudaGetLastError();
+        }
+    }
+    if (!fn || rows == 0 || (reinterpret_cast<uintptr_t>(base) & 15) || (row_stride_bytes & 15)) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {row_stride_bytes};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int pow2_at_least(int n) {
@@ -613,7 +754,11 @@ cudaError_t launch_shrink_tc(const uint16_t* x, int64_t ldx, int32_t d_in, const
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, shrink_tc_kernel, a);
+    CUtensorMap tmap_x;
+    std::memset(&tmap_x, 0, sizeof(tmap_x));
+    a.use_tma = encode_2d(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)d_in, (uint64_t)b.T,
+                          (uint64_t)ldx * 2, kKTile, kTcTileRows) ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, shrink_tc_kernel, a, tmap_x);
 }
 
 cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const BatchView& b, int32_t num_tiles,
@@ -637,9 +782,9 @@ cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const B
     a.num_units = a.n_blocks * num_tiles;
     // shared memory: V hi + lo, S stages of (B^T block, Y block); three stages when they fit
     const size_t v_bytes = (size_t)2 * kTcTileRows * ((a.kpad_max + 63) & ~63) * 2;
-    const size_t stage = (size_t)a.kpad_max * NB * 2 + (size_t)kTcTileRows * kYStride;
+    const size_t stage = (size_t)a.kpad_max * NB * 2 + (size_t)kTcTileRows * kYRowBytes;
     // the opt-in limit covers dynamic (+1 KB alignment) and static (index tables, barriers) shared memory
-    const size_t limit = (227u << 10) - 1024 - 1024 - (size_t)kMaxExpandStages * kTcTileRows * 4 -
+    const size_t limit = (227u << 10) - 1024 - 1024 - (size_t)(kMaxExpandStages + 1) * kTcTileRows * 4 -
                          (size_t)kMaxExpandStages * kMaxRank * kMaxPagesPerUnit * 4;
     const int S = (v_bytes + 3 * stage <= limit) ? 3 : 2;
     // at least 116 KB: one CTA per SM, so tensor memory (2 x NB <= 256 columns) is never oversubscribed
@@ -655,15 +800,16 @@ cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const B
     const int grid = std::min(a.num_units, sms);
     a.units_per_cta = (a.num_units + grid - 1) / grid;
     const int blocks = (a.num_units + a.units_per_cta - 1) / a.units_per_cta;
-    if (S == 3) {
-        cudaError_t e = cudaFuncSetAttribute(expand_tc_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        expand_tc_kernel<3><<<(unsigned)blocks, kExpandThreads, smem, stream>>>(a);
-    } else {
-        cudaError_t e = cudaFuncSetAttribute(expand_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        expand_tc_kernel<2><<<(unsigned)blocks, kExpandThreads, smem, stream>>>(a);
-    }
+    CUtensorMap tmap_y;
+    std::memset(&tmap_y, 0, sizeof(tmap_y));
+    const int esz = y_dtype == 0 ? 2 : 4;
+    a.use_tma = encode_2d(&tmap_y, y_dtype == 0 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, y,
+                          (uint64_t)d_out, (uint64_t)b.T, (uint64_t)ldy * esz, (uint32_t)(NB / 2), kTcTileRows) ? 1 : 0;
+    auto kern = S == 3 ? (esz == 2 ? expand_tc_kernel<3, 2> : expand_tc_kernel<3, 4>)
+                       : (esz == 2 ? expand_tc_kernel<2, 2> : expand_tc_kernel<2, 4>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)blocks, kExpandThreads, smem, stream>>>(a, tmap_y);
     return cudaGetLastError();
 }
 

@@ -102,14 +102,23 @@ struct PoolView {
 };
 
 // --------------------------------------------------------------- launchers
+// Work of the SIMT items, in stages of 8 rank rows: `sum_ng` over the items,
+// `max_ng` of the largest (items come largest first).  The launchers size the
+// CTA split with it.
+struct SimtWork {
+    int64_t sum_ng = 0;
+    int32_t max_ng = 0;
+};
 // `inl` (may be null) holds the items as launch arguments when they fit.
 cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, const BatchView& b,
-                               int32_t num_items, int32_t max_item_rows, int32_t max_rank, const PoolView& pool,
-                               float* v, int64_t ldv, const InlineTable<kInlineItems>* inl, cudaStream_t stream);
+                               int32_t num_items, int32_t max_item_rows, int32_t max_rank, const SimtWork& work,
+                               const PoolView& pool, float* v, int64_t ldv, const InlineTable<kInlineItems>* inl,
+                               cudaStream_t stream);
 // y_early: y may be read before the preceding kernel completes (that kernel is
 // the shrink of the same call, which does not write y).
 cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const BatchView& b,
-                               int32_t num_items, int32_t max_item_rows, int32_t max_rank, const PoolView& pool,
+                               int32_t num_items, int32_t max_item_rows, int32_t max_rank, const SimtWork& work,
+                               const PoolView& pool,
                                float scale, void* y, int64_t ldy, int32_t y_dtype,
                                const InlineTable<kInlineItems>* inl, bool y_early, cudaStream_t stream);
 cudaError_t launch_shrink_tc(const uint16_t* x, int64_t ldx, int32_t d_in, const BatchView& b, int32_t num_tiles,

@@ -1,5 +1,6 @@
 // C ABI entry points: argument validation, the size-based dispatch between
 // the SIMT and the tensor-core kernels, and error reporting.
+#include <algorithm>
 #include <cstdio>
 #include <mutex>
 #include <string>
@@ -87,6 +88,29 @@ bool inline_items(const sgmv_plan* plan, int32_t proj, InlineTable<kInlineItems>
         }
     }
     return true;
+}
+
+// Stage counts of the SIMT items, read from the host table (which the plan's
+// contract keeps valid until the calls); uniform by the plan's max rank if absent.
+SimtWork simt_work(const sgmv_plan* plan) {
+    SimtWork w;
+    const int32_t n = plan->num_simt_items;
+    w.max_ng = (std::max(plan->max_rank, 1) + 7) / 8;
+    if (n <= 0) return w;
+    if (!plan->host_table) {
+        w.sum_ng = (int64_t)n * w.max_ng;
+        return w;
+    }
+    const ItemRec* recs = reinterpret_cast<const ItemRec*>(static_cast<const uint8_t*>(plan->host_table) +
+                                                           plan->off_simt_items);
+    int32_t mx = 1;
+    for (int32_t i = 0; i < n; ++i) {
+        const int32_t ng = (std::max(recs[(int64_t)i * plan->n_proj].rank, 1) + 7) / 8;
+        w.sum_ng += ng;
+        mx = std::max(mx, ng);
+    }
+    w.max_ng = mx;
+    return w;
 }
 
 }  // namespace
@@ -189,8 +213,8 @@ sgmv_status sgmv::shrink_impl(const void* x, int64_t ldx, int32_t T, int32_t d_i
     const uint16_t* xb = static_cast<const uint16_t*>(x);
     InlineTable<kInlineItems> inl;
     const bool use_inl = inline_items(plan, proj, &inl);
-    SGMV_CUDA_TRY(launch_shrink_simt(xb, ldx, d_in, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, pv,
-                                     v, ldv, use_inl ? &inl : nullptr, stream));
+    SGMV_CUDA_TRY(launch_shrink_simt(xb, ldx, d_in, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank,
+                                     simt_work(plan), pv, v, ldv, use_inl ? &inl : nullptr, stream));
     SGMV_CUDA_TRY(launch_shrink_tc(xb, ldx, d_in, bv, plan->num_tc_tiles, plan->max_rank, pv, v, ldv, stream));
     return SGMV_OK;
 }
@@ -205,8 +229,9 @@ sgmv_status sgmv::expand_impl(const float* v, int64_t ldv, int32_t T, int32_t d_
     if (st != SGMV_OK || nothing) return st;
     InlineTable<kInlineItems> inl;
     const bool use_inl = inline_items(plan, proj, &inl);
-    SGMV_CUDA_TRY(launch_expand_simt(v, ldv, d_out, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, pv,
-                                     scale, y, ldy, y_dtype, use_inl ? &inl : nullptr, y_early, stream));
+    SGMV_CUDA_TRY(launch_expand_simt(v, ldv, d_out, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank,
+                                     simt_work(plan), pv, scale, y, ldy, y_dtype, use_inl ? &inl : nullptr, y_early,
+                                     stream));
     SGMV_CUDA_TRY(launch_expand_tc(v, ldv, d_out, bv, plan->num_tc_tiles, plan->max_rank, pv, scale, y, ldy, y_dtype,
                                    stream));
     return SGMV_OK;
@@ -229,12 +254,13 @@ sgmv_status sgmv::delta_impl(const void* x, int64_t ldx, int32_t T, int32_t d_in
     const uint16_t* xb = static_cast<const uint16_t*>(x);
     InlineTable<kInlineItems> inl;
     const bool use_inl = inline_items(plan, proj, &inl);
-    SGMV_CUDA_TRY(launch_shrink_simt(xb, ldx, d_in, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, pv,
-                                     v, ldv, use_inl ? &inl : nullptr, stream));
+    SGMV_CUDA_TRY(launch_shrink_simt(xb, ldx, d_in, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank,
+                                     simt_work(plan), pv, v, ldv, use_inl ? &inl : nullptr, stream));
     SGMV_CUDA_TRY(launch_shrink_tc(xb, ldx, d_in, bv, plan->num_tc_tiles, plan->max_rank, pv, v, ldv, stream));
     // the expand's predecessor is this call's shrink, which does not write y: y may be read early
-    SGMV_CUDA_TRY(launch_expand_simt(v, ldv, d_out, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, pv,
-                                     scale, y, ldy, y_dtype, use_inl ? &inl : nullptr, true, stream));
+    SGMV_CUDA_TRY(launch_expand_simt(v, ldv, d_out, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank,
+                                     simt_work(plan), pv, scale, y, ldy, y_dtype, use_inl ? &inl : nullptr, true,
+                                     stream));
     SGMV_CUDA_TRY(launch_expand_tc(v, ldv, d_out, bv, plan->num_tc_tiles, plan->max_rank, pv, scale, y, ldy, y_dtype,
                                    stream));
     return SGMV_OK;

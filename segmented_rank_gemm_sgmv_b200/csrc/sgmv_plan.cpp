@@ -123,6 +123,13 @@ extern "C" sgmv_status sgmv_build_plan(const int32_t* adapter_ids, int32_t T, co
     for (int32_t t = 0; t < T; ++t)  // ascending t keeps each segment in batch order
         if (seg_of[t] >= 0) token_idx[fill[seg_of[t]]++] = t;
     if (S > 0 || L.end > 0) std::memcpy(seg_offsets, offsets.data(), (S + 1) * sizeof(int32_t));
+    // SIMT items are emitted largest rank first (stable): their CTAs are then
+    // scheduled first, and the smaller items fill in behind them
+    struct Simt {
+        int32_t rank, s, r0, r1;
+    };
+    std::vector<Simt> simt_list;
+    simt_list.reserve(n_simt);
     int64_t i_simt = 0, i_tc = 0;
     for (int64_t s = 0; s < S; ++s) {
         seg_adapter[s] = ids[s];
@@ -139,10 +146,12 @@ extern "C" sgmv_status sgmv_build_plan(const int32_t* adapter_ids, int32_t T, co
             for (int32_t r0 = b; r0 < e; r0 += kSimtMaxItemRows) {
                 const int32_t r1 = std::min(e, r0 + kSimtMaxItemRows);
                 max_item = std::max(max_item, r1 - r0);
-                put(simt, i_simt++, (int32_t)s, r0, r1);
+                simt_list.push_back(Simt{recs[s]->rank, (int32_t)s, r0, r1});
             }
         }
     }
+    std::stable_sort(simt_list.begin(), simt_list.end(), [](const Simt& x, const Simt& y) { return x.rank > y.rank; });
+    for (const Simt& it : simt_list) put(simt, i_simt++, it.s, it.r0, it.r1);
 
     std::memset(plan, 0, sizeof(*plan));
     plan->T = T;

@@ -635,14 +635,31 @@ int resident_ctas(const void* kern, size_t smem) {
     return n;
 }
 
+// Modelled time, in stages, of a launch over `items` SIMT items with `cpi` CTAs
+// each (`slots` CTAs resident at a time), every CTA doing npass passes of its
+// item's row groups (work.sum_ng row groups over all items, work.max_ng for the
+// largest) plus a fixed prologue (page ids, pipeline fill) of about two stages.
+// Equal items run in waves; unequal ones (emitted largest first) pack into the
+// slots, bounded below by the largest CTA.  `work_passes`: passes over which
+// one row group of an item is spread in total.
+double split_time(const SimtWork& work, int64_t items, int64_t cpi, int npass, double work_passes, int64_t slots) {
+    constexpr double kPrologue = 2.0;
+    const int64_t n = items * cpi;
+    const double biggest = (double)std::max(work.max_ng, 1) * npass + kPrologue;
+    if (slots < 1) slots = 1;
+    if (work.sum_ng == items * (int64_t)work.max_ng) return (double)((n + slots - 1) / slots) * biggest;
+    const double total = (double)work.sum_ng * work_passes + (double)n * kPrologue;
+    return std::max(biggest, total / (double)slots);
+}
+
 template <typename K1, typename K2, typename K4>
 auto pick(int max_item_rows, K1 k1, K2 k2, K4 k4) {
     return max_item_rows <= 1 ? k1 : max_item_rows <= 2 ? k2 : k4;
 }
 
 cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, const BatchView& b, int32_t num_items,
-                               int32_t max_item_rows, int32_t max_rank, const PoolView& pool, float* v, int64_t ldv,
-                               const InlineTable<kInlineItems>* inl, cudaStream_t stream) {
+                               int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
+                               float* v, int64_t ldv, const InlineTable<kInlineItems>* inl, cudaStream_t stream) {
     if (num_items <= 0) return cudaSuccess;
     auto kern_inl = pick(max_item_rows, shrink_simt_kernel<1, kInlineItems>, shrink_simt_kernel<2, kInlineItems>,
                          shrink_simt_kernel<4, kInlineItems>);
@@ -657,20 +674,20 @@ cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, con
         const size_t pidb = pid_bytes_max / c;
         return (((part_bytes + 1024 + pidb + 127) & ~(size_t)127)) + ring_bytes;
     };
-    // Cluster size C: the largest split (chunks of >= 1024 columns, C <= 8,
-    // dividing the page count) whose grid still fits in one wave of resident
-    // CTAs, so that every CTA streams its share from the start and none waits
-    // for a second wave.  More CTAs per item shorten the per-item chain.
+    // Cluster size C (chunks of >= 1024 columns, C <= 8, dividing the page count):
+    // the one with the shortest modelled time (split_time).
     const int pages = d_in >> pool.page_log2;
+    const void* kp = inl ? reinterpret_cast<const void*>(kern_inl) : reinterpret_cast<const void*>(kern_tab);
     int C = 1;
-    for (int c = 8; c >= 1; --c) {
+    double best = 1e300;
+    for (int c = 1; c <= 8; ++c) {
         if (pages % c || (c > 1 && d_in / c < kPass)) continue;
-        const size_t sm = smem_for(c);
-        const void* kp = inl ? reinterpret_cast<const void*>(kern_inl) : reinterpret_cast<const void*>(kern_tab);
-        const int per_sm = resident_ctas(kp, sm);
-        if ((int64_t)num_items * c <= (int64_t)per_sm * num_sms()) {
+        const int npass = (d_in / c + kPass - 1) / kPass;
+        const double t = split_time(work, num_items, c, npass, (double)npass * c,
+                                    (int64_t)resident_ctas(kp, smem_for(c)) * num_sms());
+        if (t < best) {
+            best = t;
             C = c;
-            break;
         }
     }
     ShrinkArgs a;
@@ -710,7 +727,8 @@ cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, con
 }
 
 cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const BatchView& b, int32_t num_items,
-                               int32_t max_item_rows, int32_t max_rank, const PoolView& pool, float scale, void* y,
+                               int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
+                               float scale, void* y,
                                int64_t ldy, int32_t y_dtype, const InlineTable<kInlineItems>* inl, bool y_early,
                                cudaStream_t stream) {
     if (num_items <= 0) return cudaSuccess;
@@ -739,11 +757,15 @@ cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const
     };
     const int tiles = (d_out + kPass - 1) / kPass;
     a.npass = tiles;
+    double best = 1e300;
     for (int k = tiles; k >= 1; --k) {
         const int np = (tiles + k - 1) / k, cpi = (tiles + np - 1) / np;
-        if (k > 1 && (int64_t)num_items * cpi > (int64_t)resident_ctas(kp, smem_for(np)) * num_sms()) continue;
-        a.npass = np;
-        break;
+        const double t = split_time(work, num_items, cpi, np, (double)tiles,
+                                    (int64_t)resident_ctas(kp, smem_for(np)) * num_sms());
+        if (t < best) {
+            best = t;
+            a.npass = np;
+        }
     }
     a.ctas_per_item = (tiles + a.npass - 1) / a.npass;
     a.stages = kExpandStages;

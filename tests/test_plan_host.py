@@ -105,3 +105,18 @@ def test_errors():
     with pytest.raises(sg.SgmvError) as e:
         pool.plan([1, -2])
     assert e.value.status == 1
+
+
+def test_simt_items_largest_rank_first():
+    """SIMT work items come largest rank first (stable within a rank), so that
+    their CTAs are scheduled before the smaller ones."""
+    ranks = {0: 8, 1: 64, 2: 16, 3: 64, 4: 32}
+    pool = _pool(ranks)
+    ids = np.asarray([0, 1, 2, 3, 4] * 3 + [1, 3], dtype=np.int32)
+    plan = pool.plan(ids, long_threshold=10 ** 9)
+    rec_ranks = [int(r[0, 3]) for r in plan.simt_records]
+    assert rec_ranks == sorted(rec_ranks, reverse=True)
+    segs = [int(r[0, 0]) for r in plan.simt_records]
+    for a, b in zip(range(len(segs) - 1), range(1, len(segs))):
+        if rec_ranks[a] == rec_ranks[b]:
+            assert segs[a] <= segs[b]

@@ -141,6 +141,25 @@ def read_traffic(workload: str, kernel: str):
     return None
 
 
+# ---------------------------------------------------------------------------- ranks
+def reduce_max(x: float, device) -> float:
+    """Max of a per-rank number over all ranks (identity without a process group).
+    Every rank must call it at the same point."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(x)
+    if torch.distributed.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, tokens_per_rank: int, steps: int, total_ms: float) -> float:
+    """Whole-job tokens/s: every rank processes its own batch of the same shape each
+    step (weak scaling); the job's time is the slowest rank's."""
+    return world * tokens_per_rank * steps / (total_ms * 1e-3)
+
+
 # ---------------------------------------------------------------------------- our arm
 def setup(wl_name: str, rank: int, device: int, pool_override: int = 0):
     import segmented_rank_gemm_sgmv_b200 as sg
@@ -220,11 +239,7 @@ def run_ours(args, rank, world, device):
     sg.check_errors(stream)
     step_ms = [e[0].elapsed_time(e[-1]) for e in records]
     proj_ms = [sum(e[1 + 3 * p].elapsed_time(e[3 + 3 * p]) for p in range(n_proj)) for e in records]
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=f"cuda:{device}")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(float(sum(step_ms)), f"cuda:{device}")
 
     shrink_b = expand_b = flops = 0
     for p in range(n_proj):
@@ -298,11 +313,7 @@ def e2e_ours(sg, wl, pool, acts, args, device, stream, world):
         flush.zero_()
         torch.cuda.synchronize(device)
         times.append(one(True))
-    total = float(sum(times))
-    if world > 1:
-        t = torch.tensor([total], dtype=torch.float64, device=f"cuda:{device}")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total = float(t.item())
+    total = reduce_max(float(sum(times)), f"cuda:{device}")
     return dict(total_ms=total, h2d=h2d, d2h=d2h)
 
 
@@ -349,7 +360,7 @@ def run_reference(args, rank, world, device):
     prepared = oracle_inputs(wl, dev)
     for _ in range(args.warmup):
         time_oracle(prepared, wl, 0.0, threads)
-    per_step_budget = max(0.05, 60.0 / max(args.steps, 1))
+    per_step_budget = max(0.05, getattr(args, "ref_budget", 60.0) / max(args.steps, 1))
     t_all, reps_all, used = 0.0, 0, 1
     for _ in range(args.steps):
         _, reps, el, used = time_oracle(prepared, wl, per_step_budget, threads)
@@ -393,6 +404,8 @@ def main():
     ap.add_argument("--split-phases", action="store_true",
                     help="record an event between shrink and expand (times each phase; removes their overlap)")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--ref-budget", type=float, default=60.0,
+                    help="seconds of oracle time over all steps of --impl reference")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -416,9 +429,9 @@ def main():
         if rank != 0:
             return
         n_tok = int((wl.adapter_ids >= 0).sum())
-        value = world * n_tok * args.steps / (res["total_ms"] * 1e-3)
+        value = job_value(world, n_tok, args.steps, res["total_ms"])
         e2e = res["e2e"]
-        e2e_value = world * n_tok * args.steps / (e2e["total_ms"] * 1e-3)
+        e2e_value = job_value(world, n_tok, args.steps, e2e["total_ms"])
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["total_ms"] / args.steps, "higher_is_better": True,

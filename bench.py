@@ -188,6 +188,8 @@ def run_ours(args, rank, world, device):
         pl.build(wl.adapter_ids)
         pl.upload(stream)
     v = plans[0].new_v()
+    grouped = getattr(args, "grouped", False) and n_proj > 1
+    vs = [plans[0].new_v() for _ in range(n_proj)] if grouped else None
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=f"cuda:{device}")
     # Hold the stream for ~200 us after the flush so that the host has enqueued the
     # whole step before the device reaches it: event times are then device times.
@@ -200,6 +202,15 @@ def run_ours(args, rank, world, device):
         if evs:
             evs[0].record(stream)
         pl.upload(stream)                            # one host->device copy of the table
+        if grouped:                                  # every projection in one call
+            if evs:
+                evs[1].record(stream)
+            sg.lora_delta_grouped([(acts[p][0], acts[p][1], p, vs[p]) for p in range(n_proj)], pl, pool,
+                                  wl.scale, stream)
+            if evs:
+                evs[3].record(stream)
+                evs[-1].record(stream)
+            return
         for p in range(n_proj):
             x, y = acts[p]
             if evs:
@@ -238,7 +249,8 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize(device)
     sg.check_errors(stream)
     step_ms = [e[0].elapsed_time(e[-1]) for e in records]
-    proj_ms = [sum(e[1 + 3 * p].elapsed_time(e[3 + 3 * p]) for p in range(n_proj)) for e in records]
+    proj_ms = [sum(e[1 + 3 * p].elapsed_time(e[3 + 3 * p]) for p in range(1 if grouped else n_proj))
+               for e in records]
     total_ms = reduce_max(float(sum(step_ms)), f"cuda:{device}")
 
     shrink_b = expand_b = flops = 0
@@ -252,10 +264,12 @@ def run_ours(args, rank, world, device):
     simt, tc = plan0.num_simt_items > 0, plan0.num_tc_tiles > 0
     kinds = [k for k, on in (("simt", simt), ("tc", tc)) if on]
     names = " + ".join(f"shrink_{k}_kernel" for k in kinds) + " + " + " + ".join(f"expand_{k}_kernel" for k in kinds)
-    res = dict(total_ms=total_ms, proj_ms=float(np.mean(proj_ms)), kernel_name=f"sgmv_lora_delta ({names})",
+    api = "sgmv_lora_delta_grouped" if grouped else "sgmv_lora_delta"
+    res = dict(total_ms=total_ms, proj_ms=float(np.mean(proj_ms)), kernel_name=f"{api} ({names})",
                step_bytes=shrink_b + expand_b, flops=flops, peak=peak, peak_kind=peak_kind,
-               launches=2 * n_proj * len(kinds), clocks=clk.summary(), dom_launches=n_proj,
-               traffic=read_traffic(args.workload, "lora_delta"), split=split)
+               launches=(2 * simt + 2 * n_proj * tc) if grouped else 2 * n_proj * len(kinds),
+               clocks=clk.summary(), dom_launches=1 if grouped else n_proj,
+               traffic=read_traffic(args.workload, "lora_delta_grouped" if grouped else "lora_delta"), split=split)
     if split:
         res["phase_us_per_proj"] = {
             name: [round(1e3 * float(np.mean([e[1 + 3 * p].elapsed_time(e[2 + 3 * p]) for e in records])), 2),
@@ -279,6 +293,8 @@ def e2e_ours(sg, wl, pool, acts, args, device, stream, world):
     out_y = [torch.empty_like(h).pin_memory() for h in host_y]
     plan = sg.BatchPlan(pool, capacity_tokens=wl.T)
     v = None
+    grouped = getattr(args, "grouped", False) and n_proj > 1
+    vs = [None] * n_proj
     h2d = d2h = 0
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=f"cuda:{device}")
 
@@ -292,7 +308,19 @@ def e2e_ours(sg, wl, pool, acts, args, device, stream, world):
             b_in += int(plan.plan.table_bytes)
         if v is None:
             v = plan.new_v()
-        for p in range(n_proj):
+            if grouped:
+                vs[:] = [plan.new_v() for _ in range(n_proj)]
+        if grouped:
+            for p in range(n_proj):
+                dev_x[p].copy_(host_x[p], non_blocking=True)
+                dev_y[p].copy_(host_y[p], non_blocking=True)
+                b_in += host_x[p].numel() * 2 + host_y[p].numel() * 2
+            sg.lora_delta_grouped([(dev_x[p], dev_y[p], p, vs[p]) for p in range(n_proj)], plan, pool, wl.scale,
+                                  stream)
+            for p in range(n_proj):
+                out_y[p].copy_(dev_y[p], non_blocking=True)
+                b_out += out_y[p].numel() * 2
+        for p in range(0 if grouped else n_proj):
             dev_x[p].copy_(host_x[p], non_blocking=True)
             dev_y[p].copy_(host_y[p], non_blocking=True)
             b_in += host_x[p].numel() * 2 + host_y[p].numel() * 2
@@ -401,6 +429,9 @@ def main():
     ap.add_argument("--pool", type=int, default=0,
                     help="resident adapters of the pool (llama70b_layer only; for small profiler captures, "
                          "the kernels see the same batch shape)")
+    ap.add_argument("--per-projection", action="store_true",
+                    help="one sgmv_lora_delta call per projection instead of one sgmv_lora_delta_grouped call "
+                         "for all projections of a multi-projection workload (the default)")
     ap.add_argument("--split-phases", action="store_true",
                     help="record an event between shrink and expand (times each phase; removes their overlap)")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
@@ -408,6 +439,7 @@ def main():
                     help="seconds of oracle time over all steps of --impl reference")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    args.grouped = not args.per_projection and not args.split_phases
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

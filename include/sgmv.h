@@ -289,6 +289,44 @@ SGMV_API sgmv_status sgmv_lora_delta(const void* x, int64_t ldx, int32_t T, int3
                                      int32_t y_dtype, float* v, int64_t ldv, sgmv_stream_t stream);
 
 /*
+ * Several projections of one layer over the same batch in one call: for each
+ * entry, what sgmv_lora_delta does for it, but with one SIMT shrink launch and
+ * one SIMT expand launch covering all entries (the tensor-core tiles still take
+ * a shrink and an expand launch per entry).  A layer's projections share the
+ * batch's adapter assignment ("Multi-LoRA serving: the single translator ...",
+ * section "The maths that matters", memory table: q, k, v, o, gate, up and down
+ * of Llama-3-70B under one adapter), so one plan serves all of them; the launch
+ * boundaries between projections (each a tail and a ramp) go away.
+ *
+ * entries  host array of n_entries (1 .. 8); entry i: projection `proj` of the
+ *          pool with its d_in / d_out, x (bf16 [T][ldx]), y ([T][ldy] of
+ *          y_dtype, updated in place) and workspace v (fp32 [num_rows][ldv],
+ *          ldv >= plan->max_rank), as for sgmv_lora_delta.  Workspaces must not
+ *          overlap (SGMV_ERR_INVALID when two are the same pointer); a y must not
+ *          be another entry's x.  The same projection may appear twice (with
+ *          different x, y, v).
+ * table    the plan's device table.  NULL is accepted for a plan that needs no
+ *          device table: the entries then run one after another.
+ * Errors as for sgmv_lora_delta; all entries are checked before any launch.
+ */
+typedef struct {
+    int32_t proj;
+    int32_t d_in;
+    int32_t d_out;
+    int32_t reserved;       /* 0 */
+    const void* x;
+    int64_t ldx;
+    void* y;
+    int64_t ldy;
+    float* v;
+    int64_t ldv;
+} sgmv_delta_entry;
+
+SGMV_API sgmv_status sgmv_lora_delta_grouped(const sgmv_delta_entry* entries, int32_t n_entries, int32_t T,
+                                             const sgmv_plan* plan, const void* table, const sgmv_pool* pool,
+                                             float scale, int32_t y_dtype, sgmv_stream_t stream);
+
+/*
  * sgmv_lora_delta for callers that cannot give the library device memory.
  * No counterpart on the pages: this is a deployment convenience.
  *

@@ -32,8 +32,8 @@ _STATUS = {0: "SGMV_OK", 1: "SGMV_ERR_INVALID", 2: "SGMV_ERR_UNSUPPORTED", 3: "S
 EXPORTED = ("sgmv_status_string", "sgmv_last_error", "sgmv_pool_create", "sgmv_pool_destroy", "sgmv_pool_load",
             "sgmv_pool_evict", "sgmv_pool_get_stats", "sgmv_pool_adapter_rank", "sgmv_pool_adapter_pages",
             "sgmv_pool_shuffle_free_pages", "sgmv_pool_pages_device", "sgmv_plan_table_capacity",
-            "sgmv_build_plan", "sgmv_shrink", "sgmv_expand", "sgmv_lora_delta", "sgmv_lora_delta_noalloc",
-            "sgmv_check_errors")
+            "sgmv_build_plan", "sgmv_shrink", "sgmv_expand", "sgmv_lora_delta", "sgmv_lora_delta_grouped",
+            "sgmv_lora_delta_noalloc", "sgmv_check_errors")
 
 
 class SgmvError(RuntimeError):
@@ -48,6 +48,12 @@ class Plan(ctypes.Structure):
         "long_threshold", "max_item_rows", "needs_device_table")] + [(n, ctypes.c_int64) for n in (
             "table_bytes", "off_token_idx", "off_seg_offsets", "off_seg_adapter", "off_seg_rank",
             "off_seg_a_pt", "off_seg_b_pt", "off_simt_items", "off_tc_tiles")] + [("host_table", ctypes.c_void_p)]
+
+
+class DeltaEntry(ctypes.Structure):
+    _fields_ = [("proj", ctypes.c_int32), ("d_in", ctypes.c_int32), ("d_out", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("x", ctypes.c_void_p), ("ldx", ctypes.c_int64),
+                ("y", ctypes.c_void_p), ("ldy", ctypes.c_int64), ("v", ctypes.c_void_p), ("ldv", ctypes.c_int64)]
 
 
 class PoolStats(ctypes.Structure):
@@ -88,6 +94,8 @@ def load_library() -> ctypes.CDLL:
         "sgmv_expand": (st, [vp, i64, i32, i32, i32, ctypes.POINTER(Plan), vp, vp, f32, vp, i64, i32, vp]),
         "sgmv_lora_delta": (st, [vp, i64, i32, i32, i32, i32, ctypes.POINTER(Plan), vp, vp, f32, vp, i64, i32,
                                  vp, i64, vp]),
+        "sgmv_lora_delta_grouped": (st, [ctypes.POINTER(DeltaEntry), i32, i32, ctypes.POINTER(Plan), vp, vp, f32,
+                                         i32, vp]),
         "sgmv_lora_delta_noalloc": (st, [vp, i64, i32, i32, i32, i32, ctypes.POINTER(Plan), vp, vp, f32, vp, i64,
                                          i32, vp]),
         "sgmv_check_errors": (st, [vp, ctypes.POINTER(ctypes.c_uint32)]),
@@ -379,6 +387,30 @@ def expand(v: torch.Tensor, plan: BatchPlan, pool: AdapterPool, y: torch.Tensor,
     _check(load_library().sgmv_expand(_ptr(v), v.stride(0), plan.T, y.shape[1], int(proj), ctypes.byref(plan.plan),
                                       plan.table_ptr(stream), pool.handle, float(scale), _ptr(y), y.stride(0),
                                       0 if y.dtype == torch.bfloat16 else 1, _stream(stream)))
+
+
+def lora_delta_grouped(entries, plan: BatchPlan, pool: AdapterPool, scale: float = 1.0, stream=None):
+    """lora_delta for several projections over the same plan in one call (one SIMT
+    shrink and one SIMT expand launch for all of them).  `entries`: (x, y, proj) or
+    (x, y, proj, v) tuples, all y of one dtype.  Returns the workspaces v."""
+    assert 1 <= len(entries) <= 8
+    arr = (DeltaEntry * len(entries))()
+    vs, ydt = [], None
+    for i, e in enumerate(entries):
+        x, y, proj = e[0], e[1], int(e[2])
+        v = e[3] if len(e) > 3 and e[3] is not None else plan.new_v()
+        assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+        assert y.dim() == 2 and y.stride(1) == 1 and y.dtype in (torch.bfloat16, torch.float32)
+        assert v.dtype == torch.float32 and v.dim() == 2 and v.stride(1) == 1
+        assert ydt is None or ydt == y.dtype
+        ydt = y.dtype
+        arr[i] = DeltaEntry(proj, x.shape[1], y.shape[1], 0, _ptr(x), x.stride(0), _ptr(y), y.stride(0), _ptr(v),
+                            v.stride(0))
+        vs.append(v)
+    _check(load_library().sgmv_lora_delta_grouped(arr, len(entries), plan.T, ctypes.byref(plan.plan),
+                                                  plan.table_ptr(stream), pool.handle, float(scale),
+                                                  0 if ydt == torch.bfloat16 else 1, _stream(stream)))
+    return vs
 
 
 def lora_delta_noalloc(x: torch.Tensor, plan: BatchPlan, pool: AdapterPool, y: torch.Tensor, proj: int = 0,

@@ -80,6 +80,7 @@ struct InlineTable {
 constexpr int kTcTileRows = 128;       // rows per tensor-core tile (MMA M)
 constexpr int kDefaultLongThreshold = 16;
 constexpr int kMaxRank = 128;
+constexpr int kMaxGroup = 8;           // projections in one grouped launch
 
 // Device view of everything a kernel needs about the batch.
 struct BatchView {
@@ -109,18 +110,34 @@ struct SimtWork {
     int64_t sum_ng = 0;
     int32_t max_ng = 0;
 };
+// One projection of a SIMT launch.  A launch takes up to kMaxGroup of them over
+// the same plan (launch arguments `inl` only with one job).
+struct ShrinkJob {
+    const uint16_t* x;
+    int64_t ldx;
+    int32_t d_in;
+    int32_t proj;
+    float* v;
+    int64_t ldv;
+};
+struct ExpandJob {
+    const float* v;
+    int64_t ldv;
+    int32_t d_out;
+    int32_t proj;
+    void* y;
+    int64_t ldy;
+};
 // `inl` (may be null) holds the items as launch arguments when they fit.
-cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, const BatchView& b,
-                               int32_t num_items, int32_t max_item_rows, int32_t max_rank, const SimtWork& work,
-                               const PoolView& pool, float* v, int64_t ldv, const InlineTable<kInlineItems>* inl,
-                               cudaStream_t stream);
+cudaError_t launch_shrink_simt(const ShrinkJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,
+                               int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
+                               const InlineTable<kInlineItems>* inl, cudaStream_t stream);
 // y_early: y may be read before the preceding kernel completes (that kernel is
 // the shrink of the same call, which does not write y).
-cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const BatchView& b,
-                               int32_t num_items, int32_t max_item_rows, int32_t max_rank, const SimtWork& work,
-                               const PoolView& pool,
-                               float scale, void* y, int64_t ldy, int32_t y_dtype,
-                               const InlineTable<kInlineItems>* inl, bool y_early, cudaStream_t stream);
+cudaError_t launch_expand_simt(const ExpandJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,
+                               int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
+                               float scale, int32_t y_dtype, const InlineTable<kInlineItems>* inl, bool y_early,
+                               cudaStream_t stream);
 cudaError_t launch_shrink_tc(const uint16_t* x, int64_t ldx, int32_t d_in, const BatchView& b, int32_t num_tiles,
                              int32_t max_rank, const PoolView& pool, float* v, int64_t ldv, cudaStream_t stream);
 cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const BatchView& b, int32_t num_tiles,

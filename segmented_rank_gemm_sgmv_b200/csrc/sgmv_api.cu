@@ -120,9 +120,8 @@ sgmv_status shrink_impl(const void* x, int64_t ldx, int32_t T, int32_t d_in, int
 sgmv_status expand_impl(const float* v, int64_t ldv, int32_t T, int32_t d_out, int32_t proj, const sgmv_plan* plan,
                         const void* table, const sgmv_pool* pool, float scale, void* y, int64_t ldy, int32_t y_dtype,
                         bool y_early, cudaStream_t stream);
-sgmv_status delta_impl(const void* x, int64_t ldx, int32_t T, int32_t d_in, int32_t d_out, int32_t proj,
-                       const sgmv_plan* plan, const void* table, const sgmv_pool* pool, float scale, void* y,
-                       int64_t ldy, int32_t y_dtype, float* v, int64_t ldv, cudaStream_t stream);
+sgmv_status delta_impl(const sgmv_delta_entry* entries, int32_t n, int32_t T, const sgmv_plan* plan,
+                       const void* table, const sgmv_pool* pool, float scale, int32_t y_dtype, cudaStream_t stream);
 
 }  // namespace sgmv
 
@@ -213,8 +212,9 @@ sgmv_status sgmv::shrink_impl(const void* x, int64_t ldx, int32_t T, int32_t d_i
     const uint16_t* xb = static_cast<const uint16_t*>(x);
     InlineTable<kInlineItems> inl;
     const bool use_inl = inline_items(plan, proj, &inl);
-    SGMV_CUDA_TRY(launch_shrink_simt(xb, ldx, d_in, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank,
-                                     simt_work(plan), pv, v, ldv, use_inl ? &inl : nullptr, stream));
+    const ShrinkJob job{xb, ldx, d_in, proj, v, ldv};
+    SGMV_CUDA_TRY(launch_shrink_simt(&job, 1, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank,
+                                     simt_work(plan), pv, use_inl ? &inl : nullptr, stream));
     SGMV_CUDA_TRY(launch_shrink_tc(xb, ldx, d_in, bv, plan->num_tc_tiles, plan->max_rank, pv, v, ldv, stream));
     return SGMV_OK;
 }
@@ -229,40 +229,73 @@ sgmv_status sgmv::expand_impl(const float* v, int64_t ldv, int32_t T, int32_t d_
     if (st != SGMV_OK || nothing) return st;
     InlineTable<kInlineItems> inl;
     const bool use_inl = inline_items(plan, proj, &inl);
-    SGMV_CUDA_TRY(launch_expand_simt(v, ldv, d_out, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank,
-                                     simt_work(plan), pv, scale, y, ldy, y_dtype, use_inl ? &inl : nullptr, y_early,
-                                     stream));
+    const ExpandJob job{v, ldv, d_out, proj, y, ldy};
+    SGMV_CUDA_TRY(launch_expand_simt(&job, 1, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank,
+                                     simt_work(plan), pv, scale, y_dtype, use_inl ? &inl : nullptr, y_early, stream));
     SGMV_CUDA_TRY(launch_expand_tc(v, ldv, d_out, bv, plan->num_tc_tiles, plan->max_rank, pv, scale, y, ldy, y_dtype,
                                    stream));
     return SGMV_OK;
 }
 
-// Both phases in one call, arguments checked before anything is launched: the
-// SIMT shrink, the tensor-core shrink, then the SIMT expand as a programmatic
-// dependent launch (its adapter pages and y rows stream in while the shrinks
-// run) and the tensor-core expand.
-sgmv_status sgmv::delta_impl(const void* x, int64_t ldx, int32_t T, int32_t d_in, int32_t d_out, int32_t proj,
-                             const sgmv_plan* plan, const void* table, const sgmv_pool* pool, float scale, void* y,
-                             int64_t ldy, int32_t y_dtype, float* v, int64_t ldv, cudaStream_t stream) {
+// Both phases of every entry (projections over one plan), arguments checked
+// before anything is launched: the SIMT shrink of all entries, the tensor-core
+// shrinks, then the SIMT expand of all entries as a programmatic dependent
+// launch (its adapter pages and y rows stream in while the shrinks run) and the
+// tensor-core expands.  Launch-argument work lists carry one projection, so a
+// group over a plan without a device table runs entry by entry.
+sgmv_status sgmv::delta_impl(const sgmv_delta_entry* entries, int32_t n, int32_t T, const sgmv_plan* plan,
+                             const void* table, const sgmv_pool* pool, float scale, int32_t y_dtype,
+                             cudaStream_t stream) {
+    if (!entries || n < 1 || n > kMaxGroup)
+        return fail(SGMV_ERR_INVALID, "lora_delta: 1 to " + std::to_string(kMaxGroup) + " entries are required");
     BatchView bv;
     PoolView pv;
     bool nothing = false;
-    sgmv_status st = check_shrink(x, ldx, T, d_in, proj, plan, table, pool, v, ldv, &bv, &pv, &nothing);
-    if (st != SGMV_OK || nothing) return st;
-    st = check_expand(v, ldv, T, d_out, proj, plan, table, pool, y, ldy, y_dtype, &bv, &pv, &nothing);
-    if (st != SGMV_OK || nothing) return st;
-    const uint16_t* xb = static_cast<const uint16_t*>(x);
+    for (int32_t i = 0; i < n; ++i) {
+        const sgmv_delta_entry& e = entries[i];
+        if (plan && plan->num_rows > 0 && (plan->num_simt_items > 0 || plan->num_tc_tiles > 0) && !e.v)
+            return fail(SGMV_ERR_INVALID, "lora_delta: the workspace v is required");
+        for (int32_t k = 0; k < i; ++k)
+            if (entries[k].v == e.v && e.v)
+                return fail(SGMV_ERR_INVALID, "lora_delta: the entries of a group need distinct workspaces v");
+        sgmv_status st = check_shrink(e.x, e.ldx, T, e.d_in, e.proj, plan, table, pool, e.v, e.ldv, &bv, &pv, &nothing);
+        if (st != SGMV_OK) return st;
+        st = check_expand(e.v, e.ldv, T, e.d_out, e.proj, plan, table, pool, e.y, e.ldy, y_dtype, &bv, &pv, &nothing);
+        if (st != SGMV_OK) return st;
+    }
+    if (nothing) return SGMV_OK;
     InlineTable<kInlineItems> inl;
-    const bool use_inl = inline_items(plan, proj, &inl);
-    SGMV_CUDA_TRY(launch_shrink_simt(xb, ldx, d_in, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank,
-                                     simt_work(plan), pv, v, ldv, use_inl ? &inl : nullptr, stream));
-    SGMV_CUDA_TRY(launch_shrink_tc(xb, ldx, d_in, bv, plan->num_tc_tiles, plan->max_rank, pv, v, ldv, stream));
-    // the expand's predecessor is this call's shrink, which does not write y: y may be read early
-    SGMV_CUDA_TRY(launch_expand_simt(v, ldv, d_out, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank,
-                                     simt_work(plan), pv, scale, y, ldy, y_dtype, use_inl ? &inl : nullptr, true,
-                                     stream));
-    SGMV_CUDA_TRY(launch_expand_tc(v, ldv, d_out, bv, plan->num_tc_tiles, plan->max_rank, pv, scale, y, ldy, y_dtype,
-                                   stream));
+    const bool use_inl = n == 1 && inline_items(plan, entries[0].proj, &inl);
+    if (n > 1 && !table && plan->num_simt_items > 0) {  // items only as launch arguments: one entry at a time
+        for (int32_t i = 0; i < n; ++i) {
+            const sgmv_status st = delta_impl(&entries[i], 1, T, plan, table, pool, scale, y_dtype, stream);
+            if (st != SGMV_OK) return st;
+        }
+        return SGMV_OK;
+    }
+    const SimtWork work = simt_work(plan);
+    ShrinkJob sj[kMaxGroup];
+    ExpandJob ej[kMaxGroup];
+    for (int32_t i = 0; i < n; ++i) {
+        const sgmv_delta_entry& e = entries[i];
+        sj[i] = ShrinkJob{static_cast<const uint16_t*>(e.x), e.ldx, e.d_in, e.proj, e.v, e.ldv};
+        ej[i] = ExpandJob{e.v, e.ldv, e.d_out, e.proj, e.y, e.ldy};
+    }
+    SGMV_CUDA_TRY(launch_shrink_simt(sj, n, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, work, pv,
+                                     use_inl ? &inl : nullptr, stream));
+    for (int32_t i = 0; i < n; ++i) {
+        bv.proj = entries[i].proj;
+        SGMV_CUDA_TRY(launch_shrink_tc(sj[i].x, sj[i].ldx, sj[i].d_in, bv, plan->num_tc_tiles, plan->max_rank, pv,
+                                       sj[i].v, sj[i].ldv, stream));
+    }
+    // the expand's predecessors are this call's shrinks, which do not write y: y may be read early
+    SGMV_CUDA_TRY(launch_expand_simt(ej, n, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, work, pv,
+                                     scale, y_dtype, use_inl ? &inl : nullptr, true, stream));
+    for (int32_t i = 0; i < n; ++i) {
+        bv.proj = entries[i].proj;
+        SGMV_CUDA_TRY(launch_expand_tc(ej[i].v, ej[i].ldv, ej[i].d_out, bv, plan->num_tc_tiles, plan->max_rank, pv,
+                                       scale, ej[i].y, ej[i].ldy, y_dtype, stream));
+    }
     return SGMV_OK;
 }
 
@@ -272,8 +305,14 @@ extern "C" sgmv_status sgmv_lora_delta(const void* x, int64_t ldx, int32_t T, in
                                        sgmv_stream_t stream) {
     if (plan && plan->num_rows > 0 && (plan->num_simt_items > 0 || plan->num_tc_tiles > 0) && !v)
         return fail(SGMV_ERR_INVALID, "lora_delta: the workspace v is required");
-    return delta_impl(x, ldx, T, d_in, d_out, proj, plan, table, pool, scale, y, ldy, y_dtype, v, ldv,
-                      reinterpret_cast<cudaStream_t>(stream));
+    const sgmv_delta_entry e{proj, d_in, d_out, 0, x, ldx, y, ldy, v, ldv};
+    return delta_impl(&e, 1, T, plan, table, pool, scale, y_dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" sgmv_status sgmv_lora_delta_grouped(const sgmv_delta_entry* entries, int32_t n_entries, int32_t T,
+                                               const sgmv_plan* plan, const void* table, const sgmv_pool* pool,
+                                               float scale, int32_t y_dtype, sgmv_stream_t stream) {
+    return delta_impl(entries, n_entries, T, plan, table, pool, scale, y_dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------

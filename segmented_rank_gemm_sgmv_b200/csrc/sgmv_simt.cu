@@ -29,6 +29,8 @@
 //          updates y with one rounding, pass by pass.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+#include <cstring>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -53,34 +55,54 @@ __host__ __device__ constexpr int shrink_stages() { return MAXG == 1 ? 4 : 3; }
 constexpr int kExpandStages = 3;
 constexpr int kStageElems = kRowGroup * kPass;
 
-struct ShrinkArgs {
+// One projection of a launch.  A launch covers up to kMaxGroup projections over
+// the same batch plan (sgmv_lora_delta_grouped); every projection gets the same
+// number of CTAs per item in the shrink, its own count in the expand.
+struct ShrinkEntry {
     const uint16_t* x;
     int64_t ldx;
-    int32_t d_in;
-    BatchView b;
-    PoolView pool;
     float* v;
     int64_t ldv;
-    int32_t cluster;     // C
+    int32_t d_in;
     int32_t kc;          // columns of d_in per CTA (multiple of the page size)
+    int32_t proj;
+    int32_t pad;
+};
+
+struct ShrinkArgs {
+    ShrinkEntry ent[kMaxGroup];
+    int32_t n_entries;
+    int32_t items;       // SIMT items of the plan (each entry's CTAs: items x cluster)
+    BatchView b;         // b.proj unused: every entry names its projection
+    PoolView pool;
+    int32_t cluster;     // C
     int32_t stages;
     int32_t max_rank;
     int32_t ring_offset; // byte offset of the stage ring in shared memory
 };
 
-struct ExpandArgs {
+struct ExpandEntry {
     const float* v;
     int64_t ldv;
+    void* y;
+    int64_t ldy;
     int32_t d_out;
+    int32_t npass;       // 1024-column passes per CTA
+    int32_t cpi;         // CTAs per item
+    int32_t cta_base;    // first CTA of this entry in the grid
+    int32_t proj;
+    int32_t pad[3];
+};
+
+struct ExpandArgs {
+    ExpandEntry ent[kMaxGroup];
+    int32_t n_entries;
+    int32_t items;
     BatchView b;
     PoolView pool;
     float scale;
-    void* y;
-    int64_t ldy;
     int32_t y_dtype;
     int32_t y_early;        // y may be read before the preceding kernel (the shrink) completes
-    int32_t ctas_per_item;  // CTAs covering d_out for one item
-    int32_t npass;          // 1024-column passes per CTA
     int32_t stages;
     int32_t max_rank;
     int32_t ring_offset;    // byte offset of the stage ring in shared memory
@@ -116,9 +138,10 @@ __device__ __forceinline__ void finish_tokens(const BatchView& b, ItemInfo& m) {
 }
 
 // Work item `idx` from the device table: one 32-byte record, then the token rows.
-__device__ __forceinline__ ItemInfo load_item(const BatchView& b, int idx, int max_rows, int max_rank, int matrix) {
+__device__ __forceinline__ ItemInfo load_item(const BatchView& b, int proj, int idx, int max_rows, int max_rank,
+                                              int matrix) {
     ItemInfo m;
-    const int4* rp = reinterpret_cast<const int4*>(b.simt_items + ((int64_t)idx * b.n_proj + b.proj));
+    const int4* rp = reinterpret_cast<const int4*>(b.simt_items + ((int64_t)idx * b.n_proj + proj));
     const int4 h = rp[0], t = rp[1];  // {seg, row_begin, row_end, rank}, {a_pt, b_pt}
     m.i0 = h.y;
     m.n = h.z - h.y;
@@ -361,14 +384,17 @@ __device__ void shrink_item(const ShrinkArgs& a, const ItemInfo& m, Pipe<kStages
 
 template <int MAXG, int NI>
 __global__ void __launch_bounds__(kThreads, 3)
-    shrink_simt_kernel(const ShrinkArgs a, const __grid_constant__ InlineTable<NI> inl) {
+    shrink_simt_kernel(const __grid_constant__ ShrinkArgs a, const __grid_constant__ InlineTable<NI> inl) {
     extern __shared__ __align__(128) uint8_t smem[];
     pdl_launch_dependents();  // the expand may start staging its B^T pages now
     const int C = a.cluster;
     // First cluster phase: every CTA has started.  Its wait, just before the
     // partial tiles are pushed, makes rank 0's shared memory a valid target.
     if (C > 1) cluster_arrive_relaxed();
-    const int item_idx = blockIdx.x / C;
+    const int per_entry = a.items * C;  // a multiple of C: no cluster straddles two entries
+    const int ei = (int)blockIdx.x / per_entry;
+    const ShrinkEntry& en = a.ent[ei];
+    const int item_idx = ((int)blockIdx.x - ei * per_entry) / C;
     const uint32_t q = cluster_ctarank();
     const int slot = kSimtMaxItemRows * a.max_rank;  // floats of one partial tile
     float* part = reinterpret_cast<float*>(smem);     // [C slots][slot]; slot 0 is this CTA's own
@@ -376,15 +402,15 @@ __global__ void __launch_bounds__(kThreads, 3)
     int32_t* pid = reinterpret_cast<int32_t*>(red + 4 * 64);
 
     const ItemInfo m = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 0)
-                              : load_item(a.b, item_idx, MAXG, a.max_rank, 0);
+                              : load_item(a.b, en.proj, item_idx, MAXG, a.max_rank, 0);
     if (!m.ok && threadIdx.x == 0) atomicOr(&g_err_simt, kErrRows);
     StageGeom sg;
     sg.NG = (m.r + kRowGroup - 1) / kRowGroup;
-    sg.span = a.kc;
-    sg.npass = (a.kc + kPass - 1) / kPass;
-    sg.col_base = (int)q * a.kc;
+    sg.span = en.kc;
+    sg.npass = (en.kc + kPass - 1) / kPass;
+    sg.col_base = (int)q * en.kc;
     sg.rank = m.r;
-    sg.pages_per_row = a.d_in >> a.pool.page_log2;
+    sg.pages_per_row = en.d_in >> a.pool.page_log2;
     sg.pt = m.pt;
     constexpr int kShrinkStages = shrink_stages<MAXG>();
     Pipe<kShrinkStages> pp;
@@ -393,10 +419,10 @@ __global__ void __launch_bounds__(kThreads, 3)
     XStage xs;
     xs.ring = pp.data + (size_t)kShrinkStages * kStageElems;
     xs.maxg = MAXG;
-    xs.any = a.x;
+    xs.any = en.x;
 #pragma unroll
     for (int j = 0; j < kSimtMaxItemRows; ++j)
-        xs.rows[j] = (j < MAXG && m.tok[j] >= 0) ? a.x + (int64_t)m.tok[j] * a.ldx + (int64_t)q * a.kc : nullptr;
+        xs.rows[j] = (j < MAXG && m.tok[j] >= 0) ? en.x + (int64_t)m.tok[j] * en.ldx + (int64_t)q * en.kc : nullptr;
     if (m.ok) load_page_ids(a.pool, sg, pid, &g_err_simt);
     __syncthreads();
 #pragma unroll 1
@@ -433,15 +459,15 @@ __global__ void __launch_bounds__(kThreads, 3)
             float s = 0.f;
             for (int qq = 0; qq < C; ++qq) s += part[(size_t)qq * slot + e];
             const int jrow = e / m.r, k = e - jrow * m.r;
-            a.v[(int64_t)(m.i0 + jrow) * a.ldv + k] = s;
+            en.v[(int64_t)(m.i0 + jrow) * en.ldv + k] = s;
         }
     }
 }
 
 // ------------------------------------------------------------------ expand
 template <int G>
-__device__ void expand_item(const ExpandArgs& a, const ItemInfo& m, Pipe<kExpandStages>& pp, const StageGeom& sg,
-                            float* vs) {
+__device__ void expand_item(const ExpandArgs& a, const ExpandEntry& en, const ItemInfo& m, Pipe<kExpandStages>& pp,
+                            const StageGeom& sg, float* vs) {
     const int tid = threadIdx.x, col = kVec * tid;
     int trow[G];
 #pragma unroll
@@ -456,10 +482,10 @@ __device__ void expand_item(const ExpandArgs& a, const ItemInfo& m, Pipe<kExpand
         for (int j = 0; j < G; ++j) {
             if (active && trow[j] >= 0) {
                 if (a.y_dtype == 0) {
-                    d0[j] = *reinterpret_cast<const float4*>(static_cast<const uint16_t*>(a.y) +
-                                                             (int64_t)trow[j] * a.ldy + jcol);
+                    d0[j] = *reinterpret_cast<const float4*>(static_cast<const uint16_t*>(en.y) +
+                                                             (int64_t)trow[j] * en.ldy + jcol);
                 } else {
-                    const float* yp = static_cast<const float*>(a.y) + (int64_t)trow[j] * a.ldy + jcol;
+                    const float* yp = static_cast<const float*>(en.y) + (int64_t)trow[j] * en.ldy + jcol;
                     d0[j] = *reinterpret_cast<const float4*>(yp);
                     d1[j] = *reinterpret_cast<const float4*>(yp + 4);
                 }
@@ -470,7 +496,7 @@ __device__ void expand_item(const ExpandArgs& a, const ItemInfo& m, Pipe<kExpand
     pdl_wait();  // v (and, unless y_early, y) are final once the preceding kernel has completed
     for (int e = tid; e < m.n * m.r; e += kThreads) {
         const int jrow = e / m.r, k = e - jrow * m.r;
-        vs[e] = a.v[(int64_t)(m.i0 + jrow) * a.ldv + k];
+        vs[e] = en.v[(int64_t)(m.i0 + jrow) * en.ldv + k];
     }
     // (the first pipe_acquire's barrier publishes vs)
     for (int s = 0; s < sg.npass; ++s) {
@@ -520,10 +546,10 @@ __device__ void expand_item(const ExpandArgs& a, const ItemInfo& m, Pipe<kExpand
                     w[e] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
                            ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
                 }
-                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.y) + (int64_t)trow[j] * a.ldy + jcol) =
+                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(en.y) + (int64_t)trow[j] * en.ldy + jcol) =
                     make_uint4(w[0], w[1], w[2], w[3]);
             } else {
-                float* yp = static_cast<float*>(a.y) + (int64_t)trow[j] * a.ldy + jcol;
+                float* yp = static_cast<float*>(en.y) + (int64_t)trow[j] * en.ldy + jcol;
                 float4 o0 = y0[j], o1 = y1[j];
                 o0.x = fmaf(a.scale, acc[j][0], o0.x); o0.y = fmaf(a.scale, acc[j][1], o0.y);
                 o0.z = fmaf(a.scale, acc[j][2], o0.z); o0.w = fmaf(a.scale, acc[j][3], o0.w);
@@ -543,22 +569,26 @@ __device__ void expand_item(const ExpandArgs& a, const ItemInfo& m, Pipe<kExpand
 
 template <int MAXG, int NI>
 __global__ void __launch_bounds__(kThreads, 3)
-    expand_simt_kernel(const ExpandArgs a, const __grid_constant__ InlineTable<NI> inl) {
+    expand_simt_kernel(const __grid_constant__ ExpandArgs a, const __grid_constant__ InlineTable<NI> inl) {
     extern __shared__ __align__(128) uint8_t smem_e[];
-    const int part_idx = blockIdx.x % a.ctas_per_item, item_idx = blockIdx.x / a.ctas_per_item;
+    int ei = 0;  // this CTA's entry: the last whose first CTA is at or before it
+    while (ei + 1 < a.n_entries && (int)blockIdx.x >= a.ent[ei + 1].cta_base) ++ei;
+    const ExpandEntry& en = a.ent[ei];
+    const int local = (int)blockIdx.x - en.cta_base;
+    const int part_idx = local % en.cpi, item_idx = local / en.cpi;
     float* vs = reinterpret_cast<float*>(smem_e);
     int32_t* pid = reinterpret_cast<int32_t*>(vs + kSimtMaxItemRows * a.max_rank);
 
     const ItemInfo m = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 1)
-                              : load_item(a.b, item_idx, MAXG, a.max_rank, 1);
-    const int j0 = part_idx * a.npass * kPass;
+                              : load_item(a.b, en.proj, item_idx, MAXG, a.max_rank, 1);
+    const int j0 = part_idx * en.npass * kPass;
     StageGeom sg;
     sg.NG = (m.r + kRowGroup - 1) / kRowGroup;
-    sg.span = min(a.npass * kPass, a.d_out - j0);
+    sg.span = min(en.npass * kPass, en.d_out - j0);
     sg.npass = (sg.span + kPass - 1) / kPass;
     sg.col_base = j0;
     sg.rank = m.r;
-    sg.pages_per_row = a.d_out >> a.pool.page_log2;
+    sg.pages_per_row = en.d_out >> a.pool.page_log2;
     sg.pt = m.pt;
     const bool work = m.ok && sg.span > 0;
     Pipe<kExpandStages> pp;
@@ -575,9 +605,9 @@ __global__ void __launch_bounds__(kThreads, 3)
         cp_async_wait<0>();
         return;
     }
-    if (MAXG == 1 || m.n == 1) expand_item<1>(a, m, pp, sg, vs);
-    else if (MAXG == 2 || m.n == 2) expand_item<(MAXG < 2 ? MAXG : 2)>(a, m, pp, sg, vs);
-    else expand_item<MAXG>(a, m, pp, sg, vs);
+    if (MAXG == 1 || m.n == 1) expand_item<1>(a, en, m, pp, sg, vs);
+    else if (MAXG == 2 || m.n == 2) expand_item<(MAXG < 2 ? MAXG : 2)>(a, en, m, pp, sg, vs);
+    else expand_item<MAXG>(a, en, m, pp, sg, vs);
     cp_async_wait<0>();
 }
 
@@ -657,33 +687,65 @@ auto pick(int max_item_rows, K1 k1, K2 k2, K4 k4) {
     return max_item_rows <= 1 ? k1 : max_item_rows <= 2 ? k2 : k4;
 }
 
-cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, const BatchView& b, int32_t num_items,
+// Modelled time of a grouped launch: entries j with cpi[j] CTAs per item, each
+// doing npass[j] passes of its item's row groups; wp[j] = passes one row group
+// of an item is spread over in total.  One entry: split_time.  Several: the
+// entries' CTAs (largest first) pack into the slots, bounded by the largest.
+double group_time(const SimtWork& work, int64_t items, const int* cpi, const int* npass, const double* wp, int n,
+                  int64_t slots) {
+    if (n == 1) return split_time(work, items, cpi[0], npass[0], wp[0], slots);
+    constexpr double kPrologue = 2.0;
+    int max_np = 1;
+    double total = 0.0;
+    for (int j = 0; j < n; ++j) {
+        max_np = std::max(max_np, npass[j]);
+        total += (double)work.sum_ng * wp[j] + (double)items * cpi[j] * kPrologue;
+    }
+    const double biggest = (double)std::max(work.max_ng, 1) * max_np + kPrologue;
+    return std::max(biggest, total / (double)std::max<int64_t>(slots, 1));
+}
+
+cudaError_t launch_shrink_simt(const ShrinkJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,
                                int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
-                               float* v, int64_t ldv, const InlineTable<kInlineItems>* inl, cudaStream_t stream) {
-    if (num_items <= 0) return cudaSuccess;
+                               const InlineTable<kInlineItems>* inl, cudaStream_t stream) {
+    if (num_items <= 0 || n_jobs <= 0) return cudaSuccess;
+    if (n_jobs > kMaxGroup || (inl && n_jobs > 1)) return cudaErrorInvalidValue;
+    // entries with the most columns first: their CTAs are scheduled first
+    int order[kMaxGroup];
+    for (int j = 0; j < n_jobs; ++j) order[j] = j;
+    std::stable_sort(order, order + n_jobs, [&](int u, int w) { return jobs[u].d_in > jobs[w].d_in; });
     auto kern_inl = pick(max_item_rows, shrink_simt_kernel<1, kInlineItems>, shrink_simt_kernel<2, kInlineItems>,
                          shrink_simt_kernel<4, kInlineItems>);
     auto kern_tab = pick(max_item_rows, shrink_simt_kernel<1, 1>, shrink_simt_kernel<2, 1>, shrink_simt_kernel<4, 1>);
+    const void* kp = inl ? reinterpret_cast<const void*>(kern_inl) : reinterpret_cast<const void*>(kern_tab);
     const int mr = std::max(8, max_rank);
-    const size_t pid_bytes_max = (size_t)mr * (d_in >> pool.page_log2) * 4;
+    int max_pages = 0;
+    for (int j = 0; j < n_jobs; ++j) max_pages = std::max(max_pages, jobs[j].d_in >> pool.page_log2);
     const int maxg = max_item_rows <= 1 ? 1 : max_item_rows <= 2 ? 2 : 4;
     const int stages = maxg == 1 ? shrink_stages<1>() : shrink_stages<4>();
     const size_t ring_bytes = (size_t)stages * (kStageElems + (size_t)maxg * kPass) * 2;  // A rows + x slices
     auto smem_for = [&](int c) {
         const size_t part_bytes = (size_t)c * kSimtMaxItemRows * mr * 4;
-        const size_t pidb = pid_bytes_max / c;
+        const size_t pidb = (size_t)mr * ((max_pages + c - 1) / c) * 4;
         return (((part_bytes + 1024 + pidb + 127) & ~(size_t)127)) + ring_bytes;
     };
-    // Cluster size C (chunks of >= 1024 columns, C <= 8, dividing the page count):
-    // the one with the shortest modelled time (split_time).
-    const int pages = d_in >> pool.page_log2;
-    const void* kp = inl ? reinterpret_cast<const void*>(kern_inl) : reinterpret_cast<const void*>(kern_tab);
+    // Cluster size C (chunks of >= 1024 columns, C <= 8, dividing every entry's page
+    // count): the one with the shortest modelled time.
     int C = 1;
     double best = 1e300;
     for (int c = 1; c <= 8; ++c) {
-        if (pages % c || (c > 1 && d_in / c < kPass)) continue;
-        const int npass = (d_in / c + kPass - 1) / kPass;
-        const double t = split_time(work, num_items, c, npass, (double)npass * c,
+        bool valid = true;
+        int cpi[kMaxGroup], np[kMaxGroup];
+        double wp[kMaxGroup];
+        for (int j = 0; j < n_jobs; ++j) {
+            const int d = jobs[j].d_in;
+            if (((d >> pool.page_log2) % c) || (c > 1 && d / c < kPass)) valid = false;
+            cpi[j] = c;
+            np[j] = (d / c + kPass - 1) / kPass;
+            wp[j] = (double)np[j] * c;
+        }
+        if (!valid) continue;
+        const double t = group_time(work, num_items, cpi, np, wp, n_jobs,
                                     (int64_t)resident_ctas(kp, smem_for(c)) * num_sms());
         if (t < best) {
             best = t;
@@ -691,21 +753,22 @@ cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, con
         }
     }
     ShrinkArgs a;
-    a.x = x;
-    a.ldx = ldx;
-    a.d_in = d_in;
+    std::memset(&a, 0, sizeof(a));
+    for (int i = 0; i < n_jobs; ++i) {
+        const ShrinkJob& j = jobs[order[i]];
+        a.ent[i] = ShrinkEntry{j.x, j.ldx, j.v, j.ldv, j.d_in, j.d_in / C, j.proj, 0};
+    }
+    a.n_entries = n_jobs;
+    a.items = num_items;
     a.b = b;
     a.pool = pool;
-    a.v = v;
-    a.ldv = ldv;
     a.cluster = C;
-    a.kc = d_in / C;
-    a.max_rank = std::max(8, max_rank);
+    a.max_rank = mr;
     a.stages = stages;
     const size_t smem = smem_for(C);
     a.ring_offset = (int)(smem - ring_bytes);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(C * num_items), 1, 1);
+    cfg.gridDim = dim3((unsigned)(n_jobs * C * num_items), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -726,53 +789,73 @@ cudaError_t launch_shrink_simt(const uint16_t* x, int64_t ldx, int32_t d_in, con
     return cudaLaunchKernelEx(&cfg, kern_tab, a, InlineTable<1>{});
 }
 
-cudaError_t launch_expand_simt(const float* v, int64_t ldv, int32_t d_out, const BatchView& b, int32_t num_items,
+cudaError_t launch_expand_simt(const ExpandJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,
                                int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
-                               float scale, void* y,
-                               int64_t ldy, int32_t y_dtype, const InlineTable<kInlineItems>* inl, bool y_early,
+                               float scale, int32_t y_dtype, const InlineTable<kInlineItems>* inl, bool y_early,
                                cudaStream_t stream) {
-    if (num_items <= 0) return cudaSuccess;
-    ExpandArgs a;
-    a.v = v;
-    a.ldv = ldv;
-    a.d_out = d_out;
-    a.b = b;
-    a.pool = pool;
-    a.scale = scale;
-    a.y = y;
-    a.ldy = ldy;
-    a.y_dtype = y_dtype;
-    a.y_early = y_early ? 1 : 0;
-    // CTAs per item k, each covering npass 1024-column passes: the largest k
-    // whose grid fits in one wave of resident CTAs.
+    if (num_items <= 0 || n_jobs <= 0) return cudaSuccess;
+    if (n_jobs > kMaxGroup || (inl && n_jobs > 1)) return cudaErrorInvalidValue;
+    // entries with the most column passes first
+    int order[kMaxGroup];
+    for (int j = 0; j < n_jobs; ++j) order[j] = j;
+    std::stable_sort(order, order + n_jobs, [&](int u, int w) { return jobs[u].d_out > jobs[w].d_out; });
     auto kern_inl = pick(max_item_rows, expand_simt_kernel<1, kInlineItems>, expand_simt_kernel<2, kInlineItems>,
                          expand_simt_kernel<4, kInlineItems>);
     auto kern_tab = pick(max_item_rows, expand_simt_kernel<1, 1>, expand_simt_kernel<2, 1>, expand_simt_kernel<4, 1>);
     const void* kp = inl ? reinterpret_cast<const void*>(kern_inl) : reinterpret_cast<const void*>(kern_tab);
-    a.max_rank = std::max(8, max_rank);
+    const int mr = std::max(8, max_rank);
     auto smem_for = [&](int npass) {
-        const size_t pid_bytes = (size_t)a.max_rank * ((npass * kPass) >> pool.page_log2) * 4;
-        return (((size_t)kSimtMaxItemRows * a.max_rank * 4 + pid_bytes + 127) & ~(size_t)127) +
+        const size_t pid_bytes = (size_t)mr * ((npass * kPass) >> pool.page_log2) * 4;
+        return (((size_t)kSimtMaxItemRows * mr * 4 + pid_bytes + 127) & ~(size_t)127) +
                (size_t)kExpandStages * kStageElems * 2;
     };
-    const int tiles = (d_out + kPass - 1) / kPass;
-    a.npass = tiles;
+    int tiles[kMaxGroup], max_tiles = 1;
+    for (int j = 0; j < n_jobs; ++j) {
+        tiles[j] = (jobs[order[j]].d_out + kPass - 1) / kPass;
+        max_tiles = std::max(max_tiles, tiles[j]);
+    }
+    // passes per CTA P (each entry takes min(P, its tiles)): the shortest modelled time
+    int best_p = max_tiles;
     double best = 1e300;
-    for (int k = tiles; k >= 1; --k) {
-        const int np = (tiles + k - 1) / k, cpi = (tiles + np - 1) / np;
-        const double t = split_time(work, num_items, cpi, np, (double)tiles,
-                                    (int64_t)resident_ctas(kp, smem_for(np)) * num_sms());
+    for (int P = 1; P <= max_tiles; ++P) {
+        int cpi[kMaxGroup], np[kMaxGroup], max_np = 1;
+        double wp[kMaxGroup];
+        for (int j = 0; j < n_jobs; ++j) {
+            np[j] = std::min(P, tiles[j]);
+            cpi[j] = (tiles[j] + np[j] - 1) / np[j];
+            wp[j] = (double)tiles[j];
+            max_np = std::max(max_np, np[j]);
+        }
+        const double t = group_time(work, num_items, cpi, np, wp, n_jobs,
+                                    (int64_t)resident_ctas(kp, smem_for(max_np)) * num_sms());
         if (t < best) {
             best = t;
-            a.npass = np;
+            best_p = P;
         }
     }
-    a.ctas_per_item = (tiles + a.npass - 1) / a.npass;
+    ExpandArgs a;
+    std::memset(&a, 0, sizeof(a));
+    int ctas = 0, max_np = 1;
+    for (int i = 0; i < n_jobs; ++i) {
+        const ExpandJob& j = jobs[order[i]];
+        const int np = std::min(best_p, tiles[i]), cpi = (tiles[i] + np - 1) / np;
+        a.ent[i] = ExpandEntry{j.v, j.ldv, j.y, j.ldy, j.d_out, np, cpi, ctas, j.proj, {0, 0, 0}};
+        ctas += cpi * num_items;
+        max_np = std::max(max_np, np);
+    }
+    a.n_entries = n_jobs;
+    a.items = num_items;
+    a.b = b;
+    a.pool = pool;
+    a.scale = scale;
+    a.y_dtype = y_dtype;
+    a.y_early = y_early ? 1 : 0;
+    a.max_rank = mr;
     a.stages = kExpandStages;
-    const size_t smem = smem_for(a.npass);
+    const size_t smem = smem_for(max_np);
     a.ring_offset = (int)(smem - (size_t)kExpandStages * kStageElems * 2);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(a.ctas_per_item * num_items), 1, 1);
+    cfg.gridDim = dim3((unsigned)ctas, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;

@@ -69,8 +69,9 @@ struct ShrinkEntry {
     int32_t pad;
 };
 
+template <int NE>  // entry capacity: 1 (one projection) or kMaxGroup
 struct ShrinkArgs {
-    ShrinkEntry ent[kMaxGroup];
+    ShrinkEntry ent[NE];
     int32_t n_entries;
     int32_t items;       // SIMT items of the plan (each entry's CTAs: items x cluster)
     BatchView b;         // b.proj unused: every entry names its projection
@@ -94,8 +95,9 @@ struct ExpandEntry {
     int32_t pad[3];
 };
 
+template <int NE>
 struct ExpandArgs {
-    ExpandEntry ent[kMaxGroup];
+    ExpandEntry ent[NE];
     int32_t n_entries;
     int32_t items;
     BatchView b;
@@ -348,7 +350,7 @@ __device__ void load_page_ids(const PoolView& pool, StageGeom& sg, int32_t* pid,
 
 // ------------------------------------------------------------------ shrink
 template <int G, int kStages>
-__device__ void shrink_item(const ShrinkArgs& a, const ItemInfo& m, Pipe<kStages>& pp, const StageGeom& sg,
+__device__ void shrink_item(const PoolView& pool, const ItemInfo& m, Pipe<kStages>& pp, const StageGeom& sg,
                             const XStage& xs, float* part, float* red) {
     const int tid = threadIdx.x, col = kVec * tid;
     for (int g = 0; g < sg.NG; ++g) {
@@ -372,7 +374,7 @@ __device__ void shrink_item(const ShrinkArgs& a, const ItemInfo& m, Pipe<kStages
                     for (int j = 0; j < G; ++j) p[kk * G + j] += dot8(af, xf[j]);
                 }
             }
-            pipe_release(a.pool, pp, sg, false, xs);
+            pipe_release(pool, pp, sg, false, xs);
         }
         const float sum = block_reduce<kRowGroup * G>(p, red);
         if (tid < kRowGroup * G) {
@@ -382,9 +384,9 @@ __device__ void shrink_item(const ShrinkArgs& a, const ItemInfo& m, Pipe<kStages
     }
 }
 
-template <int MAXG, int NI>
+template <int MAXG, int NI, int NE>
 __global__ void __launch_bounds__(kThreads, 3)
-    shrink_simt_kernel(const __grid_constant__ ShrinkArgs a, const __grid_constant__ InlineTable<NI> inl) {
+    shrink_simt_kernel(const __grid_constant__ ShrinkArgs<NE> a, const __grid_constant__ InlineTable<NI> inl) {
     extern __shared__ __align__(128) uint8_t smem[];
     pdl_launch_dependents();  // the expand may start staging its B^T pages now
     const int C = a.cluster;
@@ -392,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 3)
     // partial tiles are pushed, makes rank 0's shared memory a valid target.
     if (C > 1) cluster_arrive_relaxed();
     const int per_entry = a.items * C;  // a multiple of C: no cluster straddles two entries
-    const int ei = (int)blockIdx.x / per_entry;
+    const int ei = NE == 1 ? 0 : (int)blockIdx.x / per_entry;
     const ShrinkEntry& en = a.ent[ei];
     const int item_idx = ((int)blockIdx.x - ei * per_entry) / C;
     const uint32_t q = cluster_ctarank();
@@ -428,9 +430,9 @@ __global__ void __launch_bounds__(kThreads, 3)
 #pragma unroll 1
     for (int i = 0; i < kShrinkStages; ++i) pipe_issue(a.pool, pp, sg, false, xs);
     if (m.ok) {  // MAXG bounds the token group, and with it the registers of the launch
-        if (MAXG == 1 || m.n == 1) shrink_item<1, kShrinkStages>(a, m, pp, sg, xs, part, red);
-        else if (MAXG == 2 || m.n == 2) shrink_item<(MAXG < 2 ? MAXG : 2), kShrinkStages>(a, m, pp, sg, xs, part, red);
-        else shrink_item<MAXG, kShrinkStages>(a, m, pp, sg, xs, part, red);
+        if (MAXG == 1 || m.n == 1) shrink_item<1, kShrinkStages>(a.pool, m, pp, sg, xs, part, red);
+        else if (MAXG == 2 || m.n == 2) shrink_item<(MAXG < 2 ? MAXG : 2), kShrinkStages>(a.pool, m, pp, sg, xs, part, red);
+        else shrink_item<MAXG, kShrinkStages>(a.pool, m, pp, sg, xs, part, red);
     }
     cp_async_wait<0>();
 
@@ -465,8 +467,8 @@ __global__ void __launch_bounds__(kThreads, 3)
 }
 
 // ------------------------------------------------------------------ expand
-template <int G>
-__device__ void expand_item(const ExpandArgs& a, const ExpandEntry& en, const ItemInfo& m, Pipe<kExpandStages>& pp,
+template <int G, int NE>
+__device__ void expand_item(const ExpandArgs<NE>& a, const ExpandEntry& en, const ItemInfo& m, Pipe<kExpandStages>& pp,
                             const StageGeom& sg, float* vs) {
     const int tid = threadIdx.x, col = kVec * tid;
     int trow[G];
@@ -567,12 +569,13 @@ __device__ void expand_item(const ExpandArgs& a, const ExpandEntry& en, const It
     }
 }
 
-template <int MAXG, int NI>
+template <int MAXG, int NI, int NE>
 __global__ void __launch_bounds__(kThreads, 3)
-    expand_simt_kernel(const __grid_constant__ ExpandArgs a, const __grid_constant__ InlineTable<NI> inl) {
+    expand_simt_kernel(const __grid_constant__ ExpandArgs<NE> a, const __grid_constant__ InlineTable<NI> inl) {
     extern __shared__ __align__(128) uint8_t smem_e[];
     int ei = 0;  // this CTA's entry: the last whose first CTA is at or before it
-    while (ei + 1 < a.n_entries && (int)blockIdx.x >= a.ent[ei + 1].cta_base) ++ei;
+    if (NE > 1)
+        while (ei + 1 < a.n_entries && (int)blockIdx.x >= a.ent[ei + 1].cta_base) ++ei;
     const ExpandEntry& en = a.ent[ei];
     const int local = (int)blockIdx.x - en.cta_base;
     const int part_idx = local % en.cpi, item_idx = local / en.cpi;
@@ -605,9 +608,9 @@ __global__ void __launch_bounds__(kThreads, 3)
         cp_async_wait<0>();
         return;
     }
-    if (MAXG == 1 || m.n == 1) expand_item<1>(a, en, m, pp, sg, vs);
-    else if (MAXG == 2 || m.n == 2) expand_item<(MAXG < 2 ? MAXG : 2)>(a, en, m, pp, sg, vs);
-    else expand_item<MAXG>(a, en, m, pp, sg, vs);
+    if (MAXG == 1 || m.n == 1) expand_item<1, NE>(a, en, m, pp, sg, vs);
+    else if (MAXG == 2 || m.n == 2) expand_item<(MAXG < 2 ? MAXG : 2), NE>(a, en, m, pp, sg, vs);
+    else expand_item<MAXG, NE>(a, en, m, pp, sg, vs);
     cp_async_wait<0>();
 }
 
@@ -705,18 +708,18 @@ double group_time(const SimtWork& work, int64_t items, const int* cpi, const int
     return std::max(biggest, total / (double)std::max<int64_t>(slots, 1));
 }
 
-cudaError_t launch_shrink_simt(const ShrinkJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,
-                               int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
-                               const InlineTable<kInlineItems>* inl, cudaStream_t stream) {
-    if (num_items <= 0 || n_jobs <= 0) return cudaSuccess;
-    if (n_jobs > kMaxGroup || (inl && n_jobs > 1)) return cudaErrorInvalidValue;
+template <int NE>
+cudaError_t shrink_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,
+                          int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
+                          const InlineTable<kInlineItems>* inl, cudaStream_t stream) {
     // entries with the most columns first: their CTAs are scheduled first
     int order[kMaxGroup];
     for (int j = 0; j < n_jobs; ++j) order[j] = j;
     std::stable_sort(order, order + n_jobs, [&](int u, int w) { return jobs[u].d_in > jobs[w].d_in; });
-    auto kern_inl = pick(max_item_rows, shrink_simt_kernel<1, kInlineItems>, shrink_simt_kernel<2, kInlineItems>,
-                         shrink_simt_kernel<4, kInlineItems>);
-    auto kern_tab = pick(max_item_rows, shrink_simt_kernel<1, 1>, shrink_simt_kernel<2, 1>, shrink_simt_kernel<4, 1>);
+    auto kern_inl = pick(max_item_rows, shrink_simt_kernel<1, kInlineItems, NE>, shrink_simt_kernel<2, kInlineItems, NE>,
+                         shrink_simt_kernel<4, kInlineItems, NE>);
+    auto kern_tab = pick(max_item_rows, shrink_simt_kernel<1, 1, NE>, shrink_simt_kernel<2, 1, NE>,
+                         shrink_simt_kernel<4, 1, NE>);
     const void* kp = inl ? reinterpret_cast<const void*>(kern_inl) : reinterpret_cast<const void*>(kern_tab);
     const int mr = std::max(8, max_rank);
     int max_pages = 0;
@@ -752,7 +755,7 @@ cudaError_t launch_shrink_simt(const ShrinkJob* jobs, int n_jobs, const BatchVie
             C = c;
         }
     }
-    ShrinkArgs a;
+    ShrinkArgs<NE> a;
     std::memset(&a, 0, sizeof(a));
     for (int i = 0; i < n_jobs; ++i) {
         const ShrinkJob& j = jobs[order[i]];
@@ -789,19 +792,19 @@ cudaError_t launch_shrink_simt(const ShrinkJob* jobs, int n_jobs, const BatchVie
     return cudaLaunchKernelEx(&cfg, kern_tab, a, InlineTable<1>{});
 }
 
-cudaError_t launch_expand_simt(const ExpandJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,
-                               int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
-                               float scale, int32_t y_dtype, const InlineTable<kInlineItems>* inl, bool y_early,
-                               cudaStream_t stream) {
-    if (num_items <= 0 || n_jobs <= 0) return cudaSuccess;
-    if (n_jobs > kMaxGroup || (inl && n_jobs > 1)) return cudaErrorInvalidValue;
+template <int NE>
+cudaError_t expand_launch(const ExpandJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,
+                          int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
+                          float scale, int32_t y_dtype, const InlineTable<kInlineItems>* inl, bool y_early,
+                          cudaStream_t stream) {
     // entries with the most column passes first
     int order[kMaxGroup];
     for (int j = 0; j < n_jobs; ++j) order[j] = j;
     std::stable_sort(order, order + n_jobs, [&](int u, int w) { return jobs[u].d_out > jobs[w].d_out; });
-    auto kern_inl = pick(max_item_rows, expand_simt_kernel<1, kInlineItems>, expand_simt_kernel<2, kInlineItems>,
-                         expand_simt_kernel<4, kInlineItems>);
-    auto kern_tab = pick(max_item_rows, expand_simt_kernel<1, 1>, expand_simt_kernel<2, 1>, expand_simt_kernel<4, 1>);
+    auto kern_inl = pick(max_item_rows, expand_simt_kernel<1, kInlineItems, NE>, expand_simt_kernel<2, kInlineItems, NE>,
+                         expand_simt_kernel<4, kInlineItems, NE>);
+    auto kern_tab = pick(max_item_rows, expand_simt_kernel<1, 1, NE>, expand_simt_kernel<2, 1, NE>,
+                         expand_simt_kernel<4, 1, NE>);
     const void* kp = inl ? reinterpret_cast<const void*>(kern_inl) : reinterpret_cast<const void*>(kern_tab);
     const int mr = std::max(8, max_rank);
     auto smem_for = [&](int npass) {
@@ -833,7 +836,7 @@ cudaError_t launch_expand_simt(const ExpandJob* jobs, int n_jobs, const BatchVie
             best_p = P;
         }
     }
-    ExpandArgs a;
+    ExpandArgs<NE> a;
     std::memset(&a, 0, sizeof(a));
     int ctas = 0, max_np = 1;
     for (int i = 0; i < n_jobs; ++i) {
@@ -872,6 +875,30 @@ cudaError_t launch_expand_simt(const ExpandJob* jobs, int n_jobs, const BatchVie
     cudaError_t e = set_smem(kern_tab, smem);
     if (e != cudaSuccess) return e;
     return cudaLaunchKernelEx(&cfg, kern_tab, a, InlineTable<1>{});
+}
+
+cudaError_t launch_shrink_simt(const ShrinkJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,
+                               int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
+                               const InlineTable<kInlineItems>* inl, cudaStream_t stream) {
+    if (num_items <= 0 || n_jobs <= 0) return cudaSuccess;
+    if (n_jobs > kMaxGroup || (inl && n_jobs > 1)) return cudaErrorInvalidValue;
+    // one projection: a one-entry table (small launch arguments, no per-CTA lookup)
+    if (n_jobs == 1)
+        return shrink_launch<1>(jobs, n_jobs, b, num_items, max_item_rows, max_rank, work, pool, inl, stream);
+    return shrink_launch<kMaxGroup>(jobs, n_jobs, b, num_items, max_item_rows, max_rank, work, pool, inl, stream);
+}
+
+cudaError_t launch_expand_simt(const ExpandJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,
+                               int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
+                               float scale, int32_t y_dtype, const InlineTable<kInlineItems>* inl, bool y_early,
+                               cudaStream_t stream) {
+    if (num_items <= 0 || n_jobs <= 0) return cudaSuccess;
+    if (n_jobs > kMaxGroup || (inl && n_jobs > 1)) return cudaErrorInvalidValue;
+    if (n_jobs == 1)
+        return expand_launch<1>(jobs, n_jobs, b, num_items, max_item_rows, max_rank, work, pool, scale, y_dtype, inl,
+                                y_early, stream);
+    return expand_launch<kMaxGroup>(jobs, n_jobs, b, num_items, max_item_rows, max_rank, work, pool, scale, y_dtype,
+                                    inl, y_early, stream);
 }
 
 cudaError_t read_clear_errors_simt(uint32_t* bits, cudaStream_t stream) {

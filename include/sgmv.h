@@ -211,6 +211,65 @@ typedef struct {
                                table when sgmv_shrink / sgmv_expand are called          */
 } sgmv_plan;
 
+/* ------------------------------------------------------------------------
+ * Residency manager: adapters kept in host memory and made resident in the
+ * pool on demand, batch by batch.  "Multi-LoRA serving: the single translator
+ * ...", the figure of section "SGMV: the kernel that holds it all up" (an HBM
+ * pool of hot adapters over a host-RAM cache: LRU eviction, asynchronous
+ * host-to-device copies on use) and "Operational pitfalls" (eviction: LRU by
+ * default); "Multi-LoRA Inference Serving ..." (clusterbid.com), the vLLM
+ * memory-pool paragraph (an adapter not resident is loaded from host memory
+ * into the pool, evicting a least-recently-used one).
+ *
+ * Use from one host thread with the pool (no other pool_load / pool_evict
+ * while a manager call runs).  Adapters loaded directly with sgmv_pool_load
+ * take part in the LRU order as the oldest.
+ */
+typedef struct sgmv_residency sgmv_residency;
+
+typedef struct {
+    int64_t hits;          /* batch adapters already resident                      */
+    int64_t misses;        /* batch adapters loaded from their host copies         */
+    int64_t evictions;     /* adapters evicted to make room                        */
+    int64_t bytes_loaded;  /* host -> device bytes of adapter matrices             */
+} sgmv_residency_stats;
+
+/* A manager over `pool` (not owned).  A device pool gets a device staging buffer
+ * of one largest adapter matrix and two events. */
+SGMV_API sgmv_status sgmv_residency_create(sgmv_pool* pool, sgmv_residency** out);
+/* Synchronises the pool's device, frees the manager (not the pool). */
+SGMV_API sgmv_status sgmv_residency_destroy(sgmv_residency* r);
+
+/* Host copies of an adapter: A[p] bf16 [rank][d_in_p], B[p] bf16 [d_out_p][rank]
+ * per projection (the layouts of sgmv_pool_load), owned by the caller and valid
+ * until unregistered.  Pinned (page-locked) memory lets the copies run
+ * asynchronously.  Re-registering replaces the pointers. */
+SGMV_API sgmv_status sgmv_residency_register(sgmv_residency* r, int32_t adapter_id, int32_t rank,
+                                             const void* const* A_host, const void* const* B_host);
+SGMV_API sgmv_status sgmv_residency_unregister(sgmv_residency* r, int32_t adapter_id);
+
+/*
+ * Make every adapter of a batch (adapter_ids: host int32[T], -1 = none)
+ * resident before the batch's kernels run:
+ *   - adapters already resident count as hits and become the most recently used;
+ *   - missing ones are loaded from their host copies: their page-table entries
+ *     and pages are written by copies and scatter kernels on `copy_stream`;
+ *   - when the free pages do not suffice, resident adapters that the batch does
+ *     not use are evicted, least recently used first (ties: lowest id);
+ *   - the copies that overwrite pages wait for the work already queued on
+ *     `compute_stream` (an event), and `compute_stream` waits for the copies
+ *     (another event): kernels enqueued on it afterwards see the adapters.
+ * Build the batch's plan after this call (the page-table bases may change).
+ * *loaded (optional) = adapters loaded.  Errors, with nothing changed:
+ * SGMV_ERR_NOT_RESIDENT (an adapter neither resident nor registered),
+ * SGMV_ERR_OUT_OF_PAGES (the batch's adapters do not fit even with every other
+ * adapter evicted).
+ */
+SGMV_API sgmv_status sgmv_residency_prepare(sgmv_residency* r, const int32_t* adapter_ids, int32_t T,
+                                            sgmv_stream_t copy_stream, sgmv_stream_t compute_stream,
+                                            int32_t* loaded);
+SGMV_API sgmv_status sgmv_residency_get_stats(const sgmv_residency* r, sgmv_residency_stats* out);
+
 /* Bytes a table may need for a batch of T tokens over n_proj projections. */
 SGMV_API int64_t sgmv_plan_table_capacity(int32_t T, int32_t n_proj);
 

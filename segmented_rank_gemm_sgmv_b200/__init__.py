@@ -33,7 +33,9 @@ EXPORTED = ("sgmv_status_string", "sgmv_last_error", "sgmv_pool_create", "sgmv_p
             "sgmv_pool_evict", "sgmv_pool_get_stats", "sgmv_pool_adapter_rank", "sgmv_pool_adapter_pages",
             "sgmv_pool_shuffle_free_pages", "sgmv_pool_pages_device", "sgmv_plan_table_capacity",
             "sgmv_build_plan", "sgmv_shrink", "sgmv_expand", "sgmv_lora_delta", "sgmv_lora_delta_grouped",
-            "sgmv_lora_delta_noalloc", "sgmv_check_errors")
+            "sgmv_lora_delta_noalloc", "sgmv_check_errors", "sgmv_residency_create", "sgmv_residency_destroy",
+            "sgmv_residency_register", "sgmv_residency_unregister", "sgmv_residency_prepare",
+            "sgmv_residency_get_stats")
 
 
 class SgmvError(RuntimeError):
@@ -54,6 +56,11 @@ class DeltaEntry(ctypes.Structure):
     _fields_ = [("proj", ctypes.c_int32), ("d_in", ctypes.c_int32), ("d_out", ctypes.c_int32),
                 ("reserved", ctypes.c_int32), ("x", ctypes.c_void_p), ("ldx", ctypes.c_int64),
                 ("y", ctypes.c_void_p), ("ldy", ctypes.c_int64), ("v", ctypes.c_void_p), ("ldv", ctypes.c_int64)]
+
+
+class ResidencyStats(ctypes.Structure):
+    _fields_ = [("hits", ctypes.c_int64), ("misses", ctypes.c_int64), ("evictions", ctypes.c_int64),
+                ("bytes_loaded", ctypes.c_int64)]
 
 
 class PoolStats(ctypes.Structure):
@@ -99,6 +106,12 @@ def load_library() -> ctypes.CDLL:
         "sgmv_lora_delta_noalloc": (st, [vp, i64, i32, i32, i32, i32, ctypes.POINTER(Plan), vp, vp, f32, vp, i64,
                                          i32, vp]),
         "sgmv_check_errors": (st, [vp, ctypes.POINTER(ctypes.c_uint32)]),
+        "sgmv_residency_create": (st, [vp, ctypes.POINTER(vp)]),
+        "sgmv_residency_destroy": (st, [vp]),
+        "sgmv_residency_register": (st, [vp, i32, i32, vp, vp]),
+        "sgmv_residency_unregister": (st, [vp, i32]),
+        "sgmv_residency_prepare": (st, [vp, vp, i32, vp, vp, ctypes.POINTER(i32)]),
+        "sgmv_residency_get_stats": (st, [vp, ctypes.POINTER(ResidencyStats)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -368,6 +381,69 @@ class BatchPlan:
         ldv = ldv or max(4, (self.plan.max_rank + 3) // 4 * 4)
         return torch.empty(max(self.plan.num_rows, 1), ldv, dtype=torch.float32,
                            device=torch.device("cuda", self.pool.device))
+
+
+class Residency:
+    """Adapters kept in host memory, made resident in `pool` batch by batch with
+    least-recently-used eviction (see include/sgmv.h, "Residency manager")."""
+
+    def __init__(self, pool: AdapterPool):
+        self.pool = pool
+        h = ctypes.c_void_p()
+        _check(load_library().sgmv_residency_create(pool.handle, ctypes.byref(h)))
+        self.handle = h
+        self._host = {}  # adapter -> host tensors kept alive while registered
+
+    def close(self):
+        if getattr(self, "handle", None):
+            load_library().sgmv_residency_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def register(self, adapter_id: int, rank: int, A: Optional[Sequence[torch.Tensor]] = None,
+                 B: Optional[Sequence[torch.Tensor]] = None) -> None:
+        """A[p]: bf16 [rank, d_in_p], B[p]: bf16 [d_out_p, rank] on the host (pinned if possible);
+        None for a host-only pool."""
+        if A is None:
+            _check(load_library().sgmv_residency_register(self.handle, int(adapter_id), int(rank), None, None))
+            return
+        n = len(self.pool.projections)
+        keep = []
+        for p, (d_in, d_out) in enumerate(self.pool.projections):
+            a, b = A[p].contiguous(), B[p].contiguous()
+            assert not a.is_cuda and not b.is_cuda and a.dtype == torch.bfloat16 and b.dtype == torch.bfloat16
+            assert tuple(a.shape) == (rank, d_in) and tuple(b.shape) == (d_out, rank)
+            keep += [a, b]
+        a_ptrs = (ctypes.c_void_p * n)(*[keep[2 * p].data_ptr() for p in range(n)])
+        b_ptrs = (ctypes.c_void_p * n)(*[keep[2 * p + 1].data_ptr() for p in range(n)])
+        _check(load_library().sgmv_residency_register(self.handle, int(adapter_id), int(rank),
+                                                      ctypes.cast(a_ptrs, ctypes.c_void_p),
+                                                      ctypes.cast(b_ptrs, ctypes.c_void_p)))
+        self._host[int(adapter_id)] = keep
+
+    def unregister(self, adapter_id: int) -> None:
+        _check(load_library().sgmv_residency_unregister(self.handle, int(adapter_id)))
+        self._host.pop(int(adapter_id), None)
+
+    def prepare(self, adapter_ids, copy_stream=None, compute_stream=None) -> int:
+        """Make the batch's adapters resident (see sgmv_residency_prepare); returns how many were loaded."""
+        ids = np.ascontiguousarray(np.asarray(adapter_ids, dtype=np.int32))
+        loaded = ctypes.c_int32(0)
+        dev = self.pool.device >= 0
+        _check(load_library().sgmv_residency_prepare(
+            self.handle, ids.ctypes.data if ids.size else None, int(ids.size),
+            _stream(copy_stream) if dev else None, _stream(compute_stream) if dev else None, ctypes.byref(loaded)))
+        return int(loaded.value)
+
+    def stats(self) -> ResidencyStats:
+        s = ResidencyStats()
+        _check(load_library().sgmv_residency_get_stats(self.handle, ctypes.byref(s)))
+        return s
 
 
 def shrink(x: torch.Tensor, plan: BatchPlan, pool: AdapterPool, v: torch.Tensor, proj: int = 0,

@@ -115,6 +115,33 @@ void release(sgmv_pool* p, int32_t adapter_id) {
     p->adapters.erase(it);
 }
 
+// Host bookkeeping of a load: drop the adapter's old placement, take a
+// page-table range and pages from the free stack.  False (nothing changed
+// beyond the release) when the page table has no free range that long.
+bool place(sgmv_pool* p, int32_t adapter_id, int32_t rank, AdapterRec* rec) {
+    const int64_t need = adapter_pages(p, rank);
+    release(p, adapter_id);
+    int64_t start = 0;
+    if (!pt_alloc(p, need, &start)) return false;
+    rec->rank = rank;
+    rec->pt_begin = start;
+    rec->pt_count = need;
+    rec->a_pt.resize(p->n_proj);
+    rec->b_pt.resize(p->n_proj);
+    int64_t e = start;
+    for (int i = 0; i < p->n_proj; ++i) {
+        rec->a_pt[i] = e;
+        e += (int64_t)rank * (p->d_in[i] >> p->page_log2);
+        rec->b_pt[i] = e;
+        e += (int64_t)rank * (p->d_out[i] >> p->page_log2);
+    }
+    for (int64_t k = start; k < start + need; ++k) {
+        p->pt_host[k] = (int32_t)p->free_pages.back();
+        p->free_pages.pop_back();
+    }
+    return true;
+}
+
 }  // namespace
 }  // namespace sgmv
 
@@ -194,27 +221,9 @@ extern "C" sgmv_status sgmv_pool_load(sgmv_pool* p, int32_t adapter_id, int32_t 
     auto old = p->adapters.find(adapter_id);
     if (old != p->adapters.end()) have += old->second.pt_count;
     if (need > have) return fail(SGMV_ERR_OUT_OF_PAGES, "pool_load: not enough free pages");
-    release(p, adapter_id);
-    int64_t start = 0;
-    if (!pt_alloc(p, need, &start)) return fail(SGMV_ERR_OUT_OF_PAGES, "pool_load: page table is fragmented");
-
     AdapterRec rec;
-    rec.rank = rank;
-    rec.pt_begin = start;
-    rec.pt_count = need;
-    rec.a_pt.resize(p->n_proj);
-    rec.b_pt.resize(p->n_proj);
-    int64_t e = start;
-    for (int i = 0; i < p->n_proj; ++i) {
-        rec.a_pt[i] = e;
-        e += (int64_t)rank * (p->d_in[i] >> p->page_log2);
-        rec.b_pt[i] = e;
-        e += (int64_t)rank * (p->d_out[i] >> p->page_log2);
-    }
-    for (int64_t k = start; k < start + need; ++k) {
-        p->pt_host[k] = (int32_t)p->free_pages.back();
-        p->free_pages.pop_back();
-    }
+    if (!place(p, adapter_id, rank, &rec)) return fail(SGMV_ERR_OUT_OF_PAGES, "pool_load: page table is fragmented");
+    const int64_t start = rec.pt_begin;
 
     if (p->device >= 0 && need > 0) {
         SGMV_CUDA_TRY(cudaSetDevice(p->device));
@@ -308,5 +317,203 @@ extern "C" sgmv_status sgmv_pool_shuffle_free_pages(sgmv_pool* p, uint64_t seed)
         const size_t j = (size_t)((z * 0x2545F4914F6CDD1Dull) % i);
         std::swap(p->free_pages[i - 1], p->free_pages[j]);
     }
+    return SGMV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Residency manager: adapters registered with host copies are made resident on
+// demand, batch by batch, least-recently-used adapters giving way.
+
+struct sgmv_residency {
+    sgmv_pool* pool = nullptr;
+    struct Host {
+        int32_t rank = 0;
+        std::vector<const void*> A, B;
+    };
+    std::unordered_map<int32_t, Host> host;       // registered host copies
+    std::unordered_map<int32_t, uint64_t> used;   // resident adapter -> batch tick of its last use
+    uint64_t tick = 0;
+    void* staging = nullptr;                      // device staging for host -> device copies
+    size_t staging_bytes = 0;
+    cudaEvent_t before = nullptr, after = nullptr;
+    sgmv_residency_stats stats{};
+};
+
+namespace {
+
+// Largest matrix of one adapter of rank `rank` (bytes).
+size_t largest_matrix(const sgmv_pool* p, int32_t rank) {
+    size_t m = 0;
+    for (int i = 0; i < p->n_proj; ++i) m = std::max(m, (size_t)rank * std::max(p->d_in[i], p->d_out[i]) * 2);
+    return m;
+}
+
+}  // namespace
+
+extern "C" sgmv_status sgmv_residency_create(sgmv_pool* pool, sgmv_residency** out) {
+    if (!pool || !out) return fail(SGMV_ERR_INVALID, "residency_create: NULL argument");
+    auto* r = new sgmv_residency();
+    r->pool = pool;
+    if (pool->device >= 0) {
+        SGMV_CUDA_TRY(cudaSetDevice(pool->device));
+        r->staging_bytes = std::max<size_t>(largest_matrix(pool, pool->max_rank), 16);
+        cudaError_t e = cudaMalloc(&r->staging, r->staging_bytes);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r->before, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r->after, cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            if (r->staging) cudaFree(r->staging);
+            if (r->before) cudaEventDestroy(r->before);
+            delete r;
+            return cuda_fail(e, "residency_create");
+        }
+    }
+    // adapters already resident take part in the LRU order as the oldest
+    for (const auto& kv : pool->adapters) r->used[kv.first] = 0;
+    *out = r;
+    return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_residency_destroy(sgmv_residency* r) {
+    if (!r) return SGMV_OK;
+    if (r->pool && r->pool->device >= 0) {
+        cudaSetDevice(r->pool->device);
+        cudaDeviceSynchronize();  // copies in flight read the staging buffer
+        if (r->staging) cudaFree(r->staging);
+        if (r->before) cudaEventDestroy(r->before);
+        if (r->after) cudaEventDestroy(r->after);
+    }
+    delete r;
+    return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_residency_register(sgmv_residency* r, int32_t adapter_id, int32_t rank,
+                                               const void* const* A_host, const void* const* B_host) {
+    if (!r) return fail(SGMV_ERR_INVALID, "residency_register: NULL manager");
+    if (adapter_id < 0) return fail(SGMV_ERR_INVALID, "residency_register: adapter_id must be >= 0");
+    sgmv_pool* p = r->pool;
+    if (rank < 0 || rank > p->max_rank) return fail(SGMV_ERR_INVALID, "residency_register: rank outside [0, max_rank]");
+    sgmv_residency::Host h;
+    h.rank = rank;
+    if (p->device >= 0 && rank > 0) {
+        if (!A_host || !B_host) return fail(SGMV_ERR_INVALID, "residency_register: A and B pointer arrays required");
+        for (int i = 0; i < p->n_proj; ++i) {
+            if (!A_host[i] || !B_host[i]) return fail(SGMV_ERR_INVALID, "residency_register: a matrix pointer is NULL");
+            h.A.push_back(A_host[i]);
+            h.B.push_back(B_host[i]);
+        }
+    }
+    r->host[adapter_id] = std::move(h);
+    return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_residency_unregister(sgmv_residency* r, int32_t adapter_id) {
+    if (!r) return fail(SGMV_ERR_INVALID, "residency_unregister: NULL manager");
+    if (!r->host.erase(adapter_id)) return fail(SGMV_ERR_NOT_RESIDENT, "residency_unregister: not registered");
+    return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_residency_prepare(sgmv_residency* r, const int32_t* adapter_ids, int32_t T,
+                                              sgmv_stream_t copy_stream_, sgmv_stream_t compute_stream_,
+                                              int32_t* loaded) {
+    if (!r) return fail(SGMV_ERR_INVALID, "residency_prepare: NULL manager");
+    if (T < 0 || (T > 0 && !adapter_ids)) return fail(SGMV_ERR_INVALID, "residency_prepare: bad batch");
+    sgmv_pool* p = r->pool;
+    cudaStream_t copy_stream = reinterpret_cast<cudaStream_t>(copy_stream_);
+    cudaStream_t compute_stream = reinterpret_cast<cudaStream_t>(compute_stream_);
+    const uint64_t tick = ++r->tick;
+    // the batch's distinct adapters; check all of them before changing anything
+    std::vector<int32_t> ids;
+    for (int32_t t = 0; t < T; ++t)
+        if (adapter_ids[t] >= 0) ids.push_back(adapter_ids[t]);
+    std::sort(ids.begin(), ids.end());
+    ids.erase(std::unique(ids.begin(), ids.end()), ids.end());
+    std::vector<int32_t> missing;
+    int64_t need = 0;
+    for (int32_t a : ids) {
+        if (p->adapters.count(a)) continue;
+        auto h = r->host.find(a);
+        if (h == r->host.end())
+            return fail(SGMV_ERR_NOT_RESIDENT, "residency_prepare: adapter " + std::to_string(a) +
+                                                   " is neither resident nor registered");
+        missing.push_back(a);
+        need += adapter_pages(p, h->second.rank);
+    }
+    int64_t evictable = 0;  // pages of resident adapters the batch does not use
+    for (const auto& kv : p->adapters)
+        if (!std::binary_search(ids.begin(), ids.end(), kv.first)) evictable += kv.second.pt_count;
+    if (need > (int64_t)p->free_pages.size() + evictable)
+        return fail(SGMV_ERR_OUT_OF_PAGES, "residency_prepare: the batch's adapters do not fit in the pool");
+    r->stats.hits += (int64_t)(ids.size() - missing.size());
+    r->stats.misses += (int64_t)missing.size();
+    for (int32_t a : ids)
+        if (p->adapters.count(a)) r->used[a] = tick;
+
+    // evict least recently used adapters outside the batch until the misses fit
+    while (need > (int64_t)p->free_pages.size()) {
+        int32_t victim = -1;
+        uint64_t oldest = UINT64_MAX;
+        for (const auto& kv : p->adapters) {
+            if (std::binary_search(ids.begin(), ids.end(), kv.first)) continue;
+            auto u = r->used.find(kv.first);
+            const uint64_t t = u == r->used.end() ? 0 : u->second;
+            if (t < oldest || (t == oldest && kv.first < victim)) {
+                oldest = t;
+                victim = kv.first;
+            }
+        }
+        if (victim < 0) break;
+        release(p, victim);
+        r->used.erase(victim);
+        ++r->stats.evictions;
+    }
+
+    const bool dev = p->device >= 0;
+    if (dev && !missing.empty()) {
+        SGMV_CUDA_TRY(cudaSetDevice(p->device));
+        // pages and page-table entries given up by evicted adapters may still be read
+        // by work already queued on the compute stream: the copies that overwrite
+        // them wait for it
+        SGMV_CUDA_TRY(cudaEventRecord(r->before, compute_stream));
+        SGMV_CUDA_TRY(cudaStreamWaitEvent(copy_stream, r->before, 0));
+    }
+    for (int32_t a : missing) {
+        const sgmv_residency::Host& h = r->host.at(a);
+        AdapterRec rec;
+        if (!place(p, a, h.rank, &rec))
+            return fail(SGMV_ERR_OUT_OF_PAGES, "residency_prepare: page table is fragmented");
+        if (dev && rec.pt_count > 0) {
+            SGMV_CUDA_TRY(cudaMemcpyAsync(p->pt_dev + rec.pt_begin, p->pt_host.data() + rec.pt_begin,
+                                          (size_t)rec.pt_count * sizeof(int32_t), cudaMemcpyHostToDevice,
+                                          copy_stream));
+            uint16_t* pages = static_cast<uint16_t*>(p->pages_dev);
+            for (int i = 0; i < p->n_proj; ++i) {
+                for (int m = 0; m < 2; ++m) {
+                    const int64_t cols = m == 0 ? p->d_in[i] : p->d_out[i];
+                    const size_t bytes = (size_t)h.rank * cols * 2;
+                    // the staging buffer is reused in stream order: each copy follows the
+                    // previous scatter on the copy stream
+                    SGMV_CUDA_TRY(cudaMemcpyAsync(r->staging, m == 0 ? h.A[i] : h.B[i], bytes,
+                                                  cudaMemcpyHostToDevice, copy_stream));
+                    SGMV_CUDA_TRY(launch_pool_scatter(static_cast<const uint16_t*>(r->staging), h.rank, cols, m == 1,
+                                                      p->pt_dev, m == 0 ? rec.a_pt[i] : rec.b_pt[i], p->page_log2,
+                                                      pages, copy_stream));
+                    r->stats.bytes_loaded += (int64_t)bytes;
+                }
+            }
+        }
+        p->adapters[a] = std::move(rec);
+        r->used[a] = tick;
+    }
+    if (dev && !missing.empty()) {
+        SGMV_CUDA_TRY(cudaEventRecord(r->after, copy_stream));
+        SGMV_CUDA_TRY(cudaStreamWaitEvent(compute_stream, r->after, 0));
+    }
+    if (loaded) *loaded = (int32_t)missing.size();
+    return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_residency_get_stats(const sgmv_residency* r, sgmv_residency_stats* out) {
+    if (!r || !out) return fail(SGMV_ERR_INVALID, "residency_get_stats: NULL argument");
+    *out = r->stats;
     return SGMV_OK;
 }

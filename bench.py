@@ -196,38 +196,44 @@ def run_ours(args, rank, world, device):
     gate_cycles = int(2e-4 * 2.0e9)
     split = args.split_phases
 
-    def step(i, evs=None):
+    # Events per step: `start` before the table upload, `mid` after it (only when a
+    # copy happens: with no copy, start doubles as mid), `end` after the kernels.
+    # Every event recorded between kernels adds device time, so the normal run
+    # records no others; --split-phases adds one around each projection's phases.
+    def step(i, ev=None):
         pl = plans[i % 2]
         pl.build(wl.adapter_ids)                     # host segment builder + dispatch
-        if evs:
-            evs[0].record(stream)
-        pl.upload(stream)                            # one host->device copy of the table
+        if ev:
+            ev["start"].record(stream)
+        copied = pl.upload(stream) is not None       # one host->device copy of the table (large plans)
+        if ev:
+            ev["copied"] = copied
+            if copied:
+                ev["mid"].record(stream)
         if grouped:                                  # every projection in one call
-            if evs:
-                evs[1].record(stream)
             sg.lora_delta_grouped([(acts[p][0], acts[p][1], p, vs[p]) for p in range(n_proj)], pl, pool,
                                   wl.scale, stream)
-            if evs:
-                evs[3].record(stream)
-                evs[-1].record(stream)
-            return
-        for p in range(n_proj):
-            x, y = acts[p]
-            if evs:
-                evs[1 + 3 * p].record(stream)
-            if split:                                # an event between the phases (no launch overlap)
-                sg.shrink(x, pl, pool, v, p, stream)
-                if evs:
-                    evs[2 + 3 * p].record(stream)
-                sg.expand(v, pl, pool, y, p, wl.scale, stream)
-            else:                                    # shrink, then expand overlapping it (PDL)
-                sg.lora_delta(x, pl, pool, y, p, wl.scale, v=v, stream=stream)
-            if evs:
-                evs[3 + 3 * p].record(stream)
-        if evs:
-            evs[-1].record(stream)
+        else:
+            for p in range(n_proj):
+                x, y = acts[p]
+                if split:                            # events around and between the phases (no overlap)
+                    ev and ev["ph"][p][0].record(stream)
+                    sg.shrink(x, pl, pool, v, p, stream)
+                    ev and ev["ph"][p][1].record(stream)
+                    sg.expand(v, pl, pool, y, p, wl.scale, stream)
+                    ev and ev["ph"][p][2].record(stream)
+                else:                                # shrink, then expand overlapping it (PDL)
+                    sg.lora_delta(x, pl, pool, y, p, wl.scale, v=v, stream=stream)
+        if ev:
+            ev["end"].record(stream)
 
-    n_ev = 2 + 3 * n_proj
+    def new_events():
+        mk = lambda: torch.cuda.Event(enable_timing=True)
+        ev = {"start": mk(), "mid": mk(), "end": mk()}
+        if split:
+            ev["ph"] = [[mk(), mk(), mk()] for _ in range(n_proj)]
+        return ev
+
     for i in range(args.warmup):
         flush.zero_()
         step(i)
@@ -240,17 +246,17 @@ def run_ours(args, rank, world, device):
         for i in range(args.steps):
             flush.zero_()                            # L2 flush, outside the timed window
             torch.cuda._sleep(gate_cycles)
-            evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-            step(i, evs)
-            records.append(evs)
+            ev = new_events()
+            step(i, ev)
+            records.append(ev)
         torch.cuda.synchronize(device)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(device)
     sg.check_errors(stream)
-    step_ms = [e[0].elapsed_time(e[-1]) for e in records]
-    proj_ms = [sum(e[1 + 3 * p].elapsed_time(e[3 + 3 * p]) for p in range(1 if grouped else n_proj))
-               for e in records]
+    step_ms = [e["start"].elapsed_time(e["end"]) for e in records]
+    # the kernels' time (roofline): after the table copy when there is one
+    proj_ms = [(e["mid"] if e["copied"] else e["start"]).elapsed_time(e["end"]) for e in records]
     total_ms = reduce_max(float(sum(step_ms)), f"cuda:{device}")
 
     shrink_b = expand_b = flops = 0
@@ -271,14 +277,13 @@ def run_ours(args, rank, world, device):
                clocks=clk.summary(), dom_launches=1 if grouped else n_proj,
                traffic=read_traffic(args.workload, "lora_delta_grouped" if grouped else "lora_delta"), split=split)
     if split:
+        ph = lambda e, p, k: e["ph"][p][k].elapsed_time(e["ph"][p][k + 1])
         res["phase_us_per_proj"] = {
-            name: [round(1e3 * float(np.mean([e[1 + 3 * p].elapsed_time(e[2 + 3 * p]) for e in records])), 2),
-                   round(1e3 * float(np.mean([e[2 + 3 * p].elapsed_time(e[3 + 3 * p]) for e in records])), 2)]
+            name: [round(1e3 * float(np.mean([ph(e, p, 0) for e in records])), 2),
+                   round(1e3 * float(np.mean([ph(e, p, 1) for e in records])), 2)]
             for p, (name, _, _) in enumerate(wl.projections)}
-        res["phase_ms"] = {"shrink": float(np.mean([sum(e[1 + 3 * p].elapsed_time(e[2 + 3 * p]) for p in range(n_proj))
-                                                    for e in records])),
-                           "expand": float(np.mean([sum(e[2 + 3 * p].elapsed_time(e[3 + 3 * p]) for p in range(n_proj))
-                                                    for e in records]))}
+        res["phase_ms"] = {"shrink": float(np.mean([sum(ph(e, p, 0) for p in range(n_proj)) for e in records])),
+                           "expand": float(np.mean([sum(ph(e, p, 1) for p in range(n_proj)) for e in records]))}
     res["achieved"] = res["step_bytes"] / (res["proj_ms"] * 1e-3) / 1e9
     res["e2e"] = e2e_ours(sg, wl, pool, acts, args, device, stream, world)
     return wl, res

@@ -51,9 +51,16 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def algorithmic_bytes(wl: workloads.Workload, proj: int):
+# bytes of one stored weight value, by pool weight format
+WEIGHT_BYTES = {"bf16": 2.0, "fp8_e4m3": 1.0, "int4": 0.5}
+
+
+def algorithmic_bytes(wl: workloads.Workload, proj: int, weights: str = "bf16"):
     """Minimum bytes of one shrink and one expand: each distinct adapter's A and B
-    once, x read once, v written and read in fp32, y read and written."""
+    once (codes plus one fp32 scale per rank row in a quantised pool), x read once,
+    v written and read in fp32, y read and written."""
+    wb = WEIGHT_BYTES[weights]
+    sb = 0 if weights == "bf16" else 4
     _, d_in, d_out = wl.projections[proj]
     ids = wl.adapter_ids[wl.adapter_ids >= 0]
     distinct = np.unique(ids)
@@ -61,8 +68,8 @@ def algorithmic_bytes(wl: workloads.Workload, proj: int):
     sum_r_adapters = sum(r_of.values())
     rows = [t for t in range(wl.T) if wl.adapter_ids[t] >= 0 and r_of[int(wl.adapter_ids[t])] > 0]
     sum_r_tokens = sum(r_of[int(wl.adapter_ids[t])] for t in rows)
-    shrink = 2 * sum_r_adapters * d_in + 2 * len(rows) * d_in + 4 * sum_r_tokens
-    expand = 2 * sum_r_adapters * d_out + 4 * sum_r_tokens + 4 * len(rows) * d_out
+    shrink = int(wb * sum_r_adapters * d_in) + sb * sum_r_adapters + 2 * len(rows) * d_in + 4 * sum_r_tokens
+    expand = int(wb * sum_r_adapters * d_out) + sb * sum_r_adapters + 4 * sum_r_tokens + 4 * len(rows) * d_out
     flops = 2 * sum_r_tokens * (d_in + d_out)
     return shrink, expand, flops, 4 * sum_r_tokens
 
@@ -161,14 +168,14 @@ def job_value(world: int, tokens_per_rank: int, steps: int, total_ms: float) -> 
 
 
 # ---------------------------------------------------------------------------- our arm
-def setup(wl_name: str, rank: int, device: int, pool_override: int = 0):
+def setup(wl_name: str, rank: int, device: int, pool_override: int = 0, weights: str = "bf16"):
     import segmented_rank_gemm_sgmv_b200 as sg
     wl = workloads.make(wl_name, seed=rank, **({"pool": pool_override} if pool_override else {}))
     bank = workloads.AdapterBank(wl, device=f"cuda:{device}")
     projs = [(d_in, d_out) for _, d_in, d_out in wl.projections]
     need = sum(sg.AdapterPool.pages_needed(projs, int(r)) for r in wl.pool_ranks)
     pool = sg.AdapterPool(projs, num_pages=need + 64, page_elems=512,
-                          max_rank=max(16, int(wl.pool_ranks.max())), device=device)
+                          max_rank=max(16, int(wl.pool_ranks.max())), device=device, weight_format=weights)
     pool.shuffle_free_pages(1234 + rank)
     for a, r in zip(wl.pool_ids.tolist(), wl.pool_ranks.tolist()):
         A, B = zip(*[bank.get(a, p) for p in range(len(projs))])
@@ -180,7 +187,7 @@ def setup(wl_name: str, rank: int, device: int, pool_override: int = 0):
 
 
 def run_ours(args, rank, world, device):
-    sg, wl, pool, acts = setup(args.workload, rank, device, args.pool)
+    sg, wl, pool, acts = setup(args.workload, rank, device, args.pool, args.weights)
     n_proj = len(wl.projections)
     stream = torch.cuda.current_stream(device)
     plans = [sg.BatchPlan(pool, capacity_tokens=wl.T) for _ in range(2)]
@@ -261,7 +268,7 @@ def run_ours(args, rank, world, device):
 
     shrink_b = expand_b = flops = 0
     for p in range(n_proj):
-        s_b, e_b, f, _ = algorithmic_bytes(wl, p)
+        s_b, e_b, f, _ = algorithmic_bytes(wl, p, args.weights)
         shrink_b += s_b
         expand_b += e_b
         flops += f
@@ -275,7 +282,8 @@ def run_ours(args, rank, world, device):
                step_bytes=shrink_b + expand_b, flops=flops, peak=peak, peak_kind=peak_kind,
                launches=(2 * simt + 2 * n_proj * tc) if grouped else 2 * n_proj * len(kinds),
                clocks=clk.summary(), dom_launches=1 if grouped else n_proj,
-               traffic=read_traffic(args.workload, "lora_delta_grouped" if grouped else "lora_delta"), split=split)
+               traffic=read_traffic(args.workload, ("lora_delta_grouped" if grouped else "lora_delta") +
+                                    ("" if args.weights == "bf16" else "@" + args.weights)), split=split)
     if split:
         ph = lambda e, p, k: e["ph"][p][k].elapsed_time(e["ph"][p][k + 1])
         res["phase_us_per_proj"] = {
@@ -351,16 +359,26 @@ def e2e_ours(sg, wl, pool, acts, args, device, stream, world):
 
 
 # ---------------------------------------------------------------------------- oracle arm
-def oracle_inputs(wl, device):
-    """fp64 host copies of the batch's inputs (x, y, A, B of the adapters in use)."""
+def oracle_inputs(wl, device, weights: str = "bf16"):
+    """fp64 host copies of the batch's inputs (x, y, A, B of the adapters in use; in a
+    quantised pool's format, the dequantised weights, quantised here outside any timing)."""
     bank = workloads.AdapterBank(wl, device=device)
     import oracle
+    from oracle import quant as oquant
     tix, off, seg_ad = oracle.group_by_adapter(wl.adapter_ids.tolist())
     per_proj = []
+
+    def weights_of(a, p):
+        A, B = (workloads.bf16_to_f64(m) for m in bank.get(a, p))
+        if weights == "bf16":
+            return A, B
+        return oquant.quantize_adapter(A.astype(np.float32), B.astype(np.float32), weights)[4:]
+
     for p in range(len(wl.projections)):
         x, y = workloads.activations(wl, p, device=device)
-        A = [workloads.bf16_to_f64(bank.get(a, p)[0]) for a in seg_ad]
-        B = [workloads.bf16_to_f64(bank.get(a, p)[1]) for a in seg_ad]
+        AB = [weights_of(a, p) for a in seg_ad]
+        A = [ab[0] for ab in AB]
+        B = [ab[1] for ab in AB]
         per_proj.append((workloads.bf16_to_f64(x), workloads.bf16_to_f64(y), A, B))
     ranks = [wl.rank_of(a) for a in seg_ad]
     del bank
@@ -390,7 +408,7 @@ def run_reference(args, rank, world, device):
     wl = workloads.make(args.workload, seed=0)
     threads = os.cpu_count() or 1
     dev = f"cuda:{device}" if torch.cuda.is_available() else "cpu"
-    prepared = oracle_inputs(wl, dev)
+    prepared = oracle_inputs(wl, dev, args.weights)
     for _ in range(args.warmup):
         time_oracle(prepared, wl, 0.0, threads)
     per_step_budget = max(0.05, getattr(args, "ref_budget", 60.0) / max(args.steps, 1))
@@ -404,7 +422,7 @@ def run_reference(args, rank, world, device):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_all / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": config_of(wl),
+            "data": "synthetic", "config": config_of(wl, args.weights),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
                              "sample": f"whole batch ({n_tok} tokens x {len(wl.projections)} projections) "
                                        f"repeated {reps_all} times over {args.steps} steps"},
@@ -412,12 +430,12 @@ def run_reference(args, rank, world, device):
     print(json.dumps(line), flush=True)
 
 
-def config_of(wl):
+def config_of(wl, weights: str = "bf16"):
     ranks = sorted(set(int(wl.rank_of(a)) for a in np.unique(wl.adapter_ids[wl.adapter_ids >= 0])))
     return {"workload": wl.name, "tokens": wl.T,
             "projections": [f"{n}:{a}->{b}" for n, a, b in wl.projections],
             "ranks": ranks, "pool_adapters": int(wl.pool_ids.size),
-            "distinct_adapters": wl.distinct_adapters, "page_elems": 512,
+            "distinct_adapters": wl.distinct_adapters, "page_elems": 512, "adapter_weights": weights,
             "l2": "flushed between steps (512 MiB write outside the timed window)",
             "parallelism": "replicas"}
 
@@ -439,6 +457,8 @@ def main():
                          "for all projections of a multi-projection workload (the default)")
     ap.add_argument("--split-phases", action="store_true",
                     help="record an event between shrink and expand (times each phase; removes their overlap)")
+    ap.add_argument("--weights", default="bf16", choices=sorted(WEIGHT_BYTES),
+                    help="adapter storage of the pool: bf16, or FP8 E4M3 / INT4 codes with a scale per rank row")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-budget", type=float, default=60.0,
                     help="seconds of oracle time over all steps of --impl reference")
@@ -473,7 +493,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["total_ms"] / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_of(wl),
+            "config": config_of(wl, args.weights),
             "hbm_gbs_step": res["step_bytes"] / (res["total_ms"] / args.steps * 1e-3) / 1e9,
             "roofline": {"bound": "hbm", "kernel": res["kernel_name"], "achieved": res["achieved"],
                          "peak": res["peak"], "unit": "GB/s", "frac": res["achieved"] / res["peak"],
@@ -491,7 +511,7 @@ def main():
             line["phase_ms"] = res["phase_ms"]
             line["phase_us_per_proj"] = res["phase_us_per_proj"]
         if not args.no_cpu_baseline and world == 1:
-            prepared = oracle_inputs(wl, f"cuda:{local}")
+            prepared = oracle_inputs(wl, f"cuda:{local}", args.weights)
             rate, reps, el, used = time_oracle(prepared, wl, args.cpu_budget, os.cpu_count() or 1)
             line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": used, "kind": "oracle",
                                     "sample": f"whole batch ({n_tok} tokens x {len(wl.projections)} projections)"

@@ -96,13 +96,46 @@ SGMV_API const char* sgmv_last_error(void);
  */
 typedef struct sgmv_pool sgmv_pool;
 
+/*
+ * Weight formats of a pool.  bf16 is the default and what the pool stores
+ * unless it is created with sgmv_pool_create_ex.  The two quantised formats
+ * follow [ClusterBid] (paragraph on the GPU memory budget: FP8 adapters halve
+ * the memory; paragraph on adapter weight quantization: INT4 adapters, with a
+ * dequantisation cost at inference).  [SGMV post] ("Combined pattern with
+ * quantisation and disaggregated serving") keeps adapters in BF16 in its
+ * canonical stack, which is why bf16 stays the default.
+ *
+ * Quantised layout.  A page still holds page_elems values of one rank row,
+ * now as codes: 1 byte each (FP8_E4M3) or 4 bits each (INT4, two's
+ * complement in [-7, 7], value 2i in the low nibble of byte i).  Each rank row
+ * k of A and of B^T has one fp32 scale s_k, kept beside the page table (entry
+ * of the row's first chunk), and its values are code(q) * s_k:
+ *     s_k  = max_c |w_kc| / Q    (Q = 448 for E4M3, 7 for INT4; fp32 division)
+ *     q_kc = RN(w_kc / s_k)      (fp32 division; E4M3: round to nearest even,
+ *                                 saturating; INT4: round half to even,
+ *                                 clamped to [-7, 7]); a row of zeros has s_k = 0.
+ * The load call quantises bf16 weights on the device by this rule.  Because
+ * the scale belongs to a whole rank row, it leaves both contractions
+ * exactly: v_k = s^A_k * sum_c q^A_kc x_c, and the expand multiplies v_k by
+ * s^B_k before using the codes of B^T.  The kernels therefore only convert
+ * codes (every E4M3 and INT4 value is exact in bf16 and fp32) and the delta
+ * equals the bf16 computation on the dequantised weights up to rounding.
+ */
+typedef enum {
+    SGMV_WEIGHTS_BF16 = 0,
+    SGMV_WEIGHTS_FP8_E4M3 = 1,
+    SGMV_WEIGHTS_INT4 = 2
+} sgmv_weight_format;
+
 typedef struct {
     int64_t num_pages;         /* pages in the pool                                 */
     int64_t free_pages;        /* pages not holding adapter data                    */
-    int64_t page_bytes;        /* page_elems * 2                                    */
+    int64_t page_bytes;        /* bytes of one page: page_elems * 2, 1 or 1/2       */
     int64_t payload_bytes;     /* (num_pages - free_pages) * page_bytes             */
     int32_t resident_adapters; /* adapters currently loaded                         */
     int32_t page_elems;
+    int32_t weight_format;     /* sgmv_weight_format                                */
+    int32_t reserved;
 } sgmv_pool_stats;
 
 /*
@@ -121,6 +154,15 @@ typedef struct {
 SGMV_API sgmv_status sgmv_pool_create(int device, int64_t num_pages, int32_t page_elems, int32_t n_proj,
                              const int32_t* d_in, const int32_t* d_out, int32_t max_rank,
                              sgmv_pool** out);
+/*
+ * sgmv_pool_create with a weight format (sgmv_weight_format).  A quantised
+ * pool allocates num_pages pages of page_elems codes (page_elems or
+ * page_elems / 2 bytes each) plus one fp32 scale per page-table entry, and
+ * needs page_elems >= 64 as before.  SGMV_ERR_INVALID for an unknown format.
+ */
+SGMV_API sgmv_status sgmv_pool_create_ex(int device, int64_t num_pages, int32_t page_elems, int32_t n_proj,
+                                const int32_t* d_in, const int32_t* d_out, int32_t max_rank,
+                                int32_t weight_format, sgmv_pool** out);
 SGMV_API sgmv_status sgmv_pool_destroy(sgmv_pool* pool);
 
 /*
@@ -130,7 +172,8 @@ SGMV_API sgmv_status sgmv_pool_destroy(sgmv_pool* pool);
  * arrays of n_proj pointers.  The pointed-to data is device memory when
  * src_on_device != 0, host memory otherwise.  The copies are enqueued on
  * `stream` and the call waits for them before returning, so the sources may be
- * freed afterwards.  SGMV_ERR_OUT_OF_PAGES leaves the pool unchanged.
+ * freed afterwards.  SGMV_ERR_OUT_OF_PAGES leaves the pool unchanged.  A
+ * quantised pool quantises the bf16 rows on the device as it stores them.
  */
 SGMV_API sgmv_status sgmv_pool_load(sgmv_pool* pool, int32_t adapter_id, int32_t rank,
                            const void* const* A, const void* const* B, int src_on_device,
@@ -149,12 +192,23 @@ SGMV_API sgmv_status sgmv_pool_adapter_rank(const sgmv_pool* pool, int32_t adapt
 SGMV_API sgmv_status sgmv_pool_adapter_pages(const sgmv_pool* pool, int32_t adapter_id, int32_t proj,
                                     int32_t matrix, int32_t* page_ids, int64_t cap, int64_t* n);
 /*
+ * Copy the stored form of (adapter, projection, matrix) to the host: `codes`
+ * receives its r rank rows (matrix 0 = A: rows of d_in; 1 = B^T: rows of d_out)
+ * in row order, as bf16 values (2 bytes each), E4M3 codes (1 byte each) or
+ * packed INT4 codes (d / 2 bytes a row); `scales` (may be NULL) receives the r
+ * row scales (1.0 for a bf16 pool).  Capacities are checked against cap_codes
+ * bytes and cap_scales floats.  Waits for the copies.  For export and tests.
+ */
+SGMV_API sgmv_status sgmv_pool_read(const sgmv_pool* pool, int32_t adapter_id, int32_t proj, int32_t matrix,
+                           void* codes, int64_t cap_codes, float* scales, int64_t cap_scales,
+                           sgmv_stream_t stream);
+/*
  * Reorder the free-page list pseudo-randomly (seeded), so that later loads
  * place consecutive chunks of a row on scattered pages.  Changes no resident
  * adapter.  For exercising the page-table indirection.
  */
 SGMV_API sgmv_status sgmv_pool_shuffle_free_pages(sgmv_pool* pool, uint64_t seed);
-/* Device address of the page buffer (bf16 [num_pages][page_elems]); NULL for a
+/* Device address of the page buffer ([num_pages][page_bytes]); NULL for a
  * host-only pool.  For inspection and tests. */
 SGMV_API const void* sgmv_pool_pages_device(const sgmv_pool* pool);
 

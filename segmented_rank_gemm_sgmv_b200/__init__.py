@@ -29,7 +29,8 @@ _STATUS = {0: "SGMV_OK", 1: "SGMV_ERR_INVALID", 2: "SGMV_ERR_UNSUPPORTED", 3: "S
            4: "SGMV_ERR_OUT_OF_PAGES", 5: "SGMV_ERR_CUDA", 6: "SGMV_ERR_BOUNDS", 7: "SGMV_ERR_TIMEOUT",
            8: "SGMV_ERR_CAPACITY"}
 
-EXPORTED = ("sgmv_status_string", "sgmv_last_error", "sgmv_pool_create", "sgmv_pool_destroy", "sgmv_pool_load",
+EXPORTED = ("sgmv_status_string", "sgmv_last_error", "sgmv_pool_create", "sgmv_pool_create_ex",
+            "sgmv_pool_destroy", "sgmv_pool_load", "sgmv_pool_read",
             "sgmv_pool_evict", "sgmv_pool_get_stats", "sgmv_pool_adapter_rank", "sgmv_pool_adapter_pages",
             "sgmv_pool_shuffle_free_pages", "sgmv_pool_pages_device", "sgmv_plan_table_capacity",
             "sgmv_build_plan", "sgmv_shrink", "sgmv_expand", "sgmv_lora_delta", "sgmv_lora_delta_grouped",
@@ -66,7 +67,11 @@ class ResidencyStats(ctypes.Structure):
 class PoolStats(ctypes.Structure):
     _fields_ = [("num_pages", ctypes.c_int64), ("free_pages", ctypes.c_int64), ("page_bytes", ctypes.c_int64),
                 ("payload_bytes", ctypes.c_int64), ("resident_adapters", ctypes.c_int32),
-                ("page_elems", ctypes.c_int32)]
+                ("page_elems", ctypes.c_int32), ("weight_format", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+# weight formats of a pool (sgmv_weight_format)
+WEIGHT_FORMATS = {"bf16": 0, "fp8_e4m3": 1, "int4": 2}
 
 
 _lib = None
@@ -87,6 +92,8 @@ def load_library() -> ctypes.CDLL:
         "sgmv_status_string": (ctypes.c_char_p, [st]),
         "sgmv_last_error": (ctypes.c_char_p, []),
         "sgmv_pool_create": (st, [ctypes.c_int, i64, i32, i32, vp, vp, i32, ctypes.POINTER(vp)]),
+        "sgmv_pool_create_ex": (st, [ctypes.c_int, i64, i32, i32, vp, vp, i32, i32, ctypes.POINTER(vp)]),
+        "sgmv_pool_read": (st, [vp, i32, i32, i32, vp, i64, vp, i64, vp]),
         "sgmv_pool_destroy": (st, [vp]),
         "sgmv_pool_load": (st, [vp, i32, i32, vp, vp, ctypes.c_int, vp]),
         "sgmv_pool_evict": (st, [vp, i32]),
@@ -143,17 +150,23 @@ class AdapterPool:
     """Paged adapter pool (see include/sgmv.h, "Paged adapter pool")."""
 
     def __init__(self, projections: Sequence[Tuple[int, int]], num_pages: int, page_elems: int = 512,
-                 max_rank: int = 128, device: int = 0):
+                 max_rank: int = 128, device: int = 0, weight_format: str = "bf16"):
+        """weight_format: "bf16" (default), "fp8_e4m3" or "int4" -- a quantised pool stores
+        codes with one fp32 scale per rank row and quantises bf16 weights as it loads them."""
         lib = load_library()
         self.projections = [(int(a), int(b)) for a, b in projections]
         self.device = device
         self.page_elems = page_elems
+        if weight_format not in WEIGHT_FORMATS:
+            raise ValueError(f"weight_format must be one of {sorted(WEIGHT_FORMATS)}")
+        self.weight_format = weight_format
         n = len(self.projections)
         d_in = (ctypes.c_int32 * n)(*[p[0] for p in self.projections])
         d_out = (ctypes.c_int32 * n)(*[p[1] for p in self.projections])
         h = ctypes.c_void_p()
-        _check(lib.sgmv_pool_create(device, int(num_pages), int(page_elems), n, ctypes.cast(d_in, ctypes.c_void_p),
-                                    ctypes.cast(d_out, ctypes.c_void_p), int(max_rank), ctypes.byref(h)))
+        _check(lib.sgmv_pool_create_ex(device, int(num_pages), int(page_elems), n,
+                                       ctypes.cast(d_in, ctypes.c_void_p), ctypes.cast(d_out, ctypes.c_void_p),
+                                       int(max_rank), WEIGHT_FORMATS[weight_format], ctypes.byref(h)))
         self.handle = h
 
     def close(self):
@@ -211,6 +224,23 @@ class AdapterPool:
         _check(load_library().sgmv_pool_get_stats(self.handle, ctypes.byref(s)))
         return s
 
+    def read(self, adapter_id: int, proj: int, matrix: int, stream=None) -> Tuple[np.ndarray, np.ndarray]:
+        """Stored form of (adapter, projection, matrix 0 = A / 1 = B^T): (codes, scales).
+        codes: uint16 bf16 words [r][d] (bf16 pool), uint8 E4M3 codes [r][d] or packed INT4
+        bytes [r][d/2]; scales: float32 [r] (ones for a bf16 pool)."""
+        r = self.rank_of(adapter_id)
+        d = self.projections[proj][matrix]
+        nbytes = {"bf16": 2 * d, "fp8_e4m3": d, "int4": d // 2}[self.weight_format]
+        codes = np.zeros((max(r, 1), nbytes), dtype=np.uint8)
+        scales = np.zeros(max(r, 1), dtype=np.float32)
+        _check(load_library().sgmv_pool_read(self.handle, int(adapter_id), int(proj), int(matrix),
+                                             codes.ctypes.data, codes.size, scales.ctypes.data, scales.size,
+                                             _stream(stream)))
+        codes, scales = codes[:r], scales[:r]
+        if self.weight_format == "bf16":
+            codes = codes.view(np.uint16)
+        return codes, scales
+
     def rank_of(self, adapter_id: int) -> int:
         r = ctypes.c_int32()
         _check(load_library().sgmv_pool_adapter_rank(self.handle, int(adapter_id), ctypes.byref(r)))
@@ -228,12 +258,15 @@ class AdapterPool:
         return out[:n.value]
 
     def pages_tensor(self) -> torch.Tensor:
-        """The page buffer as a bf16 [num_pages, page_elems] tensor view (device pools only)."""
+        """The page buffer as a tensor view (device pools only): bf16 [num_pages, page_elems]
+        for a bf16 pool, uint8 [num_pages, page_bytes] for a quantised one."""
         addr = load_library().sgmv_pool_pages_device(self.handle)
         s = self.stats()
         storage = torch.cuda.memory  # noqa: F841  (keeps torch.cuda initialised)
-        arr = _DevicePtr(addr, s.num_pages * s.page_elems * 2, self.device)
+        arr = _DevicePtr(addr, s.num_pages * s.page_bytes, self.device)
         t = torch.as_tensor(arr, device=f"cuda:{self.device}")
+        if self.weight_format != "bf16":
+            return t.view(s.num_pages, s.page_bytes)
         return t.view(torch.bfloat16).view(s.num_pages, s.page_elems)
 
     def plan(self, adapter_ids, long_threshold: int = 0) -> "BatchPlan":

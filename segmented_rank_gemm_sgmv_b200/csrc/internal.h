@@ -37,7 +37,11 @@ struct sgmv_pool {
     int32_t page_elems = 0, page_log2 = 0;
     int32_t n_proj = 0, max_rank = 0;
     std::vector<int32_t> d_in, d_out;
-    void* pages_dev = nullptr;       // bf16 [num_pages][page_elems]
+    int32_t wfmt = 0;                // sgmv_weight_format
+    int64_t page_bytes = 0;          // page_elems values: x2 (bf16), x1 (E4M3), x1/2 (INT4)
+    void* pages_dev = nullptr;       // [num_pages][page_bytes]
+    float* scale_dev = nullptr;      // quantised pools: fp32 [pt_capacity], scale of a rank row
+                                     // at the page-table entry of its first chunk
     int32_t* pt_dev = nullptr;       // int32 [pt_capacity]
     int64_t pt_capacity = 0;
     std::vector<int32_t> pt_host;    // mirror of the page table
@@ -94,12 +98,19 @@ struct BatchView {
     int32_t num_segments, num_rows, n_proj, proj, T;
 };
 
+// Weight format of a pool, as the kernels see it: bytes that hold 8 values.
+constexpr int kFmtBf16 = 0, kFmtFp8 = 1, kFmtInt4 = 2;
+template <int WF>
+__host__ __device__ constexpr int bytes_per_8() { return WF == kFmtBf16 ? 16 : WF == kFmtFp8 ? 8 : 4; }
+
 struct PoolView {
-    const uint16_t* pages;
+    const uint16_t* pages;       // bf16 pages; a quantised pool's code pages as the same buffer
     const int32_t* page_table;
+    const float* row_scale;      // quantised pools: scale of each rank row (first-chunk entry)
     int64_t num_pages;
     int64_t pt_capacity;
     int32_t page_log2;
+    int32_t wfmt;
 };
 
 // --------------------------------------------------------------- launchers
@@ -148,9 +159,10 @@ cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const B
 cudaError_t read_clear_errors_simt(uint32_t* bits, cudaStream_t stream);
 cudaError_t read_clear_errors_tc(uint32_t* bits, cudaStream_t stream);
 
-// Pool scatter kernels (sgmv_pool.cu).
-cudaError_t launch_pool_scatter(const uint16_t* src, int64_t rows, int64_t cols, bool transpose,
-                                const int32_t* page_table, int64_t pt_base, int32_t page_log2,
-                                uint16_t* pages, cudaStream_t stream);
+// Store a bf16 matrix (rank rows x cols; `transpose`: stored as cols x rows) into the
+// pool's pages from page-table entry pt_base on, quantising it in a quantised pool
+// (sgmv_pool.cu).
+cudaError_t write_matrix(sgmv_pool* p, const uint16_t* src, int64_t rows, int64_t cols, bool transpose,
+                         int64_t pt_base, cudaStream_t stream);
 
 }  // namespace sgmv

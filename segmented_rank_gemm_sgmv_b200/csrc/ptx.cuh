@@ -131,6 +131,20 @@ __device__ __forceinline__ void cp_async16(void* dst_smem, const void* src_gmem,
                  "r"(valid ? 16 : 0)
                  : "memory");
 }
+// 8- and 4-byte copies (through L1: the .cg form takes only 16 bytes).
+__device__ __forceinline__ void cp_async8(void* dst_smem, const void* src_gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst_smem, const void* src_gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem) : "memory");
+}
+// A copy of B bytes (16, 8 or 4) that is always valid.
+template <int B>
+__device__ __forceinline__ void cp_async_n(void* dst_smem, const void* src_gmem) {
+    if constexpr (B == 16) cp_async16(dst_smem, src_gmem, true);
+    else if constexpr (B == 8) cp_async8(dst_smem, src_gmem);
+    else cp_async4(dst_smem, src_gmem);
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
@@ -286,6 +300,40 @@ __device__ __forceinline__ void unpack8(const uint4& q, float (&f)[8]) {
     f[2] = bf16lo(q.y); f[3] = bf16hi(q.y);
     f[4] = bf16lo(q.z); f[5] = bf16hi(q.z);
     f[6] = bf16lo(q.w); f[7] = bf16hi(q.w);
+}
+
+// Eight E4M3 codes (byte i = value i) to fp32, exactly: each pair goes through
+// the hardware E4M3x2 -> f16x2 conversion (every E4M3 value is an f16 value).
+__device__ __forceinline__ void fp8x8_to_f32(const uint2& q, float (&f)[8]) {
+    const uint32_t w[2] = {q.x, q.y};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        uint32_t hh;
+        const uint16_t pair = (uint16_t)(w[h >> 1] >> (16 * (h & 1)));
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hh) : "h"(pair));
+        float lo, hi;
+        asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"((uint16_t)(hh & 0xFFFFu)));
+        asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"((uint16_t)(hh >> 16)));
+        f[2 * h] = lo;
+        f[2 * h + 1] = hi;
+    }
+}
+
+// Eight INT4 codes (two's complement nibbles, value i in bits 4i..4i+3) to fp32,
+// exactly: with n = nibble ^ 8 (0..15), the float whose bits are 0x4B000000 | n
+// is 2^23 + n, and 2^23 + n - (2^23 + 8) = n - 8 is the nibble's signed value.
+__device__ __forceinline__ void int4x8_to_f32(uint32_t q, float (&f)[8]) {
+    const uint32_t flipped = q ^ 0x88888888u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(0x4B000000u | ((flipped >> (4 * i)) & 0xFu)) - 8388616.0f;
+}
+
+// Eight stored weights of format WF at p (16, 8 or 4 bytes) to fp32.
+template <int WF>
+__device__ __forceinline__ void load_w8(const uint8_t* p, float (&f)[8]) {
+    if constexpr (WF == 0) unpack8(*reinterpret_cast<const uint4*>(p), f);
+    else if constexpr (WF == 1) fp8x8_to_f32(*reinterpret_cast<const uint2*>(p), f);
+    else int4x8_to_f32(*reinterpret_cast<const uint32_t*>(p), f);
 }
 
 }  // namespace sgmv

@@ -61,6 +61,8 @@ sgmv_status make_views(const sgmv_plan* plan, const void* table, const sgmv_pool
     pv->num_pages = pool->num_pages;
     pv->pt_capacity = pool->pt_capacity;
     pv->page_log2 = pool->page_log2;
+    pv->row_scale = pool->scale_dev;
+    pv->wfmt = pool->wfmt;
     return SGMV_OK;
 }
 

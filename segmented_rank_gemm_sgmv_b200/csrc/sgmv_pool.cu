@@ -7,7 +7,12 @@
 // blocks, so loading and evicting adapters does not fragment HBM).  For each
 // (adapter, projection) the pool keeps A as its r rank rows of d_in values and
 // B^T as r rank rows of d_out values; the page table maps every
-// (rank row, page-sized chunk) to a page.
+// (rank row, page-sized chunk) to a page.  A quantised pool (FP8 E4M3 or INT4
+// codes with one fp32 scale per rank row: "Multi-LoRA Inference Serving ..."
+// (clusterbid.com), paragraphs on the GPU memory budget and on adapter weight
+// quantization) quantises rows on the device as it stores them.
+#include <cuda_fp8.h>
+
 #include <algorithm>
 #include <cstring>
 
@@ -44,18 +49,78 @@ __global__ void pool_scatter_kernel(const uint16_t* __restrict__ src, int64_t ro
     *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(v);
 }
 
+// Quantise a logical [rows][cols] bf16 matrix row by row into a quantised pool
+// (one CTA per rank row).  Scale s = max |w| / Q (Q = 448 for E4M3, 7 for
+// INT4); code = RN(w / s), E4M3 with saturation, INT4 clamped to [-7, 7]; a
+// zero row keeps s = 0 and zero codes.  Both divisions are IEEE (round to
+// nearest), so the codes are those of any fp32 implementation of the rule.
+// The scale goes to the page-table entry of the row's first chunk.
+template <int WF>
+__global__ void __launch_bounds__(256) pool_quantize_kernel(const uint16_t* __restrict__ src, int64_t rows,
+                                                            int64_t cols, int transpose,
+                                                            const int32_t* __restrict__ page_table, int64_t pt_base,
+                                                            int32_t page_log2, uint8_t* __restrict__ pages,
+                                                            float* __restrict__ row_scale) {
+    __shared__ float red[8];
+    const int64_t row = blockIdx.x;
+    auto val = [&](int64_t c) {
+        const uint16_t h = transpose ? src[c * rows + row] : src[row * cols + c];
+        return __uint_as_float((uint32_t)h << 16);
+    };
+    float amax = 0.f;
+    for (int64_t c = threadIdx.x; c < cols; c += blockDim.x) amax = fmaxf(amax, fabsf(val(c)));
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) amax = fmaxf(amax, red[w]);
+    const float s = __fdiv_rn(amax, WF == kFmtFp8 ? 448.f : 7.f);
+    const int64_t chunks = cols >> page_log2;
+    if (threadIdx.x == 0) row_scale[pt_base + row * chunks] = s;
+    for (int64_t c0 = (int64_t)threadIdx.x * 8; c0 < cols; c0 += (int64_t)blockDim.x * 8) {
+        const int32_t page = page_table[pt_base + row * chunks + (c0 >> page_log2)];
+        const int64_t e = ((int64_t)page << page_log2) + (c0 & ((1 << page_log2) - 1));  // value index
+        if (WF == kFmtFp8) {
+            uint32_t w[2] = {0u, 0u};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float r = s > 0.f ? __fdiv_rn(val(c0 + i), s) : 0.f;
+                w[i >> 2] |= (uint32_t)__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E4M3) << (8 * (i & 3));
+            }
+            *reinterpret_cast<uint2*>(pages + e) = make_uint2(w[0], w[1]);
+        } else {
+            uint32_t w = 0u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                int q = s > 0.f ? __float2int_rn(__fdiv_rn(val(c0 + i), s)) : 0;
+                q = min(7, max(-7, q));
+                w |= ((uint32_t)q & 0xFu) << (4 * i);
+            }
+            *reinterpret_cast<uint32_t*>(pages + (e >> 1)) = w;
+        }
+    }
+}
+
 }  // namespace
 
-cudaError_t launch_pool_scatter(const uint16_t* src, int64_t rows, int64_t cols, bool transpose,
-                                const int32_t* page_table, int64_t pt_base, int32_t page_log2, uint16_t* pages,
-                                cudaStream_t stream) {
-    const int64_t n = rows * (cols >> 3);
-    if (n == 0) return cudaSuccess;
-    const int threads = 256;
-    const int64_t blocks = (n + threads - 1) / threads;
-    const int vec_ok = ((reinterpret_cast<uintptr_t>(src) & 15) == 0) ? 1 : 0;
-    pool_scatter_kernel<<<(unsigned)blocks, threads, 0, stream>>>(src, rows, cols, transpose ? 1 : 0, page_table,
-                                                                   pt_base, page_log2, pages, vec_ok);
+cudaError_t write_matrix(sgmv_pool* p, const uint16_t* src, int64_t rows, int64_t cols, bool transpose,
+                         int64_t pt_base, cudaStream_t stream) {
+    if (rows == 0 || cols == 0) return cudaSuccess;
+    if (p->wfmt == kFmtBf16) {
+        const int64_t n = rows * (cols >> 3);
+        const int threads = 256;
+        const int64_t blocks = (n + threads - 1) / threads;
+        const int vec_ok = ((reinterpret_cast<uintptr_t>(src) & 15) == 0) ? 1 : 0;
+        pool_scatter_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+            src, rows, cols, transpose ? 1 : 0, p->pt_dev, pt_base, p->page_log2,
+            static_cast<uint16_t*>(p->pages_dev), vec_ok);
+    } else {
+        auto kern = p->wfmt == kFmtFp8 ? pool_quantize_kernel<kFmtFp8> : pool_quantize_kernel<kFmtInt4>;
+        kern<<<(unsigned)rows, 256, 0, stream>>>(src, rows, cols, transpose ? 1 : 0, p->pt_dev, pt_base,
+                                                 p->page_log2, static_cast<uint8_t*>(p->pages_dev), p->scale_dev);
+    }
     return cudaGetLastError();
 }
 
@@ -150,7 +215,16 @@ using namespace sgmv;
 extern "C" sgmv_status sgmv_pool_create(int device, int64_t num_pages, int32_t page_elems, int32_t n_proj,
                                         const int32_t* d_in, const int32_t* d_out, int32_t max_rank,
                                         sgmv_pool** out) {
+    return sgmv_pool_create_ex(device, num_pages, page_elems, n_proj, d_in, d_out, max_rank, SGMV_WEIGHTS_BF16, out);
+}
+
+extern "C" sgmv_status sgmv_pool_create_ex(int device, int64_t num_pages, int32_t page_elems, int32_t n_proj,
+                                           const int32_t* d_in, const int32_t* d_out, int32_t max_rank,
+                                           int32_t weight_format, sgmv_pool** out) {
     if (!out) return fail(SGMV_ERR_INVALID, "pool_create: out is NULL");
+    if (weight_format != SGMV_WEIGHTS_BF16 && weight_format != SGMV_WEIGHTS_FP8_E4M3 &&
+        weight_format != SGMV_WEIGHTS_INT4)
+        return fail(SGMV_ERR_INVALID, "pool_create: unknown weight format");
     *out = nullptr;
     if (num_pages <= 0 || num_pages > (int64_t)INT32_MAX)
         return fail(SGMV_ERR_INVALID, "pool_create: num_pages must be in [1, 2^31-1]");
@@ -168,6 +242,9 @@ extern "C" sgmv_status sgmv_pool_create(int device, int64_t num_pages, int32_t p
     while ((1 << p->page_log2) < page_elems) ++p->page_log2;
     p->n_proj = n_proj;
     p->max_rank = max_rank;
+    p->wfmt = weight_format;
+    p->page_bytes = weight_format == SGMV_WEIGHTS_BF16 ? 2 * (int64_t)page_elems
+                    : weight_format == SGMV_WEIGHTS_FP8_E4M3 ? (int64_t)page_elems : (int64_t)page_elems / 2;
     p->d_in.assign(d_in, d_in + n_proj);
     p->d_out.assign(d_out, d_out + n_proj);
     p->pt_capacity = 2 * num_pages + 1024;
@@ -177,12 +254,17 @@ extern "C" sgmv_status sgmv_pool_create(int device, int64_t num_pages, int32_t p
     for (int64_t i = num_pages - 1; i >= 0; --i) p->free_pages.push_back(i);  // pop order 0, 1, 2, ...
     if (device >= 0) {
         cudaError_t e = cudaSetDevice(device);
-        if (e == cudaSuccess) e = cudaMalloc(&p->pages_dev, (size_t)num_pages * page_elems * 2);
+        if (e == cudaSuccess) e = cudaMalloc(&p->pages_dev, (size_t)num_pages * p->page_bytes);
         if (e == cudaSuccess) e = cudaMalloc((void**)&p->pt_dev, (size_t)p->pt_capacity * sizeof(int32_t));
         if (e == cudaSuccess) e = cudaMemset(p->pt_dev, 0xFF, (size_t)p->pt_capacity * sizeof(int32_t));
+        if (e == cudaSuccess && weight_format != SGMV_WEIGHTS_BF16) {
+            e = cudaMalloc((void**)&p->scale_dev, (size_t)p->pt_capacity * sizeof(float));
+            if (e == cudaSuccess) e = cudaMemset(p->scale_dev, 0, (size_t)p->pt_capacity * sizeof(float));
+        }
         if (e != cudaSuccess) {
             if (p->pages_dev) cudaFree(p->pages_dev);
             if (p->pt_dev) cudaFree(p->pt_dev);
+            if (p->scale_dev) cudaFree(p->scale_dev);
             delete p;
             return cuda_fail(e, "pool_create: device allocation");
         }
@@ -197,6 +279,7 @@ extern "C" sgmv_status sgmv_pool_destroy(sgmv_pool* p) {
         cudaSetDevice(p->device);
         if (p->pages_dev) cudaFree(p->pages_dev);
         if (p->pt_dev) cudaFree(p->pt_dev);
+        if (p->scale_dev) cudaFree(p->scale_dev);
         if (p->staging_dev) cudaFree(p->staging_dev);
     }
     delete p;
@@ -242,7 +325,6 @@ extern "C" sgmv_status sgmv_pool_load(sgmv_pool* p, int32_t adapter_id, int32_t 
             SGMV_CUDA_TRY(cudaMalloc(&p->staging_dev, max_bytes));
             p->staging_bytes = max_bytes;
         }
-        uint16_t* pages = static_cast<uint16_t*>(p->pages_dev);
         for (int i = 0; i < p->n_proj; ++i) {
             for (int m = 0; m < 2; ++m) {
                 const int64_t cols = m == 0 ? p->d_in[i] : p->d_out[i];
@@ -252,9 +334,8 @@ extern "C" sgmv_status sgmv_pool_load(sgmv_pool* p, int32_t adapter_id, int32_t 
                     SGMV_CUDA_TRY(cudaMemcpyAsync(p->staging_dev, src, bytes, cudaMemcpyHostToDevice, stream));
                     src = p->staging_dev;
                 }
-                SGMV_CUDA_TRY(launch_pool_scatter(static_cast<const uint16_t*>(src), rank, cols, m == 1, p->pt_dev,
-                                                  m == 0 ? rec.a_pt[i] : rec.b_pt[i], p->page_log2, pages,
-                                                  stream));
+                SGMV_CUDA_TRY(write_matrix(p, static_cast<const uint16_t*>(src), rank, cols, m == 1,
+                                           m == 0 ? rec.a_pt[i] : rec.b_pt[i], stream));
                 if (!src_on_device) SGMV_CUDA_TRY(cudaStreamSynchronize(stream));  // staging is reused
             }
         }
@@ -275,10 +356,12 @@ extern "C" sgmv_status sgmv_pool_get_stats(const sgmv_pool* p, sgmv_pool_stats* 
     if (!p || !out) return fail(SGMV_ERR_INVALID, "pool_get_stats: NULL argument");
     out->num_pages = p->num_pages;
     out->free_pages = (int64_t)p->free_pages.size();
-    out->page_bytes = (int64_t)p->page_elems * 2;
+    out->page_bytes = p->page_bytes;
     out->payload_bytes = (p->num_pages - out->free_pages) * out->page_bytes;
     out->resident_adapters = (int32_t)p->adapters.size();
     out->page_elems = p->page_elems;
+    out->weight_format = p->wfmt;
+    out->reserved = 0;
     return SGMV_OK;
 }
 
@@ -304,6 +387,41 @@ extern "C" sgmv_status sgmv_pool_adapter_pages(const sgmv_pool* p, int32_t adapt
     if (count > cap || (count > 0 && !page_ids)) return fail(SGMV_ERR_CAPACITY, "pool_adapter_pages: buffer too small");
     const int64_t base = matrix == 0 ? rec.a_pt[proj] : rec.b_pt[proj];
     for (int64_t i = 0; i < count; ++i) page_ids[i] = p->pt_host[base + i];
+    return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_pool_read(const sgmv_pool* p, int32_t adapter_id, int32_t proj, int32_t matrix,
+                                      void* codes, int64_t cap_codes, float* scales, int64_t cap_scales,
+                                      sgmv_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (!p) return fail(SGMV_ERR_INVALID, "pool_read: pool is NULL");
+    if (p->device < 0 || !p->pages_dev) return fail(SGMV_ERR_INVALID, "pool_read: pool has no device memory");
+    if (proj < 0 || proj >= p->n_proj || (matrix != 0 && matrix != 1))
+        return fail(SGMV_ERR_INVALID, "pool_read: bad projection or matrix");
+    auto it = p->adapters.find(adapter_id);
+    if (it == p->adapters.end()) return fail(SGMV_ERR_NOT_RESIDENT, "pool_read: adapter not resident");
+    const AdapterRec& rec = it->second;
+    const int64_t d = matrix == 0 ? p->d_in[proj] : p->d_out[proj];
+    const int64_t cpr = d >> p->page_log2;                  // chunks (pages) per rank row
+    const int64_t row_bytes = cpr * p->page_bytes;
+    if (codes && cap_codes < rec.rank * row_bytes) return fail(SGMV_ERR_CAPACITY, "pool_read: codes buffer too small");
+    if (scales && cap_scales < rec.rank) return fail(SGMV_ERR_CAPACITY, "pool_read: scales buffer too small");
+    const int64_t base = matrix == 0 ? rec.a_pt[proj] : rec.b_pt[proj];
+    SGMV_CUDA_TRY(cudaSetDevice(p->device));
+    const uint8_t* pages = static_cast<const uint8_t*>(p->pages_dev);
+    if (codes)
+        for (int64_t k = 0; k < rec.rank; ++k)
+            for (int64_t c = 0; c < cpr; ++c)
+                SGMV_CUDA_TRY(cudaMemcpyAsync(static_cast<uint8_t*>(codes) + k * row_bytes + c * p->page_bytes,
+                                              pages + (int64_t)p->pt_host[base + k * cpr + c] * p->page_bytes,
+                                              (size_t)p->page_bytes, cudaMemcpyDeviceToHost, stream));
+    std::vector<float> sc((size_t)std::max<int64_t>(rec.rank * cpr, 1), 1.0f);
+    if (scales && p->scale_dev && rec.rank > 0)
+        SGMV_CUDA_TRY(cudaMemcpyAsync(sc.data(), p->scale_dev + base, (size_t)(rec.rank * cpr) * sizeof(float),
+                                      cudaMemcpyDeviceToHost, stream));
+    SGMV_CUDA_TRY(cudaStreamSynchronize(stream));
+    if (scales)
+        for (int64_t k = 0; k < rec.rank; ++k) scales[k] = p->scale_dev ? sc[(size_t)(k * cpr)] : 1.0f;
     return SGMV_OK;
 }
 
@@ -485,7 +603,6 @@ extern "C" sgmv_status sgmv_residency_prepare(sgmv_residency* r, const int32_t* 
             SGMV_CUDA_TRY(cudaMemcpyAsync(p->pt_dev + rec.pt_begin, p->pt_host.data() + rec.pt_begin,
                                           (size_t)rec.pt_count * sizeof(int32_t), cudaMemcpyHostToDevice,
                                           copy_stream));
-            uint16_t* pages = static_cast<uint16_t*>(p->pages_dev);
             for (int i = 0; i < p->n_proj; ++i) {
                 for (int m = 0; m < 2; ++m) {
                     const int64_t cols = m == 0 ? p->d_in[i] : p->d_out[i];
@@ -494,9 +611,8 @@ extern "C" sgmv_status sgmv_residency_prepare(sgmv_residency* r, const int32_t* 
                     // previous scatter on the copy stream
                     SGMV_CUDA_TRY(cudaMemcpyAsync(r->staging, m == 0 ? h.A[i] : h.B[i], bytes,
                                                   cudaMemcpyHostToDevice, copy_stream));
-                    SGMV_CUDA_TRY(launch_pool_scatter(static_cast<const uint16_t*>(r->staging), h.rank, cols, m == 1,
-                                                      p->pt_dev, m == 0 ? rec.a_pt[i] : rec.b_pt[i], p->page_log2,
-                                                      pages, copy_stream));
+                    SGMV_CUDA_TRY(write_matrix(p, static_cast<const uint16_t*>(r->staging), h.rank, cols, m == 1,
+                                               m == 0 ? rec.a_pt[i] : rec.b_pt[i], copy_stream));
                     r->stats.bytes_loaded += (int64_t)bytes;
                 }
             }

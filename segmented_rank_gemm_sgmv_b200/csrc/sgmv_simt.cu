@@ -34,6 +34,7 @@
 #include <map>
 #include <mutex>
 #include <tuple>
+#include <type_traits>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -54,6 +55,9 @@ template <int MAXG>
 __host__ __device__ constexpr int shrink_stages() { return MAXG == 1 ? 4 : 3; }
 constexpr int kExpandStages = 3;
 constexpr int kStageElems = kRowGroup * kPass;
+// bytes of one stage in weight format WF (bf16 16 KB, E4M3 8 KB, INT4 4 KB)
+template <int WF>
+__host__ __device__ constexpr int stage_bytes() { return kStageElems / 8 * bytes_per_8<WF>(); }
 
 // One projection of a launch.  A launch covers up to kMaxGroup projections over
 // the same batch plan (sgmv_lora_delta_grouped); every projection gets the same
@@ -243,9 +247,9 @@ struct StageGeom {  // rows and columns of the CTA's stages
 
 // The ring: stage `issued` goes to slot `islot`, its row group / pass advance
 // incrementally (row group outer for the shrink, pass outer for the expand).
-template <int kStages>
+template <int kStages, int WF>
 struct Pipe {
-    uint16_t* data;
+    uint8_t* data;
     int issued = 0, total = 0;
     int islot = 0, cslot = 0;  // slots of the next issued / consumed stage
     int ig = 0, is = 0;        // row group and pass of the next issued stage
@@ -261,9 +265,11 @@ struct XStage {
     int maxg;
 };
 
-template <int kStages>
-__device__ __forceinline__ void pipe_issue(const PoolView& pool, Pipe<kStages>& pp, const StageGeom& sg,
+template <int kStages, int WF>
+__device__ __forceinline__ void pipe_issue(const PoolView& pool, Pipe<kStages, WF>& pp, const StageGeom& sg,
                                            bool pass_outer, const XStage& xs) {
+    constexpr int VB = bytes_per_8<WF>();  // bytes of 8 stored values
+    const uint8_t* pages = reinterpret_cast<const uint8_t*>(pool.pages);
     if (pp.issued < pp.total) {
         const int P_log2 = pool.page_log2, P = 1 << P_log2;
         const int g = pp.ig, c = pp.is * kPass;
@@ -277,19 +283,21 @@ __device__ __forceinline__ void pipe_issue(const PoolView& pool, Pipe<kStages>& 
                                xs.rows[j] != nullptr);
         }
         const int rows = min(kRowGroup, sg.rank - kRowGroup * g);
-        uint16_t* dst0 = pp.data + (size_t)pp.islot * kStageElems;
+        uint8_t* dst0 = pp.data + (size_t)pp.islot * stage_bytes<WF>();
         const int32_t* pidg = sg.pid + kRowGroup * g * sg.span_pages;
+        // a page is (1 << P_log2) values, (1 << page_shift) bytes; column c of it at byte c * VB / 8
+        const int page_shift = P_log2 + (VB == 16 ? 1 : VB == 8 ? 0 : -1);
         if (W == kPass) {  // full pass: thread t copies granule t of each of the stage's rows
             const int col = c + kVec * threadIdx.x;
             const int32_t* pidc = pidg + (col >> P_log2);
-            const uint16_t* src0 = pool.pages + (col & (P - 1));
-            uint16_t* dst = dst0 + kVec * threadIdx.x;
+            const uint8_t* src0 = pages + ((col & (P - 1)) / 8 * VB);
+            uint8_t* dst = dst0 + VB * threadIdx.x;
 #pragma unroll
             for (int kk = 0; kk < kRowGroup; ++kk)
                 if (kk < rows)
-                    cp_async16(dst + kk * kPass, src0 + ((int64_t)pidc[kk * sg.span_pages] << P_log2), true);
+                    cp_async_n<VB>(dst + kk * (kPass / 8 * VB), src0 + ((int64_t)pidc[kk * sg.span_pages] << page_shift));
         } else {
-            const int gpr = W >> 3;  // granules per row
+            const int gpr = W >> 3;  // granules (8 values) per row
 #pragma unroll
             for (int i = 0; i < kStageElems / 8 / kThreads; ++i) {
                 const int gi = threadIdx.x + kThreads * i;
@@ -297,8 +305,8 @@ __device__ __forceinline__ void pipe_issue(const PoolView& pool, Pipe<kStages>& 
                 if (kk < rows) {
                     const int col = c + cg * 8;
                     const int32_t page = pidg[kk * sg.span_pages + (col >> P_log2)];
-                    cp_async16(dst0 + (size_t)kk * W + cg * 8,
-                               pool.pages + ((int64_t)page << P_log2) + (col & (P - 1)), true);
+                    cp_async_n<VB>(dst0 + ((size_t)kk * W / 8 + cg) * VB,
+                                   pages + ((int64_t)page << page_shift) + (col & (P - 1)) / 8 * VB);
                 }
             }
         }
@@ -313,15 +321,15 @@ __device__ __forceinline__ void pipe_issue(const PoolView& pool, Pipe<kStages>& 
     cp_async_commit();
 }
 
-template <int kStages>
-__device__ __forceinline__ const uint16_t* pipe_acquire(Pipe<kStages>& pp) {
+template <int kStages, int WF>
+__device__ __forceinline__ const uint8_t* pipe_acquire(Pipe<kStages, WF>& pp) {
     cp_async_wait<kStages - 1>();
     __syncthreads();
-    return pp.data + (size_t)pp.cslot * kStageElems;
+    return pp.data + (size_t)pp.cslot * stage_bytes<WF>();
 }
 
-template <int kStages>
-__device__ __forceinline__ void pipe_release(const PoolView& pool, Pipe<kStages>& pp, const StageGeom& sg,
+template <int kStages, int WF>
+__device__ __forceinline__ void pipe_release(const PoolView& pool, Pipe<kStages, WF>& pp, const StageGeom& sg,
                                              bool pass_outer, const XStage& xs) {
     __syncthreads();  // every thread is done with the slot before it is refilled
     pp.cslot = pp.cslot + 1 == kStages ? 0 : pp.cslot + 1;
@@ -348,10 +356,25 @@ __device__ void load_page_ids(const PoolView& pool, StageGeom& sg, int32_t* pid,
     sg.pid = pid;
 }
 
+// Threads k < r: the scale of rank row k of a quantised matrix (kept at the
+// page-table entry of the row's first chunk) into rsc[k].  An entry outside
+// the table is flagged and reads as 0.
+__device__ __forceinline__ void load_row_scales(const PoolView& pool, int64_t pt, int pages_per_row, int r,
+                                                float* rsc, unsigned int* err) {
+    for (int k = threadIdx.x; k < r; k += kThreads) {
+        const int64_t e = pt + (int64_t)k * pages_per_row;
+        float v = 0.f;
+        if (e >= 0 && e < pool.pt_capacity) v = pool.row_scale[e];
+        else atomicOr(err, kErrPage);
+        rsc[k] = v;
+    }
+}
+
 // ------------------------------------------------------------------ shrink
-template <int G, int kStages>
-__device__ void shrink_item(const PoolView& pool, const ItemInfo& m, Pipe<kStages>& pp, const StageGeom& sg,
+template <int G, int kStages, int WF>
+__device__ void shrink_item(const PoolView& pool, const ItemInfo& m, Pipe<kStages, WF>& pp, const StageGeom& sg,
                             const XStage& xs, float* part, float* red) {
+    constexpr int VB = bytes_per_8<WF>();
     const int tid = threadIdx.x, col = kVec * tid;
     for (int g = 0; g < sg.NG; ++g) {
         float p[kRowGroup * G];
@@ -360,7 +383,7 @@ __device__ void shrink_item(const PoolView& pool, const ItemInfo& m, Pipe<kStage
         for (int s = 0; s < sg.npass; ++s) {
             const int c = s * kPass, W = min(kPass, sg.span - c);
             const bool active = col < W;
-            const uint16_t* st = pipe_acquire(pp);
+            const uint8_t* st = pipe_acquire(pp);
             const uint16_t* xst = xs.ring + (size_t)pp.cslot * xs.maxg * kPass + col;
             if (active) {
                 float xf[G][8];
@@ -369,7 +392,7 @@ __device__ void shrink_item(const PoolView& pool, const ItemInfo& m, Pipe<kStage
 #pragma unroll
                 for (int kk = 0; kk < kRowGroup; ++kk) {
                     float af[8];
-                    unpack8(*reinterpret_cast<const uint4*>(st + (size_t)kk * W + col), af);
+                    load_w8<WF>(st + ((size_t)kk * (W >> 3) + tid) * VB, af);
 #pragma unroll
                     for (int j = 0; j < G; ++j) p[kk * G + j] += dot8(af, xf[j]);
                 }
@@ -384,7 +407,7 @@ __device__ void shrink_item(const PoolView& pool, const ItemInfo& m, Pipe<kStage
     }
 }
 
-template <int MAXG, int NI, int NE>
+template <int MAXG, int NI, int NE, int WF>
 __global__ void __launch_bounds__(kThreads, 3)
     shrink_simt_kernel(const __grid_constant__ ShrinkArgs<NE> a, const __grid_constant__ InlineTable<NI> inl) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -401,7 +424,8 @@ __global__ void __launch_bounds__(kThreads, 3)
     const int slot = kSimtMaxItemRows * a.max_rank;  // floats of one partial tile
     float* part = reinterpret_cast<float*>(smem);     // [C slots][slot]; slot 0 is this CTA's own
     float* red = part + C * slot;                      // [4 warps][64]
-    int32_t* pid = reinterpret_cast<int32_t*>(red + 4 * 64);
+    float* rsc = red + 4 * 64;                         // [kMaxRank] row scales (quantised pools)
+    int32_t* pid = reinterpret_cast<int32_t*>(rsc + kMaxRank);
 
     const ItemInfo m = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 0)
                               : load_item(a.b, en.proj, item_idx, MAXG, a.max_rank, 0);
@@ -415,17 +439,18 @@ __global__ void __launch_bounds__(kThreads, 3)
     sg.pages_per_row = en.d_in >> a.pool.page_log2;
     sg.pt = m.pt;
     constexpr int kShrinkStages = shrink_stages<MAXG>();
-    Pipe<kShrinkStages> pp;
-    pp.data = reinterpret_cast<uint16_t*>(smem + a.ring_offset);
+    Pipe<kShrinkStages, WF> pp;
+    pp.data = smem + a.ring_offset;
     pp.total = m.ok ? sg.NG * sg.npass : 0;
     XStage xs;
-    xs.ring = pp.data + (size_t)kShrinkStages * kStageElems;
+    xs.ring = reinterpret_cast<uint16_t*>(pp.data + (size_t)kShrinkStages * stage_bytes<WF>());
     xs.maxg = MAXG;
     xs.any = en.x;
 #pragma unroll
     for (int j = 0; j < kSimtMaxItemRows; ++j)
         xs.rows[j] = (j < MAXG && m.tok[j] >= 0) ? en.x + (int64_t)m.tok[j] * en.ldx + (int64_t)q * en.kc : nullptr;
     if (m.ok) load_page_ids(a.pool, sg, pid, &g_err_simt);
+    if (WF != kFmtBf16 && m.ok && q == 0) load_row_scales(a.pool, m.pt, sg.pages_per_row, m.r, rsc, &g_err_simt);
     __syncthreads();
 #pragma unroll 1
     for (int i = 0; i < kShrinkStages; ++i) pipe_issue(a.pool, pp, sg, false, xs);
@@ -461,15 +486,17 @@ __global__ void __launch_bounds__(kThreads, 3)
             float s = 0.f;
             for (int qq = 0; qq < C; ++qq) s += part[(size_t)qq * slot + e];
             const int jrow = e / m.r, k = e - jrow * m.r;
-            en.v[(int64_t)(m.i0 + jrow) * en.ldv + k] = s;
+            // a quantised row's scale leaves the sum: v_k = s_k * sum_c q_kc x_c
+            en.v[(int64_t)(m.i0 + jrow) * en.ldv + k] = WF == kFmtBf16 ? s : s * rsc[k];
         }
     }
 }
 
 // ------------------------------------------------------------------ expand
-template <int G, int NE>
-__device__ void expand_item(const ExpandArgs<NE>& a, const ExpandEntry& en, const ItemInfo& m, Pipe<kExpandStages>& pp,
-                            const StageGeom& sg, float* vs) {
+template <int G, int NE, int WF>
+__device__ void expand_item(const ExpandArgs<NE>& a, const ExpandEntry& en, const ItemInfo& m,
+                            Pipe<kExpandStages, WF>& pp, const StageGeom& sg, float* vs, const float* rsc) {
+    constexpr int VB = bytes_per_8<WF>();
     const int tid = threadIdx.x, col = kVec * tid;
     int trow[G];
 #pragma unroll
@@ -498,7 +525,8 @@ __device__ void expand_item(const ExpandArgs<NE>& a, const ExpandEntry& en, cons
     pdl_wait();  // v (and, unless y_early, y) are final once the preceding kernel has completed
     for (int e = tid; e < m.n * m.r; e += kThreads) {
         const int jrow = e / m.r, k = e - jrow * m.r;
-        vs[e] = en.v[(int64_t)(m.i0 + jrow) * en.ldv + k];
+        const float vk = en.v[(int64_t)(m.i0 + jrow) * en.ldv + k];
+        vs[e] = WF == kFmtBf16 ? vk : vk * rsc[k];  // a quantised B^T row's scale goes onto v_k
     }
     // (the first pipe_acquire's barrier publishes vs)
     for (int s = 0; s < sg.npass; ++s) {
@@ -513,14 +541,14 @@ __device__ void expand_item(const ExpandArgs<NE>& a, const ExpandEntry& en, cons
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
         for (int g = 0; g < sg.NG; ++g) {
-            const uint16_t* st = pipe_acquire(pp);
+            const uint8_t* st = pipe_acquire(pp);
             if (active) {
 #pragma unroll
                 for (int kk = 0; kk < kRowGroup; ++kk) {
                     const int k = kRowGroup * g + kk;
                     if (k < m.r) {
                         float bf[8];
-                        unpack8(*reinterpret_cast<const uint4*>(st + (size_t)kk * W + col), bf);
+                        load_w8<WF>(st + ((size_t)kk * (W >> 3) + tid) * VB, bf);
 #pragma unroll
                         for (int j = 0; j < G; ++j) {
                             const float w = vs[min(j, m.n - 1) * m.r + k];
@@ -569,7 +597,7 @@ __device__ void expand_item(const ExpandArgs<NE>& a, const ExpandEntry& en, cons
     }
 }
 
-template <int MAXG, int NI, int NE>
+template <int MAXG, int NI, int NE, int WF>
 __global__ void __launch_bounds__(kThreads, 3)
     expand_simt_kernel(const __grid_constant__ ExpandArgs<NE> a, const __grid_constant__ InlineTable<NI> inl) {
     extern __shared__ __align__(128) uint8_t smem_e[];
@@ -580,7 +608,8 @@ __global__ void __launch_bounds__(kThreads, 3)
     const int local = (int)blockIdx.x - en.cta_base;
     const int part_idx = local % en.cpi, item_idx = local / en.cpi;
     float* vs = reinterpret_cast<float*>(smem_e);
-    int32_t* pid = reinterpret_cast<int32_t*>(vs + kSimtMaxItemRows * a.max_rank);
+    float* rsc = vs + kSimtMaxItemRows * a.max_rank;  // [kMaxRank] row scales (quantised pools)
+    int32_t* pid = reinterpret_cast<int32_t*>(rsc + kMaxRank);
 
     const ItemInfo m = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 1)
                               : load_item(a.b, en.proj, item_idx, MAXG, a.max_rank, 1);
@@ -594,10 +623,11 @@ __global__ void __launch_bounds__(kThreads, 3)
     sg.pages_per_row = en.d_out >> a.pool.page_log2;
     sg.pt = m.pt;
     const bool work = m.ok && sg.span > 0;
-    Pipe<kExpandStages> pp;
-    pp.data = reinterpret_cast<uint16_t*>(smem_e + a.ring_offset);
+    Pipe<kExpandStages, WF> pp;
+    pp.data = smem_e + a.ring_offset;
     pp.total = work ? sg.NG * sg.npass : 0;
     if (work) load_page_ids(a.pool, sg, pid, &g_err_simt);
+    if (WF != kFmtBf16 && work) load_row_scales(a.pool, m.pt, sg.pages_per_row, m.r, rsc, &g_err_simt);
     __syncthreads();
     // B^T pages do not depend on the shrink: start them before waiting for it
 #pragma unroll 1
@@ -608,9 +638,9 @@ __global__ void __launch_bounds__(kThreads, 3)
         cp_async_wait<0>();
         return;
     }
-    if (MAXG == 1 || m.n == 1) expand_item<1, NE>(a, en, m, pp, sg, vs);
-    else if (MAXG == 2 || m.n == 2) expand_item<(MAXG < 2 ? MAXG : 2), NE>(a, en, m, pp, sg, vs);
-    else expand_item<MAXG, NE>(a, en, m, pp, sg, vs);
+    if (MAXG == 1 || m.n == 1) expand_item<1, NE>(a, en, m, pp, sg, vs, rsc);
+    else if (MAXG == 2 || m.n == 2) expand_item<(MAXG < 2 ? MAXG : 2), NE>(a, en, m, pp, sg, vs, rsc);
+    else expand_item<MAXG, NE>(a, en, m, pp, sg, vs, rsc);
     cp_async_wait<0>();
 }
 
@@ -708,7 +738,7 @@ double group_time(const SimtWork& work, int64_t items, const int* cpi, const int
     return std::max(biggest, total / (double)std::max<int64_t>(slots, 1));
 }
 
-template <int NE>
+template <int NE, int WF>
 cudaError_t shrink_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,
                           int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
                           const InlineTable<kInlineItems>* inl, cudaStream_t stream) {
@@ -716,21 +746,22 @@ cudaError_t shrink_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b,
     int order[kMaxGroup];
     for (int j = 0; j < n_jobs; ++j) order[j] = j;
     std::stable_sort(order, order + n_jobs, [&](int u, int w) { return jobs[u].d_in > jobs[w].d_in; });
-    auto kern_inl = pick(max_item_rows, shrink_simt_kernel<1, kInlineItems, NE>, shrink_simt_kernel<2, kInlineItems, NE>,
-                         shrink_simt_kernel<4, kInlineItems, NE>);
-    auto kern_tab = pick(max_item_rows, shrink_simt_kernel<1, 1, NE>, shrink_simt_kernel<2, 1, NE>,
-                         shrink_simt_kernel<4, 1, NE>);
+    auto kern_inl = pick(max_item_rows, shrink_simt_kernel<1, kInlineItems, NE, WF>,
+                         shrink_simt_kernel<2, kInlineItems, NE, WF>, shrink_simt_kernel<4, kInlineItems, NE, WF>);
+    auto kern_tab = pick(max_item_rows, shrink_simt_kernel<1, 1, NE, WF>, shrink_simt_kernel<2, 1, NE, WF>,
+                         shrink_simt_kernel<4, 1, NE, WF>);
     const void* kp = inl ? reinterpret_cast<const void*>(kern_inl) : reinterpret_cast<const void*>(kern_tab);
     const int mr = std::max(8, max_rank);
     int max_pages = 0;
     for (int j = 0; j < n_jobs; ++j) max_pages = std::max(max_pages, jobs[j].d_in >> pool.page_log2);
     const int maxg = max_item_rows <= 1 ? 1 : max_item_rows <= 2 ? 2 : 4;
     const int stages = maxg == 1 ? shrink_stages<1>() : shrink_stages<4>();
-    const size_t ring_bytes = (size_t)stages * (kStageElems + (size_t)maxg * kPass) * 2;  // A rows + x slices
-    auto smem_for = [&](int c) {
+    // A rows + x slices
+    const size_t ring_bytes = (size_t)stages * ((size_t)stage_bytes<WF>() + (size_t)maxg * kPass * 2);
+    auto smem_for = [&](int c) {  // partial tiles, reduction scratch, row scales, page ids, ring
         const size_t part_bytes = (size_t)c * kSimtMaxItemRows * mr * 4;
         const size_t pidb = (size_t)mr * ((max_pages + c - 1) / c) * 4;
-        return (((part_bytes + 1024 + pidb + 127) & ~(size_t)127)) + ring_bytes;
+        return (((part_bytes + 1024 + kMaxRank * 4 + pidb + 127) & ~(size_t)127)) + ring_bytes;
     };
     // Cluster size C (chunks of >= 1024 columns, C <= 8, dividing every entry's page
     // count): the one with the shortest modelled time.
@@ -792,7 +823,7 @@ cudaError_t shrink_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b,
     return cudaLaunchKernelEx(&cfg, kern_tab, a, InlineTable<1>{});
 }
 
-template <int NE>
+template <int NE, int WF>
 cudaError_t expand_launch(const ExpandJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,
                           int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
                           float scale, int32_t y_dtype, const InlineTable<kInlineItems>* inl, bool y_early,
@@ -801,16 +832,16 @@ cudaError_t expand_launch(const ExpandJob* jobs, int n_jobs, const BatchView& b,
     int order[kMaxGroup];
     for (int j = 0; j < n_jobs; ++j) order[j] = j;
     std::stable_sort(order, order + n_jobs, [&](int u, int w) { return jobs[u].d_out > jobs[w].d_out; });
-    auto kern_inl = pick(max_item_rows, expand_simt_kernel<1, kInlineItems, NE>, expand_simt_kernel<2, kInlineItems, NE>,
-                         expand_simt_kernel<4, kInlineItems, NE>);
-    auto kern_tab = pick(max_item_rows, expand_simt_kernel<1, 1, NE>, expand_simt_kernel<2, 1, NE>,
-                         expand_simt_kernel<4, 1, NE>);
+    auto kern_inl = pick(max_item_rows, expand_simt_kernel<1, kInlineItems, NE, WF>,
+                         expand_simt_kernel<2, kInlineItems, NE, WF>, expand_simt_kernel<4, kInlineItems, NE, WF>);
+    auto kern_tab = pick(max_item_rows, expand_simt_kernel<1, 1, NE, WF>, expand_simt_kernel<2, 1, NE, WF>,
+                         expand_simt_kernel<4, 1, NE, WF>);
     const void* kp = inl ? reinterpret_cast<const void*>(kern_inl) : reinterpret_cast<const void*>(kern_tab);
     const int mr = std::max(8, max_rank);
-    auto smem_for = [&](int npass) {
+    auto smem_for = [&](int npass) {  // v of the item, row scales, page ids, ring
         const size_t pid_bytes = (size_t)mr * ((npass * kPass) >> pool.page_log2) * 4;
-        return (((size_t)kSimtMaxItemRows * mr * 4 + pid_bytes + 127) & ~(size_t)127) +
-               (size_t)kExpandStages * kStageElems * 2;
+        return (((size_t)kSimtMaxItemRows * mr * 4 + kMaxRank * 4 + pid_bytes + 127) & ~(size_t)127) +
+               (size_t)kExpandStages * stage_bytes<WF>();
     };
     int tiles[kMaxGroup], max_tiles = 1;
     for (int j = 0; j < n_jobs; ++j) {
@@ -856,7 +887,7 @@ cudaError_t expand_launch(const ExpandJob* jobs, int n_jobs, const BatchView& b,
     a.max_rank = mr;
     a.stages = kExpandStages;
     const size_t smem = smem_for(max_np);
-    a.ring_offset = (int)(smem - (size_t)kExpandStages * kStageElems * 2);
+    a.ring_offset = (int)(smem - (size_t)kExpandStages * stage_bytes<WF>());
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)ctas, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -883,9 +914,19 @@ cudaError_t launch_shrink_simt(const ShrinkJob* jobs, int n_jobs, const BatchVie
     if (num_items <= 0 || n_jobs <= 0) return cudaSuccess;
     if (n_jobs > kMaxGroup || (inl && n_jobs > 1)) return cudaErrorInvalidValue;
     // one projection: a one-entry table (small launch arguments, no per-CTA lookup)
-    if (n_jobs == 1)
-        return shrink_launch<1>(jobs, n_jobs, b, num_items, max_item_rows, max_rank, work, pool, inl, stream);
-    return shrink_launch<kMaxGroup>(jobs, n_jobs, b, num_items, max_item_rows, max_rank, work, pool, inl, stream);
+    auto go = [&](auto wf) {
+        constexpr int WF = decltype(wf)::value;
+        if (n_jobs == 1)
+            return shrink_launch<1, WF>(jobs, n_jobs, b, num_items, max_item_rows, max_rank, work, pool, inl, stream);
+        return shrink_launch<kMaxGroup, WF>(jobs, n_jobs, b, num_items, max_item_rows, max_rank, work, pool, inl,
+                                            stream);
+    };
+    switch (pool.wfmt) {
+        case kFmtBf16: return go(std::integral_constant<int, kFmtBf16>{});
+        case kFmtFp8: return go(std::integral_constant<int, kFmtFp8>{});
+        case kFmtInt4: return go(std::integral_constant<int, kFmtInt4>{});
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t launch_expand_simt(const ExpandJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,
@@ -894,11 +935,20 @@ cudaError_t launch_expand_simt(const ExpandJob* jobs, int n_jobs, const BatchVie
                                cudaStream_t stream) {
     if (num_items <= 0 || n_jobs <= 0) return cudaSuccess;
     if (n_jobs > kMaxGroup || (inl && n_jobs > 1)) return cudaErrorInvalidValue;
-    if (n_jobs == 1)
-        return expand_launch<1>(jobs, n_jobs, b, num_items, max_item_rows, max_rank, work, pool, scale, y_dtype, inl,
-                                y_early, stream);
-    return expand_launch<kMaxGroup>(jobs, n_jobs, b, num_items, max_item_rows, max_rank, work, pool, scale, y_dtype,
-                                    inl, y_early, stream);
+    auto go = [&](auto wf) {
+        constexpr int WF = decltype(wf)::value;
+        if (n_jobs == 1)
+            return expand_launch<1, WF>(jobs, n_jobs, b, num_items, max_item_rows, max_rank, work, pool, scale,
+                                        y_dtype, inl, y_early, stream);
+        return expand_launch<kMaxGroup, WF>(jobs, n_jobs, b, num_items, max_item_rows, max_rank, work, pool, scale,
+                                            y_dtype, inl, y_early, stream);
+    };
+    switch (pool.wfmt) {
+        case kFmtBf16: return go(std::integral_constant<int, kFmtBf16>{});
+        case kFmtFp8: return go(std::integral_constant<int, kFmtFp8>{});
+        case kFmtInt4: return go(std::integral_constant<int, kFmtInt4>{});
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t read_clear_errors_simt(uint32_t* bits, cudaStream_t stream) {

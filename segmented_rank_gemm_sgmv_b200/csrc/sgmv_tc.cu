@@ -26,6 +26,7 @@
 #include <algorithm>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -81,6 +82,29 @@ __device__ __forceinline__ int32_t safe_page(const PoolView& pool, int64_t entry
     return page;
 }
 
+// Codes of a quantised pool: 8 values (8 bytes E4M3 / 4 bytes INT4) of a page,
+// read through the non-coherent path, and their exact bf16 form (16 bytes).
+template <int WF>
+struct Codes8 {
+    using T = typename std::conditional<WF == kFmtFp8, uint2, uint32_t>::type;
+};
+template <int WF>
+__device__ __forceinline__ typename Codes8<WF>::T load_codes8(const uint8_t* p) {
+    return __ldg(reinterpret_cast<const typename Codes8<WF>::T*>(p));
+}
+template <int WF>
+__device__ __forceinline__ uint4 codes8_to_bf16(const typename Codes8<WF>::T& c) {
+    float f[8];
+    if constexpr (WF == kFmtFp8) fp8x8_to_f32(c, f);
+    else int4x8_to_f32(c, f);
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)  // exact: every code value has at most 4 significant bits
+        w[e] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f[2 * e])) |
+               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f[2 * e + 1])) << 16);
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // ------------------------------------------------------------------ shrink
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     const uint32_t s = smem_u32(p);
@@ -94,6 +118,7 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // once the MMAs that read it have completed (tcgen05.commit).  Every wait is
 // bounded; a wait that gives up sets kErrTimeout and the CTA's abort flag, and
 // the remaining waits of the CTA are skipped.
+template <int WF>
 __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkTcArgs a,
                                                                      const __grid_constant__ CUtensorMap tmap_x) {
     extern __shared__ uint8_t smem_raw[];
@@ -102,6 +127,7 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
     __shared__ uint32_t tmem_slot;
     __shared__ volatile int abort_flag;
     __shared__ int32_t tok_s[kTcTileRows];
+    __shared__ float rsc_s[kMaxRank];  // row scales of a quantised A
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int tile_idx = blockIdx.x / a.ks;
@@ -126,8 +152,10 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
 
     if (tid == 0) {
         abort_flag = 0;
+        // full: the producers' cp.async arrivals, plus (quantised pools) their arrivals
+        // after storing the converted A codes
         for (int i = 0; i < kShrinkStages; ++i) {
-            mbar_init(&full_bar[i], kTcTileRows);
+            mbar_init(&full_bar[i], WF == kFmtBf16 ? kTcTileRows : 2 * kTcTileRows);
             mbar_init(&empty_bar[i], 1);
         }
         mbar_init(&acc_bar, 1);
@@ -164,6 +192,11 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
         const int n = e / span_pages, pc = e - n * span_pages;
         pid_s[e] = safe_page(a.pool, a_base + (int64_t)n * pages_per_row + first_page + pc);
     }
+    if (WF != kFmtBf16)
+        for (int n = tid; n < r; n += kShrinkThreads) {
+            const int64_t e = a_base + (int64_t)n * pages_per_row;
+            rsc_s[n] = (e >= 0 && e < a.pool.pt_capacity) ? a.pool.row_scale[e] : 0.f;
+        }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -206,14 +239,40 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
             }
             // A: rank rows n < npad, zero past r; the 64 columns lie in one page
             const int page_rel = (c >> P_log2) - first_page, in_page = c & ((1 << P_log2) - 1);
-            for (int g = tid; g < npad * 8; g += kTcTileRows) {
-                const int n = g >> 3, kg = g & 7;
-                const uint32_t off = (uint32_t)(n >> 3) * 1024 + sw128_off((uint32_t)n, (uint32_t)kg);
-                const bool valid = ok && n < r;
-                const uint16_t* src = a.pool.pages;
-                if (valid)
-                    src = a.pool.pages + ((int64_t)pid_s[n * span_pages + page_rel] << P_log2) + in_page + kg * 8;
-                cp_async16(as + off, src, valid);
+            if constexpr (WF == kFmtBf16) {
+                for (int g = tid; g < npad * 8; g += kTcTileRows) {
+                    const int n = g >> 3, kg = g & 7;
+                    const uint32_t off = (uint32_t)(n >> 3) * 1024 + sw128_off((uint32_t)n, (uint32_t)kg);
+                    const bool valid = ok && n < r;
+                    const uint16_t* src = a.pool.pages;
+                    if (valid)
+                        src = a.pool.pages + ((int64_t)pid_s[n * span_pages + page_rel] << P_log2) + in_page + kg * 8;
+                    cp_async16(as + off, src, valid);
+                }
+            } else {
+                // codes through registers: all loads in flight, then converted to bf16 and
+                // stored; the stores reach the tensor core through the async proxy
+                constexpr int VB = bytes_per_8<WF>();
+                const int page_shift = P_log2 + (WF == kFmtFp8 ? 0 : -1);
+                const uint8_t* pages8 = reinterpret_cast<const uint8_t*>(a.pool.pages);
+                typename Codes8<WF>::T cw[kMaxRank * 8 / kTcTileRows];
+#pragma unroll
+                for (int i = 0; i < kMaxRank * 8 / kTcTileRows; ++i) {
+                    const int g = tid + i * kTcTileRows, n = g >> 3, kg = g & 7;
+                    cw[i] = typename Codes8<WF>::T{};
+                    if (g < npad * 8 && ok && n < r)
+                        cw[i] = load_codes8<WF>(pages8 + ((int64_t)pid_s[n * span_pages + page_rel] << page_shift) +
+                                                (in_page / 8 + kg) * VB);
+                }
+#pragma unroll
+                for (int i = 0; i < kMaxRank * 8 / kTcTileRows; ++i) {
+                    const int g = tid + i * kTcTileRows, n = g >> 3, kg = g & 7;
+                    if (g < npad * 8)
+                        *reinterpret_cast<uint4*>(as + (uint32_t)(n >> 3) * 1024 +
+                                                  sw128_off((uint32_t)n, (uint32_t)kg)) = codes8_to_bf16<WF>(cw[i]);
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&full_bar[st]);
             }
             cp_async_commit();  // close the group: the copies of every stage form their own
             cp_async_mbar_arrive_noinc(&full_bar[st]);
@@ -274,7 +333,8 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
             float sum = 0.f;
 #pragma unroll
             for (int qq = 0; qq < 8; ++qq) sum += pv[qq];
-            a.v[(int64_t)(it.row_begin + mm) * a.ldv + k] = sum;
+            // a quantised row's scale leaves the sum: v_k = s_k * sum_c q_kc x_c
+            a.v[(int64_t)(it.row_begin + mm) * a.ldv + k] = WF == kFmtBf16 ? sum : sum * rsc_s[k];
         }
     }
     cluster_sync();
@@ -311,7 +371,7 @@ constexpr int kExpandProducers = 128;
 constexpr int kMmaWarp = 12;
 constexpr int kMaxExpandStages = 3;
 
-template <int S, int ESZ>  // ESZ: bytes of a y element (2: bf16, 4: fp32)
+template <int S, int ESZ, int WF>  // ESZ: bytes of a y element (2: bf16, 4: fp32); WF: weight format
 __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const ExpandTcArgs a,
                                                                       const __grid_constant__ CUtensorMap tmap_y) {
     extern __shared__ uint8_t smem_raw[];
@@ -322,6 +382,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
     __shared__ int32_t pid_s[S][kMaxRank * kMaxPagesPerUnit];  // B^T page ids of a unit [rank row][page]
     __shared__ int32_t tok_s[S][kTcTileRows];                    // producers: token of each row of a unit
     __shared__ int32_t tok_row[2][kTcTileRows];                  // epilogue groups: token of each row, -1 = none
+    __shared__ float rsc_s[kMaxRank];                            // producers: row scales of a quantised B^T
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int u0 = blockIdx.x * a.units_per_cta, u1 = min(u0 + a.units_per_cta, a.num_units);
@@ -346,8 +407,10 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
 
     if (tid == 0) {
         abort_flag = 0;
+        // full: the producers' cp.async arrivals, plus (quantised pools) their arrivals
+        // after storing the converted B^T codes
         for (int i = 0; i < S; ++i) {
-            mbar_init(&full_bar[i], kExpandProducers);
+            mbar_init(&full_bar[i], WF == kFmtBf16 ? kExpandProducers : 2 * kExpandProducers);
             mbar_init(&yfree_bar[i], kTcTileRows);  // one epilogue group per unit
         }
         for (int i = 0; i < 2; ++i) {
@@ -435,6 +498,13 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
             if (i >= S) wait(&yfree_bar[st], (uint32_t)((i / S - 1) & 1));
             if (w.ok && w.tile != cur_tile) {
                 if (ts >= 0) wait(&vempty_bar, (uint32_t)(ts & 1));  // the MMAs of the previous tile are done
+                if (WF != kFmtBf16) {  // v_k takes the scale of B^T row k
+                    if (pt < w.r) {
+                        const int64_t e = w.b_base + (int64_t)pt * pages_per_row;
+                        rsc_s[pt] = (e >= 0 && e < a.pool.pt_capacity) ? a.pool.row_scale[e] : 0.f;
+                    }
+                    named_bar_sync(1, kExpandProducers);
+                }
                 const int m = pt, kpad = (w.r + 15) & ~15;
                 const bool row_ok = m < w.rows;
                 const float* vrow = a.v + (int64_t)(w.row_begin + (row_ok ? m : 0)) * a.ldv;
@@ -457,8 +527,10 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
                     f[0] = q0.x; f[1] = q0.y; f[2] = q0.z; f[3] = q0.w;
                     f[4] = q1.x; f[5] = q1.y; f[6] = q1.z; f[7] = q1.w;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
+                    for (int e = 0; e < 8; ++e) {
                         if (kg * 8 + e >= w.r) f[e] = 0.f;
+                        else if (WF != kFmtBf16) f[e] *= rsc_s[kg * 8 + e];
+                    }
                     uint32_t hw[4], lw[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -509,23 +581,56 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
                 // B^T block: granule (k, jg) = B^T[k][j0 + 8 jg .. +8], zero past r
                 uint8_t* bs = bst + (size_t)st * b_bytes;
                 const int kpad = (w.r + 15) & ~15;
+                constexpr int kGr = kMaxRank * (kYRowBytes / 16) / kExpandProducers;  // <= 16 granules a thread
+                if constexpr (WF == kFmtBf16) {
 #pragma unroll
-                for (int gi = 0; gi < kMaxRank * (kYRowBytes / 16) / kExpandProducers; ++gi) {  // <= 16 granules a row
-                    const int g = pt + gi * kExpandProducers;
-                    if (g >= kpad * (NB / 8)) break;
-                    const int jg = g % (NB / 8), k = g / (NB / 8);
-                    const int j = w.j0 + jg * 8;
-                    const uint32_t off = (uint32_t)(k >> 3) * sbo_b + (uint32_t)(jg >> 3) * 1024 +
-                                         sw128_off((uint32_t)k, (uint32_t)jg);
-                    const bool valid = k < w.r;
-                    const uint16_t* src = a.pool.pages;
-                    if (valid)
-                        src = a.pool.pages + ((int64_t)pid_s[st][k * npc + ((j - w.j0) >> P_log2)] << P_log2) +
-                              (j & ((1 << P_log2) - 1));
-                    cp_async16(bs + off, src, valid);
+                    for (int gi = 0; gi < kGr; ++gi) {
+                        const int g = pt + gi * kExpandProducers;
+                        if (g >= kpad * (NB / 8)) break;
+                        const int jg = g % (NB / 8), k = g / (NB / 8);
+                        const int j = w.j0 + jg * 8;
+                        const uint32_t off = (uint32_t)(k >> 3) * sbo_b + (uint32_t)(jg >> 3) * 1024 +
+                                             sw128_off((uint32_t)k, (uint32_t)jg);
+                        const bool valid = k < w.r;
+                        const uint16_t* src = a.pool.pages;
+                        if (valid)
+                            src = a.pool.pages + ((int64_t)pid_s[st][k * npc + ((j - w.j0) >> P_log2)] << P_log2) +
+                                  (j & ((1 << P_log2) - 1));
+                        cp_async16(bs + off, src, valid);
+                    }
+                } else {
+                    // codes through registers (all loads in flight), converted to bf16 and stored
+                    constexpr int VB = bytes_per_8<WF>();
+                    const int page_shift = P_log2 + (WF == kFmtFp8 ? 0 : -1);
+                    const uint8_t* pages8 = reinterpret_cast<const uint8_t*>(a.pool.pages);
+                    typename Codes8<WF>::T cw[kGr];
+#pragma unroll
+                    for (int gi = 0; gi < kGr; ++gi) {
+                        const int g = pt + gi * kExpandProducers;
+                        const int jg = g % (NB / 8), k = g / (NB / 8);
+                        const int j = w.j0 + jg * 8;
+                        cw[gi] = typename Codes8<WF>::T{};
+                        if (g < kpad * (NB / 8) && k < w.r)
+                            cw[gi] = load_codes8<WF>(
+                                pages8 + ((int64_t)pid_s[st][k * npc + ((j - w.j0) >> P_log2)] << page_shift) +
+                                ((j & ((1 << P_log2) - 1)) / 8) * VB);
+                    }
+#pragma unroll
+                    for (int gi = 0; gi < kGr; ++gi) {
+                        const int g = pt + gi * kExpandProducers;
+                        if (g >= kpad * (NB / 8)) break;
+                        const int jg = g % (NB / 8), k = g / (NB / 8);
+                        const uint32_t off = (uint32_t)(k >> 3) * sbo_b + (uint32_t)(jg >> 3) * 1024 +
+                                             sw128_off((uint32_t)k, (uint32_t)jg);
+                        *reinterpret_cast<uint4*>(bs + off) = codes8_to_bf16<WF>(cw[gi]);
+                    }
                 }
             } else if (pt == 0) {
                 atomicOr(&g_err_tc, kErrRows);
+            }
+            if (WF != kFmtBf16) {  // the converted codes, to the async proxy, then the second arrival
+                fence_proxy_async_smem();
+                mbar_arrive(&full_bar[st]);
             }
             cp_async_commit();
             cp_async_mbar_arrive_noinc(&full_bar[st]);
@@ -740,7 +845,9 @@ cudaError_t launch_shrink_tc(const uint16_t* x, int64_t ldx, int32_t d_in, const
     // >= 80 KB: at most two CTAs per SM, so tensor memory is never oversubscribed
     const size_t smem = std::max(main_bytes + pid_bytes, (size_t)80 << 10) + 1024;
     if (smem > (227u << 10)) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(shrink_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = pool.wfmt == kFmtFp8 ? shrink_tc_kernel<kFmtFp8>
+                : pool.wfmt == kFmtInt4 ? shrink_tc_kernel<kFmtInt4> : shrink_tc_kernel<kFmtBf16>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(ks * num_tiles), 1, 1);
@@ -758,7 +865,7 @@ cudaError_t launch_shrink_tc(const uint16_t* x, int64_t ldx, int32_t d_in, const
     std::memset(&tmap_x, 0, sizeof(tmap_x));
     a.use_tma = encode_2d(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)d_in, (uint64_t)b.T,
                           (uint64_t)ldx * 2, kKTile, kTcTileRows) ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, shrink_tc_kernel, a, tmap_x);
+    return cudaLaunchKernelEx(&cfg, kern, a, tmap_x);
 }
 
 cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const BatchView& b, int32_t num_tiles,
@@ -805,8 +912,14 @@ cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const B
     const int esz = y_dtype == 0 ? 2 : 4;
     a.use_tma = encode_2d(&tmap_y, y_dtype == 0 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, y,
                           (uint64_t)d_out, (uint64_t)b.T, (uint64_t)ldy * esz, (uint32_t)(NB / 2), kTcTileRows) ? 1 : 0;
-    auto kern = S == 3 ? (esz == 2 ? expand_tc_kernel<3, 2> : expand_tc_kernel<3, 4>)
-                       : (esz == 2 ? expand_tc_kernel<2, 2> : expand_tc_kernel<2, 4>);
+    auto pick = [&](auto wf) {
+        constexpr int WF = decltype(wf)::value;
+        return S == 3 ? (esz == 2 ? expand_tc_kernel<3, 2, WF> : expand_tc_kernel<3, 4, WF>)
+                      : (esz == 2 ? expand_tc_kernel<2, 2, WF> : expand_tc_kernel<2, 4, WF>);
+    };
+    auto kern = pool.wfmt == kFmtFp8    ? pick(std::integral_constant<int, kFmtFp8>{})
+                : pool.wfmt == kFmtInt4 ? pick(std::integral_constant<int, kFmtInt4>{})
+                                        : pick(std::integral_constant<int, kFmtBf16>{});
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)blocks, kExpandThreads, smem, stream>>>(a, tmap_y);

@@ -7,6 +7,9 @@ Tolerances (written here, used by every parity test):
   Gate A:  bf16 y rows   ||y_gpu - bf16(y_ref)|| / ||bf16(y_ref)||
   Gate B:  fp32 y rows   ||y_gpu - y_ref|| / ||y_ref - y_in||   (relative to the delta itself)
 Rows of tokens that use no adapter (or a rank-0 adapter) must be bit-identical to y_in.
+
+Quantised pools (weight_format "fp8_e4m3" / "int4"): the oracle computes the delta with
+the dequantised weights of oracle/quant.py (codes x row scale, fp64), under the same gates.
 """
 from __future__ import annotations
 
@@ -17,6 +20,7 @@ import numpy as np
 import torch
 
 import oracle
+from oracle import quant as oquant
 import segmented_rank_gemm_sgmv_b200 as sg
 import workloads
 
@@ -24,11 +28,12 @@ GATE_REL = 1e-3
 
 
 def build_pool(wl: workloads.Workload, bank: workloads.AdapterBank, page_elems: int = 512,
-               shuffle_seed: Optional[int] = 1, extra_pages: int = 64) -> sg.AdapterPool:
+               shuffle_seed: Optional[int] = 1, extra_pages: int = 64, weight_format: str = "bf16") -> sg.AdapterPool:
     projs = [(d_in, d_out) for _, d_in, d_out in wl.projections]
     need = sum(sg.AdapterPool.pages_needed(projs, int(r), page_elems) for r in wl.pool_ranks)
     pool = sg.AdapterPool(projs, num_pages=need + extra_pages, page_elems=page_elems,
-                          max_rank=max(16, int(wl.pool_ranks.max(initial=0))), device=0)
+                          max_rank=max(16, int(wl.pool_ranks.max(initial=0))), device=0,
+                          weight_format=weight_format)
     if shuffle_seed is not None:
         pool.shuffle_free_pages(shuffle_seed)
     for a, r in zip(wl.pool_ids.tolist(), wl.pool_ranks.tolist()):
@@ -59,8 +64,19 @@ def run_gpu(pool, wl, proj, x, y, long_threshold=0, y_dtype=torch.bfloat16, scal
     return plan, v, y_out
 
 
+def oracle_weights(bank, a, proj, weight_format: str = "bf16"):
+    """(A, B) of adapter a for the oracle, float64: the bf16 values, or their quantised and
+    dequantised form (oracle/quant.py) for a quantised pool."""
+    A16, B16 = bank.get(a, proj)
+    A, B = workloads.bf16_to_f64(A16), workloads.bf16_to_f64(B16)
+    if weight_format == "bf16":
+        return A, B
+    *_, Ad, Bd = oquant.quantize_adapter(A.astype(np.float32), B.astype(np.float32), weight_format)
+    return Ad, Bd
+
+
 def run_oracle(wl, bank, proj, x, y, rows_of_tokens: Optional[List[int]] = None, scale=None,
-               adapter_ids=None, threads: int = 0):
+               adapter_ids=None, threads: int = 0, weight_format: str = "bf16"):
     """fp64 oracle on the whole batch, or on the listed tokens only (each token's
     result depends only on its own row and adapter)."""
     ids = (wl.adapter_ids if adapter_ids is None else adapter_ids).tolist()
@@ -70,8 +86,9 @@ def run_oracle(wl, bank, proj, x, y, rows_of_tokens: Optional[List[int]] = None,
         sub_ids = [a if t in keep else -1 for t, a in enumerate(ids)]
         tix, off, seg_ad = oracle.group_by_adapter(sub_ids)
     ranks = [wl.rank_of(a) for a in seg_ad]
-    A = [workloads.bf16_to_f64(bank.get(a, proj)[0]) for a in seg_ad]
-    B = [workloads.bf16_to_f64(bank.get(a, proj)[1]) for a in seg_ad]
+    AB = [oracle_weights(bank, a, proj, weight_format) for a in seg_ad]
+    A = [ab[0] for ab in AB]
+    B = [ab[1] for ab in AB]
     v_ref, y_ref = oracle.lora_delta(workloads.bf16_to_f64(x), workloads.bf16_to_f64(y), off, ranks, A, B,
                                      token_idx=tix, scale=wl.scale if scale is None else scale,
                                      threads=threads or (os.cpu_count() or 1))

@@ -37,7 +37,7 @@ def _rank_main(rank, world, port, out):
         out[world + rank] = float(wl.T)
         out[2 * world + rank] = float(int(wl.adapter_ids.astype(np.int64).sum()))
         # the reference arm prints its line on rank 0 only
-        args = argparse.Namespace(workload="tiny", steps=1, warmup=1, cpu_budget=0.05, ref_budget=0.2)
+        args = argparse.Namespace(workload="tiny", steps=1, warmup=1, cpu_budget=0.05, ref_budget=0.2, weights="bf16")
         buf = io.StringIO()
         with contextlib.redirect_stdout(buf):
             bench.run_reference(args, rank, world, 0)

@@ -103,15 +103,17 @@ constexpr int kFmtBf16 = 0, kFmtFp8 = 1, kFmtInt4 = 2;
 template <int WF>
 __host__ __device__ constexpr int bytes_per_8() { return WF == kFmtBf16 ? 16 : WF == kFmtFp8 ? 8 : 4; }
 
+// 40 bytes, part of every kernel's parameters (page ids are int32, so is the page count).
 struct PoolView {
     const uint16_t* pages;       // bf16 pages; a quantised pool's code pages as the same buffer
     const int32_t* page_table;
     const float* row_scale;      // quantised pools: scale of each rank row (first-chunk entry)
-    int64_t num_pages;
     int64_t pt_capacity;
-    int32_t page_log2;
-    int32_t wfmt;
+    int32_t num_pages;
+    int16_t page_log2;
+    int16_t wfmt;                // sgmv_weight_format
 };
+static_assert(sizeof(PoolView) == 40, "PoolView must stay 40 bytes");
 
 // --------------------------------------------------------------- launchers
 // Work of the SIMT items, in stages of 8 rank rows: `sum_ng` over the items,

@@ -328,6 +328,26 @@ __device__ __forceinline__ void int4x8_to_f32(uint32_t q, float (&f)[8]) {
     for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(0x4B000000u | ((flipped >> (4 * i)) & 0xFu)) - 8388616.0f;
 }
 
+// Eight INT4 codes as position-scaled fp32: f[i] = q_i * 16^(i % 4), exactly, in two
+// operations a value.  With n = nibble ^ 8, the float with bits 0x4B000000 | (n << 4j)
+// (j = i % 4, the nibble kept in place inside the low 16 bits) is 2^23 + n 16^j, an
+// integer below 2^24; subtracting 2^23 + 8 * 16^j is exact and leaves (n - 8) 16^j.
+// The caller undoes the factor 16^j on the other operand (x) or on the sum, both exact
+// power-of-two scalings.
+__device__ __forceinline__ void int4x8_to_f32_pos(uint32_t q, float (&f)[8]) {
+    const uint32_t lo = q ^ 0x88888888u, hi = lo >> 16;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float c = 8388608.0f + 8.0f * (float)(1u << (4 * i));
+        f[i] = __uint_as_float(0x4B000000u | (lo & (0xFu << (4 * i)))) - c;
+        f[i + 4] = __uint_as_float(0x4B000000u | (hi & (0xFu << (4 * i)))) - c;
+    }
+}
+// 16^-(i % 4): the factor that int4x8_to_f32_pos leaves on value i
+__device__ __forceinline__ float int4_pos_unscale(int i) {
+    return i % 4 == 0 ? 1.0f : i % 4 == 1 ? 0.0625f : i % 4 == 2 ? 0.00390625f : 0.000244140625f;
+}
+
 // Eight stored weights of format WF at p (16, 8 or 4 bytes) to fp32.
 template <int WF>
 __device__ __forceinline__ void load_w8(const uint8_t* p, float (&f)[8]) {

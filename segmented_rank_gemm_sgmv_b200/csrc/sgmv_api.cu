@@ -58,11 +58,11 @@ sgmv_status make_views(const sgmv_plan* plan, const void* table, const sgmv_pool
     bv->T = T;
     pv->pages = static_cast<const uint16_t*>(pool->pages_dev);
     pv->page_table = pool->pt_dev;
-    pv->num_pages = pool->num_pages;
+    pv->num_pages = (int32_t)pool->num_pages;
     pv->pt_capacity = pool->pt_capacity;
-    pv->page_log2 = pool->page_log2;
+    pv->page_log2 = (int16_t)pool->page_log2;
     pv->row_scale = pool->scale_dev;
-    pv->wfmt = pool->wfmt;
+    pv->wfmt = (int16_t)pool->wfmt;
     return SGMV_OK;
 }
 

@@ -287,17 +287,35 @@ __device__ __forceinline__ void pipe_issue(const PoolView& pool, Pipe<kStages, W
         const int32_t* pidg = sg.pid + kRowGroup * g * sg.span_pages;
         // a page is (1 << P_log2) values, (1 << page_shift) bytes; column c of it at byte c * VB / 8
         const int page_shift = P_log2 + (VB == 16 ? 1 : VB == 8 ? 0 : -1);
-        if (W == kPass) {  // full pass: thread t copies granule t of each of the stage's rows
+        if constexpr (WF != kFmtBf16) {
+            // codes: 16-byte copies (16 E4M3 / 32 INT4 values; a row of the stage is W * VB / 8
+            // bytes, a multiple of 32 since W is a multiple of 64), consecutive threads on
+            // consecutive granules of a row; the consumers read the same bytes 8 values a thread
+            constexpr int kVals16 = 128 / VB;                  // values per 16-byte granule
+            const int gpr = W / kVals16;                       // granules per row
+#pragma unroll
+            for (int i = 0; i < stage_bytes<WF>() / 16 / kThreads; ++i) {
+                const int gi = threadIdx.x + kThreads * i;
+                const int kk = gi / gpr, cg = gi - kk * gpr;
+                if (kk < rows) {
+                    const int col = c + cg * kVals16;
+                    const int32_t page = pidg[kk * sg.span_pages + (col >> P_log2)];
+                    cp_async16(dst0 + (size_t)kk * (W / 8 * VB) + cg * 16,
+                               pages + ((int64_t)page << page_shift) + (col & (P - 1)) / 8 * VB, true);
+                }
+            }
+        } else if (W == kPass) {  // full pass: thread t copies granule t of each of the stage's rows
             const int col = c + kVec * threadIdx.x;
             const int32_t* pidc = pidg + (col >> P_log2);
-            const uint8_t* src0 = pages + ((col & (P - 1)) / 8 * VB);
-            uint8_t* dst = dst0 + VB * threadIdx.x;
+            const uint16_t* src0 = pool.pages + (col & (P - 1));
+            uint16_t* dst = reinterpret_cast<uint16_t*>(dst0) + kVec * threadIdx.x;
 #pragma unroll
             for (int kk = 0; kk < kRowGroup; ++kk)
                 if (kk < rows)
-                    cp_async_n<VB>(dst + kk * (kPass / 8 * VB), src0 + ((int64_t)pidc[kk * sg.span_pages] << page_shift));
+                    cp_async16(dst + kk * kPass, src0 + ((int64_t)pidc[kk * sg.span_pages] << P_log2), true);
         } else {
             const int gpr = W >> 3;  // granules (8 values) per row
+            uint16_t* d0 = reinterpret_cast<uint16_t*>(dst0);
 #pragma unroll
             for (int i = 0; i < kStageElems / 8 / kThreads; ++i) {
                 const int gi = threadIdx.x + kThreads * i;
@@ -305,8 +323,8 @@ __device__ __forceinline__ void pipe_issue(const PoolView& pool, Pipe<kStages, W
                 if (kk < rows) {
                     const int col = c + cg * 8;
                     const int32_t page = pidg[kk * sg.span_pages + (col >> P_log2)];
-                    cp_async_n<VB>(dst0 + ((size_t)kk * W / 8 + cg) * VB,
-                                   pages + ((int64_t)page << page_shift) + (col & (P - 1)) / 8 * VB);
+                    cp_async16(d0 + (size_t)kk * W + cg * 8, pool.pages + ((int64_t)page << P_log2) + (col & (P - 1)),
+                               true);
                 }
             }
         }
@@ -389,10 +407,21 @@ __device__ void shrink_item(const PoolView& pool, const ItemInfo& m, Pipe<kStage
                 float xf[G][8];
 #pragma unroll
                 for (int j = 0; j < G; ++j) unpack8(*reinterpret_cast<const uint4*>(xst + j * kPass), xf[j]);
+                if constexpr (WF == kFmtInt4) {  // INT4 codes arrive scaled by 16^(e % 4): x takes the inverse
+#pragma unroll
+                    for (int j = 0; j < G; ++j)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) xf[j][e] *= int4_pos_unscale(e);
+                }
 #pragma unroll
                 for (int kk = 0; kk < kRowGroup; ++kk) {
                     float af[8];
-                    load_w8<WF>(st + ((size_t)kk * (W >> 3) + tid) * VB, af);
+                    if constexpr (WF == kFmtBf16)
+                        unpack8(*reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(st) + (size_t)kk * W + col), af);
+                    else if constexpr (WF == kFmtInt4)
+                        int4x8_to_f32_pos(*reinterpret_cast<const uint32_t*>(st + ((size_t)kk * (W >> 3) + tid) * VB), af);
+                    else
+                        load_w8<WF>(st + ((size_t)kk * (W >> 3) + tid) * VB, af);
 #pragma unroll
                     for (int j = 0; j < G; ++j) p[kk * G + j] += dot8(af, xf[j]);
                 }
@@ -424,8 +453,8 @@ __global__ void __launch_bounds__(kThreads, 3)
     const int slot = kSimtMaxItemRows * a.max_rank;  // floats of one partial tile
     float* part = reinterpret_cast<float*>(smem);     // [C slots][slot]; slot 0 is this CTA's own
     float* red = part + C * slot;                      // [4 warps][64]
-    float* rsc = red + 4 * 64;                         // [kMaxRank] row scales (quantised pools)
-    int32_t* pid = reinterpret_cast<int32_t*>(rsc + kMaxRank);
+    float* rsc = red + 4 * 64;                         // [kMaxRank] row scales (quantised pools only)
+    int32_t* pid = reinterpret_cast<int32_t*>(rsc + (WF == kFmtBf16 ? 0 : kMaxRank));
 
     const ItemInfo m = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 0)
                               : load_item(a.b, en.proj, item_idx, MAXG, a.max_rank, 0);
@@ -548,7 +577,12 @@ __device__ void expand_item(const ExpandArgs<NE>& a, const ExpandEntry& en, cons
                     const int k = kRowGroup * g + kk;
                     if (k < m.r) {
                         float bf[8];
-                        load_w8<WF>(st + ((size_t)kk * (W >> 3) + tid) * VB, bf);
+                        if constexpr (WF == kFmtBf16)
+                            unpack8(*reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(st) + (size_t)kk * W + col), bf);
+                        else if constexpr (WF == kFmtInt4)  // scaled by 16^(e % 4), undone on the sums
+                            int4x8_to_f32_pos(*reinterpret_cast<const uint32_t*>(st + ((size_t)kk * (W >> 3) + tid) * VB), bf);
+                        else
+                            load_w8<WF>(st + ((size_t)kk * (W >> 3) + tid) * VB, bf);
 #pragma unroll
                         for (int j = 0; j < G; ++j) {
                             const float w = vs[min(j, m.n - 1) * m.r + k];
@@ -559,6 +593,12 @@ __device__ void expand_item(const ExpandArgs<NE>& a, const ExpandEntry& en, cons
                 }
             }
             pipe_release(a.pool, pp, sg, true, XStage{});
+        }
+        if constexpr (WF == kFmtInt4) {
+#pragma unroll
+            for (int j = 0; j < G; ++j)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[j][e] *= int4_pos_unscale(e);
         }
 #pragma unroll
         for (int j = 0; j < G; ++j) {
@@ -608,8 +648,8 @@ __global__ void __launch_bounds__(kThreads, 3)
     const int local = (int)blockIdx.x - en.cta_base;
     const int part_idx = local % en.cpi, item_idx = local / en.cpi;
     float* vs = reinterpret_cast<float*>(smem_e);
-    float* rsc = vs + kSimtMaxItemRows * a.max_rank;  // [kMaxRank] row scales (quantised pools)
-    int32_t* pid = reinterpret_cast<int32_t*>(rsc + kMaxRank);
+    float* rsc = vs + kSimtMaxItemRows * a.max_rank;  // [kMaxRank] row scales (quantised pools only)
+    int32_t* pid = reinterpret_cast<int32_t*>(rsc + (WF == kFmtBf16 ? 0 : kMaxRank));
 
     const ItemInfo m = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 1)
                               : load_item(a.b, en.proj, item_idx, MAXG, a.max_rank, 1);
@@ -761,7 +801,8 @@ cudaError_t shrink_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b,
     auto smem_for = [&](int c) {  // partial tiles, reduction scratch, row scales, page ids, ring
         const size_t part_bytes = (size_t)c * kSimtMaxItemRows * mr * 4;
         const size_t pidb = (size_t)mr * ((max_pages + c - 1) / c) * 4;
-        return (((part_bytes + 1024 + kMaxRank * 4 + pidb + 127) & ~(size_t)127)) + ring_bytes;
+        const size_t rsc_bytes = WF == kFmtBf16 ? 0 : kMaxRank * 4;
+        return (((part_bytes + 1024 + rsc_bytes + pidb + 127) & ~(size_t)127)) + ring_bytes;
     };
     // Cluster size C (chunks of >= 1024 columns, C <= 8, dividing every entry's page
     // count): the one with the shortest modelled time.
@@ -840,7 +881,8 @@ cudaError_t expand_launch(const ExpandJob* jobs, int n_jobs, const BatchView& b,
     const int mr = std::max(8, max_rank);
     auto smem_for = [&](int npass) {  // v of the item, row scales, page ids, ring
         const size_t pid_bytes = (size_t)mr * ((npass * kPass) >> pool.page_log2) * 4;
-        return (((size_t)kSimtMaxItemRows * mr * 4 + kMaxRank * 4 + pid_bytes + 127) & ~(size_t)127) +
+        const size_t rsc_bytes = WF == kFmtBf16 ? 0 : kMaxRank * 4;
+        return (((size_t)kSimtMaxItemRows * mr * 4 + rsc_bytes + pid_bytes + 127) & ~(size_t)127) +
                (size_t)kExpandStages * stage_bytes<WF>();
     };
     int tiles[kMaxGroup], max_tiles = 1;

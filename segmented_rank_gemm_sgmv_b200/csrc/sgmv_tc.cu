@@ -39,6 +39,7 @@ __device__ unsigned int g_err_tc;
 constexpr int kKTile = 64;          // K columns per pipeline stage (shrink)
 constexpr int kShrinkStages = 4;
 constexpr int kShrinkThreads = 160;  // 4 producer / epilogue warps + 1 MMA warp
+constexpr int kShrinkCodeSlots = 2;  // quantised pools: k-tiles of A codes in flight
 
 struct ShrinkTcArgs {
     const uint16_t* x;
@@ -53,6 +54,7 @@ struct ShrinkTcArgs {
     int32_t npad_max;    // largest padded rank of the launch (multiple of 16)
     int32_t tmem_cols;   // tensor-memory columns allocated per CTA
     int32_t pid_offset;  // byte offset of the page-id table in shared memory
+    int32_t raw_offset;  // quantised pools: byte offset of the ring of A codes in shared memory
     int32_t use_tma;     // tmap_x is valid: tiles whose rows are consecutive tokens load X by TMA
 };
 
@@ -71,6 +73,7 @@ struct ExpandTcArgs {
     int32_t units_per_cta;  // contiguous run of units per CTA
     int32_t kpad_max;
     int32_t use_tma;        // tmap_y is valid: tiles of consecutive tokens move y by TMA
+    int32_t raw_slots;      // quantised pools: slots of B^T codes (2: converted one unit later; 1: at once)
 };
 
 __device__ __forceinline__ int32_t safe_page(const PoolView& pool, int64_t entry) {
@@ -213,18 +216,12 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
         // 128-byte rows, 1024-byte aligned).  Granule g (16 bytes): row g >> 3,
         // chunk g & 7, so each 8-lane quarter of a warp copies one row's 128
         // contiguous bytes into one (permuted) 128-byte row of shared memory.
-        for (int kt = 0; kt < nk; ++kt) {
-            const int st = kt % kShrinkStages;
-            if (kt >= kShrinkStages && !abort_flag &&
-                !mbar_wait(&empty_bar[st], (uint32_t)((kt / kShrinkStages - 1) & 1), &g_err_tc))
-                abort_flag = 1;
-            uint8_t* xs = stage0 + (size_t)st * stage_bytes;
-            uint8_t* as = xs + x_tile_bytes;
+        auto issue_x = [&](int kt, uint8_t* xs) {
             const int c = k_begin + kt * kKTile;
             if (x_tma) {
                 if (tid == 0) {
-                    mbar_expect_tx(&full_bar[st], (uint32_t)x_tile_bytes);
-                    tma_load_2d(xs, &tmap_x, c, t0, &full_bar[st]);
+                    mbar_expect_tx(&full_bar[kt % kShrinkStages], (uint32_t)x_tile_bytes);
+                    tma_load_2d(xs, &tmap_x, c, t0, &full_bar[kt % kShrinkStages]);
                 }
             } else {
 #pragma unroll
@@ -237,9 +234,22 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
                     cp_async16(xs + off, src, t >= 0);
                 }
             }
-            // A: rank rows n < npad, zero past r; the 64 columns lie in one page
-            const int page_rel = (c >> P_log2) - first_page, in_page = c & ((1 << P_log2) - 1);
-            if constexpr (WF == kFmtBf16) {
+        };
+        auto wait_empty = [&](int kt) {
+            if (kt >= kShrinkStages && !abort_flag &&
+                !mbar_wait(&empty_bar[kt % kShrinkStages], (uint32_t)((kt / kShrinkStages - 1) & 1), &g_err_tc))
+                abort_flag = 1;
+        };
+        if constexpr (WF == kFmtBf16) {
+            for (int kt = 0; kt < nk; ++kt) {
+                const int st = kt % kShrinkStages;
+                wait_empty(kt);
+                uint8_t* xs = stage0 + (size_t)st * stage_bytes;
+                uint8_t* as = xs + x_tile_bytes;
+                const int c = k_begin + kt * kKTile;
+                issue_x(kt, xs);
+                // A: rank rows n < npad, zero past r; the 64 columns lie in one page
+                const int page_rel = (c >> P_log2) - first_page, in_page = c & ((1 << P_log2) - 1);
                 for (int g = tid; g < npad * 8; g += kTcTileRows) {
                     const int n = g >> 3, kg = g & 7;
                     const uint32_t off = (uint32_t)(n >> 3) * 1024 + sw128_off((uint32_t)n, (uint32_t)kg);
@@ -249,33 +259,60 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
                         src = a.pool.pages + ((int64_t)pid_s[n * span_pages + page_rel] << P_log2) + in_page + kg * 8;
                     cp_async16(as + off, src, valid);
                 }
-            } else {
-                // codes through registers: all loads in flight, then converted to bf16 and
-                // stored; the stores reach the tensor core through the async proxy
-                constexpr int VB = bytes_per_8<WF>();
-                const int page_shift = P_log2 + (WF == kFmtFp8 ? 0 : -1);
-                const uint8_t* pages8 = reinterpret_cast<const uint8_t*>(a.pool.pages);
-                typename Codes8<WF>::T cw[kMaxRank * 8 / kTcTileRows];
-#pragma unroll
-                for (int i = 0; i < kMaxRank * 8 / kTcTileRows; ++i) {
-                    const int g = tid + i * kTcTileRows, n = g >> 3, kg = g & 7;
-                    cw[i] = typename Codes8<WF>::T{};
-                    if (g < npad * 8 && ok && n < r)
-                        cw[i] = load_codes8<WF>(pages8 + ((int64_t)pid_s[n * span_pages + page_rel] << page_shift) +
-                                                (in_page / 8 + kg) * VB);
+                cp_async_commit();  // close the group: the copies of every stage form their own
+                cp_async_mbar_arrive_noinc(&full_bar[st]);
+            }
+        } else {
+            // Quantised A: the codes of k-tile kt travel by cp.async into raw slot kt % D,
+            // D k-tiles ahead of their use; at iteration kt a thread waits for its own
+            // copies of tile kt (one commit group per iteration), converts them to bf16
+            // into the swizzled A tile, fences them to the async proxy and arrives on the
+            // stage's barrier a second time.  Granule g (8 values) of a tile: rank row
+            // g >> 3, columns 8 (g & 7); a thread handles g = tid + 128 i.  Two slots keep
+            // the shared memory of two CTAs per SM within the limit.
+            constexpr int D = kShrinkCodeSlots;
+            constexpr int VB = bytes_per_8<WF>();
+            const int page_shift = P_log2 + (WF == kFmtFp8 ? 0 : -1);
+            const uint8_t* pages8 = reinterpret_cast<const uint8_t*>(a.pool.pages);
+            uint8_t* raw0 = smem + a.raw_offset;
+            const int raw_slot = a.npad_max * 8 * VB;
+            auto issue_codes = [&](int kt) {
+                const int c = k_begin + kt * kKTile;
+                const int page_rel = (c >> P_log2) - first_page, in_page = c & ((1 << P_log2) - 1);
+                uint8_t* raw = raw0 + (size_t)(kt % D) * raw_slot;
+                for (int g = tid; g < npad * 8; g += kTcTileRows) {
+                    const int n = g >> 3, kg = g & 7;
+                    if (ok && n < r)
+                        cp_async_n<VB>(raw + g * VB, pages8 + ((int64_t)pid_s[n * span_pages + page_rel] << page_shift) +
+                                                         (in_page / 8 + kg) * VB);
                 }
-#pragma unroll
-                for (int i = 0; i < kMaxRank * 8 / kTcTileRows; ++i) {
-                    const int g = tid + i * kTcTileRows, n = g >> 3, kg = g & 7;
-                    if (g < npad * 8)
-                        *reinterpret_cast<uint4*>(as + (uint32_t)(n >> 3) * 1024 +
-                                                  sw128_off((uint32_t)n, (uint32_t)kg)) = codes8_to_bf16<WF>(cw[i]);
+            };
+#pragma unroll 1
+            for (int kt = 0; kt < D; ++kt) {
+                if (kt < nk) issue_codes(kt);
+                cp_async_commit();
+            }
+            for (int kt = 0; kt < nk; ++kt) {
+                const int st = kt % kShrinkStages;
+                wait_empty(kt);
+                uint8_t* xs = stage0 + (size_t)st * stage_bytes;
+                uint8_t* as = xs + x_tile_bytes;
+                issue_x(kt, xs);
+                cp_async_wait<D - 1>();  // groups up to the one holding tile kt's codes
+                const uint8_t* raw = raw0 + (size_t)(kt % D) * raw_slot;
+                for (int g = tid; g < npad * 8; g += kTcTileRows) {
+                    const int n = g >> 3, kg = g & 7;
+                    typename Codes8<WF>::T cv{};
+                    if (ok && n < r) cv = *reinterpret_cast<const typename Codes8<WF>::T*>(raw + g * VB);
+                    *reinterpret_cast<uint4*>(as + (uint32_t)(n >> 3) * 1024 + sw128_off((uint32_t)n, (uint32_t)kg)) =
+                        codes8_to_bf16<WF>(cv);
                 }
                 fence_proxy_async_smem();
                 mbar_arrive(&full_bar[st]);
+                cp_async_mbar_arrive_noinc(&full_bar[st]);  // this thread's x copies (and earlier codes)
+                if (kt + D < nk) issue_codes(kt + D);        // into the slot just converted
+                cp_async_commit();
             }
-            cp_async_commit();  // close the group: the copies of every stage form their own
-            cp_async_mbar_arrive_noinc(&full_bar[st]);
         }
     } else if (tid == 4 * 32) {
         // ---- MMA issuer
@@ -369,7 +406,6 @@ constexpr int kMaxPagesPerUnit = 2;         // pages of one B^T row a unit spans
 constexpr int kExpandThreads = 416;         // 8 epilogue + 4 producer warps + 1 MMA warp
 constexpr int kExpandProducers = 128;
 constexpr int kMmaWarp = 12;
-constexpr int kMaxExpandStages = 3;
 
 template <int S, int ESZ, int WF>  // ESZ: bytes of a y element (2: bf16, 4: fp32); WF: weight format
 __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const ExpandTcArgs a,
@@ -489,6 +525,93 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
         int32_t pg_next[2];
         fetch(unit(u0), t_next, t0_next, pg_next);
         int ts = -1, cur_tile = -1;
+        // V = v split into bf16 hi + lo for the unit's tile, when the tile changes
+        auto v_split = [&](const Unit& w) {
+            if (!(w.ok && w.tile != cur_tile)) return;
+            if (ts >= 0) wait(&vempty_bar, (uint32_t)(ts & 1));  // the MMAs of the previous tile are done
+            if (WF != kFmtBf16) {  // v_k takes the scale of B^T row k
+                if (pt < w.r) {
+                    const int64_t e = w.b_base + (int64_t)pt * pages_per_row;
+                    rsc_s[pt] = (e >= 0 && e < a.pool.pt_capacity) ? a.pool.row_scale[e] : 0.f;
+                }
+                named_bar_sync(1, kExpandProducers);
+            }
+            const int m = pt, kpad = (w.r + 15) & ~15;
+            const bool row_ok = m < w.rows;
+            const float* vrow = a.v + (int64_t)(w.row_begin + (row_ok ? m : 0)) * a.ldv;
+            // v row in chunks of 64 floats, each chunk's 16-byte loads all in flight
+            // (a load starts below r and below ldv, a multiple of 4: it stays in the row)
+            float4 vq[16];
+#pragma unroll
+            for (int kg = 0; kg < kMaxRank / 8; ++kg) {
+                if (kg >= kpad / 8) break;
+                if ((kg & 7) == 0) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int k4 = kg * 8 + 4 * e;
+                        vq[e] = (row_ok && k4 < w.r && k4 < a.ldv) ? *reinterpret_cast<const float4*>(vrow + k4)
+                                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                }
+                float f[8];
+                const float4 q0 = vq[2 * (kg & 7)], q1 = vq[2 * (kg & 7) + 1];
+                f[0] = q0.x; f[1] = q0.y; f[2] = q0.z; f[3] = q0.w;
+                f[4] = q1.x; f[5] = q1.y; f[6] = q1.z; f[7] = q1.w;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    if (kg * 8 + e >= w.r) f[e] = 0.f;
+                    else if (WF != kFmtBf16) f[e] *= rsc_s[kg * 8 + e];
+                }
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const __nv_bfloat16 h0 = __float2bfloat16_rn(f[2 * e]);
+                    const __nv_bfloat16 h1 = __float2bfloat16_rn(f[2 * e + 1]);
+                    const __nv_bfloat16 l0 = __float2bfloat16_rn(f[2 * e] - __bfloat162float(h0));
+                    const __nv_bfloat16 l1 = __float2bfloat16_rn(f[2 * e + 1] - __bfloat162float(h1));
+                    hw[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+                    lw[e] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+                }
+                const uint32_t off = (uint32_t)(kg >> 3) * (kTcTileRows * 128) + (uint32_t)(m >> 3) * 1024 +
+                                     sw128_off((uint32_t)m, (uint32_t)kg);
+                *reinterpret_cast<uint4*>(vhi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4*>(vlo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+            fence_proxy_async_smem();  // the tensor core reads V through the async proxy
+            named_bar_sync(1, kExpandProducers);
+            if (pt == 0) mbar_arrive(&vfull_bar);
+            ++ts;
+            cur_tile = w.tile;
+        };
+        constexpr int kGr = kMaxRank * (kYRowBytes / 16) / kExpandProducers;  // <= 16 B^T granules a thread
+        // quantised pools: the unit's B^T codes go by cp.async into raw slot i % raw_slots
+        // (granule g = this thread's g-th B^T granule, VB bytes) and are converted to bf16
+        // into stage slot st once this thread's copies have landed: one unit later with two
+        // raw slots (their latency overlaps the next unit's copies), at once with one
+        constexpr int VB = bytes_per_8<WF>();
+        uint8_t* const rawst = yst + (size_t)S * y_bytes;
+        const size_t raw_b = (size_t)kpm * (NB / 8) * VB;
+        const int lag = a.raw_slots > 1 ? 1 : 0;
+        auto convert_codes = [&](const Unit& w, int i_unit) {
+            const int slot = i_unit % S;
+            if (w.ok) {
+                const int kpad = (w.r + 15) & ~15;
+                const uint8_t* raw = rawst + (size_t)(i_unit % a.raw_slots) * raw_b;
+                uint8_t* bs = bst + (size_t)slot * b_bytes;
+#pragma unroll
+                for (int gi = 0; gi < kGr; ++gi) {
+                    const int g = pt + gi * kExpandProducers;
+                    if (g >= kpad * (NB / 8)) break;
+                    const int jg = g % (NB / 8), k = g / (NB / 8);
+                    typename Codes8<WF>::T cv{};
+                    if (k < w.r) cv = *reinterpret_cast<const typename Codes8<WF>::T*>(raw + (size_t)g * VB);
+                    *reinterpret_cast<uint4*>(bs + (uint32_t)(k >> 3) * sbo_b + (uint32_t)(jg >> 3) * 1024 +
+                                              sw128_off((uint32_t)k, (uint32_t)jg)) = codes8_to_bf16<WF>(cv);
+                }
+            }
+            fence_proxy_async_smem();  // the converted codes, to the async proxy; then the second arrival
+            mbar_arrive(&full_bar[slot]);
+        };
         for (int u = u0; u < u1; ++u) {
             const int i = u - u0, st = i % S;
             const Unit w = unit(u);
@@ -496,62 +619,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
             const int32_t pg0 = pg_next[0], pg1 = pg_next[1];
             if (u + 1 < u1) fetch(unit(u + 1), t_next, t0_next, pg_next);
             if (i >= S) wait(&yfree_bar[st], (uint32_t)((i / S - 1) & 1));
-            if (w.ok && w.tile != cur_tile) {
-                if (ts >= 0) wait(&vempty_bar, (uint32_t)(ts & 1));  // the MMAs of the previous tile are done
-                if (WF != kFmtBf16) {  // v_k takes the scale of B^T row k
-                    if (pt < w.r) {
-                        const int64_t e = w.b_base + (int64_t)pt * pages_per_row;
-                        rsc_s[pt] = (e >= 0 && e < a.pool.pt_capacity) ? a.pool.row_scale[e] : 0.f;
-                    }
-                    named_bar_sync(1, kExpandProducers);
-                }
-                const int m = pt, kpad = (w.r + 15) & ~15;
-                const bool row_ok = m < w.rows;
-                const float* vrow = a.v + (int64_t)(w.row_begin + (row_ok ? m : 0)) * a.ldv;
-                // v row in chunks of 64 floats, each chunk's 16-byte loads all in flight
-                // (a load starts below r and below ldv, a multiple of 4: it stays in the row)
-                float4 vq[16];
-#pragma unroll
-                for (int kg = 0; kg < kMaxRank / 8; ++kg) {
-                    if (kg >= kpad / 8) break;
-                    if ((kg & 7) == 0) {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const int k4 = kg * 8 + 4 * e;
-                            vq[e] = (row_ok && k4 < w.r && k4 < a.ldv) ? *reinterpret_cast<const float4*>(vrow + k4)
-                                                                       : make_float4(0.f, 0.f, 0.f, 0.f);
-                        }
-                    }
-                    float f[8];
-                    const float4 q0 = vq[2 * (kg & 7)], q1 = vq[2 * (kg & 7) + 1];
-                    f[0] = q0.x; f[1] = q0.y; f[2] = q0.z; f[3] = q0.w;
-                    f[4] = q1.x; f[5] = q1.y; f[6] = q1.z; f[7] = q1.w;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        if (kg * 8 + e >= w.r) f[e] = 0.f;
-                        else if (WF != kFmtBf16) f[e] *= rsc_s[kg * 8 + e];
-                    }
-                    uint32_t hw[4], lw[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const __nv_bfloat16 h0 = __float2bfloat16_rn(f[2 * e]);
-                        const __nv_bfloat16 h1 = __float2bfloat16_rn(f[2 * e + 1]);
-                        const __nv_bfloat16 l0 = __float2bfloat16_rn(f[2 * e] - __bfloat162float(h0));
-                        const __nv_bfloat16 l1 = __float2bfloat16_rn(f[2 * e + 1] - __bfloat162float(h1));
-                        hw[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-                        lw[e] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
-                    }
-                    const uint32_t off = (uint32_t)(kg >> 3) * (kTcTileRows * 128) + (uint32_t)(m >> 3) * 1024 +
-                                         sw128_off((uint32_t)m, (uint32_t)kg);
-                    *reinterpret_cast<uint4*>(vhi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                    *reinterpret_cast<uint4*>(vlo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-                }
-                fence_proxy_async_smem();  // the tensor core reads V through the async proxy
-                named_bar_sync(1, kExpandProducers);
-                if (pt == 0) mbar_arrive(&vfull_bar);
-                ++ts;
-                cur_tile = w.tile;
-            }
+            if constexpr (WF == kFmtBf16) v_split(w);
             if (w.ok) {
                 if (pt < w.r * npc) pid_s[st][pt] = pg0;
                 if (pt + kExpandProducers < w.r * npc) pid_s[st][pt + kExpandProducers] = pg1;
@@ -579,10 +647,9 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
                     }
                 }
                 // B^T block: granule (k, jg) = B^T[k][j0 + 8 jg .. +8], zero past r
-                uint8_t* bs = bst + (size_t)st * b_bytes;
                 const int kpad = (w.r + 15) & ~15;
-                constexpr int kGr = kMaxRank * (kYRowBytes / 16) / kExpandProducers;  // <= 16 granules a thread
                 if constexpr (WF == kFmtBf16) {
+                    uint8_t* bs = bst + (size_t)st * b_bytes;
 #pragma unroll
                     for (int gi = 0; gi < kGr; ++gi) {
                         const int g = pt + gi * kExpandProducers;
@@ -599,41 +666,46 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
                         cp_async16(bs + off, src, valid);
                     }
                 } else {
-                    // codes through registers (all loads in flight), converted to bf16 and stored
-                    constexpr int VB = bytes_per_8<WF>();
                     const int page_shift = P_log2 + (WF == kFmtFp8 ? 0 : -1);
                     const uint8_t* pages8 = reinterpret_cast<const uint8_t*>(a.pool.pages);
-                    typename Codes8<WF>::T cw[kGr];
-#pragma unroll
-                    for (int gi = 0; gi < kGr; ++gi) {
-                        const int g = pt + gi * kExpandProducers;
-                        const int jg = g % (NB / 8), k = g / (NB / 8);
-                        const int j = w.j0 + jg * 8;
-                        cw[gi] = typename Codes8<WF>::T{};
-                        if (g < kpad * (NB / 8) && k < w.r)
-                            cw[gi] = load_codes8<WF>(
-                                pages8 + ((int64_t)pid_s[st][k * npc + ((j - w.j0) >> P_log2)] << page_shift) +
-                                ((j & ((1 << P_log2) - 1)) / 8) * VB);
-                    }
+                    uint8_t* raw = rawst + (size_t)(i % a.raw_slots) * raw_b;
 #pragma unroll
                     for (int gi = 0; gi < kGr; ++gi) {
                         const int g = pt + gi * kExpandProducers;
                         if (g >= kpad * (NB / 8)) break;
                         const int jg = g % (NB / 8), k = g / (NB / 8);
-                        const uint32_t off = (uint32_t)(k >> 3) * sbo_b + (uint32_t)(jg >> 3) * 1024 +
-                                             sw128_off((uint32_t)k, (uint32_t)jg);
-                        *reinterpret_cast<uint4*>(bs + off) = codes8_to_bf16<WF>(cw[gi]);
+                        const int j = w.j0 + jg * 8;
+                        if (k < w.r)
+                            cp_async_n<VB>(raw + (size_t)g * VB,
+                                           pages8 + ((int64_t)pid_s[st][k * npc + ((j - w.j0) >> P_log2)] << page_shift) +
+                                               ((j & ((1 << P_log2) - 1)) / 8) * VB);
                     }
                 }
             } else if (pt == 0) {
                 atomicOr(&g_err_tc, kErrRows);
             }
-            if (WF != kFmtBf16) {  // the converted codes, to the async proxy, then the second arrival
-                fence_proxy_async_smem();
-                mbar_arrive(&full_bar[st]);
-            }
             cp_async_commit();
             cp_async_mbar_arrive_noinc(&full_bar[st]);
+            if constexpr (WF != kFmtBf16) {
+                // the codes of unit i - lag (its commit group) have landed: convert them; then
+                // the V split, which may wait for the MMAs of that unit
+                if (lag) {
+                    if (i >= 1) {
+                        cp_async_wait<1>();
+                        convert_codes(unit(u - 1), i - 1);
+                    }
+                } else {
+                    cp_async_wait<0>();
+                    convert_codes(w, i);
+                }
+                v_split(w);
+            }
+        }
+        if constexpr (WF != kFmtBf16) {
+            if (lag && u1 > u0) {
+                cp_async_wait<0>();
+                convert_codes(unit(u1 - 1), u1 - 1 - u0);
+            }
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
@@ -840,10 +912,14 @@ cudaError_t launch_shrink_tc(const uint16_t* x, int64_t ldx, int32_t d_in, const
     const size_t stage_bytes = (size_t)kTcTileRows * kKTile * 2 + (size_t)a.npad_max * kKTile * 2;
     const size_t main_bytes = std::max(stage_bytes * kShrinkStages, (size_t)kTcTileRows * (a.npad_max + 1) * 4);
     const size_t span_pages = ((size_t)a.kcols >> pool.page_log2) + 2;  // pages one K range can touch
-    a.pid_offset = (int)main_bytes;
+    // quantised pools: a ring of kShrinkCodeSlots slots of A codes (npad_max rows x 64 values)
+    const size_t raw_bytes = pool.wfmt == kFmtBf16 ? 0  // 1 byte (E4M3) or half a byte (INT4) a value
+                             : (size_t)kShrinkCodeSlots * a.npad_max * kKTile / (pool.wfmt == kFmtFp8 ? 1 : 2);
+    a.raw_offset = (int)main_bytes;
+    a.pid_offset = (int)(main_bytes + raw_bytes);
     const size_t pid_bytes = ((size_t)a.npad_max * span_pages * 4 + 15) & ~(size_t)15;
     // >= 80 KB: at most two CTAs per SM, so tensor memory is never oversubscribed
-    const size_t smem = std::max(main_bytes + pid_bytes, (size_t)80 << 10) + 1024;
+    const size_t smem = std::max(main_bytes + raw_bytes + pid_bytes, (size_t)80 << 10) + 1024;
     if (smem > (227u << 10)) return cudaErrorInvalidValue;
     auto kern = pool.wfmt == kFmtFp8 ? shrink_tc_kernel<kFmtFp8>
                 : pool.wfmt == kFmtInt4 ? shrink_tc_kernel<kFmtInt4> : shrink_tc_kernel<kFmtBf16>;
@@ -889,13 +965,29 @@ cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const B
     a.num_units = a.n_blocks * num_tiles;
     // shared memory: V hi + lo, S stages of (B^T block, Y block); three stages when they fit
     const size_t v_bytes = (size_t)2 * kTcTileRows * ((a.kpad_max + 63) & ~63) * 2;
+    // a stage: B^T block (bf16) and y block; a quantised pool adds 1 or 2 slots of B^T codes
+    // (1 or 1/2 byte a value)
+    const size_t raw_slot = pool.wfmt == kFmtBf16 ? 0 : (size_t)a.kpad_max * NB / (pool.wfmt == kFmtFp8 ? 1 : 2);
     const size_t stage = (size_t)a.kpad_max * NB * 2 + (size_t)kTcTileRows * kYRowBytes;
-    // the opt-in limit covers dynamic (+1 KB alignment) and static (index tables, barriers) shared memory
-    const size_t limit = (227u << 10) - 1024 - 1024 - (size_t)(kMaxExpandStages + 1) * kTcTileRows * 4 -
-                         (size_t)kMaxExpandStages * kMaxRank * kMaxPagesPerUnit * 4;
-    const int S = (v_bytes + 3 * stage <= limit) ? 3 : 2;
+    // the opt-in limit covers dynamic (+1 KB alignment) and static shared memory (index tables,
+    // barriers, row scales: 6.1 KB with three stages, rounded up)
+    const size_t limit = (227u << 10) - 1024 - 6656;
+    // stages S and code slots R (quantised pools): three stages when they fit, two code slots
+    // when they fit (one otherwise)
+    int S = 2, R = raw_slot ? 1 : 0;
+    const int cand[3][2] = {{3, 2}, {2, 2}, {2, 1}};
+    for (const auto& c : cand) {
+        const int r = raw_slot ? c[1] : 0;
+        if (v_bytes + c[0] * stage + r * raw_slot <= limit) {
+            S = c[0];
+            R = r;
+            break;
+        }
+    }
+    a.raw_slots = std::max(R, 1);
     // at least 116 KB: one CTA per SM, so tensor memory (2 x NB <= 256 columns) is never oversubscribed
-    const size_t smem = std::max(v_bytes + S * stage, (size_t)116 << 10) + 1024;
+    const size_t smem = std::max(v_bytes + S * stage + R * raw_slot, (size_t)116 << 10) + 1024;
+    if (smem > (227u << 10)) return cudaErrorInvalidValue;
     // one CTA per SM, each a contiguous run of units
     static int sms = 0;
     if (!sms) {

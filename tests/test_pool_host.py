@@ -76,3 +76,31 @@ def test_rank_above_pool_max_is_rejected():
     pool = sg.AdapterPool([(512, 512)], num_pages=64, page_elems=512, max_rank=16, device=-1)
     with pytest.raises(sg.SgmvError):
         pool.load(0, 32)
+
+
+@pytest.mark.parametrize("fmt,page_bytes", [("bf16", 1024), ("fp8_e4m3", 512), ("int4", 256)])
+def test_quantised_pool_bookkeeping(fmt, page_bytes):
+    """A quantised pool keeps the same page table (page_elems values of a rank row a page);
+    only the bytes of a page change: 1 byte a value for E4M3, half a byte for INT4
+    ([ClusterBid] paragraph on the GPU memory budget: FP8 halves the adapter memory)."""
+    projs = [(d_in, d_out) for _, d_in, d_out in LLAMA70B_PROJECTIONS]
+    pool = sg.AdapterPool(projs, num_pages=20000, page_elems=512, max_rank=16, device=-1, weight_format=fmt)
+    pool.load(7, 16)
+    st = pool.stats()
+    assert st.weight_format == sg.WEIGHT_FORMATS[fmt] and st.page_bytes == page_bytes
+    pages = sg.AdapterPool.pages_needed(projs, 16)
+    assert st.num_pages - st.free_pages == pages
+    # payload of the rank-16 layer: 5,177,344 bytes in bf16 (the memory table), half in E4M3, a quarter in INT4
+    assert st.payload_bytes == 5177344 * page_bytes // 1024
+
+
+def test_unknown_weight_format_is_rejected():
+    lib = sg.load_library()
+    import ctypes
+    d = (ctypes.c_int32 * 1)(512)
+    h = ctypes.c_void_p()
+    st = lib.sgmv_pool_create_ex(-1, 64, 512, 1, ctypes.cast(d, ctypes.c_void_p), ctypes.cast(d, ctypes.c_void_p),
+                                 16, 3, ctypes.byref(h))
+    assert st == 1 and not h.value
+    with pytest.raises(ValueError):
+        sg.AdapterPool([(512, 512)], num_pages=8, device=-1, weight_format="fp4")

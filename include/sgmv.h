@@ -79,7 +79,8 @@ SGMV_API const char* sgmv_last_error(void);
  * interchangeable blocks) and of the fixed-size adapter pool with slots of
  * [ClusterBid] (paragraph on vLLM's GPU memory pool).
  *
- * Layout.  A page holds page_elems bf16 values.  For each adapter and each
+ * Layout.  A page holds page_elems values (bf16 by default; codes in a
+ * quantised pool, see below).  For each adapter and each
  * projection p the pool stores
  *     A   as r rows of d_in[p]  values (the logical r x d_in matrix), and
  *     B^T as r rows of d_out[p] values (the transpose of the d_out x r B),
@@ -90,9 +91,10 @@ SGMV_API const char* sgmv_last_error(void);
  * Pages are taken from a free list in any order, so consecutive chunks of a
  * row are in general not adjacent in memory.
  *
- * The payload of a rank-r adapter is exactly sum_p (d_in[p]*r + r*d_out[p])*2
- * bytes -- the bytes-per-matrix formula of [SGMV post], "The maths that
- * matters" -- because page_elems must divide every d_in[p] and d_out[p].
+ * The payload of a rank-r adapter in a bf16 pool is exactly
+ * sum_p (d_in[p]*r + r*d_out[p])*2 bytes -- the bytes-per-matrix formula of
+ * [SGMV post], "The maths that matters" -- because page_elems must divide
+ * every d_in[p] and d_out[p] (a half or a quarter of that in a quantised pool).
  */
 typedef struct sgmv_pool sgmv_pool;
 
@@ -139,7 +141,7 @@ typedef struct {
 } sgmv_pool_stats;
 
 /*
- * Create a pool on `device` (CUDA ordinal) with `num_pages` pages of
+ * Create a bf16 pool on `device` (CUDA ordinal) with `num_pages` pages of
  * `page_elems` bf16 values (a power of two in [64, 65536]), for adapters over
  * `n_proj` projections with shapes d_in[p] -> d_out[p] (host arrays of n_proj
  * entries, each a multiple of page_elems) and ranks up to max_rank (<= 128).

@@ -235,7 +235,7 @@ class AdapterPool:
         scales = np.zeros(max(r, 1), dtype=np.float32)
         _check(load_library().sgmv_pool_read(self.handle, int(adapter_id), int(proj), int(matrix),
                                              codes.ctypes.data, codes.size, scales.ctypes.data, scales.size,
-                                             _stream(stream)))
+                                             _stream(stream) if self.device >= 0 else None))
         codes, scales = codes[:r], scales[:r]
         if self.weight_format == "bf16":
             codes = codes.view(np.uint16)

@@ -104,3 +104,14 @@ def test_unknown_weight_format_is_rejected():
     assert st == 1 and not h.value
     with pytest.raises(ValueError):
         sg.AdapterPool([(512, 512)], num_pages=8, device=-1, weight_format="fp4")
+
+
+def test_read_needs_device_memory_and_a_resident_adapter():
+    pool = sg.AdapterPool([(512, 512)], num_pages=64, page_elems=512, max_rank=16, device=-1, weight_format="int4")
+    pool.load(1, 8)
+    with pytest.raises(sg.SgmvError) as e:
+        pool.read(1, 0, 0)
+    assert e.value.status == 1                       # a host-only pool has no pages to read
+    with pytest.raises(sg.SgmvError) as e:
+        pool.read(2, 0, 0)                           # not resident
+    assert e.value.status == 3

@@ -246,6 +246,9 @@ SGMV_API const void* sgmv_pool_pages_device(const sgmv_pool* pool);
  * 128-row tiles; shorter segments go to the SIMT path as items of at most
  * 4 rows (long_threshold <= 0 selects the built-in default, 16; a huge value
  * keeps every segment on the SIMT path; 1 sends every segment to tensor cores).
+ * With the default, the tensor-core path is taken only when the long segments
+ * hold at least 128 rows in total (one full tile); below that every segment
+ * goes to the SIMT path and the plan's long_threshold reads INT32_MAX.
  */
 typedef struct {
     int32_t T;              /* tokens in the batch                                   */

@@ -55,7 +55,8 @@ extern "C" sgmv_status sgmv_build_plan(const int32_t* adapter_ids, int32_t T, co
     if (T > 0 && !adapter_ids) return fail(SGMV_ERR_INVALID, "build_plan: adapter_ids is NULL");
     if (!table && table_capacity > 0) return fail(SGMV_ERR_INVALID, "build_plan: table is NULL");
     if (reinterpret_cast<uintptr_t>(table) & 15) return fail(SGMV_ERR_INVALID, "build_plan: table must be 16-byte aligned");
-    if (long_threshold <= 0) long_threshold = kDefaultLongThreshold;
+    const bool default_threshold = long_threshold <= 0;
+    if (default_threshold) long_threshold = kDefaultLongThreshold;
 
     // Distinct adapters of the batch, ascending; tokens with id -1 use none.
     std::vector<int32_t> ids;
@@ -87,6 +88,20 @@ extern "C" sgmv_status sgmv_build_plan(const int32_t* adapter_ids, int32_t T, co
     std::vector<int32_t> offsets(S + 1, 0);
     for (int64_t s = 0; s < S; ++s) offsets[s + 1] = offsets[s] + count[s + 1];
     const int32_t rows = offsets[S];
+
+    // With the default threshold, the tensor-core kernels are used only when the long
+    // segments hold at least one full 128-row tile in total: below that their fixed cost
+    // (cluster launch, tensor-memory allocation, barrier setup) outweighs the adapter
+    // re-reads of the SIMT items they would save.  The plan then reports the threshold
+    // as never reached.
+    if (default_threshold) {
+        int64_t long_rows = 0;
+        for (int64_t s = 0; s < S; ++s) {
+            const int32_t n = offsets[s + 1] - offsets[s];
+            if (recs[s]->rank > 0 && n >= long_threshold) long_rows += n;
+        }
+        if (long_rows < kTcTileRows) long_threshold = INT32_MAX;
+    }
 
     // Dispatch: long segments -> 128-row tensor-core tiles, the rest -> SIMT items.
     int64_t n_simt = 0, n_tc = 0;

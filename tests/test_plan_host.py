@@ -120,3 +120,23 @@ def test_simt_items_largest_rank_first():
     for a, b in zip(range(len(segs) - 1), range(1, len(segs))):
         if rec_ranks[a] == rec_ranks[b]:
             assert segs[a] <= segs[b]
+
+
+def test_default_dispatch_needs_one_full_tile_of_long_rows():
+    """With the default threshold (16 rows), segments go to the tensor-core kernels only
+    when the long segments hold at least 128 rows in total; otherwise every segment is
+    cut into SIMT items and the plan reports the threshold as never reached.  An
+    explicit threshold is applied as given."""
+    ranks = {0: 8, 1: 16, 2: 16, 3: 8}
+    few = [0] * 16 + [1] * 16 + [2] * 16 + [3] * 16                    # 64 long rows
+    pool = _pool(ranks)
+    plan = pool.plan(few)
+    assert plan.plan.num_tc_tiles == 0 and plan.plan.num_simt_items == 16
+    assert plan.plan.long_threshold == 2 ** 31 - 1
+    _check_plan(plan, pool, few, ranks, plan.plan.long_threshold)
+    plan = pool.plan(few, long_threshold=16)                             # explicit: applied as given
+    assert plan.plan.num_tc_tiles == 4 and plan.plan.long_threshold == 16
+    many = [0] * 100 + [1] * 28 + [2] * 3                                # 128 long rows
+    plan = pool.plan(many)
+    assert plan.plan.long_threshold == 16 and plan.plan.num_tc_tiles == 2 and plan.plan.num_simt_items == 1
+    _check_plan(plan, pool, many, ranks, 16)

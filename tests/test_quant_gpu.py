@@ -140,3 +140,17 @@ def test_quantised_pool_memory():
         pool = sg.AdapterPool(projs, num_pages=64, page_elems=512, max_rank=16, device=0, weight_format=fmt)
         assert pool.stats().page_bytes == per_page
         pool.close()
+
+
+def test_bf16_pool_read_returns_the_stored_weights():
+    d_in, d_out, r = 1024, 512, 12
+    pool = sg.AdapterPool([(d_in, d_out)], num_pages=256, page_elems=512, max_rank=16, device=0)
+    pool.shuffle_free_pages(5)
+    g = torch.Generator(device="cuda").manual_seed(2)
+    A = torch.randn(r, d_in, generator=g, device="cuda").to(torch.bfloat16)
+    B = torch.randn(d_out, r, generator=g, device="cuda").to(torch.bfloat16)
+    pool.load(3, r, [A], [B])
+    codes, scales = pool.read(3, 0, 0)
+    assert np.array_equal(codes, A.view(torch.int16).cpu().numpy().view(np.uint16)) and np.all(scales == 1.0)
+    codes, _ = pool.read(3, 0, 1)
+    assert np.array_equal(codes, B.t().contiguous().view(torch.int16).cpu().numpy().view(np.uint16))

@@ -127,19 +127,30 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-def read_traffic(workload: str, kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when the
-    kernel sources changed since the counters were taken."""
+def source_digest() -> str:
+    """sha256 (first 16 hex digits) of the library's code: csrc/* by name, with `//`
+    comments, trailing blanks and empty lines removed, so that a comment edit keeps
+    the counters while any code change drops them."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
-    if not os.path.exists(path):
-        return None
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "segmented_rank_gemm_sgmv_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
-    digest = h.hexdigest()[:16]
+        with open(os.path.join(csrc, name), encoding="utf-8", errors="replace") as f:
+            for line in f:
+                code = re.sub(r"//.*", "", line).rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
+    return h.hexdigest()[:16]
+
+
+def read_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when the
+    kernel sources changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    digest = source_digest()
     with open(path) as f:
         for line in f:
             parts = line.split()

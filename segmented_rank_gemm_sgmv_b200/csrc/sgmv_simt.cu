@@ -27,6 +27,10 @@
 //          before the kernel waits for the shrink; then v of the item is read,
 //          each thread accumulates its 8 output columns for up to 4 tokens and
 //          updates y with one rounding, pass by pass.
+// Quantised pools (template parameter WF): the stages hold E4M3 / INT4 codes
+// (8 or 4 KB, filled with 16-byte copies) and each thread converts its 8
+// values in registers; a rank row's scale multiplies v_k once, at the end of
+// the shrink, and v_k as the expand reads it.
 #include <cuda_bf16.h>
 
 #include <algorithm>

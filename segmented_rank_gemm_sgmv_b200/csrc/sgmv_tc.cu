@@ -7,18 +7,25 @@
 //   shrink  V[128 rows, r]     = X[128 rows, d_in] * A^T          (M=128, N=r padded to 16)
 //   expand  Y[128 rows, 128 j] += scale * V[128 rows, r] * B^T    (M=128, N=128, K=r padded to 16)
 //
-// Operands are staged in shared memory in the canonical no-swizzle layout
-// (8 rows x 16 bytes core matrices) with 16-byte cp.async copies -- x rows are
-// gathered through the segment's token list and A / B^T chunks through the
-// page table -- and multiplied by one thread issuing tcgen05.mma (bf16 inputs,
-// fp32 accumulator in tensor memory).  The epilogue reads the accumulator with
-// tcgen05.ld.
+// Operands are staged in shared memory in the 128-byte swizzle by producer
+// warps -- X tiles and y blocks of consecutive tokens by 2-D TMA, gathered rows
+// (through the segment's token list) and A / B^T chunks (through the page
+// table) by 16-byte cp.async -- and multiplied by one thread issuing
+// tcgen05.mma (bf16 inputs, fp32 accumulator in tensor memory); mbarriers link
+// the producer, MMA and epilogue roles, and the epilogue reads the accumulator
+// with tcgen05.ld.
 //
 // shrink: a cluster of KS CTAs splits d_in; each accumulates its K range in
 // tensor memory, and the KS partial tiles are summed in a fixed order through
 // distributed shared memory into v.
-// expand: v (fp32) is split into bf16 hi + lo parts so that the delta keeps
-// ~16 bits of v: D = V_hi B + V_lo B, both products exact, fp32 accumulation.
+// expand: persistent CTAs over (tile, column block) units with a
+// double-buffered accumulator; v (fp32) is split into bf16 hi + lo parts so
+// that the delta keeps ~16 bits of v: D = V_hi B + V_lo B, both products
+// exact, fp32 accumulation.
+// Quantised pools (template parameter WF): the producers move E4M3 / INT4
+// codes by cp.async into a small ring of code slots and convert them to bf16
+// (exact) in the swizzled operand tile; the row scales of A multiply v in the
+// shrink's epilogue, those of B^T multiply v before the hi / lo split.
 #include <cuda.h>  // CUtensorMap (the encoder is reached through the runtime's driver entry point)
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>

@@ -100,6 +100,15 @@ def test_decode_q_proj(mode):
     assert plan.plan.num_tc_tiles == 0 and plan.plan.num_segments == wl.distinct_adapters
 
 
+def test_decode_q_proj_12():
+    """The decode batch with about 12 distinct adapters among 32 requests (Zipf s = 1.5)."""
+    wl = workloads.make("decode_q_proj_12")
+    bank = workloads.AdapterBank(wl, device="cuda")
+    x, y = workloads.activations(wl, 0, device="cuda")
+    plan, *_ = check(wl, bank, x, y, 0, mode="lora_delta")
+    assert plan.plan.num_tc_tiles == 0 and plan.plan.num_segments == wl.distinct_adapters < 20
+
+
 @MODES
 @pytest.mark.parametrize("y_dtype", [torch.bfloat16, torch.float32], ids=["ybf16", "yfp32"])
 def test_mixed_rank_mlp_up(y_dtype, mode):

@@ -38,7 +38,8 @@ LLAMA70B_PROJECTIONS: Tuple[Tuple[str, int, int], ...] = (
     ("down", 28672, 8192),
 )
 
-WORKLOAD_NAMES = ("tiny", "decode_q_proj", "mixed_rank_mlp_up", "prefill_long", "llama70b_layer")
+WORKLOAD_NAMES = ("tiny", "decode_q_proj", "decode_q_proj_12", "mixed_rank_mlp_up", "prefill_long",
+                  "llama70b_layer")
 
 
 @dataclasses.dataclass
@@ -82,6 +83,8 @@ def make(name: str, seed: int = 0, **overrides) -> Workload:
     tiny              T=64, d 512->512, 4 adapters of rank 8, 4 contiguous segments of 16 tokens.
     decode_q_proj     T=32 decode tokens, q_proj 8192->8192, rank 16, adapter per token from a
                       bounded Zipf(s=1.1) over a pool of 250 resident adapters.
+    decode_q_proj_12  the same with Zipf(s=1.5): about 12 distinct adapters among the 32
+                      requests, the glossary example's "32 requests, 12 tenants".
     mixed_rank_mlp_up T=256, 4096->14336, pool of 512 adapters with ranks uniform over
                       {8,16,32,64}; 64 distinct adapters drawn, tokens assigned uniformly.
     prefill_long      8 requests x 512 tokens, 8 adapters of rank 64, 8192->8192,
@@ -99,10 +102,10 @@ def make(name: str, seed: int = 0, **overrides) -> Workload:
         ids = np.repeat(pool_ids, seg).astype(np.int32)
         d = overrides.get("d", 512)
         wl = Workload(name, seed, T, [("proj", d, d)], pool_ids, pool_ranks, ids)
-    elif name == "decode_q_proj":
+    elif name in ("decode_q_proj", "decode_q_proj_12"):
         T = overrides.get("T", 32)
         n_pool = overrides.get("pool", 250)
-        s = overrides.get("zipf_s", 1.1)
+        s = overrides.get("zipf_s", 1.1 if name == "decode_q_proj" else 1.5)
         d = overrides.get("d", 8192)
         pool_ids = np.arange(n_pool, dtype=np.int32)
         pool_ranks = np.full(n_pool, overrides.get("rank", 16), dtype=np.int32)

@@ -55,7 +55,7 @@ typedef struct CUstream_st* sgmv_stream_t; /* same type as cudaStream_t */
 typedef enum {
     SGMV_OK = 0,
     SGMV_ERR_INVALID = 1,      /* malformed argument (null pointer, bad size, misaligned row) */
-    SGMV_ERR_UNSUPPORTED = 2,  /* well-formed but outside what this build handles            */
+    SGMV_ERR_UNSUPPORTED = 2,  /* well-formed but outside what the library handles          */
     SGMV_ERR_NOT_RESIDENT = 3, /* an adapter id of the batch is not loaded in the pool        */
     SGMV_ERR_OUT_OF_PAGES = 4, /* the pool has too few free pages for an adapter              */
     SGMV_ERR_CUDA = 5,         /* a CUDA runtime call failed                                  */

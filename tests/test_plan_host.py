@@ -140,3 +140,35 @@ def test_default_dispatch_needs_one_full_tile_of_long_rows():
     plan = pool.plan(many)
     assert plan.plan.long_threshold == 16 and plan.plan.num_tc_tiles == 2 and plan.plan.num_simt_items == 1
     _check_plan(plan, pool, many, ranks, 16)
+
+
+# ---------------------------------------------------------------- property-based
+from hypothesis import given, settings, HealthCheck
+from hypothesis import strategies as st
+
+_RANKS = {a: r for a, r in zip(range(0, 24, 2), [0, 8, 16, 5, 24, 64, 128, 1, 32, 16, 8, 40])}
+_POOL = None
+
+
+def _shared_pool():
+    global _POOL
+    if _POOL is None:
+        _POOL = _pool(_RANKS)
+    return _POOL
+
+
+@settings(max_examples=150, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(ids=st.lists(st.sampled_from(list(_RANKS) + [-1]), min_size=0, max_size=400),
+       runs=st.lists(st.tuples(st.sampled_from(list(_RANKS)), st.integers(1, 200)), max_size=3),
+       thr=st.sampled_from([0, 1, 2, 5, 16, 17, 129, 10 ** 9]))
+def test_plan_properties(ids, runs, thr):
+    """Any batch (with long same-adapter runs mixed in), any threshold: the plan equals the
+    brute-force grouping and every row of a segment with rank > 0 is covered exactly once
+    by items of <= 4 rows or tiles of <= 128 rows, on the side the threshold says."""
+    batch = list(ids)
+    for a, n in runs:
+        batch += [a] * n
+    plan = _shared_pool().plan(np.asarray(batch, dtype=np.int32), long_threshold=thr)
+    _check_plan(plan, _shared_pool(), batch, _RANKS, plan.plan.long_threshold)
+    if thr > 0:
+        assert plan.plan.long_threshold == thr

@@ -115,3 +115,54 @@ def test_read_needs_device_memory_and_a_resident_adapter():
     with pytest.raises(sg.SgmvError) as e:
         pool.read(2, 0, 0)                           # not resident
     assert e.value.status == 3
+
+
+# ---------------------------------------------------------------- property-based
+from hypothesis import given, settings, HealthCheck
+from hypothesis import strategies as st
+
+_PROJS = [(512, 1024), (1024, 512)]
+
+
+@settings(max_examples=80, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(ops=st.lists(st.tuples(st.sampled_from(["load", "evict", "shuffle"]), st.integers(0, 9),
+                              st.sampled_from([0, 1, 8, 16, 32])), min_size=1, max_size=60),
+       fmt=st.sampled_from(["bf16", "fp8_e4m3", "int4"]))
+def test_pool_bookkeeping_properties(ops, fmt):
+    """Any sequence of loads (new or replacing), evictions and free-list shuffles on a
+    small pool: resident adapters own disjoint pages, the free count is the rest, a load
+    that does not fit changes nothing, and each adapter's page count matches its rank."""
+    pool = sg.AdapterPool(_PROJS, num_pages=300, page_elems=512, max_rank=32, device=-1, weight_format=fmt)
+    resident = {}
+    for op, a, r in ops:
+        if op == "load":
+            need = sg.AdapterPool.pages_needed(_PROJS, r)
+            free = pool.stats().free_pages + (sg.AdapterPool.pages_needed(_PROJS, resident[a]) if a in resident else 0)
+            if need <= free:
+                pool.load(a, r)
+                resident[a] = r
+            else:
+                before = pool.stats().free_pages
+                with pytest.raises(sg.SgmvError) as e:
+                    pool.load(a, r)
+                assert e.value.status == 4 and pool.stats().free_pages == before
+        elif op == "evict":
+            if a in resident:
+                pool.evict(a)
+                del resident[a]
+            else:
+                with pytest.raises(sg.SgmvError):
+                    pool.evict(a)
+        else:
+            pool.shuffle_free_pages(a + 1)
+        owned = []
+        for b, rb in resident.items():
+            assert pool.rank_of(b) == rb
+            for p in range(len(_PROJS)):
+                for m in range(2):
+                    ids = pool.page_ids(b, p, m)
+                    assert ids.size == rb * _PROJS[p][m] // 512
+                    owned.extend(ids.tolist())
+        assert len(owned) == len(set(owned)) and all(0 <= x < 300 for x in owned)
+        st_ = pool.stats()
+        assert st_.free_pages == 300 - len(owned) and st_.resident_adapters == len(resident)

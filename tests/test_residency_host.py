@@ -82,3 +82,51 @@ def test_adapters_loaded_directly_are_the_oldest():
     res.prepare([0])
     res.prepare([1])                                 # evicts 7, not 0
     assert _resident(pool, [0, 1, 2, 7]) == [0, 1]
+
+
+# ---------------------------------------------------------------- property-based
+from hypothesis import given, settings, HealthCheck
+from hypothesis import strategies as st
+
+
+@settings(max_examples=120, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(batches=st.lists(st.lists(st.sampled_from([-1, 0, 1, 2, 3, 4, 5]), min_size=1, max_size=6),
+                        min_size=1, max_size=25),
+       room=st.integers(1, 4))
+def test_lru_against_a_simulation(batches, room):
+    """Random batches over six equal-rank adapters with room for `room` of them: the
+    residency manager's result (what is resident, what each batch loaded, hits, misses,
+    evictions) equals an independent LRU simulation -- batch adapters touched, misses
+    loaded, least recently used outside the batch evicted first (ties: lowest id), a
+    batch that cannot fit refused with nothing changed."""
+    pool = sg.AdapterPool(PROJ, num_pages=room * PER_ADAPTER, page_elems=512, max_rank=R, device=-1)
+    res = sg.Residency(pool)
+    for a in range(6):
+        res.register(a, R)
+    resident, last, tick = set(), {}, 0
+    hits = misses = evictions = 0
+    for batch in batches:
+        want = sorted({a for a in batch if a >= 0})
+        tick += 1
+        if len(want) > room:
+            with pytest.raises(sg.SgmvError) as e:
+                res.prepare(batch)
+            assert e.value.status == 4
+        else:
+            miss = [a for a in want if a not in resident]
+            hits += len(want) - len(miss)
+            misses += len(miss)
+            for a in want:
+                if a in resident:
+                    last[a] = tick
+            while len(resident) + len(miss) > room:
+                victim = min((a for a in resident if a not in want), key=lambda a: (last[a], a))
+                resident.discard(victim)
+                evictions += 1
+            for a in miss:
+                resident.add(a)
+                last[a] = tick
+            assert res.prepare(batch) == len(miss)
+        assert _resident(pool, range(6)) == sorted(resident)
+        s = res.stats()
+        assert (s.hits, s.misses, s.evictions) == (hits, misses, evictions)

@@ -1,14 +1,16 @@
 """Benchmark of the multi-LoRA delta (SGMV shrink + expand) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--weights bf16|fp8_e4m3|int4] [--per-projection] [--split-phases]
 
 One step is one pass of the whole hot path over one batch: the host segment
 builder (run every step, overlapped with the previous device work), one
 host-to-device copy of the segment table, then SGMV-shrink and SGMV-expand for
-every adapted projection of the workload.  The device time of a step (CUDA
-events on the launching stream, from the table copy to the last expand) is
-what `value` measures; L2 is flushed (a 512 MiB write) between steps, outside
-the timed windows.  `e2e` repeats the step through the same public API with
+every adapted projection of the workload (one grouped call for a multi-projection
+workload unless --per-projection).  The device time of a step (CUDA events on the
+launching stream, from the table copy to the last expand) is what `value`
+measures; L2 is flushed (a 512 MiB write) between steps, outside the timed
+windows.  --weights runs the same batch on a pool of FP8 E4M3 or INT4 codes.  `e2e` repeats the step through the same public API with
 host buffers: the step's x and y rows go host->device from pinned memory and y
 comes back device->host, all inside the timed window, with the host builder.
 

@@ -174,8 +174,15 @@ SGMV_API sgmv_status sgmv_pool_destroy(sgmv_pool* pool);
  * arrays of n_proj pointers.  The pointed-to data is device memory when
  * src_on_device != 0, host memory otherwise.  The copies are enqueued on
  * `stream` and the call waits for them before returning, so the sources may be
- * freed afterwards.  SGMV_ERR_OUT_OF_PAGES leaves the pool unchanged.  A
- * quantised pool quantises the bf16 rows on the device as it stores them.
+ * freed afterwards.  SGMV_ERR_OUT_OF_PAGES leaves the pool unchanged (a
+ * resident adapter being replaced stays resident).  SGMV_ERR_CUDA (a copy
+ * failed) leaves the adapter not resident -- a replaced one included -- with
+ * every page back on the free list.  A quantised pool quantises the bf16 rows
+ * on the device as it stores them.
+ * Replacing a resident adapter frees its pages and may hand the same pages
+ * straight back to the new weights, which are written on `stream`: as for
+ * sgmv_pool_evict, no kernel enqueued on another stream may still read the old
+ * adapter when the call is made.
  */
 SGMV_API sgmv_status sgmv_pool_load(sgmv_pool* pool, int32_t adapter_id, int32_t rank,
                            const void* const* A, const void* const* B, int src_on_device,
@@ -459,6 +466,9 @@ SGMV_API sgmv_status sgmv_lora_delta_grouped(const sgmv_delta_entry* entries, in
  *     <= 2^19, else SGMV_ERR_CAPACITY (nothing launched).
  *   - The first call on a device looks up the array's device address, with
  *     that device current; make that first call before any stream capture.
+ *     The address is kept for the life of the process: after cudaDeviceReset
+ *     (which ends the context the address belongs to) do not call this entry
+ *     point on that device again.
  *   - All calls on a device share the array, which keeps the last call's
  *     contents (nothing in it needs to start at zero).  Calls whose kernels
  *     overlap on the same device race on it: serialise them (one stream).

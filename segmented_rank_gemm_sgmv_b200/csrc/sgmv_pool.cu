@@ -180,14 +180,31 @@ void release(sgmv_pool* p, int32_t adapter_id) {
     p->adapters.erase(it);
 }
 
-// Host bookkeeping of a load: drop the adapter's old placement, take a
-// page-table range and pages from the free stack.  False (nothing changed
-// beyond the release) when the page table has no free range that long.
+// Host bookkeeping of a load: find a page-table range for the new placement
+// (the adapter's old range, if any, counting as free), then drop the old
+// placement and take the range and pages from the free stack.  False, with
+// nothing changed (a resident adapter stays resident), when the page table has
+// no free range that long.  The caller has checked that the free pages (plus
+// the old placement's) suffice.
 bool place(sgmv_pool* p, int32_t adapter_id, int32_t rank, AdapterRec* rec) {
     const int64_t need = adapter_pages(p, rank);
-    release(p, adapter_id);
+    auto old = p->adapters.find(adapter_id);
     int64_t start = 0;
-    if (!pt_alloc(p, need, &start)) return false;
+    if (old == p->adapters.end()) {
+        if (!pt_alloc(p, need, &start)) return false;
+    } else {
+        // first fit on a copy of the free ranges with the old range returned: the same
+        // search on the real map after the release below gives the same range
+        const std::map<int64_t, int64_t> saved = p->free_pt;
+        pt_free(p, old->second.pt_begin, old->second.pt_count);
+        const bool fits = pt_alloc(p, need, &start);
+        p->free_pt = saved;
+        if (!fits) return false;
+        release(p, adapter_id);
+        int64_t again = 0;
+        pt_alloc(p, need, &again);
+        start = again;
+    }
     rec->rank = rank;
     rec->pt_begin = start;
     rec->pt_count = need;
@@ -205,6 +222,16 @@ bool place(sgmv_pool* p, int32_t adapter_id, int32_t rank, AdapterRec* rec) {
         p->free_pages.pop_back();
     }
     return true;
+}
+
+// Undo a placement that no adapter took (its copies failed): its pages and its
+// page-table range go back to the free lists.
+void unplace(sgmv_pool* p, const AdapterRec& rec) {
+    for (int64_t e = rec.pt_begin; e < rec.pt_begin + rec.pt_count; ++e) {
+        p->free_pages.push_back(p->pt_host[e]);
+        p->pt_host[e] = -1;
+    }
+    pt_free(p, rec.pt_begin, rec.pt_count);
 }
 
 }  // namespace
@@ -308,7 +335,10 @@ extern "C" sgmv_status sgmv_pool_load(sgmv_pool* p, int32_t adapter_id, int32_t 
     if (!place(p, adapter_id, rank, &rec)) return fail(SGMV_ERR_OUT_OF_PAGES, "pool_load: page table is fragmented");
     const int64_t start = rec.pt_begin;
 
-    if (p->device >= 0 && need > 0) {
+    // the copies; if one fails, the placement goes back to the free lists (the pool stays
+    // consistent, and the adapter -- a replaced one included -- is not resident)
+    auto copy_in = [&]() -> sgmv_status {
+        if (p->device < 0 || need == 0) return SGMV_OK;
         SGMV_CUDA_TRY(cudaSetDevice(p->device));
         SGMV_CUDA_TRY(cudaMemcpyAsync(p->pt_dev + start, p->pt_host.data() + start, (size_t)need * sizeof(int32_t),
                                       cudaMemcpyHostToDevice, stream));
@@ -340,6 +370,12 @@ extern "C" sgmv_status sgmv_pool_load(sgmv_pool* p, int32_t adapter_id, int32_t 
             }
         }
         SGMV_CUDA_TRY(cudaStreamSynchronize(stream));
+        return SGMV_OK;
+    };
+    const sgmv_status st = copy_in();
+    if (st != SGMV_OK) {
+        unplace(p, rec);
+        return st;
     }
     p->adapters[adapter_id] = std::move(rec);
     return SGMV_OK;
@@ -599,7 +635,11 @@ extern "C" sgmv_status sgmv_residency_prepare(sgmv_residency* r, const int32_t* 
         AdapterRec rec;
         if (!place(p, a, h.rank, &rec))
             return fail(SGMV_ERR_OUT_OF_PAGES, "residency_prepare: page table is fragmented");
-        if (dev && rec.pt_count > 0) {
+        // a failed copy returns this adapter's placement to the free lists (adapters loaded
+        // before it in this call stay resident)
+        int64_t loaded_bytes = 0;
+        auto copy_in = [&]() -> sgmv_status {
+            if (!dev || rec.pt_count == 0) return SGMV_OK;
             SGMV_CUDA_TRY(cudaMemcpyAsync(p->pt_dev + rec.pt_begin, p->pt_host.data() + rec.pt_begin,
                                           (size_t)rec.pt_count * sizeof(int32_t), cudaMemcpyHostToDevice,
                                           copy_stream));
@@ -613,10 +653,17 @@ extern "C" sgmv_status sgmv_residency_prepare(sgmv_residency* r, const int32_t* 
                                                   cudaMemcpyHostToDevice, copy_stream));
                     SGMV_CUDA_TRY(write_matrix(p, static_cast<const uint16_t*>(r->staging), h.rank, cols, m == 1,
                                                m == 0 ? rec.a_pt[i] : rec.b_pt[i], copy_stream));
-                    r->stats.bytes_loaded += (int64_t)bytes;
+                    loaded_bytes += (int64_t)bytes;
                 }
             }
+            return SGMV_OK;
+        };
+        const sgmv_status st = copy_in();
+        if (st != SGMV_OK) {
+            unplace(p, rec);
+            return st;
         }
+        r->stats.bytes_loaded += loaded_bytes;
         p->adapters[a] = std::move(rec);
         r->used[a] = tick;
     }

@@ -166,3 +166,33 @@ def test_pool_bookkeeping_properties(ops, fmt):
         assert len(owned) == len(set(owned)) and all(0 <= x < 300 for x in owned)
         st_ = pool.stats()
         assert st_.free_pages == 300 - len(owned) and st_.resident_adapters == len(resident)
+
+
+def test_replace_keeps_or_moves_the_adapter_consistently():
+    """Replacing a resident adapter: the placement is searched with the adapter's own
+    page-table range counted as free, and the old placement is dropped only once a new
+    one is found.  A replace refused for lack of pages keeps the old adapter as it was;
+    one that grows into its own freed range and the free space after it succeeds there.
+
+    (A refusal for lack of a long enough free page-table range, with enough free pages,
+    takes the same path -- nothing is released before the range is found -- but could
+    not be produced through the API: the table holds 2 * num_pages + 1024 entries, and
+    first-fit placement never fragmented it that far in randomised load / evict runs.)"""
+    # page_elems 64, one 64 -> 64 projection: rank r takes 2 r pages and 2 r table entries
+    pool = sg.AdapterPool([(64, 64)], num_pages=300, page_elems=64, max_rank=128, device=-1)
+    pool.load(1000, 40)                                   # entries [0, 80), pages 0..79
+    before = {m: pool.page_ids(1000, 0, m).tolist() for m in (0, 1)}
+    pool.load(1, 100)                                     # 200 more pages: 20 left
+    free_before = pool.stats().free_pages
+    with pytest.raises(sg.SgmvError) as e:                # 80 + 20 pages < 2 * 51
+        pool.load(1000, 51)
+    assert e.value.status == 4                            # SGMV_ERR_OUT_OF_PAGES
+    assert pool.rank_of(1000) == 40
+    assert {m: pool.page_ids(1000, 0, m).tolist() for m in (0, 1)} == before
+    assert pool.stats().free_pages == free_before
+    pool.evict(1)
+    pool.load(1000, 45)                                   # grows in place: [0, 90)
+    assert pool.rank_of(1000) == 45
+    ids = pool.page_ids(1000, 0, 0).tolist() + pool.page_ids(1000, 0, 1).tolist()
+    assert len(ids) == len(set(ids)) == 90
+    assert pool.stats().free_pages == 300 - 90

@@ -5,7 +5,7 @@ Only `tests/`, `__graft_entry__.smoke()` and the CPU-baseline leg of
 imports nothing from the CUDA library.
 
 Contents
-  lora_delta(...)        fp64 loops of y_t = W x_t + B_{a(t)} A_{a(t)} x_t (C, sgmv_oracle.c)
+  lora_delta(...)        fp64 loops of y_t = W x_t + s * s_{a(t)} B_{a(t)} A_{a(t)} x_t (C, sgmv_oracle.c)
   group_by_adapter(ids)  one segment per adapter, by brute-force sorting
   adapter_bytes(...)     the bytes-per-matrix formula of section "The maths that matters"
 
@@ -54,7 +54,7 @@ def _load():
             i64, i64, i64, dp, i64, dp, i64, i64,
             ctypes.POINTER(i64), ctypes.POINTER(i64),
             ctypes.POINTER(dp), ctypes.POINTER(dp), ctypes.POINTER(i64),
-            ctypes.c_double, dp, i64, dp, ctypes.c_int]
+            ctypes.c_double, dp, dp, i64, dp, ctypes.c_int]
         lib.oracle_threads.restype = ctypes.c_int
         lib.oracle_threads.argtypes = [ctypes.c_int]
         _lib = lib
@@ -72,7 +72,8 @@ def _dp(a: np.ndarray):
 def lora_delta(x: np.ndarray, y_in: np.ndarray, seg_offsets: Sequence[int],
                seg_rank: Sequence[int], A: List[np.ndarray], B: List[np.ndarray],
                token_idx: Optional[Sequence[int]] = None, scale: float = 1.0,
-               ldv: Optional[int] = None, threads: int = 1) -> Tuple[np.ndarray, np.ndarray]:
+               ldv: Optional[int] = None, threads: int = 1,
+               seg_scale: Optional[Sequence[float]] = None) -> Tuple[np.ndarray, np.ndarray]:
     """fp64 reference of the per-token delta ([SGMV post], "SGMV: the kernel that holds
     it all up": per-token equation, shrink then expand).
 
@@ -81,6 +82,11 @@ def lora_delta(x: np.ndarray, y_in: np.ndarray, seg_offsets: Sequence[int],
     A[s]   float64 [r_s][d_in],  B[s] float64 [d_out][r_s]   (logical orientation of
            "The bare mechanism": A in R^{r x d_in}, B in R^{d_out x r})
     seg_offsets [S+1], seg_rank [S], token_idx [rows] (row -> token) or None (identity)
+    scale      one multiplier for the whole call
+    seg_scale  [S] multiplier of each segment's adapter (LoRA's alpha/r), or None (all 1):
+               a token of segment s gets y_t + (scale * seg_scale[s]) * B_s A_s x_t.  The
+               pages give no scaling; one number per adapter, applied to its delta, is the
+               plainest reading of "W' = W + BA" with LoRA's usual alpha/r factor.
     Returns (v [rows][ldv] float64, y [T][d_out] float64).
     """
     lib = _load()
@@ -113,13 +119,19 @@ def lora_delta(x: np.ndarray, y_in: np.ndarray, seg_offsets: Sequence[int],
         tix = np.ascontiguousarray(np.asarray(token_idx, dtype=np.int64))
         assert tix.size == rows
         tix_p = tix.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+    if seg_scale is None:
+        ss, ss_p = None, None
+    else:
+        ss = np.ascontiguousarray(np.asarray(seg_scale, dtype=np.float64))
+        assert ss.size == S
+        ss_p = _dp(ss)
     v = np.zeros((max(rows, 0), ldv), dtype=np.float64)
     y = np.empty_like(y_in)
     rc = lib.oracle_lora_delta(
         T, d_in, d_out, _dp(x), d_in, _dp(y_in), d_out, S,
         off.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
         rk.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
-        A_ptrs, B_ptrs, tix_p, float(scale), _dp(v), ldv, _dp(y), int(threads))
+        A_ptrs, B_ptrs, tix_p, float(scale), ss_p, _dp(v), ldv, _dp(y), int(threads))
     if rc != 0:
         raise ValueError(f"oracle_lora_delta rejected its arguments (code {rc})")
     return v, y

@@ -16,8 +16,12 @@
  *
  * with A in R^{r x d_in} and B in R^{d_out x r} as in section "The bare
  * mechanism" (equation y = W x + B(Ax)).  The input y already holds W x.
- * `scale` is one real number per call (the pages give no LoRA scaling; the
- * plainest reading is a single multiplier, 1.0 in every workload).
+ * The pages give no LoRA scaling.  Reading taken: the delta of a token is
+ * multiplied by `scale` (one real number per call, 1.0 in every workload)
+ * times the multiplier of its segment's adapter, seg_scale[s] (LoRA's alpha/r
+ * of that adapter; all 1.0 when seg_scale is NULL):
+ *
+ *   y_t = y_t + (scale * seg_scale[s]) * B_s v_t,   t in segment s
  *
  * Tokens are visited segment by segment (one segment per adapter, "groups
  * the batch's tokens by adapter"), but every token's result depends only on
@@ -44,6 +48,7 @@ int oracle_lora_delta(int64_t T, int64_t d_in, int64_t d_out,
                       const double* const* B,               /* [S] -> [d_out][r_s]         */
                       const int64_t* token_idx,             /* [rows] row -> token, NULL = identity */
                       double scale,
+                      const double* seg_scale,              /* [S] per-segment multiplier, NULL = 1 */
                       double* v, int64_t ldv,               /* [rows][ldv] out             */
                       double* y_out,                        /* [T][ldy] out                */
                       int threads)
@@ -89,11 +94,12 @@ int oracle_lora_delta(int64_t T, int64_t d_in, int64_t d_out,
             for (int64_t c = 0; c < d_in; ++c) acc += As[k * d_in + c] * xt[c];
             vi[k] = acc;
         }
-        /* phase 2, expand: y = y + scale * B v */
+        /* phase 2, expand: y = y + (scale * seg_scale[s]) * B v */
+        const double sc = seg_scale ? scale * seg_scale[s] : scale;
         for (int64_t j = 0; j < d_out; ++j) {
             double acc = 0.0;
             for (int64_t k = 0; k < r; ++k) acc += Bs[j * r + k] * vi[k];
-            y_out[t * ldy + j] = y_in[t * ldy + j] + scale * acc;
+            y_out[t * ldy + j] = y_in[t * ldy + j] + sc * acc;
         }
     }
     return 0;

@@ -234,3 +234,74 @@ def test_threads_give_identical_bits(threads):
     v1, y1 = oracle.lora_delta(*args, token_idx=c["tix"], threads=1)
     vn, yn = oracle.lora_delta(*args, token_idx=c["tix"], threads=threads)
     assert np.array_equal(y1, yn) and np.array_equal(v1, vn)
+
+
+# -- per-segment scale (LoRA's alpha / r of each adapter) -------------------------------
+# The pages give no LoRA scaling.  Reading: each adapter carries one multiplier applied to
+# its own delta, on top of the call's scale: y_t = y_t + (scale * s_{a(t)}) B A x_t.
+def test_segment_scale_merged_weights_identity():
+    """[SGMV post] "The bare mechanism": W' = W + BA, with each adapter's delta scaled by
+    its own factor c_s: the oracle equals the explicitly merged (W + scale c_s B_s A_s) x
+    for the tokens of each segment."""
+    rng = np.random.default_rng(11)
+    c = _rand_case(rng, 31, 40, 56, [3, 7, 1, 5])
+    scale, seg_scale = 0.75, [2.0, 0.125, -1.5, 3.25]
+    _, y = oracle.lora_delta(c["x"], c["y_in"], c["off"], c["ranks"], c["A"], c["B"],
+                             token_idx=c["tix"], scale=scale, seg_scale=seg_scale)
+    for s in range(len(c["ranks"])):
+        Wm = c["W"] + scale * seg_scale[s] * (c["B"][s] @ c["A"][s])
+        for i in range(c["off"][s], c["off"][s + 1]):
+            t = c["tix"][i]
+            ref = Wm @ c["x"][t]
+            np.testing.assert_allclose(y[t], ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_equal_segment_scales_are_one_call_scale():
+    """Every segment with the same factor c is the per-call form with scale * c, bit for
+    bit; all ones is the form without per-segment factors."""
+    rng = np.random.default_rng(12)
+    c = _rand_case(rng, 27, 24, 16, [2, 5, 3])
+    args = (c["x"], c["y_in"], c["off"], c["ranks"], c["A"], c["B"])
+    _, y_seg = oracle.lora_delta(*args, token_idx=c["tix"], scale=0.75, seg_scale=[1.5] * 3)
+    _, y_call = oracle.lora_delta(*args, token_idx=c["tix"], scale=0.75 * 1.5)
+    assert np.array_equal(y_seg, y_call)
+    _, y_one = oracle.lora_delta(*args, token_idx=c["tix"], scale=0.5, seg_scale=[1.0] * 3)
+    _, y_none = oracle.lora_delta(*args, token_idx=c["tix"], scale=0.5)
+    assert np.array_equal(y_one, y_none)
+
+
+def test_segment_scale_exact_integers_match_brute_force():
+    """Integer inputs and integer factors: every value is exact in fp64, so the oracle must
+    equal Python integers y_in + scale * c_s * B (A x) element by element."""
+    rng = np.random.default_rng(13)
+    T, d_in, d_out, ranks = 13, 64, 20, [4, 1, 3, 2]
+    off, x, A, B, y_in, tix = _int_case(rng, T, d_in, d_out, ranks)
+    seg_scale, scale = [3, -2, 0, 1], 2
+    v, y = oracle.lora_delta(x.astype(float), y_in.astype(float), off, ranks,
+                             [a.astype(float) for a in A], [b.astype(float) for b in B],
+                             token_idx=tix, scale=float(scale), seg_scale=[float(q) for q in seg_scale])
+    for s, r in enumerate(ranks):
+        for i in range(off[s], off[s + 1]):
+            t = int(tix[i])
+            vv = [sum(int(A[s][k][cc]) * int(x[t][cc]) for cc in range(d_in)) for k in range(r)]
+            for j in range(d_out):
+                want = int(y_in[t][j]) + scale * seg_scale[s] * sum(int(B[s][j][k]) * vv[k] for k in range(r))
+                assert y[t, j] == want
+
+
+def test_segment_scale_acts_on_its_own_segment_only():
+    """With y_in = 0 the result is the scaled delta itself: doubling one segment's factor
+    doubles exactly that segment's rows (exact in fp64), a zero factor leaves its rows
+    at y_in, and every other row keeps its bits."""
+    rng = np.random.default_rng(14)
+    c = _rand_case(rng, 25, 16, 12, [2, 3, 4])
+    y0 = np.zeros_like(c["y_in"])
+    args = (c["x"], y0, c["off"], c["ranks"], c["A"], c["B"])
+    _, y_a = oracle.lora_delta(*args, token_idx=c["tix"], seg_scale=[1.0, 0.5, 1.25])
+    _, y_b = oracle.lora_delta(*args, token_idx=c["tix"], seg_scale=[1.0, 1.0, 1.25])
+    _, y_z = oracle.lora_delta(*args, token_idx=c["tix"], seg_scale=[1.0, 0.0, 1.25])
+    rows1 = c["tix"][c["off"][1]:c["off"][2]]
+    others = [t for t in range(25) if t not in set(rows1.tolist())]
+    assert np.array_equal(y_b[rows1], 2.0 * y_a[rows1])
+    assert np.array_equal(y_b[others], y_a[others])
+    assert np.array_equal(y_z[rows1], y0[rows1]) and np.array_equal(y_z[others], y_a[others])

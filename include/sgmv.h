@@ -4,9 +4,10 @@
  * The library computes, for every token t of a batch whose tokens carry
  * different LoRA adapters a(t),
  *
- *     y_t  <-  y_t + scale * B_{a(t)} ( A_{a(t)} x_t )
+ *     y_t  <-  y_t + scale * s_{a(t)} * B_{a(t)} ( A_{a(t)} x_t )
  *
- * where y already holds the base output W x_t.  Pages cited by title:
+ * where y already holds the base output W x_t, scale is the call's and s_a
+ * the adapter's own multiplier (1.0 unless set).  Pages cited by title:
  *
  *   [SGMV post] "Multi-LoRA serving: the single translator with a thousand
  *               glossaries -- shared base, thousands of concurrent adapters
@@ -190,6 +191,19 @@ SGMV_API sgmv_status sgmv_pool_load(sgmv_pool* pool, int32_t adapter_id, int32_t
 /* Remove an adapter and return its pages to the free list.  The caller must
  * not evict an adapter that an enqueued kernel may still read. */
 SGMV_API sgmv_status sgmv_pool_evict(sgmv_pool* pool, int32_t adapter_id);
+/*
+ * Multiplier of adapter `adapter_id`'s delta (LoRA's alpha / r for that
+ * adapter): a token on that adapter gets y_t + (scale * s_a) B_a A_a x_t,
+ * where `scale` is the expand call's argument.  The pages give no LoRA
+ * scaling ("Multi-LoRA serving: the single translator ...", section "The bare
+ * mechanism", W' = W + BA); one factor per adapter on its own delta is the
+ * reading taken.  The factor belongs to the id, resident or not: it is kept
+ * across evictions and reloads until changed, and is 1.0 for an id never set.
+ * The segment builder copies it into the plan (seg_scale), so a change takes
+ * effect for plans built afterwards.  SGMV_ERR_INVALID for a non-finite scale.
+ */
+SGMV_API sgmv_status sgmv_pool_set_adapter_scale(sgmv_pool* pool, int32_t adapter_id, float scale);
+SGMV_API sgmv_status sgmv_pool_get_adapter_scale(const sgmv_pool* pool, int32_t adapter_id, float* scale);
 SGMV_API sgmv_status sgmv_pool_get_stats(const sgmv_pool* pool, sgmv_pool_stats* out);
 /* Rank of a resident adapter; SGMV_ERR_NOT_RESIDENT otherwise. */
 SGMV_API sgmv_status sgmv_pool_adapter_rank(const sgmv_pool* pool, int32_t adapter_id, int32_t* rank);
@@ -239,6 +253,8 @@ SGMV_API const void* sgmv_pool_pages_device(const sgmv_pool* pool);
  *   seg_offsets int32 [num_segments+1]   rows of segment s: [off[s], off[s+1])
  *   seg_adapter int32 [num_segments]
  *   seg_rank    int32 [num_segments]
+ *   seg_scale   float [num_segments]     the segment's adapter multiplier
+ *                                        (sgmv_pool_set_adapter_scale) at build time
  *   seg_a_pt    int64 [num_segments*n_proj]  first page-table entry of A, per projection
  *   seg_b_pt    int64 [num_segments*n_proj]  first page-table entry of B^T
  *   simt_items  record [num_simt_items][n_proj]
@@ -275,6 +291,7 @@ typedef struct {
     int64_t off_seg_a_pt, off_seg_b_pt, off_simt_items, off_tc_tiles;
     const void* host_table; /* the host table the builder wrote; it must still hold that
                                table when sgmv_shrink / sgmv_expand are called          */
+    int64_t off_seg_scale;
 } sgmv_plan;
 
 /* ------------------------------------------------------------------------
@@ -378,9 +395,11 @@ SGMV_API sgmv_status sgmv_shrink(const void* x, int64_t ldx, int32_t T, int32_t 
  * projection r -> d_out with B_{a(t)}, accumulated into Y as in the TL;DR's
  * "Y +=" form):
  *
- *   y[t][j] <- round( y[t][j] + scale * sum_{k < r_s} B_s[j][k] * v[i][k] ),  t = token_idx[i]
+ *   y[t][j] <- round( y[t][j] + (scale * s_s) * sum_{k < r_s} B_s[j][k] * v[i][k] ),  t = token_idx[i]
  *
- * computed in fp32 with one rounding to the output type.
+ * computed in fp32 with one rounding to the output type; s_s is the multiplier
+ * of segment s's adapter (seg_scale of the plan, 1.0 unless set with
+ * sgmv_pool_set_adapter_scale).
  * y        device [T][ldy] updated in place, ldy >= d_out, rows 16-byte aligned;
  *          y_dtype 0 = bf16 (round to nearest even), 1 = fp32.
  * Rows of tokens in no segment are not read or written.
@@ -397,8 +416,9 @@ SGMV_API sgmv_status sgmv_expand(const float* v, int64_t ldv, int32_t T, int32_t
  * Both phases in one call ([SGMV post], "SGMV: the kernel that holds it all
  * up": one pass computes the delta of every token):
  *
- *   y[t][j] <- round( y[t][j] + scale * sum_k B_s[j][k] * sum_c A_s[k][c] * x[t][c] )
+ *   y[t][j] <- round( y[t][j] + (scale * s_s) * sum_k B_s[j][k] * sum_c A_s[k][c] * x[t][c] )
  *
+ * (s_s: the adapter's multiplier, as for sgmv_expand)
  * = sgmv_shrink into v, then sgmv_expand from v, on `stream`; the expand's
  * SIMT launch overlaps the shrink (programmatic dependent launch), so the
  * second launch costs little ([Glossary], "Limits and open questions", names

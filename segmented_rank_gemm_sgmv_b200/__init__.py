@@ -32,6 +32,7 @@ _STATUS = {0: "SGMV_OK", 1: "SGMV_ERR_INVALID", 2: "SGMV_ERR_UNSUPPORTED", 3: "S
 EXPORTED = ("sgmv_status_string", "sgmv_last_error", "sgmv_pool_create", "sgmv_pool_create_ex",
             "sgmv_pool_destroy", "sgmv_pool_load", "sgmv_pool_read",
             "sgmv_pool_evict", "sgmv_pool_get_stats", "sgmv_pool_adapter_rank", "sgmv_pool_adapter_pages",
+            "sgmv_pool_set_adapter_scale", "sgmv_pool_get_adapter_scale",
             "sgmv_pool_shuffle_free_pages", "sgmv_pool_pages_device", "sgmv_plan_table_capacity",
             "sgmv_build_plan", "sgmv_shrink", "sgmv_expand", "sgmv_lora_delta", "sgmv_lora_delta_grouped",
             "sgmv_lora_delta_noalloc", "sgmv_check_errors", "sgmv_residency_create", "sgmv_residency_destroy",
@@ -50,7 +51,8 @@ class Plan(ctypes.Structure):
         "T", "num_segments", "num_rows", "max_rank", "n_proj", "num_simt_items", "num_tc_tiles",
         "long_threshold", "max_item_rows", "needs_device_table")] + [(n, ctypes.c_int64) for n in (
             "table_bytes", "off_token_idx", "off_seg_offsets", "off_seg_adapter", "off_seg_rank",
-            "off_seg_a_pt", "off_seg_b_pt", "off_simt_items", "off_tc_tiles")] + [("host_table", ctypes.c_void_p)]
+            "off_seg_a_pt", "off_seg_b_pt", "off_simt_items", "off_tc_tiles")] + [("host_table", ctypes.c_void_p),
+                                                                                   ("off_seg_scale", ctypes.c_int64)]
 
 
 class DeltaEntry(ctypes.Structure):
@@ -99,6 +101,8 @@ def load_library() -> ctypes.CDLL:
         "sgmv_pool_evict": (st, [vp, i32]),
         "sgmv_pool_get_stats": (st, [vp, ctypes.POINTER(PoolStats)]),
         "sgmv_pool_adapter_rank": (st, [vp, i32, ctypes.POINTER(i32)]),
+        "sgmv_pool_set_adapter_scale": (st, [vp, i32, f32]),
+        "sgmv_pool_get_adapter_scale": (st, [vp, i32, ctypes.POINTER(f32)]),
         "sgmv_pool_adapter_pages": (st, [vp, i32, i32, i32, vp, i64, ctypes.POINTER(i64)]),
         "sgmv_pool_shuffle_free_pages": (st, [vp, ctypes.c_uint64]),
         "sgmv_pool_pages_device": (vp, [vp]),
@@ -241,6 +245,16 @@ class AdapterPool:
             codes = codes.view(np.uint16)
         return codes, scales
 
+    def set_scale(self, adapter_id: int, scale: float) -> None:
+        """Multiplier of the adapter's delta (its LoRA alpha / r), kept by id across
+        evictions and reloads; plans built afterwards carry it (sgmv_pool_set_adapter_scale)."""
+        _check(load_library().sgmv_pool_set_adapter_scale(self.handle, int(adapter_id), float(scale)))
+
+    def scale_of(self, adapter_id: int) -> float:
+        s = ctypes.c_float()
+        _check(load_library().sgmv_pool_get_adapter_scale(self.handle, int(adapter_id), ctypes.byref(s)))
+        return float(s.value)
+
     def rank_of(self, adapter_id: int) -> int:
         r = ctypes.c_int32()
         _check(load_library().sgmv_pool_adapter_rank(self.handle, int(adapter_id), ctypes.byref(r)))
@@ -336,6 +350,10 @@ class BatchPlan:
     @property
     def seg_rank(self) -> np.ndarray:
         return self._arr(self.plan.off_seg_rank, self.plan.num_segments, np.int32)
+
+    @property
+    def seg_scale(self) -> np.ndarray:
+        return self._arr(self.plan.off_seg_scale, self.plan.num_segments, np.float32)
 
     def seg_pt(self, matrix: int) -> np.ndarray:
         off = self.plan.off_seg_a_pt if matrix == 0 else self.plan.off_seg_b_pt

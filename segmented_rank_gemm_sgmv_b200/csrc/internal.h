@@ -48,6 +48,8 @@ struct sgmv_pool {
     std::vector<int64_t> free_pages; // stack of free page ids
     std::map<int64_t, int64_t> free_pt;  // free page-table ranges: start -> length
     std::unordered_map<int32_t, sgmv::AdapterRec> adapters;
+    std::unordered_map<int32_t, float> adapter_scale;  // per-adapter multiplier (1 when absent),
+                                                       // kept across evictions and reloads
     void* staging_dev = nullptr;     // device staging for host-source loads
     size_t staging_bytes = 0;
 };
@@ -80,6 +82,7 @@ template <int N>
 struct InlineTable {
     int32_t count, pad[3];
     InlineItem items[N];
+    float scale[N];              // multiplier of each item's adapter
 };
 constexpr int kTcTileRows = 128;       // rows per tensor-core tile (MMA M)
 constexpr int kDefaultLongThreshold = 16;
@@ -93,6 +96,7 @@ struct BatchView {
     const int32_t* seg_rank;
     const int64_t* seg_a_pt;
     const int64_t* seg_b_pt;
+    const float* seg_scale;      // [num_segments] multiplier of each segment's adapter
     const ItemRec* simt_items;   // [num_simt_items][n_proj]
     const ItemRec* tc_tiles;     // [num_tc_tiles][n_proj]
     int32_t num_segments, num_rows, n_proj, proj, T;

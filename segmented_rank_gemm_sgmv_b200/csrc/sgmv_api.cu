@@ -48,6 +48,7 @@ sgmv_status make_views(const sgmv_plan* plan, const void* table, const sgmv_pool
         bv->seg_rank = reinterpret_cast<const int32_t*>(base + plan->off_seg_rank);
         bv->seg_a_pt = reinterpret_cast<const int64_t*>(base + plan->off_seg_a_pt);
         bv->seg_b_pt = reinterpret_cast<const int64_t*>(base + plan->off_seg_b_pt);
+        bv->seg_scale = reinterpret_cast<const float*>(base + plan->off_seg_scale);
         bv->simt_items = reinterpret_cast<const ItemRec*>(base + plan->off_simt_items);
         bv->tc_tiles = reinterpret_cast<const ItemRec*>(base + plan->off_tc_tiles);
     }
@@ -74,6 +75,7 @@ bool inline_items(const sgmv_plan* plan, int32_t proj, InlineTable<kInlineItems>
     const uint8_t* base = static_cast<const uint8_t*>(plan->host_table);
     const ItemRec* recs = reinterpret_cast<const ItemRec*>(base + plan->off_simt_items);
     const int32_t* tix = reinterpret_cast<const int32_t*>(base + plan->off_token_idx);
+    const float* ssc = reinterpret_cast<const float*>(base + plan->off_seg_scale);
     t->count = plan->num_simt_items;
     for (int i = 0; i < plan->num_simt_items; ++i) {
         const ItemRec& r = recs[(int64_t)i * plan->n_proj + proj];
@@ -84,6 +86,7 @@ bool inline_items(const sgmv_plan* plan, int32_t proj, InlineTable<kInlineItems>
         it.rank = r.rank;
         it.a_pt = r.a_pt;
         it.b_pt = r.b_pt;
+        t->scale[i] = (r.seg >= 0 && r.seg < plan->num_segments) ? ssc[r.seg] : 1.0f;
         for (int j = 0; j < kSimtMaxItemRows; ++j) {
             const int row = r.row_begin + j;
             it.tok[j] = (row < r.row_end && row >= 0 && row < plan->num_rows) ? tix[row] : -1;

@@ -18,7 +18,7 @@ namespace {
 int64_t align16(int64_t n) { return (n + 15) & ~int64_t(15); }
 
 struct Layout {
-    int64_t token_idx, seg_offsets, seg_adapter, seg_rank, seg_a_pt, seg_b_pt, simt_items, tc_tiles, end;
+    int64_t token_idx, seg_offsets, seg_adapter, seg_rank, seg_scale, seg_a_pt, seg_b_pt, simt_items, tc_tiles, end;
 };
 
 Layout layout_for(int64_t rows, int64_t S, int64_t n_proj, int64_t n_simt, int64_t n_tc) {
@@ -28,6 +28,7 @@ Layout layout_for(int64_t rows, int64_t S, int64_t n_proj, int64_t n_simt, int64
     L.seg_offsets = o; o = align16(o + (S + 1) * 4);
     L.seg_adapter = o; o = align16(o + S * 4);
     L.seg_rank = o;    o = align16(o + S * 4);
+    L.seg_scale = o;   o = align16(o + S * 4);
     L.seg_a_pt = o;    o = align16(o + S * n_proj * 8);
     L.seg_b_pt = o;    o = align16(o + S * n_proj * 8);
     L.simt_items = o;  o = align16(o + n_simt * n_proj * 32);
@@ -123,6 +124,7 @@ extern "C" sgmv_status sgmv_build_plan(const int32_t* adapter_ids, int32_t T, co
     int32_t* seg_offsets = reinterpret_cast<int32_t*>(base + L.seg_offsets);
     int32_t* seg_adapter = reinterpret_cast<int32_t*>(base + L.seg_adapter);
     int32_t* seg_rank = reinterpret_cast<int32_t*>(base + L.seg_rank);
+    float* seg_scale = reinterpret_cast<float*>(base + L.seg_scale);
     int64_t* seg_a_pt = reinterpret_cast<int64_t*>(base + L.seg_a_pt);
     int64_t* seg_b_pt = reinterpret_cast<int64_t*>(base + L.seg_b_pt);
     auto recs_rank = [&](int32_t s) { return recs[s]->rank; };
@@ -149,6 +151,8 @@ extern "C" sgmv_status sgmv_build_plan(const int32_t* adapter_ids, int32_t T, co
     for (int64_t s = 0; s < S; ++s) {
         seg_adapter[s] = ids[s];
         seg_rank[s] = recs[s]->rank;
+        const auto sc = pool->adapter_scale.find(ids[s]);
+        seg_scale[s] = sc == pool->adapter_scale.end() ? 1.0f : sc->second;
         for (int64_t p = 0; p < n_proj; ++p) {
             seg_a_pt[s * n_proj + p] = recs[s]->a_pt[p];
             seg_b_pt[s * n_proj + p] = recs[s]->b_pt[p];
@@ -185,6 +189,7 @@ extern "C" sgmv_status sgmv_build_plan(const int32_t* adapter_ids, int32_t T, co
     plan->off_seg_offsets = L.seg_offsets;
     plan->off_seg_adapter = L.seg_adapter;
     plan->off_seg_rank = L.seg_rank;
+    plan->off_seg_scale = L.seg_scale;
     plan->off_seg_a_pt = L.seg_a_pt;
     plan->off_seg_b_pt = L.seg_b_pt;
     plan->off_simt_items = L.simt_items;

@@ -14,6 +14,7 @@
 #include <cuda_fp8.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstring>
 
 #include "internal.h"
@@ -385,6 +386,23 @@ extern "C" sgmv_status sgmv_pool_evict(sgmv_pool* p, int32_t adapter_id) {
     if (!p) return fail(SGMV_ERR_INVALID, "pool_evict: pool is NULL");
     if (!p->adapters.count(adapter_id)) return fail(SGMV_ERR_NOT_RESIDENT, "pool_evict: adapter not resident");
     release(p, adapter_id);
+    return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_pool_set_adapter_scale(sgmv_pool* p, int32_t adapter_id, float scale) {
+    if (!p) return fail(SGMV_ERR_INVALID, "pool_set_adapter_scale: pool is NULL");
+    if (adapter_id < 0) return fail(SGMV_ERR_INVALID, "pool_set_adapter_scale: adapter_id must be >= 0");
+    if (!std::isfinite(scale)) return fail(SGMV_ERR_INVALID, "pool_set_adapter_scale: scale must be finite");
+    if (scale == 1.0f) p->adapter_scale.erase(adapter_id);
+    else p->adapter_scale[adapter_id] = scale;
+    return SGMV_OK;
+}
+
+extern "C" sgmv_status sgmv_pool_get_adapter_scale(const sgmv_pool* p, int32_t adapter_id, float* scale) {
+    if (!p || !scale) return fail(SGMV_ERR_INVALID, "pool_get_adapter_scale: NULL argument");
+    if (adapter_id < 0) return fail(SGMV_ERR_INVALID, "pool_get_adapter_scale: adapter_id must be >= 0");
+    const auto it = p->adapter_scale.find(adapter_id);
+    *scale = it == p->adapter_scale.end() ? 1.0f : it->second;
     return SGMV_OK;
 }
 

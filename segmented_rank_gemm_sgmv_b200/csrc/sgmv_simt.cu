@@ -121,6 +121,7 @@ struct ExpandArgs {
 struct ItemInfo {
     int i0, n, r;
     int64_t pt;          // first page-table entry of the matrix for this projection
+    float sc;            // multiplier of the item's adapter (read for the expand only)
     bool ok;
     int tok[kSimtMaxItemRows];  // token rows of the item (-1 past n or when out of range)
 };
@@ -159,6 +160,7 @@ __device__ __forceinline__ ItemInfo load_item(const BatchView& b, int proj, int 
     check_item(b, m, h.x, h.z, max_rows, max_rank);
     m.pt = matrix == 0 ? (int64_t)(((uint64_t)(uint32_t)t.y << 32) | (uint32_t)t.x)
                        : (int64_t)(((uint64_t)(uint32_t)t.w << 32) | (uint32_t)t.z);
+    m.sc = (matrix == 1 && m.ok) ? b.seg_scale[h.x] : 1.f;  // (segment checked above)
 #pragma unroll
     for (int j = 0; j < kSimtMaxItemRows; ++j) m.tok[j] = j < m.n ? b.token_idx[m.i0 + j] : -1;
     finish_tokens(b, m);
@@ -176,6 +178,7 @@ __device__ __forceinline__ ItemInfo load_item(const BatchView& b, const InlineTa
     m.r = it.rank;
     check_item(b, m, it.seg, it.row_end, max_rows, max_rank);
     m.pt = matrix == 0 ? it.a_pt : it.b_pt;
+    m.sc = t.scale[idx];
 #pragma unroll
     for (int j = 0; j < kSimtMaxItemRows; ++j) m.tok[j] = it.tok[j];
     finish_tokens(b, m);
@@ -531,6 +534,7 @@ __device__ void expand_item(const ExpandArgs<NE>& a, const ExpandEntry& en, cons
                             Pipe<kExpandStages, WF>& pp, const StageGeom& sg, float* vs, const float* rsc) {
     constexpr int VB = bytes_per_8<WF>();
     const int tid = threadIdx.x, col = kVec * tid;
+    const float sc = a.scale * m.sc;  // the call's scale times the adapter's
     int trow[G];
 #pragma unroll
     for (int j = 0; j < G; ++j) trow[j] = m.tok[j];
@@ -615,8 +619,8 @@ __device__ void expand_item(const ExpandArgs<NE>& a, const ExpandEntry& en, cons
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float lo = fmaf(a.scale, acc[j][2 * e], yv[2 * e]);
-                    const float hi = fmaf(a.scale, acc[j][2 * e + 1], yv[2 * e + 1]);
+                    const float lo = fmaf(sc, acc[j][2 * e], yv[2 * e]);
+                    const float hi = fmaf(sc, acc[j][2 * e + 1], yv[2 * e + 1]);
                     w[e] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
                            ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
                 }
@@ -625,10 +629,10 @@ __device__ void expand_item(const ExpandArgs<NE>& a, const ExpandEntry& en, cons
             } else {
                 float* yp = static_cast<float*>(en.y) + (int64_t)trow[j] * en.ldy + jcol;
                 float4 o0 = y0[j], o1 = y1[j];
-                o0.x = fmaf(a.scale, acc[j][0], o0.x); o0.y = fmaf(a.scale, acc[j][1], o0.y);
-                o0.z = fmaf(a.scale, acc[j][2], o0.z); o0.w = fmaf(a.scale, acc[j][3], o0.w);
-                o1.x = fmaf(a.scale, acc[j][4], o1.x); o1.y = fmaf(a.scale, acc[j][5], o1.y);
-                o1.z = fmaf(a.scale, acc[j][6], o1.z); o1.w = fmaf(a.scale, acc[j][7], o1.w);
+                o0.x = fmaf(sc, acc[j][0], o0.x); o0.y = fmaf(sc, acc[j][1], o0.y);
+                o0.z = fmaf(sc, acc[j][2], o0.z); o0.w = fmaf(sc, acc[j][3], o0.w);
+                o1.x = fmaf(sc, acc[j][4], o1.x); o1.y = fmaf(sc, acc[j][5], o1.y);
+                o1.z = fmaf(sc, acc[j][6], o1.z); o1.w = fmaf(sc, acc[j][7], o1.w);
                 *reinterpret_cast<float4*>(yp) = o0;
                 *reinterpret_cast<float4*>(yp + 4) = o1;
             }

@@ -482,6 +482,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
     struct Unit {
         int tile, row_begin, rows, r, j0;
         int64_t b_base;
+        float sc;  // multiplier of the tile's adapter
         bool ok;
     };
     auto unit = [&](int u) {
@@ -495,6 +496,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
         w.b_base = it.b_pt;
         w.ok = !(it.seg < 0 || it.seg >= a.b.num_segments || it.row_begin < 0 || w.rows <= 0 ||
                  w.rows > kTcTileRows || it.row_end > a.b.num_rows || w.r <= 0 || ((w.r + 15) & ~15) > kpm);
+        w.sc = w.ok ? a.b.seg_scale[it.seg] : 1.f;
         return w;
     };
     auto wait = [&](uint64_t* bar, uint32_t parity) {
@@ -770,6 +772,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
                 if (t >= a.b.T) t = -1;
             }
             const bool row_ok = t >= 0 && !abort_flag;
+            const float sc = a.scale * w.sc;  // the call's scale times the adapter's
             for (int c00 = 0; c00 < NB; c00 += 64) {
                 uint32_t rr[2][32];  // two loads in flight per wait
                 const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(bsel * NB + c00);
@@ -792,8 +795,8 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
                             uint32_t wv[4];
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
-                                const float lo = fmaf(a.scale, __uint_as_float(regs[q4 * 8 + 2 * e]), yf[2 * e]);
-                                const float hi = fmaf(a.scale, __uint_as_float(regs[q4 * 8 + 2 * e + 1]), yf[2 * e + 1]);
+                                const float lo = fmaf(sc, __uint_as_float(regs[q4 * 8 + 2 * e]), yf[2 * e]);
+                                const float hi = fmaf(sc, __uint_as_float(regs[q4 * 8 + 2 * e + 1]), yf[2 * e + 1]);
                                 wv[e] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
                                         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
                             }
@@ -804,10 +807,10 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
                         for (int q4 = 0; q4 < 8; ++q4) {
                             float4* yp = reinterpret_cast<float4*>(yrow + ((((cc >> 2) + q4) ^ (m & 7)) << 4));
                             float4 yv = *yp;
-                            yv.x = fmaf(a.scale, __uint_as_float(regs[q4 * 4 + 0]), yv.x);
-                            yv.y = fmaf(a.scale, __uint_as_float(regs[q4 * 4 + 1]), yv.y);
-                            yv.z = fmaf(a.scale, __uint_as_float(regs[q4 * 4 + 2]), yv.z);
-                            yv.w = fmaf(a.scale, __uint_as_float(regs[q4 * 4 + 3]), yv.w);
+                            yv.x = fmaf(sc, __uint_as_float(regs[q4 * 4 + 0]), yv.x);
+                            yv.y = fmaf(sc, __uint_as_float(regs[q4 * 4 + 1]), yv.y);
+                            yv.z = fmaf(sc, __uint_as_float(regs[q4 * 4 + 2]), yv.z);
+                            yv.w = fmaf(sc, __uint_as_float(regs[q4 * 4 + 3]), yv.w);
                             *yp = yv;
                         }
                     }

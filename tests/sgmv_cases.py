@@ -76,9 +76,11 @@ def oracle_weights(bank, a, proj, weight_format: str = "bf16"):
 
 
 def run_oracle(wl, bank, proj, x, y, rows_of_tokens: Optional[List[int]] = None, scale=None,
-               adapter_ids=None, threads: int = 0, weight_format: str = "bf16"):
+               adapter_ids=None, threads: int = 0, weight_format: str = "bf16",
+               adapter_scale: Optional[Dict[int, float]] = None):
     """fp64 oracle on the whole batch, or on the listed tokens only (each token's
-    result depends only on its own row and adapter)."""
+    result depends only on its own row and adapter).  adapter_scale: the multiplier of
+    each adapter's delta (absent ids: 1), as set on the pool with set_scale."""
     ids = (wl.adapter_ids if adapter_ids is None else adapter_ids).tolist()
     tix, off, seg_ad = oracle.group_by_adapter(ids)
     if rows_of_tokens is not None:
@@ -89,9 +91,12 @@ def run_oracle(wl, bank, proj, x, y, rows_of_tokens: Optional[List[int]] = None,
     AB = [oracle_weights(bank, a, proj, weight_format) for a in seg_ad]
     A = [ab[0] for ab in AB]
     B = [ab[1] for ab in AB]
+    seg_scale = None
+    if adapter_scale:
+        seg_scale = [float(np.float32(adapter_scale.get(int(a), 1.0))) for a in seg_ad]
     v_ref, y_ref = oracle.lora_delta(workloads.bf16_to_f64(x), workloads.bf16_to_f64(y), off, ranks, A, B,
                                      token_idx=tix, scale=wl.scale if scale is None else scale,
-                                     threads=threads or (os.cpu_count() or 1))
+                                     threads=threads or (os.cpu_count() or 1), seg_scale=seg_scale)
     return dict(tix=tix, off=off, seg_ad=seg_ad, ranks=ranks, v=v_ref, y=y_ref)
 
 

@@ -172,3 +172,28 @@ def test_plan_properties(ids, runs, thr):
     _check_plan(plan, _shared_pool(), batch, _RANKS, plan.plan.long_threshold)
     if thr > 0:
         assert plan.plan.long_threshold == thr
+
+
+def test_plan_carries_each_adapter_scale():
+    """sgmv_pool_set_adapter_scale: the factor belongs to the adapter id (resident or
+    not, kept across evictions and reloads) and the builder copies it per segment."""
+    pool = sg.AdapterPool([(1024, 512)], num_pages=4000, page_elems=512, max_rank=64, device=-1)
+    for a, r in ((3, 16), (7, 8), (9, 32)):
+        pool.load(a, r)
+    pool.set_scale(7, 0.25)
+    pool.set_scale(9, -2.0)
+    pool.set_scale(11, 5.0)                      # an id that is not resident yet
+    plan = pool.plan([9, 3, -1, 7, 9, 7])
+    assert plan.seg_adapter.tolist() == [3, 7, 9]
+    assert plan.seg_scale.tolist() == [1.0, 0.25, -2.0]
+    pool.evict(7)
+    pool.load(7, 8)
+    pool.load(11, 16)
+    plan = pool.plan([11, 7])
+    assert plan.seg_scale.tolist() == [0.25, 5.0]
+    pool.set_scale(7, 1.0)
+    assert pool.scale_of(7) == 1.0 and pool.scale_of(11) == 5.0 and pool.scale_of(12345) == 1.0
+    for bad in (float("inf"), float("nan")):
+        with pytest.raises(sg.SgmvError) as e:
+            pool.set_scale(3, bad)
+        assert e.value.status == 1

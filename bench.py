@@ -7,7 +7,12 @@ One step is one pass of the whole hot path over one batch: the host segment
 builder (run every step, overlapped with the previous device work), one
 host-to-device copy of the segment table, then SGMV-shrink and SGMV-expand for
 every adapted projection of the workload (one grouped call for a multi-projection
-workload unless --per-projection).  The device time of a step (CUDA events on the
+workload unless --per-projection).  The default workload is the Llama-3-70B-shaped
+layer (7 adapted projections, 256 decode tokens each on its own rank-16 adapter of a
+pool of 2000): tokens/s per adapted layer.  At N = 1 the same run also measures every
+other workload (tiny, decode_q_proj, decode_q_proj_12, mixed_rank_mlp_up,
+prefill_long) and reports each under `per_workload` with its own step time, roofline
+and clocks (--no-per-workload skips them).  The device time of a step (CUDA events on the
 launching stream, from the table copy to the last expand) is what `value`
 measures; L2 is flushed (a 512 MiB write) between steps, outside the timed
 windows.  --weights runs the same batch on a pool of FP8 E4M3 or INT4 codes.  `e2e` repeats the step through the same public API with
@@ -17,6 +22,9 @@ comes back device->host, all inside the timed window, with the host builder.
 With N > 1 (torchrun) every rank runs its own batch of the same shape (weak
 scaling, no collective on the data path: the tokens of a batch are
 independent); the reported time is the max over ranks.
+
+The CPU baseline is the oracle on the machine's host cores, on the whole batch or, for the
+layer, on a bounded sample of its tokens (named in `cpu_baseline.sample`).
 
 Prints one JSON line (rank 0).
 """
@@ -199,7 +207,7 @@ def setup(wl_name: str, rank: int, device: int, pool_override: int = 0, weights:
     return sg, wl, pool, acts
 
 
-def run_ours(args, rank, world, device):
+def run_ours(args, rank, world, device, with_e2e=True):
     sg, wl, pool, acts = setup(args.workload, rank, device, args.pool, args.weights)
     n_proj = len(wl.projections)
     stream = torch.cuda.current_stream(device)
@@ -306,7 +314,9 @@ def run_ours(args, rank, world, device):
         res["phase_ms"] = {"shrink": float(np.mean([sum(ph(e, p, 0) for p in range(n_proj)) for e in records])),
                            "expand": float(np.mean([sum(ph(e, p, 1) for p in range(n_proj)) for e in records]))}
     res["achieved"] = res["step_bytes"] / (res["proj_ms"] * 1e-3) / 1e9
-    res["e2e"] = e2e_ours(sg, wl, pool, acts, args, device, stream, world)
+    if with_e2e:
+        res["e2e"] = e2e_ours(sg, wl, pool, acts, args, device, stream, world)
+    pool.close()
     return wl, res
 
 
@@ -372,13 +382,19 @@ def e2e_ours(sg, wl, pool, acts, args, device, stream, world):
 
 
 # ---------------------------------------------------------------------------- oracle arm
-def oracle_inputs(wl, device, weights: str = "bf16"):
+def oracle_inputs(wl, device, weights: str = "bf16", max_tokens: int = 0):
     """fp64 host copies of the batch's inputs (x, y, A, B of the adapters in use; in a
-    quantised pool's format, the dequantised weights, quantised here outside any timing)."""
+    quantised pool's format, the dequantised weights, quantised here outside any timing).
+    max_tokens > 0 keeps only the batch's first max_tokens adapted tokens (a bounded
+    sample: every token's delta depends on its own row and adapter only)."""
     bank = workloads.AdapterBank(wl, device=device)
     import oracle
     from oracle import quant as oquant
-    tix, off, seg_ad = oracle.group_by_adapter(wl.adapter_ids.tolist())
+    ids = wl.adapter_ids.tolist()
+    if max_tokens > 0:
+        keep = [t for t, a in enumerate(ids) if a >= 0][:max_tokens]
+        ids = [a if t in set(keep) else -1 for t, a in enumerate(ids)]
+    tix, off, seg_ad = oracle.group_by_adapter(ids)
     per_proj = []
 
     def weights_of(a, p):
@@ -421,7 +437,7 @@ def run_reference(args, rank, world, device):
     wl = workloads.make(args.workload, seed=0)
     threads = os.cpu_count() or 1
     dev = f"cuda:{device}" if torch.cuda.is_available() else "cpu"
-    prepared = oracle_inputs(wl, dev, args.weights)
+    prepared = oracle_inputs(wl, dev, args.weights, ORACLE_SAMPLE_TOKENS.get(wl.name, 0))
     for _ in range(args.warmup):
         time_oracle(prepared, wl, 0.0, threads)
     per_step_budget = max(0.05, getattr(args, "ref_budget", 60.0) / max(args.steps, 1))
@@ -437,10 +453,40 @@ def run_reference(args, rank, world, device):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": config_of(wl, args.weights),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
-                             "sample": f"whole batch ({n_tok} tokens x {len(wl.projections)} projections) "
-                                       f"repeated {reps_all} times over {args.steps} steps"},
+                             "sample": f"{sample_text(wl, n_tok)} repeated {reps_all} times over "
+                                       f"{args.steps} steps"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+# adapted tokens of the oracle's bounded sample, by workload (0: the whole batch)
+ORACLE_SAMPLE_TOKENS = {"llama70b_layer": 64}
+# workloads measured besides the headline one, each in the same process
+PER_WORKLOAD = ("tiny", "decode_q_proj", "decode_q_proj_12", "mixed_rank_mlp_up", "prefill_long",
+                "llama70b_layer")
+
+
+def sample_text(wl, n_tok: int) -> str:
+    whole = int((wl.adapter_ids >= 0).sum())
+    what = "whole batch" if n_tok == whole else f"first {n_tok} of the batch's {whole} tokens"
+    return f"{what} ({n_tok} tokens x {len(wl.projections)} projections)"
+
+
+def roofline_of(res) -> dict:
+    return {"bound": "hbm", "kernel": res["kernel_name"], "achieved": res["achieved"],
+            "peak": res["peak"], "unit": "GB/s", "frac": res["achieved"] / res["peak"],
+            "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if res["peak_kind"] == "measured"
+            else "fallback 6650 GB/s",
+            "algorithmic_bytes_per_step": res["step_bytes"],
+            "launches_per_step": res["dom_launches"],
+            "traffic": res["traffic"]}
+
+
+def per_workload_entry(wl, res, args, world) -> dict:
+    n_tok = int((wl.adapter_ids >= 0).sum())
+    return {"tokens": n_tok, "distinct_adapters": wl.distinct_adapters,
+            "value": job_value(world, n_tok, args.steps, res["total_ms"]), "unit": "tokens/s",
+            "ms_per_step": res["total_ms"] / args.steps, "roofline": roofline_of(res), "clocks": res["clocks"]}
 
 
 def config_of(wl, weights: str = "bf16"):
@@ -459,7 +505,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="decode_q_proj", choices=workloads.WORKLOAD_NAMES)
+    ap.add_argument("--workload", default="llama70b_layer", choices=workloads.WORKLOAD_NAMES)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--pool", type=int, default=0,
@@ -472,6 +518,8 @@ def main():
                     help="record an event between shrink and expand (times each phase; removes their overlap)")
     ap.add_argument("--weights", default="bf16", choices=sorted(WEIGHT_BYTES),
                     help="adapter storage of the pool: bf16, or FP8 E4M3 / INT4 codes with a scale per rank row")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the other workloads' lines (per_workload; measured at N = 1 only)")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-budget", type=float, default=60.0,
                     help="seconds of oracle time over all steps of --impl reference")
@@ -508,13 +556,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config_of(wl, args.weights),
             "hbm_gbs_step": res["step_bytes"] / (res["total_ms"] / args.steps * 1e-3) / 1e9,
-            "roofline": {"bound": "hbm", "kernel": res["kernel_name"], "achieved": res["achieved"],
-                         "peak": res["peak"], "unit": "GB/s", "frac": res["achieved"] / res["peak"],
-                         "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if res["peak_kind"] == "measured"
-                         else "fallback 6650 GB/s",
-                         "algorithmic_bytes_per_step": res["step_bytes"],
-                         "launches_per_step": res["dom_launches"],
-                         "traffic": res["traffic"]},
+            "roofline": roofline_of(res),
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
                     "d2h_bytes_per_step": e2e["d2h"]},
             "gpu_launches": res["launches"] * args.steps,
@@ -524,11 +566,24 @@ def main():
             line["phase_ms"] = res["phase_ms"]
             line["phase_us_per_proj"] = res["phase_us_per_proj"]
         if not args.no_cpu_baseline and world == 1:
-            prepared = oracle_inputs(wl, f"cuda:{local}", args.weights)
+            prepared = oracle_inputs(wl, f"cuda:{local}", args.weights, ORACLE_SAMPLE_TOKENS.get(wl.name, 0))
             rate, reps, el, used = time_oracle(prepared, wl, args.cpu_budget, os.cpu_count() or 1)
             line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": used, "kind": "oracle",
-                                    "sample": f"whole batch ({n_tok} tokens x {len(wl.projections)} projections)"
-                                              f" repeated {reps} times in {el:.1f} s"}
+                                    "sample": f"{sample_text(wl, len(prepared[0]))} repeated {reps} times"
+                                              f" in {el:.1f} s"}
+        if not args.no_per_workload and world == 1:
+            import copy
+            line["per_workload"] = {}
+            for name in PER_WORKLOAD:
+                if name == wl.name:
+                    continue
+                a2 = copy.copy(args)
+                a2.workload, a2.pool = name, 0
+                a2.grouped = not args.per_projection and not args.split_phases
+                wl2, res2 = run_ours(a2, rank, world, local, with_e2e=False)
+                line["per_workload"][name] = per_workload_entry(wl2, res2, a2, world)
+                del res2
+                torch.cuda.empty_cache()
         print(json.dumps(line), flush=True)
     finally:
         if world > 1:

@@ -78,23 +78,24 @@ def test_grouped_small_plan_without_device_table():
         compare(plan, vs[p], ys[p], acts[p][1], run_oracle(wl, bank, p, acts[p][0], acts[p][1]))
 
 
-def test_grouped_llama70b_layer_sampled():
-    """The 70B layer's 7 projections in one grouped call (the full pool of 2000
-    rank-16 adapters, 256 tokens on distinct adapters); the oracle recomputes a
-    sample of 32 tokens of every projection."""
+@pytest.mark.parametrize("y_dtype", [torch.bfloat16, torch.float32], ids=["ybf16", "yfp32"])
+def test_grouped_llama70b_layer(y_dtype):
+    """The 70B layer's 7 projections in one grouped call -- the launch configuration the
+    benchmark times (the full pool of 2000 rank-16 adapters, 256 tokens on distinct
+    adapters) -- against the oracle on every token of every projection: Gate A on bf16
+    y, Gate B (relative to the delta) on fp32 y."""
     wl = workloads.make("llama70b_layer")
     bank = workloads.AdapterBank(wl, device="cuda")
     pool = build_pool(wl, bank)
     acts = [workloads.activations(wl, p, device="cuda") for p in range(len(wl.projections))]
     plan = pool.plan(wl.adapter_ids)
     plan.upload()
-    ys = [y.clone() for _, y in acts]
+    ys = [y.to(y_dtype).clone() for _, y in acts]
     vs = sg.lora_delta_grouped([(acts[p][0], ys[p], p) for p in range(len(acts))], plan, pool)
     assert sg.check_errors() == 0
-    sample = sorted(np.random.default_rng(7).choice(wl.T, size=32, replace=False).tolist())
     for p in range(len(acts)):
-        ref = run_oracle(wl, bank, p, acts[p][0], acts[p][1], rows_of_tokens=sample)
-        compare(plan, vs[p], ys[p], acts[p][1], ref, check_rows=sample)
+        ref = run_oracle(wl, bank, p, acts[p][0], acts[p][1])
+        compare(plan, vs[p], ys[p], acts[p][1], ref)
 
 
 def test_grouped_argument_errors():

@@ -92,11 +92,14 @@ def test_tiny(path, y_dtype, mode):
 
 
 @MODES
-def test_decode_q_proj(mode):
+@pytest.mark.parametrize("y_dtype", [torch.bfloat16, torch.float32], ids=["ybf16", "yfp32"])
+def test_decode_q_proj(y_dtype, mode):
+    """Gate A on bf16 y, and Gate B on fp32 y: relative to the delta itself, which is
+    only ~1 % of y at d = 8192."""
     wl = workloads.make("decode_q_proj")
     bank = workloads.AdapterBank(wl, device="cuda")
     x, y = workloads.activations(wl, 0, device="cuda")
-    plan, *_ = check(wl, bank, x, y, 0, mode=mode)
+    plan, *_ = check(wl, bank, x, y, 0, y_dtype, mode=mode)
     assert plan.plan.num_tc_tiles == 0 and plan.plan.num_segments == wl.distinct_adapters
 
 
@@ -119,13 +122,15 @@ def test_mixed_rank_mlp_up(y_dtype, mode):
     assert len(set(plan.seg_rank.tolist())) == 4
 
 
-@pytest.mark.parametrize("path,mode", [(0, "separate"), (0, "lora_delta"), (SIMT, "separate")],
-                         ids=["dispatch", "dispatch-lora_delta", "simt"])
-def test_prefill_long(path, mode):
+@pytest.mark.parametrize("path,mode,y_dtype",
+                         [(0, "separate", torch.bfloat16), (0, "lora_delta", torch.bfloat16),
+                          (0, "lora_delta", torch.float32), (SIMT, "separate", torch.bfloat16)],
+                         ids=["dispatch", "dispatch-lora_delta", "dispatch-lora_delta-yfp32", "simt"])
+def test_prefill_long(path, mode, y_dtype):
     wl = workloads.make("prefill_long")
     bank = workloads.AdapterBank(wl, device="cuda")
     x, y = workloads.activations(wl, 0, device="cuda")
-    plan, *_ = check(wl, bank, x, y, path, mode=mode)
+    plan, *_ = check(wl, bank, x, y, path, y_dtype, mode=mode)
     if path == 0:
         assert plan.plan.num_tc_tiles == 32 and plan.plan.num_simt_items == 0
 
@@ -133,8 +138,9 @@ def test_prefill_long(path, mode):
 @MODES
 def test_llama70b_layer_sampled(mode):
     """Full-size layer (pool of 2000 rank-16 adapters, 7 projections, 256 tokens on
-    distinct adapters) in the launch configuration the benchmark times; the oracle
-    recomputes a sample of 32 tokens one by one for every projection."""
+    distinct adapters), one call per projection (the benchmark's grouped call over all
+    seven is checked on every token in tests/test_grouped_gpu.py); the oracle recomputes
+    a sample of 32 tokens one by one for every projection."""
     wl = workloads.make("llama70b_layer")
     bank = workloads.AdapterBank(wl, device="cuda")
     pool = build_pool(wl, bank)

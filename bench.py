@@ -67,8 +67,9 @@ WEIGHT_BYTES = {"bf16": 2.0, "fp8_e4m3": 1.0, "int4": 0.5}
 
 def algorithmic_bytes(wl: workloads.Workload, proj: int, weights: str = "bf16"):
     """Minimum bytes of one shrink and one expand: each distinct adapter's A and B
-    once (codes plus one fp32 scale per rank row in a quantised pool), x read once,
-    v written and read in fp32, y read and written."""
+    once (codes plus one fp32 scale per rank row in a quantised pool), x read once
+    (a projection that reads another's x (wl.x_source) adds none), v written and read
+    in fp32, y read and written."""
     wb = WEIGHT_BYTES[weights]
     sb = 0 if weights == "bf16" else 4
     _, d_in, d_out = wl.projections[proj]
@@ -78,7 +79,8 @@ def algorithmic_bytes(wl: workloads.Workload, proj: int, weights: str = "bf16"):
     sum_r_adapters = sum(r_of.values())
     rows = [t for t in range(wl.T) if wl.adapter_ids[t] >= 0 and r_of[int(wl.adapter_ids[t])] > 0]
     sum_r_tokens = sum(r_of[int(wl.adapter_ids[t])] for t in rows)
-    shrink = int(wb * sum_r_adapters * d_in) + sb * sum_r_adapters + 2 * len(rows) * d_in + 4 * sum_r_tokens
+    x_bytes = 2 * len(rows) * d_in if wl.x_of(proj) == proj else 0
+    shrink = int(wb * sum_r_adapters * d_in) + sb * sum_r_adapters + x_bytes + 4 * sum_r_tokens
     expand = int(wb * sum_r_adapters * d_out) + sb * sum_r_adapters + 4 * sum_r_tokens + 4 * len(rows) * d_out
     flops = 2 * sum_r_tokens * (d_in + d_out)
     return shrink, expand, flops, 4 * sum_r_tokens
@@ -202,6 +204,9 @@ def setup(wl_name: str, rank: int, device: int, pool_override: int = 0, weights:
         A, B = zip(*[bank.get(a, p) for p in range(len(projs))])
         pool.load(a, int(r), list(A), list(B))
     acts = [workloads.activations(wl, p, device=f"cuda:{device}") for p in range(len(projs))]
+    # projections that read another's input get that very tensor (the grouped call then
+    # stacks them in one shrink pass over it)
+    acts = [(acts[wl.x_of(p)][0], acts[p][1]) for p in range(len(projs))]
     del bank
     torch.cuda.empty_cache()
     return sg, wl, pool, acts
@@ -348,11 +353,13 @@ def e2e_ours(sg, wl, pool, acts, args, device, stream, world):
                 vs[:] = [plan.new_v() for _ in range(n_proj)]
         if grouped:
             for p in range(n_proj):
-                dev_x[p].copy_(host_x[p], non_blocking=True)
+                if wl.x_of(p) == p:                  # a shared input crosses once
+                    dev_x[p].copy_(host_x[p], non_blocking=True)
+                    b_in += host_x[p].numel() * 2
                 dev_y[p].copy_(host_y[p], non_blocking=True)
-                b_in += host_x[p].numel() * 2 + host_y[p].numel() * 2
-            sg.lora_delta_grouped([(dev_x[p], dev_y[p], p, vs[p]) for p in range(n_proj)], plan, pool, wl.scale,
-                                  stream)
+                b_in += host_y[p].numel() * 2
+            sg.lora_delta_grouped([(dev_x[wl.x_of(p)], dev_y[p], p, vs[p]) for p in range(n_proj)], plan, pool,
+                                  wl.scale, stream)
             for p in range(n_proj):
                 out_y[p].copy_(dev_y[p], non_blocking=True)
                 b_out += out_y[p].numel() * 2
@@ -460,10 +467,10 @@ def run_reference(args, rank, world, device):
 
 
 # adapted tokens of the oracle's bounded sample, by workload (0: the whole batch)
-ORACLE_SAMPLE_TOKENS = {"llama70b_layer": 64}
+ORACLE_SAMPLE_TOKENS = {"llama70b_layer": 64, "llama70b_layer_shared_x": 64}
 # workloads measured besides the headline one, each in the same process
 PER_WORKLOAD = ("tiny", "decode_q_proj", "decode_q_proj_12", "mixed_rank_mlp_up", "prefill_long",
-                "llama70b_layer")
+                "llama70b_layer_shared_x", "llama70b_layer")
 
 
 def sample_text(wl, n_tok: int) -> str:

@@ -127,15 +127,20 @@ struct SimtWork {
     int64_t sum_ng = 0;
     int32_t max_ng = 0;
 };
-// One projection of a SIMT launch.  A launch takes up to kMaxGroup of them over
-// the same plan (launch arguments `inl` only with one job).
+constexpr int kMaxShare = 4;           // projections that share one x in a SIMT shrink pass
+
+// One x of a SIMT shrink launch and the projections computed from it: nsub >= 1
+// projections whose A rows are stacked in the same CTAs (their shared x is read
+// once per CTA).  A launch takes up to kMaxGroup of them over the same plan
+// (launch arguments `inl` only with one job of one projection).
 struct ShrinkJob {
     const uint16_t* x;
     int64_t ldx;
     int32_t d_in;
-    int32_t proj;
-    float* v;
-    int64_t ldv;
+    int32_t nsub;
+    int32_t proj[kMaxShare];
+    float* v[kMaxShare];
+    int64_t ldv[kMaxShare];
 };
 struct ExpandJob {
     const float* v;

@@ -217,7 +217,7 @@ sgmv_status sgmv::shrink_impl(const void* x, int64_t ldx, int32_t T, int32_t d_i
     const uint16_t* xb = static_cast<const uint16_t*>(x);
     InlineTable<kInlineItems> inl;
     const bool use_inl = inline_items(plan, proj, &inl);
-    const ShrinkJob job{xb, ldx, d_in, proj, v, ldv};
+    const ShrinkJob job{xb, ldx, d_in, 1, {proj}, {v}, {ldv}};
     SGMV_CUDA_TRY(launch_shrink_simt(&job, 1, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank,
                                      simt_work(plan), pv, use_inl ? &inl : nullptr, stream));
     SGMV_CUDA_TRY(launch_shrink_tc(xb, ldx, d_in, bv, plan->num_tc_tiles, plan->max_rank, pv, v, ldv, stream));
@@ -279,19 +279,32 @@ sgmv_status sgmv::delta_impl(const sgmv_delta_entry* entries, int32_t n, int32_t
         return SGMV_OK;
     }
     const SimtWork work = simt_work(plan);
+    // entries that read the same x (same pointer, row stride and d_in) share one SIMT
+    // shrink pass: their A rows are stacked in the same CTAs and x is read once per CTA
     ShrinkJob sj[kMaxGroup];
     ExpandJob ej[kMaxGroup];
+    int n_sj = 0;
     for (int32_t i = 0; i < n; ++i) {
         const sgmv_delta_entry& e = entries[i];
-        sj[i] = ShrinkJob{static_cast<const uint16_t*>(e.x), e.ldx, e.d_in, e.proj, e.v, e.ldv};
         ej[i] = ExpandJob{e.v, e.ldv, e.d_out, e.proj, e.y, e.ldy};
+        int g = 0;
+        while (g < n_sj && !(sj[g].x == e.x && sj[g].ldx == e.ldx && sj[g].d_in == e.d_in && sj[g].nsub < kMaxShare))
+            ++g;
+        if (g == n_sj) sj[n_sj++] = ShrinkJob{static_cast<const uint16_t*>(e.x), e.ldx, e.d_in, 0, {}, {}, {}};
+        ShrinkJob& j = sj[g];
+        j.proj[j.nsub] = e.proj;
+        j.v[j.nsub] = e.v;
+        j.ldv[j.nsub] = e.ldv;
+        ++j.nsub;
     }
-    SGMV_CUDA_TRY(launch_shrink_simt(sj, n, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, work, pv,
+    if (use_inl && sj[0].nsub > 1) return fail(SGMV_ERR_INVALID, "lora_delta: internal: shared x with inline items");
+    SGMV_CUDA_TRY(launch_shrink_simt(sj, n_sj, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, work, pv,
                                      use_inl ? &inl : nullptr, stream));
     for (int32_t i = 0; i < n; ++i) {
-        bv.proj = entries[i].proj;
-        SGMV_CUDA_TRY(launch_shrink_tc(sj[i].x, sj[i].ldx, sj[i].d_in, bv, plan->num_tc_tiles, plan->max_rank, pv,
-                                       sj[i].v, sj[i].ldv, stream));
+        const sgmv_delta_entry& e = entries[i];
+        bv.proj = e.proj;
+        SGMV_CUDA_TRY(launch_shrink_tc(static_cast<const uint16_t*>(e.x), e.ldx, e.d_in, bv, plan->num_tc_tiles,
+                                       plan->max_rank, pv, e.v, e.ldv, stream));
     }
     // the expand's predecessors are this call's shrinks, which do not write y: y may be read early
     SGMV_CUDA_TRY(launch_expand_simt(ej, n, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, work, pv,

@@ -63,17 +63,21 @@ constexpr int kStageElems = kRowGroup * kPass;
 template <int WF>
 __host__ __device__ constexpr int stage_bytes() { return kStageElems / 8 * bytes_per_8<WF>(); }
 
-// One projection of a launch.  A launch covers up to kMaxGroup projections over
-// the same batch plan (sgmv_lora_delta_grouped); every projection gets the same
-// number of CTAs per item in the shrink, its own count in the expand.
+// One x of a shrink launch and the nsub projections computed from it.  A launch
+// covers up to kMaxGroup entries over the same batch plan (sgmv_lora_delta_grouped);
+// every entry gets the same number of CTAs per item.  The A rows of an entry's
+// projections are stacked in its CTAs: row group g of a CTA is row group g % NG of
+// projection g / NG (NG = row groups of one projection), so the shared x slices are
+// staged by one CTA for all of them.
 struct ShrinkEntry {
     const uint16_t* x;
     int64_t ldx;
-    float* v;
-    int64_t ldv;
+    float* v[kMaxShare];
+    int64_t ldv[kMaxShare];
     int32_t d_in;
     int32_t kc;          // columns of d_in per CTA (multiple of the page size)
-    int32_t proj;
+    int32_t proj[kMaxShare];
+    int32_t nsub;        // projections stacked over this x (1 .. kMaxShare)
     int32_t pad;
 };
 
@@ -88,6 +92,8 @@ struct ShrinkArgs {
     int32_t stages;
     int32_t max_rank;
     int32_t ring_offset; // byte offset of the stage ring in shared memory
+    int32_t nsub_max;    // largest nsub of the launch (sizes the partial tiles and page ids)
+    int32_t pad;
 };
 
 struct ExpandEntry {
@@ -247,8 +253,9 @@ __device__ __forceinline__ float block_reduce(float (&vals)[N], float* red) {
 // the newest kStages - 1 groups always means "this stage has landed".
 struct StageGeom {  // rows and columns of the CTA's stages
     int NG, npass, span, col_base, rank, pages_per_row;
+    int NGs;             // row groups of one stacked projection (NG = nsub * NGs; the expand: NG)
     int64_t pt;
-    const int32_t* pid;  // page ids of the CTA's span, [rank row][chunk], in shared memory
+    const int32_t* pid;  // page ids of the CTA's span, [row group][8 rank rows][chunk], in shared memory
     int span_pages;
 };
 
@@ -289,7 +296,8 @@ __device__ __forceinline__ void pipe_issue(const PoolView& pool, Pipe<kStages, W
                     cp_async16(xd + j * kPass, xs.rows[j] ? xs.rows[j] + c + kVec * threadIdx.x : xs.any,
                                xs.rows[j] != nullptr);
         }
-        const int rows = min(kRowGroup, sg.rank - kRowGroup * g);
+        const int gl = g - (g / sg.NGs) * sg.NGs;  // row group within its projection
+        const int rows = min(kRowGroup, sg.rank - kRowGroup * gl);
         uint8_t* dst0 = pp.data + (size_t)pp.islot * stage_bytes<WF>();
         const int32_t* pidg = sg.pid + kRowGroup * g * sg.span_pages;
         // a page is (1 << P_log2) values, (1 << page_shift) bytes; column c of it at byte c * VB / 8
@@ -362,21 +370,26 @@ __device__ __forceinline__ void pipe_release(const PoolView& pool, Pipe<kStages,
 }
 
 // All threads: fetch the page ids of every rank row over the CTA's column span
-// into shared memory in one round of independent loads.  Out-of-range ids are
-// flagged and replaced by page 0 (in bounds; the result is flagged).
-__device__ void load_page_ids(const PoolView& pool, StageGeom& sg, int32_t* pid, unsigned int* err) {
+// into shared memory in one round of independent loads; with nsub stacked
+// projections (first page-table entries pt_sub[p]), projection p's rows start at
+// row p * 8 * NGs.  Out-of-range ids are flagged and replaced by page 0 (in
+// bounds; the result is flagged).
+__device__ void load_page_ids(const PoolView& pool, StageGeom& sg, int32_t* pid, unsigned int* err,
+                              const int64_t* pt_sub = nullptr, int nsub = 1) {
     const int P_log2 = pool.page_log2;
     sg.span_pages = sg.span > 0 ? (sg.span + (1 << P_log2) - 1) >> P_log2 : 0;
-    const int n = sg.rank * sg.span_pages;
-    for (int i = threadIdx.x; i < n; i += kThreads) {
-        const int k = i / sg.span_pages, pc = i - k * sg.span_pages;
-        const int64_t e = sg.pt + (int64_t)k * sg.pages_per_row + (sg.col_base >> P_log2) + pc;
+    const int per = sg.rank * sg.span_pages;  // ids of one projection
+    for (int i = threadIdx.x; i < nsub * per; i += kThreads) {
+        const int p = i / per, ip = i - p * per;
+        const int k = ip / sg.span_pages, pc = ip - k * sg.span_pages;
+        const int64_t base = pt_sub ? pt_sub[p] : sg.pt;
+        const int64_t e = base + (int64_t)k * sg.pages_per_row + (sg.col_base >> P_log2) + pc;
         int32_t page = (e >= 0 && e < pool.pt_capacity) ? pool.page_table[e] : -1;
         if (page < 0 || page >= pool.num_pages) {
             atomicOr(err, kErrPage);
             page = 0;
         }
-        pid[i] = page;
+        pid[(p * kRowGroup * sg.NGs + k) * sg.span_pages + pc] = page;
     }
     sg.pid = pid;
 }
@@ -398,10 +411,11 @@ __device__ __forceinline__ void load_row_scales(const PoolView& pool, int64_t pt
 // ------------------------------------------------------------------ shrink
 template <int G, int kStages, int WF>
 __device__ void shrink_item(const PoolView& pool, const ItemInfo& m, Pipe<kStages, WF>& pp, const StageGeom& sg,
-                            const XStage& xs, float* part, float* red) {
+                            const XStage& xs, float* part, float* red, int nsub) {
     constexpr int VB = bytes_per_8<WF>();
     const int tid = threadIdx.x, col = kVec * tid;
     for (int g = 0; g < sg.NG; ++g) {
+        const int ps = g / sg.NGs, gl = g - ps * sg.NGs;  // stacked projection, its row group
         float p[kRowGroup * G];
 #pragma unroll
         for (int i = 0; i < kRowGroup * G; ++i) p[i] = 0.f;
@@ -436,9 +450,9 @@ __device__ void shrink_item(const PoolView& pool, const ItemInfo& m, Pipe<kStage
             pipe_release(pool, pp, sg, false, xs);
         }
         const float sum = block_reduce<kRowGroup * G>(p, red);
-        if (tid < kRowGroup * G) {
+        if (tid < kRowGroup * G) {  // partial tile [token j][projection ps][rank row]
             const int kk = tid / G, j = tid - (tid / G) * G;
-            if (kRowGroup * g + kk < m.r && j < m.n) part[j * m.r + kRowGroup * g + kk] = sum;
+            if (kRowGroup * gl + kk < m.r && j < m.n) part[(j * nsub + ps) * m.r + kRowGroup * gl + kk] = sum;
         }
     }
 }
@@ -457,17 +471,28 @@ __global__ void __launch_bounds__(kThreads, 3)
     const ShrinkEntry& en = a.ent[ei];
     const int item_idx = ((int)blockIdx.x - ei * per_entry) / C;
     const uint32_t q = cluster_ctarank();
-    const int slot = kSimtMaxItemRows * a.max_rank;  // floats of one partial tile
+    const int nsub = NI > 1 ? 1 : en.nsub;                 // projections stacked over this x
+    const int slot = kSimtMaxItemRows * a.max_rank * a.nsub_max;  // floats of one partial tile
     float* part = reinterpret_cast<float*>(smem);     // [C slots][slot]; slot 0 is this CTA's own
     float* red = part + C * slot;                      // [4 warps][64]
-    float* rsc = red + 4 * 64;                         // [kMaxRank] row scales (quantised pools only)
-    int32_t* pid = reinterpret_cast<int32_t*>(rsc + (WF == kFmtBf16 ? 0 : kMaxRank));
+    float* rsc = red + 4 * 64;                         // [nsub][kMaxRank] row scales (quantised pools only)
+    int32_t* pid = reinterpret_cast<int32_t*>(rsc + (WF == kFmtBf16 ? 0 : a.nsub_max * kMaxRank));
+    __shared__ int64_t pt_sub[kMaxShare];              // first page-table entry of A, per stacked projection
 
+    // the stacked projections' A bases come from their own records of this item (loaded
+    // alongside the item's first record; every projection of an item has its rows and rank)
+    if (NI == 1 && (int)threadIdx.x < nsub) {
+        const int4 t = reinterpret_cast<const int4*>(
+            a.b.simt_items + ((int64_t)item_idx * a.b.n_proj + en.proj[threadIdx.x]))[1];
+        pt_sub[threadIdx.x] = (int64_t)(((uint64_t)(uint32_t)t.y << 32) | (uint32_t)t.x);
+    }
     const ItemInfo m = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 0)
-                              : load_item(a.b, en.proj, item_idx, MAXG, a.max_rank, 0);
+                              : load_item(a.b, en.proj[0], item_idx, MAXG, a.max_rank, 0);
+    if (NI > 1 && threadIdx.x == 0) pt_sub[0] = m.pt;
     if (!m.ok && threadIdx.x == 0) atomicOr(&g_err_simt, kErrRows);
     StageGeom sg;
-    sg.NG = (m.r + kRowGroup - 1) / kRowGroup;
+    sg.NGs = (m.r + kRowGroup - 1) / kRowGroup;
+    sg.NG = nsub * sg.NGs;
     sg.span = en.kc;
     sg.npass = (en.kc + kPass - 1) / kPass;
     sg.col_base = (int)q * en.kc;
@@ -485,15 +510,19 @@ __global__ void __launch_bounds__(kThreads, 3)
 #pragma unroll
     for (int j = 0; j < kSimtMaxItemRows; ++j)
         xs.rows[j] = (j < MAXG && m.tok[j] >= 0) ? en.x + (int64_t)m.tok[j] * en.ldx + (int64_t)q * en.kc : nullptr;
-    if (m.ok) load_page_ids(a.pool, sg, pid, &g_err_simt);
-    if (WF != kFmtBf16 && m.ok && q == 0) load_row_scales(a.pool, m.pt, sg.pages_per_row, m.r, rsc, &g_err_simt);
+    __syncthreads();  // pt_sub
+    if (m.ok) load_page_ids(a.pool, sg, pid, &g_err_simt, pt_sub, nsub);
+    if (WF != kFmtBf16 && m.ok && q == 0)
+        for (int ps = 0; ps < nsub; ++ps)
+            load_row_scales(a.pool, pt_sub[ps], sg.pages_per_row, m.r, rsc + ps * kMaxRank, &g_err_simt);
     __syncthreads();
 #pragma unroll 1
     for (int i = 0; i < kShrinkStages; ++i) pipe_issue(a.pool, pp, sg, false, xs);
     if (m.ok) {  // MAXG bounds the token group, and with it the registers of the launch
-        if (MAXG == 1 || m.n == 1) shrink_item<1, kShrinkStages>(a.pool, m, pp, sg, xs, part, red);
-        else if (MAXG == 2 || m.n == 2) shrink_item<(MAXG < 2 ? MAXG : 2), kShrinkStages>(a.pool, m, pp, sg, xs, part, red);
-        else shrink_item<MAXG, kShrinkStages>(a.pool, m, pp, sg, xs, part, red);
+        if (MAXG == 1 || m.n == 1) shrink_item<1, kShrinkStages>(a.pool, m, pp, sg, xs, part, red, nsub);
+        else if (MAXG == 2 || m.n == 2)
+            shrink_item<(MAXG < 2 ? MAXG : 2), kShrinkStages>(a.pool, m, pp, sg, xs, part, red, nsub);
+        else shrink_item<MAXG, kShrinkStages>(a.pool, m, pp, sg, xs, part, red, nsub);
     }
     cp_async_wait<0>();
 
@@ -502,7 +531,8 @@ __global__ void __launch_bounds__(kThreads, 3)
     // barrier without waiting (it may then exit: nobody reads its memory); rank 0
     // arrives, waits for all, sums slots 0..C-1 and writes v.  Slot 0 is rank 0's
     // own tile, so the order of the sum is fixed.
-    const int E = m.n * m.r;
+    const int RS = nsub * m.r;  // values of one token row of the tile: [projection][rank row]
+    const int E = m.n * RS;
     __syncthreads();  // part[] complete in this CTA
     if (C > 1) {
         cluster_wait_acquire();
@@ -521,9 +551,10 @@ __global__ void __launch_bounds__(kThreads, 3)
         for (int e = threadIdx.x; e < E; e += kThreads) {
             float s = 0.f;
             for (int qq = 0; qq < C; ++qq) s += part[(size_t)qq * slot + e];
-            const int jrow = e / m.r, k = e - jrow * m.r;
+            const int jrow = e / RS, rem = e - jrow * RS;
+            const int ps = rem / m.r, k = rem - ps * m.r;
             // a quantised row's scale leaves the sum: v_k = s_k * sum_c q_kc x_c
-            en.v[(int64_t)(m.i0 + jrow) * en.ldv + k] = WF == kFmtBf16 ? s : s * rsc[k];
+            en.v[ps][(int64_t)(m.i0 + jrow) * en.ldv[ps] + k] = WF == kFmtBf16 ? s : s * rsc[ps * kMaxRank + k];
         }
     }
 }
@@ -664,6 +695,7 @@ __global__ void __launch_bounds__(kThreads, 3)
     const int j0 = part_idx * en.npass * kPass;
     StageGeom sg;
     sg.NG = (m.r + kRowGroup - 1) / kRowGroup;
+    sg.NGs = sg.NG;
     sg.span = min(en.npass * kPass, en.d_out - j0);
     sg.npass = (sg.span + kPass - 1) / kPass;
     sg.col_base = j0;
@@ -800,16 +832,21 @@ cudaError_t shrink_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b,
                          shrink_simt_kernel<4, 1, NE, WF>);
     const void* kp = inl ? reinterpret_cast<const void*>(kern_inl) : reinterpret_cast<const void*>(kern_tab);
     const int mr = std::max(8, max_rank);
-    int max_pages = 0;
-    for (int j = 0; j < n_jobs; ++j) max_pages = std::max(max_pages, jobs[j].d_in >> pool.page_log2);
+    int max_pages = 0, nsub_max = 1;
+    for (int j = 0; j < n_jobs; ++j) {
+        max_pages = std::max(max_pages, jobs[j].d_in >> pool.page_log2);
+        nsub_max = std::max(nsub_max, jobs[j].nsub);
+    }
     const int maxg = max_item_rows <= 1 ? 1 : max_item_rows <= 2 ? 2 : 4;
     const int stages = maxg == 1 ? shrink_stages<1>() : shrink_stages<4>();
     // A rows + x slices
     const size_t ring_bytes = (size_t)stages * ((size_t)stage_bytes<WF>() + (size_t)maxg * kPass * 2);
     auto smem_for = [&](int c) {  // partial tiles, reduction scratch, row scales, page ids, ring
-        const size_t part_bytes = (size_t)c * kSimtMaxItemRows * mr * 4;
-        const size_t pidb = (size_t)mr * ((max_pages + c - 1) / c) * 4;
-        const size_t rsc_bytes = WF == kFmtBf16 ? 0 : kMaxRank * 4;
+        const size_t part_bytes = (size_t)c * kSimtMaxItemRows * mr * nsub_max * 4;
+        // page ids: each stacked projection's rows start on a row group (multiple of 8 rows)
+        const size_t pidb = (size_t)nsub_max * ((mr + kRowGroup - 1) / kRowGroup * kRowGroup) *
+                            ((max_pages + c - 1) / c) * 4;
+        const size_t rsc_bytes = WF == kFmtBf16 ? 0 : (size_t)nsub_max * kMaxRank * 4;
         return (((part_bytes + 1024 + rsc_bytes + pidb + 127) & ~(size_t)127)) + ring_bytes;
     };
     // Cluster size C (chunks of >= 1024 columns, C <= 8, dividing every entry's page
@@ -824,7 +861,7 @@ cudaError_t shrink_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b,
             const int d = jobs[j].d_in;
             if (((d >> pool.page_log2) % c) || (c > 1 && d / c < kPass)) valid = false;
             cpi[j] = c;
-            np[j] = (d / c + kPass - 1) / kPass;
+            np[j] = jobs[j].nsub * ((d / c + kPass - 1) / kPass);  // a CTA streams every stacked projection
             wp[j] = (double)np[j] * c;
         }
         if (!valid) continue;
@@ -839,7 +876,18 @@ cudaError_t shrink_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b,
     std::memset(&a, 0, sizeof(a));
     for (int i = 0; i < n_jobs; ++i) {
         const ShrinkJob& j = jobs[order[i]];
-        a.ent[i] = ShrinkEntry{j.x, j.ldx, j.v, j.ldv, j.d_in, j.d_in / C, j.proj, 0};
+        ShrinkEntry& en = a.ent[i];
+        en.x = j.x;
+        en.ldx = j.ldx;
+        en.d_in = j.d_in;
+        en.kc = j.d_in / C;
+        en.nsub = j.nsub;
+        for (int k = 0; k < kMaxShare; ++k) {
+            const int src = k < j.nsub ? k : 0;  // unused slots repeat the first projection
+            en.proj[k] = j.proj[src];
+            en.v[k] = j.v[src];
+            en.ldv[k] = j.ldv[src];
+        }
     }
     a.n_entries = n_jobs;
     a.items = num_items;
@@ -847,6 +895,7 @@ cudaError_t shrink_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b,
     a.pool = pool;
     a.cluster = C;
     a.max_rank = mr;
+    a.nsub_max = nsub_max;
     a.stages = stages;
     const size_t smem = smem_for(C);
     a.ring_offset = (int)(smem - ring_bytes);
@@ -962,8 +1011,10 @@ cudaError_t launch_shrink_simt(const ShrinkJob* jobs, int n_jobs, const BatchVie
                                int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
                                const InlineTable<kInlineItems>* inl, cudaStream_t stream) {
     if (num_items <= 0 || n_jobs <= 0) return cudaSuccess;
-    if (n_jobs > kMaxGroup || (inl && n_jobs > 1)) return cudaErrorInvalidValue;
-    // one projection: a one-entry table (small launch arguments, no per-CTA lookup)
+    if (n_jobs > kMaxGroup || (inl && (n_jobs > 1 || jobs[0].nsub != 1))) return cudaErrorInvalidValue;
+    for (int j = 0; j < n_jobs; ++j)
+        if (jobs[j].nsub < 1 || jobs[j].nsub > kMaxShare) return cudaErrorInvalidValue;
+    // one x: a one-entry table (small launch arguments, no per-CTA lookup)
     auto go = [&](auto wf) {
         constexpr int WF = decltype(wf)::value;
         if (n_jobs == 1)

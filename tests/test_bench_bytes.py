@@ -47,3 +47,13 @@ def test_quantised_weight_bytes():
     scales = 2 * 4 * 8 * 64                # one fp32 scale per rank row of A and of B^T
     assert _total(wl, "fp8_e4m3") == rest + w16 // 2 + scales
     assert _total(wl, "int4") == rest + w16 // 4 + scales
+
+
+def test_shared_x_layer_counts_each_input_once():
+    """The layer with a real layer's inputs (q, k, v read one x; gate, up one x): the
+    same bytes as the layer with seven inputs, less the x reads of k, v and up."""
+    shared, own = workloads.make("llama70b_layer_shared_x"), workloads.make("llama70b_layer")
+    assert shared.adapter_ids.tolist() == own.adapter_ids.tolist()
+    T = 256
+    assert [shared.x_of(p) for p in range(7)] == [0, 0, 0, 3, 4, 4, 6]
+    assert _total(own) - _total(shared) == 3 * 2 * T * 8192

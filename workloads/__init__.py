@@ -39,7 +39,11 @@ LLAMA70B_PROJECTIONS: Tuple[Tuple[str, int, int], ...] = (
 )
 
 WORKLOAD_NAMES = ("tiny", "decode_q_proj", "decode_q_proj_12", "mixed_rank_mlp_up", "prefill_long",
-                  "llama70b_layer")
+                  "llama70b_layer", "llama70b_layer_shared_x")
+
+# projection whose input x each Llama-3-70B projection reads in a real layer: q, k and v the
+# attention input, o its own (the attention output), gate and up the MLP input, down its own
+LLAMA70B_X_SOURCE = (0, 0, 0, 3, 4, 4, 6)
 
 
 @dataclasses.dataclass
@@ -55,6 +59,10 @@ class Workload:
     adapter_ids: np.ndarray                  # int32[T] adapter per token, -1 = no adapter
     scale: float = 1.0
     note: str = ""
+    x_source: Optional[List[int]] = None     # projection whose x each projection reads (None: its own)
+
+    def x_of(self, proj: int) -> int:
+        return proj if self.x_source is None else int(self.x_source[proj])
 
     def rank_of(self, adapter_id: int) -> int:
         return int(self.pool_ranks[self._index()[int(adapter_id)]])
@@ -90,7 +98,11 @@ def make(name: str, seed: int = 0, **overrides) -> Workload:
     prefill_long      8 requests x 512 tokens, 8 adapters of rank 64, 8192->8192,
                       one contiguous segment per request.
     llama70b_layer    7 projections of a Llama-3-70B layer, T=256 decode tokens each on a
-                      distinct adapter drawn from a pool of 2000, rank 16.
+                      distinct adapter drawn from a pool of 2000, rank 16; every projection
+                      has its own input x.
+    llama70b_layer_shared_x  the same batch with the inputs of a real layer: q, k and v read
+                      one x (the attention input), gate and up one x (the MLP input), o and
+                      down their own -- 4 distinct x for 7 projections.
     """
     rng = np.random.default_rng(seed)
     if name == "tiny":
@@ -132,14 +144,15 @@ def make(name: str, seed: int = 0, **overrides) -> Workload:
         pool_ranks = np.full(n_req, overrides.get("rank", 64), dtype=np.int32)
         ids = np.repeat(pool_ids, L).astype(np.int32)
         wl = Workload(name, seed, T, [("proj", d, d)], pool_ids, pool_ranks, ids)
-    elif name == "llama70b_layer":
+    elif name in ("llama70b_layer", "llama70b_layer_shared_x"):
         T = overrides.get("T", 256)
         n_pool = overrides.get("pool", 2000)
         projs = overrides.get("projections", list(LLAMA70B_PROJECTIONS))
         pool_ids = np.arange(n_pool, dtype=np.int32)
         pool_ranks = np.full(n_pool, overrides.get("rank", 16), dtype=np.int32)
         ids = rng.choice(n_pool, size=T, replace=False).astype(np.int32)
-        wl = Workload(name, seed, T, [tuple(p) for p in projs], pool_ids, pool_ranks, ids)
+        wl = Workload(name, seed, T, [tuple(p) for p in projs], pool_ids, pool_ranks, ids,
+                      x_source=list(LLAMA70B_X_SOURCE) if name == "llama70b_layer_shared_x" else None)
     else:
         raise KeyError(f"unknown workload {name!r}; known: {WORKLOAD_NAMES}")
     return wl
@@ -166,9 +179,13 @@ def _randn_bf16(shape, std: float, g: torch.Generator, device) -> torch.Tensor:
 
 
 def activations(wl: Workload, proj: int, device="cpu") -> Tuple[torch.Tensor, torch.Tensor]:
-    """x bf16 [T][d_in] and y bf16 [T][d_out] (y stands for the base output W x)."""
+    """x bf16 [T][d_in] and y bf16 [T][d_out] (y stands for the base output W x).  A
+    projection that shares its input (wl.x_source) gets the same x values as the
+    projection it reads from."""
     _, d_in, d_out = wl.projections[proj]
-    x = _randn_bf16((wl.T, d_in), 1.0 / math.sqrt(d_in), _gen(device, wl.seed, proj, 1), device)
+    src = wl.x_of(proj)
+    assert wl.projections[src][1] == d_in, "projections sharing x need the same d_in"
+    x = _randn_bf16((wl.T, d_in), 1.0 / math.sqrt(d_in), _gen(device, wl.seed, src, 1), device)
     y = _randn_bf16((wl.T, d_out), 1.0, _gen(device, wl.seed, proj, 2), device)
     return x, y
 

@@ -15,9 +15,10 @@ prefill_long) and reports each under `per_workload` with its own step time, roof
 and clocks (--no-per-workload skips them).  The device time of a step (CUDA events on the
 launching stream, from the table copy to the last expand) is what `value`
 measures; L2 is flushed (a 512 MiB write) between steps, outside the timed
-windows.  --weights runs the same batch on a pool of FP8 E4M3 or INT4 codes.  `e2e` repeats the step through the same public API with
-host buffers: the step's x and y rows go host->device from pinned memory and y
-comes back device->host, all inside the timed window, with the host builder.
+windows.  --weights runs the same batch on a pool of FP8 E4M3 or INT4 codes.  `e2e` repeats
+the step through the library's host-buffer entry (sgmv_lora_delta_host): the host
+builder, the copies of every distinct x and every y from pinned memory, the delta and
+the copy of y back, all enqueued by the library in one call inside the timed window.
 
 With N > 1 (torchrun) every rank runs its own batch of the same shape (weak
 scaling, no collective on the data path: the tokens of a batch are
@@ -326,50 +327,29 @@ def run_ours(args, rank, world, device, with_e2e=True):
 
 
 def e2e_ours(sg, wl, pool, acts, args, device, stream, world):
+    """The step through the library's host-buffer entry (sgmv_lora_delta_host): the segment
+    builder, the copies of every distinct x and every y from pinned host memory, the delta
+    and the copy of y back, enqueued by the library in one call (one call per projection
+    with --per-projection).  Timed from an event before the call to an event after the
+    last copy, with the stream idle before the call."""
     n_proj = len(wl.projections)
-    host_x = [x.cpu().pin_memory() for x, _ in acts]
-    host_y = [y.cpu().pin_memory() for _, y in acts]
-    dev_x = [torch.empty_like(x) for x, _ in acts]
-    dev_y = [torch.empty_like(y) for _, y in acts]
-    out_y = [torch.empty_like(h).pin_memory() for h in host_y]
-    plan = sg.BatchPlan(pool, capacity_tokens=wl.T)
-    v = None
+    host_x = {s: acts[s][0].cpu().pin_memory() for s in sorted(set(wl.x_of(p) for p in range(n_proj)))}
+    host_y = [y.cpu().pin_memory() for _, y in acts]   # updated in place every step
+    step = sg.HostStep(pool, capacity_tokens=wl.T)
     grouped = getattr(args, "grouped", False) and n_proj > 1
-    vs = [None] * n_proj
+    entries = [(host_x[wl.x_of(p)], host_y[p], p) for p in range(n_proj)]
     h2d = d2h = 0
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=f"cuda:{device}")
 
-    def one(timed):
-        nonlocal v, h2d, d2h
-        b_in = b_out = 0
+    def one():
+        nonlocal h2d, d2h
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        plan.build(wl.adapter_ids)
-        if plan.upload(stream) is not None:          # small plans travel as launch arguments
-            b_in += int(plan.plan.table_bytes)
-        if v is None:
-            v = plan.new_v()
-            if grouped:
-                vs[:] = [plan.new_v() for _ in range(n_proj)]
-        if grouped:
-            for p in range(n_proj):
-                if wl.x_of(p) == p:                  # a shared input crosses once
-                    dev_x[p].copy_(host_x[p], non_blocking=True)
-                    b_in += host_x[p].numel() * 2
-                dev_y[p].copy_(host_y[p], non_blocking=True)
-                b_in += host_y[p].numel() * 2
-            sg.lora_delta_grouped([(dev_x[wl.x_of(p)], dev_y[p], p, vs[p]) for p in range(n_proj)], plan, pool,
-                                  wl.scale, stream)
-            for p in range(n_proj):
-                out_y[p].copy_(dev_y[p], non_blocking=True)
-                b_out += out_y[p].numel() * 2
-        for p in range(0 if grouped else n_proj):
-            dev_x[p].copy_(host_x[p], non_blocking=True)
-            dev_y[p].copy_(host_y[p], non_blocking=True)
-            b_in += host_x[p].numel() * 2 + host_y[p].numel() * 2
-            v = sg.lora_delta(dev_x[p], plan, pool, dev_y[p], p, wl.scale, v=v, stream=stream)
-            out_y[p].copy_(dev_y[p], non_blocking=True)
-            b_out += out_y[p].numel() * 2
+        b_in = b_out = 0
+        for group in ([entries] if grouped else [[e] for e in entries]):
+            i, o = step.run(wl.adapter_ids, group, wl.scale, stream)
+            b_in += i
+            b_out += o
         e1.record(stream)
         e1.synchronize()
         h2d, d2h = b_in, b_out
@@ -378,12 +358,12 @@ def e2e_ours(sg, wl, pool, acts, args, device, stream, world):
     for _ in range(max(3, args.warmup)):
         flush.zero_()
         torch.cuda.synchronize(device)
-        one(False)
+        one()
     times = []
     for _ in range(args.steps):
         flush.zero_()
         torch.cuda.synchronize(device)
-        times.append(one(True))
+        times.append(one())
     total = reduce_max(float(sum(times)), f"cuda:{device}")
     return dict(total_ms=total, h2d=h2d, d2h=d2h)
 

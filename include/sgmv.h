@@ -472,6 +472,52 @@ SGMV_API sgmv_status sgmv_lora_delta_grouped(const sgmv_delta_entry* entries, in
                                              float scale, int32_t y_dtype, sgmv_stream_t stream);
 
 /*
+ * The whole step from host buffers: the segment builder, the host-to-device
+ * copies of the step's inputs, the grouped delta and the device-to-host copy
+ * of the results, enqueued on `stream` by the library (no Python or other
+ * caller work between them).  For serving loops whose activations live in
+ * host memory, and for measuring the path end to end.
+ *
+ * adapter_ids   host int32[T] (-1 = no adapter), as for sgmv_build_plan
+ * entries       host array of n_entries (1 .. 8): projection `proj` with its
+ *               d_in / d_out, x_host (bf16 [T][d_in], rows contiguous) and
+ *               y_host ([T][d_out] of y_dtype, rows contiguous, updated in place).
+ *               Entries that name the same x_host (and d_in) share one copy
+ *               of it and one stacked shrink pass (as in sgmv_lora_delta_grouped).
+ * host_table    host memory of host_table_bytes >= sgmv_plan_table_capacity(T,
+ *               pool's n_proj), 16-byte aligned; the plan is built into it and
+ *               *plan_out (may be NULL) receives its header.
+ * workspace     device memory of workspace_bytes >= sgmv_host_workspace_bytes(...),
+ *               256-byte aligned: the device copies of the table, of every
+ *               distinct x and of every y, and the intermediates v.
+ * Host buffers should be pinned (page-locked) for the copies to run
+ * asynchronously.  The call returns once everything is enqueued: y_host holds
+ * the results, and host_table, x_host and y_host may be reused, only after the
+ * stream has completed.  *h2d_bytes / *d2h_bytes (may be NULL) receive the bytes
+ * the copies move.  Errors as for sgmv_build_plan and sgmv_lora_delta_grouped
+ * (nothing is enqueued), SGMV_ERR_CAPACITY for a workspace or table too small.
+ */
+typedef struct {
+    int32_t proj;
+    int32_t d_in;
+    int32_t d_out;
+    int32_t reserved;       /* 0 */
+    const void* x_host;
+    void* y_host;
+} sgmv_host_entry;
+
+/* Device workspace bytes sgmv_lora_delta_host needs for a batch of T tokens
+ * (an upper bound over every batch of T tokens on this pool); -1 on a bad argument. */
+SGMV_API int64_t sgmv_host_workspace_bytes(int32_t T, const sgmv_pool* pool, const sgmv_host_entry* entries,
+                                           int32_t n_entries, int32_t y_dtype);
+
+SGMV_API sgmv_status sgmv_lora_delta_host(const int32_t* adapter_ids, int32_t T, const sgmv_pool* pool,
+                                          const sgmv_host_entry* entries, int32_t n_entries, float scale,
+                                          int32_t y_dtype, void* host_table, int64_t host_table_bytes,
+                                          void* workspace, int64_t workspace_bytes, sgmv_plan* plan_out,
+                                          int64_t* h2d_bytes, int64_t* d2h_bytes, sgmv_stream_t stream);
+
+/*
  * sgmv_lora_delta for callers that cannot give the library device memory.
  * No counterpart on the pages: this is a deployment convenience.
  *

@@ -35,7 +35,8 @@ EXPORTED = ("sgmv_status_string", "sgmv_last_error", "sgmv_pool_create", "sgmv_p
             "sgmv_pool_set_adapter_scale", "sgmv_pool_get_adapter_scale",
             "sgmv_pool_shuffle_free_pages", "sgmv_pool_pages_device", "sgmv_plan_table_capacity",
             "sgmv_build_plan", "sgmv_shrink", "sgmv_expand", "sgmv_lora_delta", "sgmv_lora_delta_grouped",
-            "sgmv_lora_delta_noalloc", "sgmv_check_errors", "sgmv_residency_create", "sgmv_residency_destroy",
+            "sgmv_lora_delta_noalloc", "sgmv_host_workspace_bytes", "sgmv_lora_delta_host",
+            "sgmv_check_errors", "sgmv_residency_create", "sgmv_residency_destroy",
             "sgmv_residency_register", "sgmv_residency_unregister", "sgmv_residency_prepare",
             "sgmv_residency_get_stats")
 
@@ -59,6 +60,11 @@ class DeltaEntry(ctypes.Structure):
     _fields_ = [("proj", ctypes.c_int32), ("d_in", ctypes.c_int32), ("d_out", ctypes.c_int32),
                 ("reserved", ctypes.c_int32), ("x", ctypes.c_void_p), ("ldx", ctypes.c_int64),
                 ("y", ctypes.c_void_p), ("ldy", ctypes.c_int64), ("v", ctypes.c_void_p), ("ldv", ctypes.c_int64)]
+
+
+class HostEntry(ctypes.Structure):
+    _fields_ = [("proj", ctypes.c_int32), ("d_in", ctypes.c_int32), ("d_out", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("x_host", ctypes.c_void_p), ("y_host", ctypes.c_void_p)]
 
 
 class ResidencyStats(ctypes.Structure):
@@ -116,6 +122,9 @@ def load_library() -> ctypes.CDLL:
                                          i32, vp]),
         "sgmv_lora_delta_noalloc": (st, [vp, i64, i32, i32, i32, i32, ctypes.POINTER(Plan), vp, vp, f32, vp, i64,
                                          i32, vp]),
+        "sgmv_host_workspace_bytes": (i64, [i32, vp, ctypes.POINTER(HostEntry), i32, i32]),
+        "sgmv_lora_delta_host": (st, [vp, i32, vp, ctypes.POINTER(HostEntry), i32, f32, i32, vp, i64, vp, i64,
+                                      ctypes.POINTER(Plan), ctypes.POINTER(i64), ctypes.POINTER(i64), vp]),
         "sgmv_check_errors": (st, [vp, ctypes.POINTER(ctypes.c_uint32)]),
         "sgmv_residency_create": (st, [vp, ctypes.POINTER(vp)]),
         "sgmv_residency_destroy": (st, [vp]),
@@ -550,6 +559,62 @@ def lora_delta_noalloc(x: torch.Tensor, plan: BatchPlan, pool: AdapterPool, y: t
         _ptr(x), x.stride(0), plan.T, x.shape[1], y.shape[1], int(proj), ctypes.byref(plan.plan),
         plan.table_ptr(stream), pool.handle, float(scale), _ptr(y), y.stride(0),
         0 if y.dtype == torch.bfloat16 else 1, _stream(stream)))
+
+
+class HostStep:
+    """The whole step from host buffers in one library call (sgmv_lora_delta_host): the
+    segment builder, the copies of x and y to the device, the grouped delta and the copy
+    of y back, all enqueued on the stream by the library.  Holds the pinned host table
+    and the device workspace, grown as needed and reused across steps."""
+
+    def __init__(self, pool: AdapterPool, capacity_tokens: int):
+        self.pool = pool
+        lib = load_library()
+        self.table_bytes = int(lib.sgmv_plan_table_capacity(int(capacity_tokens), len(pool.projections)))
+        self.host_table = torch.empty(self.table_bytes, dtype=torch.uint8, pin_memory=torch.cuda.is_available())
+        self.workspace: Optional[torch.Tensor] = None
+        self.plan = Plan()
+        self.capacity = int(capacity_tokens)
+        self._done: Optional[torch.cuda.Event] = None
+
+    def run(self, adapter_ids, entries, scale: float = 1.0, stream=None) -> Tuple[int, int]:
+        """entries: (x_host, y_host, proj) with contiguous host tensors (pinned for asynchronous
+        copies), all y of one dtype; entries naming the same x_host tensor share its copy and
+        one stacked shrink pass.  y_host holds the result once the stream has completed.
+        Returns the (host-to-device, device-to-host) bytes the step's copies move."""
+        ids = np.ascontiguousarray(np.asarray(adapter_ids, dtype=np.int32).reshape(-1))
+        assert ids.size <= self.capacity and 1 <= len(entries) <= 8
+        if self._done is not None:
+            self._done.synchronize()          # the previous step's copies have read the host table
+        arr = (HostEntry * len(entries))()
+        ydt = None
+        for i, (x, y, proj) in enumerate(entries):
+            assert not x.is_cuda and not y.is_cuda and x.is_contiguous() and y.is_contiguous()
+            assert x.dtype == torch.bfloat16 and y.dtype in (torch.bfloat16, torch.float32)
+            assert ydt is None or ydt == y.dtype
+            ydt = y.dtype
+            arr[i] = HostEntry(int(proj), x.shape[1], y.shape[1], 0, x.data_ptr(), y.data_ptr())
+        y_dtype = 0 if ydt == torch.bfloat16 else 1
+        lib = load_library()
+        need = int(lib.sgmv_host_workspace_bytes(self.capacity, self.pool.handle, arr, len(entries), y_dtype))
+        if need < 0:
+            _check(1)
+        if self.workspace is None or self.workspace.numel() < need:
+            self.workspace = torch.empty(need, dtype=torch.uint8, device=torch.device("cuda", self.pool.device))
+        h2d, d2h = ctypes.c_int64(), ctypes.c_int64()
+        _check(lib.sgmv_lora_delta_host(ids.ctypes.data if ids.size else None, int(ids.size), self.pool.handle, arr,
+                                        len(entries), float(scale), y_dtype, self.host_table.data_ptr(),
+                                        self.table_bytes, self.workspace.data_ptr(), self.workspace.numel(),
+                                        ctypes.byref(self.plan), ctypes.byref(h2d), ctypes.byref(d2h),
+                                        _stream(stream)))
+        if self._done is None:
+            self._done = torch.cuda.Event()
+        s = torch.cuda.current_stream(self.pool.device) if stream is None else stream
+        if isinstance(s, torch.cuda.Stream):
+            self._done.record(s)
+        else:
+            self._done.record(torch.cuda.ExternalStream(int(s)))
+        return int(h2d.value), int(d2h.value)
 
 
 def check_errors(stream=None) -> int:

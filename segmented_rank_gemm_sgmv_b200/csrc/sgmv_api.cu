@@ -108,6 +108,8 @@ SimtWork simt_work(const sgmv_plan* plan) {
     }
     const ItemRec* recs = reinterpret_cast<const ItemRec*>(static_cast<const uint8_t*>(plan->host_table) +
                                                            plan->off_simt_items);
+    w.host_items = recs;
+    w.n_proj = plan->n_proj;
     int32_t mx = 1;
     for (int32_t i = 0; i < n; ++i) {
         const int32_t ng = (std::max(recs[(int64_t)i * plan->n_proj].rank, 1) + 7) / 8;
@@ -331,6 +333,150 @@ extern "C" sgmv_status sgmv_lora_delta_grouped(const sgmv_delta_entry* entries, 
                                                const sgmv_plan* plan, const void* table, const sgmv_pool* pool,
                                                float scale, int32_t y_dtype, sgmv_stream_t stream) {
     return delta_impl(entries, n_entries, T, plan, table, pool, scale, y_dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------------------
+// The step from host buffers: plan, copies in, grouped delta, copy out.
+
+namespace {
+
+int64_t align256(int64_t n) { return (n + 255) & ~int64_t(255); }
+
+// Device workspace layout of sgmv_lora_delta_host: the table, every distinct x,
+// every y, then every v (rows x ldv fp32); `rows` and `ldv` may be upper bounds.
+struct HostLayout {
+    int64_t table = 0, x[kMaxGroup] = {}, y[kMaxGroup] = {}, v[kMaxGroup] = {}, end = 0;
+    int x_of[kMaxGroup] = {};  // entry -> first entry with the same x
+};
+
+bool host_layout(const sgmv_host_entry* e, int32_t n, int32_t T, int64_t table_bytes, int64_t rows, int64_t ldv,
+                 int32_t y_dtype, HostLayout* L) {
+    const int64_t esz = y_dtype == 0 ? 2 : 4;
+    int64_t o = 0;
+    L->table = o;
+    o = align256(o + std::max<int64_t>(table_bytes, 16));
+    for (int32_t i = 0; i < n; ++i) {
+        L->x_of[i] = i;
+        for (int32_t k = 0; k < i; ++k)
+            if (e[k].x_host == e[i].x_host && e[k].d_in == e[i].d_in) {
+                L->x_of[i] = L->x_of[k];
+                break;
+            }
+        if (L->x_of[i] == i) {
+            L->x[i] = o;
+            o = align256(o + (int64_t)T * e[i].d_in * 2);
+        } else {
+            L->x[i] = L->x[L->x_of[i]];
+        }
+    }
+    for (int32_t i = 0; i < n; ++i) {
+        L->y[i] = o;
+        o = align256(o + (int64_t)T * e[i].d_out * esz);
+    }
+    for (int32_t i = 0; i < n; ++i) {
+        L->v[i] = o;
+        o = align256(o + std::max<int64_t>(rows, 1) * ldv * 4);
+    }
+    L->end = o;
+    return true;
+}
+
+sgmv_status check_host_entries(const sgmv_host_entry* e, int32_t n, const sgmv_pool* pool, int32_t y_dtype) {
+    if (!pool) return fail(SGMV_ERR_INVALID, "lora_delta_host: pool is NULL");
+    if (!e || n < 1 || n > kMaxGroup)
+        return fail(SGMV_ERR_INVALID, "lora_delta_host: 1 to " + std::to_string(kMaxGroup) + " entries are required");
+    if (y_dtype != 0 && y_dtype != 1) return fail(SGMV_ERR_INVALID, "lora_delta_host: y_dtype must be 0 or 1");
+    for (int32_t i = 0; i < n; ++i) {
+        if (e[i].proj < 0 || e[i].proj >= pool->n_proj) return fail(SGMV_ERR_INVALID, "lora_delta_host: bad projection");
+        if (e[i].d_in != pool->d_in[e[i].proj] || e[i].d_out != pool->d_out[e[i].proj])
+            return fail(SGMV_ERR_INVALID, "lora_delta_host: d_in / d_out differ from the pool's projection");
+        if (!e[i].x_host || !e[i].y_host) return fail(SGMV_ERR_INVALID, "lora_delta_host: x_host and y_host are required");
+        for (int32_t k = 0; k < i; ++k)
+            if (e[k].y_host == e[i].y_host) return fail(SGMV_ERR_INVALID, "lora_delta_host: two entries name one y_host");
+    }
+    return SGMV_OK;
+}
+
+}  // namespace
+
+extern "C" int64_t sgmv_host_workspace_bytes(int32_t T, const sgmv_pool* pool, const sgmv_host_entry* entries,
+                                             int32_t n_entries, int32_t y_dtype) {
+    if (T < 0 || check_host_entries(entries, n_entries, pool, y_dtype) != SGMV_OK) return -1;
+    HostLayout L;
+    const int64_t ldv = std::max<int64_t>(4, ((int64_t)pool->max_rank + 3) / 4 * 4);
+    host_layout(entries, n_entries, T, sgmv_plan_table_capacity(T, pool->n_proj), T, ldv, y_dtype, &L);
+    return L.end;
+}
+
+extern "C" sgmv_status sgmv_lora_delta_host(const int32_t* adapter_ids, int32_t T, const sgmv_pool* pool,
+                                            const sgmv_host_entry* entries, int32_t n_entries, float scale,
+                                            int32_t y_dtype, void* host_table, int64_t host_table_bytes,
+                                            void* workspace, int64_t workspace_bytes, sgmv_plan* plan_out,
+                                            int64_t* h2d_bytes, int64_t* d2h_bytes, sgmv_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    sgmv_status st = check_host_entries(entries, n_entries, pool, y_dtype);
+    if (st != SGMV_OK) return st;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return fail(SGMV_ERR_INVALID, "lora_delta_host: workspace must be a 256-byte aligned device pointer");
+    sgmv_plan plan;
+    st = sgmv_build_plan(adapter_ids, T, pool, 0, host_table, host_table_bytes, &plan);
+    if (st != SGMV_OK) return st;
+    const int64_t esz = y_dtype == 0 ? 2 : 4;
+    const int64_t ldv = std::max<int64_t>(4, ((int64_t)plan.max_rank + 3) / 4 * 4);
+    HostLayout L;
+    host_layout(entries, n_entries, T, plan.table_bytes, plan.num_rows, ldv, y_dtype, &L);
+    if (L.end > workspace_bytes) return fail(SGMV_ERR_CAPACITY, "lora_delta_host: workspace too small");
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    sgmv_delta_entry de[kMaxGroup];
+    for (int32_t i = 0; i < n_entries; ++i) {
+        const sgmv_host_entry& e = entries[i];
+        de[i] = sgmv_delta_entry{e.proj, e.d_in, e.d_out, 0, ws + L.x[i], e.d_in, ws + L.y[i], e.d_out,
+                                 reinterpret_cast<float*>(ws + L.v[i]), ldv};
+    }
+    const void* table = plan.needs_device_table ? ws + L.table : nullptr;
+    // every argument of the kernels is checked before the first copy is enqueued
+    BatchView bv;
+    PoolView pv;
+    bool nothing = false;
+    for (int32_t i = 0; i < n_entries; ++i) {
+        const sgmv_delta_entry& e = de[i];
+        st = check_shrink(e.x, e.ldx, T, e.d_in, e.proj, &plan, table ? table : ws + L.table, pool, e.v, e.ldv, &bv,
+                          &pv, &nothing);
+        if (st != SGMV_OK) return st;
+        st = check_expand(e.v, e.ldv, T, e.d_out, e.proj, &plan, table ? table : ws + L.table, pool, e.y, e.ldy,
+                          y_dtype, &bv, &pv, &nothing);
+        if (st != SGMV_OK) return st;
+    }
+    int64_t in = 0, out = 0;
+    if (plan.needs_device_table) {
+        SGMV_CUDA_TRY(cudaMemcpyAsync(ws + L.table, host_table, (size_t)plan.table_bytes, cudaMemcpyHostToDevice,
+                                      stream));
+        in += plan.table_bytes;
+    }
+    for (int32_t i = 0; i < n_entries; ++i) {
+        const sgmv_host_entry& e = entries[i];
+        if (L.x_of[i] == i && T > 0) {
+            SGMV_CUDA_TRY(cudaMemcpyAsync(ws + L.x[i], e.x_host, (size_t)T * e.d_in * 2, cudaMemcpyHostToDevice,
+                                          stream));
+            in += (int64_t)T * e.d_in * 2;
+        }
+        if (T > 0) {
+            SGMV_CUDA_TRY(cudaMemcpyAsync(ws + L.y[i], e.y_host, (size_t)T * e.d_out * esz, cudaMemcpyHostToDevice,
+                                          stream));
+            in += (int64_t)T * e.d_out * esz;
+        }
+    }
+    st = delta_impl(de, n_entries, T, &plan, table, pool, scale, y_dtype, stream);
+    if (st != SGMV_OK) return st;
+    for (int32_t i = 0; i < n_entries && T > 0; ++i) {
+        SGMV_CUDA_TRY(cudaMemcpyAsync(entries[i].y_host, ws + L.y[i], (size_t)T * entries[i].d_out * esz,
+                                      cudaMemcpyDeviceToHost, stream));
+        out += (int64_t)T * entries[i].d_out * esz;
+    }
+    if (plan_out) *plan_out = plan;
+    if (h2d_bytes) *h2d_bytes = in;
+    if (d2h_bytes) *d2h_bytes = out;
+    return SGMV_OK;
 }
 
 // ---------------------------------------------------------------------------

@@ -64,3 +64,31 @@ def test_plan_table_capacity_bounds():
     assert lib.sgmv_plan_table_capacity(-1, 1) == -1
     assert lib.sgmv_plan_table_capacity(0, 1) >= 16
     assert lib.sgmv_plan_table_capacity(1000, 7) >= 1000 * 4 * 3 + 1000 * 7 * 16 + 1000 * 32
+
+
+def test_host_step_workspace_and_argument_checks():
+    """sgmv_host_workspace_bytes: the table, each distinct x, each y and each v, every
+    region rounded up to 256 bytes; sgmv_lora_delta_host refuses bad arguments before
+    enqueueing anything."""
+    pool = sg.AdapterPool([(1024, 512), (1024, 1536), (2048, 512)], num_pages=4096, page_elems=512, max_rank=16,
+                          device=-1)
+    pool.load(0, 16)
+    lib = sg.load_library()
+    T = 37
+    r256 = lambda n: (n + 255) // 256 * 256
+    x0, x2 = ctypes.c_void_p(4096), ctypes.c_void_p(8192)          # host addresses are not touched here
+    ents = (sg.HostEntry * 3)(sg.HostEntry(0, 1024, 512, 0, x0, ctypes.c_void_p(1 << 20)),
+                              sg.HostEntry(1, 1024, 1536, 0, x0, ctypes.c_void_p(2 << 20)),
+                              sg.HostEntry(2, 2048, 512, 0, x2, ctypes.c_void_p(3 << 20)))
+    table = lib.sgmv_plan_table_capacity(T, 3)
+    for y_dtype, esz in ((0, 2), (1, 4)):
+        want = (r256(table) + r256(T * 1024 * 2) + r256(T * 2048 * 2) +
+                sum(r256(T * d * esz) for d in (512, 1536, 512)) + 3 * r256(T * 16 * 4))
+        assert lib.sgmv_host_workspace_bytes(T, pool.handle, ents, 3, y_dtype) == want
+    assert lib.sgmv_host_workspace_bytes(T, pool.handle, ents, 0, 0) == -1
+    bad = (sg.HostEntry * 1)(sg.HostEntry(0, 1024, 1536, 0, x0, ctypes.c_void_p(1 << 20)))   # d_out of proj 1
+    assert lib.sgmv_host_workspace_bytes(T, pool.handle, bad, 1, 0) == -1
+    ids = (ctypes.c_int32 * 2)(0, -1)
+    host = ctypes.create_string_buffer(4096)
+    st = lib.sgmv_lora_delta_host(ids, 2, pool.handle, ents, 3, 1.0, 0, host, 4096, None, 0, None, None, None, None)
+    assert st == 1 and b"workspace" in lib.sgmv_last_error()

@@ -815,20 +815,16 @@ __device__ __forceinline__ int64_t cta_unit(const StreamArgs& a, int k) {
     return u < a.total_units ? u : -1;
 }
 
-constexpr int kStreamStages = 3;  // three CTAs an SM, each with three 16 KB stages in flight
-
-template <int MAXG, int WF>
-__global__ void __launch_bounds__(kThreads, 3)
+template <int MAXG, int WF, int S>  // S: stages of the ring (at most one unit's passes)
+__global__ void __launch_bounds__(kThreads, 2)
     shrink_stream_kernel(const __grid_constant__ StreamArgs a) {
     extern __shared__ __align__(128) uint8_t smem_s[];
     pdl_launch_dependents();  // the expand may start staging its B^T pages as slots free up
-    constexpr int S = kStreamStages;
     constexpr int VB = bytes_per_8<WF>();
     const int tid = threadIdx.x, col = kVec * tid;
     float* red = reinterpret_cast<float*>(smem_s);  // [4 warps][64]
     uint8_t* slots = smem_s + 4 * 64 * 4;
-    uint8_t* ring = smem_s + a.ring_offset;          // S stages, then S x-slice slots
-    uint16_t* xring = reinterpret_cast<uint16_t*>(ring + (size_t)S * stage_bytes<WF>());
+    uint8_t* ring = smem_s + a.ring_offset;          // S stages of A rows
     const int P_log2 = a.pool.page_log2, P = 1 << P_log2;
     auto slot = [&](int k) { return reinterpret_cast<StreamSlot*>(slots + (size_t)(k & (kStreamSlots - 1)) * a.slot_bytes); };
 
@@ -841,6 +837,14 @@ __global__ void __launch_bounds__(kThreads, 3)
                                                         ((int64_t)id.item * a.b.n_proj + a.job[id.job].proj[id.p]));
         cp_async16(&slot(k)->rec[tid], src + tid, true);
     };
+    // is unit k's record well formed; its rank rows in its row group (0 if not)
+    auto unit_rows = [&](int k, const UnitId& id) {
+        const int4 h = slot(k)->rec[0];
+        const int n = h.z - h.y, r = h.w;
+        const bool ok = h.x >= 0 && h.x < a.b.num_segments && h.y >= 0 && n > 0 && n <= MAXG &&
+                        h.z <= a.b.num_rows && r > 0 && r <= a.max_rank && 8 * id.g < r;
+        return ok ? min(kRowGroup, r - kRowGroup * id.g) : 0;
+    };
     // the rest of unit k (its record has landed): token rows, row scales, page ids
     auto fetch_meta = [&](int k) {
         const int64_t u = cta_unit(a, k);
@@ -848,14 +852,11 @@ __global__ void __launch_bounds__(kThreads, 3)
         const UnitId id = decode_unit(a, u);
         StreamSlot* sl = slot(k);
         const int4 h = sl->rec[0], t = sl->rec[1];
-        const int n = h.z - h.y, r = h.w;
-        const bool ok = h.x >= 0 && h.x < a.b.num_segments && h.y >= 0 && n > 0 && n <= MAXG &&
-                        h.z <= a.b.num_rows && r > 0 && r <= a.max_rank && 8 * id.g < r;
-        const int rows = ok ? min(kRowGroup, r - kRowGroup * id.g) : 0;
+        const int rows = unit_rows(k, id), n = h.z - h.y;
         const int64_t a_pt = (int64_t)(((uint64_t)(uint32_t)t.y << 32) | (uint32_t)t.x);
         const int ppr = a.job[id.job].d_in >> P_log2;
         if (tid < kSimtMaxItemRows) {
-            if (ok && tid < n) cp_async4(&sl->tok[tid], a.b.token_idx + h.y + tid);
+            if (rows > 0 && tid < n) cp_async4(&sl->tok[tid], a.b.token_idx + h.y + tid);
             else sl->tok[tid] = -1;
         }
         if (WF != kFmtBf16 && tid >= 32 && tid < 32 + kRowGroup) {
@@ -871,13 +872,10 @@ __global__ void __launch_bounds__(kThreads, 3)
             else sl->pid[i] = -1;
         }
     };
-    // rank rows of unit k's row group (0 for a bad record, flagged once)
-    auto unit_rows = [&](int k, const UnitId& id) {
-        const int4 h = slot(k)->rec[0];
-        const int n = h.z - h.y, r = h.w;
-        const bool ok = h.x >= 0 && h.x < a.b.num_segments && h.y >= 0 && n > 0 && n <= MAXG &&
-                        h.z <= a.b.num_rows && r > 0 && r <= a.max_rank && 8 * id.g < r;
-        return ok ? min(kRowGroup, r - kRowGroup * id.g) : 0;
+    // unit k's token rows, checked (-1: none)
+    auto token = [&](int k, int j) {
+        const int tk = slot(k)->tok[j];
+        return (tk >= 0 && tk < a.b.T) ? tk : -1;
     };
 
     // ---- prologue: units 0 and 1 complete before the first stage
@@ -912,16 +910,6 @@ __global__ void __launch_bounds__(kThreads, 3)
             const StreamSlot* sl = slot(ki);
             const StreamJob& jb = a.job[idi.job];
             const int c = si * kPass, W = min(kPass, jb.d_in - c);
-            // x slices of the item's tokens
-            if (col < W) {
-                uint16_t* xd = xring + (size_t)islot * MAXG * kPass + col;
-#pragma unroll
-                for (int j = 0; j < MAXG; ++j) {
-                    const int tk = sl->tok[j];
-                    const bool v = rows_i > 0 && tk >= 0 && tk < a.b.T;
-                    cp_async16(xd + j * kPass, v ? jb.x + (int64_t)tk * jb.ldx + c + col : jb.x, v);
-                }
-            }
             // A rows of the row group: 16-byte copies, consecutive threads on consecutive granules
             const int ppr = jb.d_in >> P_log2;
             uint8_t* dst0 = ring + (size_t)islot * stage_bytes<WF>();
@@ -979,69 +967,132 @@ __global__ void __launch_bounds__(kThreads, 3)
     };
     for (int i = 0; i < S; ++i) issue();
 
-    // ---- consume side
-    int cslot = 0;
-    for (int kc = 0;; ++kc) {
-        const int64_t uc = cta_unit(a, kc);
-        if (uc < 0) break;
-        const UnitId idc = decode_unit(a, uc);
-        const StreamJob& jb = a.job[idc.job];
-        const int rows_c = unit_rows(kc, idc);
-        if (tid == 0) {
-            if (rows_c == 0) atomicOr(&g_err_simt, kErrRows);
-            const StreamSlot* sl = slot(kc);
-            for (int j = 0; j < sl->rec[0].z - sl->rec[0].y && j < MAXG && rows_c > 0; ++j)
-                if (sl->tok[j] < 0 || sl->tok[j] >= a.b.T) atomicOr(&g_err_simt, kErrToken);  // (its x reads as 0)
+    // ---- consume side.  Each thread's x slice of a stage (8 columns of each token) is
+    // read into registers one stage ahead; a unit's x rows are pulled into L2 when the
+    // unit before it starts.
+    int kc = 0, sc = 0, cslot = 0;
+    int64_t uc = cta_unit(a, 0);
+    if (uc < 0) {
+        cp_async_wait<0>();
+        return;
+    }
+    UnitId idc = decode_unit(a, uc);
+    int rows_c = unit_rows(0, idc);
+    // x slice of (unit k, pass s) into xr
+    auto load_x = [&](int k, const UnitId& id, int s, uint4 (&xr)[MAXG]) {
+        const StreamJob& jb = a.job[id.job];
+        const int c = s * kPass;
+#pragma unroll
+        for (int j = 0; j < MAXG; ++j) {
+            const int tk = token(k, j);
+            xr[j] = (tk >= 0 && c + col < jb.d_in)
+                        ? __ldg(reinterpret_cast<const uint4*>(jb.x + (int64_t)tk * jb.ldx + c + col))
+                        : make_uint4(0u, 0u, 0u, 0u);
         }
-        float pacc[kRowGroup * MAXG];
+    };
+    auto prefetch_x = [&](int k) {  // the x rows of unit k into L2
+        const int64_t u = cta_unit(a, k);
+        if (u < 0 || tid >= MAXG) return;
+        const UnitId id = decode_unit(a, u);
+        const int tk = token(k, tid);
+        const StreamJob& jb = a.job[id.job];
+        if (tk >= 0 && tid < slot(k)->rec[0].z - slot(k)->rec[0].y)
+            bulk_prefetch_l2(jb.x + (int64_t)tk * jb.ldx, (uint32_t)jb.d_in * 2);
+    };
+    auto flag_unit = [&](int k, int rows) {
+        if (tid != 0) return;
+        if (rows == 0) atomicOr(&g_err_simt, kErrRows);
+        const StreamSlot* sl = slot(k);
+        for (int j = 0; j < sl->rec[0].z - sl->rec[0].y && j < MAXG && rows > 0; ++j)
+            if (sl->tok[j] < 0 || sl->tok[j] >= a.b.T) atomicOr(&g_err_simt, kErrToken);  // (its x reads as 0)
+    };
+    flag_unit(0, rows_c);
+    float pacc[kRowGroup * MAXG];
 #pragma unroll
-        for (int i = 0; i < kRowGroup * MAXG; ++i) pacc[i] = 0.f;
-        for (int s = 0; s < idc.npass; ++s) {
-            cp_async_wait<S - 1>();
-            __syncthreads();
-            const int c = s * kPass, W = min(kPass, jb.d_in - c);
-            const uint8_t* st = ring + (size_t)cslot * stage_bytes<WF>();
-            const uint16_t* xst = xring + (size_t)cslot * MAXG * kPass + col;
-            if (col < W && rows_c > 0) {
-                float xf[MAXG][8];
+    for (int i = 0; i < kRowGroup * MAXG; ++i) pacc[i] = 0.f;
+    bool done = false;
+    // one stage: x of this stage in xc, x of the next one loaded into xn
+    auto step = [&](uint4 (&xc)[MAXG], uint4 (&xn)[MAXG]) {
+        // the next stage's (unit, pass): its x slice is loaded now, used one stage later
+        int kn = kc, sn = sc + 1;
+        if (sn == idc.npass) {
+            kn = kc + 1;
+            sn = 0;
+        }
+        const int64_t un = cta_unit(a, kn);
+        UnitId idn = idc;
+        if (kn != kc && un >= 0) idn = decode_unit(a, un);
+        if (un >= 0) load_x(kn, idn, sn, xn);
+        cp_async_wait<S - 1>();
+        __syncthreads();
+        // first pass of a unit: the next unit's token rows have landed (S stages after its
+        // record, no later than this one); its x rows go to L2 while this unit streams
+        if (sc == 0) prefetch_x(kc + 1);
+        const StreamJob& jb = a.job[idc.job];
+        const int c = sc * kPass, W = min(kPass, jb.d_in - c);
+        const uint8_t* st = ring + (size_t)cslot * stage_bytes<WF>();
+        if (col < W && rows_c > 0) {
+            float xf[MAXG][8];
 #pragma unroll
-                for (int j = 0; j < MAXG; ++j) unpack8(*reinterpret_cast<const uint4*>(xst + j * kPass), xf[j]);
-                if constexpr (WF == kFmtInt4) {
+            for (int j = 0; j < MAXG; ++j) unpack8(xc[j], xf[j]);
+            if constexpr (WF == kFmtInt4) {
 #pragma unroll
-                    for (int j = 0; j < MAXG; ++j)
+                for (int j = 0; j < MAXG; ++j)
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) xf[j][e] *= int4_pos_unscale(e);
-                }
+                    for (int e = 0; e < 8; ++e) xf[j][e] *= int4_pos_unscale(e);
+            }
 #pragma unroll
-                for (int kk = 0; kk < kRowGroup; ++kk) {
-                    if (kk < rows_c) {
-                        float af[8];
-                        if constexpr (WF == kFmtBf16)
-                            unpack8(*reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(st) + (size_t)kk * W + col), af);
-                        else if constexpr (WF == kFmtInt4)
-                            int4x8_to_f32_pos(*reinterpret_cast<const uint32_t*>(st + ((size_t)kk * (W >> 3) + tid) * VB), af);
-                        else
-                            load_w8<WF>(st + ((size_t)kk * (W >> 3) + tid) * VB, af);
+            for (int kk = 0; kk < kRowGroup; ++kk) {
+                if (kk < rows_c) {
+                    float af[8];
+                    if constexpr (WF == kFmtBf16)
+                        unpack8(*reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(st) + (size_t)kk * W + col), af);
+                    else if constexpr (WF == kFmtInt4)
+                        int4x8_to_f32_pos(*reinterpret_cast<const uint32_t*>(st + ((size_t)kk * (W >> 3) + tid) * VB), af);
+                    else
+                        load_w8<WF>(st + ((size_t)kk * (W >> 3) + tid) * VB, af);
 #pragma unroll
-                        for (int j = 0; j < MAXG; ++j) pacc[kk * MAXG + j] += dot8(af, xf[j]);
-                    }
+                    for (int j = 0; j < MAXG; ++j) pacc[kk * MAXG + j] += dot8(af, xf[j]);
                 }
             }
-            __syncthreads();  // every thread is done with the slot before it is refilled
-            cslot = cslot + 1 == S ? 0 : cslot + 1;
-            issue();
         }
-        // the unit's v entries: v[row][8 g + kk] of its projection
+        __syncthreads();  // every thread is done with the slot before it is refilled
+        cslot = cslot + 1 == S ? 0 : cslot + 1;
+        issue();
+        if (kn == kc) {
+            sc = sn;
+            return;
+        }
+        // last pass of the unit: its v entries v[row][8 g + kk] of its projection
         const float sum = block_reduce<kRowGroup * MAXG>(pacc, red);
         if (tid < kRowGroup * MAXG && rows_c > 0) {
             const StreamSlot* sl = slot(kc);
             const int4 h = sl->rec[0];
             const int kk = tid / MAXG, j = tid - kk * MAXG;
             if (kk < rows_c && j < h.z - h.y) {
-                const float sc = WF == kFmtBf16 ? 1.f : sl->rsc[kk];
-                jb.v[idc.p][(int64_t)(h.y + j) * jb.ldv[idc.p] + kRowGroup * idc.g + kk] = sum * sc;
+                const float rs = WF == kFmtBf16 ? 1.f : sl->rsc[kk];
+                jb.v[idc.p][(int64_t)(h.y + j) * jb.ldv[idc.p] + kRowGroup * idc.g + kk] = sum * rs;
             }
         }
+#pragma unroll
+        for (int i = 0; i < kRowGroup * MAXG; ++i) pacc[i] = 0.f;
+        kc = kn;
+        sc = 0;
+        uc = un;
+        if (uc < 0) {
+            done = true;
+            return;
+        }
+        idc = idn;
+        rows_c = unit_rows(kc, idc);
+        flag_unit(kc, rows_c);
+    };
+    uint4 x0[MAXG], x1[MAXG];
+    load_x(0, idc, 0, x0);
+    while (!done) {
+        step(x0, x1);
+        if (done) break;
+        step(x1, x0);
     }
     cp_async_wait<0>();
 }
@@ -1332,9 +1383,12 @@ cudaError_t expand_launch(const ExpandJob* jobs, int n_jobs, const BatchView& b,
 // The streaming shrink for a large plan, when it applies (*used = true); otherwise
 // nothing is launched and the caller takes the cluster kernel.  It applies when the
 // plan's items are known on the host (items come largest rank first, so their row-group
-// counts form at most 16 runs), every job streams at least kStreamStages passes a unit,
-// a row group's page ids fit a unit slot, and there are at least two units for every
-// CTA slot.
+// counts form at most 16 runs), every job streams at least as many passes a unit as the
+// ring has stages, a row group's page ids fit a unit slot, and there are at least two
+// units for every CTA slot.  The ring depth (3, 4 or 6 stages) is the one that keeps the
+// most stages in flight on an SM, given how many CTAs fit.
+constexpr int kStreamDepths[3] = {3, 4, 6};
+
 template <int WF>
 cudaError_t stream_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,
                           int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
@@ -1343,7 +1397,7 @@ cudaError_t stream_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b,
     if (!work.host_items || num_items <= 0 || !b.simt_items) return cudaSuccess;
     StreamArgs a;
     std::memset(&a, 0, sizeof(a));
-    // rank groups: runs of equal rank in the plan's item order (largest rank first)
+    // rank groups: runs of equal row-group count in the plan's item order
     int n_rg = 0;
     int64_t rg_units = 0;
     for (int32_t i = 0; i < num_items; ++i) {
@@ -1366,10 +1420,10 @@ cudaError_t stream_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b,
     for (int j = 0; j < n_jobs; ++j) order[j] = j;
     std::stable_sort(order, order + n_jobs, [&](int u, int w) { return jobs[u].d_in > jobs[w].d_in; });
     int64_t units = 0;
-    int ppr_max = 0;
+    int ppr_max = 0, npass_min = 1 << 30;
     for (int i = 0; i < n_jobs; ++i) {
         const ShrinkJob& j = jobs[order[i]];
-        if ((j.d_in + kPass - 1) / kPass < kStreamStages) return cudaSuccess;
+        npass_min = std::min(npass_min, (j.d_in + kPass - 1) / kPass);
         ppr_max = std::max(ppr_max, j.d_in >> pool.page_log2);
         StreamJob& sj = a.job[i];
         sj.x = j.x;
@@ -1387,13 +1441,31 @@ cudaError_t stream_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b,
     }
     const size_t slot_bytes = ((size_t)kStreamSlotHeader + (size_t)kRowGroup * ppr_max * 4 + 15) & ~(size_t)15;
     if (slot_bytes * kStreamSlots > 32768) return cudaSuccess;
-    const int maxg = max_item_rows <= 1 ? 1 : max_item_rows <= 2 ? 2 : 4;
-    auto kern = pick(max_item_rows, shrink_stream_kernel<1, WF>, shrink_stream_kernel<2, WF>,
-                     shrink_stream_kernel<4, WF>);
     const size_t ring_offset = ((size_t)4 * 64 * 4 + slot_bytes * kStreamSlots + 127) & ~(size_t)127;
-    const size_t smem = ring_offset + (size_t)kStreamStages * ((size_t)stage_bytes<WF>() + (size_t)maxg * kPass * 2);
-    const int64_t slots = (int64_t)resident_ctas(reinterpret_cast<const void*>(kern), smem) * num_sms();
-    if (units < 2 * slots) return cudaSuccess;
+    auto smem_for = [&](int S) { return ring_offset + (size_t)S * (size_t)stage_bytes<WF>(); };
+    auto kernel_for = [&](int S) -> const void* {
+        switch (S) {
+            case 3: return reinterpret_cast<const void*>(pick(max_item_rows, shrink_stream_kernel<1, WF, 3>,
+                                                              shrink_stream_kernel<2, WF, 3>, shrink_stream_kernel<4, WF, 3>));
+            case 4: return reinterpret_cast<const void*>(pick(max_item_rows, shrink_stream_kernel<1, WF, 4>,
+                                                              shrink_stream_kernel<2, WF, 4>, shrink_stream_kernel<4, WF, 4>));
+            default: return reinterpret_cast<const void*>(pick(max_item_rows, shrink_stream_kernel<1, WF, 6>,
+                                                               shrink_stream_kernel<2, WF, 6>, shrink_stream_kernel<4, WF, 6>));
+        }
+    };
+    // the depth with the most stages in flight on an SM (ties: fewer stages, more CTAs)
+    int S = 0, best_in_flight = 0;
+    int64_t slots = 0;
+    for (int d : kStreamDepths) {
+        if (d > npass_min) continue;
+        const int per_sm = resident_ctas(kernel_for(d), smem_for(d));
+        if (per_sm * d > best_in_flight) {
+            best_in_flight = per_sm * d;
+            S = d;
+            slots = (int64_t)per_sm * num_sms();
+        }
+    }
+    if (S == 0 || units < 2 * slots) return cudaSuccess;
     a.total_units = units;
     a.b = b;
     a.pool = pool;
@@ -1402,16 +1474,18 @@ cudaError_t stream_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b,
     a.ppr_max = ppr_max;
     a.slot_bytes = (int32_t)slot_bytes;
     a.ring_offset = (int32_t)ring_offset;
-    cudaError_t e = set_smem(kern, smem);
+    const void* kern = kernel_for(S);
+    cudaError_t e = raise_smem(kern, smem_for(S));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)slots, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = smem_for(S);
     cfg.stream = stream;
     cfg.numAttrs = 0;
     *used = true;
-    return cudaLaunchKernelEx(&cfg, kern, a);
+    void* args[] = {&a};
+    return cudaLaunchKernelExC(&cfg, kern, args);
 }
 
 cudaError_t launch_shrink_simt(const ShrinkJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,

@@ -34,7 +34,6 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
-#include <cstddef>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -725,378 +724,6 @@ __global__ void __launch_bounds__(kThreads, 3)
     cp_async_wait<0>();
 }
 
-// ------------------------------------------------------------------ streaming shrink
-// Large plans (many more row groups than CTA slots): a persistent CTA per slot
-// streams a list of work units through one continuous cp.async ring.  A unit is
-// one row group (8 rank rows) of one item for one projection over the whole of
-// d_in, so its dot products are reduced inside the CTA (no cluster, no
-// scratch).  Units are ordered job by job (largest d_in first), rank group by
-// rank group (largest rank first), then item, stacked projection and row group,
-// and dealt to the CTAs in a snake order (k-th unit of CTA c: k G + c for even
-// k, k G + G - 1 - c for odd k), which balances the sorted sizes.
-//
-// What a unit needs besides its stages -- its record, token rows, page ids and
-// (quantised pools) row scales -- travels by cp.async inside the ring's own
-// commit groups, two units ahead: the record of unit k + 2 rides with the first
-// stage of unit k, the rest of unit k + 2 (which needs the record) with the
-// stage issued kStages later.  Every job streams at least kStages passes a unit,
-// so both have landed before unit k + 2's first stage is issued, and the ring
-// never waits for an index load.  Four unit slots in shared memory hold this
-// metadata (a slot is refilled two units after it was last read).
-constexpr int kStreamMaxRankGroups = 16;
-constexpr int kStreamSlots = 4;
-
-struct StreamJob {
-    const uint16_t* x;
-    int64_t ldx;
-    float* v[kMaxShare];
-    int64_t ldv[kMaxShare];
-    int64_t unit_begin;  // first unit of this job
-    int32_t d_in;
-    int32_t nsub;
-    int32_t proj[kMaxShare];
-};
-
-struct StreamArgs {
-    StreamJob job[kMaxGroup];
-    int64_t total_units;
-    BatchView b;
-    PoolView pool;
-    int32_t n_jobs;
-    int32_t n_rg;                                  // rank groups (items of one rank, consecutive)
-    int32_t rg_item[kStreamMaxRankGroups];         // first item of each rank group
-    int32_t rg_ng[kStreamMaxRankGroups];           // row groups of one item of the group
-    int32_t rg_units[kStreamMaxRankGroups + 1];    // prefix over groups of items x row groups
-    int32_t max_rank;
-    int32_t ppr_max;                               // page ids of one rank row, largest d_in
-    int32_t slot_bytes;                            // bytes of one unit slot in shared memory
-    int32_t ring_offset;                           // byte offset of the stage ring
-};
-
-// One unit slot: the item's record for the unit's projection, its token rows, the
-// row scales of its 8 rank rows (quantised pools) and their page ids [row][chunk].
-struct StreamSlot {
-    int4 rec[2];
-    int32_t tok[kSimtMaxItemRows];
-    float rsc[kRowGroup];
-    int32_t pid[1];  // [kRowGroup][ppr]
-};
-constexpr int kStreamSlotHeader = 80;  // bytes before pid
-static_assert(offsetof(StreamSlot, pid) == kStreamSlotHeader, "slot layout");
-
-struct UnitId {
-    int job, item, p, g, npass;
-};
-
-__device__ __forceinline__ UnitId decode_unit(const StreamArgs& a, int64_t u) {
-    UnitId id;
-    int j = 0;
-    while (j + 1 < a.n_jobs && u >= a.job[j + 1].unit_begin) ++j;
-    const int64_t ul = u - a.job[j].unit_begin;
-    const int ns = a.job[j].nsub;
-    int rg = 0;
-    while (rg + 1 < a.n_rg && ul >= (int64_t)ns * a.rg_units[rg + 1]) ++rg;
-    const int64_t w = ul - (int64_t)ns * a.rg_units[rg];
-    const int per_item = ns * a.rg_ng[rg];
-    const int di = (int)(w / per_item);
-    const int rem = (int)(w - (int64_t)di * per_item);
-    id.job = j;
-    id.item = a.rg_item[rg] + di;
-    id.p = rem / a.rg_ng[rg];
-    id.g = rem - id.p * a.rg_ng[rg];
-    id.npass = (a.job[j].d_in + kPass - 1) / kPass;
-    return id;
-}
-
-// k-th unit of this CTA in the snake order, or -1 past the end.
-__device__ __forceinline__ int64_t cta_unit(const StreamArgs& a, int k) {
-    const int64_t G = gridDim.x, c = blockIdx.x;
-    const int64_t u = (int64_t)k * G + ((k & 1) ? G - 1 - c : c);
-    return u < a.total_units ? u : -1;
-}
-
-template <int MAXG, int WF, int S>  // S: stages of the ring (at most one unit's passes)
-__global__ void __launch_bounds__(kThreads, 2)
-    shrink_stream_kernel(const __grid_constant__ StreamArgs a) {
-    extern __shared__ __align__(128) uint8_t smem_s[];
-    pdl_launch_dependents();  // the expand may start staging its B^T pages as slots free up
-    constexpr int VB = bytes_per_8<WF>();
-    const int tid = threadIdx.x, col = kVec * tid;
-    float* red = reinterpret_cast<float*>(smem_s);  // [4 warps][64]
-    uint8_t* slots = smem_s + 4 * 64 * 4;
-    uint8_t* ring = smem_s + a.ring_offset;          // S stages of A rows
-    const int P_log2 = a.pool.page_log2, P = 1 << P_log2;
-    auto slot = [&](int k) { return reinterpret_cast<StreamSlot*>(slots + (size_t)(k & (kStreamSlots - 1)) * a.slot_bytes); };
-
-    // record of unit k into its slot (two 16-byte copies)
-    auto fetch_rec = [&](int k) {
-        const int64_t u = cta_unit(a, k);
-        if (u < 0 || tid >= 2) return;
-        const UnitId id = decode_unit(a, u);
-        const int4* src = reinterpret_cast<const int4*>(a.b.simt_items +
-                                                        ((int64_t)id.item * a.b.n_proj + a.job[id.job].proj[id.p]));
-        cp_async16(&slot(k)->rec[tid], src + tid, true);
-    };
-    // is unit k's record well formed; its rank rows in its row group (0 if not)
-    auto unit_rows = [&](int k, const UnitId& id) {
-        const int4 h = slot(k)->rec[0];
-        const int n = h.z - h.y, r = h.w;
-        const bool ok = h.x >= 0 && h.x < a.b.num_segments && h.y >= 0 && n > 0 && n <= MAXG &&
-                        h.z <= a.b.num_rows && r > 0 && r <= a.max_rank && 8 * id.g < r;
-        return ok ? min(kRowGroup, r - kRowGroup * id.g) : 0;
-    };
-    // the rest of unit k (its record has landed): token rows, row scales, page ids
-    auto fetch_meta = [&](int k) {
-        const int64_t u = cta_unit(a, k);
-        if (u < 0) return;
-        const UnitId id = decode_unit(a, u);
-        StreamSlot* sl = slot(k);
-        const int4 h = sl->rec[0], t = sl->rec[1];
-        const int rows = unit_rows(k, id), n = h.z - h.y;
-        const int64_t a_pt = (int64_t)(((uint64_t)(uint32_t)t.y << 32) | (uint32_t)t.x);
-        const int ppr = a.job[id.job].d_in >> P_log2;
-        if (tid < kSimtMaxItemRows) {
-            if (rows > 0 && tid < n) cp_async4(&sl->tok[tid], a.b.token_idx + h.y + tid);
-            else sl->tok[tid] = -1;
-        }
-        if (WF != kFmtBf16 && tid >= 32 && tid < 32 + kRowGroup) {
-            const int kk = tid - 32;
-            const int64_t e = a_pt + (int64_t)(kRowGroup * id.g + kk) * ppr;
-            if (kk < rows && e >= 0 && e < a.pool.pt_capacity) cp_async4(&sl->rsc[kk], a.pool.row_scale + e);
-            else sl->rsc[kk] = 0.f;
-        }
-        for (int i = tid; i < rows * ppr; i += kThreads) {
-            const int kk = i / ppr, cc = i - kk * ppr;
-            const int64_t e = a_pt + (int64_t)(kRowGroup * id.g + kk) * ppr + cc;
-            if (e >= 0 && e < a.pool.pt_capacity) cp_async4(&sl->pid[i], a.pool.page_table + e);
-            else sl->pid[i] = -1;
-        }
-    };
-    // unit k's token rows, checked (-1: none)
-    auto token = [&](int k, int j) {
-        const int tk = slot(k)->tok[j];
-        return (tk >= 0 && tk < a.b.T) ? tk : -1;
-    };
-
-    // ---- prologue: units 0 and 1 complete before the first stage
-    fetch_rec(0);
-    fetch_rec(1);
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
-    fetch_meta(0);
-    fetch_meta(1);
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
-
-    // ---- issue side: walks (unit ki, pass si); global stage index q
-    int ki = 0, si = 0, islot = 0;
-    int64_t q = 0;
-    int64_t pend_q = -1;
-    int pend_k = -1;
-    UnitId idi;
-    int64_t ui = cta_unit(a, 0);
-    if (ui >= 0) idi = decode_unit(a, ui);
-    int rows_i = ui >= 0 ? unit_rows(0, idi) : 0;
-    auto issue = [&]() {
-        if (ui >= 0) {
-            if (q == pend_q) fetch_meta(pend_k);
-            if (si == 0) {
-                fetch_rec(ki + 2);
-                pend_k = ki + 2;
-                pend_q = q + S;
-            }
-            const StreamSlot* sl = slot(ki);
-            const StreamJob& jb = a.job[idi.job];
-            const int c = si * kPass, W = min(kPass, jb.d_in - c);
-            // A rows of the row group: 16-byte copies, consecutive threads on consecutive granules
-            const int ppr = jb.d_in >> P_log2;
-            uint8_t* dst0 = ring + (size_t)islot * stage_bytes<WF>();
-            if (WF == kFmtBf16 && W == kPass) {  // full pass: thread t copies granule t of each row
-                const int cl = c + col;
-                const int32_t* pidc = sl->pid + (cl >> P_log2);
-                const uint16_t* src0 = a.pool.pages + (cl & (P - 1));
-                uint16_t* dst = reinterpret_cast<uint16_t*>(dst0) + col;
-#pragma unroll
-                for (int kk = 0; kk < kRowGroup; ++kk) {
-                    if (kk < rows_i) {
-                        int32_t page = pidc[kk * ppr];
-                        if (page < 0 || page >= a.pool.num_pages) {
-                            atomicOr(&g_err_simt, kErrPage);
-                            page = 0;
-                        }
-                        cp_async16(dst + kk * kPass, src0 + ((int64_t)page << P_log2), true);
-                    }
-                }
-            } else {
-                const uint8_t* pages = reinterpret_cast<const uint8_t*>(a.pool.pages);
-                const int page_shift = P_log2 + (VB == 16 ? 1 : VB == 8 ? 0 : -1);
-                constexpr int kVals16 = 128 / VB;  // values per 16-byte granule
-                const int gpr = W / kVals16;       // granules per row of the stage
-#pragma unroll
-                for (int i = 0; i < stage_bytes<WF>() / 16 / kThreads; ++i) {
-                    const int gi = tid + kThreads * i;
-                    const int kk = gi / gpr, cg = gi - kk * gpr;
-                    if (kk < rows_i) {
-                        const int cl = c + cg * kVals16;
-                        int32_t page = sl->pid[kk * ppr + (cl >> P_log2)];
-                        if (page < 0 || page >= a.pool.num_pages) {
-                            atomicOr(&g_err_simt, kErrPage);
-                            page = 0;
-                        }
-                        cp_async16(dst0 + (size_t)kk * (W / 8 * VB) + cg * 16,
-                                   pages + ((int64_t)page << page_shift) + (cl & (P - 1)) / 8 * VB, true);
-                    }
-                }
-            }
-            // advance
-            islot = islot + 1 == S ? 0 : islot + 1;
-            ++q;
-            if (++si == idi.npass) {
-                si = 0;
-                ++ki;
-                ui = cta_unit(a, ki);
-                if (ui >= 0) {
-                    idi = decode_unit(a, ui);
-                    rows_i = unit_rows(ki, idi);
-                }
-            }
-        }
-        cp_async_commit();
-    };
-    for (int i = 0; i < S; ++i) issue();
-
-    // ---- consume side.  Each thread's x slice of a stage (8 columns of each token) is
-    // read into registers one stage ahead; a unit's x rows are pulled into L2 when the
-    // unit before it starts.
-    int kc = 0, sc = 0, cslot = 0;
-    int64_t uc = cta_unit(a, 0);
-    if (uc < 0) {
-        cp_async_wait<0>();
-        return;
-    }
-    UnitId idc = decode_unit(a, uc);
-    int rows_c = unit_rows(0, idc);
-    // x slice of (unit k, pass s) into xr
-    auto load_x = [&](int k, const UnitId& id, int s, uint4 (&xr)[MAXG]) {
-        const StreamJob& jb = a.job[id.job];
-        const int c = s * kPass;
-#pragma unroll
-        for (int j = 0; j < MAXG; ++j) {
-            const int tk = token(k, j);
-            xr[j] = (tk >= 0 && c + col < jb.d_in)
-                        ? __ldg(reinterpret_cast<const uint4*>(jb.x + (int64_t)tk * jb.ldx + c + col))
-                        : make_uint4(0u, 0u, 0u, 0u);
-        }
-    };
-    auto prefetch_x = [&](int k) {  // the x rows of unit k into L2
-        const int64_t u = cta_unit(a, k);
-        if (u < 0 || tid >= MAXG) return;
-        const UnitId id = decode_unit(a, u);
-        const int tk = token(k, tid);
-        const StreamJob& jb = a.job[id.job];
-        if (tk >= 0 && tid < slot(k)->rec[0].z - slot(k)->rec[0].y)
-            bulk_prefetch_l2(jb.x + (int64_t)tk * jb.ldx, (uint32_t)jb.d_in * 2);
-    };
-    auto flag_unit = [&](int k, int rows) {
-        if (tid != 0) return;
-        if (rows == 0) atomicOr(&g_err_simt, kErrRows);
-        const StreamSlot* sl = slot(k);
-        for (int j = 0; j < sl->rec[0].z - sl->rec[0].y && j < MAXG && rows > 0; ++j)
-            if (sl->tok[j] < 0 || sl->tok[j] >= a.b.T) atomicOr(&g_err_simt, kErrToken);  // (its x reads as 0)
-    };
-    flag_unit(0, rows_c);
-    float pacc[kRowGroup * MAXG];
-#pragma unroll
-    for (int i = 0; i < kRowGroup * MAXG; ++i) pacc[i] = 0.f;
-    bool done = false;
-    // one stage: x of this stage in xc, x of the next one loaded into xn
-    auto step = [&](uint4 (&xc)[MAXG], uint4 (&xn)[MAXG]) {
-        // the next stage's (unit, pass): its x slice is loaded now, used one stage later
-        int kn = kc, sn = sc + 1;
-        if (sn == idc.npass) {
-            kn = kc + 1;
-            sn = 0;
-        }
-        const int64_t un = cta_unit(a, kn);
-        UnitId idn = idc;
-        if (kn != kc && un >= 0) idn = decode_unit(a, un);
-        if (un >= 0) load_x(kn, idn, sn, xn);
-        cp_async_wait<S - 1>();
-        __syncthreads();
-        // first pass of a unit: the next unit's token rows have landed (S stages after its
-        // record, no later than this one); its x rows go to L2 while this unit streams
-        if (sc == 0) prefetch_x(kc + 1);
-        const StreamJob& jb = a.job[idc.job];
-        const int c = sc * kPass, W = min(kPass, jb.d_in - c);
-        const uint8_t* st = ring + (size_t)cslot * stage_bytes<WF>();
-        if (col < W && rows_c > 0) {
-            float xf[MAXG][8];
-#pragma unroll
-            for (int j = 0; j < MAXG; ++j) unpack8(xc[j], xf[j]);
-            if constexpr (WF == kFmtInt4) {
-#pragma unroll
-                for (int j = 0; j < MAXG; ++j)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) xf[j][e] *= int4_pos_unscale(e);
-            }
-#pragma unroll
-            for (int kk = 0; kk < kRowGroup; ++kk) {
-                if (kk < rows_c) {
-                    float af[8];
-                    if constexpr (WF == kFmtBf16)
-                        unpack8(*reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(st) + (size_t)kk * W + col), af);
-                    else if constexpr (WF == kFmtInt4)
-                        int4x8_to_f32_pos(*reinterpret_cast<const uint32_t*>(st + ((size_t)kk * (W >> 3) + tid) * VB), af);
-                    else
-                        load_w8<WF>(st + ((size_t)kk * (W >> 3) + tid) * VB, af);
-#pragma unroll
-                    for (int j = 0; j < MAXG; ++j) pacc[kk * MAXG + j] += dot8(af, xf[j]);
-                }
-            }
-        }
-        __syncthreads();  // every thread is done with the slot before it is refilled
-        cslot = cslot + 1 == S ? 0 : cslot + 1;
-        issue();
-        if (kn == kc) {
-            sc = sn;
-            return;
-        }
-        // last pass of the unit: its v entries v[row][8 g + kk] of its projection
-        const float sum = block_reduce<kRowGroup * MAXG>(pacc, red);
-        if (tid < kRowGroup * MAXG && rows_c > 0) {
-            const StreamSlot* sl = slot(kc);
-            const int4 h = sl->rec[0];
-            const int kk = tid / MAXG, j = tid - kk * MAXG;
-            if (kk < rows_c && j < h.z - h.y) {
-                const float rs = WF == kFmtBf16 ? 1.f : sl->rsc[kk];
-                jb.v[idc.p][(int64_t)(h.y + j) * jb.ldv[idc.p] + kRowGroup * idc.g + kk] = sum * rs;
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < kRowGroup * MAXG; ++i) pacc[i] = 0.f;
-        kc = kn;
-        sc = 0;
-        uc = un;
-        if (uc < 0) {
-            done = true;
-            return;
-        }
-        idc = idn;
-        rows_c = unit_rows(kc, idc);
-        flag_unit(kc, rows_c);
-    };
-    uint4 x0[MAXG], x1[MAXG];
-    load_x(0, idc, 0, x0);
-    while (!done) {
-        step(x0, x1);
-        if (done) break;
-        step(x1, x0);
-    }
-    cp_async_wait<0>();
-}
-
 int num_sms() {
     static int n = 0;
     if (n == 0) {
@@ -1223,28 +850,26 @@ cudaError_t shrink_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b,
         return (((part_bytes + 1024 + rsc_bytes + pidb + 127) & ~(size_t)127)) + ring_bytes;
     };
     // Cluster size C (chunks of >= 1024 columns, C <= 8, dividing every entry's page
-    // count): the one with the shortest modelled time.
-    int C = 1;
-    double best = 1e300;
+    // count): the smallest C that still gives at least two CTAs for every CTA slot, else
+    // the largest valid one.  A CTA pays its prologue (page ids, then its first stage: two
+    // dependent DRAM round trips) once, so fewer and longer CTAs stream better as long as
+    // there are enough of them to keep every SM busy and balanced; measured on the
+    // workloads (the 70B layer: 263 us with C = 1 against 284-286 us with C = 2 or 4; the
+    // decode and mixed-rank batches, with fewer items than slots, take the largest C).
+    int C = 0, C_max = 1;
     for (int c = 1; c <= 8; ++c) {
         bool valid = true;
-        int cpi[kMaxGroup], np[kMaxGroup];
-        double wp[kMaxGroup];
         for (int j = 0; j < n_jobs; ++j) {
             const int d = jobs[j].d_in;
             if (((d >> pool.page_log2) % c) || (c > 1 && d / c < kPass)) valid = false;
-            cpi[j] = c;
-            np[j] = jobs[j].nsub * ((d / c + kPass - 1) / kPass);  // a CTA streams every stacked projection
-            wp[j] = (double)np[j] * c;
         }
         if (!valid) continue;
-        const double t = group_time(work, num_items, cpi, np, wp, n_jobs,
-                                    (int64_t)resident_ctas(kp, smem_for(c)) * num_sms());
-        if (t < best) {
-            best = t;
-            C = c;
-        }
+        C_max = c;
+        const int64_t ctas = (int64_t)n_jobs * num_items * c;
+        if (C == 0 && ctas >= 2 * (int64_t)resident_ctas(kp, smem_for(c)) * num_sms()) C = c;
     }
+    if (C == 0) C = C_max;
+    (void)work;
     ShrinkArgs<NE> a;
     std::memset(&a, 0, sizeof(a));
     for (int i = 0; i < n_jobs; ++i) {
@@ -1380,114 +1005,6 @@ cudaError_t expand_launch(const ExpandJob* jobs, int n_jobs, const BatchView& b,
     return cudaLaunchKernelEx(&cfg, kern_tab, a, InlineTable<1>{});
 }
 
-// The streaming shrink for a large plan, when it applies (*used = true); otherwise
-// nothing is launched and the caller takes the cluster kernel.  It applies when the
-// plan's items are known on the host (items come largest rank first, so their row-group
-// counts form at most 16 runs), every job streams at least as many passes a unit as the
-// ring has stages, a row group's page ids fit a unit slot, and there are at least two
-// units for every CTA slot.  The ring depth (3, 4 or 6 stages) is the one that keeps the
-// most stages in flight on an SM, given how many CTAs fit.
-constexpr int kStreamDepths[3] = {3, 4, 6};
-
-template <int WF>
-cudaError_t stream_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,
-                          int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
-                          cudaStream_t stream, bool* used) {
-    *used = false;
-    if (!work.host_items || num_items <= 0 || !b.simt_items) return cudaSuccess;
-    StreamArgs a;
-    std::memset(&a, 0, sizeof(a));
-    // rank groups: runs of equal row-group count in the plan's item order
-    int n_rg = 0;
-    int64_t rg_units = 0;
-    for (int32_t i = 0; i < num_items; ++i) {
-        const int r = work.host_items[(int64_t)i * work.n_proj].rank;
-        if (r <= 0 || r > max_rank) return cudaSuccess;
-        const int ng = (r + kRowGroup - 1) / kRowGroup;
-        if (n_rg == 0 || a.rg_ng[n_rg - 1] != ng) {  // (ranks descend: at most 16 row-group counts)
-            if (n_rg == kStreamMaxRankGroups) return cudaSuccess;
-            a.rg_item[n_rg] = i;
-            a.rg_ng[n_rg] = ng;
-            a.rg_units[n_rg] = (int32_t)rg_units;
-            ++n_rg;
-        }
-        rg_units += ng;
-    }
-    a.rg_units[n_rg] = (int32_t)rg_units;
-    a.n_rg = n_rg;
-    // jobs, largest d_in first
-    int order[kMaxGroup];
-    for (int j = 0; j < n_jobs; ++j) order[j] = j;
-    std::stable_sort(order, order + n_jobs, [&](int u, int w) { return jobs[u].d_in > jobs[w].d_in; });
-    int64_t units = 0;
-    int ppr_max = 0, npass_min = 1 << 30;
-    for (int i = 0; i < n_jobs; ++i) {
-        const ShrinkJob& j = jobs[order[i]];
-        npass_min = std::min(npass_min, (j.d_in + kPass - 1) / kPass);
-        ppr_max = std::max(ppr_max, j.d_in >> pool.page_log2);
-        StreamJob& sj = a.job[i];
-        sj.x = j.x;
-        sj.ldx = j.ldx;
-        sj.d_in = j.d_in;
-        sj.nsub = j.nsub;
-        for (int k = 0; k < kMaxShare; ++k) {
-            const int src = k < j.nsub ? k : 0;
-            sj.proj[k] = j.proj[src];
-            sj.v[k] = j.v[src];
-            sj.ldv[k] = j.ldv[src];
-        }
-        sj.unit_begin = units;
-        units += (int64_t)j.nsub * rg_units;
-    }
-    const size_t slot_bytes = ((size_t)kStreamSlotHeader + (size_t)kRowGroup * ppr_max * 4 + 15) & ~(size_t)15;
-    if (slot_bytes * kStreamSlots > 32768) return cudaSuccess;
-    const size_t ring_offset = ((size_t)4 * 64 * 4 + slot_bytes * kStreamSlots + 127) & ~(size_t)127;
-    auto smem_for = [&](int S) { return ring_offset + (size_t)S * (size_t)stage_bytes<WF>(); };
-    auto kernel_for = [&](int S) -> const void* {
-        switch (S) {
-            case 3: return reinterpret_cast<const void*>(pick(max_item_rows, shrink_stream_kernel<1, WF, 3>,
-                                                              shrink_stream_kernel<2, WF, 3>, shrink_stream_kernel<4, WF, 3>));
-            case 4: return reinterpret_cast<const void*>(pick(max_item_rows, shrink_stream_kernel<1, WF, 4>,
-                                                              shrink_stream_kernel<2, WF, 4>, shrink_stream_kernel<4, WF, 4>));
-            default: return reinterpret_cast<const void*>(pick(max_item_rows, shrink_stream_kernel<1, WF, 6>,
-                                                               shrink_stream_kernel<2, WF, 6>, shrink_stream_kernel<4, WF, 6>));
-        }
-    };
-    // the depth with the most stages in flight on an SM (ties: fewer stages, more CTAs)
-    int S = 0, best_in_flight = 0;
-    int64_t slots = 0;
-    for (int d : kStreamDepths) {
-        if (d > npass_min) continue;
-        const int per_sm = resident_ctas(kernel_for(d), smem_for(d));
-        if (per_sm * d > best_in_flight) {
-            best_in_flight = per_sm * d;
-            S = d;
-            slots = (int64_t)per_sm * num_sms();
-        }
-    }
-    if (S == 0 || units < 2 * slots) return cudaSuccess;
-    a.total_units = units;
-    a.b = b;
-    a.pool = pool;
-    a.n_jobs = n_jobs;
-    a.max_rank = max_rank;
-    a.ppr_max = ppr_max;
-    a.slot_bytes = (int32_t)slot_bytes;
-    a.ring_offset = (int32_t)ring_offset;
-    const void* kern = kernel_for(S);
-    cudaError_t e = raise_smem(kern, smem_for(S));
-    if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)slots, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem_for(S);
-    cfg.stream = stream;
-    cfg.numAttrs = 0;
-    *used = true;
-    void* args[] = {&a};
-    return cudaLaunchKernelExC(&cfg, kern, args);
-}
-
 cudaError_t launch_shrink_simt(const ShrinkJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,
                                int32_t max_item_rows, int32_t max_rank, const SimtWork& work, const PoolView& pool,
                                const InlineTable<kInlineItems>* inl, cudaStream_t stream) {
@@ -1498,12 +1015,6 @@ cudaError_t launch_shrink_simt(const ShrinkJob* jobs, int n_jobs, const BatchVie
     // one x: a one-entry table (small launch arguments, no per-CTA lookup)
     auto go = [&](auto wf) {
         constexpr int WF = decltype(wf)::value;
-        if (!inl) {  // a large plan streams through persistent CTAs
-            bool used = false;
-            const cudaError_t e =
-                stream_launch<WF>(jobs, n_jobs, b, num_items, max_item_rows, max_rank, work, pool, stream, &used);
-            if (used || e != cudaSuccess) return e;
-        }
         if (n_jobs == 1)
             return shrink_launch<1, WF>(jobs, n_jobs, b, num_items, max_item_rows, max_rank, work, pool, inl, stream);
         return shrink_launch<kMaxGroup, WF>(jobs, n_jobs, b, num_items, max_item_rows, max_rank, work, pool, inl,

@@ -298,6 +298,12 @@ sgmv_status sgmv::delta_impl(const sgmv_delta_entry* entries, int32_t n, int32_t
         ++j.nsub;
     }
     if (use_inl && sj[0].nsub > 1) return fail(SGMV_ERR_INVALID, "lora_delta: internal: shared x with inline items");
+    if (n == 1 && plan->num_tc_tiles == 0) {  // decode-sized: both phases in one kernel when it fits
+        bool used = false;
+        SGMV_CUDA_TRY(launch_fused_simt(sj[0], ej[0], bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank,
+                                        pv, scale, y_dtype, use_inl ? &inl : nullptr, stream, &used));
+        if (used) return SGMV_OK;
+    }
     SGMV_CUDA_TRY(launch_shrink_simt(sj, n_sj, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, work, pv,
                                      use_inl ? &inl : nullptr, stream));
     for (int32_t i = 0; i < n; ++i) {

@@ -724,6 +724,274 @@ __global__ void __launch_bounds__(kThreads, 3)
     cp_async_wait<0>();
 }
 
+// ------------------------------------------------------------------ one-shot fused decode
+// A decode-sized call (one projection; every SIMT item's cluster resident in one wave; a
+// CTA's slices of A, x, B^T and y small enough to stage whole) runs both phases in one
+// kernel.  A cluster of C CTAs per item: CTA q owns d_in columns [q kc, (q+1) kc) and d_out
+// columns [q ko, (q+1) ko).  After one round of page-id loads every CTA issues all of its
+// copies at once -- A rows and x slices as one commit group, B^T rows and y rows as a second
+// -- so the whole call pays one DRAM round trip for its data.  The shrink's partial tile is
+// pushed to every CTA of the cluster (distributed shared memory); after the cluster barrier
+// each CTA sums the C tiles in a fixed order (the same bits as the two-kernel path) and
+// runs its share of the expand from shared memory.  The loops and their orders are those of
+// shrink_item and expand_item, so the result equals the two-kernel path's bit for bit.
+struct FusedArgs {
+    const uint16_t* x;
+    int64_t ldx;
+    float* v;
+    int64_t ldv;
+    void* y;
+    int64_t ldy;
+    BatchView b;
+    PoolView pool;
+    int32_t d_in, d_out;
+    int32_t kc, ko;          // d_in / d_out columns per CTA (multiples of the page size)
+    int32_t proj;
+    int32_t cluster;         // C
+    int32_t max_rank;        // rank capacity of the shared-memory tiles (>= 8)
+    int32_t y_dtype;
+    float scale;
+    // byte offsets in shared memory
+    int32_t off_part, off_vs, off_rsc, off_pid_a, off_pid_b, off_a, off_x, off_b, off_y;
+};
+
+template <int MAXG, int NI, int WF>
+__global__ void __launch_bounds__(kThreads, 1)
+    fused_simt_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ InlineTable<NI> inl) {
+    extern __shared__ __align__(128) uint8_t smem_f[];
+    constexpr int VB = bytes_per_8<WF>();
+    const int tid = threadIdx.x, col = kVec * tid;
+    const int C = a.cluster;
+    // every CTA of the cluster is running before any pushes into another's shared memory
+    if (C > 1) cluster_arrive_relaxed();
+    const int item_idx = (int)blockIdx.x / C;
+    const uint32_t q = cluster_ctarank();
+    float* red = reinterpret_cast<float*>(smem_f);                       // [4 warps][64]
+    float* part = reinterpret_cast<float*>(smem_f + a.off_part);         // [C][4 x max_rank]
+    float* vs = reinterpret_cast<float*>(smem_f + a.off_vs);             // [4 x max_rank]
+    float* rsc_a = reinterpret_cast<float*>(smem_f + a.off_rsc);         // [kMaxRank] (quantised)
+    float* rsc_b = rsc_a + kMaxRank;
+    int32_t* pid_a = reinterpret_cast<int32_t*>(smem_f + a.off_pid_a);  // [r][kc / P]
+    int32_t* pid_b = reinterpret_cast<int32_t*>(smem_f + a.off_pid_b);  // [r][ko / P]
+    uint8_t* As = smem_f + a.off_a;                                      // [r][kc] weights
+    uint16_t* xs = reinterpret_cast<uint16_t*>(smem_f + a.off_x);        // [MAXG][kc]
+    uint8_t* Bs = smem_f + a.off_b;                                      // [r][ko] weights
+    uint8_t* ys = smem_f + a.off_y;                                      // [MAXG][ko] of y's type
+    const int slot = kSimtMaxItemRows * a.max_rank;
+
+    ItemInfo ma = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 0)
+                         : load_item(a.b, a.proj, item_idx, MAXG, a.max_rank, 0);
+    const ItemInfo mb = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 1)
+                               : load_item(a.b, a.proj, item_idx, MAXG, a.max_rank, 1);
+    if (!ma.ok && tid == 0) atomicOr(&g_err_simt, kErrRows);
+    const int r = ma.r, n = ma.n;
+    const int P_log2 = a.pool.page_log2, P = 1 << P_log2;
+    const int ppr_a = a.d_in >> P_log2, ppr_b = a.d_out >> P_log2;
+    const int cpa = a.kc >> P_log2, cpb = a.ko >> P_log2;  // pages of a row in this CTA's slices
+    const int ca0 = (int)q * a.kc, cb0 = (int)q * a.ko;     // first column of the slices
+
+    // page ids of both slices (one round of independent loads), row scales of quantised pools
+    if (ma.ok) {
+        for (int i = tid; i < r * (cpa + cpb); i += kThreads) {
+            const bool isa = i < r * cpa;
+            const int ii = isa ? i : i - r * cpa, cp = isa ? cpa : cpb;
+            const int k = ii / cp, pc = ii - k * cp;
+            const int64_t e = isa ? ma.pt + (int64_t)k * ppr_a + (ca0 >> P_log2) + pc
+                                  : mb.pt + (int64_t)k * ppr_b + (cb0 >> P_log2) + pc;
+            int32_t page = (e >= 0 && e < a.pool.pt_capacity) ? a.pool.page_table[e] : -1;
+            if (page < 0 || page >= a.pool.num_pages) {
+                atomicOr(&g_err_simt, kErrPage);
+                page = 0;
+            }
+            (isa ? pid_a : pid_b)[ii] = page;
+        }
+        if (WF != kFmtBf16) {
+            load_row_scales(a.pool, ma.pt, ppr_a, r, rsc_a, &g_err_simt);
+            load_row_scales(a.pool, mb.pt, ppr_b, r, rsc_b, &g_err_simt);
+        }
+    }
+    __syncthreads();
+
+    // every copy at once: group 1 = A rows + x slices, group 2 = B^T rows + y rows
+    const uint8_t* pages = reinterpret_cast<const uint8_t*>(a.pool.pages);
+    const int page_shift = P_log2 + (VB == 16 ? 1 : VB == 8 ? 0 : -1);
+    constexpr int kVals16 = 128 / VB;  // values per 16-byte granule
+    if (ma.ok) {
+        const int gpr_a = a.kc / kVals16;
+        for (int gi = tid; gi < r * gpr_a; gi += kThreads) {
+            const int k = gi / gpr_a, cg = gi - k * gpr_a, cl = cg * kVals16;
+            cp_async16(As + (size_t)k * (a.kc / 8 * VB) + cg * 16,
+                       pages + ((int64_t)pid_a[k * cpa + (cl >> P_log2)] << page_shift) + (cl & (P - 1)) / 8 * VB,
+                       true);
+        }
+        for (int gi = tid; gi < MAXG * (a.kc / 8); gi += kThreads) {
+            const int j = gi / (a.kc / 8), cg = gi - j * (a.kc / 8);
+            const int t = ma.tok[j];
+            cp_async16(xs + (size_t)j * a.kc + cg * 8,
+                       t >= 0 ? a.x + (int64_t)t * a.ldx + ca0 + cg * 8 : a.x, t >= 0);
+        }
+    }
+    cp_async_commit();
+    const int esz = a.y_dtype == 0 ? 2 : 4;
+    if (ma.ok) {
+        const int gpr_b = a.ko / kVals16;
+        for (int gi = tid; gi < r * gpr_b; gi += kThreads) {
+            const int k = gi / gpr_b, cg = gi - k * gpr_b, cl = cg * kVals16;
+            cp_async16(Bs + (size_t)k * (a.ko / 8 * VB) + cg * 16,
+                       pages + ((int64_t)pid_b[k * cpb + (cl >> P_log2)] << page_shift) + (cl & (P - 1)) / 8 * VB,
+                       true);
+        }
+        const int gy = a.ko * esz / 16;  // granules of one y row slice
+        for (int gi = tid; gi < MAXG * gy; gi += kThreads) {
+            const int j = gi / gy, cg = gi - j * gy;
+            const int t = mb.tok[j];
+            const uint8_t* src = static_cast<const uint8_t*>(a.y);
+            cp_async16(ys + (size_t)j * a.ko * esz + cg * 16,
+                       t >= 0 ? src + ((int64_t)t * a.ldy + cb0) * esz + cg * 16 : src, t >= 0);
+        }
+    }
+    cp_async_commit();
+
+    // ---- shrink over this CTA's d_in slice: row groups outer, 1024-column passes inner
+    cp_async_wait<1>();
+    __syncthreads();
+    float* mine = part + (size_t)q * slot;  // this CTA's partial tile [token][rank row]
+    if (ma.ok) {
+        const int NG = (r + kRowGroup - 1) / kRowGroup, npass = (a.kc + kPass - 1) / kPass;
+        for (int g = 0; g < NG; ++g) {
+            float p[kRowGroup * MAXG];
+#pragma unroll
+            for (int i = 0; i < kRowGroup * MAXG; ++i) p[i] = 0.f;
+            for (int s = 0; s < npass; ++s) {
+                const int c = s * kPass, W = min(kPass, a.kc - c);
+                if (col < W) {
+                    float xf[MAXG][8];
+#pragma unroll
+                    for (int j = 0; j < MAXG; ++j)
+                        unpack8(*reinterpret_cast<const uint4*>(xs + (size_t)j * a.kc + c + col), xf[j]);
+                    if constexpr (WF == kFmtInt4) {
+#pragma unroll
+                        for (int j = 0; j < MAXG; ++j)
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) xf[j][e] *= int4_pos_unscale(e);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < kRowGroup; ++kk) {
+                        const int k = kRowGroup * g + kk;
+                        if (k < r) {
+                            float af[8];
+                            const uint8_t* w = As + (size_t)k * (a.kc / 8 * VB) + (size_t)(c + col) / 8 * VB;
+                            if constexpr (WF == kFmtInt4) int4x8_to_f32_pos(*reinterpret_cast<const uint32_t*>(w), af);
+                            else load_w8<WF>(w, af);
+#pragma unroll
+                            for (int j = 0; j < MAXG; ++j) p[kk * MAXG + j] += dot8(af, xf[j]);
+                        }
+                    }
+                }
+            }
+            const float sum = block_reduce<kRowGroup * MAXG>(p, red);
+            if (tid < kRowGroup * MAXG) {
+                const int kk = tid / MAXG, j = tid - kk * MAXG;
+                if (kRowGroup * g + kk < r && j < n) mine[j * r + kRowGroup * g + kk] = sum;
+            }
+        }
+    }
+    __syncthreads();  // this CTA's partial tile is complete
+
+    // ---- push the tile to every other CTA of the cluster, then sum the C tiles in order
+    const int E = n * r;
+    if (C > 1) {
+        cluster_wait_acquire();  // (first phase: every CTA of the cluster has started)
+        for (int qq = 0; qq < C; ++qq) {
+            if (qq == (int)q) continue;
+            const uint32_t dst = map_cluster(smem_u32(mine), (uint32_t)qq);
+            for (int e = tid; e < E; e += kThreads) st_cluster_f32(dst + 4u * (uint32_t)e, mine[e]);
+        }
+        cluster_arrive_release();
+        cluster_wait_acquire();
+    }
+    if (ma.ok) {
+        for (int e = tid; e < E; e += kThreads) {
+            float s = 0.f;
+            for (int qq = 0; qq < C; ++qq) s += part[(size_t)qq * slot + e];
+            const int k = e - (e / r) * r;
+            const float vk = WF == kFmtBf16 ? s : s * rsc_a[k];
+            if (q == 0) a.v[(int64_t)(ma.i0 + e / r) * a.ldv + k] = vk;
+            vs[e] = WF == kFmtBf16 ? vk : vk * rsc_b[k];  // a quantised B^T row's scale goes onto v_k
+        }
+    }
+    cp_async_wait<0>();
+    __syncthreads();  // vs, and the B^T and y slices, are visible to every thread
+
+    // ---- expand over this CTA's d_out slice: 1024-column passes, each over every rank row
+    if (!mb.ok) return;
+    const float sc = a.scale * mb.sc;  // the call's scale times the adapter's
+    const int NG = (r + kRowGroup - 1) / kRowGroup, npass = (a.ko + kPass - 1) / kPass;
+    for (int s = 0; s < npass; ++s) {
+        const int c = s * kPass, W = min(kPass, a.ko - c);
+        if (col >= W) continue;
+        float acc[MAXG][8];
+#pragma unroll
+        for (int j = 0; j < MAXG; ++j)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+        for (int g = 0; g < NG; ++g) {
+#pragma unroll
+            for (int kk = 0; kk < kRowGroup; ++kk) {
+                const int k = kRowGroup * g + kk;
+                if (k < r) {
+                    float bf[8];
+                    const uint8_t* w = Bs + (size_t)k * (a.ko / 8 * VB) + (size_t)(c + col) / 8 * VB;
+                    if constexpr (WF == kFmtInt4) int4x8_to_f32_pos(*reinterpret_cast<const uint32_t*>(w), bf);
+                    else load_w8<WF>(w, bf);
+#pragma unroll
+                    for (int j = 0; j < MAXG; ++j) {
+                        const float wv = vs[min(j, n - 1) * r + k];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[j][e] = fmaf(wv, bf[e], acc[j][e]);
+                    }
+                }
+            }
+        }
+        if constexpr (WF == kFmtInt4) {
+#pragma unroll
+            for (int j = 0; j < MAXG; ++j)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[j][e] *= int4_pos_unscale(e);
+        }
+        const int jcol = cb0 + c + col;
+#pragma unroll
+        for (int j = 0; j < MAXG; ++j) {
+            const int t = mb.tok[j];
+            if (t < 0) continue;
+            if (a.y_dtype == 0) {
+                float yv[8];
+                unpack8(*reinterpret_cast<const uint4*>(ys + ((size_t)j * a.ko + c + col) * 2), yv);
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float lo = fmaf(sc, acc[j][2 * e], yv[2 * e]);
+                    const float hi = fmaf(sc, acc[j][2 * e + 1], yv[2 * e + 1]);
+                    w[e] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+                           ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+                }
+                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.y) + (int64_t)t * a.ldy + jcol) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+            } else {
+                const float* yp = reinterpret_cast<const float*>(ys + ((size_t)j * a.ko + c + col) * 4);
+                float4 o0 = *reinterpret_cast<const float4*>(yp), o1 = *reinterpret_cast<const float4*>(yp + 4);
+                o0.x = fmaf(sc, acc[j][0], o0.x); o0.y = fmaf(sc, acc[j][1], o0.y);
+                o0.z = fmaf(sc, acc[j][2], o0.z); o0.w = fmaf(sc, acc[j][3], o0.w);
+                o1.x = fmaf(sc, acc[j][4], o1.x); o1.y = fmaf(sc, acc[j][5], o1.y);
+                o1.z = fmaf(sc, acc[j][6], o1.z); o1.w = fmaf(sc, acc[j][7], o1.w);
+                float* yo = static_cast<float*>(a.y) + (int64_t)t * a.ldy + jcol;
+                *reinterpret_cast<float4*>(yo) = o0;
+                *reinterpret_cast<float4*>(yo + 4) = o1;
+            }
+        }
+    }
+}
+
 int num_sms() {
     static int n = 0;
     if (n == 0) {
@@ -1003,6 +1271,119 @@ cudaError_t expand_launch(const ExpandJob* jobs, int n_jobs, const BatchView& b,
     cudaError_t e = set_smem(kern_tab, smem);
     if (e != cudaSuccess) return e;
     return cudaLaunchKernelEx(&cfg, kern_tab, a, InlineTable<1>{});
+}
+
+// The one-shot fused kernel for a single projection, when every item's cluster fits in
+// one wave and a CTA's slices fit in shared memory (*used = true); otherwise nothing is
+// launched.  The largest cluster size that fits is taken (the most CTAs loading at once).
+template <int WF>
+cudaError_t fused_launch(const ShrinkJob& sj, const ExpandJob& ej, const BatchView& b, int32_t num_items,
+                         int32_t max_item_rows, int32_t max_rank, const PoolView& pool, float scale, int32_t y_dtype,
+                         const InlineTable<kInlineItems>* inl, cudaStream_t stream, bool* used) {
+    *used = false;
+    if (num_items <= 0 || sj.nsub != 1 || sj.d_in <= 0 || ej.d_out <= 0) return cudaSuccess;
+    const int maxg = max_item_rows <= 1 ? 1 : max_item_rows <= 2 ? 2 : 4;
+    const int mr = std::max(8, max_rank);
+    const int esz = y_dtype == 0 ? 2 : 4;
+    const int pa = sj.d_in >> pool.page_log2, pb = ej.d_out >> pool.page_log2;
+    auto al = [](size_t v) { return (v + 127) & ~(size_t)127; };
+    auto kern_for = [&](bool use_inl) -> const void* {
+        if (use_inl)
+            return reinterpret_cast<const void*>(pick(max_item_rows, fused_simt_kernel<1, kInlineItems, WF>,
+                                                      fused_simt_kernel<2, kInlineItems, WF>,
+                                                      fused_simt_kernel<4, kInlineItems, WF>));
+        return reinterpret_cast<const void*>(pick(max_item_rows, fused_simt_kernel<1, 1, WF>,
+                                                  fused_simt_kernel<2, 1, WF>, fused_simt_kernel<4, 1, WF>));
+    };
+    const void* kern = kern_for(inl != nullptr);
+    for (int C = 8; C >= 1; --C) {
+        if ((pa % C) || (pb % C)) continue;
+        const int kc = sj.d_in / C, ko = ej.d_out / C;
+        FusedArgs a;
+        std::memset(&a, 0, sizeof(a));
+        size_t o = 4 * 64 * 4;  // block-reduction scratch
+        a.off_part = (int32_t)(o = al(o));
+        o += (size_t)C * kSimtMaxItemRows * mr * 4;
+        a.off_vs = (int32_t)(o = al(o));
+        o += (size_t)kSimtMaxItemRows * mr * 4;
+        a.off_rsc = (int32_t)(o = al(o));
+        o += WF == kFmtBf16 ? 0 : 2 * kMaxRank * 4;
+        a.off_pid_a = (int32_t)(o = al(o));
+        o += (size_t)mr * (pa / C) * 4;
+        a.off_pid_b = (int32_t)(o = al(o));
+        o += (size_t)mr * (pb / C) * 4;
+        a.off_a = (int32_t)(o = al(o));
+        o += (size_t)mr * kc / 8 * bytes_per_8<WF>();
+        a.off_x = (int32_t)(o = al(o));
+        o += (size_t)maxg * kc * 2;
+        a.off_b = (int32_t)(o = al(o));
+        o += (size_t)mr * ko / 8 * bytes_per_8<WF>();
+        a.off_y = (int32_t)(o = al(o));
+        o += (size_t)maxg * ko * esz;
+        const size_t smem = al(o);
+        if (smem > 227 * 1024) continue;
+        const int per_sm = resident_ctas(kern, smem);
+        if ((int64_t)num_items * C > (int64_t)per_sm * num_sms()) continue;  // one wave
+        a.x = sj.x;
+        a.ldx = sj.ldx;
+        a.v = sj.v[0];
+        a.ldv = sj.ldv[0];
+        a.y = ej.y;
+        a.ldy = ej.ldy;
+        a.b = b;
+        a.pool = pool;
+        a.d_in = sj.d_in;
+        a.d_out = ej.d_out;
+        a.kc = kc;
+        a.ko = ko;
+        a.proj = sj.proj[0];
+        a.cluster = C;
+        a.max_rank = mr;
+        a.y_dtype = y_dtype;
+        a.scale = scale;
+        cudaError_t e = raise_smem(kern, smem);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(num_items * C), 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        *used = true;
+        if (inl) {
+            void* args[] = {&a, const_cast<InlineTable<kInlineItems>*>(inl)};
+            return cudaLaunchKernelExC(&cfg, kern, args);
+        }
+        InlineTable<1> none{};
+        void* args[] = {&a, &none};
+        return cudaLaunchKernelExC(&cfg, kern, args);
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_fused_simt(const ShrinkJob& sj, const ExpandJob& ej, const BatchView& b, int32_t num_items,
+                              int32_t max_item_rows, int32_t max_rank, const PoolView& pool, float scale,
+                              int32_t y_dtype, const InlineTable<kInlineItems>* inl, cudaStream_t stream,
+                              bool* used) {
+    *used = false;
+    switch (pool.wfmt) {
+        case kFmtBf16:
+            return fused_launch<kFmtBf16>(sj, ej, b, num_items, max_item_rows, max_rank, pool, scale, y_dtype, inl,
+                                          stream, used);
+        case kFmtFp8:
+            return fused_launch<kFmtFp8>(sj, ej, b, num_items, max_item_rows, max_rank, pool, scale, y_dtype, inl,
+                                         stream, used);
+        case kFmtInt4:
+            return fused_launch<kFmtInt4>(sj, ej, b, num_items, max_item_rows, max_rank, pool, scale, y_dtype, inl,
+                                          stream, used);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t launch_shrink_simt(const ShrinkJob* jobs, int n_jobs, const BatchView& b, int32_t num_items,

@@ -560,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 3)
 }
 
 // ------------------------------------------------------------------ expand
-template <int G, int NE, int WF>
+template <int G, int NE, int WF, int YT>  // YT: y type, 0 = bf16, 1 = fp32
 __device__ void expand_item(const ExpandArgs<NE>& a, const ExpandEntry& en, const ItemInfo& m,
                             Pipe<kExpandStages, WF>& pp, const StageGeom& sg, float* vs, const float* rsc) {
     constexpr int VB = bytes_per_8<WF>();
@@ -570,7 +570,7 @@ __device__ void expand_item(const ExpandArgs<NE>& a, const ExpandEntry& en, cons
 #pragma unroll
     for (int j = 0; j < G; ++j) trow[j] = m.tok[j];
     // y of a pass is loaded one pass ahead of its update (two buffers)
-    // (bf16 y: the 16 bytes live in the first float4)
+    // (bf16 y: the 16 bytes live in the first float4; the second is used for fp32 y only)
     float4 y0[G], y1[G], n0[G], n1[G];
     auto load_y = [&](int s, float4 (&d0)[G], float4 (&d1)[G]) {
         const int c = s * kPass, jcol = sg.col_base + c + col;
@@ -578,7 +578,7 @@ __device__ void expand_item(const ExpandArgs<NE>& a, const ExpandEntry& en, cons
 #pragma unroll
         for (int j = 0; j < G; ++j) {
             if (active && trow[j] >= 0) {
-                if (a.y_dtype == 0) {
+                if constexpr (YT == 0) {
                     d0[j] = *reinterpret_cast<const float4*>(static_cast<const uint16_t*>(en.y) +
                                                              (int64_t)trow[j] * en.ldy + jcol);
                 } else {
@@ -642,7 +642,7 @@ __device__ void expand_item(const ExpandArgs<NE>& a, const ExpandEntry& en, cons
 #pragma unroll
         for (int j = 0; j < G; ++j) {
             if (!active || trow[j] < 0) continue;
-            if (a.y_dtype == 0) {
+            if constexpr (YT == 0) {
                 float yv[8];
                 const float4 q = y0[j];
                 unpack8(make_uint4(__float_as_uint(q.x), __float_as_uint(q.y), __float_as_uint(q.z),
@@ -671,13 +671,13 @@ __device__ void expand_item(const ExpandArgs<NE>& a, const ExpandEntry& en, cons
 #pragma unroll
         for (int j = 0; j < G; ++j) {
             y0[j] = n0[j];
-            y1[j] = n1[j];
+            if constexpr (YT == 1) y1[j] = n1[j];
         }
     }
 }
 
-template <int MAXG, int NI, int NE, int WF>
-__global__ void __launch_bounds__(kThreads, 3)
+template <int MAXG, int NI, int NE, int WF, int YT>
+__global__ void __launch_bounds__(kThreads, 4)
     expand_simt_kernel(const __grid_constant__ ExpandArgs<NE> a, const __grid_constant__ InlineTable<NI> inl) {
     extern __shared__ __align__(128) uint8_t smem_e[];
     int ei = 0;  // this CTA's entry: the last whose first CTA is at or before it
@@ -718,9 +718,9 @@ __global__ void __launch_bounds__(kThreads, 3)
         cp_async_wait<0>();
         return;
     }
-    if (MAXG == 1 || m.n == 1) expand_item<1, NE>(a, en, m, pp, sg, vs, rsc);
-    else if (MAXG == 2 || m.n == 2) expand_item<(MAXG < 2 ? MAXG : 2), NE>(a, en, m, pp, sg, vs, rsc);
-    else expand_item<MAXG, NE>(a, en, m, pp, sg, vs, rsc);
+    if (MAXG == 1 || m.n == 1) expand_item<1, NE, WF, YT>(a, en, m, pp, sg, vs, rsc);
+    else if (MAXG == 2 || m.n == 2) expand_item<(MAXG < 2 ? MAXG : 2), NE, WF, YT>(a, en, m, pp, sg, vs, rsc);
+    else expand_item<MAXG, NE, WF, YT>(a, en, m, pp, sg, vs, rsc);
     cp_async_wait<0>();
 }
 
@@ -1196,10 +1196,16 @@ cudaError_t expand_launch(const ExpandJob* jobs, int n_jobs, const BatchView& b,
     int order[kMaxGroup];
     for (int j = 0; j < n_jobs; ++j) order[j] = j;
     std::stable_sort(order, order + n_jobs, [&](int u, int w) { return jobs[u].d_out > jobs[w].d_out; });
-    auto kern_inl = pick(max_item_rows, expand_simt_kernel<1, kInlineItems, NE, WF>,
-                         expand_simt_kernel<2, kInlineItems, NE, WF>, expand_simt_kernel<4, kInlineItems, NE, WF>);
-    auto kern_tab = pick(max_item_rows, expand_simt_kernel<1, 1, NE, WF>, expand_simt_kernel<2, 1, NE, WF>,
-                         expand_simt_kernel<4, 1, NE, WF>);
+    auto kern_inl = y_dtype == 0 ? pick(max_item_rows, expand_simt_kernel<1, kInlineItems, NE, WF, 0>,
+                                        expand_simt_kernel<2, kInlineItems, NE, WF, 0>,
+                                        expand_simt_kernel<4, kInlineItems, NE, WF, 0>)
+                                 : pick(max_item_rows, expand_simt_kernel<1, kInlineItems, NE, WF, 1>,
+                                        expand_simt_kernel<2, kInlineItems, NE, WF, 1>,
+                                        expand_simt_kernel<4, kInlineItems, NE, WF, 1>);
+    auto kern_tab = y_dtype == 0 ? pick(max_item_rows, expand_simt_kernel<1, 1, NE, WF, 0>,
+                                        expand_simt_kernel<2, 1, NE, WF, 0>, expand_simt_kernel<4, 1, NE, WF, 0>)
+                                 : pick(max_item_rows, expand_simt_kernel<1, 1, NE, WF, 1>,
+                                        expand_simt_kernel<2, 1, NE, WF, 1>, expand_simt_kernel<4, 1, NE, WF, 1>);
     const void* kp = inl ? reinterpret_cast<const void*>(kern_inl) : reinterpret_cast<const void*>(kern_tab);
     const int mr = std::max(8, max_rank);
     auto smem_for = [&](int npass) {  // v of the item, row scales, page ids, ring

@@ -365,7 +365,51 @@ def e2e_ours(sg, wl, pool, acts, args, device, stream, world):
         torch.cuda.synchronize(device)
         times.append(one())
     total = reduce_max(float(sum(times)), f"cuda:{device}")
-    return dict(total_ms=total, h2d=h2d, d2h=d2h)
+    return dict(total_ms=total, h2d=h2d, d2h=d2h, breakdown=e2e_breakdown(sg, wl, pool, host_x, host_y, stream, flush))
+
+
+def e2e_breakdown(sg, wl, pool, host_x, host_y, stream, flush, reps: int = 10):
+    """Where an end-to-end step's time goes: the same work as sgmv_lora_delta_host, issued
+    phase by phase through the binding with events between the phases (the stream idle
+    before each step): the host segment builder (host clock), the host-to-device copies
+    (table, distinct x, y), the kernels, and the copy of y back.  Median microseconds."""
+    n_proj = len(wl.projections)
+    dev_x = {s: torch.empty_like(h, device=f"cuda:{pool.device}") for s, h in host_x.items()}
+    dev_y = [torch.empty_like(h, device=f"cuda:{pool.device}") for h in host_y]
+    plan = sg.BatchPlan(pool, capacity_tokens=wl.T)
+    plan.build(wl.adapter_ids)
+    vs = [plan.new_v() for _ in range(n_proj)]
+    rows = {"build": [], "h2d": [], "kernels": [], "d2h": []}
+    for i in range(reps + 2):
+        flush.zero_()
+        torch.cuda.synchronize(pool.device)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        t0 = time.perf_counter()
+        plan.build(wl.adapter_ids)
+        t1 = time.perf_counter()
+        ev[0].record(stream)
+        plan.upload(stream)
+        for s_, h in host_x.items():
+            dev_x[s_].copy_(h, non_blocking=True)
+        for p in range(n_proj):
+            dev_y[p].copy_(host_y[p], non_blocking=True)
+        ev[1].record(stream)
+        if n_proj > 1:
+            sg.lora_delta_grouped([(dev_x[wl.x_of(p)], dev_y[p], p, vs[p]) for p in range(n_proj)], plan, pool,
+                                  wl.scale, stream)
+        else:
+            sg.lora_delta(dev_x[wl.x_of(0)], plan, pool, dev_y[0], 0, wl.scale, v=vs[0], stream=stream)
+        ev[2].record(stream)
+        for p in range(n_proj):
+            host_y[p].copy_(dev_y[p], non_blocking=True)
+        ev[3].record(stream)
+        ev[3].synchronize()
+        if i >= 2:
+            rows["build"].append((t1 - t0) * 1e6)
+            rows["h2d"].append(ev[0].elapsed_time(ev[1]) * 1e3)
+            rows["kernels"].append(ev[1].elapsed_time(ev[2]) * 1e3)
+            rows["d2h"].append(ev[2].elapsed_time(ev[3]) * 1e3)
+    return {k + "_us": round(float(statistics.median(v)), 1) for k, v in rows.items()}
 
 
 # ---------------------------------------------------------------------------- oracle arm
@@ -545,7 +589,7 @@ def main():
             "hbm_gbs_step": res["step_bytes"] / (res["total_ms"] / args.steps * 1e-3) / 1e9,
             "roofline": roofline_of(res),
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
-                    "d2h_bytes_per_step": e2e["d2h"]},
+                    "d2h_bytes_per_step": e2e["d2h"], "breakdown": e2e["breakdown"]},
             "gpu_launches": res["launches"] * args.steps,
             "clocks": res["clocks"],
         }

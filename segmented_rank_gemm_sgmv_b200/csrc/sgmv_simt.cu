@@ -734,7 +734,8 @@ __global__ void __launch_bounds__(kThreads, 4)
 // pushed to every CTA of the cluster (distributed shared memory); after the cluster barrier
 // each CTA sums the C tiles in a fixed order (the same bits as the two-kernel path) and
 // runs its share of the expand from shared memory.  The loops and their orders are those of
-// shrink_item and expand_item, so the result equals the two-kernel path's bit for bit.
+// shrink_item and expand_item: with the same cluster size the result equals the two-kernel
+// path's bit for bit.
 struct FusedArgs {
     const uint16_t* x;
     int64_t ldx;
@@ -1281,7 +1282,9 @@ cudaError_t expand_launch(const ExpandJob* jobs, int n_jobs, const BatchView& b,
 
 // The one-shot fused kernel for a single projection, when every item's cluster fits in
 // one wave and a CTA's slices fit in shared memory (*used = true); otherwise nothing is
-// launched.  The largest cluster size that fits is taken (the most CTAs loading at once).
+// launched.  The largest cluster size that fits is taken (the most CTAs loading at once,
+// and the least dependent work per thread): 16 CTAs, a non-portable cluster size that
+// sm_100 allows on request, when the device can hold every item's cluster at once.
 template <int WF>
 cudaError_t fused_launch(const ShrinkJob& sj, const ExpandJob& ej, const BatchView& b, int32_t num_items,
                          int32_t max_item_rows, int32_t max_rank, const PoolView& pool, float scale, int32_t y_dtype,
@@ -1302,8 +1305,8 @@ cudaError_t fused_launch(const ShrinkJob& sj, const ExpandJob& ej, const BatchVi
                                                   fused_simt_kernel<2, 1, WF>, fused_simt_kernel<4, 1, WF>));
     };
     const void* kern = kern_for(inl != nullptr);
-    for (int C = 8; C >= 1; --C) {
-        if ((pa % C) || (pb % C)) continue;
+    for (int C = 16; C >= 1; --C) {
+        if ((pa % C) || (pb % C) || (C > 8 && C != 16)) continue;
         const int kc = sj.d_in / C, ko = ej.d_out / C;
         FusedArgs a;
         std::memset(&a, 0, sizeof(a));
@@ -1328,8 +1331,30 @@ cudaError_t fused_launch(const ShrinkJob& sj, const ExpandJob& ej, const BatchVi
         o += (size_t)maxg * ko * esz;
         const size_t smem = al(o);
         if (smem > 227 * 1024) continue;
-        const int per_sm = resident_ctas(kern, smem);
-        if ((int64_t)num_items * C > (int64_t)per_sm * num_sms()) continue;  // one wave
+        cudaError_t e = raise_smem(kern, smem);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(num_items * C), 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (C > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+            cudaGetLastError();
+            continue;
+        }
+        int clusters = 0;  // every item's cluster resident at once: one wave
+        if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            continue;
+        }
+        if (clusters < num_items) continue;
         a.x = sj.x;
         a.ldx = sj.ldx;
         a.v = sj.v[0];
@@ -1347,20 +1372,6 @@ cudaError_t fused_launch(const ShrinkJob& sj, const ExpandJob& ej, const BatchVi
         a.max_rank = mr;
         a.y_dtype = y_dtype;
         a.scale = scale;
-        cudaError_t e = raise_smem(kern, smem);
-        if (e != cudaSuccess) return e;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)(num_items * C), 1, 1);
-        cfg.blockDim = dim3(kThreads, 1, 1);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = (unsigned)C;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
         *used = true;
         if (inl) {
             void* args[] = {&a, const_cast<InlineTable<kInlineItems>*>(inl)};

@@ -762,15 +762,18 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
         for (int u = u0 + grp; u < u1; u += 2) {
             const int i = u - u0, st = i % S, bsel = i & 1;
             const Unit w = unit(u);
-            wait(&accf_bar[bsel], (uint32_t)((i / 2) & 1));
-            wait(&full_bar[st], (uint32_t)((i / S) & 1));  // (completed: makes the staged y visible here)
-            tc_fence_after();
-            uint8_t* ys = yst + (size_t)st * y_bytes;
-            int t = -1;  // the row's token (the producer flags a bad one and leaves the row alone)
+            // the row's token and the tile's first token are loaded before the waits, so their
+            // latency is spent waiting for the accumulator rather than after it
+            int t = -1;  // (the producer flags a bad token and leaves the row alone)
             if (w.ok && m < w.rows) {
                 t = a.b.token_idx[w.row_begin + m];
                 if (t >= a.b.T) t = -1;
             }
+            const int t0 = w.ok ? a.b.token_idx[w.row_begin] : -1;
+            wait(&accf_bar[bsel], (uint32_t)((i / 2) & 1));
+            wait(&full_bar[st], (uint32_t)((i / S) & 1));  // (completed: makes the staged y visible here)
+            tc_fence_after();
+            uint8_t* ys = yst + (size_t)st * y_bytes;
             const bool row_ok = t >= 0 && !abort_flag;
             const float sc = a.scale * w.sc;  // the call's scale times the adapter's
             for (int c00 = 0; c00 < NB; c00 += 64) {
@@ -821,7 +824,6 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
             tok_row[grp][m] = t;
             // a full tile of consecutive tokens goes back by TMA (a partial one must not
             // touch the rows past it)
-            const int t0 = w.ok ? a.b.token_idx[w.row_begin] : -1;
             const bool full = named_bar_and(2 + grp, kTcTileRows, w.ok && w.rows == kTcTileRows && t0 >= 0 &&
                                                                       t == t0 + m && !abort_flag);
             if (full && a.use_tma) {

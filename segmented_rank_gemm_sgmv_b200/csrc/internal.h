@@ -126,10 +126,7 @@ static_assert(sizeof(PoolView) == 40, "PoolView must stay 40 bytes");
 struct SimtWork {
     int64_t sum_ng = 0;
     int32_t max_ng = 0;
-    const ItemRec* host_items = nullptr;  // the plan's host records [items][n_proj] (may be null)
-    int32_t n_proj = 0;
 };
-constexpr int kMaxRuns = 16;           // runs of items with equal row-group counts (<= 128 / 8)
 constexpr int kMaxShare = 4;           // projections that share one x in a SIMT shrink pass
 
 // One x of a SIMT shrink launch and the projections computed from it: nsub >= 1

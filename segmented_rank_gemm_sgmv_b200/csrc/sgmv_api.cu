@@ -108,8 +108,6 @@ SimtWork simt_work(const sgmv_plan* plan) {
     }
     const ItemRec* recs = reinterpret_cast<const ItemRec*>(static_cast<const uint8_t*>(plan->host_table) +
                                                            plan->off_simt_items);
-    w.host_items = recs;
-    w.n_proj = plan->n_proj;
     int32_t mx = 1;
     for (int32_t i = 0; i < n; ++i) {
         const int32_t ng = (std::max(recs[(int64_t)i * plan->n_proj].rank, 1) + 7) / 8;

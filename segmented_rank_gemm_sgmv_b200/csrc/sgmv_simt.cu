@@ -93,14 +93,7 @@ struct ShrinkArgs {
     int32_t max_rank;
     int32_t ring_offset; // byte offset of the stage ring in shared memory
     int32_t nsub_max;    // largest nsub of the launch (sizes the partial tiles and page ids)
-    // row_split: a CTA per (item, row group) over all of d_in -- one projection, no cluster,
-    // no reduction between CTAs.  Items come largest rank first, so their row-group counts
-    // form runs: run k = items [rg_item[k], ...) of rg_ng[k] row groups, CTAs from rg_cta[k]
-    int32_t row_split;
-    int32_t n_rg;
-    int32_t rg_item[kMaxRuns];
-    int32_t rg_ng[kMaxRuns];
-    int32_t rg_cta[kMaxRuns + 1];
+    int32_t pad;
 };
 
 struct ExpandEntry {
@@ -129,15 +122,6 @@ struct ExpandArgs {
     int32_t stages;
     int32_t max_rank;
     int32_t ring_offset;    // byte offset of the stage ring in shared memory
-    // by_rank (one entry): CTAs per item and passes per CTA by the item's row-group run, so a
-    // CTA streams about the same number of stages whatever its item's rank: run k = items
-    // [rg_item[k], ...) with rg_cpi[k] CTAs of rg_np[k] passes each, CTAs from rg_cta[k]
-    int32_t by_rank;
-    int32_t n_rg;
-    int32_t rg_item[kMaxRuns];
-    int32_t rg_cpi[kMaxRuns];
-    int32_t rg_np[kMaxRuns];
-    int32_t rg_cta[kMaxRuns + 1];
 };
 
 struct ItemInfo {
@@ -485,14 +469,7 @@ __global__ void __launch_bounds__(kThreads, 3)
     const int per_entry = a.items * C;  // a multiple of C: no cluster straddles two entries
     const int ei = NE == 1 ? 0 : (int)blockIdx.x / per_entry;
     const ShrinkEntry& en = a.ent[ei];
-    int item_idx = ((int)blockIdx.x - ei * per_entry) / C, g0 = 0;
-    if (NE == 1 && a.row_split) {  // this CTA's item and row group
-        int k = 0;
-        while (k + 1 < a.n_rg && (int)blockIdx.x >= a.rg_cta[k + 1]) ++k;
-        const int local = (int)blockIdx.x - a.rg_cta[k];
-        item_idx = a.rg_item[k] + local / a.rg_ng[k];
-        g0 = local - (local / a.rg_ng[k]) * a.rg_ng[k];
-    }
+    const int item_idx = ((int)blockIdx.x - ei * per_entry) / C;
     const uint32_t q = cluster_ctarank();
     const int nsub = NI > 1 ? 1 : en.nsub;                 // projections stacked over this x
     const int slot = kSimtMaxItemRows * a.max_rank * a.nsub_max;  // floats of one partial tile
@@ -509,21 +486,10 @@ __global__ void __launch_bounds__(kThreads, 3)
             a.b.simt_items + ((int64_t)item_idx * a.b.n_proj + en.proj[threadIdx.x]))[1];
         pt_sub[threadIdx.x] = (int64_t)(((uint64_t)(uint32_t)t.y << 32) | (uint32_t)t.x);
     }
-    ItemInfo m = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 0)
-                        : load_item(a.b, en.proj[0], item_idx, MAXG, a.max_rank, 0);
+    const ItemInfo m = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 0)
+                              : load_item(a.b, en.proj[0], item_idx, MAXG, a.max_rank, 0);
+    if (NI > 1 && threadIdx.x == 0) pt_sub[0] = m.pt;
     if (!m.ok && threadIdx.x == 0) atomicOr(&g_err_simt, kErrRows);
-    // row split: this CTA's rank rows [k_off, k_off + 8) of the item, as an item of their own
-    const int k_off = kRowGroup * g0;
-    if (NE == 1 && a.row_split && m.ok) {
-        if (k_off >= m.r) {
-            m.ok = false;
-            m.n = m.r = 0;
-        } else {
-            m.r = min(kRowGroup, m.r - k_off);
-            m.pt += (int64_t)k_off * (en.d_in >> a.pool.page_log2);
-        }
-    }
-    if ((NI > 1 || (NE == 1 && a.row_split)) && threadIdx.x == 0) pt_sub[0] = m.pt;
     StageGeom sg;
     sg.NGs = (m.r + kRowGroup - 1) / kRowGroup;
     sg.NG = nsub * sg.NGs;
@@ -588,8 +554,7 @@ __global__ void __launch_bounds__(kThreads, 3)
             const int jrow = e / RS, rem = e - jrow * RS;
             const int ps = rem / m.r, k = rem - ps * m.r;
             // a quantised row's scale leaves the sum: v_k = s_k * sum_c q_kc x_c
-            en.v[ps][(int64_t)(m.i0 + jrow) * en.ldv[ps] + k_off + k] =
-                WF == kFmtBf16 ? s : s * rsc[ps * kMaxRank + k];
+            en.v[ps][(int64_t)(m.i0 + jrow) * en.ldv[ps] + k] = WF == kFmtBf16 ? s : s * rsc[ps * kMaxRank + k];
         }
     }
 }
@@ -719,27 +684,19 @@ __global__ void __launch_bounds__(kThreads, 4)
     if (NE > 1)
         while (ei + 1 < a.n_entries && (int)blockIdx.x >= a.ent[ei + 1].cta_base) ++ei;
     const ExpandEntry& en = a.ent[ei];
-    int local = (int)blockIdx.x - en.cta_base;
-    int part_idx = local % en.cpi, item_idx = local / en.cpi, npass = en.npass;
-    if (NE == 1 && a.by_rank) {  // this CTA's item, part and passes by its item's run
-        int k = 0;
-        while (k + 1 < a.n_rg && (int)blockIdx.x >= a.rg_cta[k + 1]) ++k;
-        local = (int)blockIdx.x - a.rg_cta[k];
-        item_idx = a.rg_item[k] + local / a.rg_cpi[k];
-        part_idx = local - (local / a.rg_cpi[k]) * a.rg_cpi[k];
-        npass = a.rg_np[k];
-    }
+    const int local = (int)blockIdx.x - en.cta_base;
+    const int part_idx = local % en.cpi, item_idx = local / en.cpi;
     float* vs = reinterpret_cast<float*>(smem_e);
     float* rsc = vs + kSimtMaxItemRows * a.max_rank;  // [kMaxRank] row scales (quantised pools only)
     int32_t* pid = reinterpret_cast<int32_t*>(rsc + (WF == kFmtBf16 ? 0 : kMaxRank));
 
     const ItemInfo m = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 1)
                               : load_item(a.b, en.proj, item_idx, MAXG, a.max_rank, 1);
-    const int j0 = part_idx * npass * kPass;
+    const int j0 = part_idx * en.npass * kPass;
     StageGeom sg;
     sg.NG = (m.r + kRowGroup - 1) / kRowGroup;
     sg.NGs = sg.NG;
-    sg.span = min(npass * kPass, en.d_out - j0);
+    sg.span = min(en.npass * kPass, en.d_out - j0);
     sg.npass = (sg.span + kPass - 1) / kPass;
     sg.col_base = j0;
     sg.rank = m.r;
@@ -1107,30 +1064,6 @@ double split_time(const SimtWork& work, int64_t items, int64_t cpi, int npass, d
     return std::max(biggest, total / (double)slots);
 }
 
-// Runs of consecutive SIMT items with equal row-group counts (items come largest rank
-// first, so there are at most kMaxRuns): first item and row groups of each; false when the
-// plan's items are not on the host.
-struct Runs {
-    int n = 0;
-    int32_t item[kMaxRuns], ng[kMaxRuns], count[kMaxRuns];
-};
-bool item_runs(const SimtWork& work, int32_t num_items, Runs* runs) {
-    runs->n = 0;
-    if (!work.host_items || num_items <= 0) return false;
-    for (int32_t i = 0; i < num_items; ++i) {
-        const int ng = (std::max(work.host_items[(int64_t)i * work.n_proj].rank, 1) + kRowGroup - 1) / kRowGroup;
-        if (runs->n == 0 || runs->ng[runs->n - 1] != ng) {
-            if (runs->n == kMaxRuns) return false;
-            runs->item[runs->n] = i;
-            runs->ng[runs->n] = ng;
-            runs->count[runs->n] = 0;
-            ++runs->n;
-        }
-        ++runs->count[runs->n - 1];
-    }
-    return true;
-}
-
 template <typename K1, typename K2, typename K4>
 auto pick(int max_item_rows, K1 k1, K2 k2, K4 k4) {
     return max_item_rows <= 1 ? k1 : max_item_rows <= 2 ? k2 : k4;
@@ -1205,16 +1138,7 @@ cudaError_t shrink_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b,
         if (C == 0 && ctas >= 2 * (int64_t)resident_ctas(kp, smem_for(c)) * num_sms()) C = c;
     }
     if (C == 0) C = C_max;
-    // One projection with at least a full wave of row groups: a CTA per (item, row group)
-    // over all of d_in instead -- every CTA streams the same number of stages whatever its
-    // item's rank, and no reduction crosses CTAs.
-    Runs runs;
-    bool row_split = false;
-    if (n_jobs == 1 && jobs[0].nsub == 1 && !inl && item_runs(work, num_items, &runs) &&
-        work.sum_ng >= (int64_t)resident_ctas(kp, smem_for(1)) * num_sms()) {
-        row_split = true;
-        C = 1;
-    }
+    (void)work;
     ShrinkArgs<NE> a;
     std::memset(&a, 0, sizeof(a));
     for (int i = 0; i < n_jobs; ++i) {
@@ -1240,24 +1164,10 @@ cudaError_t shrink_launch(const ShrinkJob* jobs, int n_jobs, const BatchView& b,
     a.max_rank = mr;
     a.nsub_max = nsub_max;
     a.stages = stages;
-    unsigned grid = (unsigned)(n_jobs * C * num_items);
-    if (row_split) {
-        a.row_split = 1;
-        a.n_rg = runs.n;
-        int cta = 0;
-        for (int k = 0; k < runs.n; ++k) {
-            a.rg_item[k] = runs.item[k];
-            a.rg_ng[k] = runs.ng[k];
-            a.rg_cta[k] = cta;
-            cta += runs.count[k] * runs.ng[k];
-        }
-        a.rg_cta[runs.n] = cta;
-        grid = (unsigned)cta;
-    }
     const size_t smem = smem_for(C);
     a.ring_offset = (int)(smem - ring_bytes);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.gridDim = dim3((unsigned)(n_jobs * C * num_items), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -1329,33 +1239,10 @@ cudaError_t expand_launch(const ExpandJob* jobs, int n_jobs, const BatchView& b,
             best_p = P;
         }
     }
-    // One entry over items of several ranks: passes per CTA by the item's run, about
-    // kExpandStagesPerCta stages a CTA (a rank-64 item's CTAs take one 1024-column pass,
-    // a rank-8 item's eight), instead of one pass count for every item.
-    Runs runs;
-    const bool by_rank = n_jobs == 1 && !inl && item_runs(work, num_items, &runs) && runs.n > 1;
     ExpandArgs<NE> a;
     std::memset(&a, 0, sizeof(a));
     int ctas = 0, max_np = 1;
-    if (by_rank) {
-        constexpr int kExpandStagesPerCta = 8;
-        a.by_rank = 1;
-        a.n_rg = runs.n;
-        for (int k = 0; k < runs.n; ++k) {
-            const int np = std::max(1, std::min(tiles[0], kExpandStagesPerCta / runs.ng[k]));
-            const int cpi = (tiles[0] + np - 1) / np;
-            a.rg_item[k] = runs.item[k];
-            a.rg_np[k] = np;
-            a.rg_cpi[k] = cpi;
-            a.rg_cta[k] = ctas;
-            ctas += runs.count[k] * cpi;
-            max_np = std::max(max_np, np);
-        }
-        a.rg_cta[runs.n] = ctas;
-        const ExpandJob& j = jobs[order[0]];
-        a.ent[0] = ExpandEntry{j.v, j.ldv, j.y, j.ldy, j.d_out, max_np, 1, 0, j.proj, {0, 0, 0}};
-    }
-    for (int i = 0; i < n_jobs && !by_rank; ++i) {
+    for (int i = 0; i < n_jobs; ++i) {
         const ExpandJob& j = jobs[order[i]];
         const int np = std::min(best_p, tiles[i]), cpi = (tiles[i] + np - 1) / np;
         a.ent[i] = ExpandEntry{j.v, j.ldv, j.y, j.ldy, j.d_out, np, cpi, ctas, j.proj, {0, 0, 0}};

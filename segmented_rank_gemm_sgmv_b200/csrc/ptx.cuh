@@ -1,8 +1,10 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, bulk async copies (no
-// multicast), thread-block-cluster shared memory, cp.async, and the tcgen05
-// tensor-core / tensor-memory instructions.  Every wait here is bounded.
+// multicast), thread-block-cluster shared memory, cp.async, the tcgen05
+// tensor-core / tensor-memory instructions, and the warp-level ldmatrix / mma.sync
+// pair the SIMT kernels use for their small contractions.  Every wait here is bounded.
 #pragma once
 #include <cstdint>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 namespace sgmv {
@@ -346,6 +348,39 @@ __device__ __forceinline__ void int4x8_to_f32_pos(uint32_t q, float (&f)[8]) {
 // 16^-(i % 4): the factor that int4x8_to_f32_pos leaves on value i
 __device__ __forceinline__ float int4_pos_unscale(int i) {
     return i % 4 == 0 ? 1.0f : i % 4 == 1 ? 0.0625f : i % 4 == 2 ? 0.00390625f : 0.000244140625f;
+}
+
+// ------------------------------------------------------------------ warp-level mma
+// ldmatrix: lanes 8i..8i+7 give the row addresses (16 bytes each) of 8x8 matrix i;
+// lane l receives, of every matrix, the pair (row l/4, columns 2(l%4), 2(l%4)+1), or with
+// .trans the pair (rows 2(l%4), 2(l%4)+1, column l/4).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t (&r)[2]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
+}
+// D(16x8, fp32) += A(16x16, bf16, row-major fragment) x B(16x8, bf16, column fragment).
+// Fragments, with g = lane / 4 and t = lane % 4: a = {A[g][2t..], A[g+8][2t..], A[g][2t+8..],
+// A[g+8][2t+8..]}, b = {B[2t..][g], B[2t+8..][g]}, d = {D[g][2t], D[g][2t+1], D[g+8][2t],
+// D[g+8][2t+1]}; each 32-bit register holds two bf16, the lower index in the low half.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Two fp32 to a bf16 pair (round to nearest even), lo in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+           ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
 }
 
 // Eight stored weights of format WF at p (16, 8 or 4 bytes) to fp32.

@@ -732,10 +732,23 @@ __global__ void __launch_bounds__(kThreads, 4)
 // copies at once -- A rows and x slices as one commit group, B^T rows and y rows as a second
 // -- so the whole call pays one DRAM round trip for its data.  The shrink's partial tile is
 // pushed to every CTA of the cluster (distributed shared memory); after the cluster barrier
-// each CTA sums the C tiles in a fixed order (the same bits as the two-kernel path) and
-// runs its share of the expand from shared memory.  The loops and their orders are those of
-// shrink_item and expand_item: with the same cluster size the result equals the two-kernel
-// path's bit for bit.
+// each CTA sums the C tiles in a fixed order and runs its share of the expand from shared
+// memory.
+//
+// bf16 pools run eight warps a CTA:
+//   shrink: warp-level bf16 mma (m16n8k16, fp32 accumulation): M = rank rows (16 a tile), N =
+//           tokens (8: the item's <= 4 and padding), K = 16 columns of d_in; warp w takes K
+//           steps w, w + 8, ... with two accumulator sets, and the eight warp tiles are summed
+//           in warp order.  A and x are staged with their 16-byte granules XOR-swizzled by row
+//           (granule c of row k at c ^ (k % 8)), so the ldmatrix row reads are conflict-free.
+//           Three instructions per 16 x 16 block of A replace some thirty FMA, conversion and
+//           shared-memory instructions: the phase is latency-bound, and this shortens it.
+//   expand: thread t owns 4 columns of the slice and runs over every rank row with FMA; v is
+//           kept transposed, [rank row][4 tokens], so one 16-byte load gives the row's weights
+//           for every token of the item.  (An mma expand, with v split into bf16 hi + lo, was
+//           measured twice as slow: each tile needs two dependent mma, and the legacy warp-level
+//           mma's latency dominates a phase this short.)
+// Quantised pools keep four warps and the loops of the two-kernel path.
 struct FusedArgs {
     const uint16_t* x;
     int64_t ldx;
@@ -753,15 +766,54 @@ struct FusedArgs {
     int32_t y_dtype;
     float scale;
     // byte offsets in shared memory
-    int32_t off_part, off_vs, off_rsc, off_pid_a, off_pid_b, off_a, off_x, off_b, off_y;
+    int32_t off_part, off_vs, off_rsc, off_pid_a, off_pid_b, off_a, off_x, off_b, off_y, off_wp;
 };
 
+// The cells of a rows x cols grid that thread `start` visits with stride `stride` in
+// row-major order: (k, c), advanced without a division per step.
+struct GridWalk {
+    int k, c, dk, dc, cols;
+    __device__ __forceinline__ GridWalk(int cols_, int start, int stride) : cols(cols_) {
+        k = start / cols;
+        c = start - k * cols;
+        dk = stride / cols;
+        dc = stride - dk * cols;
+    }
+    __device__ __forceinline__ void next() {
+        k += dk;
+        c += dc;
+        if (c >= cols) {
+            c -= cols;
+            ++k;
+        }
+    }
+};
+
+// Token row j of an item (j a run-time value): selected from the registers, no local memory.
+__device__ __forceinline__ int tok_at(const ItemInfo& m, int j) {
+    int t = -1;
+#pragma unroll
+    for (int i = 0; i < kSimtMaxItemRows; ++i)
+        if (j == i) t = m.tok[i];
+    return t;
+}
+
+// Threads of the fused kernel: eight warps for bf16 pools (two a scheduler), four for the
+// loops of quantised pools.
+template <int WF>
+__host__ __device__ constexpr int fused_threads() { return WF == kFmtBf16 ? 2 * kThreads : kThreads; }
+constexpr int kFusedWideMaxRank = 64;  // bf16 pools: ranks up to 64 (four 16-row tiles) take the fused kernel
+
 template <int MAXG, int NI, int WF>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(fused_threads<WF>(), 1)
     fused_simt_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ InlineTable<NI> inl) {
     extern __shared__ __align__(128) uint8_t smem_f[];
     constexpr int VB = bytes_per_8<WF>();
-    const int tid = threadIdx.x, col = kVec * tid;
+    constexpr bool kWide = WF == kFmtBf16;
+    constexpr int TPB = fused_threads<WF>();
+    constexpr int kWarps = TPB / 32;
+    constexpr int kMT = kFusedWideMaxRank / 16;  // 16-row tiles of the largest rank
+    const int tid = threadIdx.x, col = kVec * tid, lane = tid & 31, warp = tid >> 5;
     const int C = a.cluster;
     // every CTA of the cluster is running before any pushes into another's shared memory
     if (C > 1) cluster_arrive_relaxed();
@@ -769,7 +821,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t q = cluster_ctarank();
     float* red = reinterpret_cast<float*>(smem_f);                       // [4 warps][64]
     float* part = reinterpret_cast<float*>(smem_f + a.off_part);         // [C][4 x max_rank]
-    float* vs = reinterpret_cast<float*>(smem_f + a.off_vs);             // [4 x max_rank]
+    float* vs = reinterpret_cast<float*>(smem_f + a.off_vs);             // [4 x max_rank] (bf16: [max_rank][4])
     float* rsc_a = reinterpret_cast<float*>(smem_f + a.off_rsc);         // [kMaxRank] (quantised)
     float* rsc_b = rsc_a + kMaxRank;
     int32_t* pid_a = reinterpret_cast<int32_t*>(smem_f + a.off_pid_a);  // [r][kc / P]
@@ -778,6 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint16_t* xs = reinterpret_cast<uint16_t*>(smem_f + a.off_x);        // [MAXG][kc]
     uint8_t* Bs = smem_f + a.off_b;                                      // [r][ko] weights
     uint8_t* ys = smem_f + a.off_y;                                      // [MAXG][ko] of y's type
+    float* wpart = reinterpret_cast<float*>(smem_f + a.off_wp);          // [warps][MAXG][max_rank] (bf16)
     const int slot = kSimtMaxItemRows * a.max_rank;
 
     ItemInfo ma = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 0)
@@ -793,7 +846,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // page ids of both slices (one round of independent loads), row scales of quantised pools
     if (ma.ok) {
-        for (int i = tid; i < r * (cpa + cpb); i += kThreads) {
+        for (int i = tid; i < r * (cpa + cpb); i += TPB) {
             const bool isa = i < r * cpa;
             const int ii = isa ? i : i - r * cpa, cp = isa ? cpa : cpb;
             const int k = ii / cp, pc = ii - k * cp;
@@ -814,50 +867,116 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
 
     // every copy at once: group 1 = A rows + x slices, group 2 = B^T rows + y rows
+    // (bf16: granule c of an A or x row k lands at granule c ^ (k % 8) of the row)
     const uint8_t* pages = reinterpret_cast<const uint8_t*>(a.pool.pages);
     const int page_shift = P_log2 + (VB == 16 ? 1 : VB == 8 ? 0 : -1);
     constexpr int kVals16 = 128 / VB;  // values per 16-byte granule
+    const int gx = a.kc / 8;           // 16-byte granules of an x row slice
     if (ma.ok) {
         const int gpr_a = a.kc / kVals16;
-        for (int gi = tid; gi < r * gpr_a; gi += kThreads) {
-            const int k = gi / gpr_a, cg = gi - k * gpr_a, cl = cg * kVals16;
-            cp_async16(As + (size_t)k * (a.kc / 8 * VB) + cg * 16,
-                       pages + ((int64_t)pid_a[k * cpa + (cl >> P_log2)] << page_shift) + (cl & (P - 1)) / 8 * VB,
+        for (GridWalk w(gpr_a, tid, TPB); w.k < r; w.next()) {
+            const int cl = w.c * kVals16;
+            cp_async16(As + (size_t)w.k * (a.kc / 8 * VB) + (kWide ? (w.c ^ (w.k & 7)) : w.c) * 16,
+                       pages + ((int64_t)pid_a[w.k * cpa + (cl >> P_log2)] << page_shift) + (cl & (P - 1)) / 8 * VB,
                        true);
         }
-        for (int gi = tid; gi < MAXG * (a.kc / 8); gi += kThreads) {
-            const int j = gi / (a.kc / 8), cg = gi - j * (a.kc / 8);
+#pragma unroll
+        for (int j = 0; j < MAXG; ++j) {
             const int t = ma.tok[j];
-            cp_async16(xs + (size_t)j * a.kc + cg * 8,
-                       t >= 0 ? a.x + (int64_t)t * a.ldx + ca0 + cg * 8 : a.x, t >= 0);
+            for (int cg = tid; cg < gx; cg += TPB)
+                cp_async16(xs + (size_t)j * a.kc + (kWide ? (cg ^ (j & 7)) : cg) * 8,
+                           t >= 0 ? a.x + (int64_t)t * a.ldx + ca0 + cg * 8 : a.x, t >= 0);
         }
     }
     cp_async_commit();
     const int esz = a.y_dtype == 0 ? 2 : 4;
     if (ma.ok) {
         const int gpr_b = a.ko / kVals16;
-        for (int gi = tid; gi < r * gpr_b; gi += kThreads) {
-            const int k = gi / gpr_b, cg = gi - k * gpr_b, cl = cg * kVals16;
-            cp_async16(Bs + (size_t)k * (a.ko / 8 * VB) + cg * 16,
-                       pages + ((int64_t)pid_b[k * cpb + (cl >> P_log2)] << page_shift) + (cl & (P - 1)) / 8 * VB,
+        for (GridWalk w(gpr_b, tid, TPB); w.k < r; w.next()) {
+            const int cl = w.c * kVals16;
+            cp_async16(Bs + (size_t)w.k * (a.ko / 8 * VB) + w.c * 16,
+                       pages + ((int64_t)pid_b[w.k * cpb + (cl >> P_log2)] << page_shift) + (cl & (P - 1)) / 8 * VB,
                        true);
         }
         const int gy = a.ko * esz / 16;  // granules of one y row slice
-        for (int gi = tid; gi < MAXG * gy; gi += kThreads) {
-            const int j = gi / gy, cg = gi - j * gy;
+        const uint8_t* src = static_cast<const uint8_t*>(a.y);
+#pragma unroll
+        for (int j = 0; j < MAXG; ++j) {
             const int t = mb.tok[j];
-            const uint8_t* src = static_cast<const uint8_t*>(a.y);
-            cp_async16(ys + (size_t)j * a.ko * esz + cg * 16,
-                       t >= 0 ? src + ((int64_t)t * a.ldy + cb0) * esz + cg * 16 : src, t >= 0);
+            for (int cg = tid; cg < gy; cg += TPB)
+                cp_async16(ys + (size_t)j * a.ko * esz + cg * 16,
+                           t >= 0 ? src + ((int64_t)t * a.ldy + cb0) * esz + cg * 16 : src, t >= 0);
         }
     }
     cp_async_commit();
 
-    // ---- shrink over this CTA's d_in slice: row groups outer, 1024-column passes inner
+    // ---- shrink over this CTA's d_in slice
     cp_async_wait<1>();
     __syncthreads();
     float* mine = part + (size_t)q * slot;  // this CTA's partial tile [token][rank row]
-    if (ma.ok) {
+    if constexpr (kWide) {
+        if (ma.ok) {
+            const int MT = (r + 15) >> 4, ksteps = a.kc >> 4;
+            // two accumulator sets (K steps ks and ks + warps) keep two mma chains in flight
+            float d[kMT][4], d1[kMT][4];
+#pragma unroll
+            for (int mt = 0; mt < kMT; ++mt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) d[mt][i] = d1[mt][i] = 0.f;
+            // lane addresses: x rows are the tokens (padding lanes read row 0; their columns of
+            // D are not used), A rows the rank rows of each tile (rows past r read row 0)
+            const int mi = lane >> 3;
+            const int xrow = (lane & 7) < MAXG ? (lane & 7) : 0;
+            const uint32_t xbase = smem_u32(xs) + (uint32_t)(xrow * a.kc * 2);
+            uint32_t arow[kMT];
+            int asw[kMT];
+#pragma unroll
+            for (int mt = 0; mt < kMT; ++mt) {
+                int row = mt * 16 + ((mi & 1) << 3) + (lane & 7);
+                row = row < r ? row : 0;
+                arow[mt] = smem_u32(As) + (uint32_t)(row * a.kc * 2);
+                asw[mt] = row & 7;
+            }
+            for (int ks = warp; ks < ksteps; ks += 2 * kWarps) {
+                const int ks1 = ks + kWarps;
+                const bool two = ks1 < ksteps;
+                uint32_t xb[2], xb1[2];
+                ldsm_x2(xbase + ((((ks << 1) | (mi & 1)) ^ (xrow & 7)) << 4), xb);
+                if (two) ldsm_x2(xbase + ((((ks1 << 1) | (mi & 1)) ^ (xrow & 7)) << 4), xb1);
+#pragma unroll
+                for (int mt = 0; mt < kMT; ++mt) {
+                    if (mt < MT) {
+                        uint32_t af[4], af1[4];
+                        ldsm_x4(arow[mt] + ((((ks << 1) | (mi >> 1)) ^ asw[mt]) << 4), af);
+                        if (two) ldsm_x4(arow[mt] + ((((ks1 << 1) | (mi >> 1)) ^ asw[mt]) << 4), af1);
+                        mma_bf16_16816(d[mt], af, xb[0], xb[1]);
+                        if (two) mma_bf16_16816(d1[mt], af1, xb1[0], xb1[1]);
+                    }
+                }
+            }
+            // warp tiles: d[mt] = {(row 16mt + g, tokens 2t, 2t+1), (row 16mt + g + 8, same tokens)}
+            const int g = lane >> 2, t2 = 2 * (lane & 3);
+#pragma unroll
+            for (int mt = 0; mt < kMT; ++mt) {
+                if (mt < MT) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int k = mt * 16 + g + ((i >> 1) << 3), j = t2 + (i & 1);
+                        if (j < MAXG && k < r) wpart[(warp * MAXG + j) * a.max_rank + k] = d[mt][i] + d1[mt][i];
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        if (ma.ok)
+            for (int e = tid; e < n * r; e += TPB) {
+                const int j = e / r, k = e - j * r;
+                float sum = 0.f;
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) sum += wpart[(w * MAXG + j) * a.max_rank + k];
+                mine[e] = sum;
+            }
+    } else if (ma.ok) {  // rank row groups outer, 1024-column passes inner
         const int NG = (r + kRowGroup - 1) / kRowGroup, npass = (a.kc + kPass - 1) / kPass;
         for (int g = 0; g < NG; ++g) {
             float p[kRowGroup * MAXG];
@@ -906,27 +1025,67 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int qq = 0; qq < C; ++qq) {
             if (qq == (int)q) continue;
             const uint32_t dst = map_cluster(smem_u32(mine), (uint32_t)qq);
-            for (int e = tid; e < E; e += kThreads) st_cluster_f32(dst + 4u * (uint32_t)e, mine[e]);
+            for (int e = tid; e < E; e += TPB) st_cluster_f32(dst + 4u * (uint32_t)e, mine[e]);
         }
         cluster_arrive_release();
         cluster_wait_acquire();
     }
     if (ma.ok) {
-        for (int e = tid; e < E; e += kThreads) {
+        for (int e = tid; e < E; e += TPB) {
             float s = 0.f;
             for (int qq = 0; qq < C; ++qq) s += part[(size_t)qq * slot + e];
             const int k = e - (e / r) * r;
             const float vk = WF == kFmtBf16 ? s : s * rsc_a[k];
             if (q == 0) a.v[(int64_t)(ma.i0 + e / r) * a.ldv + k] = vk;
-            vs[e] = WF == kFmtBf16 ? vk : vk * rsc_b[k];  // a quantised B^T row's scale goes onto v_k
+            if (kWide) vs[k * 4 + e / r] = vk;                // [rank row][token]
+            else vs[e] = WF == kFmtBf16 ? vk : vk * rsc_b[k];  // a quantised B^T row's scale goes onto v_k
         }
     }
     cp_async_wait<0>();
     __syncthreads();  // vs, and the B^T and y slices, are visible to every thread
 
-    // ---- expand over this CTA's d_out slice: 1024-column passes, each over every rank row
+    // ---- expand over this CTA's d_out slice
     if (!mb.ok) return;
     const float sc = a.scale * mb.sc;  // the call's scale times the adapter's
+    if constexpr (kWide) {
+        for (int c4 = tid; c4 < (a.ko >> 2); c4 += TPB) {  // 4 columns of the slice a thread
+            float acc[MAXG][4];
+#pragma unroll
+            for (int j = 0; j < MAXG; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+            const uint8_t* bp = Bs + (size_t)c4 * 8;
+#pragma unroll 4
+            for (int k = 0; k < r; ++k) {
+                const uint2 bw = *reinterpret_cast<const uint2*>(bp + (size_t)k * a.ko * 2);
+                const float b4[4] = {bf16lo(bw.x), bf16hi(bw.x), bf16lo(bw.y), bf16hi(bw.y)};
+                const float4 w = *reinterpret_cast<const float4*>(vs + k * 4);
+                const float wj[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int j = 0; j < MAXG; ++j)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[j][e] = fmaf(wj[j], b4[e], acc[j][e]);
+            }
+            const int jcol = cb0 + 4 * c4;
+#pragma unroll
+            for (int j = 0; j < MAXG; ++j) {
+                const int t = mb.tok[j];
+                if (j >= n || t < 0) continue;
+                if (a.y_dtype == 0) {
+                    const uint2 yv = *reinterpret_cast<const uint2*>(ys + ((size_t)j * a.ko + 4 * c4) * 2);
+                    *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.y) + (int64_t)t * a.ldy + jcol) =
+                        make_uint2(pack_bf16x2(fmaf(sc, acc[j][0], bf16lo(yv.x)), fmaf(sc, acc[j][1], bf16hi(yv.x))),
+                                   pack_bf16x2(fmaf(sc, acc[j][2], bf16lo(yv.y)), fmaf(sc, acc[j][3], bf16hi(yv.y))));
+                } else {
+                    float4 o = *reinterpret_cast<const float4*>(ys + ((size_t)j * a.ko + 4 * c4) * 4);
+                    o.x = fmaf(sc, acc[j][0], o.x); o.y = fmaf(sc, acc[j][1], o.y);
+                    o.z = fmaf(sc, acc[j][2], o.z); o.w = fmaf(sc, acc[j][3], o.w);
+                    *reinterpret_cast<float4*>(static_cast<float*>(a.y) + (int64_t)t * a.ldy + jcol) = o;
+                }
+            }
+        }
+        return;
+    }
     const int NG = (r + kRowGroup - 1) / kRowGroup, npass = (a.ko + kPass - 1) / kPass;
     for (int s = 0; s < npass; ++s) {
         const int c = s * kPass, W = min(kPass, a.ko - c);
@@ -1291,6 +1450,7 @@ cudaError_t fused_launch(const ShrinkJob& sj, const ExpandJob& ej, const BatchVi
                          const InlineTable<kInlineItems>* inl, cudaStream_t stream, bool* used) {
     *used = false;
     if (num_items <= 0 || sj.nsub != 1 || sj.d_in <= 0 || ej.d_out <= 0) return cudaSuccess;
+    if (WF == kFmtBf16 && max_rank > kFusedWideMaxRank) return cudaSuccess;
     const int maxg = max_item_rows <= 1 ? 1 : max_item_rows <= 2 ? 2 : 4;
     const int mr = std::max(8, max_rank);
     const int esz = y_dtype == 0 ? 2 : 4;
@@ -1329,13 +1489,15 @@ cudaError_t fused_launch(const ShrinkJob& sj, const ExpandJob& ej, const BatchVi
         o += (size_t)mr * ko / 8 * bytes_per_8<WF>();
         a.off_y = (int32_t)(o = al(o));
         o += (size_t)maxg * ko * esz;
+        a.off_wp = (int32_t)(o = al(o));
+        o += WF == kFmtBf16 ? (size_t)(fused_threads<WF>() / 32) * maxg * mr * 4 : 0;
         const size_t smem = al(o);
         if (smem > 227 * 1024) continue;
         cudaError_t e = raise_smem(kern, smem);
         if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)(num_items * C), 1, 1);
-        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.blockDim = dim3(fused_threads<WF>(), 1, 1);
         cfg.dynamicSmemBytes = smem;
         cfg.stream = stream;
         cudaLaunchAttribute attr[1];

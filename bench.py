@@ -316,14 +316,27 @@ def run_ours(args, rank, world, device, with_e2e=True):
         expand_b += e_b
         flops += f
     peak, peak_kind = measured_peaks()
-    plan0 = plans[0].plan
-    simt, tc = plan0.num_simt_items > 0, plan0.num_tc_tiles > 0
-    kinds = [k for k, on in (("simt", simt), ("tc", tc)) if on]
-    names = " + ".join(f"shrink_{k}_kernel" for k in kinds) + " + " + " + ".join(f"expand_{k}_kernel" for k in kinds)
+    # the kernels the calls launch, as the library reports them (sgmv_lora_delta_kernels)
+    y_dt = acts[0][1].dtype
+    if split:                                        # separate shrink and expand calls
+        plan0 = plans[0].plan
+        mask = (sg.KERNELS_SIMT if plan0.num_simt_items > 0 else 0) | (sg.KERNELS_TC if plan0.num_tc_tiles > 0 else 0)
+        launches = 2 * n_proj * bin(mask).count("1")
+    elif grouped:
+        mask, launches = sg.lora_delta_kernels(plans[0], pool, list(range(n_proj)), y_dt, stream)
+    else:
+        mask = launches = 0
+        for p in range(n_proj):
+            k, n_l = sg.lora_delta_kernels(plans[0], pool, [p], y_dt, stream)
+            mask |= k
+            launches += n_l
+    names = " + ".join(n for bit, n in ((sg.KERNELS_FUSED, "fused_simt_kernel"),
+                                        (sg.KERNELS_SIMT, "shrink_simt_kernel + expand_simt_kernel"),
+                                        (sg.KERNELS_TC, "shrink_tc_kernel + expand_tc_kernel")) if mask & bit)
     api = "sgmv_lora_delta_grouped" if grouped else "sgmv_lora_delta"
     res = dict(total_ms=total_ms, proj_ms=float(np.mean(proj_ms)), kernel_name=f"{api} ({names})",
                step_bytes=shrink_b + expand_b, flops=flops, peak=peak, peak_kind=peak_kind,
-               launches=(2 * simt + 2 * n_proj * tc) if grouped else 2 * n_proj * len(kinds),
+               launches=launches,
                clocks=clk.summary(), dom_launches=1 if grouped else n_proj,
                traffic=read_traffic(args.workload, ("lora_delta_grouped" if grouped else "lora_delta") +
                                     ("" if args.weights == "bf16" else "@" + args.weights)), split=split)
@@ -525,7 +538,8 @@ def roofline_of(res) -> dict:
             "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if res["peak_kind"] == "measured"
             else "fallback 6650 GB/s",
             "algorithmic_bytes_per_step": res["step_bytes"],
-            "launches_per_step": res["dom_launches"],
+            "calls_per_step": res["dom_launches"],
+            "launches_per_step": res["launches"],
             "traffic": res["traffic"]}
 
 

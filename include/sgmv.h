@@ -472,6 +472,32 @@ SGMV_API sgmv_status sgmv_lora_delta_grouped(const sgmv_delta_entry* entries, in
                                              float scale, int32_t y_dtype, sgmv_stream_t stream);
 
 /*
+ * Which kernels sgmv_lora_delta (n_entries = 1) or sgmv_lora_delta_grouped (the
+ * entries' projections `projs`, with the same `table`, NULL or not) launch for
+ * this plan and pool, without launching anything.  The calls' own choices are
+ * made, including the test of the one-shot fused kernel (every SIMT item's
+ * cluster resident in one wave: an occupancy query on the pool's device, which
+ * becomes the calling thread's current device).
+ *
+ * kinds     out: a mask of SGMV_KERNELS_FUSED (the one-shot fused SIMT kernel),
+ *           SGMV_KERNELS_SIMT (the SIMT shrink and expand pair) and
+ *           SGMV_KERNELS_TC (the tensor-core shrink and expand of long segments);
+ *           0 when the plan has no work.
+ * launches  out: kernel launches the call makes.
+ * Errors: SGMV_ERR_INVALID (null pointers, a pool without device memory,
+ * n_entries outside 1..8, a projection outside the pool, y_dtype not 0 or 1, a
+ * plan built for another pool), SGMV_ERR_CUDA.
+ */
+enum {
+    SGMV_KERNELS_FUSED = 1,
+    SGMV_KERNELS_SIMT = 2,
+    SGMV_KERNELS_TC = 4,
+};
+SGMV_API sgmv_status sgmv_lora_delta_kernels(const sgmv_plan* plan, const sgmv_pool* pool, const int32_t* projs,
+                                             int32_t n_entries, const void* table, int32_t y_dtype,
+                                             int32_t* kinds, int32_t* launches);
+
+/*
  * The whole step from host buffers: the segment builder, the host-to-device
  * copies of the step's inputs, the grouped delta and the device-to-host copy
  * of the results, enqueued on `stream` by the library (no Python or other

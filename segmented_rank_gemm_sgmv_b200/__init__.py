@@ -35,7 +35,7 @@ EXPORTED = ("sgmv_status_string", "sgmv_last_error", "sgmv_pool_create", "sgmv_p
             "sgmv_pool_set_adapter_scale", "sgmv_pool_get_adapter_scale",
             "sgmv_pool_shuffle_free_pages", "sgmv_pool_pages_device", "sgmv_plan_table_capacity",
             "sgmv_build_plan", "sgmv_shrink", "sgmv_expand", "sgmv_lora_delta", "sgmv_lora_delta_grouped",
-            "sgmv_lora_delta_noalloc", "sgmv_host_workspace_bytes", "sgmv_lora_delta_host",
+            "sgmv_lora_delta_noalloc", "sgmv_lora_delta_kernels", "sgmv_host_workspace_bytes", "sgmv_lora_delta_host",
             "sgmv_check_errors", "sgmv_residency_create", "sgmv_residency_destroy",
             "sgmv_residency_register", "sgmv_residency_unregister", "sgmv_residency_prepare",
             "sgmv_residency_get_stats")
@@ -122,6 +122,8 @@ def load_library() -> ctypes.CDLL:
                                          i32, vp]),
         "sgmv_lora_delta_noalloc": (st, [vp, i64, i32, i32, i32, i32, ctypes.POINTER(Plan), vp, vp, f32, vp, i64,
                                          i32, vp]),
+        "sgmv_lora_delta_kernels": (st, [ctypes.POINTER(Plan), vp, vp, i32, vp, i32, ctypes.POINTER(i32),
+                                         ctypes.POINTER(i32)]),
         "sgmv_host_workspace_bytes": (i64, [i32, vp, ctypes.POINTER(HostEntry), i32, i32]),
         "sgmv_lora_delta_host": (st, [vp, i32, vp, ctypes.POINTER(HostEntry), i32, f32, i32, vp, i64, vp, i64,
                                       ctypes.POINTER(Plan), ctypes.POINTER(i64), ctypes.POINTER(i64), vp]),
@@ -547,6 +549,25 @@ def lora_delta_grouped(entries, plan: BatchPlan, pool: AdapterPool, scale: float
                                                   plan.table_ptr(stream), pool.handle, float(scale),
                                                   0 if ydt == torch.bfloat16 else 1, _stream(stream)))
     return vs
+
+
+# kernel kinds reported by lora_delta_kernels (SGMV_KERNELS_* in include/sgmv.h)
+KERNELS_FUSED, KERNELS_SIMT, KERNELS_TC = 1, 2, 4
+
+
+def lora_delta_kernels(plan: BatchPlan, pool: AdapterPool, projs: Sequence[int], y_dtype=torch.bfloat16,
+                       stream=None) -> Tuple[int, int]:
+    """(kinds, launches): which kernels lora_delta (one projection) or lora_delta_grouped (the
+    projections `projs`) launch for this plan and pool -- a mask of KERNELS_FUSED,
+    KERNELS_SIMT and KERNELS_TC -- and how many launches; nothing is launched."""
+    n = len(projs)
+    arr = (ctypes.c_int32 * n)(*[int(p) for p in projs])
+    kinds, launches = ctypes.c_int32(), ctypes.c_int32()
+    _check(load_library().sgmv_lora_delta_kernels(ctypes.byref(plan.plan), pool.handle,
+                                                  ctypes.cast(arr, ctypes.c_void_p), n, plan.table_ptr(stream),
+                                                  0 if y_dtype == torch.bfloat16 else 1, ctypes.byref(kinds),
+                                                  ctypes.byref(launches)))
+    return int(kinds.value), int(launches.value)
 
 
 def lora_delta_noalloc(x: torch.Tensor, plan: BatchPlan, pool: AdapterPool, y: torch.Tensor, proj: int = 0,

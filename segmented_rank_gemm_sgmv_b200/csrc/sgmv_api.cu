@@ -339,6 +339,56 @@ extern "C" sgmv_status sgmv_lora_delta_grouped(const sgmv_delta_entry* entries, 
     return delta_impl(entries, n_entries, T, plan, table, pool, scale, y_dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
+// Which kernels sgmv_lora_delta / sgmv_lora_delta_grouped launch for a plan, pool and set of
+// projections: the same choices the calls make (including the one-wave test of the fused
+// kernel, an occupancy query), with nothing launched.
+extern "C" sgmv_status sgmv_lora_delta_kernels(const sgmv_plan* plan, const sgmv_pool* pool, const int32_t* projs,
+                                               int32_t n_entries, const void* table, int32_t y_dtype,
+                                               int32_t* kinds, int32_t* launches) {
+    if (!plan || !pool || !projs || !kinds || !launches)
+        return fail(SGMV_ERR_INVALID, "lora_delta_kernels: plan, pool, projs, kinds and launches are required");
+    if (pool->device < 0 || !pool->pages_dev)
+        return fail(SGMV_ERR_INVALID, "lora_delta_kernels: pool has no device memory");
+    if (n_entries < 1 || n_entries > kMaxGroup)
+        return fail(SGMV_ERR_INVALID, "lora_delta_kernels: 1 to " + std::to_string(kMaxGroup) + " entries are required");
+    if (y_dtype != 0 && y_dtype != 1) return fail(SGMV_ERR_INVALID, "lora_delta_kernels: y_dtype must be 0 or 1");
+    if (plan->n_proj != pool->n_proj) return fail(SGMV_ERR_INVALID, "lora_delta_kernels: plan was built for another pool");
+    for (int32_t i = 0; i < n_entries; ++i)
+        if (projs[i] < 0 || projs[i] >= pool->n_proj)
+            return fail(SGMV_ERR_INVALID, "lora_delta_kernels: projection index out of range");
+    *kinds = 0;
+    *launches = 0;
+    if (plan->num_rows <= 0 || (plan->num_simt_items <= 0 && plan->num_tc_tiles <= 0)) return SGMV_OK;
+    const bool simt = plan->num_simt_items > 0, tc = plan->num_tc_tiles > 0;
+    if (tc) {
+        *kinds |= SGMV_KERNELS_TC;
+        *launches += 2 * n_entries;  // a shrink and an expand per entry
+    }
+    if (!simt) return SGMV_OK;
+    SGMV_CUDA_TRY(cudaSetDevice(pool->device));
+    const bool per_entry = n_entries > 1 && !table;  // the calls then run the entries one at a time
+    const int32_t calls = per_entry ? n_entries : 1;
+    for (int32_t c = 0; c < calls; ++c) {
+        bool fused = false;
+        if ((per_entry || n_entries == 1) && !tc) {
+            const int32_t p = projs[c];
+            PoolView pv{};
+            pv.page_log2 = (int16_t)pool->page_log2;
+            pv.wfmt = (int16_t)pool->wfmt;
+            const ShrinkJob sj{nullptr, 0, pool->d_in[p], 1, {p}, {}, {}};
+            const ExpandJob ej{nullptr, 0, pool->d_out[p], p, nullptr, 0};
+            InlineTable<kInlineItems> inl;
+            const bool use_inl = inline_items(plan, p, &inl);
+            SGMV_CUDA_TRY(launch_fused_simt(sj, ej, BatchView{}, plan->num_simt_items, plan->max_item_rows,
+                                            plan->max_rank, pv, 1.0f, y_dtype, use_inl ? &inl : nullptr, nullptr,
+                                            &fused, true));
+        }
+        *kinds |= fused ? SGMV_KERNELS_FUSED : SGMV_KERNELS_SIMT;
+        *launches += fused ? 1 : 2;
+    }
+    return SGMV_OK;
+}
+
 // ---------------------------------------------------------------------------
 // The step from host buffers: plan, copies in, grouped delta, copy out.
 

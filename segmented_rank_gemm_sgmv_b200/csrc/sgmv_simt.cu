@@ -789,15 +789,6 @@ struct GridWalk {
     }
 };
 
-// Token row j of an item (j a run-time value): selected from the registers, no local memory.
-__device__ __forceinline__ int tok_at(const ItemInfo& m, int j) {
-    int t = -1;
-#pragma unroll
-    for (int i = 0; i < kSimtMaxItemRows; ++i)
-        if (j == i) t = m.tok[i];
-    return t;
-}
-
 // Threads of the fused kernel: eight warps for bf16 pools (two a scheduler), four for the
 // loops of quantised pools.
 template <int WF>
@@ -1441,13 +1432,14 @@ cudaError_t expand_launch(const ExpandJob* jobs, int n_jobs, const BatchView& b,
 
 // The one-shot fused kernel for a single projection, when every item's cluster fits in
 // one wave and a CTA's slices fit in shared memory (*used = true); otherwise nothing is
-// launched.  The largest cluster size (up to 8) that fits is taken: the most CTAs loading at
-// once, and the least dependent work per thread.  (Clusters of 16, a non-portable size,
-// were measured slower on decode: 18.5 against 16.5 us per step.)
+// launched.  With `dry`, the choice is made and reported but nothing is launched.  The
+// largest cluster size (up to 8) that fits is taken: the most CTAs loading at once, and the
+// least dependent work per thread.  (Clusters of 16, a non-portable size, were measured
+// slower on decode: 18.5 against 16.5 us per step.)
 template <int WF>
 cudaError_t fused_launch(const ShrinkJob& sj, const ExpandJob& ej, const BatchView& b, int32_t num_items,
                          int32_t max_item_rows, int32_t max_rank, const PoolView& pool, float scale, int32_t y_dtype,
-                         const InlineTable<kInlineItems>* inl, cudaStream_t stream, bool* used) {
+                         const InlineTable<kInlineItems>* inl, cudaStream_t stream, bool* used, bool dry) {
     *used = false;
     if (num_items <= 0 || sj.nsub != 1 || sj.d_in <= 0 || ej.d_out <= 0) return cudaSuccess;
     if (WF == kFmtBf16 && max_rank > kFusedWideMaxRank) return cudaSuccess;
@@ -1513,6 +1505,10 @@ cudaError_t fused_launch(const ShrinkJob& sj, const ExpandJob& ej, const BatchVi
             continue;
         }
         if (clusters < num_items) continue;
+        if (dry) {
+            *used = true;
+            return cudaSuccess;
+        }
         a.x = sj.x;
         a.ldx = sj.ldx;
         a.v = sj.v[0];
@@ -1545,18 +1541,18 @@ cudaError_t fused_launch(const ShrinkJob& sj, const ExpandJob& ej, const BatchVi
 cudaError_t launch_fused_simt(const ShrinkJob& sj, const ExpandJob& ej, const BatchView& b, int32_t num_items,
                               int32_t max_item_rows, int32_t max_rank, const PoolView& pool, float scale,
                               int32_t y_dtype, const InlineTable<kInlineItems>* inl, cudaStream_t stream,
-                              bool* used) {
+                              bool* used, bool dry) {
     *used = false;
     switch (pool.wfmt) {
         case kFmtBf16:
             return fused_launch<kFmtBf16>(sj, ej, b, num_items, max_item_rows, max_rank, pool, scale, y_dtype, inl,
-                                          stream, used);
+                                          stream, used, dry);
         case kFmtFp8:
             return fused_launch<kFmtFp8>(sj, ej, b, num_items, max_item_rows, max_rank, pool, scale, y_dtype, inl,
-                                         stream, used);
+                                         stream, used, dry);
         case kFmtInt4:
             return fused_launch<kFmtInt4>(sj, ej, b, num_items, max_item_rows, max_rank, pool, scale, y_dtype, inl,
-                                          stream, used);
+                                          stream, used, dry);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -92,3 +92,22 @@ def test_host_step_workspace_and_argument_checks():
     host = ctypes.create_string_buffer(4096)
     st = lib.sgmv_lora_delta_host(ids, 2, pool.handle, ents, 3, 1.0, 0, host, 4096, None, 0, None, None, None, None)
     assert st == 1 and b"workspace" in lib.sgmv_last_error()
+
+
+def test_kernels_query_argument_checks():
+    """sgmv_lora_delta_kernels refuses malformed arguments before any CUDA call."""
+    lib = sg.load_library()
+    pool = sg.AdapterPool([(512, 512)], num_pages=64, page_elems=512, max_rank=16, device=-1)
+    pool.load(0, 8)
+    plan = pool.plan([0, 0, -1])
+    projs = (ctypes.c_int32 * 1)(0)
+    kinds, launches = ctypes.c_int32(7), ctypes.c_int32(7)
+    pp = ctypes.cast(projs, ctypes.c_void_p)
+    st = lib.sgmv_lora_delta_kernels(None, pool.handle, pp, 1, None, 0, ctypes.byref(kinds), ctypes.byref(launches))
+    assert st == 1 and b"required" in lib.sgmv_last_error()
+    st = lib.sgmv_lora_delta_kernels(ctypes.byref(plan.plan), pool.handle, pp, 1, None, 0, None, ctypes.byref(launches))
+    assert st == 1
+    st = lib.sgmv_lora_delta_kernels(ctypes.byref(plan.plan), pool.handle, pp, 1, None, 0, ctypes.byref(kinds),
+                                     ctypes.byref(launches))
+    assert st == 1 and b"no device memory" in lib.sgmv_last_error()
+    pool.close()

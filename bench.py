@@ -330,8 +330,8 @@ def run_ours(args, rank, world, device, with_e2e=True):
             k, n_l = sg.lora_delta_kernels(plans[0], pool, [p], y_dt, stream)
             mask |= k
             launches += n_l
-    names = " + ".join(n for bit, n in ((sg.KERNELS_FUSED, "fused_simt_kernel"),
-                                        (sg.KERNELS_SIMT, "shrink_simt_kernel + expand_simt_kernel"),
+    simt_pair = ("shrink_slab_kernel" if mask & sg.KERNELS_SLAB else "shrink_simt_kernel") + " + expand_simt_kernel"
+    names = " + ".join(n for bit, n in ((sg.KERNELS_FUSED, "fused_simt_kernel"), (sg.KERNELS_SIMT, simt_pair),
                                         (sg.KERNELS_TC, "shrink_tc_kernel + expand_tc_kernel")) if mask & bit)
     api = "sgmv_lora_delta_grouped" if grouped else "sgmv_lora_delta"
     res = dict(total_ms=total_ms, proj_ms=float(np.mean(proj_ms)), kernel_name=f"{api} ({names})",

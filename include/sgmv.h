@@ -480,9 +480,11 @@ SGMV_API sgmv_status sgmv_lora_delta_grouped(const sgmv_delta_entry* entries, in
  * becomes the calling thread's current device).
  *
  * kinds     out: a mask of SGMV_KERNELS_FUSED (the one-shot fused SIMT kernel),
- *           SGMV_KERNELS_SIMT (the SIMT shrink and expand pair) and
- *           SGMV_KERNELS_TC (the tensor-core shrink and expand of long segments);
- *           0 when the plan has no work.
+ *           SGMV_KERNELS_SIMT (a SIMT shrink and expand pair), SGMV_KERNELS_SLAB
+ *           (set with SGMV_KERNELS_SIMT: the pair's shrink is the one-shot slab
+ *           kernel, each CTA's whole slice of A staged at once, instead of the
+ *           streaming one) and SGMV_KERNELS_TC (the tensor-core shrink and expand
+ *           of long segments); 0 when the plan has no work.
  * launches  out: kernel launches the call makes.
  * Errors: SGMV_ERR_INVALID (null pointers, a pool without device memory,
  * n_entries outside 1..8, a projection outside the pool, y_dtype not 0 or 1, a
@@ -492,6 +494,7 @@ enum {
     SGMV_KERNELS_FUSED = 1,
     SGMV_KERNELS_SIMT = 2,
     SGMV_KERNELS_TC = 4,
+    SGMV_KERNELS_SLAB = 8,
 };
 SGMV_API sgmv_status sgmv_lora_delta_kernels(const sgmv_plan* plan, const sgmv_pool* pool, const int32_t* projs,
                                              int32_t n_entries, const void* table, int32_t y_dtype,

@@ -552,14 +552,15 @@ def lora_delta_grouped(entries, plan: BatchPlan, pool: AdapterPool, scale: float
 
 
 # kernel kinds reported by lora_delta_kernels (SGMV_KERNELS_* in include/sgmv.h)
-KERNELS_FUSED, KERNELS_SIMT, KERNELS_TC = 1, 2, 4
+KERNELS_FUSED, KERNELS_SIMT, KERNELS_TC, KERNELS_SLAB = 1, 2, 4, 8
 
 
 def lora_delta_kernels(plan: BatchPlan, pool: AdapterPool, projs: Sequence[int], y_dtype=torch.bfloat16,
                        stream=None) -> Tuple[int, int]:
     """(kinds, launches): which kernels lora_delta (one projection) or lora_delta_grouped (the
     projections `projs`) launch for this plan and pool -- a mask of KERNELS_FUSED,
-    KERNELS_SIMT and KERNELS_TC -- and how many launches; nothing is launched."""
+    KERNELS_SIMT (with KERNELS_SLAB when its shrink is the slab kernel) and KERNELS_TC --
+    and how many launches; nothing is launched."""
     n = len(projs)
     arr = (ctypes.c_int32 * n)(*[int(p) for p in projs])
     kinds, launches = ctypes.c_int32(), ctypes.c_int32()

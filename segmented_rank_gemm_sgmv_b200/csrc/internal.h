@@ -166,6 +166,11 @@ cudaError_t launch_fused_simt(const ShrinkJob& sj, const ExpandJob& ej, const Ba
                               int32_t max_item_rows, int32_t max_rank, const PoolView& pool, float scale,
                               int32_t y_dtype, const InlineTable<kInlineItems>* inl, cudaStream_t stream,
                               bool* used, bool dry = false);
+// The one-shot slab shrink of one x over a bf16 pool, when it applies (*used = true; with
+// `dry` the choice is made and nothing is launched).  launch_shrink_simt tries it first.
+cudaError_t slab_shrink_launch(const ShrinkJob& j, const BatchView& b, int32_t num_items, int32_t max_item_rows,
+                               int32_t max_rank, const PoolView& pool, const InlineTable<kInlineItems>* inl,
+                               cudaStream_t stream, bool* used, bool dry);
 cudaError_t launch_shrink_tc(const uint16_t* x, int64_t ldx, int32_t d_in, const BatchView& b, int32_t num_tiles,
                              int32_t max_rank, const PoolView& pool, float* v, int64_t ldv, cudaStream_t stream);
 cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const BatchView& b, int32_t num_tiles,

@@ -385,6 +385,19 @@ extern "C" sgmv_status sgmv_lora_delta_kernels(const sgmv_plan* plan, const sgmv
         }
         *kinds |= fused ? SGMV_KERNELS_FUSED : SGMV_KERNELS_SIMT;
         *launches += fused ? 1 : 2;
+        if (!fused && (per_entry || n_entries == 1)) {  // one x, one projection: the slab shrink may run
+            const int32_t p = projs[c];
+            PoolView pv{};
+            pv.page_log2 = (int16_t)pool->page_log2;
+            pv.wfmt = (int16_t)pool->wfmt;
+            const ShrinkJob sj{nullptr, 0, pool->d_in[p], 1, {p}, {}, {}};
+            InlineTable<kInlineItems> inl;
+            const bool use_inl = inline_items(plan, p, &inl);
+            bool slab = false;
+            SGMV_CUDA_TRY(slab_shrink_launch(sj, BatchView{}, plan->num_simt_items, plan->max_item_rows,
+                                             plan->max_rank, pv, use_inl ? &inl : nullptr, nullptr, &slab, true));
+            if (slab) *kinds |= SGMV_KERNELS_SLAB;
+        }
     }
     return SGMV_OK;
 }

@@ -736,13 +736,7 @@ __global__ void __launch_bounds__(kThreads, 4)
 // memory.
 //
 // bf16 pools run eight warps a CTA:
-//   shrink: warp-level bf16 mma (m16n8k16, fp32 accumulation): M = rank rows (16 a tile), N =
-//           tokens (8: the item's <= 4 and padding), K = 16 columns of d_in; warp w takes K
-//           steps w, w + 8, ... with two accumulator sets, and the eight warp tiles are summed
-//           in warp order.  A and x are staged with their 16-byte granules XOR-swizzled by row
-//           (granule c of row k at c ^ (k % 8)), so the ldmatrix row reads are conflict-free.
-//           Three instructions per 16 x 16 block of A replace some thirty FMA, conversion and
-//           shared-memory instructions: the phase is latency-bound, and this shortens it.
+//   shrink: mma_shrink_slab over the staged A and x slices (XOR-swizzled granules).
 //   expand: thread t owns 4 columns of the slice and runs over every rank row with FMA; v is
 //           kept transposed, [rank row][4 tokens], so one 16-byte load gives the row's weights
 //           for every token of the item.  (An mma expand, with v split into bf16 hi + lo, was
@@ -789,6 +783,81 @@ struct GridWalk {
     }
 };
 
+// The shrink of a CTA's staged bf16 slab on warp-level bf16 mma (m16n8k16, fp32
+// accumulation): A rows [r][kc] and token rows x [MAXG][kc] in shared memory at As_u / xs_u,
+// both with 16-byte granule c of row k stored at granule c ^ (k % 8), so that the ldmatrix row
+// reads are conflict-free.  M = rank rows (16 a tile, up to MT_MAX tiles), N = tokens (8: the
+// item's <= 4 and padding), K = 16 columns; warp w takes K steps w, w + W, ... with two
+// accumulator sets, and the W warp tiles are summed in warp order into tile[j * r + k] (j < n,
+// k < r).  Three instructions per 16 x 16 block of A replace some thirty FMA, conversion and
+// shared-memory instructions.  wpart: W x MAXG x ldw floats of scratch.  Every thread of the
+// CTA calls it (it holds a barrier); `ok` false leaves the tile untouched.
+template <int MAXG, int W, int MT_MAX>
+__device__ __forceinline__ void mma_shrink_slab(uint32_t As_u, uint32_t xs_u, int kc, int r, int n, bool ok,
+                                                float* wpart, int ldw, float* tile) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (ok) {
+        const int MT = (r + 15) >> 4, ksteps = kc >> 4;
+        float d[MT_MAX][4], d1[MT_MAX][4];
+#pragma unroll
+        for (int mt = 0; mt < MT_MAX; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d[mt][i] = d1[mt][i] = 0.f;
+        // lane addresses: x rows are the tokens (padding lanes read row 0; their columns of D
+        // are not used), A rows the rank rows of each tile (rows past r read row 0)
+        const int mi = lane >> 3;
+        const int xrow = (lane & 7) < MAXG ? (lane & 7) : 0;
+        const uint32_t xbase = xs_u + (uint32_t)(xrow * kc * 2);
+        uint32_t arow[MT_MAX];
+        int asw[MT_MAX];
+#pragma unroll
+        for (int mt = 0; mt < MT_MAX; ++mt) {
+            int row = mt * 16 + ((mi & 1) << 3) + (lane & 7);
+            row = row < r ? row : 0;
+            arow[mt] = As_u + (uint32_t)(row * kc * 2);
+            asw[mt] = row & 7;
+        }
+        for (int ks = warp; ks < ksteps; ks += 2 * W) {
+            const int ks1 = ks + W;
+            const bool two = ks1 < ksteps;
+            uint32_t xb[2], xb1[2];
+            ldsm_x2(xbase + ((((ks << 1) | (mi & 1)) ^ (xrow & 7)) << 4), xb);
+            if (two) ldsm_x2(xbase + ((((ks1 << 1) | (mi & 1)) ^ (xrow & 7)) << 4), xb1);
+#pragma unroll
+            for (int mt = 0; mt < MT_MAX; ++mt) {
+                if (mt < MT) {
+                    uint32_t af[4], af1[4];
+                    ldsm_x4(arow[mt] + ((((ks << 1) | (mi >> 1)) ^ asw[mt]) << 4), af);
+                    if (two) ldsm_x4(arow[mt] + ((((ks1 << 1) | (mi >> 1)) ^ asw[mt]) << 4), af1);
+                    mma_bf16_16816(d[mt], af, xb[0], xb[1]);
+                    if (two) mma_bf16_16816(d1[mt], af1, xb1[0], xb1[1]);
+                }
+            }
+        }
+        // warp tiles: d[mt] = {(row 16mt + g, tokens 2t, 2t+1), (row 16mt + g + 8, same tokens)}
+        const int g = lane >> 2, t2 = 2 * (lane & 3);
+#pragma unroll
+        for (int mt = 0; mt < MT_MAX; ++mt) {
+            if (mt < MT) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int k = mt * 16 + g + ((i >> 1) << 3), j = t2 + (i & 1);
+                    if (j < MAXG && k < r) wpart[(warp * MAXG + j) * ldw + k] = d[mt][i] + d1[mt][i];
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (ok)
+        for (int e = tid; e < n * r; e += W * 32) {
+            const int j = e / r, k = e - j * r;
+            float sum = 0.f;
+#pragma unroll
+            for (int w = 0; w < W; ++w) sum += wpart[(w * MAXG + j) * ldw + k];
+            tile[e] = sum;
+        }
+}
+
 // Threads of the fused kernel: eight warps for bf16 pools (two a scheduler), four for the
 // loops of quantised pools.
 template <int WF>
@@ -804,7 +873,7 @@ __global__ void __launch_bounds__(fused_threads<WF>(), 1)
     constexpr int TPB = fused_threads<WF>();
     constexpr int kWarps = TPB / 32;
     constexpr int kMT = kFusedWideMaxRank / 16;  // 16-row tiles of the largest rank
-    const int tid = threadIdx.x, col = kVec * tid, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x, col = kVec * tid;
     const int C = a.cluster;
     // every CTA of the cluster is running before any pushes into another's shared memory
     if (C > 1) cluster_arrive_relaxed();
@@ -906,67 +975,7 @@ __global__ void __launch_bounds__(fused_threads<WF>(), 1)
     __syncthreads();
     float* mine = part + (size_t)q * slot;  // this CTA's partial tile [token][rank row]
     if constexpr (kWide) {
-        if (ma.ok) {
-            const int MT = (r + 15) >> 4, ksteps = a.kc >> 4;
-            // two accumulator sets (K steps ks and ks + warps) keep two mma chains in flight
-            float d[kMT][4], d1[kMT][4];
-#pragma unroll
-            for (int mt = 0; mt < kMT; ++mt)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) d[mt][i] = d1[mt][i] = 0.f;
-            // lane addresses: x rows are the tokens (padding lanes read row 0; their columns of
-            // D are not used), A rows the rank rows of each tile (rows past r read row 0)
-            const int mi = lane >> 3;
-            const int xrow = (lane & 7) < MAXG ? (lane & 7) : 0;
-            const uint32_t xbase = smem_u32(xs) + (uint32_t)(xrow * a.kc * 2);
-            uint32_t arow[kMT];
-            int asw[kMT];
-#pragma unroll
-            for (int mt = 0; mt < kMT; ++mt) {
-                int row = mt * 16 + ((mi & 1) << 3) + (lane & 7);
-                row = row < r ? row : 0;
-                arow[mt] = smem_u32(As) + (uint32_t)(row * a.kc * 2);
-                asw[mt] = row & 7;
-            }
-            for (int ks = warp; ks < ksteps; ks += 2 * kWarps) {
-                const int ks1 = ks + kWarps;
-                const bool two = ks1 < ksteps;
-                uint32_t xb[2], xb1[2];
-                ldsm_x2(xbase + ((((ks << 1) | (mi & 1)) ^ (xrow & 7)) << 4), xb);
-                if (two) ldsm_x2(xbase + ((((ks1 << 1) | (mi & 1)) ^ (xrow & 7)) << 4), xb1);
-#pragma unroll
-                for (int mt = 0; mt < kMT; ++mt) {
-                    if (mt < MT) {
-                        uint32_t af[4], af1[4];
-                        ldsm_x4(arow[mt] + ((((ks << 1) | (mi >> 1)) ^ asw[mt]) << 4), af);
-                        if (two) ldsm_x4(arow[mt] + ((((ks1 << 1) | (mi >> 1)) ^ asw[mt]) << 4), af1);
-                        mma_bf16_16816(d[mt], af, xb[0], xb[1]);
-                        if (two) mma_bf16_16816(d1[mt], af1, xb1[0], xb1[1]);
-                    }
-                }
-            }
-            // warp tiles: d[mt] = {(row 16mt + g, tokens 2t, 2t+1), (row 16mt + g + 8, same tokens)}
-            const int g = lane >> 2, t2 = 2 * (lane & 3);
-#pragma unroll
-            for (int mt = 0; mt < kMT; ++mt) {
-                if (mt < MT) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int k = mt * 16 + g + ((i >> 1) << 3), j = t2 + (i & 1);
-                        if (j < MAXG && k < r) wpart[(warp * MAXG + j) * a.max_rank + k] = d[mt][i] + d1[mt][i];
-                    }
-                }
-            }
-        }
-        __syncthreads();
-        if (ma.ok)
-            for (int e = tid; e < n * r; e += TPB) {
-                const int j = e / r, k = e - j * r;
-                float sum = 0.f;
-#pragma unroll
-                for (int w = 0; w < kWarps; ++w) sum += wpart[(w * MAXG + j) * a.max_rank + k];
-                mine[e] = sum;
-            }
+        mma_shrink_slab<MAXG, kWarps, kMT>(smem_u32(As), smem_u32(xs), a.kc, r, n, ma.ok, wpart, a.max_rank, mine);
     } else if (ma.ok) {  // rank row groups outer, 1024-column passes inner
         const int NG = (r + kRowGroup - 1) / kRowGroup, npass = (a.kc + kPass - 1) / kPass;
         for (int g = 0; g < NG; ++g) {
@@ -1143,6 +1152,114 @@ __global__ void __launch_bounds__(fused_threads<WF>(), 1)
     }
 }
 
+// ------------------------------------------------------------------ one-shot shrink (bf16)
+// The shrink of a single x over bf16 pools when the streaming ring would be latency-bound
+// (items whose rank rows take many stages: a rank-64 item streams eight 8-row stages one after
+// another).  A cluster of C CTAs per item, CTA q owning d_in columns [q kc, (q+1) kc), with C
+// chosen so that the whole slice of A (r x kc) and of x fits in shared memory: after one round
+// of page-id loads every copy of the CTA is issued at once (one DRAM round trip), the slab is
+// contracted by mma_shrink_slab, and the partial tiles are summed on rank 0 as in the streaming
+// shrink (pushed into its shared memory, fixed order).  Launched like the streaming shrink: its
+// dependent expand may start as soon as the CTAs have started.
+struct SlabShrinkArgs {
+    const uint16_t* x;
+    int64_t ldx;
+    float* v;
+    int64_t ldv;
+    BatchView b;
+    PoolView pool;
+    int32_t d_in, kc, proj, cluster, max_rank;
+    int32_t off_part, off_wp, off_pid, off_a, off_x;
+};
+constexpr int kSlabThreads = 2 * kThreads;
+constexpr int kSlabMaxRank = 64;            // four 16-row mma tiles
+constexpr size_t kSlabBytes = 64 * 1024;    // A slice of one CTA, at most
+
+template <int MAXG, int NI>
+__global__ void __launch_bounds__(kSlabThreads, 2)
+    shrink_slab_kernel(const __grid_constant__ SlabShrinkArgs a, const __grid_constant__ InlineTable<NI> inl) {
+    extern __shared__ __align__(128) uint8_t smem_s[];
+    constexpr int kWarps = kSlabThreads / 32;
+    pdl_launch_dependents();  // the expand may start staging its B^T pages now
+    const int C = a.cluster;
+    if (C > 1) cluster_arrive_relaxed();  // (waited on before the partial tiles are pushed)
+    const int tid = threadIdx.x;
+    const int item_idx = (int)blockIdx.x / C;
+    const uint32_t q = cluster_ctarank();
+    float* part = reinterpret_cast<float*>(smem_s + a.off_part);       // [C][4 x max_rank]; slot 0 this CTA's own
+    float* wpart = reinterpret_cast<float*>(smem_s + a.off_wp);        // [warps][MAXG][max_rank]
+    int32_t* pid = reinterpret_cast<int32_t*>(smem_s + a.off_pid);     // [r][kc / P]
+    uint16_t* As = reinterpret_cast<uint16_t*>(smem_s + a.off_a);      // [r][kc]
+    uint16_t* xs = reinterpret_cast<uint16_t*>(smem_s + a.off_x);      // [MAXG][kc]
+    const int slot = kSimtMaxItemRows * a.max_rank;
+
+    const ItemInfo m = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 0)
+                              : load_item(a.b, a.proj, item_idx, MAXG, a.max_rank, 0);
+    if (!m.ok && tid == 0) atomicOr(&g_err_simt, kErrRows);
+    const int r = m.r, n = m.n;
+    const int P_log2 = a.pool.page_log2, P = 1 << P_log2;
+    const int ppr = a.d_in >> P_log2, cpa = a.kc >> P_log2;
+    const int c0 = (int)q * a.kc;
+    const int gx = a.kc / 8;  // 16-byte granules of a row slice
+    if (m.ok) {
+        // x slices need no page ids: issued first; granule c of row j at c ^ (j % 8)
+#pragma unroll
+        for (int j = 0; j < MAXG; ++j) {
+            const int t = m.tok[j];
+            for (int cg = tid; cg < gx; cg += kSlabThreads)
+                cp_async16(xs + (size_t)j * a.kc + (cg ^ (j & 7)) * 8,
+                           t >= 0 ? a.x + (int64_t)t * a.ldx + c0 + cg * 8 : a.x, t >= 0);
+        }
+        for (int i = tid; i < r * cpa; i += kSlabThreads) {
+            const int k = i / cpa, pc = i - k * cpa;
+            const int64_t e = m.pt + (int64_t)k * ppr + (c0 >> P_log2) + pc;
+            int32_t page = (e >= 0 && e < a.pool.pt_capacity) ? a.pool.page_table[e] : -1;
+            if (page < 0 || page >= a.pool.num_pages) {
+                atomicOr(&g_err_simt, kErrPage);
+                page = 0;
+            }
+            pid[i] = page;
+        }
+    }
+    __syncthreads();
+    if (m.ok)
+        for (GridWalk w(gx, tid, kSlabThreads); w.k < r; w.next()) {
+            const int cl = w.c * 8;
+            cp_async16(As + (size_t)w.k * a.kc + (w.c ^ (w.k & 7)) * 8,
+                       a.pool.pages + ((int64_t)pid[w.k * cpa + (cl >> P_log2)] << P_log2) + (cl & (P - 1)), true);
+        }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    float* mine = part;  // slot 0
+    mma_shrink_slab<MAXG, kWarps, kSlabMaxRank / 16>(smem_u32(As), smem_u32(xs), a.kc, r, n, m.ok, wpart,
+                                                     a.max_rank, mine);
+    __syncthreads();
+
+    // partial tiles into rank 0's slots 1..C-1 (the other CTAs then exit); rank 0 sums 0..C-1
+    const int E = n * r;
+    if (C > 1) {
+        cluster_wait_acquire();
+        if (q != 0) {
+            if (m.ok) {
+                const uint32_t dst = map_cluster(smem_u32(part + (size_t)q * slot), 0u);
+                for (int e = tid; e < E; e += kSlabThreads) st_cluster_f32(dst + 4u * (uint32_t)e, mine[e]);
+            }
+            cluster_arrive_release();
+            return;
+        }
+        cluster_arrive_release();
+        cluster_wait_acquire();
+    }
+    if (m.ok)
+        for (int e = tid; e < E; e += kSlabThreads) {
+            float sum = 0.f;
+            for (int qq = 0; qq < C; ++qq) sum += part[(size_t)qq * slot + e];
+            const int jrow = e / r, k = e - jrow * r;
+            a.v[(int64_t)(m.i0 + jrow) * a.ldv + k] = sum;
+        }
+}
+
 int num_sms() {
     static int n = 0;
     if (n == 0) {
@@ -1235,6 +1352,89 @@ double group_time(const SimtWork& work, int64_t items, const int* cpi, const int
     }
     const double biggest = (double)std::max(work.max_ng, 1) * max_np + kPrologue;
     return std::max(biggest, total / (double)std::max<int64_t>(slots, 1));
+}
+
+// The one-shot slab shrink, when it applies: bf16 pool, one x with one projection, ranks up to
+// 64, a cluster size C <= 8 dividing the page count with an A slice r x (d_in / C) of at most
+// kSlabBytes, and at most two waves of clusters.  Then *used = true and the kernel is launched
+// (unless `dry`); otherwise nothing happens.  Measured against the streaming shrink (per step,
+// L2 flushed): 200 decode tokens on 8192 -> 8192, rank 16: 29.6 against 35.8 us; 64 tokens of
+// ranks 8-64 on 4096 -> 14336: 27.7 against 29.7 us; beyond two waves it loses (256 tokens of
+// ranks 8-64: 42.0 against 39.9 us; the 70B layer's down projection: 70.6 against 68.6 us),
+// the streaming ring overlapping each CTA's loads with its arithmetic.
+cudaError_t slab_shrink_launch(const ShrinkJob& j, const BatchView& b, int32_t num_items, int32_t max_item_rows,
+                               int32_t max_rank, const PoolView& pool, const InlineTable<kInlineItems>* inl,
+                               cudaStream_t stream, bool* used, bool dry) {
+    *used = false;
+    if (pool.wfmt != kFmtBf16 || j.nsub != 1 || max_rank > kSlabMaxRank || j.d_in <= 0) return cudaSuccess;
+    const int mr = std::max(8, max_rank);
+    const int maxg = max_item_rows <= 1 ? 1 : max_item_rows <= 2 ? 2 : 4;
+    const int pa = j.d_in >> pool.page_log2;
+    int C = 0;
+    for (int c = 1; c <= 8 && !C; ++c)
+        if (pa % c == 0 && (size_t)mr * (j.d_in / c) * 2 <= kSlabBytes) C = c;
+    if (!C) return cudaSuccess;
+    const int kc = j.d_in / C;
+    auto al = [](size_t v) { return (v + 127) & ~(size_t)127; };
+    SlabShrinkArgs a;
+    std::memset(&a, 0, sizeof(a));
+    size_t o = 0;
+    a.off_part = (int32_t)(o = al(o));
+    o += (size_t)C * kSimtMaxItemRows * mr * 4;
+    a.off_wp = (int32_t)(o = al(o));
+    o += (size_t)(kSlabThreads / 32) * maxg * mr * 4;
+    a.off_pid = (int32_t)(o = al(o));
+    o += (size_t)mr * (kc >> pool.page_log2) * 4;
+    a.off_a = (int32_t)(o = al(o));
+    o += (size_t)mr * kc * 2;
+    a.off_x = (int32_t)(o = al(o));
+    o += (size_t)maxg * kc * 2;
+    const size_t smem = al(o);
+    a.x = j.x;
+    a.ldx = j.ldx;
+    a.v = j.v[0];
+    a.ldv = j.ldv[0];
+    a.b = b;
+    a.pool = pool;
+    a.d_in = j.d_in;
+    a.kc = kc;
+    a.proj = j.proj[0];
+    a.cluster = C;
+    a.max_rank = mr;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(num_items * C), 1, 1);
+    cfg.blockDim = dim3(kSlabThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const void* kern =
+        inl ? reinterpret_cast<const void*>(pick(max_item_rows, shrink_slab_kernel<1, kInlineItems>,
+                                                 shrink_slab_kernel<2, kInlineItems>, shrink_slab_kernel<4, kInlineItems>))
+            : reinterpret_cast<const void*>(pick(max_item_rows, shrink_slab_kernel<1, 1>, shrink_slab_kernel<2, 1>,
+                                                 shrink_slab_kernel<4, 1>));
+    cudaError_t e = raise_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    int clusters = 0;  // clusters resident at once
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return cudaSuccess;
+    }
+    if (clusters <= 0 || num_items > 2 * clusters) return cudaSuccess;
+    *used = true;
+    if (dry) return cudaSuccess;
+    if (inl) {
+        void* args[] = {&a, const_cast<InlineTable<kInlineItems>*>(inl)};
+        return cudaLaunchKernelExC(&cfg, kern, args);
+    }
+    InlineTable<1> none{};
+    void* args[] = {&a, &none};
+    return cudaLaunchKernelExC(&cfg, kern, args);
 }
 
 template <int NE, int WF>
@@ -1564,6 +1764,12 @@ cudaError_t launch_shrink_simt(const ShrinkJob* jobs, int n_jobs, const BatchVie
     if (n_jobs > kMaxGroup || (inl && (n_jobs > 1 || jobs[0].nsub != 1))) return cudaErrorInvalidValue;
     for (int j = 0; j < n_jobs; ++j)
         if (jobs[j].nsub < 1 || jobs[j].nsub > kMaxShare) return cudaErrorInvalidValue;
+    if (n_jobs == 1) {
+        bool used = false;
+        cudaError_t e = slab_shrink_launch(jobs[0], b, num_items, max_item_rows, max_rank, pool, inl, stream, &used,
+                                           false);
+        if (e != cudaSuccess || used) return e;
+    }
     // one x: a one-entry table (small launch arguments, no per-CTA lookup)
     auto go = [&](auto wf) {
         constexpr int WF = decltype(wf)::value;

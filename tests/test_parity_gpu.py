@@ -155,6 +155,33 @@ def test_llama70b_layer_sampled(mode):
         assert plan.plan.num_segments == 256 and plan.plan.num_simt_items == 256
 
 
+# ------------------------------------------------------------------ slab shrink
+@pytest.mark.parametrize("y_dtype", [torch.bfloat16, torch.float32], ids=["ybf16", "yfp32"])
+@pytest.mark.parametrize("case", ["decode200", "mixed64", "ragged"])
+def test_slab_shrink(case, y_dtype):
+    """Single-projection batches that take the one-shot slab shrink (each CTA's whole slice of
+    A staged at once, contracted with warp-level mma): 200 decode tokens, 64 mixed-rank tokens,
+    and ragged segments with ranks that are not multiples of 16 (padding rows of the mma
+    tiles) and a d_in of 3 pages (cluster of 3)."""
+    if case == "decode200":
+        wl = workloads.make("decode_q_proj", T=200)
+    elif case == "mixed64":
+        wl = workloads.make("mixed_rank_mlp_up", T=64)
+    if case == "ragged":
+        wl, bank, x, y = custom_case([1, 2, 3, 4, 5, 7, 9, 2, 1], [3, 24, 40, 57, 64, 9, 16, 1, 33], 1536, 1024,
+                                     seed=11, minus_one=3)
+    else:
+        bank = workloads.AdapterBank(wl, device="cuda")
+        x, y = workloads.activations(wl, 0, device="cuda")
+    pool = build_pool(wl, bank)
+    plan = pool.plan(wl.adapter_ids, long_threshold=SIMT)
+    kinds, _ = sg.lora_delta_kernels(plan, pool, [0], y_dtype)
+    assert kinds == sg.KERNELS_SIMT | sg.KERNELS_SLAB, kinds
+    pool.close()
+    for mode in ("separate", "lora_delta"):
+        check(wl, bank, x, y, SIMT, y_dtype, mode=mode)
+
+
 # ------------------------------------------------------------------ exact pins
 @MODES
 @pytest.mark.parametrize("path", [SIMT, TC], ids=["simt", "tc"])

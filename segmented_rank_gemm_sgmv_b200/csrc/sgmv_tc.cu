@@ -396,12 +396,18 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
 //     copy each y row segment (256 bytes) with one bulk copy that completes on
 //     the stage's mbarrier by bytes, and the B^T block with 16-byte cp.async;
 //     when the tile changes, write V_hi / V_lo (v split into bf16 hi + lo)
-//   warp 12 (one lane): tcgen05.mma  acc[i & 1] = V_hi B + V_lo B  (N = block)
+//   warp 12 (one lane): tcgen05.mma  acc[i & 1] = V_hi B + V_lo B  (N = block);
+//     with bf16 y (YM), V carries the scale and the MMAs go on with acc += Y I:
+//     the staged y block, already in the K-major 128-byte swizzle of an A
+//     operand, times a 128 x 128 identity kept in shared memory (each product
+//     y * 1 exact), so the accumulator ends as y + scale V B^T
 //   warps 0-7 (epilogue): two groups of four warps take alternate units (the
 //     group of unit i reads acc[i & 1]); warp w reads rows 32 (w % 4) .. + 31 of
-//     the accumulator (tcgen05.ld) and adds scale * acc to its y rows in shared
-//     memory; the group then stores the block: one TMA store per half for a full
-//     tile of consecutive tokens, coalesced 16-byte stores otherwise
+//     the accumulator (tcgen05.ld) and either rounds it to bf16 into its y rows in
+//     shared memory (YM) or adds scale * acc to them; the group then stores the
+//     block: one TMA store per half for a full tile of consecutive tokens,
+//     coalesced 16-byte stores otherwise.  (Measured on the long-prefill batch
+//     without YM: the read-modify-write of y took 2 us of a unit's epilogue.)
 // mbarriers: full[s] (producers' copies landed: 128 cp.async arrivals plus the
 // TMA bytes), yfree[s] (the unit's epilogue group has stored slot s), accf[b]
 // (MMAs done, tcgen05.commit), acce[b] (the group has read acc[b] out),
@@ -414,7 +420,9 @@ constexpr int kExpandThreads = 416;         // 8 epilogue + 4 producer warps + 1
 constexpr int kExpandProducers = 128;
 constexpr int kMmaWarp = 12;
 
-template <int S, int ESZ, int WF>  // ESZ: bytes of a y element (2: bf16, 4: fp32); WF: weight format
+// ESZ: bytes of a y element (2: bf16, 4: fp32); WF: weight format; YM: y enters the accumulator
+// by an identity MMA (bf16 y only)
+template <int S, int ESZ, int WF, bool YM>
 __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const ExpandTcArgs a,
                                                                       const __grid_constant__ CUtensorMap tmap_y) {
     extern __shared__ uint8_t smem_raw[];
@@ -448,6 +456,24 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
     constexpr int kYHalf = kTcTileRows * (kYRowBytes / 2);
     const size_t y_bytes = 2 * (size_t)kYHalf;
 
+    static_assert(!YM || ESZ == 2, "the identity MMA adds bf16 y only");
+    // YM: the identity I[k][n] (k, n < NB = 128) in the layout of a B^T block with 128 K rows
+    uint8_t* ident = nullptr;
+    if constexpr (YM) {
+        constexpr int VBq = bytes_per_8<WF>();
+        uint8_t* const after = yst + (size_t)S * y_bytes +
+                               (WF == kFmtBf16 ? 0 : (size_t)a.raw_slots * ((size_t)kpm * (NB / 8) * VBq));
+        ident = align1024(after);
+        for (int i = tid; i < NB * NB * 2 / 16; i += kExpandThreads)
+            reinterpret_cast<uint4*>(ident)[i] = make_uint4(0u, 0u, 0u, 0u);
+        __syncthreads();
+        if (tid < NB) {
+            const int k = tid;  // element (k, k): granule k / 8 of row k, value k % 8 inside it
+            *reinterpret_cast<uint16_t*>(ident + (uint32_t)(k >> 3) * sbo_b + (uint32_t)(k >> 6) * 1024 +
+                                         sw128_off((uint32_t)k, (uint32_t)(k >> 3)) + (k & 7) * 2) = 0x3F80;  // 1.0
+        }
+        fence_proxy_async_smem();  // the identity, to the async proxy (the barrier below orders it)
+    }
     if (tid == 0) {
         abort_flag = 0;
         // full: the producers' cp.async arrivals, plus (quantised pools) their arrivals
@@ -477,14 +503,14 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
     const int pages_per_row = a.d_out >> P_log2;
     uint8_t* const ybase = static_cast<uint8_t*>(a.y);
 
-    // unit u: its tile record; ok depends on the tile only, so it is the same for
-    // every unit of a tile and for every thread
     struct Unit {
         int tile, row_begin, rows, r, j0;
         int64_t b_base;
         float sc;  // multiplier of the tile's adapter
         bool ok;
     };
+    // unit u: its tile record; ok depends on the tile only, so it is the same for
+    // every unit of a tile and for every thread
     auto unit = [&](int u) {
         Unit w;
         w.tile = u / a.n_blocks;
@@ -547,6 +573,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
             }
             const int m = pt, kpad = (w.r + 15) & ~15;
             const bool row_ok = m < w.rows;
+            const float vsc = a.scale * w.sc;
             const float* vrow = a.v + (int64_t)(w.row_begin + (row_ok ? m : 0)) * a.ldv;
             // v row in chunks of 64 floats, each chunk's 16-byte loads all in flight
             // (a load starts below r and below ldv, a multiple of 4: it stays in the row)
@@ -570,6 +597,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
                 for (int e = 0; e < 8; ++e) {
                     if (kg * 8 + e >= w.r) f[e] = 0.f;
                     else if (WF != kFmtBf16) f[e] *= rsc_s[kg * 8 + e];
+                    if (YM) f[e] *= vsc;  // the call's scale times the adapter's
                 }
                 uint32_t hw[4], lw[4];
 #pragma unroll
@@ -745,6 +773,12 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
                     for (int ks = 0; ks < kpad / 16; ++ks)
                         tc_mma_bf16(acc, smem_desc_sw128(al + (ks >> 2) * (kTcTileRows * 128) + (ks & 3) * 32, 16, 1024),
                                     smem_desc_sw128(bb + ks * 2 * sbo_b, 1024, sbo_b), idesc, true);
+                    if constexpr (YM) {  // acc += Y I: the y block (two 64-column halves) as the A operand
+                        const uint32_t yb = smem_u32(yst + (size_t)st * y_bytes), ib = smem_u32(ident);
+                        for (int ks = 0; ks < NB / 16; ++ks)
+                            tc_mma_bf16(acc, smem_desc_sw128(yb + (ks >> 2) * kYHalf + (ks & 3) * 32, 16, 1024),
+                                        smem_desc_sw128(ib + ks * 2 * sbo_b, 1024, sbo_b), idesc, true);
+                    }
                 }
                 tc_commit(&accf_bar[bsel]);
                 if (w.ok && (u + 1 == u1 || (u + 1) / a.n_blocks != w.tile))
@@ -789,7 +823,18 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
                     const int hf = c0 / (NB / 2), cc = c0 % (NB / 2);  // half, column within it
                     uint8_t* yrow = ys + (size_t)hf * kYHalf + (size_t)m * 128;  // swizzled row
                     const uint32_t (&regs)[32] = rr[h];
-                    if (ESZ == 2) {
+                    if (YM) {  // the accumulator already holds y + scale V B^T
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint32_t wv[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                wv[e] = pack_bf16x2(__uint_as_float(regs[q4 * 8 + 2 * e]),
+                                                    __uint_as_float(regs[q4 * 8 + 2 * e + 1]));
+                            *reinterpret_cast<uint4*>(yrow + ((((cc >> 3) + q4) ^ (m & 7)) << 4)) =
+                                make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                        }
+                    } else if (ESZ == 2) {
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4) {
                             uint4* yp = reinterpret_cast<uint4*>(yrow + ((((cc >> 3) + q4) ^ (m & 7)) << 4));
@@ -986,19 +1031,27 @@ cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const B
     const size_t limit = (227u << 10) - 1024 - 6656;
     // stages S and code slots R (quantised pools): three stages when they fit, two code slots
     // when they fit (one otherwise)
+    // bf16 y: the identity of the Y I products (32 KB, 1 KB aligned) when it fits, with three
+    // stages before two
+    const size_t ident_bytes = (size_t)NB * NB * 2 + 1024;
     int S = 2, R = raw_slot ? 1 : 0;
-    const int cand[3][2] = {{3, 2}, {2, 2}, {2, 1}};
+    bool ym = false;
+    const int cand[6][3] = {{3, 2, 1}, {2, 2, 1}, {2, 1, 1}, {3, 2, 0}, {2, 2, 0}, {2, 1, 0}};
     for (const auto& c : cand) {
         const int r = raw_slot ? c[1] : 0;
-        if (v_bytes + c[0] * stage + r * raw_slot <= limit) {
+        const bool with_ident = c[2] != 0;
+        if (with_ident && y_dtype != 0) continue;
+        if (v_bytes + c[0] * stage + r * raw_slot + (with_ident ? ident_bytes : 0) <= limit) {
             S = c[0];
             R = r;
+            ym = with_ident;
             break;
         }
     }
     a.raw_slots = std::max(R, 1);
     // at least 116 KB: one CTA per SM, so tensor memory (2 x NB <= 256 columns) is never oversubscribed
-    const size_t smem = std::max(v_bytes + S * stage + R * raw_slot, (size_t)116 << 10) + 1024;
+    const size_t smem =
+        std::max(v_bytes + S * stage + R * raw_slot + (ym ? ident_bytes : 0), (size_t)116 << 10) + 1024;
     if (smem > (227u << 10)) return cudaErrorInvalidValue;
     // one CTA per SM, each a contiguous run of units
     static int sms = 0;
@@ -1018,8 +1071,9 @@ cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const B
                           (uint64_t)d_out, (uint64_t)b.T, (uint64_t)ldy * esz, (uint32_t)(NB / 2), kTcTileRows) ? 1 : 0;
     auto pick = [&](auto wf) {
         constexpr int WF = decltype(wf)::value;
-        return S == 3 ? (esz == 2 ? expand_tc_kernel<3, 2, WF> : expand_tc_kernel<3, 4, WF>)
-                      : (esz == 2 ? expand_tc_kernel<2, 2, WF> : expand_tc_kernel<2, 4, WF>);
+        if (ym) return S == 3 ? expand_tc_kernel<3, 2, WF, true> : expand_tc_kernel<2, 2, WF, true>;
+        return S == 3 ? (esz == 2 ? expand_tc_kernel<3, 2, WF, false> : expand_tc_kernel<3, 4, WF, false>)
+                      : (esz == 2 ? expand_tc_kernel<2, 2, WF, false> : expand_tc_kernel<2, 4, WF, false>);
     };
     auto kern = pool.wfmt == kFmtFp8    ? pick(std::integral_constant<int, kFmtFp8>{})
                 : pool.wfmt == kFmtInt4 ? pick(std::integral_constant<int, kFmtInt4>{})

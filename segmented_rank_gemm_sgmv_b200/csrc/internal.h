@@ -68,7 +68,7 @@ struct ItemRec {
 static_assert(sizeof(ItemRec) == 32, "ItemRec must be 32 bytes");
 
 constexpr int kSimtMaxItemRows = 4;    // rows per SIMT work item
-constexpr int kInlineItems = 64;       // SIMT items that can travel as launch arguments
+constexpr int kInlineItems = 256;      // SIMT items that can travel as launch arguments (13 KB of parameters)
 
 // A SIMT work item passed by value in the kernel's parameters: the record for
 // the launch's projection plus the item's token rows.

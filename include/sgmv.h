@@ -284,8 +284,10 @@ typedef struct {
     int32_t long_threshold; /* the threshold actually used                           */
     int32_t max_item_rows;  /* largest SIMT item                                     */
     int32_t needs_device_table; /* 0: the kernels take everything from `host_table` as
-                               launch arguments (<= 256 SIMT items, no tensor-core tiles);
-                               the device table may then be NULL and need not be copied */
+                               launch arguments (no tensor-core tiles and <= 256 SIMT
+                               items, or <= 64 for a pool of several projections, whose
+                               grouped calls need the table); the device table may then
+                               be NULL and need not be copied */
     int64_t table_bytes;    /* bytes of the table to copy to the device              */
     int64_t off_token_idx, off_seg_offsets, off_seg_adapter, off_seg_rank;
     int64_t off_seg_a_pt, off_seg_b_pt, off_simt_items, off_tc_tiles;

@@ -69,6 +69,10 @@ static_assert(sizeof(ItemRec) == 32, "ItemRec must be 32 bytes");
 
 constexpr int kSimtMaxItemRows = 4;    // rows per SIMT work item
 constexpr int kInlineItems = 256;      // SIMT items that can travel as launch arguments (13 KB of parameters)
+// A plan over a pool of several projections keeps a device table above this many items: a
+// launch-argument list carries one projection, and a grouped call over the pool's
+// projections (one launch pair for all of them) needs the table.
+constexpr int kInlineItemsMultiProj = 64;
 
 // A SIMT work item passed by value in the kernel's parameters: the record for
 // the launch's projection plus the item's token rows.

@@ -182,7 +182,8 @@ extern "C" sgmv_status sgmv_build_plan(const int32_t* adapter_ids, int32_t T, co
     plan->num_tc_tiles = (int32_t)n_tc;
     plan->long_threshold = long_threshold;
     plan->max_item_rows = max_item;
-    plan->needs_device_table = (n_tc > 0 || n_simt > kInlineItems) ? 1 : 0;
+    const int32_t inline_cap = plan->n_proj > 1 ? kInlineItemsMultiProj : kInlineItems;
+    plan->needs_device_table = (n_tc > 0 || n_simt > inline_cap) ? 1 : 0;
     plan->host_table = table;
     plan->table_bytes = L.end;
     plan->off_token_idx = L.token_idx;

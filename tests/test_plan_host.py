@@ -197,3 +197,19 @@ def test_plan_carries_each_adapter_scale():
         with pytest.raises(sg.SgmvError) as e:
             pool.set_scale(3, bad)
         assert e.value.status == 1
+
+
+@pytest.mark.parametrize("projs,n_items,want_table", [
+    ([(512, 512)], 64, 0), ([(512, 512)], 256, 0), ([(512, 512)], 257, 1),
+    ([(512, 512), (512, 1024)], 64, 0), ([(512, 512), (512, 1024)], 65, 1),
+])
+def test_launch_argument_threshold(projs, n_items, want_table):
+    """Up to 256 SIMT items travel as launch arguments for a single-projection pool; a pool
+    of several projections keeps its device table above 64 (its grouped calls need it)."""
+    pool = sg.AdapterPool(projs, num_pages=20000, page_elems=512, max_rank=8, device=-1)
+    for a in range(n_items):
+        pool.load(a, 8)
+    plan = pool.plan(np.arange(n_items, dtype=np.int32))
+    assert plan.plan.num_simt_items == n_items and plan.plan.num_tc_tiles == 0
+    assert plan.plan.needs_device_table == want_table
+    pool.close()

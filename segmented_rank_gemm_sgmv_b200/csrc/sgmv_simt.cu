@@ -735,14 +735,15 @@ __global__ void __launch_bounds__(kThreads, 4)
 // each CTA sums the C tiles in a fixed order and runs its share of the expand from shared
 // memory.
 //
-// bf16 pools run eight warps a CTA:
-//   shrink: mma_shrink_slab over the staged A and x slices (XOR-swizzled granules).
-//   expand: thread t owns 4 columns of the slice and runs over every rank row with FMA; v is
-//           kept transposed, [rank row][4 tokens], so one 16-byte load gives the row's weights
-//           for every token of the item.  (An mma expand, with v split into bf16 hi + lo, was
-//           measured twice as slow: each tile needs two dependent mma, and the legacy warp-level
-//           mma's latency dominates a phase this short.)
-// Quantised pools keep four warps and the loops of the two-kernel path.
+// Eight warps a CTA:
+//   shrink: mma_shrink_slab over the staged A and x slices (XOR-swizzled granules); a quantised
+//           pool's A codes land in row order and are converted once into the bf16 slab (exact).
+//   expand: thread t owns 4 columns of the slice and runs over every rank row with FMA,
+//           converting a quantised B^T row's codes in registers; v is kept transposed,
+//           [rank row][4 tokens] (with the B^T row's scale folded in), so one 16-byte load
+//           gives the row's weights for every token of the item.  (An mma expand, with v
+//           split into bf16 hi + lo, was measured twice as slow: each tile needs two dependent
+//           mma, and the legacy warp-level mma's latency dominates a phase this short.)
 struct FusedArgs {
     const uint16_t* x;
     int64_t ldx;
@@ -760,7 +761,7 @@ struct FusedArgs {
     int32_t y_dtype;
     float scale;
     // byte offsets in shared memory
-    int32_t off_part, off_vs, off_rsc, off_pid_a, off_pid_b, off_a, off_x, off_b, off_y, off_wp;
+    int32_t off_part, off_vs, off_rsc, off_pid_a, off_pid_b, off_a, off_ac, off_x, off_b, off_y, off_wp;
 };
 
 // The cells of a rows x cols grid that thread `start` visits with stride `stride` in
@@ -858,39 +859,62 @@ __device__ __forceinline__ void mma_shrink_slab(uint32_t As_u, uint32_t xs_u, in
         }
 }
 
-// Threads of the fused kernel: eight warps for bf16 pools (two a scheduler), four for the
-// loops of quantised pools.
+// Four stored weights of format WF, values c .. c + 3 of a row (c a multiple of 4), to fp32,
+// exactly: bf16 halves, E4M3 pairs through the hardware E4M3x2 -> f16x2 conversion, INT4
+// nibbles (two's complement, value i in bits 4i .. 4i + 3 of the pair of bytes).
 template <int WF>
-__host__ __device__ constexpr int fused_threads() { return WF == kFmtBf16 ? 2 * kThreads : kThreads; }
-constexpr int kFusedWideMaxRank = 64;  // bf16 pools: ranks up to 64 (four 16-row tiles) take the fused kernel
+__device__ __forceinline__ void load_w4(const uint8_t* row, int c, float (&f)[4]) {
+    if constexpr (WF == kFmtBf16) {
+        const uint2 w = *reinterpret_cast<const uint2*>(row + (size_t)c * 2);
+        f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
+    } else if constexpr (WF == kFmtFp8) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(row + c);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t hh;
+            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hh) : "h"((uint16_t)(w >> (16 * h))));
+            float lo, hi;
+            asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"((uint16_t)(hh & 0xFFFFu)));
+            asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"((uint16_t)(hh >> 16)));
+            f[2 * h] = lo;
+            f[2 * h + 1] = hi;
+        }
+    } else {
+        const uint32_t w = (uint32_t)*reinterpret_cast<const uint16_t*>(row + c / 2) ^ 0x8888u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) f[i] = __uint_as_float(0x4B000000u | ((w >> (4 * i)) & 0xFu)) - 8388616.0f;
+    }
+}
+
+constexpr int kFusedThreads = 2 * kThreads;  // eight warps, two a scheduler
+constexpr int kFusedMaxRank = 64;             // four 16-row mma tiles
 
 template <int MAXG, int NI, int WF>
-__global__ void __launch_bounds__(fused_threads<WF>(), 1)
+__global__ void __launch_bounds__(kFusedThreads, 1)
     fused_simt_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ InlineTable<NI> inl) {
     extern __shared__ __align__(128) uint8_t smem_f[];
     constexpr int VB = bytes_per_8<WF>();
-    constexpr bool kWide = WF == kFmtBf16;
-    constexpr int TPB = fused_threads<WF>();
+    constexpr int TPB = kFusedThreads;
     constexpr int kWarps = TPB / 32;
-    constexpr int kMT = kFusedWideMaxRank / 16;  // 16-row tiles of the largest rank
-    const int tid = threadIdx.x, col = kVec * tid;
+    constexpr int kMT = kFusedMaxRank / 16;  // 16-row tiles of the largest rank
+    const int tid = threadIdx.x;
     const int C = a.cluster;
     // every CTA of the cluster is running before any pushes into another's shared memory
     if (C > 1) cluster_arrive_relaxed();
     const int item_idx = (int)blockIdx.x / C;
     const uint32_t q = cluster_ctarank();
-    float* red = reinterpret_cast<float*>(smem_f);                       // [4 warps][64]
     float* part = reinterpret_cast<float*>(smem_f + a.off_part);         // [C][4 x max_rank]
-    float* vs = reinterpret_cast<float*>(smem_f + a.off_vs);             // [4 x max_rank] (bf16: [max_rank][4])
+    float* vs = reinterpret_cast<float*>(smem_f + a.off_vs);             // [max_rank][4 tokens]
     float* rsc_a = reinterpret_cast<float*>(smem_f + a.off_rsc);         // [kMaxRank] (quantised)
     float* rsc_b = rsc_a + kMaxRank;
     int32_t* pid_a = reinterpret_cast<int32_t*>(smem_f + a.off_pid_a);  // [r][kc / P]
     int32_t* pid_b = reinterpret_cast<int32_t*>(smem_f + a.off_pid_b);  // [r][ko / P]
-    uint8_t* As = smem_f + a.off_a;                                      // [r][kc] weights
-    uint16_t* xs = reinterpret_cast<uint16_t*>(smem_f + a.off_x);        // [MAXG][kc]
+    uint16_t* As = reinterpret_cast<uint16_t*>(smem_f + a.off_a);        // [r][kc] bf16, swizzled
+    uint8_t* Ac = smem_f + a.off_ac;                                     // [r][kc] codes (quantised)
+    uint16_t* xs = reinterpret_cast<uint16_t*>(smem_f + a.off_x);        // [MAXG][kc] bf16, swizzled
     uint8_t* Bs = smem_f + a.off_b;                                      // [r][ko] weights
     uint8_t* ys = smem_f + a.off_y;                                      // [MAXG][ko] of y's type
-    float* wpart = reinterpret_cast<float*>(smem_f + a.off_wp);          // [warps][MAXG][max_rank] (bf16)
+    float* wpart = reinterpret_cast<float*>(smem_f + a.off_wp);          // [warps][MAXG][max_rank]
     const int slot = kSimtMaxItemRows * a.max_rank;
 
     ItemInfo ma = NI > 1 ? load_item(a.b, inl, item_idx, MAXG, a.max_rank, 0)
@@ -926,25 +950,28 @@ __global__ void __launch_bounds__(fused_threads<WF>(), 1)
     }
     __syncthreads();
 
-    // every copy at once: group 1 = A rows + x slices, group 2 = B^T rows + y rows
-    // (bf16: granule c of an A or x row k lands at granule c ^ (k % 8) of the row)
+    // every copy at once: group 1 = A rows + x slices, group 2 = B^T rows + y rows.  Granule c
+    // of a bf16 A or x row k lands at granule c ^ (k % 8) of the row; quantised A codes land
+    // in row order and are converted into the swizzled bf16 slab below.
     const uint8_t* pages = reinterpret_cast<const uint8_t*>(a.pool.pages);
     const int page_shift = P_log2 + (VB == 16 ? 1 : VB == 8 ? 0 : -1);
     constexpr int kVals16 = 128 / VB;  // values per 16-byte granule
-    const int gx = a.kc / 8;           // 16-byte granules of an x row slice
+    const int gx = a.kc / 8;           // 16-byte granules of an x row slice (and of a bf16 A row)
     if (ma.ok) {
         const int gpr_a = a.kc / kVals16;
         for (GridWalk w(gpr_a, tid, TPB); w.k < r; w.next()) {
             const int cl = w.c * kVals16;
-            cp_async16(As + (size_t)w.k * (a.kc / 8 * VB) + (kWide ? (w.c ^ (w.k & 7)) : w.c) * 16,
-                       pages + ((int64_t)pid_a[w.k * cpa + (cl >> P_log2)] << page_shift) + (cl & (P - 1)) / 8 * VB,
-                       true);
+            const uint8_t* src = pages + ((int64_t)pid_a[w.k * cpa + (cl >> P_log2)] << page_shift) + (cl & (P - 1)) / 8 * VB;
+            if constexpr (WF == kFmtBf16)
+                cp_async16(As + (size_t)w.k * a.kc + (w.c ^ (w.k & 7)) * 8, src, true);
+            else
+                cp_async16(Ac + (size_t)w.k * (a.kc / 8 * VB) + w.c * 16, src, true);
         }
 #pragma unroll
         for (int j = 0; j < MAXG; ++j) {
             const int t = ma.tok[j];
             for (int cg = tid; cg < gx; cg += TPB)
-                cp_async16(xs + (size_t)j * a.kc + (kWide ? (cg ^ (j & 7)) : cg) * 8,
+                cp_async16(xs + (size_t)j * a.kc + (cg ^ (j & 7)) * 8,
                            t >= 0 ? a.x + (int64_t)t * a.ldx + ca0 + cg * 8 : a.x, t >= 0);
         }
     }
@@ -973,49 +1000,21 @@ __global__ void __launch_bounds__(fused_threads<WF>(), 1)
     // ---- shrink over this CTA's d_in slice
     cp_async_wait<1>();
     __syncthreads();
-    float* mine = part + (size_t)q * slot;  // this CTA's partial tile [token][rank row]
-    if constexpr (kWide) {
-        mma_shrink_slab<MAXG, kWarps, kMT>(smem_u32(As), smem_u32(xs), a.kc, r, n, ma.ok, wpart, a.max_rank, mine);
-    } else if (ma.ok) {  // rank row groups outer, 1024-column passes inner
-        const int NG = (r + kRowGroup - 1) / kRowGroup, npass = (a.kc + kPass - 1) / kPass;
-        for (int g = 0; g < NG; ++g) {
-            float p[kRowGroup * MAXG];
-#pragma unroll
-            for (int i = 0; i < kRowGroup * MAXG; ++i) p[i] = 0.f;
-            for (int s = 0; s < npass; ++s) {
-                const int c = s * kPass, W = min(kPass, a.kc - c);
-                if (col < W) {
-                    float xf[MAXG][8];
-#pragma unroll
-                    for (int j = 0; j < MAXG; ++j)
-                        unpack8(*reinterpret_cast<const uint4*>(xs + (size_t)j * a.kc + c + col), xf[j]);
-                    if constexpr (WF == kFmtInt4) {
-#pragma unroll
-                        for (int j = 0; j < MAXG; ++j)
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) xf[j][e] *= int4_pos_unscale(e);
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < kRowGroup; ++kk) {
-                        const int k = kRowGroup * g + kk;
-                        if (k < r) {
-                            float af[8];
-                            const uint8_t* w = As + (size_t)k * (a.kc / 8 * VB) + (size_t)(c + col) / 8 * VB;
-                            if constexpr (WF == kFmtInt4) int4x8_to_f32_pos(*reinterpret_cast<const uint32_t*>(w), af);
-                            else load_w8<WF>(w, af);
-#pragma unroll
-                            for (int j = 0; j < MAXG; ++j) p[kk * MAXG + j] += dot8(af, xf[j]);
-                        }
-                    }
-                }
+    if constexpr (WF != kFmtBf16) {  // codes -> bf16 (exact for E4M3 and INT4), 8 values a granule
+        if (ma.ok)
+            for (GridWalk w(gx, tid, TPB); w.k < r; w.next()) {
+                float f[8];
+                const uint8_t* cp = Ac + (size_t)w.k * (a.kc / 8 * VB) + (size_t)w.c * VB;
+                if constexpr (WF == kFmtFp8) fp8x8_to_f32(*reinterpret_cast<const uint2*>(cp), f);
+                else int4x8_to_f32(*reinterpret_cast<const uint32_t*>(cp), f);
+                *reinterpret_cast<uint4*>(As + (size_t)w.k * a.kc + (w.c ^ (w.k & 7)) * 8) =
+                    make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                               pack_bf16x2(f[6], f[7]));
             }
-            const float sum = block_reduce<kRowGroup * MAXG>(p, red);
-            if (tid < kRowGroup * MAXG) {
-                const int kk = tid / MAXG, j = tid - kk * MAXG;
-                if (kRowGroup * g + kk < r && j < n) mine[j * r + kRowGroup * g + kk] = sum;
-            }
-        }
+        __syncthreads();
     }
+    float* mine = part + (size_t)q * slot;  // this CTA's partial tile [token][rank row]
+    mma_shrink_slab<MAXG, kWarps, kMT>(smem_u32(As), smem_u32(xs), a.kc, r, n, ma.ok, wpart, a.max_rank, mine);
     __syncthreads();  // this CTA's partial tile is complete
 
     // ---- push the tile to every other CTA of the cluster, then sum the C tiles in order
@@ -1035,118 +1034,50 @@ __global__ void __launch_bounds__(fused_threads<WF>(), 1)
             float s = 0.f;
             for (int qq = 0; qq < C; ++qq) s += part[(size_t)qq * slot + e];
             const int k = e - (e / r) * r;
-            const float vk = WF == kFmtBf16 ? s : s * rsc_a[k];
+            const float vk = WF == kFmtBf16 ? s : s * rsc_a[k];  // a quantised A row's scale leaves the sum
             if (q == 0) a.v[(int64_t)(ma.i0 + e / r) * a.ldv + k] = vk;
-            if (kWide) vs[k * 4 + e / r] = vk;                // [rank row][token]
-            else vs[e] = WF == kFmtBf16 ? vk : vk * rsc_b[k];  // a quantised B^T row's scale goes onto v_k
+            vs[k * 4 + e / r] = WF == kFmtBf16 ? vk : vk * rsc_b[k];  // [rank row][token]; B^T row's scale
         }
     }
     cp_async_wait<0>();
     __syncthreads();  // vs, and the B^T and y slices, are visible to every thread
 
-    // ---- expand over this CTA's d_out slice
+    // ---- expand over this CTA's d_out slice: 4 columns a thread, every rank row
     if (!mb.ok) return;
     const float sc = a.scale * mb.sc;  // the call's scale times the adapter's
-    if constexpr (kWide) {
-        for (int c4 = tid; c4 < (a.ko >> 2); c4 += TPB) {  // 4 columns of the slice a thread
-            float acc[MAXG][4];
-#pragma unroll
-            for (int j = 0; j < MAXG; ++j)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
-            const uint8_t* bp = Bs + (size_t)c4 * 8;
-#pragma unroll 4
-            for (int k = 0; k < r; ++k) {
-                const uint2 bw = *reinterpret_cast<const uint2*>(bp + (size_t)k * a.ko * 2);
-                const float b4[4] = {bf16lo(bw.x), bf16hi(bw.x), bf16lo(bw.y), bf16hi(bw.y)};
-                const float4 w = *reinterpret_cast<const float4*>(vs + k * 4);
-                const float wj[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                for (int j = 0; j < MAXG; ++j)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[j][e] = fmaf(wj[j], b4[e], acc[j][e]);
-            }
-            const int jcol = cb0 + 4 * c4;
-#pragma unroll
-            for (int j = 0; j < MAXG; ++j) {
-                const int t = mb.tok[j];
-                if (j >= n || t < 0) continue;
-                if (a.y_dtype == 0) {
-                    const uint2 yv = *reinterpret_cast<const uint2*>(ys + ((size_t)j * a.ko + 4 * c4) * 2);
-                    *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.y) + (int64_t)t * a.ldy + jcol) =
-                        make_uint2(pack_bf16x2(fmaf(sc, acc[j][0], bf16lo(yv.x)), fmaf(sc, acc[j][1], bf16hi(yv.x))),
-                                   pack_bf16x2(fmaf(sc, acc[j][2], bf16lo(yv.y)), fmaf(sc, acc[j][3], bf16hi(yv.y))));
-                } else {
-                    float4 o = *reinterpret_cast<const float4*>(ys + ((size_t)j * a.ko + 4 * c4) * 4);
-                    o.x = fmaf(sc, acc[j][0], o.x); o.y = fmaf(sc, acc[j][1], o.y);
-                    o.z = fmaf(sc, acc[j][2], o.z); o.w = fmaf(sc, acc[j][3], o.w);
-                    *reinterpret_cast<float4*>(static_cast<float*>(a.y) + (int64_t)t * a.ldy + jcol) = o;
-                }
-            }
-        }
-        return;
-    }
-    const int NG = (r + kRowGroup - 1) / kRowGroup, npass = (a.ko + kPass - 1) / kPass;
-    for (int s = 0; s < npass; ++s) {
-        const int c = s * kPass, W = min(kPass, a.ko - c);
-        if (col >= W) continue;
-        float acc[MAXG][8];
+    const size_t brow = (size_t)a.ko / 8 * VB;  // bytes of a B^T row slice
+    for (int c4 = tid; c4 < (a.ko >> 2); c4 += TPB) {
+        float acc[MAXG][4];
 #pragma unroll
         for (int j = 0; j < MAXG; ++j)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
-        for (int g = 0; g < NG; ++g) {
-#pragma unroll
-            for (int kk = 0; kk < kRowGroup; ++kk) {
-                const int k = kRowGroup * g + kk;
-                if (k < r) {
-                    float bf[8];
-                    const uint8_t* w = Bs + (size_t)k * (a.ko / 8 * VB) + (size_t)(c + col) / 8 * VB;
-                    if constexpr (WF == kFmtInt4) int4x8_to_f32_pos(*reinterpret_cast<const uint32_t*>(w), bf);
-                    else load_w8<WF>(w, bf);
-#pragma unroll
-                    for (int j = 0; j < MAXG; ++j) {
-                        const float wv = vs[min(j, n - 1) * r + k];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) acc[j][e] = fmaf(wv, bf[e], acc[j][e]);
-                    }
-                }
-            }
-        }
-        if constexpr (WF == kFmtInt4) {
+            for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+#pragma unroll 4
+        for (int k = 0; k < r; ++k) {
+            float b4[4];
+            load_w4<WF>(Bs + (size_t)k * brow, 4 * c4, b4);
+            const float4 w = *reinterpret_cast<const float4*>(vs + k * 4);
+            const float wj[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int j = 0; j < MAXG; ++j)
 #pragma unroll
-                for (int e = 0; e < 8; ++e) acc[j][e] *= int4_pos_unscale(e);
+                for (int e = 0; e < 4; ++e) acc[j][e] = fmaf(wj[j], b4[e], acc[j][e]);
         }
-        const int jcol = cb0 + c + col;
+        const int jcol = cb0 + 4 * c4;
 #pragma unroll
         for (int j = 0; j < MAXG; ++j) {
             const int t = mb.tok[j];
-            if (t < 0) continue;
+            if (j >= n || t < 0) continue;
             if (a.y_dtype == 0) {
-                float yv[8];
-                unpack8(*reinterpret_cast<const uint4*>(ys + ((size_t)j * a.ko + c + col) * 2), yv);
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float lo = fmaf(sc, acc[j][2 * e], yv[2 * e]);
-                    const float hi = fmaf(sc, acc[j][2 * e + 1], yv[2 * e + 1]);
-                    w[e] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
-                           ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
-                }
-                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.y) + (int64_t)t * a.ldy + jcol) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
+                const uint2 yv = *reinterpret_cast<const uint2*>(ys + ((size_t)j * a.ko + 4 * c4) * 2);
+                *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.y) + (int64_t)t * a.ldy + jcol) =
+                    make_uint2(pack_bf16x2(fmaf(sc, acc[j][0], bf16lo(yv.x)), fmaf(sc, acc[j][1], bf16hi(yv.x))),
+                               pack_bf16x2(fmaf(sc, acc[j][2], bf16lo(yv.y)), fmaf(sc, acc[j][3], bf16hi(yv.y))));
             } else {
-                const float* yp = reinterpret_cast<const float*>(ys + ((size_t)j * a.ko + c + col) * 4);
-                float4 o0 = *reinterpret_cast<const float4*>(yp), o1 = *reinterpret_cast<const float4*>(yp + 4);
-                o0.x = fmaf(sc, acc[j][0], o0.x); o0.y = fmaf(sc, acc[j][1], o0.y);
-                o0.z = fmaf(sc, acc[j][2], o0.z); o0.w = fmaf(sc, acc[j][3], o0.w);
-                o1.x = fmaf(sc, acc[j][4], o1.x); o1.y = fmaf(sc, acc[j][5], o1.y);
-                o1.z = fmaf(sc, acc[j][6], o1.z); o1.w = fmaf(sc, acc[j][7], o1.w);
-                float* yo = static_cast<float*>(a.y) + (int64_t)t * a.ldy + jcol;
-                *reinterpret_cast<float4*>(yo) = o0;
-                *reinterpret_cast<float4*>(yo + 4) = o1;
+                float4 o = *reinterpret_cast<const float4*>(ys + ((size_t)j * a.ko + 4 * c4) * 4);
+                o.x = fmaf(sc, acc[j][0], o.x); o.y = fmaf(sc, acc[j][1], o.y);
+                o.z = fmaf(sc, acc[j][2], o.z); o.w = fmaf(sc, acc[j][3], o.w);
+                *reinterpret_cast<float4*>(static_cast<float*>(a.y) + (int64_t)t * a.ldy + jcol) = o;
             }
         }
     }
@@ -1642,7 +1573,7 @@ cudaError_t fused_launch(const ShrinkJob& sj, const ExpandJob& ej, const BatchVi
                          const InlineTable<kInlineItems>* inl, cudaStream_t stream, bool* used, bool dry) {
     *used = false;
     if (num_items <= 0 || sj.nsub != 1 || sj.d_in <= 0 || ej.d_out <= 0) return cudaSuccess;
-    if (WF == kFmtBf16 && max_rank > kFusedWideMaxRank) return cudaSuccess;
+    if (max_rank > kFusedMaxRank) return cudaSuccess;
     const int maxg = max_item_rows <= 1 ? 1 : max_item_rows <= 2 ? 2 : 4;
     const int mr = std::max(8, max_rank);
     const int esz = y_dtype == 0 ? 2 : 4;
@@ -1662,7 +1593,7 @@ cudaError_t fused_launch(const ShrinkJob& sj, const ExpandJob& ej, const BatchVi
         const int kc = sj.d_in / C, ko = ej.d_out / C;
         FusedArgs a;
         std::memset(&a, 0, sizeof(a));
-        size_t o = 4 * 64 * 4;  // block-reduction scratch
+        size_t o = 0;
         a.off_part = (int32_t)(o = al(o));
         o += (size_t)C * kSimtMaxItemRows * mr * 4;
         a.off_vs = (int32_t)(o = al(o));
@@ -1673,8 +1604,10 @@ cudaError_t fused_launch(const ShrinkJob& sj, const ExpandJob& ej, const BatchVi
         o += (size_t)mr * (pa / C) * 4;
         a.off_pid_b = (int32_t)(o = al(o));
         o += (size_t)mr * (pb / C) * 4;
-        a.off_a = (int32_t)(o = al(o));
-        o += (size_t)mr * kc / 8 * bytes_per_8<WF>();
+        a.off_a = (int32_t)(o = al(o));  // the bf16 slab of A
+        o += (size_t)mr * kc * 2;
+        a.off_ac = (int32_t)(o = al(o));  // a quantised pool's codes of A
+        o += WF == kFmtBf16 ? 0 : (size_t)mr * kc / 8 * bytes_per_8<WF>();
         a.off_x = (int32_t)(o = al(o));
         o += (size_t)maxg * kc * 2;
         a.off_b = (int32_t)(o = al(o));
@@ -1682,14 +1615,14 @@ cudaError_t fused_launch(const ShrinkJob& sj, const ExpandJob& ej, const BatchVi
         a.off_y = (int32_t)(o = al(o));
         o += (size_t)maxg * ko * esz;
         a.off_wp = (int32_t)(o = al(o));
-        o += WF == kFmtBf16 ? (size_t)(fused_threads<WF>() / 32) * maxg * mr * 4 : 0;
+        o += (size_t)(kFusedThreads / 32) * maxg * mr * 4;
         const size_t smem = al(o);
         if (smem > 227 * 1024) continue;
         cudaError_t e = raise_smem(kern, smem);
         if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)(num_items * C), 1, 1);
-        cfg.blockDim = dim3(fused_threads<WF>(), 1, 1);
+        cfg.blockDim = dim3(kFusedThreads, 1, 1);
         cfg.dynamicSmemBytes = smem;
         cfg.stream = stream;
         cudaLaunchAttribute attr[1];

@@ -331,6 +331,8 @@ def run_ours(args, rank, world, device, with_e2e=True):
             mask |= k
             launches += n_l
     simt_pair = ("shrink_slab_kernel" if mask & sg.KERNELS_SLAB else "shrink_simt_kernel") + " + expand_simt_kernel"
+    if plans[0].plan.needs_device_table:
+        launches += 1                                # the table upload (sgmv_upload_table) of every step
     names = " + ".join(n for bit, n in ((sg.KERNELS_FUSED, "fused_simt_kernel"), (sg.KERNELS_SIMT, simt_pair),
                                         (sg.KERNELS_TC, "shrink_tc_kernel + expand_tc_kernel")) if mask & bit)
     api = "sgmv_lora_delta_grouped" if grouped else "sgmv_lora_delta"

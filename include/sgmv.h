@@ -474,6 +474,19 @@ SGMV_API sgmv_status sgmv_lora_delta_grouped(const sgmv_delta_entry* entries, in
                                              float scale, int32_t y_dtype, sgmv_stream_t stream);
 
 /*
+ * Copy the plan's table (plan->table_bytes from plan->host_table) to its device
+ * copy `device_table` (16-byte aligned, at least table_bytes), in stream order.
+ * When the host table is pinned (cudaHostAlloc / cudaMallocHost, device-visible
+ * through unified addressing) a small kernel reads it across the bus with
+ * coalesced 16-byte loads, which costs a few microseconds where a copy-engine
+ * transfer of a table this small takes about ten; pageable memory takes a
+ * cudaMemcpyAsync.  The host table must keep its contents until the copy has run
+ * (stream order).  Errors: SGMV_ERR_INVALID (null or misaligned tables, a
+ * table_bytes that is not a multiple of 16), SGMV_ERR_CUDA.
+ */
+SGMV_API sgmv_status sgmv_upload_table(const sgmv_plan* plan, void* device_table, sgmv_stream_t stream);
+
+/*
  * Which kernels sgmv_lora_delta (n_entries = 1) or sgmv_lora_delta_grouped (the
  * entries' projections `projs`, with the same `table`, NULL or not) launch for
  * this plan and pool, without launching anything.  The calls' own choices are

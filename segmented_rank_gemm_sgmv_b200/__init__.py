@@ -35,7 +35,8 @@ EXPORTED = ("sgmv_status_string", "sgmv_last_error", "sgmv_pool_create", "sgmv_p
             "sgmv_pool_set_adapter_scale", "sgmv_pool_get_adapter_scale",
             "sgmv_pool_shuffle_free_pages", "sgmv_pool_pages_device", "sgmv_plan_table_capacity",
             "sgmv_build_plan", "sgmv_shrink", "sgmv_expand", "sgmv_lora_delta", "sgmv_lora_delta_grouped",
-            "sgmv_lora_delta_noalloc", "sgmv_lora_delta_kernels", "sgmv_host_workspace_bytes", "sgmv_lora_delta_host",
+            "sgmv_lora_delta_noalloc", "sgmv_lora_delta_kernels", "sgmv_upload_table", "sgmv_host_workspace_bytes",
+            "sgmv_lora_delta_host",
             "sgmv_check_errors", "sgmv_residency_create", "sgmv_residency_destroy",
             "sgmv_residency_register", "sgmv_residency_unregister", "sgmv_residency_prepare",
             "sgmv_residency_get_stats")
@@ -124,6 +125,7 @@ def load_library() -> ctypes.CDLL:
                                          i32, vp]),
         "sgmv_lora_delta_kernels": (st, [ctypes.POINTER(Plan), vp, vp, i32, vp, i32, ctypes.POINTER(i32),
                                          ctypes.POINTER(i32)]),
+        "sgmv_upload_table": (st, [ctypes.POINTER(Plan), vp, vp]),
         "sgmv_host_workspace_bytes": (i64, [i32, vp, ctypes.POINTER(HostEntry), i32, i32]),
         "sgmv_lora_delta_host": (st, [vp, i32, vp, ctypes.POINTER(HostEntry), i32, f32, i32, vp, i64, vp, i64,
                                       ctypes.POINTER(Plan), ctypes.POINTER(i64), ctypes.POINTER(i64), vp]),
@@ -423,8 +425,9 @@ class BatchPlan:
         return self.device_table.data_ptr()
 
     def upload(self, stream=None) -> Optional[torch.Tensor]:
-        """Copy the table to the device on `stream` (one host-to-device copy); nothing to do
-        when the plan's work items travel as launch arguments."""
+        """Copy the table to the device on `stream` (sgmv_upload_table: a small kernel reading
+        the pinned host table); nothing to do when the plan's work items travel as launch
+        arguments."""
         if not self.plan.needs_device_table:
             return None
         n = max(int(self.plan.table_bytes), 16)
@@ -432,8 +435,8 @@ class BatchPlan:
         if self.device_table is None or self.device_table.numel() < max(n, self.capacity):
             self.device_table = torch.empty(max(n, self.capacity), dtype=torch.uint8, device=dev)
         s = torch.cuda.current_stream(dev) if stream is None else stream
+        _check(load_library().sgmv_upload_table(ctypes.byref(self.plan), self.device_table.data_ptr(), _stream(s)))
         with torch.cuda.stream(s):
-            self.device_table[:n].copy_(self.host[:n], non_blocking=True)
             if self._uploaded is None:
                 self._uploaded = torch.cuda.Event()
             self._uploaded.record(s)

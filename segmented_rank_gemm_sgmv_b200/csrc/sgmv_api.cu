@@ -339,6 +339,56 @@ extern "C" sgmv_status sgmv_lora_delta_grouped(const sgmv_delta_entry* entries, 
     return delta_impl(entries, n_entries, T, plan, table, pool, scale, y_dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
+namespace sgmv {
+namespace {
+// The plan table from pinned host memory to the device: coalesced 16-byte loads through
+// unified addressing (the host buffer is read across the bus by the kernel), stores to the
+// device copy.  Four granules a thread, loads before stores.
+constexpr int kUploadThreads = 256, kUploadPer = 4;
+__global__ void __launch_bounds__(kUploadThreads) table_upload_kernel(const uint4* __restrict__ src,
+                                                                      uint4* __restrict__ dst, int64_t n16) {
+    const int64_t base = (int64_t)blockIdx.x * kUploadThreads * kUploadPer + threadIdx.x;
+    uint4 r[kUploadPer];
+#pragma unroll
+    for (int i = 0; i < kUploadPer; ++i) {
+        const int64_t g = base + (int64_t)i * kUploadThreads;
+        if (g < n16) r[i] = src[g];
+    }
+#pragma unroll
+    for (int i = 0; i < kUploadPer; ++i) {
+        const int64_t g = base + (int64_t)i * kUploadThreads;
+        if (g < n16) dst[g] = r[i];
+    }
+}
+}  // namespace
+}  // namespace sgmv
+
+extern "C" sgmv_status sgmv_upload_table(const sgmv_plan* plan, void* device_table, sgmv_stream_t stream) {
+    if (!plan || !device_table) return fail(SGMV_ERR_INVALID, "upload_table: plan and device_table are required");
+    if (!plan->host_table) return fail(SGMV_ERR_INVALID, "upload_table: plan->host_table is NULL");
+    if (!aligned16(device_table) || !aligned16(plan->host_table))
+        return fail(SGMV_ERR_INVALID, "upload_table: both tables must be 16-byte aligned");
+    const int64_t bytes = plan->table_bytes;
+    if (bytes <= 0) return SGMV_OK;
+    if (bytes % 16) return fail(SGMV_ERR_INVALID, "upload_table: table_bytes is not a multiple of 16");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaPointerAttributes at{};
+    const void* src = nullptr;
+    if (cudaPointerGetAttributes(&at, plan->host_table) == cudaSuccess && at.type == cudaMemoryTypeHost)
+        src = at.devicePointer;
+    cudaGetLastError();  // (an unregistered pointer is not an error here)
+    if (!src) {  // pageable host memory: a copy-engine transfer
+        SGMV_CUDA_TRY(cudaMemcpyAsync(device_table, plan->host_table, (size_t)bytes, cudaMemcpyHostToDevice, s));
+        return SGMV_OK;
+    }
+    const int64_t n16 = bytes / 16;
+    const int64_t per_cta = (int64_t)kUploadThreads * kUploadPer;
+    table_upload_kernel<<<(unsigned)((n16 + per_cta - 1) / per_cta), kUploadThreads, 0, s>>>(
+        static_cast<const uint4*>(src), static_cast<uint4*>(device_table), n16);
+    SGMV_CUDA_TRY(cudaGetLastError());
+    return SGMV_OK;
+}
+
 // Which kernels sgmv_lora_delta / sgmv_lora_delta_grouped launch for a plan, pool and set of
 // projections: the same choices the calls make (including the one-wave test of the fused
 // kernel, an occupancy query), with nothing launched.
@@ -516,8 +566,8 @@ extern "C" sgmv_status sgmv_lora_delta_host(const int32_t* adapter_ids, int32_t 
     }
     int64_t in = 0, out = 0;
     if (plan.needs_device_table) {
-        SGMV_CUDA_TRY(cudaMemcpyAsync(ws + L.table, host_table, (size_t)plan.table_bytes, cudaMemcpyHostToDevice,
-                                      stream));
+        const sgmv_status st_up = sgmv_upload_table(&plan, ws + L.table, stream_);
+        if (st_up != SGMV_OK) return st_up;
         in += plan.table_bytes;
     }
     for (int32_t i = 0; i < n_entries; ++i) {

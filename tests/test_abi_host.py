@@ -111,3 +111,16 @@ def test_kernels_query_argument_checks():
                                      ctypes.byref(launches))
     assert st == 1 and b"no device memory" in lib.sgmv_last_error()
     pool.close()
+
+
+def test_upload_table_argument_checks():
+    """sgmv_upload_table refuses null or misaligned tables before any CUDA call."""
+    lib = sg.load_library()
+    pool = sg.AdapterPool([(512, 512)], num_pages=64, page_elems=512, max_rank=16, device=-1)
+    pool.load(0, 8)
+    plan = pool.plan([0, 0, -1])
+    assert lib.sgmv_upload_table(None, 16, None) == 1
+    assert lib.sgmv_upload_table(ctypes.byref(plan.plan), None, None) == 1
+    assert lib.sgmv_upload_table(ctypes.byref(plan.plan), 17, None) == 1
+    assert b"aligned" in lib.sgmv_last_error()
+    pool.close()

@@ -177,9 +177,13 @@ cudaError_t slab_shrink_launch(const ShrinkJob& j, const BatchView& b, int32_t n
                                cudaStream_t stream, bool* used, bool dry);
 cudaError_t launch_shrink_tc(const uint16_t* x, int64_t ldx, int32_t d_in, const BatchView& b, int32_t num_tiles,
                              int32_t max_rank, const PoolView& pool, float* v, int64_t ldv, cudaStream_t stream);
+// after_shrink: the preceding kernel of the stream is this call's tensor-core shrink, an
+// ordinary launch that wrote v and nothing else this kernel reads; the expand is then a
+// programmatic dependent launch that reads the plan, the pool and y at once and waits for
+// the shrink's completion only before it reads v.
 cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const BatchView& b, int32_t num_tiles,
                              int32_t max_rank, const PoolView& pool, float scale, void* y, int64_t ldy,
-                             int32_t y_dtype, cudaStream_t stream);
+                             int32_t y_dtype, bool after_shrink, cudaStream_t stream);
 
 // Read and clear the device error words of every translation unit.
 cudaError_t read_clear_errors_simt(uint32_t* bits, cudaStream_t stream);

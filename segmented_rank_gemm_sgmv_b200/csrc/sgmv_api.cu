@@ -238,7 +238,7 @@ sgmv_status sgmv::expand_impl(const float* v, int64_t ldv, int32_t T, int32_t d_
     SGMV_CUDA_TRY(launch_expand_simt(&job, 1, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank,
                                      simt_work(plan), pv, scale, y_dtype, use_inl ? &inl : nullptr, y_early, stream));
     SGMV_CUDA_TRY(launch_expand_tc(v, ldv, d_out, bv, plan->num_tc_tiles, plan->max_rank, pv, scale, y, ldy, y_dtype,
-                                   stream));
+                                   false, stream));
     return SGMV_OK;
 }
 
@@ -315,10 +315,13 @@ sgmv_status sgmv::delta_impl(const sgmv_delta_entry* entries, int32_t n, int32_t
     // the expand's predecessors are this call's shrinks, which do not write y: y may be read early
     SGMV_CUDA_TRY(launch_expand_simt(ej, n, bv, plan->num_simt_items, plan->max_item_rows, plan->max_rank, work, pv,
                                      scale, y_dtype, use_inl ? &inl : nullptr, true, stream));
+    // the first tensor-core expand directly follows a tensor-core shrink when there are no
+    // SIMT items: it may then start while that shrink finishes
     for (int32_t i = 0; i < n; ++i) {
         bv.proj = entries[i].proj;
         SGMV_CUDA_TRY(launch_expand_tc(ej[i].v, ej[i].ldv, ej[i].d_out, bv, plan->num_tc_tiles, plan->max_rank, pv,
-                                       scale, ej[i].y, ej[i].ldy, y_dtype, stream));
+                                       scale, ej[i].y, ej[i].ldy, y_dtype, i == 0 && plan->num_simt_items == 0,
+                                       stream));
     }
     return SGMV_OK;
 }

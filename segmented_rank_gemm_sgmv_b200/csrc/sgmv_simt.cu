@@ -191,11 +191,6 @@ __device__ __forceinline__ ItemInfo load_item(const BatchView& b, const InlineTa
     return m;
 }
 
-__device__ __forceinline__ void pdl_launch_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
 __device__ __forceinline__ float dot8(const float (&a)[8], const float (&b)[8]) {
     float s = a[0] * b[0];
 #pragma unroll

@@ -140,6 +140,9 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
     __shared__ float rsc_s[kMaxRank];  // row scales of a quantised A
 
     const int tid = threadIdx.x, warp = tid >> 5;
+    // a dependent expand may be scheduled now: its CTAs take SMs as these CTAs leave, and
+    // wait for this grid's completion before they read v
+    pdl_launch_dependents();
     const int tile_idx = blockIdx.x / a.ks;
     const uint32_t q = cluster_ctarank();
     const ItemRec it = a.b.tc_tiles[(int64_t)tile_idx * a.b.n_proj + a.b.proj];
@@ -248,6 +251,14 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
                 abort_flag = 1;
         };
         if constexpr (WF == kFmtBf16) {
+            // A: rank rows n < npad (zero past r); the thread's granules g = tid + 128 i are
+            // rank rows (tid >> 3) + 16 i at column chunk tid & 7.  Their page ids stay in
+            // registers while the K tiles stay in one page, so a stage issues its copies
+            // back to back without a shared-memory load in front of each.
+            constexpr int kMaxI = kMaxRank * 8 / kTcTileRows;
+            const int n_i = npad / 16, kg = tid & 7;
+            int32_t pg[kMaxI];
+            int cur_rel = -1;
             for (int kt = 0; kt < nk; ++kt) {
                 const int st = kt % kShrinkStages;
                 wait_empty(kt);
@@ -255,16 +266,26 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
                 uint8_t* as = xs + x_tile_bytes;
                 const int c = k_begin + kt * kKTile;
                 issue_x(kt, xs);
-                // A: rank rows n < npad, zero past r; the 64 columns lie in one page
+                // the 64 columns lie in one page
                 const int page_rel = (c >> P_log2) - first_page, in_page = c & ((1 << P_log2) - 1);
-                for (int g = tid; g < npad * 8; g += kTcTileRows) {
-                    const int n = g >> 3, kg = g & 7;
-                    const uint32_t off = (uint32_t)(n >> 3) * 1024 + sw128_off((uint32_t)n, (uint32_t)kg);
-                    const bool valid = ok && n < r;
-                    const uint16_t* src = a.pool.pages;
-                    if (valid)
-                        src = a.pool.pages + ((int64_t)pid_s[n * span_pages + page_rel] << P_log2) + in_page + kg * 8;
-                    cp_async16(as + off, src, valid);
+                if (page_rel != cur_rel) {
+                    cur_rel = page_rel;
+#pragma unroll
+                    for (int i = 0; i < kMaxI; ++i) {
+                        const int n = (tid >> 3) + 16 * i;
+                        pg[i] = (i < n_i && ok && n < r) ? pid_s[n * span_pages + page_rel] : 0;
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < kMaxI; ++i) {
+                    if (i < n_i) {
+                        const int n = (tid >> 3) + 16 * i;
+                        const uint32_t off = (uint32_t)(n >> 3) * 1024 + sw128_off((uint32_t)n, (uint32_t)kg);
+                        const bool valid = ok && n < r;
+                        const uint16_t* src =
+                            valid ? a.pool.pages + ((int64_t)pg[i] << P_log2) + in_page + kg * 8 : a.pool.pages;
+                        cp_async16(as + off, src, valid);
+                    }
                 }
                 cp_async_commit();  // close the group: the copies of every stage form their own
                 cp_async_mbar_arrive_noinc(&full_bar[st]);
@@ -283,15 +304,30 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
             const uint8_t* pages8 = reinterpret_cast<const uint8_t*>(a.pool.pages);
             uint8_t* raw0 = smem + a.raw_offset;
             const int raw_slot = a.npad_max * 8 * VB;
+            // granules g = tid + 128 i: rank row (tid >> 3) + 16 i, column chunk tid & 7; their
+            // page ids stay in registers while the K tiles stay in one page
+            constexpr int kMaxI = kMaxRank * 8 / kTcTileRows;
+            const int n_i = npad / 16, kg = tid & 7;
+            int32_t pg[kMaxI];
+            int cur_rel = -1;
             auto issue_codes = [&](int kt) {
                 const int c = k_begin + kt * kKTile;
                 const int page_rel = (c >> P_log2) - first_page, in_page = c & ((1 << P_log2) - 1);
                 uint8_t* raw = raw0 + (size_t)(kt % D) * raw_slot;
-                for (int g = tid; g < npad * 8; g += kTcTileRows) {
-                    const int n = g >> 3, kg = g & 7;
-                    if (ok && n < r)
-                        cp_async_n<VB>(raw + g * VB, pages8 + ((int64_t)pid_s[n * span_pages + page_rel] << page_shift) +
-                                                         (in_page / 8 + kg) * VB);
+                if (page_rel != cur_rel) {
+                    cur_rel = page_rel;
+#pragma unroll
+                    for (int i = 0; i < kMaxI; ++i) {
+                        const int n = (tid >> 3) + 16 * i;
+                        pg[i] = (i < n_i && ok && n < r) ? pid_s[n * span_pages + page_rel] : 0;
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < kMaxI; ++i) {
+                    const int n = (tid >> 3) + 16 * i;
+                    if (i < n_i && ok && n < r)
+                        cp_async_n<VB>(raw + (tid + kTcTileRows * i) * VB,
+                                       pages8 + ((int64_t)pg[i] << page_shift) + (in_page / 8 + kg) * VB);
                 }
             };
 #pragma unroll 1
@@ -344,9 +380,12 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
     }
     __syncwarp();  // warp 4 reconverges before the warp-collective instructions below
 
-    // ---- epilogue: tensor memory -> red[128][RS] (reuses the stages; RS odd: conflict-free)
+    // ---- epilogue: tensor memory -> red[128][RS] (reuses the stages).  RS = npad_max + 4 is
+    // 4 or 20 modulo 32 words, so the 16-byte stores of 8 consecutive rows (one store
+    // phase) fall into 8 different 4-bank groups, and every 4 columns are one 16-byte word
+    // for the cluster reduction below.
     float* red = reinterpret_cast<float*>(smem);
-    const int RS = a.npad_max + 1;
+    const int RS = a.npad_max + 4;
     if (warp < 4) {
         if (!abort_flag && !mbar_wait(&acc_bar, 0u, &g_err_tc)) abort_flag = 1;
         tc_fence_after();
@@ -356,29 +395,42 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
             tmem_ld_32x32b_x32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, regs);
             tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-                if (c0 + e < a.npad_max) red[m * RS + c0 + e] = __uint_as_float(regs[e]);
+            for (int e = 0; e < 32; e += 4)
+                if (c0 + e < a.npad_max)
+                    *reinterpret_cast<float4*>(red + m * RS + c0 + e) =
+                        make_float4(__uint_as_float(regs[e]), __uint_as_float(regs[e + 1]),
+                                    __uint_as_float(regs[e + 2]), __uint_as_float(regs[e + 3]));
         }
     }
     tc_fence_before();
     cluster_sync();
 
     if (ok && !abort_flag) {
-        const int KS = a.ks;
+        // CTA q sums rows [m0, m1) of the KS partial tiles, 4 rank columns per 16-byte load
+        const int KS = a.ks, G = npad / 4;
         const int m0 = (int)((kTcTileRows * q) / KS), m1 = (int)((kTcTileRows * (q + 1)) / KS);
         const uint32_t red_s = smem_u32(red);
-        for (int e = tid; e < (m1 - m0) * r; e += kShrinkThreads) {
-            const int mm = m0 + e / r, k = e % r;
-            if (mm >= rows) continue;
-            float pv[8];
+        for (int e = tid; e < (m1 - m0) * G; e += kShrinkThreads) {
+            const int mm = m0 + e / G, k4 = (e % G) * 4;
+            if (mm >= rows || k4 >= r) continue;
+            float4 pv[8];
 #pragma unroll
             for (int qq = 0; qq < 8; ++qq)  // all loads in flight before the fixed-order sum
-                pv[qq] = qq < KS ? ld_cluster_f32(map_cluster(red_s + 4u * (uint32_t)(mm * RS + k), (uint32_t)qq)) : 0.f;
-            float sum = 0.f;
+                pv[qq] = qq < KS ? ld_cluster_v4(map_cluster(red_s + 4u * (uint32_t)(mm * RS + k4), (uint32_t)qq))
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            float sum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int qq = 0; qq < 8; ++qq) sum += pv[qq];
-            // a quantised row's scale leaves the sum: v_k = s_k * sum_c q_kc x_c
-            a.v[(int64_t)(it.row_begin + mm) * a.ldv + k] = WF == kFmtBf16 ? sum : sum * rsc_s[k];
+            for (int qq = 0; qq < 8; ++qq) {
+                sum[0] += pv[qq].x;
+                sum[1] += pv[qq].y;
+                sum[2] += pv[qq].z;
+                sum[3] += pv[qq].w;
+            }
+            float* vrow = a.v + (int64_t)(it.row_begin + mm) * a.ldv;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                // a quantised row's scale leaves the sum: v_k = s_k * sum_c q_kc x_c
+                if (k4 + c < r) vrow[k4 + c] = WF == kFmtBf16 ? sum[c] : sum[c] * rsc_s[k4 + c];
         }
     }
     cluster_sync();
@@ -563,6 +615,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
         // V = v split into bf16 hi + lo for the unit's tile, when the tile changes
         auto v_split = [&](const Unit& w) {
             if (!(w.ok && w.tile != cur_tile)) return;
+            pdl_wait();  // v is final once the preceding kernel (the shrink) has completed
             if (ts >= 0) wait(&vempty_bar, (uint32_t)(ts & 1));  // the MMAs of the previous tile are done
             if (WF != kFmtBf16) {  // v_k takes the scale of B^T row k
                 if (pt < w.r) {
@@ -656,7 +709,6 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
             const int32_t pg0 = pg_next[0], pg1 = pg_next[1];
             if (u + 1 < u1) fetch(unit(u + 1), t_next, t0_next, pg_next);
             if (i >= S) wait(&yfree_bar[st], (uint32_t)((i / S - 1) & 1));
-            if constexpr (WF == kFmtBf16) v_split(w);
             if (w.ok) {
                 if (pt < w.r * npc) pid_s[st][pt] = pg0;
                 if (pt + kExpandProducers < w.r * npc) pid_s[st][pt + kExpandProducers] = pg1;
@@ -723,6 +775,9 @@ __global__ void __launch_bounds__(kExpandThreads, 1) expand_tc_kernel(const Expa
             }
             cp_async_commit();
             cp_async_mbar_arrive_noinc(&full_bar[st]);
+            // V after the unit's copies: with a programmatic launch, the first unit's y and
+            // B^T copies go out before the wait for the shrink
+            if constexpr (WF == kFmtBf16) v_split(w);
             if constexpr (WF != kFmtBf16) {
                 // the codes of unit i - lag (its commit group) have landed: convert them; then
                 // the V split, which may wait for the MMAs of that unit
@@ -967,7 +1022,7 @@ cudaError_t launch_shrink_tc(const uint16_t* x, int64_t ldx, int32_t d_in, const
     a.ks = ks;
     a.kcols = d_in / ks;
     const size_t stage_bytes = (size_t)kTcTileRows * kKTile * 2 + (size_t)a.npad_max * kKTile * 2;
-    const size_t main_bytes = std::max(stage_bytes * kShrinkStages, (size_t)kTcTileRows * (a.npad_max + 1) * 4);
+    const size_t main_bytes = std::max(stage_bytes * kShrinkStages, (size_t)kTcTileRows * (a.npad_max + 4) * 4);
     const size_t span_pages = ((size_t)a.kcols >> pool.page_log2) + 2;  // pages one K range can touch
     // quantised pools: a ring of kShrinkCodeSlots slots of A codes (npad_max rows x 64 values)
     const size_t raw_bytes = pool.wfmt == kFmtBf16 ? 0  // 1 byte (E4M3) or half a byte (INT4) a value
@@ -1003,7 +1058,7 @@ cudaError_t launch_shrink_tc(const uint16_t* x, int64_t ldx, int32_t d_in, const
 
 cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const BatchView& b, int32_t num_tiles,
                              int32_t max_rank, const PoolView& pool, float scale, void* y, int64_t ldy,
-                             int32_t y_dtype, cudaStream_t stream) {
+                             int32_t y_dtype, bool after_shrink, cudaStream_t stream) {
     if (num_tiles <= 0) return cudaSuccess;
     ExpandTcArgs a;
     a.v = v;
@@ -1080,8 +1135,17 @@ cudaError_t launch_expand_tc(const float* v, int64_t ldv, int32_t d_out, const B
                                         : pick(std::integral_constant<int, kFmtBf16>{});
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)blocks, kExpandThreads, smem, stream>>>(a, tmap_y);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks, 1, 1);
+    cfg.blockDim = dim3(kExpandThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_shrink ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, a, tmap_y);
 }
 
 cudaError_t read_clear_errors_tc(uint32_t* bits, cudaStream_t stream) {

@@ -422,8 +422,10 @@ SGMV_API sgmv_status sgmv_expand(const float* v, int64_t ldv, int32_t T, int32_t
  *
  * (s_s: the adapter's multiplier, as for sgmv_expand)
  * = sgmv_shrink into v, then sgmv_expand from v, on `stream`; the expand's
- * SIMT launch overlaps the shrink (programmatic dependent launch), so the
- * second launch costs little ([Glossary], "Limits and open questions", names
+ * SIMT launch overlaps the shrink (programmatic dependent launch), and so does
+ * its tensor-core launch when the plan has no SIMT items (it follows the
+ * tensor-core shrink directly and reads v only after that shrink completes), so
+ * the second launch costs little ([Glossary], "Limits and open questions", names
  * the extra launch per adapted layer as a cost of unmerged adapters).
  * x, y, y_dtype, d_in, d_out, proj as for sgmv_shrink / sgmv_expand.
  * v        device fp32 [plan->num_rows][ldv], ldv >= plan->max_rank: workspace

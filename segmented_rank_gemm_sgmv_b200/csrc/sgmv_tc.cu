@@ -444,10 +444,13 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_tc_kernel(const ShrinkT
 // Persistent: CTA b takes a contiguous run of units (tile of <= 128 rows, block
 // of kYRowBytes of y columns), so consecutive units mostly share the tile and
 // its v rows.  Warp roles:
-//   warps 8-11 (producers): per unit, fetch the token rows and B^T page ids;
-//     copy each y row segment (256 bytes) with one bulk copy that completes on
-//     the stage's mbarrier by bytes, and the B^T block with 16-byte cp.async;
-//     when the tile changes, write V_hi / V_lo (v split into bf16 hi + lo)
+//   warps 8-11 (producers): per unit, fetch the token rows and B^T page ids (one
+//     unit ahead); copy the y block (two 2-D TMA boxes that complete on the stage's
+//     mbarrier by bytes when the tile's rows are consecutive tokens, else 16-byte
+//     cp.async) and the B^T block (16-byte cp.async); then, when the tile changes,
+//     write V_hi / V_lo (v split into bf16 hi + lo).  Launched as a programmatic
+//     dependent of the shrink, they wait for it (griddepcontrol.wait) only there,
+//     before the first read of v.
 //   warp 12 (one lane): tcgen05.mma  acc[i & 1] = V_hi B + V_lo B  (N = block);
 //     with bf16 y (YM), V carries the scale and the MMAs go on with acc += Y I:
 //     the staged y block, already in the K-major 128-byte swizzle of an A
